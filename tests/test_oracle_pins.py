@@ -1,0 +1,388 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+None of these tests retypes the oracle's own formulas: each compares the
+oracle with a worked example printed on the pages (``tests/golden``), a closed
+form, an invariant, or an independent library routine (``math.fsum``, torch's
+fp64 norms, numpy integer matmul, torch's bf16 cast).
+"""
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from w8a8_int8_quantized_norm_b200 import synthetic as S
+
+RNG = np.random.default_rng(1234)
+
+
+def _golden(golden_dir, name):
+    with open(os.path.join(golden_dir, name)) as f:
+        return json.load(f)
+
+
+def _ulp32(x):
+    x = np.abs(np.asarray(x, np.float32))
+    return np.spacing(np.maximum(x, np.float32(np.finfo(np.float32).tiny)))
+
+
+# --------------------------------------------------------------------------
+# exact summation (the norm statistics)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("case", range(6))
+def test_exact_sum_matches_fsum(case):
+    n = [1, 7, 100, 4096, 9216, 28672][case]
+    x = RNG.standard_normal(n) * np.exp2(RNG.integers(-60, 60, n))
+    assert oracle.exact_sum(x) == math.fsum(x)
+
+
+def test_exact_sum_adversarial():
+    cases = [
+        [1e308, 1e308, -1e308, -1e308, 1.0],
+        [1.0, 1e-300, -1.0],
+        [2.0 ** 53, 1.0, -(2.0 ** 53)],
+        [2.0 ** 53, 1.0, 1e-30],            # sticky bit breaks the tie upward
+        [2.0 ** 53, 1.0],                   # exact tie, rounds to even
+        [2.0 ** 53 + 2, 1.0],               # exact tie, rounds up to even
+        [5e-324, 5e-324, 5e-324],
+        [-3.5, 1.25, -0.0, 0.0],
+        [0.1] * 10,
+        list(-np.arange(1000, dtype=np.float64) ** 2),
+    ]
+    for c in cases:
+        # exact rational sum, rounded once by CPython's correctly rounded int division
+        exact = float(sum((Fraction(v) for v in c), Fraction(0)))
+        assert oracle.exact_sum(np.array(c)) == exact, c
+
+
+# --------------------------------------------------------------------------
+# bf16 rounding of the epilogue output
+# --------------------------------------------------------------------------
+
+def test_bf16_rounding_matches_torch():
+    x = np.concatenate([
+        RNG.standard_normal(20000).astype(np.float32) * np.float32(3.0),
+        np.array([0.0, -0.0, 1.0, 1.00390625, 1.01171875, 65504.0, 3.0e38, -3.0e38,
+                  1e-40, -1e-40, np.inf, -np.inf], np.float32),
+        # exact ties between two bf16 neighbours
+        (np.arange(1, 200, dtype=np.uint32) << 16 | 0x8000).view(np.float32),
+    ])
+    ours = oracle.f32_to_bf16_bits(x)
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, ref)
+
+
+# --------------------------------------------------------------------------
+# norms (step 4) against torch's fp64 implementations
+# --------------------------------------------------------------------------
+
+def _torch_norm64(x32, kind, gamma, beta, eps):
+    t = torch.from_numpy(x32.astype(np.float64))
+    K = t.shape[1]
+    g = torch.from_numpy(gamma.astype(np.float64)) if gamma is not None else None
+    b = torch.from_numpy(beta.astype(np.float64)) if beta is not None else None
+    if kind == oracle.NORM_RMS:
+        return torch.nn.functional.rms_norm(t, (K,), g, eps).numpy()
+    return torch.nn.functional.layer_norm(t, (K,), g, b, eps).numpy()
+
+
+@pytest.mark.parametrize("kind", [oracle.NORM_RMS, oracle.NORM_LAYER])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_norm_matches_torch_fp64(kind, dtype):
+    M, K = 37, 1000
+    x = RNG.standard_normal((M, K)).astype(np.float32)
+    x[:, [3, 500]] *= 60.0
+    x[5] += 7.0  # a row with a large mean (cancellation in the variance)
+    gamma = RNG.uniform(0.5, 1.5, K).astype(np.float32)
+    beta = (RNG.standard_normal(K) * 0.1).astype(np.float32) if kind == oracle.NORM_LAYER else None
+    if dtype == "bf16":
+        xin = S.to_bf16_bits(x)
+        x32 = torch.from_numpy(xin.view(np.int16)).view(torch.bfloat16).float().numpy()
+    else:
+        xin, x32 = x, x
+    y, mu, r = oracle.norm(xin, kind, gamma, beta, 1e-5)
+    ref = _torch_norm64(x32, kind, gamma, beta, 1e-5)
+    # the oracle rounds r (and mu) to fp32 and then does 2-4 fp32 operations
+    err = np.abs(y.astype(np.float64) - ref)
+    bound = 6 * _ulp32(ref).astype(np.float64) + 4 * np.finfo(np.float32).eps * np.abs(ref) \
+        + (1e-6 if kind == oracle.NORM_LAYER else 0.0)
+    assert np.all(err <= bound), float((err / bound).max())
+
+
+def test_norm_closed_forms():
+    K = 64
+    c = np.float32(3.0)
+    x = np.full((1, K), c, np.float32)
+    y, _, r = oracle.norm(x, oracle.NORM_RMS, None, None, 0.0)
+    assert r[0] == np.float32(1.0 / 3.0) and np.all(y == np.float32(c * np.float32(1.0 / 3.0)))
+    # LayerNorm of a constant row is beta exactly (x - mu == 0)
+    beta = RNG.standard_normal(K).astype(np.float32)
+    y, mu, _ = oracle.norm(x, oracle.NORM_LAYER, None, beta, 1e-5)
+    assert mu[0] == c and np.array_equal(y[0], beta)
+    # all-zero RMS row: y = 0; r = 1/sqrt(eps)
+    z = np.zeros((1, K), np.float32)
+    y, _, r = oracle.norm(z, oracle.NORM_RMS, None, None, 1e-5)
+    assert np.all(y == 0) and r[0] == np.float32(1.0 / math.sqrt(np.float64(np.float32(1e-5))))
+    # NONE with a multiplier is an element-wise product
+    g = RNG.uniform(0.5, 2, K).astype(np.float32)
+    xx = RNG.standard_normal((3, K)).astype(np.float32)
+    y, _, _ = oracle.norm(xx, oracle.NORM_NONE, g, None, 1e-5)
+    assert np.array_equal(y, (xx * g[None, :]).astype(np.float32))
+
+
+# --------------------------------------------------------------------------
+# per-token quantisation (steps 5/6)
+# --------------------------------------------------------------------------
+
+def test_worked_example_token_row(golden_dir):
+    g = _golden(golden_dir, "token_row_outliers.json")
+    K = g["row_width"]
+    lo, hi = g["ordinary_range"]
+    row = RNG.uniform(lo, hi, K).astype(np.float32)
+    row[[0, 1]] = [lo, hi]  # the range ends are present
+    for ch, v in g["outliers"].items():
+        row[int(ch)] = v
+    q, step = oracle.quantize_rows(row[None, :])
+    p, tol = g["printed"], g["printed_precision"]
+    assert abs(step[0] - p["step_with_outliers"]) <= tol["step_with_outliers"]
+    assert step[0] == np.float32(np.float32(60.0) / np.float32(127.0))
+    ordinary = np.ones(K, bool)
+    ordinary[[int(c) for c in g["outliers"]]] = False
+    levels = np.unique(q[0, ordinary])
+    assert levels.min() == -4 and levels.max() == 4
+    assert len(levels) == p["ordinary_levels_with_outliers"]
+    assert q[0, 2817] == -127 and q[0, 1512] == 95  # 45 / (60/127) = 95.25
+    # without the outliers: step = 2/127, about 30 times finer
+    row2 = row.copy()
+    row2[~ordinary] = 0
+    q2, step2 = oracle.quantize_rows(row2[None, :])
+    assert abs(step2[0] - p["step_without_outliers"]) <= tol["step_without_outliers"]
+    assert step2[0] == np.float32(np.float32(2.0) / np.float32(127.0))
+    assert abs(step[0] / step2[0] - p["finer_factor"]) <= tol["finer_factor"]
+    assert q2[0].min() == -127 and q2[0].max() == 127
+
+
+def test_quantize_ties_round_half_even():
+    # absmax 127 makes the step exactly 1.0, so y/step are the values themselves
+    y = np.array([[127.0, 0.5, 1.5, 2.5, -0.5, -1.5, -2.5, 126.5, -126.5, 3.4999998]], np.float32)
+    q, step = oracle.quantize_rows(y)
+    assert step[0] == 1.0
+    assert q[0].tolist() == [127, 0, 2, 2, 0, -2, -2, 126, -126, 3]
+
+
+def test_quantize_clamp_and_zero_rows():
+    # a subnormal absmax: step = fl32(2^-140 / 127) = 2^-147 and the quotient
+    # 2^-140 / 2^-147 = 128 must clamp to 127 (and -128 to -127)
+    a = np.float32(2.0 ** -140)
+    y = np.array([[a, -a, 0.0], [0.0, 0.0, 0.0]], np.float32)
+    q, step = oracle.quantize_rows(y)
+    assert step[0] == np.float32(2.0 ** -147)
+    assert q[0].tolist() == [127, -127, 0]
+    assert step[1] == 0.0 and q[1].tolist() == [0, 0, 0]
+    # the symmetric range never produces -128
+    yy = RNG.standard_normal((200, 333)).astype(np.float32)
+    qq, _ = oracle.quantize_rows(yy)
+    assert qq.min() >= -127 and qq.max() <= 127
+    assert np.all(np.abs(qq).max(axis=1) == 127)
+
+
+def test_try_it_steps(golden_dir):
+    g = _golden(golden_dir, "try_it_steps.json")
+    for key, big in (("x_step", g["largest_abs_x"]), ("w_step", g["largest_abs_w"])):
+        t = np.array([[big, -0.25 * big, 0.0]], np.float32)
+        _, step = oracle.quantize_rows(t)
+        assert abs(step[0] - g["printed"][key]) <= g["printed_precision"][key], key
+
+
+# --------------------------------------------------------------------------
+# smoothing factors, fold and weight smoothing (steps 1-3)
+# --------------------------------------------------------------------------
+
+def _two_channel_weights():
+    # nn.Linear layout [N_out=3, K_in=2]; column maxima are (0.2, 0.5) while
+    # the row maxima are different, so a max over the wrong axis is caught
+    return np.array([[0.2, -0.05], [-0.1, 0.5], [0.15, 0.3]], np.float32)
+
+
+def test_worked_example_two_channels(golden_dir):
+    g = _golden(golden_dir, "two_channel_alpha.json")
+    act_max = np.array(g["act_max"], np.float32)
+    W = _two_channel_weights()
+    assert np.allclose(np.abs(W).max(axis=0), g["w_max"])
+    token = act_max[None, :].copy()  # a token that reaches both channel maxima
+    p, tol = g["printed"], g["printed_precision"]
+
+    q0, st0 = oracle.quantize_rows(token)
+    assert abs(st0[0] - p["unsmoothed"]["step"]) <= tol["step"]
+    assert q0[0, 1] == p["unsmoothed"]["ch2_levels"]
+
+    res = {}
+    for alpha in (0.5, 0.8):
+        s, _ = oracle.smooth_scales(act_max, [W], alpha)
+        gf, _ = oracle.fold_norm(s)                      # gamma = 1: gamma' = 1/s
+        y, _, _ = oracle.norm(token, oracle.NORM_NONE, gf, None)
+        q, st = oracle.quantize_rows(y)
+        What = oracle.smooth_weights(W, s)
+        res[alpha] = (s, y, q, st, np.abs(What).max(axis=0))
+
+    s, y, q, st, wmax = res[0.5]
+    pa = p["alpha_0.5"]
+    assert abs(float(np.abs(y).max()) - pa["step_numerator"]) <= tol["step_numerator"]
+    assert abs(st[0] - pa["step"]) <= tol["step"]
+    assert q[0, 1] == pa["ch2_levels"]
+    s, y, q, st, wmax = res[0.8]
+    pb = p["alpha_0.8"]
+    assert q[0, 1] == pb["ch2_levels"]
+    assert abs(wmax.max() / wmax.min() - pb["weight_spread"]) <= tol["weight_spread"]
+
+
+def test_geometric_mean_at_half_alpha():
+    """At alpha = 0.5 the smoothed activation and weight channel maxima are both
+    sqrt(max|X_j| * max|W_j|) (the page 'LLM.int8() and SmoothQuant', going deeper)."""
+    w = S.SMALL
+    inp = S.make_inputs(w)
+    xc = inp.x_cal["x"]
+    W = inp.W["fc"]
+    act_max = oracle.calibrate_absmax(xc, oracle.NORM_NONE)
+    s, _ = oracle.smooth_scales(act_max, [W], 0.5)
+    gf, _ = oracle.fold_norm(s)
+    y, _, _ = oracle.norm(xc, oracle.NORM_NONE, gf, None)
+    x_hat_max = np.abs(y).max(axis=0).astype(np.float64)
+    w_hat_max = np.abs(oracle.smooth_weights(W, s)).max(axis=0).astype(np.float64)
+    gm = np.sqrt(act_max.astype(np.float64) * np.abs(W).max(axis=0).astype(np.float64))
+    assert np.all(np.abs(x_hat_max - gm) <= 4e-7 * gm)
+    assert np.all(np.abs(w_hat_max - gm) <= 4e-7 * gm)
+
+
+def test_equivalence_fp64():
+    """Y = (X diag(s)^-1)(diag(s) W) to 1e-12 relative in fp64, with the oracle's s."""
+    w = S.SMALL
+    inp = S.make_inputs(w)
+    X = inp.x["x"].astype(np.float64)
+    W = inp.W["fc"]
+    act_max = oracle.calibrate_absmax(inp.x_cal["x"], oracle.NORM_NONE)
+    for alpha in (0.5, 0.8):
+        s, _ = oracle.smooth_scales(act_max, [W], alpha)
+        s = s.astype(np.float64)
+        Y = X @ W.astype(np.float64).T
+        Ys = (X / s[None, :]) @ (W.astype(np.float64) * s[None, :]).T
+        assert np.max(np.abs(Ys - Y)) <= 1e-12 * np.max(np.abs(Y))
+
+
+@pytest.mark.parametrize("kind", [oracle.NORM_RMS, oracle.NORM_LAYER])
+def test_fold_keeps_the_layer_output(kind):
+    """The folded norm times the smoothed weights reproduces the unsmoothed
+    product within fp32 rounding; folding in the wrong direction does not."""
+    M, K, N = 24, 256, 48
+    x = RNG.standard_normal((M, K)).astype(np.float32)
+    x[:, [7, 100]] *= 50
+    gamma = RNG.uniform(0.5, 1.5, K).astype(np.float32)
+    beta = (RNG.standard_normal(K) * 0.1).astype(np.float32) if kind == oracle.NORM_LAYER else None
+    W = (RNG.standard_normal((N, K)) * 0.02).astype(np.float32)
+    act_max = oracle.calibrate_absmax(x, kind, gamma, beta)
+    s, _ = oracle.smooth_scales(act_max, [W], 0.5)
+    gf, bf = oracle.fold_norm(s, gamma, beta)
+    y, _, _ = oracle.norm(x, kind, gamma, beta)
+    yf, _, _ = oracle.norm(x, kind, gf, bf)
+    What = oracle.smooth_weights(W, s)
+    Y = y.astype(np.float64) @ W.astype(np.float64).T
+    Yf = yf.astype(np.float64) @ What.astype(np.float64).T
+    scale = np.abs(y).astype(np.float64) @ np.abs(W).astype(np.float64).T
+    assert np.all(np.abs(Yf - Y) <= 1e-6 * scale + 1e-30)
+    # the check discriminates: a fold in the wrong direction (gamma * s, so
+    # the norm would emit y * s while the weights also carry s) fails it
+    s64 = s.astype(np.float64)
+    wrong = (y.astype(np.float64) * s64[None, :]) @ What.astype(np.float64).T
+    assert np.max(np.abs(wrong - Y)) > 1e-2 * np.max(np.abs(Y))
+
+
+def test_shared_scale_is_max_over_all_linears():
+    """Linears reading one norm share s from the element-wise max of their
+    weights: equal to treating them as one stacked weight."""
+    K = 96
+    act_max = np.abs(RNG.standard_normal(K)).astype(np.float32) * 10
+    Ws = [(RNG.standard_normal((n, K)) * 0.02).astype(np.float32) for n in (16, 40, 8)]
+    Ws[2][3, 11] = 0.9  # one large weight in the third matrix decides channel 11
+    s_list, _ = oracle.smooth_scales(act_max, Ws, 0.8)
+    s_cat, _ = oracle.smooth_scales(act_max, [np.concatenate(Ws, axis=0)], 0.8)
+    s_first, _ = oracle.smooth_scales(act_max, [Ws[0]], 0.8)
+    assert np.array_equal(s_list, s_cat)
+    assert s_list[11] != s_first[11]
+
+
+def test_smoothing_clamps():
+    K = 4
+    act_max = np.array([0.0, 1e-9, 5.0, 5.0], np.float32)
+    W = np.array([[0.0, 0.3, 0.0, 1e-9]], np.float32)
+    s, s64 = oracle.smooth_scales(act_max, [W], 0.5)
+    eps = float(np.float32(1e-5))
+    assert np.all(s >= np.float32(1e-5))
+    # channel 0: both maxima clamp to eps -> s = eps^0.5 / eps^0.5 = 1
+    assert abs(s64[0] - 1.0) < 1e-15
+    # channel 2: w clamps to eps -> s = sqrt(5) / sqrt(eps)
+    assert abs(s64[2] - math.sqrt(5.0) / math.sqrt(eps)) < 1e-12 * s64[2]
+
+
+def test_calibration_running_max():
+    inp = S.make_inputs(S.OPT_QKV, rows=8, weights=False)
+    xc = inp.x_cal["attn_norm"]
+    g = inp.gamma["attn_norm"]
+    full = oracle.calibrate_absmax(xc, oracle.NORM_RMS, g)
+    run = oracle.calibrate_absmax(xc[:200], oracle.NORM_RMS, g)
+    run = oracle.calibrate_absmax(xc[200:], oracle.NORM_RMS, g, act_max=run)
+    assert np.array_equal(full, run)
+    x32 = torch.from_numpy(xc.view(np.int16)).view(torch.bfloat16).float().numpy()
+    ref = np.abs(_torch_norm64(x32, oracle.NORM_RMS, g, None, 1e-5)).max(axis=0)
+    assert np.all(np.abs(full - ref) <= 4 * _ulp32(ref))
+    ch, _ = S.outlier_channels(S.OPT_QKV, "attn_norm")
+    others = np.setdiff1d(np.arange(xc.shape[1]), ch)
+    assert full[ch].min() > 3 * full[others].max()  # the outlier channels stand out
+
+
+# --------------------------------------------------------------------------
+# the integer GEMM and the epilogue (steps 7/8)
+# --------------------------------------------------------------------------
+
+def test_gemm_brute_force():
+    for (M, N, K) in [(1, 1, 1), (3, 5, 7), (4, 6, 33)]:
+        A = RNG.integers(-127, 128, (M, K)).astype(np.int8)
+        B = RNG.integers(-127, 128, (N, K)).astype(np.int8)
+        acc = oracle.gemm_i64(A, B)
+        for m in range(M):
+            for n in range(N):
+                t = 0
+                for k in range(K):
+                    t += int(A[m, k]) * int(B[n, k])
+                assert acc[m, n] == t
+
+
+def test_gemm_matches_numpy_and_extremes():
+    M, N, K = 17, 29, 4112
+    A = RNG.integers(-127, 128, (M, K)).astype(np.int8)
+    B = RNG.integers(-127, 128, (N, K)).astype(np.int8)
+    assert np.array_equal(oracle.gemm_i64(A, B), A.astype(np.int64) @ B.astype(np.int64).T)
+    A[:] = -127
+    B[:] = -127
+    assert np.all(oracle.gemm_i64(A, B) == 127 * 127 * K)
+
+
+def test_epilogue_matches_float32_and_torch_bf16():
+    M, N = 9, 31
+    acc = RNG.integers(-(2 ** 31) + 1, 2 ** 31 - 1, (M, N)).astype(np.int64)
+    acc[0, :5] = [0, 1, -1, 2 ** 24 + 1, -(2 ** 24) - 3]
+    xs = (RNG.random(M) * 0.05).astype(np.float32)
+    ws = (RNG.random(N) * 0.002).astype(np.float32)
+    for relu in (False, True):
+        o32, out = oracle.epilogue(acc, xs, ws, relu)
+        ref = (acc.astype(np.float32) * xs[:, None]).astype(np.float32) * ws[None, :]
+        ref = ref.astype(np.float32)
+        if relu:
+            ref = np.maximum(ref, np.float32(0))
+        assert np.array_equal(o32, ref)
+        tb = torch.from_numpy(ref).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        assert np.array_equal(out, tb)
