@@ -1,0 +1,252 @@
+/*
+ * sq.h -- C ABI of the SmoothQuant W8A8 linear layer for NVIDIA B200 (sm_100a).
+ *
+ * What the library computes (source pages cited by title and section):
+ *
+ *   [SQ-depth] "SmoothQuant, in depth: where the scales fold, how calibration
+ *              feeds them, and a W8A8 pipeline you can ship"
+ *   [LLMint8]  "LLM.int8() and SmoothQuant"
+ *
+ *   1. calibration: per input channel j, the running max over calibration
+ *      tokens of |x_j| at a smoothed Linear's input ([SQ-depth] "The
+ *      calibration data flow");
+ *   2. smoothing factors s_j = max|X_j|^alpha / max|W_j|^(1-alpha), shared by
+ *      all Linears that read one norm, and the fold of 1/s into that norm's
+ *      gamma (and beta) ([LLMint8] "Fix 2" and "going deeper"; [SQ-depth]
+ *      "Where the scales go in a decoder block");
+ *   3. smoothed weights diag(s) W quantised to INT8 with one scale per output
+ *      channel ([LLMint8] "going deeper"; [SQ-depth] "Granularity");
+ *   4. at run time: the norm (carrying 1/s) and a per-token dynamic absmax
+ *      INT8 quantisation of its output ([SQ-depth] "Granularity");
+ *   5. an INT8 x INT8 GEMM with exact INT32 accumulation and an epilogue
+ *      out = acc * scale_token[i] * scale_channel[j] emitted as bf16
+ *      ([SQ-depth] "Granularity"; "The problem SmoothQuant solves").
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Layout: activations are row-major [M, K] (M tokens, K input channels) with
+ *   a row stride ld (elements); weights are nn.Linear-shaped row-major [N, K]
+ *   (N output channels); outputs are row-major [M, N] with stride ldo.
+ * - Memory: every tensor pointer is DEVICE memory owned by the caller.  Except
+ *   where a call says otherwise the library allocates nothing and frees
+ *   nothing.  Pointer arguments marked "host" are host memory read during the
+ *   call only.
+ * - Execution: every call enqueues work on `stream` (a cudaStream_t; NULL is
+ *   the legacy default stream) and returns without synchronising.  Calls keep
+ *   no state between them and may be made from several threads.
+ * - Arithmetic: rounding is IEEE round-to-nearest-even everywhere; INT8 codes
+ *   are symmetric, clamped to [-127, 127]; a row whose absmax is 0 gets scale 0
+ *   and codes 0.  Results are bit-identical from run to run.
+ * - Alignment: tensor base pointers must be 16-byte aligned and K, every ld
+ *   and ldo must keep rows 16-byte aligned (K % 16 == 0 for the INT8 tensors,
+ *   ld % 8 == 0 for bf16 rows, ld % 4 == 0 for fp32 rows); otherwise the call
+ *   returns SQ_ERR_ALIGNMENT and launches nothing.
+ * - Errors: arguments are checked on the host before anything is launched; a
+ *   failing call returns a non-zero sq_status and leaves its outputs
+ *   untouched.  Faults the GPU can only discover later (a pipeline wait that
+ *   ran out) are recorded in a device error word that sq_get_device_error()
+ *   reads.  No call aborts the process.
+ */
+#ifndef SQ_H_
+#define SQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SQ_OK = 0,
+  SQ_ERR_INVALID_ARG = 1,      /* NULL pointer, negative size, bad enum, ld < K */
+  SQ_ERR_UNSUPPORTED = 2,      /* dtype / shape this build does not handle */
+  SQ_ERR_ALIGNMENT = 3,        /* pointer or row stride not 16-byte aligned */
+  SQ_ERR_OVERFLOW_RISK = 4,    /* K so large that 127*127*K could overflow INT32 */
+  SQ_ERR_CUDA = 5,             /* a CUDA runtime call or launch failed */
+  SQ_ERR_PIPELINE_TIMEOUT = 6, /* a device-side wait gave up (read later) */
+  SQ_ERR_WORKSPACE = 7         /* workspace missing or smaller than required */
+} sq_status;
+
+typedef enum { SQ_F32 = 0, SQ_BF16 = 1 } sq_dtype;
+
+typedef enum { SQ_NORM_NONE = 0, SQ_NORM_RMS = 1, SQ_NORM_LAYER = 2 } sq_norm;
+
+typedef enum {
+  SQ_EPI_BF16 = 0,      /* out bf16 = bf16(fp32(fp32(float(acc) * xs[m]) * ws[n])) */
+  SQ_EPI_BF16_RELU = 1, /* the same with max(., 0) before the bf16 rounding */
+  SQ_EPI_I32_RAW = 2    /* out int32 = acc (no scaling; for exactness checks) */
+} sq_epilogue;
+
+/* Largest K for which |sum_k q_a q_b| <= 127*127*K fits in INT32. */
+#define SQ_MAX_K 133144
+
+/*
+ * sq_calibrate_absmax -- running per-channel absmax of the norm output.
+ * [SQ-depth] "The calibration data flow": record, for every smoothed Linear,
+ * the running maximum over all calibration tokens of |x_j| at its input,
+ * combining batches with an element-wise maximum.  The Linear's input is the
+ * output of its (unsmoothed) norm: y = norm(x; gamma, beta, eps).
+ *   x        device [M, K] with row stride ldx, fp32 or bf16 (dtype)
+ *   norm     SQ_NORM_RMS, SQ_NORM_LAYER, or SQ_NORM_NONE (y = x, or
+ *            y = x * gamma when gamma is given)
+ *   gamma    device [K] fp32, or NULL for gamma = 1
+ *   beta     device [K] fp32, or NULL for beta = 0 (LayerNorm only)
+ *   eps      norm epsilon, added to the mean square / variance in fp64
+ *   act_max  device [K] fp32, IN/OUT: act_max[j] = max(act_max[j],
+ *            max_m |y[m, j]|).  The caller zero-fills it before the first
+ *            batch.  M == 0 is a no-op.
+ * Errors: SQ_ERR_INVALID_ARG, SQ_ERR_ALIGNMENT, SQ_ERR_CUDA.
+ */
+sq_status sq_calibrate_absmax(const void* x, sq_dtype dtype, int64_t M, int64_t K,
+                              int64_t ldx, sq_norm norm, const float* gamma,
+                              const float* beta, float eps, float* act_max, void* stream);
+
+/*
+ * sq_compute_smooth_scales -- smoothing factors and the folded norm.
+ * [LLMint8] "going deeper": s_j = max_t|X_tj|^alpha / max|W_j|^(1-alpha);
+ * [SQ-depth] "Where the scales go in a decoder block": all Linears reading one
+ * norm share one s from the element-wise maximum of their weights, and gamma
+ * (and beta) are divided by s; [SQ-depth] "The calibration data flow": both
+ * maxima are clamped below at clamp_eps before the powers, s itself after.
+ *   act_max   device [K] fp32 (from sq_calibrate_absmax)
+ *   W         HOST array of num_w DEVICE pointers, weight l is [N[l], K]
+ *             row-major (stride K), all of one dtype
+ *   N         HOST array of num_w output sizes
+ *   alpha     migration strength in [0, 1]
+ *   clamp_eps lower clamp of both maxima and of s (1e-5 on the page)
+ *   gamma     device [K] fp32 norm weight, or NULL for gamma = 1 (a Linear
+ *             with no norm in front: gamma_folded = 1/s is then applied as a
+ *             per-channel multiplier by SQ_NORM_NONE)
+ *   beta      device [K] fp32 or NULL
+ *   s         device [K] fp32 OUT: fl32 of the fp64 value
+ *             max(max(a,eps)^alpha / max(w,eps)^(1-alpha), eps); it is also
+ *             used as scratch during the call
+ *   gamma_folded  device [K] fp32 OUT: fl32(gamma / s)
+ *   beta_folded   device [K] fp32 OUT or NULL: fl32(beta / s)
+ * Errors: SQ_ERR_INVALID_ARG (alpha outside [0,1], num_w < 1, ...),
+ *         SQ_ERR_ALIGNMENT, SQ_ERR_CUDA.
+ */
+sq_status sq_compute_smooth_scales(const float* act_max, const void* const* W,
+                                   const int64_t* N, int num_w, sq_dtype dtype, int64_t K,
+                                   double alpha, float clamp_eps, const float* gamma,
+                                   const float* beta, float* s, float* gamma_folded,
+                                   float* beta_folded, void* stream);
+
+/*
+ * sq_smooth_quantize_weights -- W-hat = W diag(s), INT8 per output channel.
+ * [LLMint8] "going deeper": W-hat = diag(s) W (column j of an nn.Linear
+ * weight times s_j), then quantised per channel; [SQ-depth] "Granularity":
+ * per-output-channel weight scales.
+ *   W      device [N, K] row stride ldw, fp32 or bf16
+ *   s      device [K] fp32, or NULL for an unsmoothed Linear (s = 1)
+ *   Wq     device [N, K] int8 OUT (dense, stride K)
+ *   w_scale device [N] fp32 OUT: fl32(max_k |W-hat[n,k]| / 127)
+ * Codes: Wq = clamp(rne(fl32(W-hat / w_scale)), -127, 127).
+ * Errors: SQ_ERR_INVALID_ARG, SQ_ERR_ALIGNMENT, SQ_ERR_CUDA.
+ */
+sq_status sq_smooth_quantize_weights(const void* W, sq_dtype dtype, int64_t N, int64_t K,
+                                     int64_t ldw, const float* s, int8_t* Wq, float* w_scale,
+                                     void* stream);
+
+/*
+ * sq_norm_smooth_quant_per_token -- fused norm (with the folded 1/s) and
+ * per-token dynamic absmax INT8 quantisation.
+ * [SQ-depth] "Where the scales go in a decoder block": the norm with gamma/s
+ * (and beta/s) emits X/s with no extra kernel; [SQ-depth] "Granularity":
+ * per-token dynamic activation scales; [LLMint8] "Try it": step = max / 127.
+ *   x        device [M, K] row stride ldx, fp32 or bf16
+ *   norm     SQ_NORM_RMS / SQ_NORM_LAYER, or SQ_NORM_NONE for a Linear with
+ *            no norm in front (y = x, or x * gamma_folded when given)
+ *   gamma_folded device [K] fp32 or NULL (= 1)
+ *   beta_folded  device [K] fp32 or NULL (= 0; LayerNorm only)
+ *   Xq       device [M, K] int8 OUT (dense, stride K)
+ *   x_scale  device [M] fp32 OUT: fl32(max_k |y[m,k]| / 127)
+ * Norm arithmetic: row sums of x and x^2 in fp64, then
+ *   RMS:  r = fl32(1 / sqrt(S2/K + eps));  y = fl32(fl32(x r) gamma)
+ *   LN:   mu = S1/K, var = max(0, S2/K - mu^2), r = fl32(1/sqrt(var + eps)),
+ *         y = fl32(fl32(fl32(fl32(x - fl32(mu)) r) gamma) + beta)
+ * (every fp64 step is one IEEE operation).
+ * Errors: SQ_ERR_INVALID_ARG, SQ_ERR_ALIGNMENT, SQ_ERR_UNSUPPORTED (K too
+ *         large for one CTA per row), SQ_ERR_CUDA.
+ */
+sq_status sq_norm_smooth_quant_per_token(const void* x, sq_dtype dtype, int64_t M, int64_t K,
+                                         int64_t ldx, sq_norm norm, const float* gamma_folded,
+                                         const float* beta_folded, float eps, int8_t* Xq,
+                                         float* x_scale, void* stream);
+
+/*
+ * sq_w8a8_gemm_workspace_size -- bytes of device workspace that
+ * sq_w8a8_gemm_dequant needs for this shape and split factor (0 when the
+ * chosen path needs none).  split_k = 0 asks for the automatic choice.
+ */
+size_t sq_w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int split_k);
+
+/*
+ * sq_w8a8_gemm_dequant -- INT8 x INT8 -> INT32 GEMM with the dequantising
+ * epilogue fused.
+ * [SQ-depth] "Granularity": the GEMM computes an INT32 accumulator and applies
+ * both scales in its epilogue, out = acc x scale_token[i] x scale_channel[j],
+ * before converting to BF16; "The problem SmoothQuant solves": both operands
+ * are 8-bit integers accumulated in INT32.
+ *   Xq       device [M, K] int8 (stride K)
+ *   Wq       device [N, K] int8 (stride K)
+ *   x_scale  device [M] fp32;  w_scale device [N] fp32 (ignored for I32_RAW)
+ *   epi      SQ_EPI_BF16, SQ_EPI_BF16_RELU (out is bf16 [M, N], stride ldo)
+ *            or SQ_EPI_I32_RAW (out is int32 [M, N], stride ldo)
+ *   workspace / ws_bytes  device scratch for split-K partial sums; at least
+ *            sq_w8a8_gemm_workspace_size(M, N, K, split_k) bytes when that is
+ *            non-zero, else may be NULL
+ *   path_hint 0 = automatic, 1 = prefill tiles (tokens on the MMA M side),
+ *            2 = decode tiles (weight rows on the MMA M side, M <= 256)
+ *   split_k  0 = automatic, else the number of K slices (decode path only;
+ *            the INT32 partial sums are added exactly, so the result does not
+ *            depend on it)
+ * Accumulation is exact for K <= SQ_MAX_K (else SQ_ERR_OVERFLOW_RISK).
+ * Errors: SQ_ERR_INVALID_ARG, SQ_ERR_ALIGNMENT, SQ_ERR_OVERFLOW_RISK,
+ *         SQ_ERR_WORKSPACE, SQ_ERR_UNSUPPORTED, SQ_ERR_CUDA.
+ */
+sq_status sq_w8a8_gemm_dequant(const int8_t* Xq, const int8_t* Wq, const float* x_scale,
+                               const float* w_scale, int64_t M, int64_t N, int64_t K,
+                               sq_epilogue epi, void* out, int64_t ldo, void* workspace,
+                               size_t ws_bytes, int path_hint, int split_k, void* stream);
+
+/*
+ * sq_linear_w8a8 -- the whole runtime layer: sq_norm_smooth_quant_per_token
+ * into Xq_scratch / xscale_scratch, then sq_w8a8_gemm_dequant (automatic
+ * path and split).
+ *   Xq_scratch     device [M, K] int8, caller-owned
+ *   xscale_scratch device [M] fp32, caller-owned
+ *   workspace      as for sq_w8a8_gemm_dequant with split_k = 0
+ * Errors: the union of the two calls'.
+ */
+sq_status sq_linear_w8a8(const void* x, sq_dtype dtype, int64_t M, int64_t K, int64_t ldx,
+                         sq_norm norm, const float* gamma_folded, const float* beta_folded,
+                         float eps, const int8_t* Wq, const float* w_scale, int64_t N,
+                         sq_epilogue epi, void* out, int64_t ldo, int8_t* Xq_scratch,
+                         float* xscale_scratch, void* workspace, size_t ws_bytes, void* stream);
+
+/* Human-readable name of a status code (static storage). */
+const char* sq_status_string(sq_status status);
+
+/*
+ * sq_get_device_error -- synchronises `stream`, then reads and clears the
+ * device error word of the current device.  Returns SQ_OK, or the first
+ * device-side error recorded since the last call (SQ_ERR_PIPELINE_TIMEOUT), or
+ * SQ_ERR_CUDA if the synchronisation itself failed.
+ */
+sq_status sq_get_device_error(void* stream);
+
+/*
+ * sq_set_wait_limit -- diagnostics: the number of polls after which a GEMM
+ * pipeline wait gives up, records SQ_ERR_PIPELINE_TIMEOUT and lets the kernel
+ * drain and return (default 0 = the built-in limit of about one second).
+ * Affects launches made after the call, from any thread.
+ */
+void sq_set_wait_limit(int64_t polls);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SQ_H_ */

@@ -1,0 +1,350 @@
+"""GPU (libsq.so through the C ABI) versus the CPU oracle, element by element.
+
+Stage tests feed both sides the same seeded inputs (for a later stage, the
+oracle's own upstream results); workload tests run the whole path on the GPU
+and the oracle on the full tensors (small workloads) or on sampled token rows
+(full-size workloads, which the GPU processes at full size in the same launch
+configuration as the benchmark).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from w8a8_int8_quantized_norm_b200 import pipeline, sq
+from w8a8_int8_quantized_norm_b200 import synthetic as S
+
+from _oracle_pipeline import forward_rows, prepare
+from _parity import (bf16_bits, bf16_ulp_diff, compare_rows_quant, norm_near_tie_rows,
+                     scale_near_tie_channels, to_gpu)
+
+pytestmark = pytest.mark.gpu
+
+RNG = np.random.default_rng(20261202)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    sq.lib()
+    yield
+    assert sq.get_device_error() == 0
+
+
+def _acts(M, K, dtype, outliers=3, scale=1.0):
+    x = RNG.standard_normal((M, K)).astype(np.float32) * np.float32(scale)
+    if K >= 8 and outliers:
+        ch = RNG.choice(K, size=min(outliers, K), replace=False)
+        x[:, ch] *= RNG.uniform(20, 100, ch.size).astype(np.float32)
+    return S.to_bf16_bits(x) if dtype == "bf16" else x
+
+
+# ---------------------------------------------------------------------------
+# K1: fused norm + per-token quantisation
+# ---------------------------------------------------------------------------
+
+SHAPES = [(1, 16), (3, 48), (17, 64), (129, 4112), (64, 8192), (5, 28672), (3, 36864),
+          (2, 40960)]
+KINDS = [("none", oracle.NORM_NONE, False), ("none_mult", oracle.NORM_NONE, True),
+         ("rms", oracle.NORM_RMS, True), ("rms_nogamma", oracle.NORM_RMS, False),
+         ("layer", oracle.NORM_LAYER, True)]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "%dx%d" % s)
+@pytest.mark.parametrize("kind", KINDS, ids=lambda k: k[0])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_norm_quant_matches_oracle(shape, kind, dtype):
+    M, K = shape
+    _, norm, with_params = kind
+    x = _acts(M, K, dtype)
+    if M >= 3:
+        x[1] = 0  # an all-zero row: scale 0, codes 0 (LayerNorm: y = beta)
+    g = RNG.uniform(0.5, 1.5, K).astype(np.float32) if with_params else None
+    b = (RNG.standard_normal(K) * 0.1).astype(np.float32) if (with_params and norm == oracle.NORM_LAYER) else None
+    Xq_o, xs_o = oracle.norm_quant(x, norm, g, b, 1e-5)
+    Xq_g, xs_g = sq.norm_smooth_quant_per_token(to_gpu(x), norm, None if g is None else to_gpu(g),
+                                                None if b is None else to_gpu(b), 1e-5)
+    tol = compare_rows_quant(Xq_g.cpu().numpy(), xs_g.cpu().numpy(), Xq_o, xs_o,
+                             norm_near_tie_rows(x, norm, 1e-5))
+    assert tol == 0
+
+
+def test_norm_quant_strided_rows_and_canaries():
+    M, K, ld = 33, 4096, 4096 + 64
+    big = S.to_bf16_bits(RNG.standard_normal((M, ld)).astype(np.float32))
+    x = np.ascontiguousarray(big[:, :K])
+    g = RNG.uniform(0.5, 1.5, K).astype(np.float32)
+    Xq_o, xs_o = oracle.norm_quant(x, oracle.NORM_RMS, g, None, 1e-5)
+    xg = to_gpu(big)[:, :K]
+    assert xg.stride(0) == ld
+    # outputs with guard regions around them
+    q_buf = torch.full((M + 2, K), 77, dtype=torch.int8, device="cuda")
+    s_buf = torch.full((M + 8,), -3.0, dtype=torch.float32, device="cuda")
+    Xq_g, xs_g = sq.norm_smooth_quant_per_token(xg, oracle.NORM_RMS, to_gpu(g), None, 1e-5,
+                                                Xq=q_buf[1:M + 1], x_scale=s_buf[4:M + 4])
+    assert torch.all(q_buf[0] == 77) and torch.all(q_buf[M + 1] == 77)
+    assert torch.all(s_buf[:4] == -3.0) and torch.all(s_buf[M + 4:] == -3.0)
+    compare_rows_quant(Xq_g.cpu().numpy(), xs_g.cpu().numpy(), Xq_o, xs_o,
+                       norm_near_tie_rows(x, oracle.NORM_RMS, 1e-5))
+
+
+def test_worked_example_row_on_gpu(golden_dir):
+    """The pages' 4096-wide row with outliers 45 and -60: step 60/127 on the GPU too."""
+    import json, os
+    g = json.load(open(os.path.join(golden_dir, "token_row_outliers.json")))
+    row = RNG.uniform(-2, 2, g["row_width"]).astype(np.float32)
+    for ch, v in g["outliers"].items():
+        row[int(ch)] = v
+    Xq, xs = sq.norm_smooth_quant_per_token(to_gpu(row[None, :]), oracle.NORM_NONE)
+    assert float(xs[0]) == float(np.float32(60.0) / np.float32(127.0))
+    q = Xq.cpu().numpy()[0]
+    mask = np.ones(row.size, bool)
+    mask[[int(c) for c in g["outliers"]]] = False
+    assert q[mask].min() >= -4 and q[mask].max() <= 4
+
+
+# ---------------------------------------------------------------------------
+# K2: calibration, smoothing factors + fold, weight smoothing + quantisation
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("kind", [oracle.NORM_NONE, oracle.NORM_RMS, oracle.NORM_LAYER])
+@pytest.mark.parametrize("K", [64, 4096, 9216])
+def test_calibration_running_max(kind, K):
+    g = RNG.uniform(0.5, 1.5, K).astype(np.float32)
+    b = (RNG.standard_normal(K) * 0.1).astype(np.float32) if kind == oracle.NORM_LAYER else None
+    x1, x2 = _acts(300, K, "bf16"), _acts(213, K, "bf16")
+    am_o = oracle.calibrate_absmax(x1, kind, g, b)
+    am_o = oracle.calibrate_absmax(x2, kind, g, b, act_max=am_o)
+    gg, bb = to_gpu(g), (to_gpu(b) if b is not None else None)
+    am_g = sq.calibrate_absmax(to_gpu(x1), kind, gg, bb)
+    am_g = sq.calibrate_absmax(to_gpu(x2), kind, gg, bb, act_max=am_g).cpu().numpy()
+    ties = norm_near_tie_rows(np.concatenate([x1, x2]), kind, 1e-5)
+    if not ties.any():
+        assert np.array_equal(am_g.view(np.uint32), am_o.view(np.uint32))
+    else:
+        assert np.all(np.abs(am_g - am_o) <= 2 * np.spacing(am_o))
+
+
+@pytest.mark.parametrize("alpha", [0.0, 0.5, 0.8, 1.0])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_smooth_scales_and_fold(alpha, dtype):
+    K = 4096
+    act_max = np.abs(RNG.standard_normal(K)).astype(np.float32) * 3
+    act_max[[5, 77, 300]] = [60.0, 0.0, 1e-7]
+    Ws = [(RNG.standard_normal((n, K)) * 0.02).astype(np.float32) for n in (1024, 512, 512)]
+    Ws[1][:, 9] = 0.0
+    Ws[0][:, 9] = 0.0
+    Ws[2][:, 9] = 0.0
+    if dtype == "bf16":
+        Ws = [S.to_bf16_bits(w) for w in Ws]
+    g = RNG.uniform(0.5, 1.5, K).astype(np.float32)
+    b = (RNG.standard_normal(K) * 0.1).astype(np.float32)
+    s_o, s64 = oracle.smooth_scales(act_max, Ws, alpha, 1e-5)
+    gf_o, bf_o = oracle.fold_norm(s_o, g, b)
+    s_g, gf_g, bf_g = sq.compute_smooth_scales(to_gpu(act_max), [to_gpu(w) for w in Ws], alpha,
+                                               1e-5, to_gpu(g), to_gpu(b))
+    s_g, gf_g, bf_g = s_g.cpu().numpy(), gf_g.cpu().numpy(), bf_g.cpu().numpy()
+    diff = s_g.view(np.uint32) != s_o.view(np.uint32)
+    ties = scale_near_tie_channels(s64)
+    assert not np.any(diff & ~ties), np.nonzero(diff & ~ties)[0][:10]
+    assert np.all(np.abs(s_g[diff] - s_o[diff]) <= np.spacing(s_o[diff]))
+    same = ~diff
+    assert np.array_equal(gf_g[same].view(np.uint32), gf_o[same].view(np.uint32))
+    assert np.array_equal(bf_g[same].view(np.uint32), bf_o[same].view(np.uint32))
+    # no norm in front: gamma = 1, gamma' = 1/s
+    _, gf1, bf1 = sq.compute_smooth_scales(to_gpu(act_max), [to_gpu(Ws[0])], alpha, 1e-5)
+    s1, _ = oracle.smooth_scales(act_max, [Ws[0]], alpha, 1e-5)
+    gfo1, _ = oracle.fold_norm(s1)
+    assert bf1 is None
+    assert np.array_equal(gf1.cpu().numpy().view(np.uint32), gfo1.view(np.uint32))
+
+
+@pytest.mark.parametrize("NK", [(1, 16), (7, 48), (300, 4096), (129, 4112), (64, 28672)])
+@pytest.mark.parametrize("smoothed", [True, False])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_weight_quant_matches_oracle(NK, smoothed, dtype):
+    N, K = NK
+    W = (RNG.standard_normal((N, K)) * 0.02).astype(np.float32)
+    if N > 3:
+        W[2] = 0.0
+    if dtype == "bf16":
+        W = S.to_bf16_bits(W)
+    s = RNG.uniform(0.05, 20.0, K).astype(np.float32) if smoothed else None
+    Wq_o, ws_o = oracle.quantize_weights(W, s)
+    Wq_g, ws_g = sq.smooth_quantize_weights(to_gpu(W), None if s is None else to_gpu(s))
+    assert np.array_equal(Wq_g.cpu().numpy(), Wq_o)
+    assert np.array_equal(ws_g.cpu().numpy().view(np.uint32), ws_o.view(np.uint32))
+
+
+# ---------------------------------------------------------------------------
+# K3 / K4: the INT8 GEMM and its epilogue
+# ---------------------------------------------------------------------------
+
+GEMM_SHAPES = [(16, 64, 64), (3, 5, 16), (1, 300, 48), (129, 257, 4112), (256, 512, 1024),
+               (200, 1000, 128), (300, 777, 160), (1024, 768, 2048)]
+
+
+def _codes(M, K, extreme=False):
+    if extreme:
+        return np.full((M, K), -127, np.int8)
+    return RNG.integers(-127, 128, (M, K)).astype(np.int8)
+
+
+@pytest.mark.parametrize("shape", GEMM_SHAPES, ids=lambda s: "%dx%dx%d" % s)
+@pytest.mark.parametrize("path", [1, 2])
+def test_gemm_int32_exact(shape, path):
+    M, N, K = shape
+    if path == 2 and M > 256:
+        pytest.skip("decode tiles take at most 256 tokens")
+    A, B = _codes(M, K), _codes(N, K)
+    acc_o = oracle.gemm_i64(A, B)
+    out = sq.w8a8_gemm_dequant(to_gpu(A), to_gpu(B), None, None, "i32", path_hint=path)
+    assert np.array_equal(out.cpu().numpy().astype(np.int64), acc_o)
+
+
+def test_gemm_int32_extremes_and_max_k():
+    # |acc| = 127*127*K at the largest K whose products fit INT32
+    K = sq.MAX_K // 16 * 16
+    A, B = _codes(3, K, extreme=True), _codes(130, K, extreme=True)
+    B[1] = 127
+    acc_o = oracle.gemm_i64(A, B)
+    assert acc_o.max() == 127 * 127 * K and acc_o.min() == -127 * 127 * K
+    for path in (1, 2):
+        out = sq.w8a8_gemm_dequant(to_gpu(A), to_gpu(B), None, None, "i32", path_hint=path)
+        assert np.array_equal(out.cpu().numpy().astype(np.int64), acc_o)
+
+
+@pytest.mark.parametrize("M", [1, 8, 32, 128])
+def test_split_k_invariance(M):
+    N, K = 640, 4096
+    A, B = _codes(M, K), _codes(N, K)
+    acc_o = oracle.gemm_i64(A, B)
+    for split in (1, 2, 4, 8):
+        out = sq.w8a8_gemm_dequant(to_gpu(A), to_gpu(B), None, None, "i32", path_hint=2,
+                                   split_k=split)
+        assert np.array_equal(out.cpu().numpy().astype(np.int64), acc_o), split
+
+
+@pytest.mark.parametrize("shape", [(16, 64, 64), (129, 257, 4112), (7, 1000, 512), (512, 384, 256)],
+                         ids=lambda s: "%dx%dx%d" % s)
+@pytest.mark.parametrize("relu", [False, True])
+@pytest.mark.parametrize("path", [1, 2])
+def test_gemm_bf16_epilogue(shape, relu, path):
+    M, N, K = shape
+    if path == 2 and M > 256:
+        pytest.skip("decode tiles take at most 256 tokens")
+    A, B = _codes(M, K), _codes(N, K)
+    xs = (RNG.random(M) * 0.05 + 1e-3).astype(np.float32)
+    ws = (RNG.random(N) * 0.002 + 1e-5).astype(np.float32)
+    acc = oracle.gemm_i64(A, B)
+    o32, out_o = oracle.epilogue(acc, xs, ws, relu)
+    ldo = N + 24 if (N + 24) % 8 == 0 else (N + 24 + 7) // 8 * 8
+    buf = torch.full((M, ldo), 1.5, dtype=torch.bfloat16, device="cuda")
+    view = buf[:, :N]
+    sq.w8a8_gemm_dequant(to_gpu(A), to_gpu(B), to_gpu(xs), to_gpu(ws),
+                         "bf16_relu" if relu else "bf16", out=view, path_hint=path)
+    assert torch.all(buf[:, N:] == 1.5)  # the padding columns are untouched
+    out_g = bf16_bits(view.contiguous())
+    assert bf16_ulp_diff(out_g, out_o).max() <= 1
+    assert np.array_equal(out_g, out_o)
+
+
+# ---------------------------------------------------------------------------
+# whole workloads
+# ---------------------------------------------------------------------------
+
+def _gpu_inputs(inp):
+    dev = lambda a: None if a is None else to_gpu(a)
+    return ({k: dev(v) for k, v in inp.x.items()}, {k: dev(v) for k, v in inp.x_cal.items()},
+            {k: dev(v) for k, v in inp.W.items()}, {k: dev(v) for k, v in inp.gamma.items()},
+            {k: dev(v) for k, v in inp.beta.items()})
+
+
+_FAMILY = {}
+
+
+def _family_state(w, seed=0):
+    """Weights, calibration and both sides' offline preparation, shared by
+    every workload drawn from the same weights (the decode sweep reuses the
+    prefill block's)."""
+    fam = S._family(w)
+    if fam not in _FAMILY:
+        _FAMILY.clear()
+        base = S.WORKLOADS[fam]
+        inp = S.make_inputs(base, seed=seed, rows=1)
+        _, xc, W, g, b = _gpu_inputs(inp)
+        prep_g = pipeline.prepare(base, xc, W, g, b)
+        del W, xc
+        torch.cuda.synchronize()
+        _FAMILY[fam] = (inp, prepare(base, inp), prep_g)
+    return _FAMILY[fam]
+
+
+def _check_workload(w, rows=None, seed=0):
+    inp_w, prep_o, prep_g = _family_state(w, seed)
+    inp = S.make_inputs(w, seed=seed, weights=False)
+    inp.W = inp_w.W
+    x = {k: to_gpu(v) for k, v in inp.x.items()}
+    fwd = pipeline.Forward(prep_g, w.M, "cuda")
+    out_g = fwd(x)
+    torch.cuda.synchronize()
+    # offline results: bit-exact on the full tensors
+    for site in w.sites:
+        so, sg = prep_o["sites"][site.name], prep_g.sites[site.name]
+        if site.smoothed:
+            ties = scale_near_tie_channels(so["s64"])
+            s_g = sg.s.cpu().numpy()
+            diff = s_g.view(np.uint32) != so["s"].view(np.uint32)
+            assert not np.any(diff & ~ties)
+            if diff.any():
+                pytest.skip("certified smoothing-factor near-tie: downstream not comparable")
+            assert np.array_equal(sg.act_max.cpu().numpy().view(np.uint32), so["act_max"].view(np.uint32))
+            assert np.array_equal(sg.gamma_folded.cpu().numpy().view(np.uint32), so["gamma_f"].view(np.uint32))
+    for lin in w.linears:
+        lo, lg = prep_o["linears"][lin.name], prep_g.linears[lin.name]
+        assert np.array_equal(lg.Wq.cpu().numpy(), lo["Wq"]), lin.name
+        assert np.array_equal(lg.w_scale.cpu().numpy().view(np.uint32), lo["w_scale"].view(np.uint32))
+    # runtime path on the chosen rows
+    rows = np.arange(w.M) if rows is None else np.asarray(rows)
+    res = forward_rows(w, prep_o, inp, rows)
+    idx = torch.from_numpy(rows).cuda()
+    for site in w.sites:
+        r = res["sites"][site.name]
+        Xq_g = fwd.xq[site.name][idx].cpu().numpy()
+        xs_g = fwd.xs[site.name][idx].cpu().numpy()
+        compare_rows_quant(Xq_g, xs_g, r["Xq"], r["xs"], norm_near_tie_rows(r["x"], site.norm, w.eps))
+    for lin in w.linears:
+        o = res["linears"][lin.name]
+        out_rows = bf16_bits(out_g[lin.name][idx].contiguous())
+        d = bf16_ulp_diff(out_rows, o["out"])
+        assert d.max() <= 1, (lin.name, int(d.max()))
+        assert np.array_equal(out_rows, o["out"]), lin.name
+    return fwd
+
+
+def test_workload_small_smoothed_linear():
+    _check_workload(S.SMALL)
+
+
+def test_workload_opt_prefill_qkv():
+    _check_workload(S.OPT_QKV)
+
+
+def _sample_rows(M, n=16, seed=7):
+    r = np.random.default_rng(seed)
+    rows = np.unique(np.concatenate([[0, M - 1], r.choice(M, size=min(n, M), replace=False)]))
+    return rows
+
+
+def test_workload_opt66b_mlp_sampled():
+    _check_workload(S.OPT66B_MLP, rows=_sample_rows(S.OPT66B_MLP.M))
+
+
+def test_workload_llama_block_prefill_sampled():
+    _check_workload(S.LLAMA_BLOCK, rows=_sample_rows(S.LLAMA_BLOCK.M, n=8))
+
+
+@pytest.mark.parametrize("M", [1, 8, 32, 128])
+def test_workload_llama_block_decode(M):
+    _check_workload(S.WORKLOADS["llama-block-8192-decode-m%d" % M])

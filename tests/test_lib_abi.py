@@ -1,0 +1,138 @@
+"""The C-ABI library loads, exports every symbol include/sq.h declares, and
+rejects bad arguments on the host before any launch (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from w8a8_int8_quantized_norm_b200 import build as sqbuild
+from w8a8_int8_quantized_norm_b200 import sq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sq.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    sqbuild.build()
+    return sq.lib()
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _declared()
+    assert len(names) >= 10
+    assert set(names) == set(sq.EXPORTS)
+    for n in names:
+        assert getattr(L, n) is not None
+
+
+def test_header_constants_match_binding():
+    text = open(HEADER).read()
+    for name, val in [("SQ_OK", 0), ("SQ_ERR_INVALID_ARG", 1), ("SQ_ERR_UNSUPPORTED", 2),
+                      ("SQ_ERR_ALIGNMENT", 3), ("SQ_ERR_OVERFLOW_RISK", 4), ("SQ_ERR_CUDA", 5),
+                      ("SQ_ERR_PIPELINE_TIMEOUT", 6), ("SQ_ERR_WORKSPACE", 7), ("SQ_F32", 0),
+                      ("SQ_BF16", 1), ("SQ_NORM_NONE", 0), ("SQ_NORM_RMS", 1),
+                      ("SQ_NORM_LAYER", 2), ("SQ_EPI_BF16", 0), ("SQ_EPI_BF16_RELU", 1),
+                      ("SQ_EPI_I32_RAW", 2)]:
+        assert re.search(r"\b%s\s*=\s*%d\b" % (name, val), text), name
+    assert re.search(r"#define SQ_MAX_K %d\b" % sq.MAX_K, text)
+    assert 127 * 127 * sq.MAX_K < 2 ** 31 <= 127 * 127 * (sq.MAX_K + 1)
+
+
+def test_status_strings(L):
+    for code, name in sq.STATUS_NAMES.items():
+        assert L.sq_status_string(code).decode().startswith(name)
+    assert b"unknown" in L.sq_status_string(99)
+
+
+# Fake, never-dereferenced device addresses: every call below must be rejected
+# by the host-side checks before it touches CUDA.
+A16 = ctypes.c_void_p(0x10000)
+A8 = ctypes.c_void_p(0x10008)
+
+
+def test_rows_calls_reject_bad_arguments(L):
+    f = L.sq_norm_smooth_quant_per_token
+    ok_args = dict(x=A16, dt=1, M=4, K=64, ld=64, norm=1, g=None, b=None, eps=1e-5, q=A16, s=A16)
+
+    def call(**kw):
+        a = dict(ok_args, **kw)
+        return f(a["x"], a["dt"], a["M"], a["K"], a["ld"], a["norm"], a["g"], a["b"], a["eps"],
+                 a["q"], a["s"], None)
+
+    assert call(dt=7) == 1
+    assert call(norm=9) == 1
+    assert call(M=-1) == 1
+    assert call(K=0) == 1
+    assert call(ld=32) == 1          # ld < K
+    assert call(x=None) == 1
+    assert call(q=None) == 1
+    assert call(s=None) == 1
+    assert call(eps=-1.0) == 1
+    assert call(K=40, ld=40) == 3    # K % 16
+    assert call(x=A8) == 3           # misaligned base
+    assert call(ld=68) == 3          # bf16 row stride not 16-byte multiple
+    assert call(q=A8) == 3
+    assert call(g=A8) == 3
+    assert call(K=65536 * 4, ld=65536 * 4) == 2  # row too wide for one CTA
+    c = L.sq_calibrate_absmax
+    assert c(A16, 1, 4, 64, 64, 1, None, None, 1e-5, None, None) == 1
+    assert c(A16, 1, 4, 64, 64, 5, None, None, 1e-5, A16, None) == 1
+    w = L.sq_smooth_quantize_weights
+    assert w(A16, 1, 4, 64, 64, None, None, A16, None) == 1
+    assert w(A16, 1, 4, 64, 64, A8, A16, A16, None) == 3
+
+
+def test_smooth_scales_rejects_bad_arguments(L):
+    f = L.sq_compute_smooth_scales
+    ptrs = (ctypes.c_void_p * 1)(0x10000)
+    ns = (ctypes.c_int64 * 1)(64)
+    P = ctypes.cast(ptrs, ctypes.c_void_p)
+    Nn = ctypes.cast(ns, ctypes.c_void_p)
+    assert f(A16, P, Nn, 1, 1, 64, 1.5, 1e-5, None, None, A16, A16, None, None) == 1  # alpha
+    assert f(A16, P, Nn, 1, 1, 64, -0.1, 1e-5, None, None, A16, A16, None, None) == 1
+    assert f(A16, P, Nn, 1, 1, 64, float("nan"), 1e-5, None, None, A16, A16, None, None) == 1
+    assert f(A16, P, Nn, 0, 1, 64, 0.5, 1e-5, None, None, A16, A16, None, None) == 1  # num_w
+    assert f(A16, P, Nn, 1, 1, 64, 0.5, 0.0, None, None, A16, A16, None, None) == 1   # eps
+    assert f(A16, None, Nn, 1, 1, 64, 0.5, 1e-5, None, None, A16, A16, None, None) == 1
+    assert f(A16, P, Nn, 1, 1, 64, 0.5, 1e-5, None, None, None, A16, None, None) == 1  # s
+    assert f(A8, P, Nn, 1, 1, 64, 0.5, 1e-5, None, None, A16, A16, None, None) == 3
+
+
+def test_gemm_rejects_bad_arguments(L):
+    f = L.sq_w8a8_gemm_dequant
+
+    def call(Xq=A16, Wq=A16, xs=A16, ws=A16, M=16, N=64, K=64, epi=0, out=A16, ldo=64,
+             wsp=None, wsb=0, path=0, split=0):
+        return f(Xq, Wq, xs, ws, M, N, K, epi, out, ldo, wsp, wsb, path, split, None)
+
+    assert call(M=-1) == 1
+    assert call(K=0) == 1
+    assert call(epi=5) == 1
+    assert call(path=3) == 1
+    assert call(split=-2) == 1
+    assert call(ldo=32) == 1
+    assert call(Xq=None) == 1
+    assert call(out=None) == 1
+    assert call(xs=None) == 1           # scales needed for the bf16 epilogue
+    assert call(K=sq.MAX_K + 16) == 4   # INT32 overflow risk
+    assert call(K=40) == 3
+    assert call(Wq=A8) == 3
+    assert call(ldo=68) == 3            # bf16 output rows not 16-byte aligned
+    assert call(ws=A8) == 3
+    assert call(path=2, M=300) == 2     # decode tiles take at most 256 tokens
+    # empty problems are valid no-ops that touch nothing
+    assert call(M=0, Xq=None, xs=None, out=None) == 0
+    assert call(N=0, ldo=0, Wq=None, ws=None, out=None) == 0
+
+
+def test_workspace_size_is_host_only_for_empty_shapes(L):
+    assert L.sq_w8a8_gemm_workspace_size(0, 10, 64, 0) == 0
+    assert L.sq_w8a8_gemm_workspace_size(10, 10, 64, -1) == 0

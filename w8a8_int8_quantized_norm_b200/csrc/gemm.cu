@@ -1,0 +1,589 @@
+// gemm.cu -- INT8 x INT8 -> INT32 GEMM with the fused dequantising epilogue,
+// written for the sm_100a tensor cores (tcgen05 + tensor memory + TMA).
+//
+// Source pages (by title and section): "SmoothQuant, in depth" --
+// "Granularity: O1, O2, O3 and what kernels run today" (an INT32 accumulator,
+// both scales applied in the epilogue, out = acc x scale_token[i] x
+// scale_channel[j], converted to BF16) and "The problem SmoothQuant solves"
+// (both operands 8-bit integers, INT32 accumulation); "SmoothQuant, in depth"
+// -- "Serving and operations" (prefill is compute-bound, small-batch decode is
+// memory-bound: it streams the INT8 weights once).
+//
+// One kernel template serves both regimes.  The MMA's M side ("P", 128 rows
+// per tile) and N side ("Q", BN rows per tile) are both K-major INT8 tiles:
+//   prefill: P = activation rows (tokens), Q = weight rows (channels), BN=256;
+//   decode:  P = weight rows, Q = the few token rows (BN = 16..256), so the
+//            weight stream fills the 128-row MMA and split-K spreads the
+//            weight bytes over all SMs; INT32 partial sums are added exactly
+//            by a second kernel.
+// Persistent CTAs (one per SM), warp-specialised:
+//   warp 0      TMA producer: 128-byte-swizzled K-major tiles into an
+//               mbarrier ring of STAGES stages (no cluster multicast);
+//   warp 1      allocates tensor memory and issues tcgen05.mma.kind::i8
+//               (one thread), committing each stage back to the producer and
+//               each finished tile to the epilogue;
+//   warps 2-5   epilogue: tcgen05.ld of the INT32 accumulator (double
+//               buffered in tensor memory, 2 x BN columns), the two scales,
+//               bf16 rounding and the global stores, overlapping the next
+//               tile's main loop.
+// Every mbarrier wait is bounded; a wait that runs out records
+// SQ_ERR_PIPELINE_TIMEOUT in the device error word, and the CTA drains its
+// outstanding TMA loads and MMAs, frees its tensor memory and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "sq_device.cuh"
+#include "sq_launch.h"
+
+namespace sq {
+namespace {
+
+constexpr int BM = 128;  // MMA M (rows of P per tile)
+constexpr int BK = 128;  // K bytes per stage = one 128-byte swizzle atom row
+constexpr int UMMA_K = 32;  // K of one kind::i8 MMA
+constexpr int kThreads = 192;
+
+template <int BN>
+struct Cfg {
+  static constexpr int A_BYTES = BM * BK;
+  static constexpr int B_BYTES = BN * BK;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES_FIT = (196 * 1024) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
+  static constexpr int TMEM_COLS =
+      2 * BN <= 32 ? 32 : 2 * BN <= 64 ? 64 : 2 * BN <= 128 ? 128 : 2 * BN <= 256 ? 256 : 512;
+  static constexpr int NUM_BARS = 2 * STAGES + 5;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 8 * NUM_BARS + 16;
+  static constexpr int CHUNK = BN < 32 ? BN : 32;  // accumulator columns per tcgen05.ld
+  static_assert(STAGES >= 2, "pipeline too shallow");
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "invalid MMA N for M = 128");
+};
+
+struct Params {
+  int P, Q, K;                     // rows on the MMA M side, rows on the N side, reduction
+  int p_blocks, q_blocks, k_blocks, splits, group, units;
+  const float* p_scale;            // scale per P row
+  const float* q_scale;            // scale per Q row
+  void* out;
+  int64_t ldo;
+  int epi;                         // SQ_EPI_*
+  int swap;                        // 0: out[p][q]; 1: out[q][p]
+  int32_t* partial;                // split-K: raw sums [split][M][N] (M = token extent)
+  int64_t wait_polls;              // > 0: poll budget per wait; 0: ~2 s by the global timer
+  int* error_word;                 // device error word of this device
+};
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait on an mbarrier phase; `abort` may be null.
+__device__ bool wait_phase(uint32_t bar, uint32_t parity, int64_t polls, const volatile int* abort) {
+  if (polls > 0) {
+    for (int64_t i = 0; i < polls; ++i) {
+      if (mbar_try_wait(bar, parity)) return true;
+      if (abort && *abort) return false;
+    }
+    return false;
+  }
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 0;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (abort && *abort) return false;
+    if ((i & 255u) == 255u && global_ns() - t0 > 2000000000ull) return false;
+  }
+}
+
+__device__ __forceinline__ void fail(int* word, volatile int* abort) {
+  record_device_error(word, SQ_ERR_PIPELINE_TIMEOUT);
+  *abort = 1;
+}
+
+__device__ __forceinline__ void decode_unit(const Params& p, int u, int& pb, int& qb, int& kb0,
+                                            int& kb1, int& split) {
+  split = u % p.splits;
+  const int tile = u / p.splits;
+  const int band_tiles = p.group * p.q_blocks;
+  const int band = tile / band_tiles;
+  const int rem = tile - band * band_tiles;
+  const int first = band * p.group;
+  const int gsize = min(p.group, p.p_blocks - first);
+  pb = first + rem % gsize;
+  qb = rem / gsize;
+  kb0 = static_cast<int>((static_cast<int64_t>(split) * p.k_blocks) / p.splits);
+  kb1 = static_cast<int>((static_cast<int64_t>(split + 1) * p.k_blocks) / p.splits);
+}
+
+// Epilogue for one CHUNK of accumulator columns held by this thread (row p of
+// the P side, columns q0 .. q0 + CHUNK - 1 of the Q side).
+template <int CHUNK>
+__device__ __forceinline__ void store_chunk(const Params& prm, const uint32_t (&r)[32], int p,
+                                            int q0, int split) {
+  if (p >= prm.P) return;
+  if (prm.partial) {  // split-K partial sums, [split][M][N] with M = Q (tokens), N = P
+#pragma unroll
+    for (int j = 0; j < CHUNK; ++j) {
+      const int q = q0 + j;
+      if (q < prm.Q)
+        prm.partial[(static_cast<int64_t>(split) * prm.Q + q) * prm.P + p] =
+            static_cast<int32_t>(r[j]);
+    }
+    return;
+  }
+  if (prm.epi == SQ_EPI_I32_RAW) {
+    int32_t* o = static_cast<int32_t*>(prm.out);
+    if (!prm.swap) {
+      int32_t* dst = o + static_cast<int64_t>(p) * prm.ldo + q0;
+      if (q0 + CHUNK <= prm.Q) {
+#pragma unroll
+        for (int j = 0; j < CHUNK; j += 4)
+          *reinterpret_cast<uint4*>(dst + j) = make_uint4(r[j], r[j + 1], r[j + 2], r[j + 3]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < CHUNK; ++j)
+          if (q0 + j < prm.Q) dst[j] = static_cast<int32_t>(r[j]);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < CHUNK; ++j)
+        if (q0 + j < prm.Q) o[static_cast<int64_t>(q0 + j) * prm.ldo + p] = static_cast<int32_t>(r[j]);
+    }
+    return;
+  }
+  const bool relu = prm.epi == SQ_EPI_BF16_RELU;
+  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(prm.out);
+  if (!prm.swap) {
+    // token scale for this row, channel scale per column
+    const float xs = __ldg(prm.p_scale + p);
+    float ws[CHUNK];
+    if (q0 + CHUNK <= prm.Q) {
+#pragma unroll
+      for (int j = 0; j < CHUNK; j += 4) {
+        const float4 t = __ldg(reinterpret_cast<const float4*>(prm.q_scale + q0 + j));
+        ws[j] = t.x; ws[j + 1] = t.y; ws[j + 2] = t.z; ws[j + 3] = t.w;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < CHUNK; ++j) ws[j] = (q0 + j < prm.Q) ? __ldg(prm.q_scale + q0 + j) : 0.0f;
+    }
+    float v[CHUNK];
+#pragma unroll
+    for (int j = 0; j < CHUNK; ++j) {
+      float t = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(r[j])), xs), ws[j]);
+      if (relu) t = fmaxf(t, 0.0f);
+      v[j] = t;
+    }
+    __nv_bfloat16* dst = o + static_cast<int64_t>(p) * prm.ldo + q0;
+    if (q0 + CHUNK <= prm.Q) {
+#pragma unroll
+      for (int j = 0; j < CHUNK; j += 8) {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const __nv_bfloat162 h = __floats2bfloat162_rn(v[j + 2 * i], v[j + 2 * i + 1]);
+          w[i] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        *reinterpret_cast<uint4*>(dst + j) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < CHUNK; ++j)
+        if (q0 + j < prm.Q) dst[j] = __float2bfloat16_rn(v[j]);
+    }
+  } else {
+    // channel scale for this row (weight row p), token scale per column
+    const float ws = __ldg(prm.p_scale + p);
+#pragma unroll
+    for (int j = 0; j < CHUNK; ++j) {
+      const int q = q0 + j;
+      if (q < prm.Q) {
+        const float xs = __ldg(prm.q_scale + q);
+        float t = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(r[j])), xs), ws);
+        if (relu) t = fmaxf(t, 0.0f);
+        o[static_cast<int64_t>(q) * prm.ldo + p] = __float2bfloat16_rn(t);
+      }
+    }
+  }
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+    w8a8_gemm_kernel(const __grid_constant__ CUtensorMap mapP,
+                     const __grid_constant__ CUtensorMap mapQ, const Params prm) {
+  using C = Cfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_u32 = smem_u32(smem_raw);
+  const uint32_t base = (raw_u32 + 1023u) & ~1023u;
+  uint8_t* base_ptr = smem_raw + (base - raw_u32);
+  const uint32_t a_base = base;
+  const uint32_t b_base = base + C::STAGES * C::A_BYTES;
+  const uint32_t bar_base = base + C::STAGES * C::STAGE_BYTES;
+  const uint32_t drain_bar = bar_base + 8u * (2 * C::STAGES + 4);
+  uint32_t* tmem_slot =
+      reinterpret_cast<uint32_t*>(base_ptr + C::STAGES * C::STAGE_BYTES + 8 * C::NUM_BARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+#define FULL_BAR(s) (bar_base + 8u * static_cast<uint32_t>(s))
+#define EMPTY_BAR(s) (bar_base + 8u * static_cast<uint32_t>(C::STAGES + (s)))
+#define TFULL_BAR(a) (bar_base + 8u * static_cast<uint32_t>(2 * C::STAGES + (a)))
+#define TEMPTY_BAR(a) (bar_base + 8u * static_cast<uint32_t>(2 * C::STAGES + 2 + (a)))
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(FULL_BAR(s), 1);
+      mbar_init(EMPTY_BAR(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(TFULL_BAR(a), 1);
+      mbar_init(TEMPTY_BAR(a), 4);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&mapP);
+    tma_prefetch_desc(&mapQ);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int64_t polls = prm.wait_polls;
+  int64_t producer_issued = 0;  // TMA stage loads issued (warp 0)
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    int stage = 0;
+    uint32_t phase = 0;
+    int64_t issued = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < prm.units && ok; u += gridDim.x) {
+      int pb, qb, kb0, kb1, split;
+      decode_unit(prm, u, pb, qb, kb0, kb1, split);
+      for (int kb = kb0; kb < kb1; ++kb) {
+        bool w = false;
+        if (lane == 0) w = wait_phase(EMPTY_BAR(stage), phase ^ 1u, polls, abort_flag);
+        w = __shfl_sync(0xffffffffu, w, 0);
+        if (!w) {
+          if (lane == 0) fail(prm.error_word, abort_flag);
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(FULL_BAR(stage), C::STAGE_BYTES);
+          tma_load_2d(a_base + stage * C::A_BYTES, &mapP, FULL_BAR(stage), kb * BK, pb * BM);
+          tma_load_2d(b_base + stage * C::B_BYTES, &mapQ, FULL_BAR(stage), kb * BK, qb * BN);
+        }
+        ++issued;
+        if (++stage == C::STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    producer_issued = issued;
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t kIdesc = idesc_i8(BM, BN);
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < prm.units && ok; u += gridDim.x) {
+      int pb, qb, kb0, kb1, split;
+      decode_unit(prm, u, pb, qb, kb0, kb1, split);
+      bool w = false;
+      if (lane == 0) w = wait_phase(TEMPTY_BAR(acc), acc_phase ^ 1u, polls, abort_flag);
+      w = __shfl_sync(0xffffffffu, w, 0);
+      if (!w) {
+        if (lane == 0) fail(prm.error_word, abort_flag);
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+      for (int kb = kb0; kb < kb1; ++kb) {
+        w = false;
+        if (lane == 0) w = wait_phase(FULL_BAR(stage), phase, polls, abort_flag);
+        w = __shfl_sync(0xffffffffu, w, 0);
+        if (!w) {
+          if (lane == 0) fail(prm.error_word, abort_flag);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t sa = a_base + stage * C::A_BYTES;
+          const uint32_t sb = b_base + stage * C::B_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+            mma_i8(d_tmem, smem_desc_k_sw128(sa + kk * UMMA_K), smem_desc_k_sw128(sb + kk * UMMA_K),
+                   kIdesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(EMPTY_BAR(stage));
+        }
+        __syncwarp();
+        if (++stage == C::STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      if (lane == 0) mma_commit(TFULL_BAR(acc));
+      __syncwarp();
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+    if (lane == 0) {
+      // every MMA issued by this thread completes before tensor memory is freed
+      mma_commit(drain_bar);
+      wait_phase(drain_bar, 0, 0, nullptr);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;  // tensor-memory lanes this warp may access
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int u = blockIdx.x; u < prm.units; u += gridDim.x) {
+      int pb, qb, kb0, kb1, split;
+      decode_unit(prm, u, pb, qb, kb0, kb1, split);
+      bool w = false;
+      if (lane == 0) w = wait_phase(TFULL_BAR(acc), acc_phase, polls, abort_flag);
+      w = __shfl_sync(0xffffffffu, w, 0);
+      if (!w) {
+        if (lane == 0) fail(prm.error_word, abort_flag);
+        break;
+      }
+      tc_fence_after();
+      const int p = pb * BM + quarter * 32 + lane;
+#pragma unroll 1
+      for (int c = 0; c < BN / C::CHUNK; ++c) {
+        uint32_t r[32];
+        __syncwarp();  // tcgen05.ld is .sync.aligned: the warp must be converged
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                               static_cast<uint32_t>(acc * BN + c * C::CHUNK);
+        if constexpr (C::CHUNK == 32)
+          tmem_ld_32x32b_x32(taddr, r);
+        else
+          tmem_ld_32x32b_x16(taddr, r);
+        tmem_wait_ld();
+        store_chunk<C::CHUNK>(prm, r, p, qb * BN + c * C::CHUNK, split);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(TEMPTY_BAR(acc));
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+  if (warp == 0 && lane == 0 && *abort_flag) {
+    // after an abort some issued TMA loads may not have been consumed: let
+    // every one of them land before the CTA releases its shared memory
+    for (int s = 0; s < C::STAGES; ++s) {
+      const int64_t n = producer_issued / C::STAGES + (s < producer_issued % C::STAGES ? 1 : 0);
+      if (n > 0) wait_phase(FULL_BAR(s), static_cast<uint32_t>((n - 1) & 1), 0, nullptr);
+    }
+  }
+#undef FULL_BAR
+#undef EMPTY_BAR
+#undef TFULL_BAR
+#undef TEMPTY_BAR
+}
+
+// out[m][n] = epilogue(sum_s partial[s][m][n]); INT32 addition is exact, so
+// the split does not change the result.
+__global__ void splitk_reduce_kernel(const int32_t* __restrict__ partial, int splits, int64_t M,
+                                     int64_t N, const float* __restrict__ x_scale,
+                                     const float* __restrict__ w_scale, int epi, void* out,
+                                     int64_t ldo) {
+  const int64_t total = M * N;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t m = i / N, n = i - m * N;
+    int32_t acc = 0;
+    for (int s = 0; s < splits; ++s) acc += partial[s * total + i];
+    if (epi == SQ_EPI_I32_RAW) {
+      static_cast<int32_t*>(out)[m * ldo + n] = acc;
+    } else {
+      float t = __fmul_rn(__fmul_rn(__int2float_rn(acc), x_scale[m]), w_scale[n]);
+      if (epi == SQ_EPI_BF16_RELU) t = fmaxf(t, 0.0f);
+      static_cast<__nv_bfloat16*>(out)[m * ldo + n] = __float2bfloat16_rn(t);
+    }
+  }
+}
+
+// --------------------------------------------------------------------------
+// host side
+// --------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// K-major INT8 matrix [rows, K] (row pitch K bytes), box = box_rows x 128
+// bytes, 128-byte swizzle, zero fill outside the matrix.
+bool make_map(CUtensorMap* map, const int8_t* ptr, int64_t rows, int64_t K, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+                        const_cast<void*>(static_cast<const void*>(ptr)), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN>
+cudaError_t launch_bn(const Params& prm, const CUtensorMap& mp, const CUtensorMap& mq, int grid,
+                      cudaStream_t st) {
+  using C = Cfg<BN>;
+  // the attribute is per device; setting it is cheap and idempotent
+  cudaError_t e = cudaFuncSetAttribute(w8a8_gemm_kernel<BN>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  w8a8_gemm_kernel<BN><<<grid, kThreads, C::SMEM_BYTES, st>>>(mp, mq, prm);
+  return cudaGetLastError();
+}
+
+int bn_for_tokens(int64_t M) {
+  return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
+}
+
+}  // namespace
+
+int num_sms_current_device() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int path_hint, int split_k, int num_sms) {
+  GemmPlan p{};
+  const int64_t kblocks = (K + BK - 1) / BK;
+  p.swap = (path_hint == 2 || (path_hint == 0 && M <= 128)) ? 1 : 0;
+  if (!p.swap) {
+    p.bn = 256;
+    p.splits = 1;
+  } else {
+    p.bn = bn_for_tokens(M);
+    const int64_t tiles = (N + BM - 1) / BM;
+    int splits = split_k;
+    if (splits <= 0) {
+      // pick the split that best fills the SMs, keeping the INT32 partial
+      // traffic (splits * M * N * 4 bytes) under a quarter of the weight bytes
+      const int64_t sms = num_sms > 0 ? num_sms : 148;
+      int64_t cap = K / (16 * (M > 0 ? M : 1));
+      if (cap > 8) cap = 8;
+      if (cap > kblocks) cap = kblocks;
+      if (cap < 1) cap = 1;
+      double best = -1.0;
+      splits = 1;
+      for (int64_t s = 1; s <= cap; ++s) {
+        const int64_t units = tiles * s;
+        const int64_t waves = (units + sms - 1) / sms;
+        const double eff = static_cast<double>(units) / static_cast<double>(waves * sms);
+        if (eff > best + 0.02) {
+          best = eff;
+          splits = static_cast<int>(s);
+        }
+      }
+    }
+    if (splits > kblocks) splits = static_cast<int>(kblocks > 0 ? kblocks : 1);
+    p.splits = splits < 1 ? 1 : splits;
+  }
+  p.workspace_bytes =
+      p.splits > 1 ? static_cast<size_t>(p.splits) * static_cast<size_t>(M) * static_cast<size_t>(N) * 4u
+                   : 0u;
+  return p;
+}
+
+cudaError_t launch_gemm(const GemmPlan& plan, const int8_t* Xq, const int8_t* Wq,
+                        const float* x_scale, const float* w_scale, int64_t M, int64_t N,
+                        int64_t K, int epi, void* out, int64_t ldo, void* workspace, int num_sms,
+                        int64_t wait_polls, int* error_word, cudaStream_t st) {
+  if (M == 0 || N == 0) return cudaSuccess;
+  Params prm{};
+  const int8_t* Pptr = plan.swap ? Wq : Xq;
+  const int8_t* Qptr = plan.swap ? Xq : Wq;
+  prm.P = static_cast<int>(plan.swap ? N : M);
+  prm.Q = static_cast<int>(plan.swap ? M : N);
+  prm.K = static_cast<int>(K);
+  prm.p_blocks = (prm.P + BM - 1) / BM;
+  prm.q_blocks = (prm.Q + plan.bn - 1) / plan.bn;
+  prm.k_blocks = static_cast<int>((K + BK - 1) / BK);
+  prm.splits = plan.splits;
+  prm.group = plan.swap ? 1 : 16;
+  prm.units = prm.p_blocks * prm.q_blocks * prm.splits;
+  prm.p_scale = plan.swap ? w_scale : x_scale;
+  prm.q_scale = plan.swap ? x_scale : w_scale;
+  prm.out = out;
+  prm.ldo = ldo;
+  prm.epi = epi;
+  prm.swap = plan.swap;
+  prm.partial = plan.splits > 1 ? static_cast<int32_t*>(workspace) : nullptr;
+  prm.wait_polls = wait_polls;
+  prm.error_word = error_word;
+
+  CUtensorMap mp, mq;
+  if (K == 0) return cudaErrorInvalidValue;
+  if (!make_map(&mp, Pptr, prm.P, K, BM) || !make_map(&mq, Qptr, prm.Q, K, plan.bn))
+    return cudaErrorInvalidValue;
+  const int sms = num_sms > 0 ? num_sms : 148;
+  const int grid = prm.units < sms ? prm.units : sms;
+  cudaError_t e;
+  switch (plan.bn) {
+    case 16: e = launch_bn<16>(prm, mp, mq, grid, st); break;
+    case 32: e = launch_bn<32>(prm, mp, mq, grid, st); break;
+    case 64: e = launch_bn<64>(prm, mp, mq, grid, st); break;
+    case 128: e = launch_bn<128>(prm, mp, mq, grid, st); break;
+    case 256: e = launch_bn<256>(prm, mp, mq, grid, st); break;
+    default: return cudaErrorInvalidValue;
+  }
+  if (e != cudaSuccess || plan.splits <= 1) return e;
+  const int64_t total = M * N;
+  int blocks = static_cast<int>((total + 255) / 256);
+  if (blocks > sms * 8) blocks = sms * 8;
+  splitk_reduce_kernel<<<blocks, 256, 0, st>>>(static_cast<const int32_t*>(workspace), plan.splits,
+                                               M, N, x_scale, w_scale, epi, out, ldo);
+  return cudaGetLastError();
+}
+
+}  // namespace sq

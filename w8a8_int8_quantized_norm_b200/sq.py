@@ -1,0 +1,271 @@
+"""Thin Python binding of ``libsq.so`` (include/sq.h).
+
+Argument marshalling only: every call checks the tensors it is given, turns
+them into device pointers and sizes, and calls the C ABI on the current torch
+CUDA stream.  Output tensors are allocated here with torch when the caller
+does not pass them; the library itself never allocates.  There is no CPU or
+PyTorch fallback: if the library is missing or a call fails, an exception is
+raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence, Tuple
+
+import torch
+
+from . import build as _build
+
+SQ_OK = 0
+STATUS_NAMES = {
+    0: "SQ_OK", 1: "SQ_ERR_INVALID_ARG", 2: "SQ_ERR_UNSUPPORTED", 3: "SQ_ERR_ALIGNMENT",
+    4: "SQ_ERR_OVERFLOW_RISK", 5: "SQ_ERR_CUDA", 6: "SQ_ERR_PIPELINE_TIMEOUT",
+    7: "SQ_ERR_WORKSPACE",
+}
+SQ_F32, SQ_BF16 = 0, 1
+NORM_NONE, NORM_RMS, NORM_LAYER = 0, 1, 2
+EPI = {"bf16": 0, "bf16_relu": 1, "i32": 2}
+MAX_K = 133144
+
+# Every symbol include/sq.h declares.
+EXPORTS = (
+    "sq_calibrate_absmax", "sq_compute_smooth_scales", "sq_smooth_quantize_weights",
+    "sq_norm_smooth_quant_per_token", "sq_w8a8_gemm_workspace_size", "sq_w8a8_gemm_dequant",
+    "sq_linear_w8a8", "sq_status_string", "sq_get_device_error", "sq_set_wait_limit",
+)
+
+
+class SQError(RuntimeError):
+    def __init__(self, status: int, call: str):
+        self.status = status
+        super().__init__("%s failed: %s" % (call, _status_text(status)))
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def lib() -> ctypes.CDLL:
+    """Load libsq.so (built in-tree); raises if it is not there."""
+    global _lib
+    if _lib is None:
+        path = library_path()
+        if not os.path.exists(path):
+            raise RuntimeError("libsq.so is not built (%s); run python -m "
+                               "w8a8_int8_quantized_norm_b200.build" % path)
+        L = ctypes.CDLL(path)
+        _declare(L)
+        _lib = L
+    return _lib
+
+
+_P, _I64, _I32, _F32, _F64, _SZ = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float,
+                                   ctypes.c_double, ctypes.c_size_t)
+
+
+def _declare(L):
+    L.sq_calibrate_absmax.argtypes = [_P, _I32, _I64, _I64, _I64, _I32, _P, _P, _F32, _P, _P]
+    L.sq_compute_smooth_scales.argtypes = [_P, _P, _P, _I32, _I32, _I64, _F64, _F32, _P, _P, _P,
+                                           _P, _P, _P]
+    L.sq_smooth_quantize_weights.argtypes = [_P, _I32, _I64, _I64, _I64, _P, _P, _P, _P]
+    L.sq_norm_smooth_quant_per_token.argtypes = [_P, _I32, _I64, _I64, _I64, _I32, _P, _P, _F32,
+                                                 _P, _P, _P]
+    L.sq_w8a8_gemm_workspace_size.argtypes = [_I64, _I64, _I64, _I32]
+    L.sq_w8a8_gemm_workspace_size.restype = _SZ
+    L.sq_w8a8_gemm_dequant.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _I32, _P, _I64, _P, _SZ,
+                                       _I32, _I32, _P]
+    L.sq_linear_w8a8.argtypes = [_P, _I32, _I64, _I64, _I64, _I32, _P, _P, _F32, _P, _P, _I64,
+                                 _I32, _P, _I64, _P, _P, _P, _SZ, _P]
+    L.sq_status_string.argtypes = [_I32]
+    L.sq_status_string.restype = ctypes.c_char_p
+    L.sq_get_device_error.argtypes = [_P]
+    L.sq_set_wait_limit.argtypes = [_I64]
+    L.sq_set_wait_limit.restype = None
+    for name in EXPORTS:
+        f = getattr(L, name)
+        if name not in ("sq_w8a8_gemm_workspace_size", "sq_status_string", "sq_set_wait_limit"):
+            f.restype = _I32
+
+
+def _status_text(status: int) -> str:
+    try:
+        return lib().sq_status_string(status).decode()
+    except Exception:  # the library may be what failed to load
+        return STATUS_NAMES.get(status, str(status))
+
+
+def _check(status: int, call: str):
+    if status != SQ_OK:
+        raise SQError(status, call)
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return SQ_BF16
+    if t.dtype == torch.float32:
+        return SQ_F32
+    raise TypeError("activations and weights are bf16 or fp32, got %s" % t.dtype)
+
+
+def _rows(t: torch.Tensor, name: str):
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError("%s must be 2-D with unit column stride" % name)
+    return t.shape[0], t.shape[1], t.stride(0)
+
+
+def _vec(t: Optional[torch.Tensor], K: int, name: str):
+    if t is None:
+        return None
+    if not (t.is_cuda and t.dtype == torch.float32 and t.dim() == 1 and t.numel() == K
+            and t.is_contiguous()):
+        raise ValueError("%s must be a contiguous fp32 CUDA vector of length %d" % (name, K))
+    return t
+
+
+# ---------------------------------------------------------------------------
+# the six calls of the C ABI
+# ---------------------------------------------------------------------------
+
+def calibrate_absmax(x: torch.Tensor, norm: int, gamma=None, beta=None, eps: float = 1e-5,
+                     act_max: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    M, K, ld = _rows(x, "x")
+    if act_max is None:
+        act_max = torch.zeros(K, dtype=torch.float32, device=x.device)
+    _vec(act_max, K, "act_max")
+    _check(lib().sq_calibrate_absmax(_ptr(x), _dtype_code(x), M, K, ld, norm,
+                                     _ptr(_vec(gamma, K, "gamma")), _ptr(_vec(beta, K, "beta")),
+                                     eps, _ptr(act_max), _stream(stream)), "sq_calibrate_absmax")
+    return act_max
+
+
+def compute_smooth_scales(act_max: torch.Tensor, weights: Sequence[torch.Tensor], alpha: float,
+                          clamp_eps: float = 1e-5, gamma=None, beta=None, stream=None
+                          ) -> Tuple[torch.Tensor, torch.Tensor, Optional[torch.Tensor]]:
+    K = act_max.numel()
+    _vec(act_max, K, "act_max")
+    dt = _dtype_code(weights[0])
+    for w in weights:
+        _rows(w, "W")
+        if not w.is_contiguous() or w.shape[1] != K or _dtype_code(w) != dt:
+            raise ValueError("weights must be contiguous [N, K] of one dtype")
+    ptrs = (ctypes.c_void_p * len(weights))(*[w.data_ptr() for w in weights])
+    ns = (ctypes.c_int64 * len(weights))(*[w.shape[0] for w in weights])
+    dev = act_max.device
+    s = torch.empty(K, dtype=torch.float32, device=dev)
+    gf = torch.empty(K, dtype=torch.float32, device=dev)
+    bf = torch.empty(K, dtype=torch.float32, device=dev) if beta is not None else None
+    _check(lib().sq_compute_smooth_scales(_ptr(act_max), ctypes.cast(ptrs, ctypes.c_void_p),
+                                          ctypes.cast(ns, ctypes.c_void_p), len(weights), dt, K,
+                                          float(alpha), clamp_eps, _ptr(_vec(gamma, K, "gamma")),
+                                          _ptr(_vec(beta, K, "beta")), _ptr(s), _ptr(gf), _ptr(bf),
+                                          _stream(stream)), "sq_compute_smooth_scales")
+    return s, gf, bf
+
+
+def smooth_quantize_weights(W: torch.Tensor, s: Optional[torch.Tensor] = None, Wq=None,
+                            w_scale=None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    N, K, ld = _rows(W, "W")
+    if Wq is None:
+        Wq = torch.empty((N, K), dtype=torch.int8, device=W.device)
+    if w_scale is None:
+        w_scale = torch.empty(N, dtype=torch.float32, device=W.device)
+    _check(lib().sq_smooth_quantize_weights(_ptr(W), _dtype_code(W), N, K, ld,
+                                            _ptr(_vec(s, K, "s")), _ptr(Wq), _ptr(w_scale),
+                                            _stream(stream)), "sq_smooth_quantize_weights")
+    return Wq, w_scale
+
+
+def norm_smooth_quant_per_token(x: torch.Tensor, norm: int, gamma_folded=None, beta_folded=None,
+                                eps: float = 1e-5, Xq=None, x_scale=None, stream=None
+                                ) -> Tuple[torch.Tensor, torch.Tensor]:
+    M, K, ld = _rows(x, "x")
+    if Xq is None:
+        Xq = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    if x_scale is None:
+        x_scale = torch.empty(M, dtype=torch.float32, device=x.device)
+    _check(lib().sq_norm_smooth_quant_per_token(
+        _ptr(x), _dtype_code(x), M, K, ld, norm, _ptr(_vec(gamma_folded, K, "gamma_folded")),
+        _ptr(_vec(beta_folded, K, "beta_folded")), eps, _ptr(Xq), _ptr(x_scale), _stream(stream)),
+        "sq_norm_smooth_quant_per_token")
+    return Xq, x_scale
+
+
+def gemm_workspace_size(M: int, N: int, K: int, split_k: int = 0) -> int:
+    return int(lib().sq_w8a8_gemm_workspace_size(M, N, K, split_k))
+
+
+def w8a8_gemm_dequant(Xq: torch.Tensor, Wq: torch.Tensor, x_scale: Optional[torch.Tensor],
+                      w_scale: Optional[torch.Tensor], epi: str = "bf16", out=None,
+                      path_hint: int = 0, split_k: int = 0, workspace=None, stream=None
+                      ) -> torch.Tensor:
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    if Xq.dtype != torch.int8 or Wq.dtype != torch.int8 or not Xq.is_contiguous() \
+            or not Wq.is_contiguous() or Wq.shape[1] != K:
+        raise ValueError("Xq [M,K] and Wq [N,K] must be contiguous int8")
+    code = EPI[epi]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.int32 if epi == "i32" else torch.bfloat16,
+                          device=Xq.device)
+    need = gemm_workspace_size(M, N, K, split_k)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=Xq.device)
+    wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().sq_w8a8_gemm_dequant(_ptr(Xq), _ptr(Wq), _ptr(x_scale), _ptr(w_scale), M, N, K,
+                                      code, _ptr(out), out.stride(0), _ptr(workspace), wsb,
+                                      path_hint, split_k, _stream(stream)),
+           "sq_w8a8_gemm_dequant")
+    return out
+
+
+def linear_w8a8(x: torch.Tensor, norm: int, gamma_folded, beta_folded, eps: float,
+                Wq: torch.Tensor, w_scale: torch.Tensor, epi: str = "bf16", out=None,
+                Xq_scratch=None, xscale_scratch=None, workspace=None, stream=None) -> torch.Tensor:
+    M, K, ld = _rows(x, "x")
+    N = Wq.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.int32 if epi == "i32" else torch.bfloat16,
+                          device=x.device)
+    if Xq_scratch is None:
+        Xq_scratch = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    if xscale_scratch is None:
+        xscale_scratch = torch.empty(M, dtype=torch.float32, device=x.device)
+    need = gemm_workspace_size(M, N, K, 0)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().sq_linear_w8a8(_ptr(x), _dtype_code(x), M, K, ld, norm,
+                                _ptr(_vec(gamma_folded, K, "gamma_folded")),
+                                _ptr(_vec(beta_folded, K, "beta_folded")), eps, _ptr(Wq),
+                                _ptr(w_scale), N, EPI[epi], _ptr(out), out.stride(0),
+                                _ptr(Xq_scratch), _ptr(xscale_scratch), _ptr(workspace), wsb,
+                                _stream(stream)), "sq_linear_w8a8")
+    return out
+
+
+def get_device_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device error word."""
+    return int(lib().sq_get_device_error(_stream(stream)))
+
+
+def set_wait_limit(polls: int) -> None:
+    lib().sq_set_wait_limit(int(polls))
+
+
+def status_string(status: int) -> str:
+    return _status_text(status)
