@@ -37,10 +37,13 @@
  * - Arithmetic: rounding is IEEE round-to-nearest-even everywhere; INT8 codes
  *   are symmetric, clamped to [-127, 127]; a row whose absmax is 0 gets scale 0
  *   and codes 0.  Results are bit-identical from run to run.
- * - Alignment: tensor base pointers must be 16-byte aligned and K, every ld
- *   and ldo must keep rows 16-byte aligned (K % 16 == 0 for the INT8 tensors,
- *   ld % 8 == 0 for bf16 rows, ld % 4 == 0 for fp32 rows); otherwise the call
- *   returns SQ_ERR_ALIGNMENT and launches nothing.
+ * - Alignment: input tensor and parameter-vector base pointers must be
+ *   16-byte aligned and K and every input row stride ld must keep rows 16-byte
+ *   aligned (K % 16 == 0 for the INT8 tensors, ld % 8 == 0 for bf16 rows,
+ *   ld % 4 == 0 for fp32 rows); otherwise the call returns SQ_ERR_ALIGNMENT
+ *   and launches nothing.  GEMM outputs need only element alignment: rows
+ *   that are 16-byte aligned are written with 128-bit stores, others element
+ *   by element.
  * - Errors: arguments are checked on the host before anything is launched; a
  *   failing call returns a non-zero sq_status and leaves its outputs
  *   untouched.  Faults the GPU can only discover later (a pipeline wait that

@@ -274,8 +274,7 @@ def _family_state(w, seed=0):
         base = S.WORKLOADS[fam]
         inp = S.make_inputs(base, seed=seed, rows=1)
         _, xc, W, g, b = _gpu_inputs(inp)
-        prep_g = pipeline.prepare(base, xc, W, g, b)
-        del W, xc
+        prep_g = {"xc": xc, "W": W, "g": g, "b": b}
         torch.cuda.synchronize()
         _FAMILY[fam] = (inp, prepare(base, inp), prep_g)
     return _FAMILY[fam]
@@ -286,33 +285,40 @@ def _check_workload(w, rows=None, seed=0):
     inp = S.make_inputs(w, seed=seed, weights=False)
     inp.W = inp_w.W
     x = {k: to_gpu(v) for k, v in inp.x.items()}
-    fwd = pipeline.Forward(prep_g, w.M, "cuda")
-    out_g = fwd(x)
+    blk = pipeline.Block(w, w.M, "cuda")
+    blk.prepare(prep_g["xc"], prep_g["W"], prep_g["g"], prep_g["b"])
+    out_g = blk.forward(x)
     torch.cuda.synchronize()
     # offline results: bit-exact on the full tensors
     for site in w.sites:
-        so, sg = prep_o["sites"][site.name], prep_g.sites[site.name]
+        so = prep_o["sites"][site.name]
         if site.smoothed:
             ties = scale_near_tie_channels(so["s64"])
-            s_g = sg.s.cpu().numpy()
+            s_g = blk.s[site.name].cpu().numpy()
             diff = s_g.view(np.uint32) != so["s"].view(np.uint32)
             assert not np.any(diff & ~ties)
             if diff.any():
                 pytest.skip("certified smoothing-factor near-tie: downstream not comparable")
-            assert np.array_equal(sg.act_max.cpu().numpy().view(np.uint32), so["act_max"].view(np.uint32))
-            assert np.array_equal(sg.gamma_folded.cpu().numpy().view(np.uint32), so["gamma_f"].view(np.uint32))
+            assert np.array_equal(blk.act_max[site.name].cpu().numpy().view(np.uint32),
+                                  so["act_max"].view(np.uint32))
+            assert np.array_equal(blk.gamma_f[site.name].cpu().numpy().view(np.uint32),
+                                  so["gamma_f"].view(np.uint32))
+            if so["beta_f"] is not None:
+                assert np.array_equal(blk.beta_f[site.name].cpu().numpy().view(np.uint32),
+                                      so["beta_f"].view(np.uint32))
     for lin in w.linears:
-        lo, lg = prep_o["linears"][lin.name], prep_g.linears[lin.name]
-        assert np.array_equal(lg.Wq.cpu().numpy(), lo["Wq"]), lin.name
-        assert np.array_equal(lg.w_scale.cpu().numpy().view(np.uint32), lo["w_scale"].view(np.uint32))
+        lo = prep_o["linears"][lin.name]
+        assert np.array_equal(blk.Wq[lin.name].cpu().numpy(), lo["Wq"]), lin.name
+        assert np.array_equal(blk.w_scale[lin.name].cpu().numpy().view(np.uint32),
+                              lo["w_scale"].view(np.uint32))
     # runtime path on the chosen rows
     rows = np.arange(w.M) if rows is None else np.asarray(rows)
     res = forward_rows(w, prep_o, inp, rows)
     idx = torch.from_numpy(rows).cuda()
     for site in w.sites:
         r = res["sites"][site.name]
-        Xq_g = fwd.xq[site.name][idx].cpu().numpy()
-        xs_g = fwd.xs[site.name][idx].cpu().numpy()
+        Xq_g = blk.xq[site.name][idx].cpu().numpy()
+        xs_g = blk.xs[site.name][idx].cpu().numpy()
         compare_rows_quant(Xq_g, xs_g, r["Xq"], r["xs"], norm_near_tie_rows(r["x"], site.norm, w.eps))
     for lin in w.linears:
         o = res["linears"][lin.name]
@@ -320,7 +326,7 @@ def _check_workload(w, rows=None, seed=0):
         d = bf16_ulp_diff(out_rows, o["out"])
         assert d.max() <= 1, (lin.name, int(d.max()))
         assert np.array_equal(out_rows, o["out"]), lin.name
-    return fwd
+    return blk
 
 
 def test_workload_small_smoothed_linear():

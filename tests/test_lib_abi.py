@@ -125,7 +125,7 @@ def test_gemm_rejects_bad_arguments(L):
     assert call(K=sq.MAX_K + 16) == 4   # INT32 overflow risk
     assert call(K=40) == 3
     assert call(Wq=A8) == 3
-    assert call(ldo=68) == 3            # bf16 output rows not 16-byte aligned
+    assert call(out=ctypes.c_void_p(0x10001)) == 3  # output not element aligned
     assert call(ws=A8) == 3
     assert call(path=2, M=300) == 2     # decode tiles take at most 256 tokens
     # empty problems are valid no-ops that touch nothing

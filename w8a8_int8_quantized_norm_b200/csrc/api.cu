@@ -80,9 +80,9 @@ sq_status check_gemm(const int8_t* Xq, const int8_t* Wq, const float* x_scale,
   if (K > SQ_MAX_K) return SQ_ERR_OVERFLOW_RISK;
   if (M > 0x7fffffff || N > 0x7fffffff) return SQ_ERR_UNSUPPORTED;
   if (path_hint == 2 && M > 256) return SQ_ERR_UNSUPPORTED;
-  const int64_t esz = epi == SQ_EPI_I32_RAW ? 4 : 2;
-  if (K % 16 != 0 || !aligned16(Xq) || !aligned16(Wq) || !aligned16(out) ||
-      (ldo * esz) % 16 != 0)
+  const uintptr_t esz = epi == SQ_EPI_I32_RAW ? 4 : 2;
+  if (K % 16 != 0 || !aligned16(Xq) || !aligned16(Wq) ||
+      (reinterpret_cast<uintptr_t>(out) % esz) != 0)
     return SQ_ERR_ALIGNMENT;
   if ((x_scale && !aligned16(x_scale)) || (w_scale && !aligned16(w_scale))) return SQ_ERR_ALIGNMENT;
   return SQ_OK;

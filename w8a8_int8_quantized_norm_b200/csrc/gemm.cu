@@ -75,6 +75,7 @@ struct Params {
   int32_t* partial;                // split-K: raw sums [split][M][N] (M = token extent)
   int64_t wait_polls;              // > 0: poll budget per wait; 0: ~2 s by the global timer
   int* error_word;                 // device error word of this device
+  int vec_out;                     // output rows 16-byte aligned: 128-bit stores allowed
 };
 
 __device__ __forceinline__ uint64_t global_ns() {
@@ -140,7 +141,7 @@ __device__ __forceinline__ void store_chunk(const Params& prm, const uint32_t (&
     int32_t* o = static_cast<int32_t*>(prm.out);
     if (!prm.swap) {
       int32_t* dst = o + static_cast<int64_t>(p) * prm.ldo + q0;
-      if (q0 + CHUNK <= prm.Q) {
+      if (prm.vec_out && q0 + CHUNK <= prm.Q) {
 #pragma unroll
         for (int j = 0; j < CHUNK; j += 4)
           *reinterpret_cast<uint4*>(dst + j) = make_uint4(r[j], r[j + 1], r[j + 2], r[j + 3]);
@@ -180,7 +181,7 @@ __device__ __forceinline__ void store_chunk(const Params& prm, const uint32_t (&
       v[j] = t;
     }
     __nv_bfloat16* dst = o + static_cast<int64_t>(p) * prm.ldo + q0;
-    if (q0 + CHUNK <= prm.Q) {
+    if (prm.vec_out && q0 + CHUNK <= prm.Q) {
 #pragma unroll
       for (int j = 0; j < CHUNK; j += 8) {
         uint32_t w[4];
@@ -561,6 +562,10 @@ cudaError_t launch_gemm(const GemmPlan& plan, const int8_t* Xq, const int8_t* Wq
   prm.partial = plan.splits > 1 ? static_cast<int32_t*>(workspace) : nullptr;
   prm.wait_polls = wait_polls;
   prm.error_word = error_word;
+  {
+    const int64_t esz = epi == SQ_EPI_I32_RAW ? 4 : 2;
+    prm.vec_out = ((reinterpret_cast<uintptr_t>(out) & 15u) == 0 && (ldo * esz) % 16 == 0) ? 1 : 0;
+  }
 
   CUtensorMap mp, mq;
   if (K == 0) return cudaErrorInvalidValue;

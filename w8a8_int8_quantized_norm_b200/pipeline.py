@@ -9,12 +9,11 @@ still quantised per token.  A Linear with no norm in front that *is* smoothed
 gets its 1/s as a per-channel multiplier (the fold with gamma = 1).
 
 Every arithmetic step runs in libsq.so; this module only sequences the calls
-and owns the device buffers (allocated once, reused by every forward).
+and owns the device buffers (allocated once, reused by every call).
 """
 from __future__ import annotations
 
-import dataclasses
-from typing import Dict, Optional
+from typing import Callable, Dict, Optional
 
 import torch
 
@@ -22,96 +21,120 @@ from . import sq
 from .synthetic import Workload
 
 
-@dataclasses.dataclass
-class SiteState:
-    norm: int
-    K: int
-    act_max: Optional[torch.Tensor] = None
-    s: Optional[torch.Tensor] = None
-    gamma_folded: Optional[torch.Tensor] = None
-    beta_folded: Optional[torch.Tensor] = None
+class Block:
+    """Device state of one workload for M tokens per forward.
 
+    ``prepare`` runs the offline rows (calibration, smoothing factors + fold,
+    weight smoothing + quantisation); ``forward`` the runtime rows (fused norm
+    + per-token quantisation, INT8 GEMM with the dequant epilogue).  Optional
+    ``around_gemm(fn)`` hooks let a caller bracket every GEMM launch (the
+    benchmark records CUDA events there)."""
 
-@dataclasses.dataclass
-class LinearState:
-    Wq: torch.Tensor
-    w_scale: torch.Tensor
-
-
-@dataclasses.dataclass
-class Prepared:
-    workload: Workload
-    sites: Dict[str, SiteState]
-    linears: Dict[str, LinearState]
-
-
-def prepare(w: Workload, x_cal: Dict[str, torch.Tensor], W: Dict[str, torch.Tensor],
-            gamma: Dict[str, Optional[torch.Tensor]], beta: Dict[str, Optional[torch.Tensor]],
-            stream=None) -> Prepared:
-    """Offline steps: calibrate every smoothed site, compute its s from the
-    weights of all Linears reading it, fold 1/s, smooth and quantise every
-    weight (unsmoothed Linears with s = 1)."""
-    sites: Dict[str, SiteState] = {}
-    for site in w.sites:
-        st = SiteState(norm=site.norm, K=site.K)
-        if site.smoothed:
-            g, b = gamma.get(site.name), beta.get(site.name)
-            st.act_max = sq.calibrate_absmax(x_cal[site.name], site.norm, g, b, w.eps,
-                                             stream=stream)
-            ws = [W[l.name] for l in w.linears_of(site.name)]
-            st.s, st.gamma_folded, st.beta_folded = sq.compute_smooth_scales(
-                st.act_max, ws, w.alpha, w.clamp_eps, g, b, stream=stream)
-        else:
-            st.gamma_folded, st.beta_folded = gamma.get(site.name), beta.get(site.name)
-        sites[site.name] = st
-    linears: Dict[str, LinearState] = {}
-    for lin in w.linears:
-        Wq, wsc = sq.smooth_quantize_weights(W[lin.name], sites[lin.site].s, stream=stream)
-        linears[lin.name] = LinearState(Wq, wsc)
-    return Prepared(w, sites, linears)
-
-
-class Forward:
-    """Runtime path with preallocated buffers for M tokens."""
-
-    def __init__(self, prep: Prepared, M: int, device, epi_raw: bool = False):
-        self.prep = prep
+    def __init__(self, w: Workload, M: int, device):
+        self.w = w
         self.M = M
-        w = prep.workload
-        self.xq: Dict[str, torch.Tensor] = {}
-        self.xs: Dict[str, torch.Tensor] = {}
+        dev = torch.device(device)
+        f32 = dict(dtype=torch.float32, device=dev)
+        self.act_max: Dict[str, torch.Tensor] = {}
+        self.s: Dict[str, Optional[torch.Tensor]] = {}
+        self.gamma_f: Dict[str, Optional[torch.Tensor]] = {}
+        self.beta_f: Dict[str, Optional[torch.Tensor]] = {}
+        self.has_beta: Dict[str, bool] = {}
+        for site in w.sites:
+            self.s[site.name] = None
+            self.gamma_f[site.name] = None
+            self.beta_f[site.name] = None
+            if site.smoothed:
+                self.act_max[site.name] = torch.zeros(site.K, **f32)
+                self.s[site.name] = torch.empty(site.K, **f32)
+                self.gamma_f[site.name] = torch.empty(site.K, **f32)
+        self.Wq: Dict[str, torch.Tensor] = {}
+        self.w_scale: Dict[str, torch.Tensor] = {}
         self.out: Dict[str, torch.Tensor] = {}
         self.ws: Dict[str, Optional[torch.Tensor]] = {}
-        for site in w.sites:
-            self.xq[site.name] = torch.empty((M, site.K), dtype=torch.int8, device=device)
-            self.xs[site.name] = torch.empty(M, dtype=torch.float32, device=device)
         for lin in w.linears:
-            self.out[lin.name] = torch.empty((M, lin.N), dtype=torch.bfloat16, device=device)
             K = w.site(lin.site).K
+            self.Wq[lin.name] = torch.empty((lin.N, K), dtype=torch.int8, device=dev)
+            self.w_scale[lin.name] = torch.empty(lin.N, **f32)
+            self.out[lin.name] = torch.empty((M, lin.N), dtype=torch.bfloat16, device=dev)
             need = sq.gemm_workspace_size(M, lin.N, K, 0)
-            self.ws[lin.name] = (torch.empty(need, dtype=torch.uint8, device=device)
-                                 if need else None)
+            self.ws[lin.name] = torch.empty(need, dtype=torch.uint8, device=dev) if need else None
+        self.xq: Dict[str, torch.Tensor] = {}
+        self.xs: Dict[str, torch.Tensor] = {}
+        for site in w.sites:
+            self.xq[site.name] = torch.empty((M, site.K), dtype=torch.int8, device=dev)
+            self.xs[site.name] = torch.empty(M, **f32)
 
-    def __call__(self, x: Dict[str, torch.Tensor], stream=None) -> Dict[str, torch.Tensor]:
-        w = self.prep.workload
+    # -- offline rows -------------------------------------------------------
+    def prepare(self, x_cal: Dict[str, torch.Tensor], W: Dict[str, torch.Tensor],
+                gamma: Dict[str, Optional[torch.Tensor]], beta: Dict[str, Optional[torch.Tensor]],
+                stream=None) -> "Block":
+        w = self.w
+        for site in w.sites:
+            g, b = gamma.get(site.name), beta.get(site.name)
+            if site.smoothed:
+                if b is not None and self.beta_f[site.name] is None:
+                    self.beta_f[site.name] = torch.empty_like(self.gamma_f[site.name])
+                am = self.act_max[site.name]
+                am.zero_()
+                sq.calibrate_absmax(x_cal[site.name], site.norm, g, b, w.eps, act_max=am,
+                                    stream=stream)
+                sq.compute_smooth_scales(am, [W[l.name] for l in w.linears_of(site.name)],
+                                         w.alpha, w.clamp_eps, g, b, s=self.s[site.name],
+                                         gamma_folded=self.gamma_f[site.name],
+                                         beta_folded=self.beta_f[site.name], stream=stream)
+            else:
+                self.gamma_f[site.name], self.beta_f[site.name] = g, b
+        for lin in w.linears:
+            sq.smooth_quantize_weights(W[lin.name], self.s[lin.site], Wq=self.Wq[lin.name],
+                                       w_scale=self.w_scale[lin.name], stream=stream)
+        return self
+
+    # -- runtime rows -------------------------------------------------------
+    def forward(self, x: Dict[str, torch.Tensor], stream=None,
+                around_gemm: Optional[Callable] = None) -> Dict[str, torch.Tensor]:
+        w = self.w
         for site in w.sites:
             src = next((l.source for l in w.linears if l.site == site.name and l.source), None)
             xin = self.out[src] if src else x[site.name]
-            st = self.prep.sites[site.name]
-            sq.norm_smooth_quant_per_token(xin, st.norm, st.gamma_folded, st.beta_folded, w.eps,
-                                           self.xq[site.name], self.xs[site.name], stream=stream)
+            sq.norm_smooth_quant_per_token(xin, site.norm, self.gamma_f[site.name],
+                                           self.beta_f[site.name], w.eps, self.xq[site.name],
+                                           self.xs[site.name], stream=stream)
             for lin in w.linears_of(site.name):
-                L = self.prep.linears[lin.name]
-                sq.w8a8_gemm_dequant(self.xq[site.name], L.Wq, self.xs[site.name], L.w_scale,
-                                     "bf16_relu" if lin.relu else "bf16", out=self.out[lin.name],
-                                     workspace=self.ws[lin.name], stream=stream)
+                def gemm(lin=lin, site=site):
+                    sq.w8a8_gemm_dequant(self.xq[site.name], self.Wq[lin.name],
+                                         self.xs[site.name], self.w_scale[lin.name],
+                                         "bf16_relu" if lin.relu else "bf16",
+                                         out=self.out[lin.name], workspace=self.ws[lin.name],
+                                         stream=stream)
+                if around_gemm is None:
+                    gemm()
+                else:
+                    around_gemm(lin, gemm)
         return self.out
 
-    def kernel_launches(self) -> int:
-        """Kernels one forward launches (norm-quant per site, GEMM per Linear,
-        plus the split-K reduction where the plan splits K)."""
-        w = self.prep.workload
-        n = len(w.sites)
-        for lin in w.linears:
+    # -- launch accounting ---------------------------------------------------
+    def prepare_launches(self) -> int:
+        """Kernels of this library one ``prepare`` launches: per smoothed site
+        calibration + one column-max per Linear reading it + the finalise
+        kernel; one weight-quantisation kernel per Linear."""
+        n = 0
+        for site in self.w.sites:
+            if site.smoothed:
+                n += 2 + len(self.w.linears_of(site.name))
+        return n + len(self.w.linears)
+
+    def forward_launches(self) -> int:
+        """Kernels one ``forward`` launches: norm-quant per site, the GEMM per
+        Linear, plus the split-K reduction where the plan splits K."""
+        n = len(self.w.sites)
+        for lin in self.w.linears:
             n += 2 if self.ws[lin.name] is not None else 1
         return n
+
+
+# Thin functional wrappers (used by tests and the smoke check).
+
+def prepare(w: Workload, x_cal, W, gamma, beta, M: Optional[int] = None, device="cuda",
+            stream=None) -> Block:
+    return Block(w, w.M if M is None else M, device).prepare(x_cal, W, gamma, beta, stream)

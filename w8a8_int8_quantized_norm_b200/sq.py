@@ -123,9 +123,11 @@ def _dtype_code(t: torch.Tensor) -> int:
 def _rows(t: torch.Tensor, name: str):
     if not t.is_cuda:
         raise ValueError("%s must be a CUDA tensor" % name)
-    if t.dim() != 2 or t.stride(1) != 1:
+    if t.dim() != 2 or (t.stride(1) != 1 and t.shape[1] > 1):
         raise ValueError("%s must be 2-D with unit column stride" % name)
-    return t.shape[0], t.shape[1], t.stride(0)
+    # a single row's stride is arbitrary (numpy / torch may report 0 for it)
+    ld = t.stride(0) if t.shape[0] > 1 else t.shape[1]
+    return t.shape[0], t.shape[1], ld
 
 
 def _vec(t: Optional[torch.Tensor], K: int, name: str):
@@ -154,7 +156,8 @@ def calibrate_absmax(x: torch.Tensor, norm: int, gamma=None, beta=None, eps: flo
 
 
 def compute_smooth_scales(act_max: torch.Tensor, weights: Sequence[torch.Tensor], alpha: float,
-                          clamp_eps: float = 1e-5, gamma=None, beta=None, stream=None
+                          clamp_eps: float = 1e-5, gamma=None, beta=None, s=None,
+                          gamma_folded=None, beta_folded=None, stream=None
                           ) -> Tuple[torch.Tensor, torch.Tensor, Optional[torch.Tensor]]:
     K = act_max.numel()
     _vec(act_max, K, "act_max")
@@ -166,9 +169,13 @@ def compute_smooth_scales(act_max: torch.Tensor, weights: Sequence[torch.Tensor]
     ptrs = (ctypes.c_void_p * len(weights))(*[w.data_ptr() for w in weights])
     ns = (ctypes.c_int64 * len(weights))(*[w.shape[0] for w in weights])
     dev = act_max.device
-    s = torch.empty(K, dtype=torch.float32, device=dev)
-    gf = torch.empty(K, dtype=torch.float32, device=dev)
-    bf = torch.empty(K, dtype=torch.float32, device=dev) if beta is not None else None
+    s = torch.empty(K, dtype=torch.float32, device=dev) if s is None else _vec(s, K, "s")
+    gf = (torch.empty(K, dtype=torch.float32, device=dev) if gamma_folded is None
+          else _vec(gamma_folded, K, "gamma_folded"))
+    bf = None
+    if beta is not None:
+        bf = (torch.empty(K, dtype=torch.float32, device=dev) if beta_folded is None
+              else _vec(beta_folded, K, "beta_folded"))
     _check(lib().sq_compute_smooth_scales(_ptr(act_max), ctypes.cast(ptrs, ctypes.c_void_p),
                                           ctypes.cast(ns, ctypes.c_void_p), len(weights), dt, K,
                                           float(alpha), clamp_eps, _ptr(_vec(gamma, K, "gamma")),
