@@ -229,6 +229,41 @@ sq_status sq_linear_w8a8(const void* x, sq_dtype dtype, int64_t M, int64_t K, in
                          sq_epilogue epi, void* out, int64_t ldo, int8_t* Xq_scratch,
                          float* xscale_scratch, void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * sq_w8a8_gemm_dequant_noalloc -- sq_w8a8_gemm_dequant for callers that cannot
+ * allocate device memory when they call it.  (This entry point is an
+ * engineering addition: the source pages have no counterpart.)
+ *
+ * Who needs it: code whose launch path may not allocate -- for example a
+ * plugin inside an inference engine that owns all device memory, where a
+ * cudaMalloc / cudaFree would also synchronise the device, or a serving loop
+ * whose memory was reserved up front by a framework's allocator.
+ *
+ * It takes the same arguments as sq_w8a8_gemm_dequant minus the workspace.
+ * The split-K partial sums go to a scratch array owned by the library: a
+ * static device array of SQ_NOALLOC_SCRATCH_BYTES that every GPU which loads
+ * the library keeps until the process exits.  This call allocates nothing
+ * and calls no allocating routine.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - All calls share the one array: calls whose kernels overlap on the GPU
+ *     (different streams, or different host threads) race on it.  Calls in
+ *     one stream are ordered and safe.  No state carries over between calls:
+ *     every partial sum is written before it is read.
+ *   - If the chosen plan needs more split-K scratch than
+ *     SQ_NOALLOC_SCRATCH_BYTES (sq_w8a8_gemm_workspace_size tells), the call
+ *     returns SQ_ERR_WORKSPACE and launches nothing; pass split_k = 1 (no
+ *     scratch) or a smaller split.
+ * Results are bit-identical to sq_w8a8_gemm_dequant's for the same plan.
+ * Errors: those of sq_w8a8_gemm_dequant.
+ */
+#define SQ_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+sq_status sq_w8a8_gemm_dequant_noalloc(const int8_t* Xq, const int8_t* Wq,
+                                       const float* x_scale, const float* w_scale, int64_t M,
+                                       int64_t N, int64_t K, sq_epilogue epi, void* out,
+                                       int64_t ldo, int path_hint, int split_k, void* stream);
+
 /* Human-readable name of a status code (static storage). */
 const char* sq_status_string(sq_status status);
 

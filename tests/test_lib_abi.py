@@ -43,6 +43,8 @@ def test_header_constants_match_binding():
                       ("SQ_EPI_I32_RAW", 2)]:
         assert re.search(r"\b%s\s*=\s*%d\b" % (name, val), text), name
     assert re.search(r"#define SQ_MAX_K %d\b" % sq.MAX_K, text)
+    assert re.search(r"#define SQ_NOALLOC_SCRATCH_BYTES \(8u << 20\)", text)
+    assert sq.NOALLOC_SCRATCH_BYTES == 8 << 20
     assert 127 * 127 * sq.MAX_K < 2 ** 31 <= 127 * 127 * (sq.MAX_K + 1)
 
 

@@ -1,0 +1,74 @@
+// noalloc.cu -- an entry point of the INT8 GEMM that never allocates.
+//
+// sq_w8a8_gemm_dequant asks its caller for a split-K workspace.  Some callers
+// cannot provide one on demand: a plugin inside an inference engine whose
+// enqueue path may not allocate (the engine owns the device memory, and
+// cudaMalloc / cudaFree can synchronise the whole device), or a serving loop
+// whose memory has been reserved up front by a framework's caching allocator.
+// sq_w8a8_gemm_dequant_noalloc serves them: its split-K partial sums live in a
+// fixed array of device memory that belongs to the library itself.
+//
+// The array is a file-scope __device__ variable, so every GPU that loads the
+// library holds SQ_NOALLOC_SCRATCH_BYTES of it until the process exits.  Host
+// code cannot use the array's name as a device address; the address is looked
+// up once per device with cudaGetSymbolAddress, with that device current, on
+// the first call made on it.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "../../include/sq.h"
+#include "sq_launch.h"
+
+// The library's own split-K scratch: one copy per device, for the life of the
+// process.  Nothing needs to start at zero (every partial sum a call reads was
+// written earlier in the same call).
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SQ_NOALLOC_SCRATCH_BYTES];
+
+namespace sq {
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+// Device address of the scratch array for the current device (set up on the
+// first call on that device); nullptr if the lookup failed.
+void* scratch_address() {
+  static void* addr[kMaxDevices] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    addr[dev] = p;
+  }
+  return addr[dev];
+}
+
+}  // namespace
+}  // namespace sq
+
+extern "C" sq_status sq_w8a8_gemm_dequant_noalloc(const int8_t* Xq, const int8_t* Wq,
+                                                  const float* x_scale, const float* w_scale,
+                                                  int64_t M, int64_t N, int64_t K,
+                                                  sq_epilogue epi, void* out, int64_t ldo,
+                                                  int path_hint, int split_k, void* stream) {
+  using namespace sq;
+  if (M < 0 || N < 0 || K <= 0 || split_k < 0 || path_hint < 0 || path_hint > 2)
+    return SQ_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) {
+    return sq_w8a8_gemm_dequant(Xq, Wq, x_scale, w_scale, M, N, K, epi, out, ldo, nullptr, 0,
+                                path_hint, split_k, stream);
+  }
+  const int sms = num_sms_current_device();
+  const GemmPlan plan = plan_gemm(M, N, K, path_hint, split_k, sms);
+  if (plan.workspace_bytes > SQ_NOALLOC_SCRATCH_BYTES) return SQ_ERR_WORKSPACE;
+  void* scratch = plan.workspace_bytes > 0 ? scratch_address() : nullptr;
+  if (plan.workspace_bytes > 0 && !scratch) return SQ_ERR_CUDA;
+  // the allocating entry point does the remaining checks and the launches;
+  // the library's own array stands in for the caller's workspace
+  return sq_w8a8_gemm_dequant(Xq, Wq, x_scale, w_scale, M, N, K, epi, out, ldo, scratch,
+                              scratch ? SQ_NOALLOC_SCRATCH_BYTES : 0, path_hint, split_k, stream);
+}

@@ -33,7 +33,9 @@ EXPORTS = (
     "sq_calibrate_absmax", "sq_compute_smooth_scales", "sq_smooth_quantize_weights",
     "sq_norm_smooth_quant_per_token", "sq_w8a8_gemm_workspace_size", "sq_w8a8_gemm_dequant",
     "sq_linear_w8a8", "sq_status_string", "sq_get_device_error", "sq_set_wait_limit",
+    "sq_w8a8_gemm_dequant_noalloc",
 )
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 class SQError(RuntimeError):
@@ -78,6 +80,8 @@ def _declare(L):
     L.sq_w8a8_gemm_workspace_size.restype = _SZ
     L.sq_w8a8_gemm_dequant.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _I32, _P, _I64, _P, _SZ,
                                        _I32, _I32, _P]
+    L.sq_w8a8_gemm_dequant_noalloc.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _I32, _P, _I64,
+                                               _I32, _I32, _P]
     L.sq_linear_w8a8.argtypes = [_P, _I32, _I64, _I64, _I64, _I32, _P, _P, _F32, _P, _P, _I64,
                                  _I32, _P, _I64, _P, _P, _P, _SZ, _P]
     L.sq_status_string.argtypes = [_I32]
@@ -237,6 +241,25 @@ def w8a8_gemm_dequant(Xq: torch.Tensor, Wq: torch.Tensor, x_scale: Optional[torc
                                       code, _ptr(out), out.stride(0), _ptr(workspace), wsb,
                                       path_hint, split_k, _stream(stream)),
            "sq_w8a8_gemm_dequant")
+    return out
+
+
+def w8a8_gemm_dequant_noalloc(Xq: torch.Tensor, Wq: torch.Tensor,
+                              x_scale: Optional[torch.Tensor], w_scale: Optional[torch.Tensor],
+                              out: torch.Tensor, epi: str = "bf16", path_hint: int = 0,
+                              split_k: int = 0, stream=None) -> torch.Tensor:
+    """The GEMM for callers that cannot allocate: the caller passes every input
+    and the output; split-K scratch comes from the library's own fixed array
+    (see include/sq.h).  Calls that overlap on the GPU share that array."""
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    if Xq.dtype != torch.int8 or Wq.dtype != torch.int8 or not Xq.is_contiguous() \
+            or not Wq.is_contiguous() or Wq.shape[1] != K:
+        raise ValueError("Xq [M,K] and Wq [N,K] must be contiguous int8")
+    _check(lib().sq_w8a8_gemm_dequant_noalloc(_ptr(Xq), _ptr(Wq), _ptr(x_scale), _ptr(w_scale),
+                                              M, N, K, EPI[epi], _ptr(out), out.stride(0),
+                                              path_hint, split_k, _stream(stream)),
+           "sq_w8a8_gemm_dequant_noalloc")
     return out
 
 
