@@ -21,7 +21,6 @@ import json
 import os
 import re
 import statistics
-import subprocess
 import sys
 import time
 
@@ -95,49 +94,54 @@ def _sample_rows(n, k, seed=11):
     return np.sort(np.random.default_rng(seed).choice(n, size=k, replace=False))
 
 
-def oracle_sample_step(w, inp, token_rows=16, weight_elems=48 << 20):
-    """One oracle step on a bounded sample.  Offline rows run on the full
-    calibration batch and on a sample of weight rows (all rows when the
-    weights are small); the runtime rows on `token_rows` sampled tokens.
+def oracle_sample_step(w, inp, cal_rows=512, weight_elems=48 << 20, token_rows=16):
+    """One oracle step on a bounded sample: `cal_rows` calibration tokens, up
+    to `weight_elems` weight elements per Linear (whole rows) and `token_rows`
+    runtime tokens.  Each phase's time is scaled linearly to the full workload.
     Returns (extrapolated seconds for the full step, seconds spent, text)."""
     import oracle
     spent = 0.0
     full = 0.0
     prep = {}
-    wfrac = {}
+
+    def wrows(Wl):
+        n = max(1, min(Wl.shape[0], weight_elems // Wl.shape[1]))
+        return _sample_rows(Wl.shape[0], n)
+
     for site in w.sites:
         g, b = inp.gamma[site.name], inp.beta[site.name]
         s = None
         gf, bf = g, b
         if site.smoothed:
-            t0 = time.perf_counter()
-            am = oracle.calibrate_absmax(inp.x_cal[site.name], site.norm, g, b, w.eps)
-            Ws = []
-            fr = []
+            xc = inp.x_cal[site.name]
+            cr = _sample_rows(xc.shape[0], cal_rows)
+            xcs = np.ascontiguousarray(xc[cr])
+            Ws, fr = [], []
             for l in w.linears_of(site.name):
                 Wl = inp.W[l.name]
-                n = max(1, min(Wl.shape[0], weight_elems // Wl.shape[1]))
-                Ws.append(np.ascontiguousarray(Wl[_sample_rows(Wl.shape[0], n)]))
-                fr.append(n / Wl.shape[0])
+                r = wrows(Wl)
+                Ws.append(np.ascontiguousarray(Wl[r]))
+                fr.append(len(r) / Wl.shape[0])
+            t0 = time.perf_counter()
+            am = oracle.calibrate_absmax(xcs, site.norm, g, b, w.eps)
             t1 = time.perf_counter()
             s, _ = oracle.smooth_scales(am, Ws, w.alpha, w.clamp_eps)
             gf, bf = oracle.fold_norm(s, g, b)
             t2 = time.perf_counter()
             spent += t2 - t0
-            full += (t1 - t0) + (t2 - t1) / max(min(fr), 1e-12)
+            full += (t1 - t0) * xc.shape[0] / len(cr) + (t2 - t1) / min(fr)
         prep[site.name] = (s, gf, bf)
     lin_q = {}
     for lin in w.linears:
         Wl = inp.W[lin.name]
-        n = max(1, min(Wl.shape[0], weight_elems // Wl.shape[1]))
-        rows = _sample_rows(Wl.shape[0], n)
-        Wsub = np.ascontiguousarray(Wl[rows])
+        r = wrows(Wl)
+        Wsub = np.ascontiguousarray(Wl[r])
         t0 = time.perf_counter()
         Wq, ws = oracle.quantize_weights(Wsub, prep[lin.site][0])
         dt = time.perf_counter() - t0
         spent += dt
-        full += dt * Wl.shape[0] / n
-        lin_q[lin.name] = (Wq, ws, n, Wl.shape[0])
+        full += dt * Wl.shape[0] / len(r)
+        lin_q[lin.name] = (Wq, ws, len(r), Wl.shape[0])
     rows = _sample_rows(w.M, token_rows)
     R = len(rows)
     t_rows = 0.0
@@ -155,6 +159,7 @@ def oracle_sample_step(w, inp, token_rows=16, weight_elems=48 << 20):
             acc = oracle.gemm_i64(Xq, Wq)
             _, out = oracle.epilogue(acc, xs, ws, lin.relu)
             dt = time.perf_counter() - t0
+            spent += dt
             t_rows += dt * N / n  # the GEMM scales with the output channels too
             if any(l.source == lin.name for l in w.linears):
                 # a downstream site reads this output: it needs every channel
@@ -163,10 +168,22 @@ def oracle_sample_step(w, inp, token_rows=16, weight_elems=48 << 20):
                 outs[lin.name] = np.ascontiguousarray(out)
     spent += t_rows
     full += t_rows * w.M / R
-    desc = ("oracle on %d of %d tokens and up to %d weight elements per Linear "
-            "(full calibration batch), extrapolated linearly to the full step" %
-            (R, w.M, weight_elems))
+    desc = ("oracle on %d of %d tokens, %d of %d calibration tokens and up to %d weight "
+            "elements per Linear, each phase extrapolated linearly to the full step" %
+            (R, w.M, min(cal_rows, w.M_cal), w.M_cal, weight_elems))
     return full, spent, desc
+
+
+def reference_sample_sizes(w, inp, steps, budget_s=150.0):
+    """Sample sizes for `steps` oracle steps to fit in about `budget_s`
+    seconds: a tiny probe step measures the cost, the sizes scale from it."""
+    probe = dict(cal_rows=8, weight_elems=1 << 20, token_rows=1)
+    _, spent, _ = oracle_sample_step(w, inp, **probe)
+    per_step = max(0.05, (budget_s - spent) / max(1, steps))
+    k = max(1.0, per_step / max(spent, 1e-3))
+    return dict(cal_rows=int(min(w.M_cal, 8 * k)),
+                weight_elems=int(min(48 << 20, (1 << 20) * k)),
+                token_rows=int(max(1, min(16, k))))
 
 
 def run_reference(args, w):
@@ -176,10 +193,11 @@ def run_reference(args, w):
     oracle.build()
     inp = S.make_inputs(w, seed=0)
     cores = oracle.num_threads()
+    sizes = reference_sample_sizes(w, inp, args.warmup + args.steps)
     times = []
     desc = ""
     for i in range(args.warmup + args.steps):
-        full, spent, desc = oracle_sample_step(w, inp, token_rows=args.ref_rows)
+        full, spent, desc = oracle_sample_step(w, inp, **sizes)
         if i >= args.warmup:
             times.append(full)
     t = sum(times) / len(times)
@@ -209,58 +227,68 @@ REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_pow
 
 
 class ClockSampler:
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "utilization.gpu")
+    """Samples the SM clock, power and clock-event reasons of one GPU through
+    NVML every few milliseconds on a background thread while the timed region
+    runs (the same counters nvidia-smi's clocks query reads)."""
 
-    def __init__(self, gpu_id):
-        self.proc = None
-        self.path = None
-        self.gpu_id = gpu_id
+    def __init__(self, pci_bus_id=None, period_s=0.005):
+        self.period = period_s
+        self.pci = pci_bus_id
+        self.samples = []
+        self._stop = None
+        self._thr = None
+        self._nvml = None
 
     def start(self):
-        import tempfile
-        fd, self.path = tempfile.mkstemp(prefix="sq_clocks_", suffix=".csv")
-        os.close(fd)
-        cmd = ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
-               "-lms", "200"]
-        if self.gpu_id:
-            cmd += ["-i", self.gpu_id]
+        import threading
         try:
-            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"),
-                                         stderr=subprocess.DEVNULL)
-        except OSError:
-            self.proc = None
+            import pynvml
+            pynvml.nvmlInit()
+            h = (pynvml.nvmlDeviceGetHandleByPciBusId(self.pci) if self.pci
+                 else pynvml.nvmlDeviceGetHandleByIndex(0))
+            self._nvml = (pynvml, h)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+        except Exception:
+            self._nvml = None
+            return
+        self._stop = threading.Event()
+
+        def loop():
+            pn, h = self._nvml
+            while not self._stop.is_set():
+                try:
+                    self.samples.append((
+                        float(pn.nvmlDeviceGetClockInfo(h, pn.NVML_CLOCK_SM)),
+                        pn.nvmlDeviceGetPowerUsage(h) / 1000.0,
+                        int(pn.nvmlDeviceGetCurrentClocksEventReasons(h)),
+                        float(pn.nvmlDeviceGetUtilizationRates(h).gpu)))
+                except Exception:
+                    pass
+                self._stop.wait(self.period)
+
+        self._thr = threading.Thread(target=loop, daemon=True)
+        self._thr.start()
 
     def stop(self):
-        if self.proc is None:
+        if self._nvml is None:
             return None
-        self.proc.terminate()
+        self._stop.set()
+        self._thr.join(timeout=2)
         try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 5:
-                    continue
-                try:
-                    rows.append((float(parts[0]), float(parts[1]), float(parts[2]),
-                                 int(parts[3], 16), float(parts[4])))
-                except ValueError:
-                    continue
-        os.unlink(self.path)
+            self._nvml[0].nvmlShutdown()
+        except Exception:
+            pass
+        rows = self.samples
         if not rows:
             return None
-        busy = [r for r in rows if r[4] > 0] or rows
         reasons = 0
-        for r in busy:
-            reasons |= r[3]
-        return {"sm_mhz": statistics.median(r[0] for r in busy),
-                "sm_max_mhz": max(r[1] for r in rows),
-                "power_w_max": max(r[2] for r in rows),
-                "samples": len(rows),
+        for r in rows:
+            reasons |= r[2]
+        return {"sm_mhz": statistics.median(r[0] for r in rows),
+                "sm_max_mhz": self.max_mhz,
+                "sm_mhz_min": min(r[0] for r in rows),
+                "power_w_max": max(r[1] for r in rows),
+                "samples": len(rows), "source": "NVML, every 5 ms during the timed region",
                 "reasons": [name for bit, name in REASON_BITS.items() if reasons & bit]}
 
 
@@ -331,19 +359,19 @@ def run_gpu(args, w):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    gemm_events = []
+    events = []  # (kind, units, start event, end event) of every library call
 
-    def around_gemm(lin, fn):
+    def timer(kind, units, fn):
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         fn()
         e1.record(stream)
-        gemm_events.append((lin, e0, e1))
+        events.append((kind, units, e0, e1))
 
     def step(timed):
-        blk.prepare(xc, W, g, b)
-        blk.forward(x, around_gemm=around_gemm if timed else None)
+        blk.prepare(xc, W, g, b, timer=timer if timed else None)
+        blk.forward(x, timer=timer if timed else None)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -353,12 +381,13 @@ def run_gpu(args, w):
         dist.barrier()
     torch.cuda.synchronize(dev)
 
-    gpu_id = None
+    pci = None
     try:
-        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+        p = torch.cuda.get_device_properties(dev)
+        pci = "%08X:%02X:%02X.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
     except Exception:
         pass
-    sampler = ClockSampler(gpu_id)
+    sampler = ClockSampler(pci)
     sampler.start()
     wall0 = time.perf_counter()
     step_ev = []
@@ -387,16 +416,27 @@ def run_gpu(args, w):
     value = tops_total / 1e12
     tokens_per_s = w.M * args.steps * world / t_max
 
-    # dominant kernel: the GEMM (every launch timed with events on its stream)
-    g_ms = [a.elapsed_time(b_) for (_, a, b_) in gemm_events]
-    g_ops = 0
-    g_bytes = 0
-    for (lin, _, _) in gemm_events:
-        K = w.site(lin.site).K
-        g_ops += 2 * w.M * lin.N * K
-        g_bytes += gemm_bytes(w.M, lin.N, K)
-    g_time = sum(g_ms) / 1e3
+    # per library call: CUDA events on the launching stream around every call
+    kinds = {}
+    for (kind, units, a, b_) in events:
+        k = kinds.setdefault(kind, [0, 0.0, 0.0])
+        k[0] += 1
+        k[1] += units
+        k[2] += a.elapsed_time(b_) / 1e3
     peaks, peak_src = load_peaks()
+    kernels = {}
+    for kind, (n, units, secs) in kinds.items():
+        if kind == "gemm":
+            continue
+        gbs = units / secs / 1e9
+        kernels[kind] = {"calls": n // args.steps, "ms_per_call": secs * 1e3 / n,
+                         "achieved_gbs": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
+                         "bytes_per_call": units / n}
+    # dominant kernel: the GEMM
+    g_n, g_ops, g_time = kinds["gemm"]
+    g_bytes = 0
+    for lin in w.linears:
+        g_bytes += gemm_bytes(w.M, lin.N, w.site(lin.site).K) * args.steps
     decode = w.M <= 128
     if decode:
         achieved = g_bytes / g_time / 1e9
@@ -411,12 +451,11 @@ def run_gpu(args, w):
                 "peak_sustained": peaks.get("bf16_tflops_sustained", 0.0) * INT8_PER_BF16}
     roof["peak_source"] = "%s (%s)" % (peak_src, "HBM copy" if decode else
                                        "2 x bf16 cuBLAS, the nominal INT8:BF16 ratio")
-    n_gemm_launches = len(gemm_events) // args.steps
     tr = profile_traffic("w8a8_gemm_kernel", w.name)
     roof["traffic"] = None if tr is None else tr
-    roof["algorithmic_per_launch"] = (g_bytes if decode else g_ops) / len(gemm_events)
+    roof["algorithmic_per_launch"] = (g_bytes if decode else g_ops) / g_n
     roof["kernel"] = "w8a8_gemm_kernel"
-    roof["launch_ms_mean"] = g_time * 1e3 / len(gemm_events)
+    roof["launch_ms_mean"] = g_time * 1e3 / g_n
 
     line = {
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
@@ -431,11 +470,11 @@ def run_gpu(args, w):
         "tokens_per_s": tokens_per_s,
         "forward_gemm_tops": g_ops / g_time / 1e12,
         "roofline": roof,
+        "kernels": kernels,
         "gpu_launches": args.steps * (blk.prepare_launches() + blk.forward_launches()),
         "clocks": clocks,
         "wall_s_timed": wall,
     }
-    del n_gemm_launches
 
     # end to end through the public API: pinned host inputs in, results out
     if not args.no_e2e:
@@ -448,7 +487,7 @@ def run_gpu(args, w):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         oracle.build()
-        full, spent, desc = oracle_sample_step(w, inp, token_rows=args.ref_rows)
+        full, spent, desc = oracle_sample_step(w, inp)
         line["cpu_baseline"] = {"value": workload_ops(w) / full / 1e12, "unit": "TOPS",
                                 "cores": oracle.num_threads(), "kind": "oracle",
                                 "sample": desc + " (%.1f s of CPU time)" % spent}
@@ -514,13 +553,11 @@ def e2e_leg(args, w, inp, blk, dev, stream, world):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--ref-rows", type=int, default=16,
-                    help="tokens per oracle sample step (reference arm / CPU baseline)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

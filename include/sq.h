@@ -200,8 +200,10 @@ size_t sq_w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int split_k)
  *   workspace / ws_bytes  device scratch for split-K partial sums; at least
  *            sq_w8a8_gemm_workspace_size(M, N, K, split_k) bytes when that is
  *            non-zero, else may be NULL
- *   path_hint 0 = automatic, 1 = prefill tiles (tokens on the MMA M side),
- *            2 = decode tiles (weight rows on the MMA M side, M <= 256)
+ *   path_hint 0 = automatic, 1 = prefill tiles (tokens on the MMA M side;
+ *            CTA pairs, 256 x 256 tiles on two SMs), 2 = decode tiles (weight
+ *            rows on the MMA M side, M <= 256), 3 = prefill tiles on single
+ *            SMs (128 x 256)
  *   split_k  0 = automatic, else the number of K slices (decode path only;
  *            the INT32 partial sums are added exactly, so the result does not
  *            depend on it)

@@ -182,7 +182,8 @@ def test_weight_quant_matches_oracle(NK, smoothed, dtype):
 # ---------------------------------------------------------------------------
 
 GEMM_SHAPES = [(16, 64, 64), (3, 5, 16), (1, 300, 48), (129, 257, 4112), (256, 512, 1024),
-               (200, 1000, 128), (300, 777, 160), (1024, 768, 2048)]
+               (200, 1000, 128), (300, 777, 160), (1024, 768, 2048), (2048, 1536, 512),
+               (600, 2304, 4096)]
 
 
 def _codes(M, K, extreme=False):
@@ -191,8 +192,9 @@ def _codes(M, K, extreme=False):
     return RNG.integers(-127, 128, (M, K)).astype(np.int8)
 
 
+# path hints: 1 = prefill on CTA pairs (2-SM MMA), 2 = decode tiles, 3 = prefill on one SM
 @pytest.mark.parametrize("shape", GEMM_SHAPES, ids=lambda s: "%dx%dx%d" % s)
-@pytest.mark.parametrize("path", [1, 2])
+@pytest.mark.parametrize("path", [1, 2, 3])
 def test_gemm_int32_exact(shape, path):
     M, N, K = shape
     if path == 2 and M > 256:
@@ -210,7 +212,7 @@ def test_gemm_int32_extremes_and_max_k():
     B[1] = 127
     acc_o = oracle.gemm_i64(A, B)
     assert acc_o.max() == 127 * 127 * K and acc_o.min() == -127 * 127 * K
-    for path in (1, 2):
+    for path in (1, 2, 3):
         out = sq.w8a8_gemm_dequant(to_gpu(A), to_gpu(B), None, None, "i32", path_hint=path)
         assert np.array_equal(out.cpu().numpy().astype(np.int64), acc_o)
 
@@ -229,7 +231,7 @@ def test_split_k_invariance(M):
 @pytest.mark.parametrize("shape", [(16, 64, 64), (129, 257, 4112), (7, 1000, 512), (512, 384, 256)],
                          ids=lambda s: "%dx%dx%d" % s)
 @pytest.mark.parametrize("relu", [False, True])
-@pytest.mark.parametrize("path", [1, 2])
+@pytest.mark.parametrize("path", [1, 2, 3])
 def test_gemm_bf16_epilogue(shape, relu, path):
     M, N, K = shape
     if path == 2 and M > 256:

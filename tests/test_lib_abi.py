@@ -118,7 +118,7 @@ def test_gemm_rejects_bad_arguments(L):
     assert call(M=-1) == 1
     assert call(K=0) == 1
     assert call(epi=5) == 1
-    assert call(path=3) == 1
+    assert call(path=4) == 1
     assert call(split=-2) == 1
     assert call(ldo=32) == 1
     assert call(Xq=None) == 1

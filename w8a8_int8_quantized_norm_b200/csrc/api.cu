@@ -72,7 +72,7 @@ sq_status check_gemm(const int8_t* Xq, const int8_t* Wq, const float* x_scale,
   if (M < 0 || N < 0 || K <= 0 || split_k < 0) return SQ_ERR_INVALID_ARG;
   if (epi != SQ_EPI_BF16 && epi != SQ_EPI_BF16_RELU && epi != SQ_EPI_I32_RAW)
     return SQ_ERR_INVALID_ARG;
-  if (path_hint < 0 || path_hint > 2) return SQ_ERR_INVALID_ARG;
+  if (path_hint < 0 || path_hint > 3) return SQ_ERR_INVALID_ARG;
   if (ldo < N) return SQ_ERR_INVALID_ARG;
   if (M == 0 || N == 0) return SQ_OK;
   if (!Xq || !Wq || !out) return SQ_ERR_INVALID_ARG;

@@ -411,6 +411,273 @@ __global__ void __launch_bounds__(kThreads, 1)
 #undef TEMPTY_BAR
 }
 
+// ---------------------------------------------------------------------------
+// 2-SM variant for prefill: a CTA pair computes a 256 x 256 tile with
+// tcgen05.mma.cta_group::2.  Each CTA loads its own 128 rows of A and its own
+// 128-row half of B (no multicast), so every SM pulls 32 KB of operands per
+// 128-deep K step instead of 48 KB.  The leader CTA (rank 0) owns the
+// operand-ready barriers (it expects the bytes of both CTAs; the peer's loads
+// complete on the leader's barrier) and issues the MMAs; it signals both CTAs'
+// stage-free and accumulator-ready barriers with one commit each; both CTAs'
+// epilogue warps drain their own 128 accumulator rows and tell the leader.
+// ---------------------------------------------------------------------------
+namespace pair {
+constexpr int ROWS = 128;                    // rows of A and of B per CTA
+constexpr int A_BYTES = ROWS * BK;
+constexpr int B_BYTES = ROWS * BK;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // per CTA
+constexpr int STAGES = 6;
+constexpr int TILE = 256;                    // pair tile: 256 x 256
+constexpr int TMEM_COLS = 512;               // 2 accumulators x 256 INT32 columns
+constexpr int NUM_BARS = 2 * STAGES + 5;
+constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 8 * NUM_BARS + 16;
+}  // namespace pair
+
+__device__ __forceinline__ void mbar_complete_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.complete_tx.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+// Stage loads issued to stage s after `total` loads round-robin over STAGES.
+__device__ __forceinline__ int64_t loads_on_stage(int64_t total, int s, int stages) {
+  return total / stages + (s < total % stages ? 1 : 0);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    w8a8_gemm_pair_kernel(const __grid_constant__ CUtensorMap mapP,
+                          const __grid_constant__ CUtensorMap mapQ, const Params prm) {
+  using namespace pair;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_u32 = smem_u32(smem_raw);
+  const uint32_t base = (raw_u32 + 1023u) & ~1023u;
+  uint8_t* base_ptr = smem_raw + (base - raw_u32);
+  const uint32_t a_base = base;
+  const uint32_t b_base = base + STAGES * A_BYTES;
+  const uint32_t bar_base = base + STAGES * STAGE_BYTES;
+  const uint32_t drain_bar = bar_base + 8u * (2 * STAGES + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + STAGES * STAGE_BYTES + 8 * NUM_BARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int64_t* peer_issued_slot = reinterpret_cast<volatile int64_t*>(tmem_slot + 2);
+#define FULL_BAR(s) (bar_base + 8u * static_cast<uint32_t>(s))
+#define EMPTY_BAR(s) (bar_base + 8u * static_cast<uint32_t>(STAGES + (s)))
+#define TFULL_BAR(a) (bar_base + 8u * static_cast<uint32_t>(2 * STAGES + (a)))
+#define TEMPTY_BAR(a) (bar_base + 8u * static_cast<uint32_t>(2 * STAGES + 2 + (a)))
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair_id = static_cast<int>(blockIdx.x >> 1);
+  const int num_pairs = static_cast<int>(gridDim.x >> 1);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(FULL_BAR(s), 1);
+      mbar_init(EMPTY_BAR(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(TFULL_BAR(a), 1);
+      mbar_init(TEMPTY_BAR(a), 8);  // 4 epilogue warps in each CTA of the pair
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    *peer_issued_slot = 0;
+    mbar_fence_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&mapP);
+    tma_prefetch_desc(&mapQ);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers exist before any cross-CTA signal
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int64_t polls = prm.wait_polls;
+  // the partner's abort flag, so a failing CTA stops its partner quickly
+  const uint32_t partner_abort = map_to_cta(smem_u32(const_cast<int*>(abort_flag)), rank ^ 1u);
+  int64_t producer_issued = 0;
+
+  auto fail_pair = [&]() {
+    fail(prm.error_word, abort_flag);
+    st_cluster_u32(partner_abort, 1u);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    int stage = 0;
+    uint32_t phase = 0;
+    int64_t issued = 0;
+    bool ok = true;
+    for (int u = pair_id; u < prm.units && ok; u += num_pairs) {
+      int pb, qb, kb0, kb1, split;
+      decode_unit(prm, u, pb, qb, kb0, kb1, split);
+      for (int kb = kb0; kb < kb1; ++kb) {
+        bool w = false;
+        if (lane == 0) w = wait_phase(EMPTY_BAR(stage), phase ^ 1u, polls, abort_flag);
+        w = __shfl_sync(0xffffffffu, w, 0);
+        if (!w) {
+          if (lane == 0) fail_pair();
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          const uint32_t fb = leader ? FULL_BAR(stage) : map_to_cta(FULL_BAR(stage), 0);
+          if (leader) mbar_arrive_expect_tx(FULL_BAR(stage), 2 * STAGE_BYTES);
+          tma_load_2d_pair(a_base + stage * A_BYTES, &mapP, fb, kb * BK,
+                           pb * TILE + static_cast<int>(rank) * ROWS);
+          tma_load_2d_pair(b_base + stage * B_BYTES, &mapQ, fb, kb * BK,
+                           qb * TILE + static_cast<int>(rank) * ROWS);
+        }
+        ++issued;
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    producer_issued = issued;
+    if (lane == 0 && !leader)  // the leader needs the peer's count to drain after an abort
+      st_cluster_u32(map_to_cta(smem_u32(const_cast<int64_t*>(peer_issued_slot)), 0),
+                     static_cast<uint32_t>(issued));
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader only)
+    if (leader) {
+      constexpr uint32_t kIdesc = idesc_i8(2 * ROWS, TILE);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int u = pair_id; u < prm.units && ok; u += num_pairs) {
+        int pb, qb, kb0, kb1, split;
+        decode_unit(prm, u, pb, qb, kb0, kb1, split);
+        bool w = false;
+        if (lane == 0) w = wait_phase(TEMPTY_BAR(acc), acc_phase ^ 1u, polls, abort_flag);
+        w = __shfl_sync(0xffffffffu, w, 0);
+        if (!w) {
+          if (lane == 0) fail_pair();
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * TILE);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          w = false;
+          if (lane == 0) w = wait_phase(FULL_BAR(stage), phase, polls, abort_flag);
+          w = __shfl_sync(0xffffffffu, w, 0);
+          if (!w) {
+            if (lane == 0) fail_pair();
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t sa = a_base + stage * A_BYTES;
+            const uint32_t sb = b_base + stage * B_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+              mma_i8_pair(d_tmem, smem_desc_k_sw128(sa + kk * UMMA_K),
+                          smem_desc_k_sw128(sb + kk * UMMA_K), kIdesc,
+                          (kb > kb0 || kk > 0) ? 1u : 0u);
+            }
+            // the stage is free in both CTAs once these MMAs have read it
+            mma_commit_pair(EMPTY_BAR(stage));
+            mma_commit_pair(map_to_cta(EMPTY_BAR(stage), 1));
+          }
+          __syncwarp();
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        if (lane == 0) {
+          mma_commit_pair(TFULL_BAR(acc));
+          mma_commit_pair(map_to_cta(TFULL_BAR(acc), 1));
+        }
+        __syncwarp();
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      if (lane == 0) {
+        mma_commit_pair(drain_bar);
+        wait_phase(drain_bar, 0, 0, nullptr);
+      }
+      __syncwarp();
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int quarter = warp & 3;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    const uint32_t leader_tempty0 = leader ? TEMPTY_BAR(0) : map_to_cta(TEMPTY_BAR(0), 0);
+    const uint32_t leader_tempty1 = leader ? TEMPTY_BAR(1) : map_to_cta(TEMPTY_BAR(1), 0);
+    for (int u = pair_id; u < prm.units; u += num_pairs) {
+      int pb, qb, kb0, kb1, split;
+      decode_unit(prm, u, pb, qb, kb0, kb1, split);
+      bool w = false;
+      if (lane == 0) w = wait_phase(TFULL_BAR(acc), acc_phase, polls, abort_flag);
+      w = __shfl_sync(0xffffffffu, w, 0);
+      if (!w) {
+        if (lane == 0) fail_pair();
+        break;
+      }
+      tc_fence_after();
+      const int p = pb * TILE + static_cast<int>(rank) * ROWS + quarter * 32 + lane;
+#pragma unroll 1
+      for (int c = 0; c < TILE / 32; ++c) {
+        uint32_t r[32];
+        __syncwarp();
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                               static_cast<uint32_t>(acc * TILE + c * 32);
+        tmem_ld_32x32b_x32(taddr, r);
+        tmem_wait_ld();
+        store_chunk<32>(prm, r, p, qb * TILE + c * 32, 0);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        const uint32_t t = acc ? leader_tempty1 : leader_tempty0;
+        if (leader)
+          mbar_arrive(t);
+        else
+          mbar_arrive_cluster(t);
+      }
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+  __syncthreads();
+  cluster_sync_all();  // no MMA, TMA signal or remote arrive of this tile loop is pending
+  if (warp == 0 && lane == 0 && leader && *abort_flag) {
+    // after an abort, every stage load either CTA issued lands before either
+    // CTA releases its shared memory (the peer's loads complete on the
+    // leader's barriers; the two producers are at most one round apart)
+    const int64_t peer_issued = *peer_issued_slot;
+    for (int s = 0; s < STAGES; ++s) {
+      const int64_t nl = loads_on_stage(producer_issued, s, STAGES);
+      const int64_t np = loads_on_stage(peer_issued, s, STAGES);
+      if (np > nl) mbar_arrive_expect_tx(FULL_BAR(s), STAGE_BYTES);  // the missing leader arrival
+      else if (nl > np) mbar_complete_tx(FULL_BAR(s), STAGE_BYTES);  // peer bytes never sent
+      const int64_t n = nl > np ? nl : np;
+      if (n > 0) wait_phase(FULL_BAR(s), static_cast<uint32_t>((n - 1) & 1), 0, nullptr);
+    }
+  }
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+#undef FULL_BAR
+#undef EMPTY_BAR
+#undef TFULL_BAR
+#undef TEMPTY_BAR
+}
+
 // out[m][n] = epilogue(sum_s partial[s][m][n]); INT32 addition is exact, so
 // the split does not change the result.
 __global__ void splitk_reduce_kernel(const int32_t* __restrict__ partial, int splits, int64_t M,
@@ -483,6 +750,43 @@ cudaError_t launch_bn(const Params& prm, const CUtensorMap& mp, const CUtensorMa
   return cudaGetLastError();
 }
 
+cudaError_t launch_pair(const Params& prm, const CUtensorMap& mp, const CUtensorMap& mq,
+                        int max_pairs, cudaStream_t st) {
+  cudaError_t e = cudaFuncSetAttribute(w8a8_gemm_pair_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       pair::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = pair::SMEM_BYTES;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // as many co-resident CTA pairs as the device holds (one per SM pair)
+  static int max_clusters[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && max_clusters[dev] == 0) {
+    cfg.gridDim = dim3(2 * max_pairs);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, w8a8_gemm_pair_kernel, &cfg) != cudaSuccess || n <= 0)
+      n = max_pairs;
+    max_clusters[dev] = n;
+  }
+  int pairs = (dev >= 0 && dev < 64) ? max_clusters[dev] : max_pairs;
+  if (pairs > max_pairs) pairs = max_pairs;
+  if (pairs > prm.units) pairs = prm.units;
+  cfg.gridDim = dim3(2 * pairs);
+  e = cudaLaunchKernelEx(&cfg, w8a8_gemm_pair_kernel, mp, mq, prm);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 int bn_for_tokens(int64_t M) {
   return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
 }
@@ -500,9 +804,11 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int path_hint, int split_k, 
   GemmPlan p{};
   const int64_t kblocks = (K + BK - 1) / BK;
   p.swap = (path_hint == 2 || (path_hint == 0 && M <= 128)) ? 1 : 0;
+  p.pair = 0;
   if (!p.swap) {
     p.bn = 256;
     p.splits = 1;
+    p.pair = path_hint == 3 ? 0 : 1;
   } else {
     p.bn = bn_for_tokens(M);
     const int64_t tiles = (N + BM - 1) / BM;
@@ -547,7 +853,8 @@ cudaError_t launch_gemm(const GemmPlan& plan, const int8_t* Xq, const int8_t* Wq
   prm.P = static_cast<int>(plan.swap ? N : M);
   prm.Q = static_cast<int>(plan.swap ? M : N);
   prm.K = static_cast<int>(K);
-  prm.p_blocks = (prm.P + BM - 1) / BM;
+  const int p_tile = plan.pair ? pair::TILE : BM;
+  prm.p_blocks = (prm.P + p_tile - 1) / p_tile;
   prm.q_blocks = (prm.Q + plan.bn - 1) / plan.bn;
   prm.k_blocks = static_cast<int>((K + BK - 1) / BK);
   prm.splits = plan.splits;
@@ -569,9 +876,15 @@ cudaError_t launch_gemm(const GemmPlan& plan, const int8_t* Xq, const int8_t* Wq
 
   CUtensorMap mp, mq;
   if (K == 0) return cudaErrorInvalidValue;
+  const int sms = num_sms > 0 ? num_sms : 148;
+  if (plan.pair) {
+    // each CTA of a pair loads 128 rows of A and 128 rows of B
+    if (!make_map(&mp, Pptr, prm.P, K, pair::ROWS) || !make_map(&mq, Qptr, prm.Q, K, pair::ROWS))
+      return cudaErrorInvalidValue;
+    return launch_pair(prm, mp, mq, sms / 2, st);
+  }
   if (!make_map(&mp, Pptr, prm.P, K, BM) || !make_map(&mq, Qptr, prm.Q, K, plan.bn))
     return cudaErrorInvalidValue;
-  const int sms = num_sms > 0 ? num_sms : 148;
   const int grid = prm.units < sms ? prm.units : sms;
   cudaError_t e;
   switch (plan.bn) {

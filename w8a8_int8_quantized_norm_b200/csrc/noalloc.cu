@@ -56,7 +56,7 @@ extern "C" sq_status sq_w8a8_gemm_dequant_noalloc(const int8_t* Xq, const int8_t
                                                   sq_epilogue epi, void* out, int64_t ldo,
                                                   int path_hint, int split_k, void* stream) {
   using namespace sq;
-  if (M < 0 || N < 0 || K <= 0 || split_k < 0 || path_hint < 0 || path_hint > 2)
+  if (M < 0 || N < 0 || K <= 0 || split_k < 0 || path_hint < 0 || path_hint > 3)
     return SQ_ERR_INVALID_ARG;
   if (M == 0 || N == 0) {
     return sq_w8a8_gemm_dequant(Xq, Wq, x_scale, w_scale, M, N, K, epi, out, ldo, nullptr, 0,

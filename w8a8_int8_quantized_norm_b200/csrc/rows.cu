@@ -236,7 +236,19 @@ __global__ void __launch_bounds__(256) weight_colmax_kernel(const void* __restri
   float m[kChunk];
 #pragma unroll
   for (int i = 0; i < kChunk; ++i) m[i] = 0.0f;
-  for (int64_t n = r0; n < r1; ++n) {
+  // eight independent 128-bit loads in flight per thread
+  constexpr int U = 8;
+  int64_t n = r0;
+  for (; n + U <= r1; n += U) {
+    float v[U][kChunk];
+#pragma unroll
+    for (int u = 0; u < U; ++u) load_chunk<kBF16>(W, (n + u) * (int64_t)K + (int64_t)ch * kChunk, v[u]);
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int i = 0; i < kChunk; ++i) m[i] = fmaxf(m[i], fabsf(v[u][i]));
+  }
+  for (; n < r1; ++n) {
     float v[kChunk];
     load_chunk<kBF16>(W, n * (int64_t)K + (int64_t)ch * kChunk, v);
 #pragma unroll
@@ -313,7 +325,12 @@ cudaError_t launch_calibrate(const void* x, bool bf16, int64_t M, int K, int64_t
   if (M == 0) return cudaSuccess;
   const int ch = pick_ch(K);
   const int threads = threads_for(K, ch);
-  const int rows_per_cta = 8;
+  // about two CTAs per SM: enough parallelism, few atomics per channel
+  int sms = 0, dev = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t target = 2 * static_cast<int64_t>(sms > 0 ? sms : 148);
+  const int rows_per_cta = static_cast<int>((M + target - 1) / target);
   const dim3 grid(static_cast<unsigned>((M + rows_per_cta - 1) / rows_per_cta));
   const size_t smem = static_cast<size_t>(K) * sizeof(float);
   auto go = [&](auto kernel) {

@@ -25,6 +25,7 @@ cudaError_t launch_smooth_finalize(const float* act_max, float* s, int K, double
 // gemm.cu
 struct GemmPlan {
   int swap;       // 0: tokens on the MMA M side (prefill); 1: weight rows (decode)
+  int pair;       // prefill on CTA pairs (2-SM MMA, 256 x 256 tiles)
   int bn;         // MMA N (tile width on the Q side)
   int splits;     // K slices
   size_t workspace_bytes;

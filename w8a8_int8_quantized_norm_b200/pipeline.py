@@ -20,15 +20,27 @@ import torch
 from . import sq
 from .synthetic import Workload
 
+# timer(kind, algorithmic_units, fn): a caller hook around every library call;
+# kind names the kernel family, units are its algorithmic bytes (row kernels)
+# or integer ops (the GEMM).
+Timer = Optional[Callable[[str, float, Callable[[], None]], None]]
+
+
+def _run(timer: Timer, kind: str, units: float, fn: Callable[[], None]) -> None:
+    if timer is None:
+        fn()
+    else:
+        timer(kind, units, fn)
+
 
 class Block:
     """Device state of one workload for M tokens per forward.
 
     ``prepare`` runs the offline rows (calibration, smoothing factors + fold,
     weight smoothing + quantisation); ``forward`` the runtime rows (fused norm
-    + per-token quantisation, INT8 GEMM with the dequant epilogue).  Optional
-    ``around_gemm(fn)`` hooks let a caller bracket every GEMM launch (the
-    benchmark records CUDA events there)."""
+    + per-token quantisation, INT8 GEMM with the dequant epilogue).  An optional
+    ``timer`` hook brackets every library call (the benchmark records CUDA
+    events there)."""
 
     def __init__(self, w: Workload, M: int, device):
         self.w = w
@@ -68,7 +80,7 @@ class Block:
     # -- offline rows -------------------------------------------------------
     def prepare(self, x_cal: Dict[str, torch.Tensor], W: Dict[str, torch.Tensor],
                 gamma: Dict[str, Optional[torch.Tensor]], beta: Dict[str, Optional[torch.Tensor]],
-                stream=None) -> "Block":
+                stream=None, timer: Timer = None) -> "Block":
         w = self.w
         for site in w.sites:
             g, b = gamma.get(site.name), beta.get(site.name)
@@ -76,30 +88,43 @@ class Block:
                 if b is not None and self.beta_f[site.name] is None:
                     self.beta_f[site.name] = torch.empty_like(self.gamma_f[site.name])
                 am = self.act_max[site.name]
+                xc = x_cal[site.name]
                 am.zero_()
-                sq.calibrate_absmax(x_cal[site.name], site.norm, g, b, w.eps, act_max=am,
-                                    stream=stream)
-                sq.compute_smooth_scales(am, [W[l.name] for l in w.linears_of(site.name)],
-                                         w.alpha, w.clamp_eps, g, b, s=self.s[site.name],
-                                         gamma_folded=self.gamma_f[site.name],
-                                         beta_folded=self.beta_f[site.name], stream=stream)
+                _run(timer, "calibrate", xc.numel() * xc.element_size() + 4 * site.K,
+                     lambda: sq.calibrate_absmax(xc, site.norm, g, b, w.eps, act_max=am,
+                                                 stream=stream))
+                Ws = [W[l.name] for l in w.linears_of(site.name)]
+                _run(timer, "smooth_scales",
+                     sum(t.numel() * t.element_size() for t in Ws) + 16 * site.K,
+                     lambda: sq.compute_smooth_scales(am, Ws, w.alpha, w.clamp_eps, g, b,
+                                                      s=self.s[site.name],
+                                                      gamma_folded=self.gamma_f[site.name],
+                                                      beta_folded=self.beta_f[site.name],
+                                                      stream=stream))
             else:
                 self.gamma_f[site.name], self.beta_f[site.name] = g, b
         for lin in w.linears:
-            sq.smooth_quantize_weights(W[lin.name], self.s[lin.site], Wq=self.Wq[lin.name],
-                                       w_scale=self.w_scale[lin.name], stream=stream)
+            Wl = W[lin.name]
+            _run(timer, "weight_quant", Wl.numel() * (Wl.element_size() + 1) + 4 * lin.N,
+                 lambda: sq.smooth_quantize_weights(Wl, self.s[lin.site], Wq=self.Wq[lin.name],
+                                                    w_scale=self.w_scale[lin.name],
+                                                    stream=stream))
         return self
 
     # -- runtime rows -------------------------------------------------------
-    def forward(self, x: Dict[str, torch.Tensor], stream=None,
-                around_gemm: Optional[Callable] = None) -> Dict[str, torch.Tensor]:
+    def forward(self, x: Dict[str, torch.Tensor], stream=None, timer: Timer = None
+                ) -> Dict[str, torch.Tensor]:
         w = self.w
         for site in w.sites:
             src = next((l.source for l in w.linears if l.site == site.name and l.source), None)
             xin = self.out[src] if src else x[site.name]
-            sq.norm_smooth_quant_per_token(xin, site.norm, self.gamma_f[site.name],
-                                           self.beta_f[site.name], w.eps, self.xq[site.name],
-                                           self.xs[site.name], stream=stream)
+            nparam = (self.gamma_f[site.name] is not None) + (self.beta_f[site.name] is not None)
+            _run(timer, "norm_quant",
+                 xin.numel() * (xin.element_size() + 1) + 4 * self.M + 4 * site.K * nparam,
+                 lambda: sq.norm_smooth_quant_per_token(xin, site.norm, self.gamma_f[site.name],
+                                                        self.beta_f[site.name], w.eps,
+                                                        self.xq[site.name], self.xs[site.name],
+                                                        stream=stream))
             for lin in w.linears_of(site.name):
                 def gemm(lin=lin, site=site):
                     sq.w8a8_gemm_dequant(self.xq[site.name], self.Wq[lin.name],
@@ -107,10 +132,7 @@ class Block:
                                          "bf16_relu" if lin.relu else "bf16",
                                          out=self.out[lin.name], workspace=self.ws[lin.name],
                                          stream=stream)
-                if around_gemm is None:
-                    gemm()
-                else:
-                    around_gemm(lin, gemm)
+                _run(timer, "gemm", 2.0 * self.M * lin.N * site.K, gemm)
         return self.out
 
     # -- launch accounting ---------------------------------------------------
