@@ -70,6 +70,44 @@ def test_norm_quant_matches_oracle(shape, kind, dtype):
     assert tol == 0
 
 
+@pytest.mark.parametrize("shape", [(1000, 4096), (777, 8192), (4099, 64), (300, 9216)],
+                         ids=lambda s: "%dx%d" % s)
+@pytest.mark.parametrize("kind", [oracle.NORM_RMS, oracle.NORM_LAYER, oracle.NORM_NONE])
+def test_norm_quant_many_rows(shape, kind):
+    """More rows than resident CTAs: every CTA loops over several rows."""
+    M, K = shape
+    x = _acts(M, K, "bf16")
+    g = RNG.uniform(0.5, 1.5, K).astype(np.float32)
+    b = (RNG.standard_normal(K) * 0.1).astype(np.float32) if kind == oracle.NORM_LAYER else None
+    Xq_o, xs_o = oracle.norm_quant(x, kind, g, b, 1e-5)
+    Xq_g, xs_g = sq.norm_smooth_quant_per_token(to_gpu(x), kind, to_gpu(g),
+                                                None if b is None else to_gpu(b), 1e-5)
+    assert compare_rows_quant(Xq_g.cpu().numpy(), xs_g.cpu().numpy(), Xq_o, xs_o,
+                              norm_near_tie_rows(x, kind, 1e-5)) == 0
+
+
+def test_quantizer_half_integer_quotients():
+    """Values whose quotient by the step is a half-integer or within an ulp of
+    one: the rounding must follow the exact fp32 quotient (ties to even)."""
+    K = 4096
+    rows = []
+    for am in (100.0, 3.0, 0.1234, 77.7):
+        step = np.float32(np.float32(am) / np.float32(127.0))
+        k = RNG.integers(-126, 126, K).astype(np.float32)
+        y = ((k + np.float32(0.5)) * step).astype(np.float32)
+        y = np.nextafter(y, y + RNG.choice([-1.0, 0.0, 1.0], K).astype(np.float32) * np.float32(1e30))
+        y = y.astype(np.float32)
+        y[0] = am
+        y[1] = -am
+        y = np.clip(y, -am, am).astype(np.float32)
+        rows.append(y)
+    x = np.stack(rows)
+    Xq_o, xs_o = oracle.norm_quant(x, oracle.NORM_NONE)
+    Xq_g, xs_g = sq.norm_smooth_quant_per_token(to_gpu(x), oracle.NORM_NONE)
+    assert np.array_equal(xs_g.cpu().numpy(), xs_o)
+    assert np.array_equal(Xq_g.cpu().numpy(), Xq_o)
+
+
 def test_norm_quant_strided_rows_and_canaries():
     M, K, ld = 33, 4096, 4096 + 64
     big = S.to_bf16_bits(RNG.standard_normal((M, ld)).astype(np.float32))

@@ -177,8 +177,10 @@ sq_status sq_smooth_quantize_weights(const void* W, sq_dtype dtype, int64_t N, i
     if ((st = check_vec(w_scale, true)) != SQ_OK) return st;
   }
   // a weight row smoothed by s is the no-norm row path with s as multiplier
+  int* err = device_error_word();
+  if (!err) return SQ_ERR_CUDA;
   return from_cuda(launch_norm_quant(W, dtype == SQ_BF16, N, static_cast<int>(K), ldw,
-                                     SQ_NORM_NONE, s, nullptr, 0.0f, Wq, w_scale,
+                                     SQ_NORM_NONE, s, nullptr, 0.0f, Wq, w_scale, err,
                                      as_stream(stream)));
 }
 
@@ -196,8 +198,10 @@ sq_status sq_norm_smooth_quant_per_token(const void* x, sq_dtype dtype, int64_t 
     if (!aligned16(Xq)) return SQ_ERR_ALIGNMENT;
     if ((st = check_vec(x_scale, true)) != SQ_OK) return st;
   }
+  int* err = device_error_word();
+  if (!err) return SQ_ERR_CUDA;
   return from_cuda(launch_norm_quant(x, dtype == SQ_BF16, M, static_cast<int>(K), ldx, norm,
-                                     gamma_folded, beta_folded, eps, Xq, x_scale,
+                                     gamma_folded, beta_folded, eps, Xq, x_scale, err,
                                      as_stream(stream)));
 }
 
@@ -257,7 +261,8 @@ sq_status sq_linear_w8a8(const void* x, sq_dtype dtype, int64_t M, int64_t K, in
   if (!err) return SQ_ERR_CUDA;
   cudaStream_t cs = as_stream(stream);
   cudaError_t e = launch_norm_quant(x, dtype == SQ_BF16, M, static_cast<int>(K), ldx, norm,
-                                    gamma_folded, beta_folded, eps, Xq_scratch, xscale_scratch, cs);
+                                    gamma_folded, beta_folded, eps, Xq_scratch, xscale_scratch,
+                                    err, cs);
   if (e != cudaSuccess) return SQ_ERR_CUDA;
   return from_cuda(launch_gemm(plan, Xq_scratch, Wq, xscale_scratch, w_scale, M, N, K, epi, out,
                                ldo, workspace, sms, g_wait_polls.load(), err, cs));

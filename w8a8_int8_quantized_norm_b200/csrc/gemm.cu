@@ -73,31 +73,33 @@ struct Params {
   int epi;                         // SQ_EPI_*
   int swap;                        // 0: out[p][q]; 1: out[q][p]
   int32_t* partial;                // split-K: raw sums [split][M][N] (M = token extent)
-  int64_t wait_polls;              // > 0: poll budget per wait; 0: ~2 s by the global timer
+  int64_t wait_polls;              // > 0: poll budget per wait; 0: ~2 s of SM clock cycles
   int* error_word;                 // device error word of this device
   int vec_out;                     // output rows 16-byte aligned: 128-bit stores allowed
 };
 
-__device__ __forceinline__ uint64_t global_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
+// Give-up point of a pipeline wait, in SM clock cycles (about 2 s at the
+// B200's 1.965 GHz maximum clock, longer at lower clocks).
+constexpr long long kWaitBudgetCycles = 4000000000LL;
 
-// Bounded wait on an mbarrier phase; `abort` may be null.
+// Bounded wait on an mbarrier phase; `abort` may be null.  The first probe is
+// free of any timer read (the common case: the phase is already complete);
+// the budget is kept with the SM-local cycle counter, which is cheap to read
+// (the global nanosecond timer costs a few hundred cycles per read).
 __device__ bool wait_phase(uint32_t bar, uint32_t parity, int64_t polls, const volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
   if (polls > 0) {
-    for (int64_t i = 0; i < polls; ++i) {
+    for (int64_t i = 1; i < polls; ++i) {
       if (mbar_try_wait(bar, parity)) return true;
       if (abort && *abort) return false;
     }
     return false;
   }
-  const uint64_t t0 = global_ns();
+  const long long t0 = clock64();
   for (uint32_t i = 0;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if (abort && *abort) return false;
-    if ((i & 255u) == 255u && global_ns() - t0 > 2000000000ull) return false;
+    if ((i & 63u) == 63u && clock64() - t0 > kWaitBudgetCycles) return false;
   }
 }
 

@@ -300,8 +300,12 @@ int threads_for(int K, int ch) {
 
 cudaError_t launch_norm_quant(const void* x, bool bf16, int64_t M, int K, int64_t ldx, int norm,
                               const float* gamma, const float* beta, float eps, int8_t* q,
-                              float* scale, cudaStream_t st) {
+                              float* scale, int* err, cudaStream_t st) {
   if (M == 0) return cudaSuccess;
+  // rows that fit the shared-memory ring take the pipelined kernel; very wide
+  // rows keep everything in registers instead
+  if (norm_quant_pipe_supported(K, bf16))
+    return launch_norm_quant_pipe(x, bf16, M, K, ldx, norm, gamma, beta, eps, q, scale, err, st);
   const int ch = pick_ch(K);
   const int threads = threads_for(K, ch);
   const dim3 grid(static_cast<unsigned>(M));

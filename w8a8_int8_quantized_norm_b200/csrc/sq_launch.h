@@ -12,7 +12,13 @@ namespace sq {
 bool rows_supported(int K);
 cudaError_t launch_norm_quant(const void* x, bool bf16, int64_t M, int K, int64_t ldx, int norm,
                               const float* gamma, const float* beta, float eps, int8_t* q,
-                              float* scale, cudaStream_t st);
+                              float* scale, int* err, cudaStream_t st);
+
+// normquant.cu
+bool norm_quant_pipe_supported(int K, bool bf16);
+cudaError_t launch_norm_quant_pipe(const void* x, bool bf16, int64_t M, int K, int64_t ldx,
+                                   int norm, const float* gamma, const float* beta, float eps,
+                                   int8_t* q, float* scale, int* err, cudaStream_t st);
 cudaError_t launch_calibrate(const void* x, bool bf16, int64_t M, int K, int64_t ldx, int norm,
                              const float* gamma, const float* beta, float eps, float* act_max,
                              cudaStream_t st);
