@@ -89,6 +89,12 @@ sq_status check_gemm(const int8_t* Xq, const int8_t* Wq, const float* x_scale,
 }
 
 }  // namespace
+
+LaunchCache& launch_cache() {
+  static LaunchCache cache;
+  return cache;
+}
+
 }  // namespace sq
 
 using namespace sq;

@@ -744,9 +744,8 @@ template <int BN>
 cudaError_t launch_bn(const Params& prm, const CUtensorMap& mp, const CUtensorMap& mq, int grid,
                       cudaStream_t st) {
   using C = Cfg<BN>;
-  // the attribute is per device; setting it is cheap and idempotent
-  cudaError_t e = cudaFuncSetAttribute(w8a8_gemm_kernel<BN>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  cudaError_t e = launch_cache().ensure_smem(reinterpret_cast<const void*>(w8a8_gemm_kernel<BN>),
+                                             C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   w8a8_gemm_kernel<BN><<<grid, kThreads, C::SMEM_BYTES, st>>>(mp, mq, prm);
   return cudaGetLastError();
@@ -754,9 +753,8 @@ cudaError_t launch_bn(const Params& prm, const CUtensorMap& mp, const CUtensorMa
 
 cudaError_t launch_pair(const Params& prm, const CUtensorMap& mp, const CUtensorMap& mq,
                         int max_pairs, cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(w8a8_gemm_pair_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       pair::SMEM_BYTES);
+  cudaError_t e = launch_cache().ensure_smem(reinterpret_cast<const void*>(w8a8_gemm_pair_kernel),
+                                             pair::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -771,8 +769,7 @@ cudaError_t launch_pair(const Params& prm, const CUtensorMap& mp, const CUtensor
   cfg.numAttrs = 1;
   // as many co-resident CTA pairs as the device holds (one per SM pair)
   static int max_clusters[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
+  const int dev = LaunchCache::device();
   if (dev >= 0 && dev < 64 && max_clusters[dev] == 0) {
     cfg.gridDim = dim3(2 * max_pairs);
     int n = 0;
@@ -795,12 +792,7 @@ int bn_for_tokens(int64_t M) {
 
 }  // namespace
 
-int num_sms_current_device() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  return n;
-}
+int num_sms_current_device() { return launch_cache().sms(); }
 
 GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int path_hint, int split_k, int num_sms) {
   GemmPlan p{};

@@ -77,11 +77,6 @@ __device__ __forceinline__ double warp_sum(double v) {
   for (int o = 16; o > 0; o >>= 1) v = __dadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
   return v;
 }
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
 
 // INT8 codes of 8 values, packed little-endian into two words:
 // clamp(rne(fl32(v / step)), -127, 127).  Fast path: one fused multiply-add
@@ -384,16 +379,11 @@ cudaError_t launch_pipe_k(const void* x, int64_t M, int K, int64_t ldx, const fl
                           const float* beta, float eps, int8_t* q, float* scale,
                           const PipeShape& ps, int* err, cudaStream_t st) {
   auto kern = norm_quant_pipe_kernel<kBF16, NORMK, CH, kG, kB, kF>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(ps.smem));
+  LaunchCache& lc = launch_cache();
+  const cudaError_t e = lc.ensure_smem(reinterpret_cast<const void*>(kern), ps.smem);
   if (e != cudaSuccess) return e;
-  int per_sm = 0, dev = 0, sms = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, ps.threads, ps.smem);
-  if (e != cudaSuccess) return e;
-  if (per_sm < 1) per_sm = 1;
-  int64_t grid = static_cast<int64_t>(per_sm) * (sms > 0 ? sms : 148);
+  const int per_sm = lc.blocks_per_sm(reinterpret_cast<const void*>(kern), ps.threads, ps.smem);
+  int64_t grid = static_cast<int64_t>(per_sm) * lc.sms();
   if (grid > M) grid = M;
   kern<<<static_cast<unsigned>(grid), ps.threads, ps.smem, st>>>(x, ldx, M, K, gamma, beta, eps,
                                                                    q, scale, ps.nbuf, err);

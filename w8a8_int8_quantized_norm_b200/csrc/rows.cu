@@ -330,16 +330,12 @@ cudaError_t launch_calibrate(const void* x, bool bf16, int64_t M, int K, int64_t
   const int ch = pick_ch(K);
   const int threads = threads_for(K, ch);
   // about two CTAs per SM: enough parallelism, few atomics per channel
-  int sms = 0, dev = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t target = 2 * static_cast<int64_t>(sms > 0 ? sms : 148);
+  const int64_t target = 2 * static_cast<int64_t>(launch_cache().sms());
   const int rows_per_cta = static_cast<int>((M + target - 1) / target);
   const dim3 grid(static_cast<unsigned>((M + rows_per_cta - 1) / rows_per_cta));
   const size_t smem = static_cast<size_t>(K) * sizeof(float);
   auto go = [&](auto kernel) {
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    cudaError_t e = launch_cache().ensure_smem(reinterpret_cast<const void*>(kernel), smem);
     if (e != cudaSuccess) return e;
     kernel<<<grid, threads, smem, st>>>(x, ldx, M, K, rows_per_cta, norm, gamma, beta, eps, act_max);
     return cudaGetLastError();

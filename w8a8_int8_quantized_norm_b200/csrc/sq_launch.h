@@ -6,7 +6,68 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <map>
+#include <mutex>
+#include <tuple>
+
 namespace sq {
+
+// Host-side launch queries (function attributes, occupancy, SM counts) are
+// answered once per device and shape and remembered: they cost microseconds,
+// comparable to the small kernels they launch.
+class LaunchCache {
+ public:
+  // Makes sure `kernel` may use `smem` bytes of dynamic shared memory on the
+  // current device; returns the CUDA error of the attribute call, if made.
+  cudaError_t ensure_smem(const void* kernel, size_t smem) {
+    const int dev = device();
+    std::lock_guard<std::mutex> lock(mu_);
+    size_t& have = smem_[std::make_pair(dev, kernel)];
+    if (smem <= have) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(smem));
+    if (e == cudaSuccess) have = smem;
+    return e;
+  }
+  // Resident CTAs per SM of `kernel` for (threads, smem) on the current device.
+  int blocks_per_sm(const void* kernel, int threads, size_t smem) {
+    const int dev = device();
+    std::lock_guard<std::mutex> lock(mu_);
+    auto key = std::make_tuple(dev, kernel, threads, smem);
+    auto it = occ_.find(key);
+    if (it != occ_.end()) return it->second;
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem) != cudaSuccess)
+      n = 1;
+    if (n < 1) n = 1;
+    occ_[key] = n;
+    return n;
+  }
+  int sms() {
+    const int dev = device();
+    std::lock_guard<std::mutex> lock(mu_);
+    auto it = sms_.find(dev);
+    if (it != sms_.end()) return it->second;
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    sms_[dev] = n;
+    return n;
+  }
+  static int device() {
+    int d = 0;
+    cudaGetDevice(&d);
+    return d;
+  }
+
+ private:
+  std::mutex mu_;
+  std::map<std::pair<int, const void*>, size_t> smem_;
+  std::map<std::tuple<int, const void*, int, size_t>, int> occ_;
+  std::map<int, int> sms_;
+};
+
+LaunchCache& launch_cache();
 
 // rows.cu
 bool rows_supported(int K);
