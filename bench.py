@@ -78,6 +78,14 @@ def max_over_ranks(value: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+def rank_inputs(w, seed: int, rank: int):
+    """One data-parallel replica's inputs: weights, norm parameters and the
+    calibration batch are the same on every rank; the token batch is the
+    rank's own (weak scaling: a fixed batch per GPU)."""
+    from w8a8_int8_quantized_norm_b200 import synthetic as S
+    return S.make_inputs(w, seed=seed, token_seed=seed + 1000003 * rank)
+
+
 def aggregate(units_per_rank: float, seconds_per_rank: float, world: int, device=None):
     """Whole-job throughput: units all ranks processed over the slowest rank's time."""
     t = max_over_ranks(seconds_per_rank, world, device)
@@ -191,7 +199,7 @@ def run_reference(args, w):
     import oracle
     from w8a8_int8_quantized_norm_b200 import synthetic as S
     oracle.build()
-    inp = S.make_inputs(w, seed=0)
+    inp = S.make_inputs(w, seed=args.seed)
     cores = oracle.num_threads()
     sizes = reference_sample_sizes(w, inp, args.warmup + args.steps)
     times = []
@@ -340,8 +348,7 @@ def run_gpu(args, w):
                                 device_id=dev)
     sq.lib()
 
-    # inputs: each rank draws its own token batch (weak scaling)
-    inp = S.make_inputs(w, seed=args.seed + rank)
+    inp = rank_inputs(w, args.seed, rank)
 
     def to_dev(a):
         if a is None:

@@ -280,7 +280,7 @@ sq_status sq_get_device_error(void* stream);
 /*
  * sq_set_wait_limit -- diagnostics: the number of polls after which a GEMM
  * pipeline wait gives up, records SQ_ERR_PIPELINE_TIMEOUT and lets the kernel
- * drain and return (default 0 = the built-in limit of about one second).
+ * drain and return (default 0 = the built-in limit of about two seconds of SM clock).
  * Affects launches made after the call, from any thread.
  */
 void sq_set_wait_limit(int64_t polls);

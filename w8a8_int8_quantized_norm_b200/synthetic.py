@@ -235,15 +235,18 @@ class Inputs:
 
 
 def make_inputs(w: Workload, seed: int = 0, rows: Optional[int] = None,
-                weights: bool = True) -> Inputs:
+                weights: bool = True, token_seed: Optional[int] = None) -> Inputs:
     """All inputs of one workload.  ``rows`` limits the runtime token count
-    (a prefix of the full token stream)."""
+    (a prefix of the full token stream).  ``token_seed`` (default ``seed``)
+    draws the runtime tokens alone: data-parallel replicas share weights, norm
+    parameters and the calibration batch and differ only in their tokens."""
     M = w.M if rows is None else rows
+    ts = seed if token_seed is None else token_seed
     fed = {l.site for l in w.linears if l.source is not None}
     x, xc, Ws, g, b = {}, {}, {}, {}, {}
     for s in w.sites:
         if s.name not in fed:
-            x[s.name] = activations(w, s.name, M, "x", seed)
+            x[s.name] = activations(w, s.name, M, "x", ts)
         if s.smoothed and s.calibrated:
             xc[s.name] = activations(_cal_workload(w), s.name, w.M_cal, "x_cal", seed)
         g[s.name], b[s.name] = norm_params(w, s.name, seed)
