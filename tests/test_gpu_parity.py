@@ -70,7 +70,8 @@ def test_norm_quant_matches_oracle(shape, kind, dtype):
     assert tol == 0
 
 
-@pytest.mark.parametrize("shape", [(1000, 4096), (777, 8192), (4099, 64), (300, 9216)],
+@pytest.mark.parametrize("shape", [(1000, 4096), (777, 8192), (4099, 64), (300, 9216),
+                                   (2048, 4096), (700, 4112), (5000, 1024), (150, 40960)],
                          ids=lambda s: "%dx%d" % s)
 @pytest.mark.parametrize("kind", [oracle.NORM_RMS, oracle.NORM_LAYER, oracle.NORM_NONE])
 def test_norm_quant_many_rows(shape, kind):
@@ -147,7 +148,7 @@ def test_worked_example_row_on_gpu(golden_dir):
 # ---------------------------------------------------------------------------
 
 @pytest.mark.parametrize("kind", [oracle.NORM_NONE, oracle.NORM_RMS, oracle.NORM_LAYER])
-@pytest.mark.parametrize("K", [64, 4096, 9216])
+@pytest.mark.parametrize("K", [64, 4096, 9216, 16384, 28672])
 def test_calibration_running_max(kind, K):
     g = RNG.uniform(0.5, 1.5, K).astype(np.float32)
     b = (RNG.standard_normal(K) * 0.1).astype(np.float32) if kind == oracle.NORM_LAYER else None
@@ -162,6 +163,45 @@ def test_calibration_running_max(kind, K):
         assert np.array_equal(am_g.view(np.uint32), am_o.view(np.uint32))
     else:
         assert np.all(np.abs(am_g - am_o) <= 2 * np.spacing(am_o))
+
+
+@pytest.mark.parametrize("kind", [oracle.NORM_NONE, oracle.NORM_RMS, oracle.NORM_LAYER])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("shape", [(3000, 4096), (1500, 4112), (2, 8192)],
+                         ids=lambda s: "%dx%d" % s)
+def test_calibration_many_rows(kind, dtype, shape):
+    """Several rows per CTA, ragged chunk counts, a row count below the CTA count."""
+    M, K = shape
+    g = RNG.uniform(0.5, 1.5, K).astype(np.float32)
+    b = (RNG.standard_normal(K) * 0.1).astype(np.float32) if kind == oracle.NORM_LAYER else None
+    x = _acts(M, K, dtype)
+    am_o = oracle.calibrate_absmax(x, kind, g, b)
+    am_g = sq.calibrate_absmax(to_gpu(x), kind, to_gpu(g),
+                               None if b is None else to_gpu(b)).cpu().numpy()
+    ties = norm_near_tie_rows(x, kind, 1e-5)
+    if not ties.any():
+        assert np.array_equal(am_g.view(np.uint32), am_o.view(np.uint32))
+    else:
+        assert np.all(np.abs(am_g - am_o) <= 2 * np.spacing(am_o))
+
+
+@pytest.mark.parametrize("NK", [(5000, 4112), (20000, 64), (3, 2056)], ids=lambda s: "%dx%d" % s)
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_weight_column_max_through_scales(NK, dtype):
+    """alpha = 0 makes s_j = 1 / max(w_j, eps): the column maxima of a tall,
+    ragged weight come back exactly through s."""
+    N, K = NK
+    W = (RNG.standard_normal((N, K)) * 0.02).astype(np.float32)
+    W[RNG.integers(0, N, 40), RNG.integers(0, K, 40)] = 3.5  # isolated column peaks
+    W[:, 7] = 0.0
+    if dtype == "bf16":
+        W = S.to_bf16_bits(W)
+    act_max = np.ones(K, np.float32)
+    s_o, s64 = oracle.smooth_scales(act_max, [W], 0.0, 1e-5)
+    s_g, _, _ = sq.compute_smooth_scales(to_gpu(act_max), [to_gpu(W)], 0.0, 1e-5)
+    s_g = s_g.cpu().numpy()
+    diff = s_g.view(np.uint32) != s_o.view(np.uint32)
+    assert not np.any(diff & ~scale_near_tie_channels(s64))
 
 
 @pytest.mark.parametrize("alpha", [0.0, 0.5, 0.8, 1.0])

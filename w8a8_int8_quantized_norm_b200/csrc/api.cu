@@ -137,8 +137,10 @@ sq_status sq_calibrate_absmax(const void* x, sq_dtype dtype, int64_t M, int64_t 
   if ((st = check_vec(act_max, true)) != SQ_OK) return st;
   if ((st = check_vec(gamma, false)) != SQ_OK) return st;
   if ((st = check_vec(beta, false)) != SQ_OK) return st;
+  int* err = device_error_word();
+  if (!err) return SQ_ERR_CUDA;
   return from_cuda(launch_calibrate(x, dtype == SQ_BF16, M, static_cast<int>(K), ldx, norm, gamma,
-                                    beta, eps, act_max, as_stream(stream)));
+                                    beta, eps, act_max, err, as_stream(stream)));
 }
 
 sq_status sq_compute_smooth_scales(const float* act_max, const void* const* W, const int64_t* N,

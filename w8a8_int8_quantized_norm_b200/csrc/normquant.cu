@@ -123,21 +123,72 @@ __device__ __forceinline__ uint2 codes8(const float2 (&v)[4], float rstep, float
   return make_uint2(lo, hi);
 }
 
+// fl32(a / 127) for every non-negative finite binary32 a, in three
+// instructions: q0 = fl32(a c) with c = fl32(1/127) is within an ulp of the
+// quotient, the remainder a - 127 q0 is exact in one fused multiply-add, and a
+// second one corrects q0.  The sequence was compared with the IEEE quotient
+// for all 2^31 - 2^23 such inputs (subnormals included) and agrees on every
+// one; infinities take the division.
+__device__ __forceinline__ float div127(float a) {
+  constexpr float c = 1.0f / 127.0f;
+  if (!(a <= FLT_MAX)) return __fdiv_rn(a, 127.0f);
+  const float q0 = __fmul_rn(a, c);
+  const float r = __fmaf_rn(-q0, 127.0f, a);
+  return __fmaf_rn(r, c, q0);
+}
+
+// Bounded wait for the copy of the CTA's row number `i` (buffer i mod nbuf).
+__device__ __forceinline__ bool row_landed(uint32_t bar_base, int nbuf, int i) {
+  const uint32_t bar = bar_base + 8u * static_cast<uint32_t>(i % nbuf);
+  const uint32_t parity = static_cast<uint32_t>((i / nbuf) & 1);
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long c0 = clock64();
+  for (uint32_t k = 0;; ++k) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((k & 63u) == 63u && clock64() - c0 > kWaitBudgetCycles) return false;
+  }
+}
+
+// The buffer of row number `i` has been read: load the row nbuf further on
+// into it (if there is one).  Returns the new count of issued copies.
+__device__ __forceinline__ int refill_row(uint32_t smem_base, uint32_t bar_base,
+                                          uint32_t buf_stride, uint32_t row_bytes, int nbuf, int i,
+                                          int64_t row, int64_t G, int64_t M, const uint8_t* xb,
+                                          int64_t row_pitch, int issued) {
+  const int pb = i % nbuf;
+  const int64_t nrow = row + static_cast<int64_t>(nbuf) * G;
+  if (nrow >= M) return issued;
+  mbar_arrive_expect_tx(bar_base + 8u * pb, row_bytes);
+  bulk_load(smem_base + pb * buf_stride, xb + nrow * row_pitch, row_bytes, bar_base + 8u * pb);
+  return i + nbuf + 1;
+}
+
 // NORMK: 0 = no norm (optional per-channel multiplier), 1 = RMSNorm, 2 = LayerNorm.
-template <int CH>
+template <int CH, bool kCalib>
 struct PipeBounds {
   static constexpr int kMaxThreads = CH <= 4 ? 512 : 640;
-  // 4-chunk CTAs keep to 64 registers a thread so four 256-thread CTAs fit an SM
-  static constexpr int kMinBlocks = CH <= 4 ? 2 : 1;
+  // 4-chunk quantising CTAs keep to 64 registers a thread so four 256-thread
+  // CTAs fit an SM; calibration also keeps a running column max per element
+  static constexpr int kMinBlocks = (CH <= 4 && !kCalib) ? 2 : 1;
 };
 
+// One row per iteration, three CTA barriers per row (two when calibrating):
+//   A  the warps' partial sums are in shared memory (norm kinds only); the
+//      row buffer has been read into registers, so it is refilled here;
+//   B  warp 0 has turned the sums into r (and mu);
+//   C  the warps' partial absmax is merged, and thread 0 has seen the next
+//      row land (a bounded wait; a timeout aborts the CTA).
+// Calibrating (kCalib) folds C into B and keeps a per-thread running max of
+// |y| over the rows it sees, merged into act_max at the end.
+//
 // kFull: every thread owns all CH of its chunks (T * CH == K / 8): no bounds checks.
-template <bool kBF16, int NORMK, int CH, bool kGamma, bool kBeta, bool kFull>
-__global__ void __launch_bounds__(PipeBounds<CH>::kMaxThreads, PipeBounds<CH>::kMinBlocks)
-    norm_quant_pipe_kernel(
-    const void* __restrict__ x, int64_t ldx, int64_t M, int K, const float* __restrict__ gamma,
-    const float* __restrict__ beta, float eps, int8_t* __restrict__ q, float* __restrict__ scale,
-    int nbuf, int* error_word) {
+template <bool kBF16, int NORMK, int CH, bool kGamma, bool kBeta, bool kFull, bool kCalib>
+__global__ void __launch_bounds__(PipeBounds<CH, kCalib>::kMaxThreads,
+                                  PipeBounds<CH, kCalib>::kMinBlocks)
+    norm_rows_pipe_kernel(const void* __restrict__ x, int64_t ldx, int64_t M, int K,
+                          const float* __restrict__ gamma, const float* __restrict__ beta,
+                          float eps, int8_t* __restrict__ q, float* __restrict__ scale,
+                          float* __restrict__ act_max, int nbuf, int* error_word) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int kEsz = kBF16 ? 2 : 4;
   const uint32_t row_bytes = static_cast<uint32_t>(K) * kEsz;
@@ -145,7 +196,10 @@ __global__ void __launch_bounds__(PipeBounds<CH>::kMaxThreads, PipeBounds<CH>::k
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + nbuf * buf_stride);
   double* dscr = reinterpret_cast<double*>(bars + nbuf);      // [64]: sum x^2, sum x per warp
   float* fscr = reinterpret_cast<float*>(dscr + 64);           // [2]: r, mu of the row
-  unsigned int* smax = reinterpret_cast<unsigned int*>(fscr + 2);  // [2]: row absmax bits
+  // [3]: row absmax bits, rotating: row i merges into slot i mod 3 before
+  // barrier C and reads it after; thread 0 clears the slot of row i + 2 after
+  // C, which every thread passes again (C of row i + 1) before touching it
+  unsigned int* smax = reinterpret_cast<unsigned int*>(fscr + 2);
   const uint32_t smem_base = smem_u32(smem);
   const uint32_t bar_base = smem_u32(bars);
 
@@ -161,61 +215,43 @@ __global__ void __launch_bounds__(PipeBounds<CH>::kMaxThreads, PipeBounds<CH>::k
     for (int b = 0; b < nbuf; ++b) mbar_init(bar_base + 8u * b, 1);
     smax[0] = 0u;
     smax[1] = 0u;
+    smax[2] = 0u;
     mbar_fence_init();
   }
   __syncthreads();
-  int last_phase[8];  // thread 0: phase of the latest copy issued into each buffer (-1: none)
-#pragma unroll
-  for (int b = 0; b < 8; ++b) last_phase[b] = (b < nbuf && first + b * G < M) ? 0 : -1;
+  // thread 0: row copies issued so far, in the CTA's row order (the first
+  // nbuf at once, then one refill per iteration, each into the buffer of the
+  // row it replaces)
+  int issued = 0;
   if (t == 0) {
     for (int b = 0; b < nbuf; ++b) {
       const int64_t row = first + b * G;
       if (row < M) {
         mbar_arrive_expect_tx(bar_base + 8u * b, row_bytes);
         bulk_load(smem_base + b * buf_stride, xb + row * row_pitch, row_bytes, bar_base + 8u * b);
+        issued = b + 1;
       }
     }
   }
+  bool aborted = false;
+  {
+    const bool ok = (t != 0 || first >= M) ? true : row_landed(bar_base, nbuf, 0);
+    if (__syncthreads_or(!ok)) aborted = true;
+  }
+  float2 cm[kCalib ? CH : 1][4];  // calibration: running max of |y| per owned element
+  if constexpr (kCalib) {
+#pragma unroll
+    for (int c = 0; c < CH; ++c)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) cm[c][i] = make_float2(0.0f, 0.0f);
+  }
 
   int it = 0;
-  bool aborted = false;
-  for (int64_t row = first; row < M; row += G, ++it) {
-    const int b = it % nbuf;
-    const int slot = it & 1;
-    // one thread watches the row's barrier; the others sleep in the CTA barrier
-    bool ok = true;
-    if (t == 0) {
-      const uint32_t parity = static_cast<uint32_t>((it / nbuf) & 1);
-      ok = mbar_try_wait(bar_base + 8u * b, parity);
-      if (!ok) {
-        const long long c0 = clock64();
-        for (uint32_t i = 0; !ok; ++i) {
-          ok = mbar_try_wait(bar_base + 8u * b, parity);
-          if (!ok && (i & 63u) == 63u && clock64() - c0 > kWaitBudgetCycles) break;
-        }
-      }
-    }
-    if (__syncthreads_or(!ok)) {
-      if (t == 0) record_device_error(error_word, SQ_ERR_PIPELINE_TIMEOUT);
-      aborted = true;
-      break;
-    }
-    // all threads are past the previous row: refill its buffer
-    if (t == 0 && it > 0) {
-      const int pb = (it - 1) % nbuf;
-      const int64_t nrow = row - G + static_cast<int64_t>(nbuf) * G;
-      if (nrow < M) {
-        mbar_arrive_expect_tx(bar_base + 8u * pb, row_bytes);
-        bulk_load(smem_base + pb * buf_stride, xb + nrow * row_pitch, row_bytes,
-                  bar_base + 8u * pb);
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          if (k == pb) ++last_phase[k];
-      }
-    }
-    const uint8_t* rowp = smem + b * buf_stride;
+  for (int64_t row = first; row < M && !aborted; row += G, ++it) {
+    const int slot = it % 3;
+    const uint8_t* rowp = smem + (it % nbuf) * buf_stride;
 
-    // ---- load this thread's chunks of the row from shared memory
+    // ---- this thread's chunks of the row, from shared memory
     float2 v[CH][4];
 #pragma unroll
     for (int c = 0; c < CH; ++c) {
@@ -228,7 +264,6 @@ __global__ void __launch_bounds__(PipeBounds<CH>::kMaxThreads, PipeBounds<CH>::k
       }
     }
     // ---- row statistics in fp64 (two accumulators per sum for ILP)
-    float mu = 0.0f, r = 1.0f;
     if constexpr (NORMK != 0) {
       double s1a = 0.0, s1b = 0.0, s2a = 0.0, s2b = 0.0;
 #pragma unroll
@@ -251,7 +286,10 @@ __global__ void __launch_bounds__(PipeBounds<CH>::kMaxThreads, PipeBounds<CH>::k
         dscr[warp] = s2;
         if constexpr (NORMK == 2) dscr[32 + warp] = s1;
       }
-      __syncthreads();
+      __syncthreads();  // A
+      if (t == 0)
+        issued = refill_row(smem_base, bar_base, buf_stride, row_bytes, nbuf, it, row, G, M, xb,
+                            row_pitch, issued);
       // one warp turns the sums into the row's scalars (the fp64 divide and
       // square root are long instruction sequences: not worth repeating in
       // every warp)
@@ -278,13 +316,28 @@ __global__ void __launch_bounds__(PipeBounds<CH>::kMaxThreads, PipeBounds<CH>::k
           fscr[1] = mu32;
         }
       }
-      __syncthreads();
+    }
+    if constexpr (kCalib) {
+      // B (with C folded in): the row scalars are published and the next row is in
+      const bool ok = (t != 0 || row + G >= M) ? true : row_landed(bar_base, nbuf, it + 1);
+      if (__syncthreads_or(!ok)) {
+        aborted = true;
+        break;
+      }
+      if (NORMK == 0 && t == 0)
+        issued = refill_row(smem_base, bar_base, buf_stride, row_bytes, nbuf, it, row, G, M, xb,
+                            row_pitch, issued);
+    } else if constexpr (NORMK != 0) {
+      __syncthreads();  // B
+    }
+    float mu = 0.0f, r = 1.0f;
+    if constexpr (NORMK != 0) {
       r = fscr[0];
       mu = fscr[1];
     }
-    // ---- the norm output and its absmax (paired fp32 ops, same roundings;
-    // a multiply followed by an add uses the scalar intrinsics, which are
-    // never contracted into a fused multiply-add)
+    // ---- the norm output (paired fp32 ops, same roundings; a multiply
+    // followed by an add uses the scalar intrinsics, which are never
+    // contracted into a fused multiply-add)
     float am = 0.0f;
     const float2 r2 = make_float2(r, r), nmu2 = make_float2(-mu, -mu);
 #pragma unroll
@@ -309,38 +362,77 @@ __global__ void __launch_bounds__(PipeBounds<CH>::kMaxThreads, PipeBounds<CH>::k
         } else if constexpr (kGamma) {
           y = __fmul2_rn(y, g[i]);
         }
-        v[c][i] = y;
-        am = fmaxf(am, fmaxf(fabsf(y.x), fabsf(y.y)));
+        if constexpr (kCalib) {
+          cm[c][i].x = fmaxf(cm[c][i].x, fabsf(y.x));
+          cm[c][i].y = fmaxf(cm[c][i].y, fabsf(y.y));
+        } else {
+          v[c][i] = y;
+          am = fmaxf(am, fmaxf(fabsf(y.x), fabsf(y.y)));
+        }
       }
     }
-    // non-negative floats order like their bit patterns: integer max reduce
-    const unsigned int wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(am));
-    if (lane == 0) atomicMax(&smax[slot], wmax);
-    __syncthreads();
-    am = __uint_as_float(smax[slot]);
-    if (t == 0) smax[slot ^ 1] = 0u;  // the next row's slot starts from zero
+    if constexpr (!kCalib) {
+      // non-negative floats order like their bit patterns: integer max reduce
+      const unsigned int wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(am));
+      if (lane == 0) atomicMax(&smax[slot], wmax);
+      const bool ok = (t != 0 || row + G >= M) ? true : row_landed(bar_base, nbuf, it + 1);
+      if (__syncthreads_or(!ok)) {  // C
+        aborted = true;
+        break;
+      }
+      if (NORMK == 0 && t == 0)
+        issued = refill_row(smem_base, bar_base, buf_stride, row_bytes, nbuf, it, row, G, M, xb,
+                            row_pitch, issued);
+      am = __uint_as_float(smax[slot]);
+      if (t == 0) smax[slot == 0 ? 2 : slot - 1] = 0u;  // the slot of row it + 2
 
-    // ---- per-token INT8 quantisation
-    const float step = __fdiv_rn(am, 127.0f);
-    const bool exact_only = step < FLT_MIN;  // zero or subnormal step: no reciprocal
-    const float rstep = exact_only ? 0.0f : __fdiv_rn(1.0f, step);
-    if (t == 0) scale[row] = step;
-    int8_t* qrow = q + row * static_cast<int64_t>(K);
+      // ---- per-token INT8 quantisation
+      const float step = div127(am);
+      const bool exact_only = step < FLT_MIN;  // zero or subnormal step: no reciprocal
+      const float rstep = exact_only ? 0.0f : __frcp_rn(step);
+      if (t == 0) scale[row] = step;
+      int8_t* qrow = q + row * static_cast<int64_t>(K);
+#pragma unroll
+      for (int c = 0; c < CH; ++c) {
+        const int ch = t + c * T;
+        if (!kFull && ch >= nchunks) continue;
+        *reinterpret_cast<uint2*>(qrow + ch * kChunk) = codes8(v[c], rstep, step, exact_only);
+      }
+    }
+  }
+  if (aborted) {
+    if (t == 0) {
+      record_device_error(error_word, SQ_ERR_PIPELINE_TIMEOUT);
+      // let every bulk copy still in flight land before the CTA exits: the
+      // latest copy into buffer b is the one of row number s (s = b mod nbuf,
+      // s < issued), which completes phase s / nbuf of the buffer's barrier
+      for (int b = 0; b < nbuf && b < issued; ++b) {
+        const int s_last = b + (issued - 1 - b) / nbuf * nbuf;
+        const uint32_t par = static_cast<uint32_t>((s_last / nbuf) & 1);
+        const long long c0 = clock64();
+        while (!mbar_try_wait(bar_base + 8u * b, par) && clock64() - c0 < kWaitBudgetCycles) {
+        }
+      }
+    }
+    return;
+  }
+  if constexpr (kCalib) {
+    // merge into the running maximum: an atomic only where this CTA's value is
+    // larger than what act_max already holds (the maximum only grows, so a
+    // stale read costs an extra atomic, never a lost update)
+    unsigned int* am_bits = reinterpret_cast<unsigned int*>(act_max);
 #pragma unroll
     for (int c = 0; c < CH; ++c) {
       const int ch = t + c * T;
       if (!kFull && ch >= nchunks) continue;
-      *reinterpret_cast<uint2*>(qrow + ch * kChunk) = codes8(v[c], rstep, step, exact_only);
-    }
-  }
-  if (aborted && t == 0) {
-    // let every bulk copy still in flight land before the CTA exits
+      const uint4 cur0 = __ldcg(reinterpret_cast<const uint4*>(am_bits + ch * kChunk));
+      const uint4 cur1 = __ldcg(reinterpret_cast<const uint4*>(am_bits + ch * kChunk + 4));
+      const unsigned int cur[8] = {cur0.x, cur0.y, cur0.z, cur0.w, cur1.x, cur1.y, cur1.z, cur1.w};
 #pragma unroll
-    for (int b = 0; b < 8; ++b) {
-      if (last_phase[b] < 0) continue;
-      const uint32_t par = static_cast<uint32_t>(last_phase[b] & 1);
-      const long long c0 = clock64();
-      while (!mbar_try_wait(bar_base + 8u * b, par) && clock64() - c0 < kWaitBudgetCycles) {
+      for (int i = 0; i < 4; ++i) {
+        const unsigned int a0 = __float_as_uint(cm[c][i].x), a1 = __float_as_uint(cm[c][i].y);
+        if (a0 > cur[2 * i]) atomicMax(am_bits + ch * kChunk + 2 * i, a0);
+        if (a1 > cur[2 * i + 1]) atomicMax(am_bits + ch * kChunk + 2 * i + 1, a1);
       }
     }
   }
@@ -351,11 +443,14 @@ struct PipeShape {
   size_t smem;
 };
 
+// row buffers, their barriers, 64 doubles of partial sums, r and mu, 3 absmax slots
+size_t pipe_smem(size_t stride, int nbuf) { return nbuf * stride + 8 * nbuf + 64 * 8 + 4 * 8; }
+
 bool pipe_shape(int K, bool bf16, PipeShape* ps) {
   const int nchunks = K / kChunk;
   // chunks per thread and threads per CTA within the variant's register budget
-  int ch = nchunks <= 4 * PipeBounds<4>::kMaxThreads ? 4
-           : (nchunks <= 8 * PipeBounds<8>::kMaxThreads ? 8 : 0);
+  int ch = nchunks <= 4 * PipeBounds<4, false>::kMaxThreads ? 4
+           : (nchunks <= 8 * PipeBounds<8, false>::kMaxThreads ? 8 : 0);
   if (!ch) return false;
   int threads = (nchunks + ch - 1) / ch;
   threads = (threads + 31) / 32 * 32;
@@ -370,61 +465,90 @@ bool pipe_shape(int K, bool bf16, PipeShape* ps) {
   ps->ch = ch;
   ps->threads = threads;
   ps->nbuf = nbuf;
-  ps->smem = nbuf * stride + 8 * nbuf + 64 * 8 + 4 * 4;
+  ps->smem = pipe_smem(stride, nbuf);
   return true;
 }
 
-template <bool kBF16, int NORMK, int CH, bool kG, bool kB, bool kF>
-cudaError_t launch_pipe_k(const void* x, int64_t M, int K, int64_t ldx, const float* gamma,
-                          const float* beta, float eps, int8_t* q, float* scale,
-                          const PipeShape& ps, int* err, cudaStream_t st) {
-  auto kern = norm_quant_pipe_kernel<kBF16, NORMK, CH, kG, kB, kF>;
+struct RowArgs {
+  const void* x;
+  int64_t M;
+  int K;
+  int64_t ldx;
+  const float* gamma;
+  const float* beta;
+  float eps;
+  int8_t* q;
+  float* scale;
+  float* act_max;
+  int* err;
+};
+
+template <bool kBF16, int NORMK, int CH, bool kG, bool kB, bool kF, bool kC>
+cudaError_t launch_pipe_k(const RowArgs& a, PipeShape ps, cudaStream_t st) {
+  auto kern = norm_rows_pipe_kernel<kBF16, NORMK, CH, kG, kB, kF, kC>;
+  const void* key = reinterpret_cast<const void*>(kern);
   LaunchCache& lc = launch_cache();
-  const cudaError_t e = lc.ensure_smem(reinterpret_cast<const void*>(kern), ps.smem);
-  if (e != cudaSuccess) return e;
-  const int per_sm = lc.blocks_per_sm(reinterpret_cast<const void*>(kern), ps.threads, ps.smem);
+  int per_sm = 0;
+  // fewer row buffers when each CTA sees only a few rows: more CTAs fit an SM
+  const size_t stride = (static_cast<size_t>(a.K) * (kBF16 ? 2 : 4) + 127) / 128 * 128;
+  for (;;) {
+    cudaError_t e = lc.ensure_smem(key, ps.smem);
+    if (e != cudaSuccess) return e;
+    per_sm = lc.blocks_per_sm(key, ps.threads, ps.smem);
+    const int64_t ctas = static_cast<int64_t>(per_sm) * lc.sms();
+    const int64_t rows_per_cta = (a.M + ctas - 1) / ctas;
+    if (ps.nbuf <= 2 || rows_per_cta >= ps.nbuf) break;
+    ps.nbuf = rows_per_cta < 2 ? 2 : static_cast<int>(rows_per_cta);
+    ps.smem = pipe_smem(stride, ps.nbuf);
+  }
   int64_t grid = static_cast<int64_t>(per_sm) * lc.sms();
-  if (grid > M) grid = M;
-  kern<<<static_cast<unsigned>(grid), ps.threads, ps.smem, st>>>(x, ldx, M, K, gamma, beta, eps,
-                                                                   q, scale, ps.nbuf, err);
+  if (grid > a.M) grid = a.M;
+  kern<<<static_cast<unsigned>(grid), ps.threads, ps.smem, st>>>(
+      a.x, a.ldx, a.M, a.K, a.gamma, a.beta, a.eps, a.q, a.scale, a.act_max, ps.nbuf, a.err);
   return cudaGetLastError();
 }
 
-template <bool kBF16, int NORMK, int CH, bool kG, bool kB>
-cudaError_t launch_pipe_t(const void* x, int64_t M, int K, int64_t ldx, const float* gamma,
-                          const float* beta, float eps, int8_t* q, float* scale,
-                          const PipeShape& ps, int* err, cudaStream_t st) {
+template <bool kBF16, int NORMK, int CH, bool kG, bool kB, bool kC>
+cudaError_t launch_pipe_t(const RowArgs& a, const PipeShape& ps, cudaStream_t st) {
   // bf16 rows whose chunks split evenly over the threads skip the bounds checks
   if constexpr (kBF16) {
-    if (ps.threads * ps.ch == K / kChunk)
-      return launch_pipe_k<kBF16, NORMK, CH, kG, kB, true>(x, M, K, ldx, gamma, beta, eps, q,
-                                                           scale, ps, err, st);
+    if (ps.threads * ps.ch == a.K / kChunk)
+      return launch_pipe_k<kBF16, NORMK, CH, kG, kB, true, kC>(a, ps, st);
   }
-  return launch_pipe_k<kBF16, NORMK, CH, kG, kB, false>(x, M, K, ldx, gamma, beta, eps, q, scale,
-                                                        ps, err, st);
+  return launch_pipe_k<kBF16, NORMK, CH, kG, kB, false, kC>(a, ps, st);
 }
 
-template <bool kBF16, int NORMK, int CH>
-cudaError_t launch_pipe_c(const void* x, int64_t M, int K, int64_t ldx, const float* gamma,
-                          const float* beta, float eps, int8_t* q, float* scale,
-                          const PipeShape& ps, int* err, cudaStream_t st) {
+template <bool kBF16, int NORMK, int CH, bool kC>
+cudaError_t launch_pipe_c(const RowArgs& a, const PipeShape& ps, cudaStream_t st) {
   // beta only matters for LayerNorm
-  const bool hb = NORMK == 2 && beta != nullptr;
-  if (gamma) {
-    if (hb) return launch_pipe_t<kBF16, NORMK, CH, true, NORMK == 2>(x, M, K, ldx, gamma, beta, eps, q, scale, ps, err, st);
-    return launch_pipe_t<kBF16, NORMK, CH, true, false>(x, M, K, ldx, gamma, beta, eps, q, scale, ps, err, st);
+  const bool hb = NORMK == 2 && a.beta != nullptr;
+  if (a.gamma) {
+    if (hb) return launch_pipe_t<kBF16, NORMK, CH, true, NORMK == 2, kC>(a, ps, st);
+    return launch_pipe_t<kBF16, NORMK, CH, true, false, kC>(a, ps, st);
   }
-  if (hb) return launch_pipe_t<kBF16, NORMK, CH, false, NORMK == 2>(x, M, K, ldx, gamma, beta, eps, q, scale, ps, err, st);
-  return launch_pipe_t<kBF16, NORMK, CH, false, false>(x, M, K, ldx, gamma, beta, eps, q, scale, ps, err, st);
+  if (hb) return launch_pipe_t<kBF16, NORMK, CH, false, NORMK == 2, kC>(a, ps, st);
+  return launch_pipe_t<kBF16, NORMK, CH, false, false, kC>(a, ps, st);
 }
 
-template <bool kBF16, int NORMK>
-cudaError_t launch_pipe_n(const void* x, int64_t M, int K, int64_t ldx, const float* gamma,
-                          const float* beta, float eps, int8_t* q, float* scale,
-                          const PipeShape& ps, int* err, cudaStream_t st) {
-  if (ps.ch == 4)
-    return launch_pipe_c<kBF16, NORMK, 4>(x, M, K, ldx, gamma, beta, eps, q, scale, ps, err, st);
-  return launch_pipe_c<kBF16, NORMK, 8>(x, M, K, ldx, gamma, beta, eps, q, scale, ps, err, st);
+template <bool kBF16, int NORMK, bool kC>
+cudaError_t launch_pipe_n(const RowArgs& a, const PipeShape& ps, cudaStream_t st) {
+  if (ps.ch == 4) return launch_pipe_c<kBF16, NORMK, 4, kC>(a, ps, st);
+  if constexpr (kC) return cudaErrorInvalidValue;  // calibration: 4-chunk shapes only
+  else return launch_pipe_c<kBF16, NORMK, 8, kC>(a, ps, st);
+}
+
+template <bool kC>
+cudaError_t launch_rows(const RowArgs& a, bool bf16, int norm, cudaStream_t st) {
+  PipeShape ps;
+  if (!pipe_shape(a.K, bf16, &ps)) return cudaErrorInvalidValue;
+  if (bf16) {
+    if (norm == SQ_NORM_RMS) return launch_pipe_n<true, 1, kC>(a, ps, st);
+    if (norm == SQ_NORM_LAYER) return launch_pipe_n<true, 2, kC>(a, ps, st);
+    return launch_pipe_n<true, 0, kC>(a, ps, st);
+  }
+  if (norm == SQ_NORM_RMS) return launch_pipe_n<false, 1, kC>(a, ps, st);
+  if (norm == SQ_NORM_LAYER) return launch_pipe_n<false, 2, kC>(a, ps, st);
+  return launch_pipe_n<false, 0, kC>(a, ps, st);
 }
 
 }  // namespace
@@ -434,24 +558,25 @@ bool norm_quant_pipe_supported(int K, bool bf16) {
   return pipe_shape(K, bf16, &ps);
 }
 
+bool calibrate_pipe_supported(int K, bool bf16) {
+  PipeShape ps;
+  return pipe_shape(K, bf16, &ps) && ps.ch == 4;
+}
+
 cudaError_t launch_norm_quant_pipe(const void* x, bool bf16, int64_t M, int K, int64_t ldx,
                                    int norm, const float* gamma, const float* beta, float eps,
                                    int8_t* q, float* scale, int* err, cudaStream_t st) {
   if (M == 0) return cudaSuccess;
-  PipeShape ps;
-  if (!pipe_shape(K, bf16, &ps)) return cudaErrorInvalidValue;
-  if (bf16) {
-    if (norm == SQ_NORM_RMS)
-      return launch_pipe_n<true, 1>(x, M, K, ldx, gamma, beta, eps, q, scale, ps, err, st);
-    if (norm == SQ_NORM_LAYER)
-      return launch_pipe_n<true, 2>(x, M, K, ldx, gamma, beta, eps, q, scale, ps, err, st);
-    return launch_pipe_n<true, 0>(x, M, K, ldx, gamma, beta, eps, q, scale, ps, err, st);
-  }
-  if (norm == SQ_NORM_RMS)
-    return launch_pipe_n<false, 1>(x, M, K, ldx, gamma, beta, eps, q, scale, ps, err, st);
-  if (norm == SQ_NORM_LAYER)
-    return launch_pipe_n<false, 2>(x, M, K, ldx, gamma, beta, eps, q, scale, ps, err, st);
-  return launch_pipe_n<false, 0>(x, M, K, ldx, gamma, beta, eps, q, scale, ps, err, st);
+  const RowArgs a{x, M, K, ldx, gamma, beta, eps, q, scale, nullptr, err};
+  return launch_rows<false>(a, bf16, norm, st);
+}
+
+cudaError_t launch_calibrate_pipe(const void* x, bool bf16, int64_t M, int K, int64_t ldx,
+                                  int norm, const float* gamma, const float* beta, float eps,
+                                  float* act_max, int* err, cudaStream_t st) {
+  if (M == 0) return cudaSuccess;
+  const RowArgs a{x, M, K, ldx, gamma, beta, eps, nullptr, nullptr, act_max, err};
+  return launch_rows<true>(a, bf16, norm, st);
 }
 
 }  // namespace sq

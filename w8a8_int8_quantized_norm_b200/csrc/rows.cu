@@ -222,42 +222,60 @@ __global__ void __launch_bounds__(RowBounds<CH>::kMaxThreads) calib_kernel(
                 __float_as_uint(colmax[ch * kChunk + i]));
 }
 
-// Column absmax of a weight [N, K]: thread owns one 8-column chunk and a run
-// of rows; merged with an atomic max on the bit pattern into wmax[K].
+// Column absmax of a weight [N, K].  A CTA owns a slab of 256 columns (one
+// 8-column chunk per lane, so every warp reads 512 contiguous bytes of a bf16
+// row) and a run of rows, split over its 8 warps with 8 independent 16-byte
+// loads in flight per thread; the warps' maxima meet in shared memory, and
+// each column is merged into wmax with an atomic max on the bit pattern --
+// issued only where this CTA's value beats the one already there.
 template <bool kBF16>
 __global__ void __launch_bounds__(256) weight_colmax_kernel(const void* __restrict__ W, int64_t N,
-                                                            int K, int rows_per_cta,
+                                                            int K, int64_t rows_per_cta,
                                                             float* __restrict__ wmax) {
+  __shared__ __align__(16) float red[8][kChunk * 32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nchunks = K / kChunk;
-  const int ch = blockIdx.x * blockDim.x + threadIdx.x;
-  if (ch >= nchunks) return;
-  const int64_t r0 = (int64_t)blockIdx.y * rows_per_cta;
-  const int64_t r1 = min(N, r0 + rows_per_cta);
+  const int ch = blockIdx.x * 32 + lane;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rows_per_cta;
+  const int64_t r1 = r0 + rows_per_cta < N ? r0 + rows_per_cta : N;
   float m[kChunk];
 #pragma unroll
   for (int i = 0; i < kChunk; ++i) m[i] = 0.0f;
-  // eight independent 128-bit loads in flight per thread
-  constexpr int U = 8;
-  int64_t n = r0;
-  for (; n + U <= r1; n += U) {
-    float v[U][kChunk];
+  if (ch < nchunks) {
+    constexpr int U = 8;
+    int64_t n = r0 + warp;
+    for (; n + 8 * (U - 1) < r1; n += 8 * U) {
+      float v[U][kChunk];
 #pragma unroll
-    for (int u = 0; u < U; ++u) load_chunk<kBF16>(W, (n + u) * (int64_t)K + (int64_t)ch * kChunk, v[u]);
+      for (int u = 0; u < U; ++u)
+        load_chunk<kBF16>(W, (n + 8 * u) * static_cast<int64_t>(K) + static_cast<int64_t>(ch) * kChunk,
+                          v[u]);
 #pragma unroll
-    for (int u = 0; u < U; ++u)
+      for (int u = 0; u < U; ++u)
 #pragma unroll
-      for (int i = 0; i < kChunk; ++i) m[i] = fmaxf(m[i], fabsf(v[u][i]));
+        for (int i = 0; i < kChunk; ++i) m[i] = fmaxf(m[i], fabsf(v[u][i]));
+    }
+    for (; n < r1; n += 8) {
+      float v[kChunk];
+      load_chunk<kBF16>(W, n * static_cast<int64_t>(K) + static_cast<int64_t>(ch) * kChunk, v);
+#pragma unroll
+      for (int i = 0; i < kChunk; ++i) m[i] = fmaxf(m[i], fabsf(v[i]));
+    }
   }
-  for (; n < r1; ++n) {
-    float v[kChunk];
-    load_chunk<kBF16>(W, n * (int64_t)K + (int64_t)ch * kChunk, v);
+  float4* dst = reinterpret_cast<float4*>(&red[warp][lane * kChunk]);
+  dst[0] = make_float4(m[0], m[1], m[2], m[3]);
+  dst[1] = make_float4(m[4], m[5], m[6], m[7]);
+  __syncthreads();
+  const int j = threadIdx.x;  // column of the slab
+  float v = red[0][j];
 #pragma unroll
-    for (int i = 0; i < kChunk; ++i) m[i] = fmaxf(m[i], fabsf(v[i]));
+  for (int w = 1; w < 8; ++w) v = fmaxf(v, red[w][j]);
+  const int64_t col = static_cast<int64_t>(blockIdx.x) * (kChunk * 32) + j;
+  if (col < K) {
+    unsigned int* p = reinterpret_cast<unsigned int*>(wmax) + col;
+    const unsigned int bits = __float_as_uint(v);
+    if (bits > __ldcg(p)) atomicMax(p, bits);
   }
-#pragma unroll
-  for (int i = 0; i < kChunk; ++i)
-    atomicMax(reinterpret_cast<unsigned int*>(wmax) + (int64_t)ch * kChunk + i,
-              __float_as_uint(m[i]));
 }
 
 // s_j = max(max(a,eps)^alpha / max(w,eps)^(1-alpha), eps) in binary64, stored
@@ -325,8 +343,12 @@ cudaError_t launch_norm_quant(const void* x, bool bf16, int64_t M, int K, int64_
 
 cudaError_t launch_calibrate(const void* x, bool bf16, int64_t M, int K, int64_t ldx, int norm,
                              const float* gamma, const float* beta, float eps, float* act_max,
-                             cudaStream_t st) {
+                             int* err, cudaStream_t st) {
   if (M == 0) return cudaSuccess;
+  // rows that fit the shared-memory ring (and a 4-chunk thread layout) take
+  // the pipelined kernel; wider rows keep a column max in shared memory
+  if (calibrate_pipe_supported(K, bf16))
+    return launch_calibrate_pipe(x, bf16, M, K, ldx, norm, gamma, beta, eps, act_max, err, st);
   const int ch = pick_ch(K);
   const int threads = threads_for(K, ch);
   // about two CTAs per SM: enough parallelism, few atomics per channel
@@ -348,16 +370,22 @@ cudaError_t launch_weight_colmax(const void* W, bool bf16, int64_t N, int K, flo
                                  cudaStream_t st) {
   if (N == 0) return cudaSuccess;
   const int nchunks = K / kChunk;
-  const int threads = 256;
-  // at least 64 rows per CTA, more when N would overflow gridDim.y
-  const int64_t rpc = (N + 65534) / 65535;
-  const int rows_per_cta = static_cast<int>(rpc > 64 ? rpc : 64);
-  const dim3 grid((nchunks + threads - 1) / threads,
-                  static_cast<unsigned>((N + rows_per_cta - 1) / rows_per_cta));
+  const int slabs = (nchunks + 31) / 32;
+  // about eight CTAs per SM, at least 64 rows (8 per warp) each, and no more
+  // row runs than gridDim.y allows
+  const int64_t target = 8 * static_cast<int64_t>(launch_cache().sms());
+  int64_t runs = target / slabs;
+  if (runs < 1) runs = 1;
+  int64_t rows = (N + runs - 1) / runs;
+  if (rows < 64) rows = 64;
+  const int64_t min_rows = (N + 65534) / 65535;
+  if (rows < min_rows) rows = min_rows;
+  rows = (rows + 7) / 8 * 8;
+  const dim3 grid(static_cast<unsigned>(slabs), static_cast<unsigned>((N + rows - 1) / rows));
   if (bf16)
-    weight_colmax_kernel<true><<<grid, threads, 0, st>>>(W, N, K, rows_per_cta, wmax);
+    weight_colmax_kernel<true><<<grid, 256, 0, st>>>(W, N, K, rows, wmax);
   else
-    weight_colmax_kernel<false><<<grid, threads, 0, st>>>(W, N, K, rows_per_cta, wmax);
+    weight_colmax_kernel<false><<<grid, 256, 0, st>>>(W, N, K, rows, wmax);
   return cudaGetLastError();
 }
 

@@ -80,9 +80,13 @@ bool norm_quant_pipe_supported(int K, bool bf16);
 cudaError_t launch_norm_quant_pipe(const void* x, bool bf16, int64_t M, int K, int64_t ldx,
                                    int norm, const float* gamma, const float* beta, float eps,
                                    int8_t* q, float* scale, int* err, cudaStream_t st);
+bool calibrate_pipe_supported(int K, bool bf16);
+cudaError_t launch_calibrate_pipe(const void* x, bool bf16, int64_t M, int K, int64_t ldx,
+                                  int norm, const float* gamma, const float* beta, float eps,
+                                  float* act_max, int* err, cudaStream_t st);
 cudaError_t launch_calibrate(const void* x, bool bf16, int64_t M, int K, int64_t ldx, int norm,
                              const float* gamma, const float* beta, float eps, float* act_max,
-                             cudaStream_t st);
+                             int* err, cudaStream_t st);
 cudaError_t launch_weight_colmax(const void* W, bool bf16, int64_t N, int K, float* wmax,
                                  cudaStream_t st);
 cudaError_t launch_smooth_finalize(const float* act_max, float* s, int K, double alpha,

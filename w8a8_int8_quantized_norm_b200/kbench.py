@@ -4,6 +4,7 @@
     python -m w8a8_int8_quantized_norm_b200.kbench gemm --M 2048 --N 12288 --K 4096 --path 1
     python -m w8a8_int8_quantized_norm_b200.kbench calibrate --M 4096 --K 8192 --norm layer
     python -m w8a8_int8_quantized_norm_b200.kbench weight_quant --N 28672 --K 8192
+    python -m w8a8_int8_quantized_norm_b200.kbench smooth_scales --N 12288 --K 4096
 
 Each timed call is bracketed by CUDA events on the launching stream, with the
 L2 cache overwritten (256 MiB, untimed) before every call, so the operands come
@@ -70,7 +71,8 @@ def _time(fn, iters, warmup, flush, stream):
 
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
-    ap.add_argument("op", choices=["norm_quant", "gemm", "calibrate", "weight_quant"])
+    ap.add_argument("op", choices=["norm_quant", "gemm", "calibrate", "weight_quant",
+                                   "smooth_scales"])
     ap.add_argument("--M", type=int, default=4096)
     ap.add_argument("--N", type=int, default=4096)
     ap.add_argument("--K", type=int, default=4096)
@@ -122,6 +124,17 @@ def main(argv=None):
         wsc = torch.empty(N, dtype=torch.float32, device=dev)
         fn = lambda: sq.smooth_quantize_weights(W, s, Wq=wq, w_scale=wsc, stream=stream)
         units = N * K * (esz + 1) + 4 * N + 4 * K
+        shape = {"N": N, "K": K, "dtype": a.dtype}
+    elif a.op == "smooth_scales":
+        W = (torch.randn((N, K), generator=gen, device=dev) * 0.02)
+        W = W.to(torch.bfloat16) if a.dtype == "bf16" else W
+        am = torch.empty(K, device=dev).uniform_(0.1, 60.0, generator=gen)
+        g = torch.empty(K, device=dev).uniform_(0.5, 1.5, generator=gen)
+        s = torch.empty(K, dtype=torch.float32, device=dev)
+        gf = torch.empty(K, dtype=torch.float32, device=dev)
+        fn = lambda: sq.compute_smooth_scales(am, [W], 0.5, 1e-5, g, None, s=s, gamma_folded=gf,
+                                              stream=stream)
+        units = N * K * esz + 16 * K
         shape = {"N": N, "K": K, "dtype": a.dtype}
     else:
         A, B = _codes(M, K, gen, dev), _codes(N, K, gen, dev)
