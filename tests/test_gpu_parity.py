@@ -185,7 +185,7 @@ def test_calibration_many_rows(kind, dtype, shape):
         assert np.all(np.abs(am_g - am_o) <= 2 * np.spacing(am_o))
 
 
-@pytest.mark.parametrize("NK", [(5000, 4112), (20000, 64), (3, 2056)], ids=lambda s: "%dx%d" % s)
+@pytest.mark.parametrize("NK", [(5000, 4112), (20000, 64), (3, 2064)], ids=lambda s: "%dx%d" % s)
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_weight_column_max_through_scales(NK, dtype):
     """alpha = 0 makes s_j = 1 / max(w_j, eps): the column maxima of a tall,
