@@ -366,23 +366,26 @@ def run_gpu(args, w):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    events = []  # (kind, units, start event, end event) of every library call
+    events = []  # (kind, units, start event, end event) of every library call in a step
 
     def timer(kind, units, fn):
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
+        e0.record()
         fn()
-        e1.record(stream)
+        e1.record()
         events.append((kind, units, e0, e1))
 
-    def step(timed):
-        blk.prepare(xc, W, g, b, timer=timer if timed else None)
-        blk.forward(x, timer=timer if timed else None)
-
+    # eager warm-up, then the whole step captured once as a CUDA graph (the
+    # per-call event records are captured with it and time every replay)
     for _ in range(args.warmup):
         flush.zero_()
-        step(False)
+        blk.prepare(xc, W, g, b)
+        blk.forward(x)
+    graph = blk.capture(xc, W, g, b, x, timer=timer)
+    for _ in range(args.warmup):
+        flush.zero_()
+        graph.replay()
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
@@ -397,15 +400,22 @@ def run_gpu(args, w):
     sampler = ClockSampler(pci)
     sampler.start()
     wall0 = time.perf_counter()
-    step_ev = []
+    step_ms = []
+    kinds = {}  # kind -> [calls, units, seconds]
     for _ in range(args.steps):
-        flush.zero_()  # L2 holds nothing of the step's inputs when it starts
+        flush.zero_()  # L2 holds nothing of the step's inputs when it starts (untimed)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        step(True)
+        graph.replay()
         e1.record(stream)
-        step_ev.append((e0, e1))
+        e1.synchronize()
+        step_ms.append(e0.elapsed_time(e1))
+        for (kind, units, a, b_) in events:
+            k = kinds.setdefault(kind, [0, 0.0, 0.0])
+            k[0] += 1
+            k[1] += units
+            k[2] += a.elapsed_time(b_) / 1e3
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
@@ -416,20 +426,13 @@ def run_gpu(args, w):
     if err:
         raise SystemExit("device error %s during the benchmark" % sq.status_string(err))
 
-    step_ms = [a.elapsed_time(b_) for a, b_ in step_ev]
     t_rank = sum(step_ms) / 1e3
     ops = workload_ops(w)
     tops_total, t_max = aggregate(ops * args.steps, t_rank, world, dev)
     value = tops_total / 1e12
     tokens_per_s = w.M * args.steps * world / t_max
 
-    # per library call: CUDA events on the launching stream around every call
-    kinds = {}
-    for (kind, units, a, b_) in events:
-        k = kinds.setdefault(kind, [0, 0.0, 0.0])
-        k[0] += 1
-        k[1] += units
-        k[2] += a.elapsed_time(b_) / 1e3
+    # per library call: CUDA events recorded around every call inside the graph
     peaks, peak_src = load_peaks()
     kernels = {}
     for kind, (n, units, secs) in kinds.items():
@@ -458,11 +461,17 @@ def run_gpu(args, w):
                 "peak_sustained": peaks.get("bf16_tflops_sustained", 0.0) * INT8_PER_BF16}
     roof["peak_source"] = "%s (%s)" % (peak_src, "HBM copy" if decode else
                                        "2 x bf16 cuBLAS, the nominal INT8:BF16 ratio")
-    tr = profile_traffic("w8a8_gemm_kernel", w.name)
+    plan = sq.gemm_plan(w.M, w.linears[0].N, w.site(w.linears[0].site).K)
+    kname = sq.GemmPlanInfo.KERNELS[plan.kernel].split(" ")[0]
+    tr = profile_traffic(kname, w.name)
     roof["traffic"] = None if tr is None else tr
     roof["algorithmic_per_launch"] = (g_bytes if decode else g_ops) / g_n
-    roof["kernel"] = "w8a8_gemm_kernel"
+    roof["kernel"] = kname
+    roof["plan"] = {k: v for k, v in plan.as_dict().items() if k != "kernel"}
     roof["launch_ms_mean"] = g_time * 1e3 / g_n
+    roof["timing"] = ("CUDA events recorded around each GEMM call inside the captured step "
+                      "graph, every timed replay (a call = the main kernel plus its fix-up "
+                      "kernel when the plan has one)")
 
     line = {
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
@@ -472,6 +481,7 @@ def run_gpu(args, w):
         "config": {"workload": w.name, "tokens": w.M, "calib_tokens": w.M_cal, "alpha": w.alpha,
                    "linears": ["%s %dx%d" % (l.name, w.site(l.site).K, l.N) for l in w.linears],
                    "step": "calibrate + smooth scales/fold + weight quant + norm-quant + GEMM",
+                   "launch": "the whole step replayed as one CUDA graph",
                    "l2": "flushed before every step (256 MiB write, not timed)",
                    "parallelism": "dp%d (independent token batches, weights replicated)" % world},
         "tokens_per_s": tokens_per_s,

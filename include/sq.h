@@ -185,6 +185,27 @@ sq_status sq_norm_smooth_quant_per_token(const void* x, sq_dtype dtype, int64_t 
  */
 size_t sq_w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int split_k);
 
+/* What sq_w8a8_gemm_dequant will run for a shape (filled by sq_w8a8_gemm_plan). */
+typedef struct sq_gemm_plan_info {
+  int kernel;      /* 0: single-SM prefill tiles, 1: CTA-pair prefill tiles, 2: decode tiles */
+  int tile_m;      /* rows of a tile on the MMA M side (tokens, or weight rows for decode) */
+  int tile_n;      /* columns of a tile on the MMA N side */
+  int split_k;     /* K slices per tile (1: none) */
+  int stream_k;    /* 1: balanced K ranges per SM with a fix-up kernel */
+  int ctas;        /* CTAs of the main kernel (persistent: at most one per SM) */
+  int launches;    /* kernels the call launches */
+  size_t workspace_bytes;
+} sq_gemm_plan_info;
+
+/*
+ * sq_w8a8_gemm_plan -- host-only: the plan sq_w8a8_gemm_dequant would choose
+ * for these arguments on the current device (no launch, no allocation).
+ * Errors: SQ_ERR_INVALID_ARG (negative sizes, K <= 0, bad hint or split,
+ * null info), SQ_ERR_UNSUPPORTED (a split on a prefill path).
+ */
+sq_status sq_w8a8_gemm_plan(int64_t M, int64_t N, int64_t K, int path_hint, int split_k,
+                            sq_gemm_plan_info* info);
+
 /*
  * sq_w8a8_gemm_dequant -- INT8 x INT8 -> INT32 GEMM with the dequantising
  * epilogue fused.
@@ -197,16 +218,19 @@ size_t sq_w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int split_k)
  *   x_scale  device [M] fp32;  w_scale device [N] fp32 (ignored for I32_RAW)
  *   epi      SQ_EPI_BF16, SQ_EPI_BF16_RELU (out is bf16 [M, N], stride ldo)
  *            or SQ_EPI_I32_RAW (out is int32 [M, N], stride ldo)
- *   workspace / ws_bytes  device scratch for split-K partial sums; at least
+ *   workspace / ws_bytes  device scratch for partial sums (split-K slices,
+ *            or the stream-K slots of decode tiles); at least
  *            sq_w8a8_gemm_workspace_size(M, N, K, split_k) bytes when that is
- *            non-zero, else may be NULL
+ *            non-zero, else may be NULL.  Nothing in it outlives the call.
  *   path_hint 0 = automatic, 1 = prefill tiles (tokens on the MMA M side;
  *            CTA pairs, 256 x 256 tiles on two SMs), 2 = decode tiles (weight
  *            rows on the MMA M side, M <= 256), 3 = prefill tiles on single
  *            SMs (128 x 256)
  *   split_k  0 = automatic, else the number of K slices (decode path only;
  *            the INT32 partial sums are added exactly, so the result does not
- *            depend on it)
+ *            depend on it).  The automatic decode plan is stream-K: every SM
+ *            runs the same number of 128-deep K steps across tile boundaries,
+ *            and tiles shared by two SMs are summed by a second, small kernel.
  * Accumulation is exact for K <= SQ_MAX_K (else SQ_ERR_OVERFLOW_RISK).
  * Errors: SQ_ERR_INVALID_ARG, SQ_ERR_ALIGNMENT, SQ_ERR_OVERFLOW_RISK,
  *         SQ_ERR_WORKSPACE, SQ_ERR_UNSUPPORTED, SQ_ERR_CUDA.
@@ -252,10 +276,11 @@ sq_status sq_linear_w8a8(const void* x, sq_dtype dtype, int64_t M, int64_t K, in
  *     (different streams, or different host threads) race on it.  Calls in
  *     one stream are ordered and safe.  No state carries over between calls:
  *     every partial sum is written before it is read.
- *   - If the chosen plan needs more split-K scratch than
- *     SQ_NOALLOC_SCRATCH_BYTES (sq_w8a8_gemm_workspace_size tells), the call
- *     returns SQ_ERR_WORKSPACE and launches nothing; pass split_k = 1 (no
- *     scratch) or a smaller split.
+ *   - With split_k = 0, a decode plan whose stream-K slots would not fit the
+ *     array runs whole tiles instead (split_k = 1, no scratch).  An explicit
+ *     split whose partial sums need more than SQ_NOALLOC_SCRATCH_BYTES
+ *     (sq_w8a8_gemm_workspace_size tells) returns SQ_ERR_WORKSPACE and
+ *     launches nothing; pass split_k = 1 (no scratch) or a smaller split.
  * Results are bit-identical to sq_w8a8_gemm_dequant's for the same plan.
  * Errors: those of sq_w8a8_gemm_dequant.
  */

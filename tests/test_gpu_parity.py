@@ -434,3 +434,35 @@ def test_workload_llama_block_prefill_sampled():
 @pytest.mark.parametrize("M", [1, 8, 32, 128])
 def test_workload_llama_block_decode(M):
     _check_workload(S.WORKLOADS["llama-block-8192-decode-m%d" % M])
+
+
+@pytest.mark.parametrize("wname", ["opt-prefill-rmsnorm-qkv-2048x4096x12288",
+                                   "llama-block-8192-decode-m1"])
+def test_graph_replay_matches_eager_step(wname):
+    """The benchmark replays the whole step as one CUDA graph: every buffer the
+    step writes must come out bit-identical to the eager calls' results."""
+    w = S.WORKLOADS[wname]
+    inp_w, _, prep_g = _family_state(w)
+    inp = S.make_inputs(w, seed=0, weights=False)
+    x = {k: to_gpu(v) for k, v in inp.x.items()}
+    blk = pipeline.Block(w, w.M, "cuda")
+    blk.prepare(prep_g["xc"], prep_g["W"], prep_g["g"], prep_g["b"])
+    blk.forward(x)
+    torch.cuda.synchronize()
+
+    def snapshot():
+        bufs = [blk.out, blk.xq, blk.xs, blk.Wq, blk.w_scale, blk.act_max, blk.s, blk.gamma_f]
+        return {(i, k): v.clone() for i, d in enumerate(bufs) for k, v in d.items()
+                if v is not None}
+
+    eager = snapshot()
+    graph = blk.capture(prep_g["xc"], prep_g["W"], prep_g["g"], prep_g["b"], x)
+    for d in (blk.out, blk.xq, blk.Wq):
+        for v in d.values():
+            v.zero_()
+    for _ in range(2):
+        graph.replay()
+    torch.cuda.synchronize()
+    for key, v in snapshot().items():
+        assert torch.equal(v, eager[key]), key
+    del graph

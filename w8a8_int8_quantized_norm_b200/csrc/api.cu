@@ -224,6 +224,33 @@ size_t sq_w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int split_k)
   return need;
 }
 
+sq_status sq_w8a8_gemm_plan(int64_t M, int64_t N, int64_t K, int path_hint, int split_k,
+                            sq_gemm_plan_info* info) {
+  if (!info || M < 0 || N < 0 || K <= 0 || split_k < 0 || path_hint < 0 || path_hint > 3)
+    return SQ_ERR_INVALID_ARG;
+  const int sms = sms_cached();
+  const GemmPlan plan = plan_gemm(M, N, K, path_hint, split_k, sms);
+  if (!plan.swap && split_k > 1) return SQ_ERR_UNSUPPORTED;
+  sq_gemm_plan_info r{};
+  r.kernel = plan.swap ? 2 : (plan.pair ? 1 : 0);
+  r.tile_m = plan.pair ? 256 : 128;
+  r.tile_n = plan.pair ? 256 : plan.bn;
+  r.split_k = plan.splits;
+  r.stream_k = plan.streamk;
+  const int64_t p_rows = plan.swap ? N : M, q_rows = plan.swap ? M : N;
+  const int64_t tiles = ((p_rows + r.tile_m - 1) / r.tile_m) * ((q_rows + r.tile_n - 1) / r.tile_n);
+  int64_t ctas = plan.streamk ? plan.grid : tiles * plan.splits;
+  const int64_t sm_count = sms > 0 ? sms : 148;  // the planner's own default
+  const int64_t cap = plan.pair ? (sm_count / 2) * 2 : sm_count;
+  if (plan.pair) ctas *= 2;
+  if (ctas > cap) ctas = cap;
+  r.ctas = static_cast<int>(M == 0 || N == 0 ? 0 : ctas);
+  r.launches = (M == 0 || N == 0) ? 0 : 1 + (plan.workspace_bytes > 0 ? 1 : 0);
+  r.workspace_bytes = plan.workspace_bytes;
+  *info = r;
+  return SQ_OK;
+}
+
 sq_status sq_w8a8_gemm_dequant(const int8_t* Xq, const int8_t* Wq, const float* x_scale,
                                const float* w_scale, int64_t M, int64_t N, int64_t K,
                                sq_epilogue epi, void* out, int64_t ldo, void* workspace,

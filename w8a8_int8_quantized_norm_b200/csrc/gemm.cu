@@ -76,6 +76,14 @@ struct Params {
   int64_t wait_polls;              // > 0: poll budget per wait; 0: ~2 s of SM clock cycles
   int* error_word;                 // device error word of this device
   int vec_out;                     // output rows 16-byte aligned: 128-bit stores allowed
+  // stream-K (decode tiles): CTA c runs the flattened (tile, k-block)
+  // iterations [c * sk_iters / G, (c + 1) * sk_iters / G); a tile whose K
+  // range is split between CTAs leaves partial sums in slots 2c (the CTA's
+  // first tile) and 2c + 1 (its last), [slot][Q][128], summed afterwards by
+  // streamk_fixup_kernel
+  int streamk;
+  int64_t sk_iters;
+  int32_t* sk_partial;
 };
 
 // Give-up point of a pipeline wait, in SM clock cycles (about 2 s at the
@@ -108,10 +116,9 @@ __device__ __forceinline__ void fail(int* word, volatile int* abort) {
   *abort = 1;
 }
 
-__device__ __forceinline__ void decode_unit(const Params& p, int u, int& pb, int& qb, int& kb0,
-                                            int& kb1, int& split) {
-  split = u % p.splits;
-  const int tile = u / p.splits;
+// Tile number -> (P block, Q block): bands of `group` P blocks sweep all Q
+// blocks before the next band starts, so a band's Q operand stays in L2.
+__device__ __forceinline__ void tile_coords(const Params& p, int tile, int& pb, int& qb) {
   const int band_tiles = p.group * p.q_blocks;
   const int band = tile / band_tiles;
   const int rem = tile - band * band_tiles;
@@ -119,16 +126,73 @@ __device__ __forceinline__ void decode_unit(const Params& p, int u, int& pb, int
   const int gsize = min(p.group, p.p_blocks - first);
   pb = first + rem % gsize;
   qb = rem / gsize;
+}
+
+__device__ __forceinline__ void decode_unit(const Params& p, int u, int& pb, int& qb, int& kb0,
+                                            int& kb1, int& split) {
+  split = u % p.splits;
+  tile_coords(p, u / p.splits, pb, qb);
   kb0 = static_cast<int>((static_cast<int64_t>(split) * p.k_blocks) / p.splits);
   kb1 = static_cast<int>((static_cast<int64_t>(split + 1) * p.k_blocks) / p.splits);
+}
+
+// The work units of one CTA, in order: round-robin tiles (or split-K slices),
+// or the CTA's stream-K range cut at tile boundaries.  All three warp roles
+// walk the same sequence.
+struct Work {
+  int u;               // round-robin unit
+  int64_t it, it_end;  // stream-K iteration range still to run
+  bool first;          // stream-K: the next unit is the CTA's first
+};
+
+__device__ __forceinline__ int64_t sk_start(const Params& p, int64_t c) {
+  return c * p.sk_iters / gridDim.x;
+}
+
+__device__ __forceinline__ void work_init(const Params& p, Work& w) {
+  w.u = blockIdx.x;
+  w.it = sk_start(p, blockIdx.x);
+  w.it_end = sk_start(p, blockIdx.x + 1);
+  w.first = true;
+}
+
+// Next unit of the CTA, or false.  slot < 0: the unit ends in the output (or
+// its split-K slice); slot >= 0: a stream-K partial-sum slot.
+__device__ __forceinline__ bool work_next(const Params& p, Work& w, int& pb, int& qb, int& kb0,
+                                          int& kb1, int& split, int& slot) {
+  if (p.streamk) {
+    if (w.it >= w.it_end) return false;
+    const int tile = static_cast<int>(w.it / p.k_blocks);
+    kb0 = static_cast<int>(w.it - static_cast<int64_t>(tile) * p.k_blocks);
+    const int64_t left = w.it_end - w.it;
+    kb1 = left < p.k_blocks - kb0 ? kb0 + static_cast<int>(left) : p.k_blocks;
+    w.it += kb1 - kb0;
+    tile_coords(p, tile, pb, qb);
+    split = 0;
+    slot = (kb0 == 0 && kb1 == p.k_blocks) ? -1 : 2 * static_cast<int>(blockIdx.x) + (w.first ? 0 : 1);
+    w.first = false;
+    return true;
+  }
+  if (w.u >= p.units) return false;
+  decode_unit(p, w.u, pb, qb, kb0, kb1, split);
+  slot = -1;
+  w.u += gridDim.x;
+  return true;
 }
 
 // Epilogue for one CHUNK of accumulator columns held by this thread (row p of
 // the P side, columns q0 .. q0 + CHUNK - 1 of the Q side).
 template <int CHUNK>
 __device__ __forceinline__ void store_chunk(const Params& prm, const uint32_t (&r)[32], int p,
-                                            int q0, int split) {
+                                            int q0, int split, int slot) {
   if (p >= prm.P) return;
+  if (slot >= 0) {  // stream-K partial sums of a decode tile: [slot][Q][128]
+    int32_t* dst = prm.sk_partial + static_cast<int64_t>(slot) * prm.Q * BM + (p % BM);
+#pragma unroll
+    for (int j = 0; j < CHUNK; ++j)
+      if (q0 + j < prm.Q) dst[static_cast<int64_t>(q0 + j) * BM] = static_cast<int32_t>(r[j]);
+    return;
+  }
   if (prm.partial) {  // split-K partial sums, [split][M][N] with M = Q (tokens), N = P
 #pragma unroll
     for (int j = 0; j < CHUNK; ++j) {
@@ -272,9 +336,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t phase = 0;
     int64_t issued = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < prm.units && ok; u += gridDim.x) {
-      int pb, qb, kb0, kb1, split;
-      decode_unit(prm, u, pb, qb, kb0, kb1, split);
+    Work wk;
+    work_init(prm, wk);
+    int pb, qb, kb0, kb1, split, slot;
+    while (ok && work_next(prm, wk, pb, qb, kb0, kb1, split, slot)) {
       for (int kb = kb0; kb < kb1; ++kb) {
         bool w = false;
         if (lane == 0) w = wait_phase(EMPTY_BAR(stage), phase ^ 1u, polls, abort_flag);
@@ -306,9 +371,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < prm.units && ok; u += gridDim.x) {
-      int pb, qb, kb0, kb1, split;
-      decode_unit(prm, u, pb, qb, kb0, kb1, split);
+    Work wk;
+    work_init(prm, wk);
+    int pb, qb, kb0, kb1, split, slot;
+    while (ok && work_next(prm, wk, pb, qb, kb0, kb1, split, slot)) {
       bool w = false;
       if (lane == 0) w = wait_phase(TEMPTY_BAR(acc), acc_phase ^ 1u, polls, abort_flag);
       w = __shfl_sync(0xffffffffu, w, 0);
@@ -362,9 +428,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;  // tensor-memory lanes this warp may access
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int u = blockIdx.x; u < prm.units; u += gridDim.x) {
-      int pb, qb, kb0, kb1, split;
-      decode_unit(prm, u, pb, qb, kb0, kb1, split);
+    Work wk;
+    work_init(prm, wk);
+    int pb, qb, kb0, kb1, split, slot;
+    while (work_next(prm, wk, pb, qb, kb0, kb1, split, slot)) {
       bool w = false;
       if (lane == 0) w = wait_phase(TFULL_BAR(acc), acc_phase, polls, abort_flag);
       w = __shfl_sync(0xffffffffu, w, 0);
@@ -385,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         else
           tmem_ld_32x32b_x16(taddr, r);
         tmem_wait_ld();
-        store_chunk<C::CHUNK>(prm, r, p, qb * BN + c * C::CHUNK, split);
+        store_chunk<C::CHUNK>(prm, r, p, qb * BN + c * C::CHUNK, split, slot);
       }
       tc_fence_before();
       __syncwarp();
@@ -638,7 +705,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                static_cast<uint32_t>(acc * TILE + c * 32);
         tmem_ld_32x32b_x32(taddr, r);
         tmem_wait_ld();
-        store_chunk<32>(prm, r, p, qb * TILE + c * 32, 0);
+        store_chunk<32>(prm, r, p, qb * TILE + c * 32, 0, -1);
       }
       tc_fence_before();
       __syncwarp();
@@ -678,6 +745,46 @@ __global__ void __launch_bounds__(kThreads, 1)
 #undef EMPTY_BAR
 #undef TFULL_BAR
 #undef TEMPTY_BAR
+}
+
+// Stream-K fix-up for decode tiles (weight rows on the P side, tokens on the
+// Q side, one Q block).  Block b looks at the start of CTA c = b + 1: if that
+// iteration lies inside a tile and no earlier CTA starts inside the same
+// tile, the block sums the tile's partial slots (CTA c - 1 up to the last CTA
+// starting before the tile ends) and applies the epilogue; thread = row of
+// the tile's 128 P rows.  INT32 addition is exact, so the result equals the
+// unsplit accumulation.
+__global__ void __launch_bounds__(BM) streamk_fixup_kernel(const Params prm, int G) {
+  const int c = static_cast<int>(blockIdx.x) + 1;
+  const int64_t kbt = prm.k_blocks;
+  const int64_t b = static_cast<int64_t>(c) * prm.sk_iters / G;
+  if (b % kbt == 0) return;
+  const int64_t tile = b / kbt;
+  const int64_t t0 = tile * kbt, t1 = t0 + kbt;
+  if (static_cast<int64_t>(c - 1) * prm.sk_iters / G > t0) return;  // not the first boundary
+  int pb, qb;
+  tile_coords(prm, static_cast<int>(tile), pb, qb);
+  const int pl = static_cast<int>(threadIdx.x);
+  const int p = pb * BM + pl;
+  if (p >= prm.P) return;
+  const float ws = prm.epi == SQ_EPI_I32_RAW ? 0.0f : __ldg(prm.p_scale + p);
+  for (int q = 0; q < prm.Q; ++q) {
+    int32_t acc = 0;
+    for (int cc = c - 1; cc < G; ++cc) {
+      const int64_t sc = static_cast<int64_t>(cc) * prm.sk_iters / G;
+      if (sc >= t1) break;
+      const int64_t slot = (sc / kbt == tile) ? 2 * cc : 2 * cc + 1;
+      acc += __ldcg(prm.sk_partial + (slot * prm.Q + q) * BM + pl);
+    }
+    if (prm.epi == SQ_EPI_I32_RAW) {
+      static_cast<int32_t*>(prm.out)[static_cast<int64_t>(q) * prm.ldo + p] = acc;
+    } else {
+      float t = __fmul_rn(__fmul_rn(__int2float_rn(acc), __ldg(prm.q_scale + q)), ws);
+      if (prm.epi == SQ_EPI_BF16_RELU) t = fmaxf(t, 0.0f);
+      static_cast<__nv_bfloat16*>(prm.out)[static_cast<int64_t>(q) * prm.ldo + p] =
+          __float2bfloat16_rn(t);
+    }
+  }
 }
 
 // out[m][n] = epilogue(sum_s partial[s][m][n]); INT32 addition is exact, so
@@ -803,6 +910,22 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int path_hint, int split_k, 
     p.bn = 256;
     p.splits = 1;
     p.pair = path_hint == 3 ? 0 : 1;
+  } else if (split_k <= 0) {
+    // decode tiles, stream-K: every SM streams the same number of k-blocks
+    p.bn = bn_for_tokens(M);
+    const int64_t tiles = (N + BM - 1) / BM;
+    const int64_t iters = tiles * kblocks;
+    const int64_t sms = num_sms > 0 ? num_sms : 148;
+    const int64_t G = iters < sms ? iters : sms;
+    p.splits = 1;
+    p.streamk = 1;
+    p.grid = static_cast<int>(G);
+    p.sk_iters = iters;
+    bool split_tiles = false;
+    for (int64_t c = 1; c < G && !split_tiles; ++c) split_tiles = (c * iters / G) % kblocks != 0;
+    p.workspace_bytes = split_tiles ? static_cast<size_t>(2 * G) * BM * static_cast<size_t>(M) * 4u
+                                    : 0u;
+    return p;
   } else {
     p.bn = bn_for_tokens(M);
     const int64_t tiles = (N + BM - 1) / BM;
@@ -861,6 +984,9 @@ cudaError_t launch_gemm(const GemmPlan& plan, const int8_t* Xq, const int8_t* Wq
   prm.epi = epi;
   prm.swap = plan.swap;
   prm.partial = plan.splits > 1 ? static_cast<int32_t*>(workspace) : nullptr;
+  prm.streamk = plan.streamk;
+  prm.sk_iters = plan.sk_iters;
+  prm.sk_partial = plan.streamk ? static_cast<int32_t*>(workspace) : nullptr;
   prm.wait_polls = wait_polls;
   prm.error_word = error_word;
   {
@@ -879,7 +1005,7 @@ cudaError_t launch_gemm(const GemmPlan& plan, const int8_t* Xq, const int8_t* Wq
   }
   if (!make_map(&mp, Pptr, prm.P, K, BM) || !make_map(&mq, Qptr, prm.Q, K, plan.bn))
     return cudaErrorInvalidValue;
-  const int grid = prm.units < sms ? prm.units : sms;
+  const int grid = plan.streamk ? plan.grid : (prm.units < sms ? prm.units : sms);
   cudaError_t e;
   switch (plan.bn) {
     case 16: e = launch_bn<16>(prm, mp, mq, grid, st); break;
@@ -889,7 +1015,13 @@ cudaError_t launch_gemm(const GemmPlan& plan, const int8_t* Xq, const int8_t* Wq
     case 256: e = launch_bn<256>(prm, mp, mq, grid, st); break;
     default: return cudaErrorInvalidValue;
   }
-  if (e != cudaSuccess || plan.splits <= 1) return e;
+  if (e != cudaSuccess) return e;
+  if (plan.streamk) {
+    if (plan.workspace_bytes == 0 || plan.grid < 2) return cudaSuccess;
+    streamk_fixup_kernel<<<plan.grid - 1, BM, 0, st>>>(prm, plan.grid);
+    return cudaGetLastError();
+  }
+  if (plan.splits <= 1) return e;
   const int64_t total = M * N;
   int blocks = static_cast<int>((total + 255) / 256);
   if (blocks > sms * 8) blocks = sms * 8;

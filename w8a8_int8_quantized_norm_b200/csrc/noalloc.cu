@@ -63,7 +63,12 @@ extern "C" sq_status sq_w8a8_gemm_dequant_noalloc(const int8_t* Xq, const int8_t
                                 path_hint, split_k, stream);
   }
   const int sms = num_sms_current_device();
-  const GemmPlan plan = plan_gemm(M, N, K, path_hint, split_k, sms);
+  GemmPlan plan = plan_gemm(M, N, K, path_hint, split_k, sms);
+  if (plan.workspace_bytes > SQ_NOALLOC_SCRATCH_BYTES && split_k == 0 && plan.streamk) {
+    // the automatic decode plan's stream-K slots do not fit: whole tiles, no scratch
+    split_k = 1;
+    plan = plan_gemm(M, N, K, path_hint, split_k, sms);
+  }
   if (plan.workspace_bytes > SQ_NOALLOC_SCRATCH_BYTES) return SQ_ERR_WORKSPACE;
   void* scratch = plan.workspace_bytes > 0 ? scratch_address() : nullptr;
   if (plan.workspace_bytes > 0 && !scratch) return SQ_ERR_CUDA;

@@ -99,6 +99,9 @@ struct GemmPlan {
   int pair;       // prefill on CTA pairs (2-SM MMA, 256 x 256 tiles)
   int bn;         // MMA N (tile width on the Q side)
   int splits;     // K slices
+  int streamk;    // decode tiles: balanced k-block ranges per CTA + a fix-up pass
+  int grid;       // stream-K: CTAs
+  int64_t sk_iters;  // stream-K: tiles x k-blocks
   size_t workspace_bytes;
 };
 GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int path_hint, int split_k, int num_sms);

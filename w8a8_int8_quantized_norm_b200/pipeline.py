@@ -147,12 +147,34 @@ class Block:
         return n + len(self.w.linears)
 
     def forward_launches(self) -> int:
-        """Kernels one ``forward`` launches: norm-quant per site, the GEMM per
-        Linear, plus the split-K reduction where the plan splits K."""
+        """Kernels one ``forward`` launches: norm-quant per site, and per Linear
+        the kernels of its GEMM plan (the main kernel, plus the split-K
+        reduction or stream-K fix-up where the plan has one)."""
         n = len(self.w.sites)
         for lin in self.w.linears:
-            n += 2 if self.ws[lin.name] is not None else 1
+            n += sq.gemm_plan(self.M, lin.N, self.w.site(lin.site).K).launches
         return n
+
+    # -- CUDA graph ----------------------------------------------------------
+    def capture(self, x_cal, W, gamma, beta, x, timer: Timer = None, warmup: int = 1):
+        """Records one whole step (``prepare`` then ``forward``) into a CUDA
+        graph and returns it; ``graph.replay()`` reruns every kernel of the
+        step on the current stream with no host work per kernel.  The step's
+        tensors must stay where they are between replays (the graph holds their
+        addresses).  ``timer`` hooks are captured too (e.g. CUDA event records,
+        which then time each call inside every replay)."""
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):  # first use of each kernel outside the capture
+            for _ in range(warmup):
+                self.prepare(x_cal, W, gamma, beta)
+                self.forward(x)
+        torch.cuda.current_stream().wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            self.prepare(x_cal, W, gamma, beta, timer=timer)
+            self.forward(x, timer=timer)
+        return graph
 
 
 # Thin functional wrappers (used by tests and the smoke check).

@@ -33,9 +33,23 @@ EXPORTS = (
     "sq_calibrate_absmax", "sq_compute_smooth_scales", "sq_smooth_quantize_weights",
     "sq_norm_smooth_quant_per_token", "sq_w8a8_gemm_workspace_size", "sq_w8a8_gemm_dequant",
     "sq_linear_w8a8", "sq_status_string", "sq_get_device_error", "sq_set_wait_limit",
-    "sq_w8a8_gemm_dequant_noalloc",
+    "sq_w8a8_gemm_dequant_noalloc", "sq_w8a8_gemm_plan",
 )
 NOALLOC_SCRATCH_BYTES = 8 << 20
+
+
+class GemmPlanInfo(ctypes.Structure):
+    """sq_gemm_plan_info: what sq_w8a8_gemm_dequant runs for a shape."""
+    _fields_ = [("kernel", ctypes.c_int), ("tile_m", ctypes.c_int), ("tile_n", ctypes.c_int),
+                ("split_k", ctypes.c_int), ("stream_k", ctypes.c_int), ("ctas", ctypes.c_int),
+                ("launches", ctypes.c_int), ("workspace_bytes", ctypes.c_size_t)]
+
+    KERNELS = ("w8a8_gemm_kernel", "w8a8_gemm_pair_kernel", "w8a8_gemm_kernel (decode tiles)")
+
+    def as_dict(self):
+        d = {f: getattr(self, f) for f, _ in self._fields_}
+        d["kernel_name"] = self.KERNELS[self.kernel]
+        return d
 
 
 class SQError(RuntimeError):
@@ -87,6 +101,7 @@ def _declare(L):
     L.sq_status_string.argtypes = [_I32]
     L.sq_status_string.restype = ctypes.c_char_p
     L.sq_get_device_error.argtypes = [_P]
+    L.sq_w8a8_gemm_plan.argtypes = [_I64, _I64, _I64, _I32, _I32, ctypes.POINTER(GemmPlanInfo)]
     L.sq_set_wait_limit.argtypes = [_I64]
     L.sq_set_wait_limit.restype = None
     for name in EXPORTS:
@@ -214,6 +229,13 @@ def norm_smooth_quant_per_token(x: torch.Tensor, norm: int, gamma_folded=None, b
         _ptr(_vec(beta_folded, K, "beta_folded")), eps, _ptr(Xq), _ptr(x_scale), _stream(stream)),
         "sq_norm_smooth_quant_per_token")
     return Xq, x_scale
+
+
+def gemm_plan(M: int, N: int, K: int, path_hint: int = 0, split_k: int = 0) -> GemmPlanInfo:
+    info = GemmPlanInfo()
+    _check(lib().sq_w8a8_gemm_plan(M, N, K, path_hint, split_k, ctypes.byref(info)),
+           "sq_w8a8_gemm_plan")
+    return info
 
 
 def gemm_workspace_size(M: int, N: int, K: int, split_k: int = 0) -> int:
