@@ -748,12 +748,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Stream-K fix-up for decode tiles (weight rows on the P side, tokens on the
-// Q side, one Q block).  Block b looks at the start of CTA c = b + 1: if that
-// iteration lies inside a tile and no earlier CTA starts inside the same
+// Q side, one Q block).  Block (b, y) looks at the start of CTA c = b + 1: if
+// that iteration lies inside a tile and no earlier CTA starts inside the same
 // tile, the block sums the tile's partial slots (CTA c - 1 up to the last CTA
-// starting before the tile ends) and applies the epilogue; thread = row of
-// the tile's 128 P rows.  INT32 addition is exact, so the result equals the
+// starting before the tile ends) for tokens q = y * kFixQ ... and applies the
+// epilogue; thread = row of the tile's 128 P rows, so every load and store is
+// 128 consecutive words.  INT32 addition is exact, so the result equals the
 // unsplit accumulation.
+constexpr int kFixQ = 8;  // tokens per fix-up block
+
 __global__ void __launch_bounds__(BM) streamk_fixup_kernel(const Params prm, int G) {
   const int c = static_cast<int>(blockIdx.x) + 1;
   const int64_t kbt = prm.k_blocks;
@@ -767,22 +770,31 @@ __global__ void __launch_bounds__(BM) streamk_fixup_kernel(const Params prm, int
   const int pl = static_cast<int>(threadIdx.x);
   const int p = pb * BM + pl;
   if (p >= prm.P) return;
+  const int q0 = static_cast<int>(blockIdx.y) * kFixQ;
+  const int nq = min(kFixQ, prm.Q - q0);
+  int32_t acc[kFixQ];
+#pragma unroll
+  for (int j = 0; j < kFixQ; ++j) acc[j] = 0;
+  for (int cc = c - 1; cc < G; ++cc) {
+    const int64_t sc = static_cast<int64_t>(cc) * prm.sk_iters / G;
+    if (sc >= t1) break;
+    const int64_t slot = (sc / kbt == tile) ? 2 * cc : 2 * cc + 1;
+    const int32_t* src = prm.sk_partial + (slot * prm.Q + q0) * BM + pl;
+#pragma unroll
+    for (int j = 0; j < kFixQ; ++j)
+      if (j < nq) acc[j] += __ldcg(src + j * BM);
+  }
   const float ws = prm.epi == SQ_EPI_I32_RAW ? 0.0f : __ldg(prm.p_scale + p);
-  for (int q = 0; q < prm.Q; ++q) {
-    int32_t acc = 0;
-    for (int cc = c - 1; cc < G; ++cc) {
-      const int64_t sc = static_cast<int64_t>(cc) * prm.sk_iters / G;
-      if (sc >= t1) break;
-      const int64_t slot = (sc / kbt == tile) ? 2 * cc : 2 * cc + 1;
-      acc += __ldcg(prm.sk_partial + (slot * prm.Q + q) * BM + pl);
-    }
+#pragma unroll
+  for (int j = 0; j < kFixQ; ++j) {
+    if (j >= nq) break;
+    const int64_t o = static_cast<int64_t>(q0 + j) * prm.ldo + p;
     if (prm.epi == SQ_EPI_I32_RAW) {
-      static_cast<int32_t*>(prm.out)[static_cast<int64_t>(q) * prm.ldo + p] = acc;
+      static_cast<int32_t*>(prm.out)[o] = acc[j];
     } else {
-      float t = __fmul_rn(__fmul_rn(__int2float_rn(acc), __ldg(prm.q_scale + q)), ws);
+      float t = __fmul_rn(__fmul_rn(__int2float_rn(acc[j]), __ldg(prm.q_scale + q0 + j)), ws);
       if (prm.epi == SQ_EPI_BF16_RELU) t = fmaxf(t, 0.0f);
-      static_cast<__nv_bfloat16*>(prm.out)[static_cast<int64_t>(q) * prm.ldo + p] =
-          __float2bfloat16_rn(t);
+      static_cast<__nv_bfloat16*>(prm.out)[o] = __float2bfloat16_rn(t);
     }
   }
 }
@@ -1018,7 +1030,9 @@ cudaError_t launch_gemm(const GemmPlan& plan, const int8_t* Xq, const int8_t* Wq
   if (e != cudaSuccess) return e;
   if (plan.streamk) {
     if (plan.workspace_bytes == 0 || plan.grid < 2) return cudaSuccess;
-    streamk_fixup_kernel<<<plan.grid - 1, BM, 0, st>>>(prm, plan.grid);
+    const dim3 fgrid(static_cast<unsigned>(plan.grid - 1),
+                     static_cast<unsigned>((prm.Q + kFixQ - 1) / kFixQ));
+    streamk_fixup_kernel<<<fgrid, BM, 0, st>>>(prm, plan.grid);
     return cudaGetLastError();
   }
   if (plan.splits <= 1) return e;
