@@ -380,9 +380,9 @@ def run_gpu(args, w):
         blk.prepare(xc, W, g, b, timer=timer if timed else None)
         blk.forward(x, timer=timer if timed else None)
 
-    # warm-up; the host time to enqueue one step sets the GPU-side head start
-    # (a spin kernel before each timed step, untimed) that keeps the launch
-    # queue ahead of the GPU, so every event brackets device work only
+    # warm-up (eager), then the step captured once as a CUDA graph: the timed
+    # region replays it, each replay bracketed by events on the launching
+    # stream after an untimed L2 overwrite
     enqueue_s = 0.0
     for _ in range(args.warmup):
         flush.zero_()
@@ -391,7 +391,10 @@ def run_gpu(args, w):
         step(True)
         enqueue_s = max(enqueue_s, time.perf_counter() - t0)
         events.clear()
-    head_cycles = int(2.0e9 * (2.0 * enqueue_s + 50e-6))
+    graph = blk.capture(xc, W, g, b, x)
+    for _ in range(args.warmup):
+        flush.zero_()
+        graph.replay()
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
@@ -409,50 +412,44 @@ def run_gpu(args, w):
     step_ev = []
     for _ in range(args.steps):
         flush.zero_()  # L2 holds nothing of the step's inputs when it starts (untimed)
-        torch.cuda._sleep(head_cycles)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        step(True)
+        graph.replay()
         e1.record(stream)
         step_ev.append((e0, e1))
-        if len(step_ev) % 16 == 0:
-            e1.synchronize()  # bound the queue (the spin must outlast each enqueue)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     wall = time.perf_counter() - wall0
+    step_ms = [a.elapsed_time(b_) for a, b_ in step_ev]
+
+    # per-call breakdown: the same step run eagerly, each call bracketed by
+    # events; every step waits behind an untimed GPU spin sized from the host's
+    # enqueue time, so the queue runs ahead and no host gap enters an interval
+    # (each event record still drains the stream: a few microseconds per call)
+    head_cycles = int(2.0e9 * (2.0 * enqueue_s + 50e-6))
+    n_calls = max(1, min(args.steps, 50))
+    for i in range(n_calls):
+        flush.zero_()
+        torch.cuda._sleep(head_cycles)
+        step(True)
+        if i % 8 == 7:
+            torch.cuda.synchronize(dev)
+    torch.cuda.synchronize(dev)
     clocks = sampler.stop()
     err = sq.get_device_error()
     if err:
         raise SystemExit("device error %s during the benchmark" % sq.status_string(err))
-    step_ms = [a.elapsed_time(b_) for a, b_ in step_ev]
+    del graph
     kinds = {}  # kind -> [calls, units, seconds]
     for (kind, units, a, b_) in events:
         k = kinds.setdefault(kind, [0, 0.0, 0.0])
         k[0] += 1
         k[1] += units
         k[2] += a.elapsed_time(b_) / 1e3
-
-    # the same step captured once as a CUDA graph and replayed (the launch mode
-    # a serving loop would use); reported beside the eager number
-    graph = blk.capture(xc, W, g, b, x)
-    graph_ms = []
-    for i in range(args.warmup + min(args.steps, 50)):
-        flush.zero_()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        graph.replay()
-        e1.record(stream)
-        if i >= args.warmup:
-            graph_ms.append((e0, e1))
-    torch.cuda.synchronize(dev)
-    graph_ms = [a.elapsed_time(b_) for a, b_ in graph_ms]
-    del graph
-    if sq.get_device_error():
-        raise SystemExit("device error during the graph replays")
+    calls_steps = n_calls
 
     t_rank = sum(step_ms) / 1e3
     ops = workload_ops(w)
@@ -467,14 +464,14 @@ def run_gpu(args, w):
         if kind == "gemm":
             continue
         gbs = units / secs / 1e9
-        kernels[kind] = {"calls": n // args.steps, "ms_per_call": secs * 1e3 / n,
+        kernels[kind] = {"calls": n // calls_steps, "ms_per_call": secs * 1e3 / n,
                          "achieved_gbs": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
                          "bytes_per_call": units / n}
     # dominant kernel: the GEMM
     g_n, g_ops, g_time = kinds["gemm"]
     g_bytes = 0
     for lin in w.linears:
-        g_bytes += gemm_bytes(w.M, lin.N, w.site(lin.site).K) * args.steps
+        g_bytes += gemm_bytes(w.M, lin.N, w.site(lin.site).K) * calls_steps
     decode = w.M <= 128
     if decode:
         achieved = g_bytes / g_time / 1e9
@@ -497,9 +494,10 @@ def run_gpu(args, w):
     roof["kernel"] = kname
     roof["plan"] = {k: v for k, v in plan.as_dict().items() if k != "kernel"}
     roof["launch_ms_mean"] = g_time * 1e3 / g_n
-    roof["timing"] = ("CUDA events on the launching stream around each GEMM call of every "
-                      "timed step (a call = the main kernel plus its fix-up kernel when the "
-                      "plan has one)")
+    roof["timing"] = ("CUDA events on the launching stream around each GEMM call, in %d eager "
+                      "steps run right after the graph-timed ones (a call = the main kernel "
+                      "plus its fix-up kernel when the plan has one; the interval includes "
+                      "the event records' own drain)" % calls_steps)
 
     line = {
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
@@ -509,12 +507,10 @@ def run_gpu(args, w):
         "config": {"workload": w.name, "tokens": w.M, "calib_tokens": w.M_cal, "alpha": w.alpha,
                    "linears": ["%s %dx%d" % (l.name, w.site(l.site).K, l.N) for l in w.linears],
                    "step": "calibrate + smooth scales/fold + weight quant + norm-quant + GEMM",
-                   "launch": "eager C-ABI calls, each step queued behind an untimed GPU spin "
-                             "so no host gap enters the events",
+                   "launch": "the whole step as one CUDA graph, replayed per timed step",
                    "l2": "flushed before every step (256 MiB write, not timed)",
                    "parallelism": "dp%d (independent token batches, weights replicated)" % world},
         "tokens_per_s": tokens_per_s,
-        "graph_ms_per_step": sum(graph_ms) / len(graph_ms),
         "forward_gemm_tops": g_ops / g_time / 1e12,
         "roofline": roof,
         "kernels": kernels,

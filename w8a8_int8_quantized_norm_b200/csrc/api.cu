@@ -234,7 +234,7 @@ sq_status sq_w8a8_gemm_plan(int64_t M, int64_t N, int64_t K, int path_hint, int 
   sq_gemm_plan_info r{};
   r.kernel = plan.swap ? 2 : (plan.pair ? 1 : 0);
   r.tile_m = plan.pair ? 256 : 128;
-  r.tile_n = plan.pair ? 256 : plan.bn;
+  r.tile_n = plan.bn;
   r.split_k = plan.splits;
   r.stream_k = plan.streamk;
   const int64_t p_rows = plan.swap ? N : M, q_rows = plan.swap ? M : N;

@@ -490,17 +490,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 // stage-free and accumulator-ready barriers with one commit each; both CTAs'
 // epilogue warps drain their own 128 accumulator rows and tell the leader.
 // ---------------------------------------------------------------------------
-namespace pair {
-constexpr int ROWS = 128;                    // rows of A and of B per CTA
-constexpr int A_BYTES = ROWS * BK;
-constexpr int B_BYTES = ROWS * BK;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // per CTA
-constexpr int STAGES = 6;
-constexpr int TILE = 256;                    // pair tile: 256 x 256
-constexpr int TMEM_COLS = 512;               // 2 accumulators x 256 INT32 columns
-constexpr int NUM_BARS = 2 * STAGES + 5;
-constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 8 * NUM_BARS + 16;
-}  // namespace pair
+// TN: the pair tile's N (Q-side) width, 256, 192 or 128; each CTA loads
+// TN / 2 rows of B.  As many stages as fit 227 KB of shared memory (at most 8).
+template <int TN>
+struct PairCfg {
+  static constexpr int ROWS = 128;             // rows of A per CTA
+  static constexpr int TILE_M = 2 * ROWS;      // P side of the pair tile
+  static constexpr int B_ROWS = TN / 2;        // rows of B per CTA
+  static constexpr int A_BYTES = ROWS * BK;
+  static constexpr int B_BYTES = B_ROWS * BK;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // per CTA
+  static constexpr int STAGES_FIT = (227 * 1024 - 1024 - 256) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_FIT < 8 ? STAGES_FIT : 8;
+  static constexpr int TMEM_COLS = 512;        // 2 accumulators x TN INT32 columns
+  static constexpr int NUM_BARS = 2 * STAGES + 5;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 8 * NUM_BARS + 16;
+  static_assert(TN % 32 == 0 && TN >= 64 && TN <= 256, "pair tile width");
+  static_assert(B_BYTES % 1024 == 0, "swizzle atoms need 1024-byte aligned stages");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+};
 
 __device__ __forceinline__ void mbar_complete_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.complete_tx.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
@@ -511,10 +519,14 @@ __device__ __forceinline__ int64_t loads_on_stage(int64_t total, int s, int stag
   return total / stages + (s < total % stages ? 1 : 0);
 }
 
+template <int TN>
 __global__ void __launch_bounds__(kThreads, 1)
     w8a8_gemm_pair_kernel(const __grid_constant__ CUtensorMap mapP,
                           const __grid_constant__ CUtensorMap mapQ, const Params prm) {
-  using namespace pair;
+  using C = PairCfg<TN>;
+  constexpr int ROWS = C::ROWS, TILE_M = C::TILE_M, B_ROWS = C::B_ROWS;
+  constexpr int A_BYTES = C::A_BYTES, B_BYTES = C::B_BYTES, STAGE_BYTES = C::STAGE_BYTES;
+  constexpr int STAGES = C::STAGES, TMEM_COLS = C::TMEM_COLS, NUM_BARS = C::NUM_BARS;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = smem_u32(smem_raw);
   const uint32_t base = (raw_u32 + 1023u) & ~1023u;
@@ -596,9 +608,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t fb = leader ? FULL_BAR(stage) : map_to_cta(FULL_BAR(stage), 0);
           if (leader) mbar_arrive_expect_tx(FULL_BAR(stage), 2 * STAGE_BYTES);
           tma_load_2d_pair(a_base + stage * A_BYTES, &mapP, fb, kb * BK,
-                           pb * TILE + static_cast<int>(rank) * ROWS);
+                           pb * TILE_M + static_cast<int>(rank) * ROWS);
           tma_load_2d_pair(b_base + stage * B_BYTES, &mapQ, fb, kb * BK,
-                           qb * TILE + static_cast<int>(rank) * ROWS);
+                           qb * TN + static_cast<int>(rank) * B_ROWS);
         }
         ++issued;
         if (++stage == STAGES) {
@@ -615,7 +627,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader only)
     if (leader) {
-      constexpr uint32_t kIdesc = idesc_i8(2 * ROWS, TILE);
+      constexpr uint32_t kIdesc = idesc_i8(TILE_M, TN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -633,7 +645,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * TILE);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * TN);
         for (int kb = kb0; kb < kb1; ++kb) {
           w = false;
           if (lane == 0) w = wait_phase(FULL_BAR(stage), phase, polls, abort_flag);
@@ -696,16 +708,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const int p = pb * TILE + static_cast<int>(rank) * ROWS + quarter * 32 + lane;
+      const int p = pb * TILE_M + static_cast<int>(rank) * ROWS + quarter * 32 + lane;
 #pragma unroll 1
-      for (int c = 0; c < TILE / 32; ++c) {
+      for (int c = 0; c < TN / 32; ++c) {
         uint32_t r[32];
         __syncwarp();
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                               static_cast<uint32_t>(acc * TILE + c * 32);
+                               static_cast<uint32_t>(acc * TN + c * 32);
         tmem_ld_32x32b_x32(taddr, r);
         tmem_wait_ld();
-        store_chunk<32>(prm, r, p, qb * TILE + c * 32, 0, -1);
+        store_chunk<32>(prm, r, p, qb * TN + c * 32, 0, -1);
       }
       tc_fence_before();
       __syncwarp();
@@ -870,10 +882,12 @@ cudaError_t launch_bn(const Params& prm, const CUtensorMap& mp, const CUtensorMa
   return cudaGetLastError();
 }
 
+template <int TN>
 cudaError_t launch_pair(const Params& prm, const CUtensorMap& mp, const CUtensorMap& mq,
                         int max_pairs, cudaStream_t st) {
-  cudaError_t e = launch_cache().ensure_smem(reinterpret_cast<const void*>(w8a8_gemm_pair_kernel),
-                                             pair::SMEM_BYTES);
+  using C = PairCfg<TN>;
+  auto kern = w8a8_gemm_pair_kernel<TN>;
+  cudaError_t e = launch_cache().ensure_smem(reinterpret_cast<const void*>(kern), C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -882,7 +896,7 @@ cudaError_t launch_pair(const Params& prm, const CUtensorMap& mp, const CUtensor
   attr[0].val.clusterDim.z = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = pair::SMEM_BYTES;
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
@@ -892,15 +906,14 @@ cudaError_t launch_pair(const Params& prm, const CUtensorMap& mp, const CUtensor
   if (dev >= 0 && dev < 64 && max_clusters[dev] == 0) {
     cfg.gridDim = dim3(2 * max_pairs);
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, w8a8_gemm_pair_kernel, &cfg) != cudaSuccess || n <= 0)
-      n = max_pairs;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) n = max_pairs;
     max_clusters[dev] = n;
   }
   int pairs = (dev >= 0 && dev < 64) ? max_clusters[dev] : max_pairs;
   if (pairs > max_pairs) pairs = max_pairs;
   if (pairs > prm.units) pairs = prm.units;
   cfg.gridDim = dim3(2 * pairs);
-  e = cudaLaunchKernelEx(&cfg, w8a8_gemm_pair_kernel, mp, mq, prm);
+  e = cudaLaunchKernelEx(&cfg, kern, mp, mq, prm);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -922,6 +935,22 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int path_hint, int split_k, 
     p.bn = 256;
     p.splits = 1;
     p.pair = path_hint == 3 ? 0 : 1;
+    if (p.pair) {
+      // pair tile width: the fewest rounds of tiles over the SM pairs, each
+      // round costing its width plus a fixed share for the A operand (whose
+      // bytes do not shrink with the width)
+      const int64_t pairs = (num_sms > 0 ? num_sms : 148) / 2;
+      const int64_t p_blocks = (M + 255) / 256;
+      int64_t best = -1;
+      for (int tn : {256, 192, 128}) {
+        const int64_t tiles = p_blocks * ((N + tn - 1) / tn);
+        const int64_t cost = ((tiles + pairs - 1) / pairs) * (tn + 64);
+        if (best < 0 || cost < best) {
+          best = cost;
+          p.bn = tn;
+        }
+      }
+    }
   } else if (split_k <= 0) {
     // decode tiles, stream-K: every SM streams the same number of k-blocks
     p.bn = bn_for_tokens(M);
@@ -982,7 +1011,7 @@ cudaError_t launch_gemm(const GemmPlan& plan, const int8_t* Xq, const int8_t* Wq
   prm.P = static_cast<int>(plan.swap ? N : M);
   prm.Q = static_cast<int>(plan.swap ? M : N);
   prm.K = static_cast<int>(K);
-  const int p_tile = plan.pair ? pair::TILE : BM;
+  const int p_tile = plan.pair ? 256 : BM;
   prm.p_blocks = (prm.P + p_tile - 1) / p_tile;
   prm.q_blocks = (prm.Q + plan.bn - 1) / plan.bn;
   prm.k_blocks = static_cast<int>((K + BK - 1) / BK);
@@ -1011,9 +1040,14 @@ cudaError_t launch_gemm(const GemmPlan& plan, const int8_t* Xq, const int8_t* Wq
   const int sms = num_sms > 0 ? num_sms : 148;
   if (plan.pair) {
     // each CTA of a pair loads 128 rows of A and 128 rows of B
-    if (!make_map(&mp, Pptr, prm.P, K, pair::ROWS) || !make_map(&mq, Qptr, prm.Q, K, pair::ROWS))
+    if (!make_map(&mp, Pptr, prm.P, K, 128) || !make_map(&mq, Qptr, prm.Q, K, plan.bn / 2))
       return cudaErrorInvalidValue;
-    return launch_pair(prm, mp, mq, sms / 2, st);
+    switch (plan.bn) {
+      case 256: return launch_pair<256>(prm, mp, mq, sms / 2, st);
+      case 192: return launch_pair<192>(prm, mp, mq, sms / 2, st);
+      case 128: return launch_pair<128>(prm, mp, mq, sms / 2, st);
+      default: return cudaErrorInvalidValue;
+    }
   }
   if (!make_map(&mp, Pptr, prm.P, K, BM) || !make_map(&mq, Qptr, prm.Q, K, plan.bn))
     return cudaErrorInvalidValue;

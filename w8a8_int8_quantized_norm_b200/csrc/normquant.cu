@@ -457,7 +457,9 @@ bool pipe_shape(int K, bool bf16, PipeShape* ps) {
   if (threads < 32) threads = 32;
   const size_t row_bytes = static_cast<size_t>(K) * (bf16 ? 2 : 4);
   const size_t stride = (row_bytes + 127) / 128 * 128;
-  int nbuf = static_cast<int>((48u << 10) / stride);
+  // about 24 KB of row buffers per CTA: with small rows that leaves room for
+  // eight CTAs per SM (more rows in flight, shorter per-CTA row chains)
+  int nbuf = static_cast<int>((24u << 10) / stride);
   if (nbuf < 3) nbuf = 3;
   if (nbuf > 8) nbuf = 8;
   while (nbuf > 2 && nbuf * stride > (150u << 10)) --nbuf;
@@ -495,14 +497,18 @@ cudaError_t launch_pipe_k(const RowArgs& a, PipeShape ps, cudaStream_t st) {
     cudaError_t e = lc.ensure_smem(key, ps.smem);
     if (e != cudaSuccess) return e;
     per_sm = lc.blocks_per_sm(key, ps.threads, ps.smem);
-    const int64_t ctas = static_cast<int64_t>(per_sm) * lc.sms();
+    int64_t ctas = static_cast<int64_t>(per_sm) * lc.sms();
+    if (kC && ctas > (a.M + 3) / 4) ctas = (a.M + 3) / 4;
     const int64_t rows_per_cta = (a.M + ctas - 1) / ctas;
     if (ps.nbuf <= 2 || rows_per_cta >= ps.nbuf) break;
     ps.nbuf = rows_per_cta < 2 ? 2 : static_cast<int>(rows_per_cta);
     ps.smem = pipe_smem(stride, ps.nbuf);
   }
   int64_t grid = static_cast<int64_t>(per_sm) * lc.sms();
-  if (grid > a.M) grid = a.M;
+  // calibration merges every CTA's column maxima with atomics: at least four
+  // rows per CTA keeps their number (CTAs x K) down
+  const int64_t max_grid = kC ? (a.M + 3) / 4 : a.M;
+  if (grid > max_grid) grid = max_grid;
   kern<<<static_cast<unsigned>(grid), ps.threads, ps.smem, st>>>(
       a.x, a.ldx, a.M, a.K, a.gamma, a.beta, a.eps, a.q, a.scale, a.act_max, ps.nbuf, a.err);
   return cudaGetLastError();

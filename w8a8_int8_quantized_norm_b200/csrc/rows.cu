@@ -371,9 +371,10 @@ cudaError_t launch_weight_colmax(const void* W, bool bf16, int64_t N, int K, flo
   if (N == 0) return cudaSuccess;
   const int nchunks = K / kChunk;
   const int slabs = (nchunks + 31) / 32;
-  // about eight CTAs per SM, at least 64 rows (8 per warp) each, and no more
-  // row runs than gridDim.y allows
-  const int64_t target = 8 * static_cast<int64_t>(launch_cache().sms());
+  // about four CTAs per SM (what fits at once: one wave of long-lived CTAs),
+  // at least 64 rows (8 per warp) each, and no more row runs than gridDim.y
+  // allows; fewer runs also mean fewer atomics (runs x K)
+  const int64_t target = 4 * static_cast<int64_t>(launch_cache().sms());
   int64_t runs = target / slabs;
   if (runs < 1) runs = 1;
   int64_t rows = (N + runs - 1) / runs;

@@ -6,9 +6,10 @@
     python -m w8a8_int8_quantized_norm_b200.kbench weight_quant --N 28672 --K 8192
     python -m w8a8_int8_quantized_norm_b200.kbench smooth_scales --N 12288 --K 4096
 
-Each timed call is bracketed by CUDA events on the launching stream, with the
-L2 cache overwritten (256 MiB, untimed) before every call, so the operands come
-from HBM.  Prints one JSON line: mean time per call, the call's algorithmic
+Each call is captured once as a CUDA graph; every timed replay is bracketed by
+CUDA events on the launching stream, with the L2 cache overwritten (256 MiB,
+untimed) before it, so the operands come from HBM and no host work falls
+inside the interval.  Prints one JSON line: mean time per call, the call's algorithmic
 bytes (row kernels, GEMMs with at most 128 tokens) or integer ops (other
 GEMMs), and the fraction of the measured peak.  Inputs are seeded synthetic
 tensors made on the device: N(0, 1) activations with a few outlier channels
@@ -52,20 +53,30 @@ def _codes(R, K, gen, dev):
     return torch.randint(-127, 128, (R, K), generator=gen, device=dev, dtype=torch.int8)
 
 
-def _time(fn, iters, warmup, flush, stream):
+def _time(fn, iters, warmup, flush):
+    """Mean device time of one call: the call is captured once as a CUDA graph
+    (no host work inside the timed interval) and each replay is bracketed by
+    events, after an untimed L2 overwrite."""
     for _ in range(warmup):
         fn()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        fn()
+    for _ in range(warmup):
+        graph.replay()
     torch.cuda.synchronize()
     total = 0.0
     for _ in range(iters):
         flush.zero_()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        fn()
-        e1.record(stream)
+        e0.record()
+        graph.replay()
+        e1.record()
         e1.synchronize()
         total += e0.elapsed_time(e1)
+    del graph
     return total / iters * 1e3  # microseconds per call
 
 
@@ -92,7 +103,6 @@ def main(argv=None):
     sq.lib()
     gen = torch.Generator(device=dev)
     gen.manual_seed(a.seed)
-    stream = torch.cuda.current_stream(dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     hbm, bf16, src = _peaks()
     M, N, K = a.M, a.N, a.K
@@ -105,7 +115,7 @@ def main(argv=None):
         b = torch.randn(K, generator=gen, device=dev) * 0.1 if norm == sq.NORM_LAYER else None
         xq = torch.empty((M, K), dtype=torch.int8, device=dev)
         xs = torch.empty(M, dtype=torch.float32, device=dev)
-        fn = lambda: sq.norm_smooth_quant_per_token(x, norm, g, b, 1e-5, xq, xs, stream=stream)
+        fn = lambda: sq.norm_smooth_quant_per_token(x, norm, g, b, 1e-5, xq, xs)
         units = M * K * (esz + 1) + 4 * M + 4 * K * ((g is not None) + (b is not None))
         shape = {"M": M, "K": K, "norm": a.norm, "dtype": a.dtype}
     elif a.op == "calibrate":
@@ -113,7 +123,8 @@ def main(argv=None):
         g = torch.empty(K, device=dev).uniform_(0.5, 1.5, generator=gen) if norm else None
         b = torch.randn(K, generator=gen, device=dev) * 0.1 if norm == sq.NORM_LAYER else None
         am = torch.zeros(K, dtype=torch.float32, device=dev)
-        fn = lambda: sq.calibrate_absmax(x, norm, g, b, 1e-5, act_max=am, stream=stream)
+        # the running max starts from zero every call, as in a calibration pass
+        fn = lambda: (am.zero_(), sq.calibrate_absmax(x, norm, g, b, 1e-5, act_max=am))
         units = M * K * esz + 4 * K
         shape = {"M": M, "K": K, "norm": a.norm, "dtype": a.dtype}
     elif a.op == "weight_quant":
@@ -122,7 +133,7 @@ def main(argv=None):
         s = torch.empty(K, device=dev).uniform_(0.25, 4.0, generator=gen)
         wq = torch.empty((N, K), dtype=torch.int8, device=dev)
         wsc = torch.empty(N, dtype=torch.float32, device=dev)
-        fn = lambda: sq.smooth_quantize_weights(W, s, Wq=wq, w_scale=wsc, stream=stream)
+        fn = lambda: sq.smooth_quantize_weights(W, s, Wq=wq, w_scale=wsc)
         units = N * K * (esz + 1) + 4 * N + 4 * K
         shape = {"N": N, "K": K, "dtype": a.dtype}
     elif a.op == "smooth_scales":
@@ -132,8 +143,7 @@ def main(argv=None):
         g = torch.empty(K, device=dev).uniform_(0.5, 1.5, generator=gen)
         s = torch.empty(K, dtype=torch.float32, device=dev)
         gf = torch.empty(K, dtype=torch.float32, device=dev)
-        fn = lambda: sq.compute_smooth_scales(am, [W], 0.5, 1e-5, g, None, s=s, gamma_folded=gf,
-                                              stream=stream)
+        fn = lambda: sq.compute_smooth_scales(am, [W], 0.5, 1e-5, g, None, s=s, gamma_folded=gf)
         units = N * K * esz + 16 * K
         shape = {"N": N, "K": K, "dtype": a.dtype}
     else:
@@ -146,11 +156,10 @@ def main(argv=None):
         ws = torch.empty(need, dtype=torch.uint8, device=dev) if need else None
         scales = (None, None) if a.epi == "i32" else (xs, wsc)
         fn = lambda: sq.w8a8_gemm_dequant(A, B, scales[0], scales[1], a.epi, out=out,
-                                          path_hint=a.path, split_k=a.split, workspace=ws,
-                                          stream=stream)
+                                          path_hint=a.path, split_k=a.split, workspace=ws)
         shape = {"M": M, "N": N, "K": K, "path": a.path, "split": a.split, "epi": a.epi}
         units = None
-    us = _time(fn, a.iters, a.warmup, flush, stream)
+    us = _time(fn, a.iters, a.warmup, flush)
     err = sq.get_device_error()
     if err:
         raise SystemExit("device error: %s" % sq.status_string(err))
