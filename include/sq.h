@@ -223,8 +223,8 @@ sq_status sq_w8a8_gemm_plan(int64_t M, int64_t N, int64_t K, int path_hint, int 
  *            sq_w8a8_gemm_workspace_size(M, N, K, split_k) bytes when that is
  *            non-zero, else may be NULL.  Nothing in it outlives the call.
  *   path_hint 0 = automatic, 1 = prefill tiles (tokens on the MMA M side;
- *            CTA pairs, 256-row tiles 256, 192 or 128 wide on two SMs, the
- *            width chosen to fill the SMs evenly), 2 = decode tiles (weight
+ *            CTA pairs, 256-row tiles 256 or 192 wide on two SMs, the width
+ *            chosen to fill the SMs evenly), 2 = decode tiles (weight
  *            rows on the MMA M side, M <= 256), 3 = prefill tiles on single
  *            SMs (128 x 256)
  *   split_k  0 = automatic, else the number of K slices (decode path only;

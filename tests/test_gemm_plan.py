@@ -31,10 +31,12 @@ def test_plan_kinds_and_workspace_agree_with_the_size_query(L):
     assert (p.kernel, p.stream_k, p.split_k, p.tile_m, p.tile_n) == (2, 1, 1, 128, 16)
     assert p.ctas == SMS and p.launches == 2
     assert p.workspace_bytes == 2 * SMS * 128 * 1 * 4
-    # 8 x 48 tiles of 256 x 256 fill 74 SM pairs 5.2 times (6 rounds); 8 x 64 of
-    # 256 x 192 take 7 rounds of a narrower tile: the planner takes the latter
+    # 8 x 48 tiles of 256 x 256 fill 74 SM pairs in 6 rounds; 8 x 64 of 256 x 192
+    # need 7 rounds of a step that is not proportionally shorter: 256 wins
     p = _plan(2048, 12288, 4096)
-    assert (p.kernel, p.tile_m, p.tile_n, p.launches, p.workspace_bytes) == (1, 256, 192, 1, 0)
+    assert (p.kernel, p.tile_m, p.tile_n, p.launches, p.workspace_bytes) == (1, 256, 256, 1, 0)
+    # 4 x 12 tiles of 256 x 256 or 4 x 16 of 256 x 192 are one round either way
+    assert _plan(1024, 3000, 272).tile_n == 192
     p = _plan(16384, 57344, 8192)
     assert (p.kernel, p.tile_m, p.tile_n) == (1, 256, 256)
     p = _plan(2048, 12288, 4096, path=3)

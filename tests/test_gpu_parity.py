@@ -259,9 +259,8 @@ def test_weight_quant_matches_oracle(NK, smoothed, dtype):
 # K3 / K4: the INT8 GEMM and its epilogue
 # ---------------------------------------------------------------------------
 
-# the automatic pair-tile width differs by shape: (600, 2304, 4096) and most
-# small shapes take 256 x 128 tiles, (1024, 3000, 272) and (2048, 1536, 512)
-# 256 x 192, (2048, 9472, 128) 256 x 256
+# the automatic pair-tile width differs by shape: most small shapes take
+# 256 x 192 tiles (fewer rounds over the SM pairs), (2048, 9472, 128) 256 x 256
 GEMM_SHAPES = [(16, 64, 64), (3, 5, 16), (1, 300, 48), (129, 257, 4112), (256, 512, 1024),
                (200, 1000, 128), (300, 777, 160), (1024, 768, 2048), (2048, 1536, 512),
                (600, 2304, 4096), (1024, 3000, 272), (2048, 9472, 128)]

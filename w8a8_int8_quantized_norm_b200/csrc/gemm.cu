@@ -547,7 +547,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // stage-free and accumulator-ready barriers with one commit each; both CTAs'
 // epilogue warps drain their own 128 accumulator rows and tell the leader.
 // ---------------------------------------------------------------------------
-// TN: the pair tile's N (Q-side) width, 256, 192 or 128; each CTA loads
+// TN: the pair tile's N (Q-side) width, 256 or 192; each CTA loads
 // TN / 2 rows of B.  As many stages as fit 227 KB of shared memory (at most 8).
 template <int TN>
 struct PairCfg {
@@ -1022,15 +1022,17 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int path_hint, int split_k, 
     p.splits = 1;
     p.pair = path_hint == 3 ? 0 : 1;
     if (p.pair) {
-      // pair tile width: the fewest rounds of tiles over the SM pairs, each
-      // round costing its width plus a fixed share for the A operand (whose
-      // bytes do not shrink with the width)
+      // pair tile width: rounds of tiles over the SM pairs times the time of
+      // a tile's 128-deep K step, which is the MMA's (proportional to the
+      // width) for 256 but does not drop below about 240/256 of it for
+      // narrower tiles (operand delivery and per-step overhead; measured
+      // 600 vs 640 cycles per step at widths 192 and 256)
       const int64_t pairs = (num_sms > 0 ? num_sms : 148) / 2;
       const int64_t p_blocks = (M + 255) / 256;
       int64_t best = -1;
-      for (int tn : {256, 192, 128}) {
+      for (int tn : {256, 192}) {
         const int64_t tiles = p_blocks * ((N + tn - 1) / tn);
-        const int64_t cost = ((tiles + pairs - 1) / pairs) * (tn + 64);
+        const int64_t cost = ((tiles + pairs - 1) / pairs) * (tn > 240 ? tn : 240);
         if (best < 0 || cost < best) {
           best = cost;
           p.bn = tn;
@@ -1131,7 +1133,6 @@ cudaError_t launch_gemm(const GemmPlan& plan, const int8_t* Xq, const int8_t* Wq
     switch (plan.bn) {
       case 256: return launch_pair<256>(prm, mp, mq, sms / 2, st);
       case 192: return launch_pair<192>(prm, mp, mq, sms / 2, st);
-      case 128: return launch_pair<128>(prm, mp, mq, sms / 2, st);
       default: return cudaErrorInvalidValue;
     }
   }
