@@ -84,6 +84,12 @@ def _declare(L):
     L.oracle_f32_to_bf16_bits.argtypes = [ctypes.c_float]
     L.oracle_row_sums.restype = None
     L.oracle_row_sums.argtypes = [_P, ctypes.c_int, _I64, _I64, _I64, _P, _P, _P]
+    L.oracle_absmax_all.restype = None
+    L.oracle_absmax_all.argtypes = [_P, _I64, _I64, _P]
+    L.oracle_step_of.restype = ctypes.c_float
+    L.oracle_step_of.argtypes = [ctypes.c_float]
+    L.oracle_quantize_with_step.restype = None
+    L.oracle_quantize_with_step.argtypes = [_P, _I64, _I64, ctypes.c_float, _P]
     L.oracle_num_threads.restype = ctypes.c_int
     L.oracle_num_threads.argtypes = []
 
@@ -151,6 +157,45 @@ def quantize_rows(y: np.ndarray):
     return q, step
 
 
+def absmax_all(y: np.ndarray, absmax: float = 0.0) -> np.float32:
+    """Per-tensor variants: running max of |y| over every element."""
+    y = np.ascontiguousarray(y, dtype=np.float32).reshape(-1, y.shape[-1] if y.ndim else 1)
+    M, K = y.shape
+    am = np.array([absmax], np.float32)
+    lib().oracle_absmax_all(_ptr(y), M, K, _ptr(am))
+    return am[0]
+
+
+def step_of(absmax) -> np.float32:
+    """fl32(absmax / 127)."""
+    return np.float32(lib().oracle_step_of(float(np.float32(absmax))))
+
+
+def quantize_with_step(y: np.ndarray, step) -> np.ndarray:
+    """Every element with one step: clamp(rne(fl32(y / step)), +-127)."""
+    y = np.ascontiguousarray(y, dtype=np.float32)
+    M, K = y.shape
+    q = np.empty((M, K), np.int8)
+    lib().oracle_quantize_with_step(_ptr(y), M, K, float(np.float32(step)), _ptr(q))
+    return q
+
+
+def quantize_tensor(y: np.ndarray):
+    """O2 on a tensor (or per-tensor weights): (q int8, step fp32)."""
+    step = step_of(absmax_all(y))
+    return quantize_with_step(y, step), step
+
+
+def norm_quant_per_tensor(x, norm_kind, gamma_f=None, beta_f=None, eps=1e-5, absmax=None):
+    """Steps 4+5 with one activation scale for the whole tensor: O2 (``absmax``
+    None: the tensor's own max |y|) or O3 (``absmax`` given: the calibrated
+    static max; larger values saturate).  Returns (Xq, step)."""
+    y, _, _ = norm(x, norm_kind, gamma_f, beta_f, eps)
+    am = absmax_all(y) if absmax is None else np.float32(absmax)
+    step = step_of(am)
+    return quantize_with_step(y, step), step
+
+
 def norm_quant(x, norm_kind, gamma_f=None, beta_f=None, eps=1e-5):
     """Steps 4+5 (the runtime activation path): returns (Xq, x_scale)."""
     y, _, _ = norm(x, norm_kind, gamma_f, beta_f, eps)
@@ -216,6 +261,12 @@ def smooth_weights(W, s=None):
 def quantize_weights(W, s=None):
     """Steps 3+6: (Wq int8 [N,K], w_scale fp32 [N])."""
     return quantize_rows(smooth_weights(W, s))
+
+
+def quantize_weights_per_tensor(W, s=None):
+    """Steps 3+6 with one weight scale for the whole matrix (the paper's
+    O1-O3 weights): (Wq int8 [N,K], step fp32)."""
+    return quantize_tensor(smooth_weights(W, s))
 
 
 def gemm_i64(Xq, Wq):

@@ -305,6 +305,40 @@ void oracle_quantize_rows(const float* y, int64_t M, int64_t K, int8_t* q,
 }
 
 /* ------------------------------------------------------------------------ */
+/* Per-tensor variants (O2 dynamic, O3 static)                               */
+/* ------------------------------------------------------------------------ */
+/*
+ * [SQ-depth] "Granularity: O1, O2, O3 and what kernels run today": the paper's
+ * three levels all use per-tensor weight scales; O2 shares one dynamic
+ * activation scale across the whole tensor, O3 uses a static activation
+ * scale fixed offline (the page warns that O3's static scales break on inputs
+ * outside the calibration distribution: values beyond it saturate).
+ * [LLMint8] "Try it": plain INT8 with one scale per tensor, step = max / 127.
+ * oracle_absmax_all: the running max over every element of |y| (in/out, the
+ * caller starts it at zero).  oracle_quantize_with_step: every element with
+ * the same step, q = clamp(rne(fl32(y / step)), -127, 127), step 0 -> q 0.
+ * O2 is step = fl32(absmax_all / 127) on the tensor itself; O3 the same on
+ * the calibration batch passed through the runtime (folded) norm, then
+ * applied to every later tensor.
+ * Parity: pinned by the one-row case (identical to the per-row quantiser),
+ * the "Try it" steps, and the clamp of values beyond a static range.
+ */
+void oracle_absmax_all(const float* y, int64_t M, int64_t K, float* absmax) {
+  float am = *absmax;
+  for (int64_t i = 0; i < M * K; ++i) {
+    float a = fabsf(y[i]);
+    if (a > am) am = a;
+  }
+  *absmax = am;
+}
+
+float oracle_step_of(float absmax) { return absmax / 127.0f; }
+
+void oracle_quantize_with_step(const float* y, int64_t M, int64_t K, float step, int8_t* q) {
+  for (int64_t i = 0; i < M * K; ++i) q[i] = quantize_one(y[i], step);
+}
+
+/* ------------------------------------------------------------------------ */
 /* Step 1: calibration -- running per-channel absmax of the norm output      */
 /* ------------------------------------------------------------------------ */
 /*

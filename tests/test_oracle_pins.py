@@ -200,6 +200,82 @@ def test_try_it_steps(golden_dir):
 
 
 # --------------------------------------------------------------------------
+# per-tensor variants (O2 dynamic, O3 static)
+# --------------------------------------------------------------------------
+
+def test_per_tensor_one_row_is_the_per_token_quantiser():
+    rng = np.random.default_rng(5)
+    for K in (1, 7, 4096):
+        y = (rng.standard_normal((1, K)) * rng.uniform(0.01, 100)).astype(np.float32)
+        q_t, st_t = oracle.quantize_tensor(y)
+        q_r, st_r = oracle.quantize_rows(y)
+        assert st_t == st_r[0] and np.array_equal(q_t, q_r)
+
+
+def test_per_tensor_step_is_the_largest_row_step_and_order_free():
+    rng = np.random.default_rng(6)
+    y = rng.standard_normal((37, 300)).astype(np.float32)
+    y[11, 250] = -41.0
+    q, step = oracle.quantize_tensor(y)
+    _, row_steps = oracle.quantize_rows(y)
+    assert step == row_steps.max() == np.float32(np.float32(41.0) / np.float32(127.0))
+    assert q[11, 250] == -127 and np.abs(q).max() == 127
+    perm_r, perm_c = rng.permutation(37), rng.permutation(300)
+    q2, step2 = oracle.quantize_tensor(y[perm_r][:, perm_c])
+    assert step2 == step and np.array_equal(q2, q[perm_r][:, perm_c])
+    # every element with the one step, against numpy's float32 arithmetic
+    ref = np.clip(np.rint((y / step).astype(np.float32)), -127, 127).astype(np.int8)
+    assert np.array_equal(q, ref)
+
+
+def test_try_it_per_tensor(golden_dir):
+    """The demo quantises each whole tensor with one step: a 64 x 64 block of
+    ordinary values whose largest magnitude is the printed max gives the
+    printed step, and ordinary values use only a few levels."""
+    g = _golden(golden_dir, "try_it_steps.json")
+    rng = np.random.default_rng(7)
+    for key, big in (("x_step", g["largest_abs_x"]), ("w_step", g["largest_abs_w"])):
+        t = np.clip(rng.standard_normal((64, 64)), -2.5, 2.5).astype(np.float32) * np.float32(
+            big / 84.3 if key == "w_step" else 1.0)
+        t[17, 3] = np.float32(big)
+        q, step = oracle.quantize_tensor(t)
+        assert abs(step - g["printed"][key]) <= g["printed_precision"][key], key
+        if key == "x_step":  # about +-4 of the 127 levels for the ordinary channels
+            mask = np.ones_like(t, bool)
+            mask[17, 3] = False
+            assert np.abs(q[mask]).max() <= 4
+
+
+def test_static_step_saturates_beyond_the_calibrated_range():
+    # a static max of 127 gives step 1 exactly; values outside [-127, 127] clamp
+    assert oracle.step_of(127.0) == np.float32(1.0)
+    y = np.array([[254.0, -381.0, 127.0, -127.0, 63.5, 62.5, -0.5, 126.49]], np.float32)
+    q = oracle.quantize_with_step(y, oracle.step_of(127.0))
+    assert q.tolist() == [[127, -127, 127, -127, 64, 62, 0, 126]]
+    assert not oracle.quantize_with_step(y, 0.0).any()
+    # O3 on a norm: the static max comes from the calibration tokens through
+    # the folded norm; a runtime row twice as large saturates
+    rng = np.random.default_rng(8)
+    xc = rng.standard_normal((16, 64)).astype(np.float32)
+    g = rng.uniform(0.5, 1.5, 64).astype(np.float32)
+    yc, _, _ = oracle.norm(xc, oracle.NORM_NONE, g)
+    am = oracle.absmax_all(yc)
+    q_run, step = oracle.norm_quant_per_tensor(2 * xc, oracle.NORM_NONE, g, absmax=am)
+    assert step == oracle.step_of(am)
+    assert np.count_nonzero(np.abs(q_run) == 127) > 1
+
+
+def test_per_tensor_weights():
+    rng = np.random.default_rng(9)
+    W = (rng.standard_normal((48, 96)) * 0.02).astype(np.float32)
+    s = rng.uniform(0.5, 4.0, 96).astype(np.float32)
+    q, step = oracle.quantize_weights_per_tensor(W, s)
+    _, row_steps = oracle.quantize_weights(W, s)
+    assert step == row_steps.max()
+    assert np.array_equal(q, oracle.quantize_with_step(oracle.smooth_weights(W, s), step))
+
+
+# --------------------------------------------------------------------------
 # smoothing factors, fold and weight smoothing (steps 1-3)
 # --------------------------------------------------------------------------
 
