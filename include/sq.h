@@ -179,6 +179,55 @@ sq_status sq_norm_smooth_quant_per_token(const void* x, sq_dtype dtype, int64_t 
                                          float* x_scale, void* stream);
 
 /*
+ * Per-tensor variants (the paper's O2 and O3 levels).
+ * [SQ-depth] "Granularity: O1, O2, O3 and what kernels run today": all three
+ * levels use per-tensor weight scales; O2 shares one dynamic activation scale
+ * over the whole tensor, O3 one static scale fixed offline (values beyond the
+ * calibrated range saturate).  [LLMint8] "Try it": one step = max / 127 per
+ * tensor.  The per-row scale outputs below hold that one step in every entry,
+ * so sq_w8a8_gemm_dequant's epilogue applies it unchanged.  These calls take
+ * rows up to 40960 elements (bf16) / 25600 (fp32) (else SQ_ERR_UNSUPPORTED).
+ *
+ * sq_norm_smooth_absmax -- running max over all of |y|, y the norm output of
+ * sq_norm_smooth_quant_per_token (same arithmetic), into absmax[0].
+ *   absmax   device [1] fp32 IN/OUT (the caller starts it at zero; a running
+ *            max over calls).  O2: the tensor itself; O3: the calibration
+ *            tokens through the folded norm, once, offline.
+ * Errors: those of sq_norm_smooth_quant_per_token.
+ */
+sq_status sq_norm_smooth_absmax(const void* x, sq_dtype dtype, int64_t M, int64_t K, int64_t ldx,
+                                sq_norm norm, const float* gamma_folded,
+                                const float* beta_folded, float eps, float* absmax,
+                                void* stream);
+
+/*
+ * sq_norm_smooth_quant_per_tensor -- the norm output quantised with one step,
+ * step = fl32(absmax[0] / 127); Xq = clamp(rne(fl32(y / step)), -127, 127)
+ * (0 where the step is 0); x_scale[m] = step for every row.
+ *   absmax   device [1] fp32 IN: max |y| (sq_norm_smooth_absmax)
+ *   Xq, x_scale as for sq_norm_smooth_quant_per_token
+ * Errors: those of sq_norm_smooth_quant_per_token.
+ */
+sq_status sq_norm_smooth_quant_per_tensor(const void* x, sq_dtype dtype, int64_t M, int64_t K,
+                                          int64_t ldx, sq_norm norm, const float* gamma_folded,
+                                          const float* beta_folded, float eps,
+                                          const float* absmax, int8_t* Xq, float* x_scale,
+                                          void* stream);
+
+/*
+ * sq_smooth_quantize_weights_per_tensor -- W-hat = W diag(s) quantised with
+ * one step for the whole matrix, fl32(max |W-hat| / 127).
+ *   w_scale  device [N] fp32 OUT: the step in every entry
+ *   w_absmax device [1] fp32 OUT: max |W-hat| (scratch the call overwrites)
+ *   other arguments as for sq_smooth_quantize_weights
+ * Errors: those of sq_smooth_quantize_weights, SQ_ERR_UNSUPPORTED.
+ */
+sq_status sq_smooth_quantize_weights_per_tensor(const void* W, sq_dtype dtype, int64_t N,
+                                                int64_t K, int64_t ldw, const float* s,
+                                                int8_t* Wq, float* w_scale, float* w_absmax,
+                                                void* stream);
+
+/*
  * sq_w8a8_gemm_workspace_size -- bytes of device workspace that
  * sq_w8a8_gemm_dequant needs for this shape and split factor (0 when the
  * chosen path needs none).  split_k = 0 asks for the automatic choice.

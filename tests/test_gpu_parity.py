@@ -468,3 +468,88 @@ def test_graph_replay_matches_eager_step(wname):
     for key, v in snapshot().items():
         assert torch.equal(v, eager[key]), key
     del graph
+
+
+# ---------------------------------------------------------------------------
+# per-tensor variants (O2 dynamic, O3 static; per-tensor weights)
+# ---------------------------------------------------------------------------
+
+PT_KINDS = [("none_mult", oracle.NORM_NONE), ("rms", oracle.NORM_RMS),
+            ("layer", oracle.NORM_LAYER)]
+
+
+@pytest.mark.parametrize("shape", [(1, 64), (17, 4096), (300, 4112), (2048, 4096), (40, 28672)],
+                         ids=lambda s: "%dx%d" % s)
+@pytest.mark.parametrize("kind", PT_KINDS, ids=lambda k: k[0])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_per_tensor_dynamic_matches_oracle(shape, kind, dtype):
+    M, K = shape
+    _, norm = kind
+    x = _acts(M, K, dtype)
+    g = RNG.uniform(0.5, 1.5, K).astype(np.float32)
+    b = (RNG.standard_normal(K) * 0.1).astype(np.float32) if norm == oracle.NORM_LAYER else None
+    gg, bb = to_gpu(g), (None if b is None else to_gpu(b))
+    y_o, _, _ = oracle.norm(x, norm, g, b, 1e-5)
+    ties = norm_near_tie_rows(x, norm, 1e-5)
+    am_o = oracle.absmax_all(y_o)
+    xg = to_gpu(x)
+    am_g = sq.norm_smooth_absmax(xg, norm, gg, bb)
+    am_gv = np.float32(am_g.item())
+    if not ties.any():
+        assert am_gv.view(np.uint32) == am_o.view(np.uint32)
+    else:
+        assert abs(am_gv - am_o) <= 2 * np.spacing(am_o)
+    # a second call keeps the running max
+    sq.norm_smooth_absmax(xg[: max(1, M // 2)], norm, gg, bb, absmax=am_g)
+    assert np.float32(am_g.item()) == am_gv
+    # O2: one step from the tensor's own max (the GPU's, equal to the oracle's
+    # unless a certified near-tie moved it)
+    Xq_g, xs_g = sq.norm_smooth_quant_per_tensor(xg, norm, am_g, gg, bb)
+    step = oracle.step_of(am_gv)
+    Xq_o = oracle.quantize_with_step(y_o, step)
+    xs_o = np.full(M, step, np.float32)
+    compare_rows_quant(Xq_g.cpu().numpy(), xs_g.cpu().numpy(), Xq_o, xs_o, ties)
+
+
+@pytest.mark.parametrize("kind", PT_KINDS, ids=lambda k: k[0])
+def test_per_tensor_static_saturates_like_the_oracle(kind):
+    """O3: the step comes from a calibrated max below this tensor's own, so
+    the largest values clamp at +-127."""
+    _, norm = kind
+    M, K = 257, 4096
+    x = _acts(M, K, "bf16")
+    g = RNG.uniform(0.5, 1.5, K).astype(np.float32)
+    b = (RNG.standard_normal(K) * 0.1).astype(np.float32) if norm == oracle.NORM_LAYER else None
+    y_o, _, _ = oracle.norm(x, norm, g, b, 1e-5)
+    am_static = np.float32(0.37 * oracle.absmax_all(y_o))
+    Xq_g, xs_g = sq.norm_smooth_quant_per_tensor(
+        to_gpu(x), norm, to_gpu(np.array([am_static], np.float32)), to_gpu(g),
+        None if b is None else to_gpu(b))
+    step = oracle.step_of(am_static)
+    Xq_o = oracle.quantize_with_step(y_o, step)
+    assert np.count_nonzero(np.abs(Xq_o) == 127) > 0
+    compare_rows_quant(Xq_g.cpu().numpy(), xs_g.cpu().numpy(), Xq_o, np.full(M, step, np.float32),
+                       norm_near_tie_rows(x, norm, 1e-5))
+    # a zero static max gives step 0 and all-zero codes
+    Xq0, xs0 = sq.norm_smooth_quant_per_tensor(to_gpu(x), norm, torch.zeros(1, device="cuda"),
+                                               to_gpu(g), None if b is None else to_gpu(b))
+    assert not Xq0.any() and not xs0.any()
+
+
+@pytest.mark.parametrize("NK", [(1, 16), (300, 4096), (129, 4112), (64, 28672)],
+                         ids=lambda s: "%dx%d" % s)
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_per_tensor_weights_match_oracle(NK, dtype):
+    N, K = NK
+    W = (RNG.standard_normal((N, K)) * 0.02).astype(np.float32)
+    if N > 3:
+        W[2] = 0.0
+    if dtype == "bf16":
+        W = S.to_bf16_bits(W)
+    s = RNG.uniform(0.25, 4.0, K).astype(np.float32)
+    q_o, step_o = oracle.quantize_weights_per_tensor(W, s)
+    am = torch.full((1,), 123.0, device="cuda")  # overwritten by the call
+    Wq_g, ws_g = sq.smooth_quantize_weights_per_tensor(to_gpu(W), to_gpu(s), w_absmax=am)
+    assert np.array_equal(Wq_g.cpu().numpy(), q_o)
+    assert np.all(ws_g.cpu().numpy().view(np.uint32) == np.float32(step_o).view(np.uint32))
+    assert np.float32(am.item()) * 0 == 0 and oracle.step_of(am.item()) == step_o

@@ -213,6 +213,82 @@ sq_status sq_norm_smooth_quant_per_token(const void* x, sq_dtype dtype, int64_t 
                                      as_stream(stream)));
 }
 
+namespace {
+
+// Shared checks of the per-tensor row calls.
+sq_status check_tensor_rows(const void* x, sq_dtype dtype, int64_t M, int64_t K, int64_t ldx,
+                            sq_norm norm, const float* gamma, const float* beta, float eps) {
+  if (!valid_norm(norm) || !(eps >= 0.0f)) return SQ_ERR_INVALID_ARG;
+  sq_status st = check_rows(x, dtype, M, K, ldx);
+  if (st != SQ_OK) return st;
+  if ((st = check_vec(gamma, false)) != SQ_OK) return st;
+  if ((st = check_vec(beta, false)) != SQ_OK) return st;
+  if (!norm_quant_pipe_supported(static_cast<int>(K), dtype == SQ_BF16)) return SQ_ERR_UNSUPPORTED;
+  return SQ_OK;
+}
+
+}  // namespace
+
+sq_status sq_norm_smooth_absmax(const void* x, sq_dtype dtype, int64_t M, int64_t K, int64_t ldx,
+                                sq_norm norm, const float* gamma_folded,
+                                const float* beta_folded, float eps, float* absmax,
+                                void* stream) {
+  sq_status st = check_tensor_rows(x, dtype, M, K, ldx, norm, gamma_folded, beta_folded, eps);
+  if (st != SQ_OK) return st;
+  if (!absmax) return SQ_ERR_INVALID_ARG;
+  int* err = device_error_word();
+  if (!err) return SQ_ERR_CUDA;
+  return from_cuda(launch_tensor_absmax_pipe(x, dtype == SQ_BF16, M, static_cast<int>(K), ldx,
+                                             norm, gamma_folded, beta_folded, eps, absmax, err,
+                                             as_stream(stream)));
+}
+
+sq_status sq_norm_smooth_quant_per_tensor(const void* x, sq_dtype dtype, int64_t M, int64_t K,
+                                          int64_t ldx, sq_norm norm, const float* gamma_folded,
+                                          const float* beta_folded, float eps,
+                                          const float* absmax, int8_t* Xq, float* x_scale,
+                                          void* stream) {
+  sq_status st = check_tensor_rows(x, dtype, M, K, ldx, norm, gamma_folded, beta_folded, eps);
+  if (st != SQ_OK) return st;
+  if (!absmax) return SQ_ERR_INVALID_ARG;
+  if (M > 0) {
+    if (!Xq) return SQ_ERR_INVALID_ARG;
+    if (!aligned16(Xq)) return SQ_ERR_ALIGNMENT;
+    if ((st = check_vec(x_scale, true)) != SQ_OK) return st;
+  }
+  int* err = device_error_word();
+  if (!err) return SQ_ERR_CUDA;
+  return from_cuda(launch_quant_fixed_pipe(x, dtype == SQ_BF16, M, static_cast<int>(K), ldx, norm,
+                                           gamma_folded, beta_folded, eps, absmax, Xq, x_scale,
+                                           err, as_stream(stream)));
+}
+
+sq_status sq_smooth_quantize_weights_per_tensor(const void* W, sq_dtype dtype, int64_t N,
+                                                int64_t K, int64_t ldw, const float* s,
+                                                int8_t* Wq, float* w_scale, float* w_absmax,
+                                                void* stream) {
+  sq_status st = check_tensor_rows(W, dtype, N, K, ldw, SQ_NORM_NONE, s, nullptr, 0.0f);
+  if (st != SQ_OK) return st;
+  if (!w_absmax) return SQ_ERR_INVALID_ARG;
+  if (N > 0) {
+    if (!Wq) return SQ_ERR_INVALID_ARG;
+    if (!aligned16(Wq)) return SQ_ERR_ALIGNMENT;
+    if ((st = check_vec(w_scale, true)) != SQ_OK) return st;
+  }
+  int* err = device_error_word();
+  if (!err) return SQ_ERR_CUDA;
+  cudaStream_t cs = as_stream(stream);
+  // a weight row smoothed by s is the no-norm row path with s as multiplier
+  cudaError_t e = cudaMemsetAsync(w_absmax, 0, sizeof(float), cs);
+  if (e == cudaSuccess)
+    e = launch_tensor_absmax_pipe(W, dtype == SQ_BF16, N, static_cast<int>(K), ldw, SQ_NORM_NONE,
+                                  s, nullptr, 0.0f, w_absmax, err, cs);
+  if (e == cudaSuccess)
+    e = launch_quant_fixed_pipe(W, dtype == SQ_BF16, N, static_cast<int>(K), ldw, SQ_NORM_NONE, s,
+                                nullptr, 0.0f, w_absmax, Wq, w_scale, err, cs);
+  return from_cuda(e);
+}
+
 size_t sq_w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int split_k) {
   if (M <= 0 || N <= 0 || K <= 0 || split_k < 0) return 0;
   const int sms = sms_cached();

@@ -164,12 +164,20 @@ __device__ __forceinline__ int refill_row(uint32_t smem_base, uint32_t bar_base,
 }
 
 // NORMK: 0 = no norm (optional per-channel multiplier), 1 = RMSNorm, 2 = LayerNorm.
-template <int CH, bool kCalib>
+// What a launch of the row pipeline produces.
+enum RowMode : int {
+  kModeRowQuant = 0,    // per-row (per-token) step and codes
+  kModeColMax = 1,      // calibration: running per-column max of |y|
+  kModeTensorMax = 2,   // one running max of |y| over the whole tensor
+  kModeFixedQuant = 3,  // codes with one given step (per-tensor: O2 / O3)
+};
+
+template <int CH, int kMode>
 struct PipeBounds {
   static constexpr int kMaxThreads = CH <= 4 ? 512 : 640;
-  // 4-chunk quantising CTAs keep to 64 registers a thread so four 256-thread
-  // CTAs fit an SM; calibration also keeps a running column max per element
-  static constexpr int kMinBlocks = (CH <= 4 && !kCalib) ? 2 : 1;
+  // 4-chunk CTAs keep to 64 registers a thread so four 256-thread CTAs fit
+  // an SM; calibration also keeps a running column max per element
+  static constexpr int kMinBlocks = (CH <= 4 && kMode != kModeColMax) ? 2 : 1;
 };
 
 // One row per iteration, three CTA barriers per row (two when calibrating):
@@ -178,13 +186,16 @@ struct PipeBounds {
 //   B  warp 0 has turned the sums into r (and mu);
 //   C  the warps' partial absmax is merged, and thread 0 has seen the next
 //      row land (a bounded wait; a timeout aborts the CTA).
-// Calibrating (kCalib) folds C into B and keeps a per-thread running max of
-// |y| over the rows it sees, merged into act_max at the end.
+// Modes without a per-row absmax (calibration column max, fixed-step codes)
+// fold C into B.  Calibration keeps a per-thread running max of |y| over the
+// rows it sees, merged into act_max[K] at the end; the tensor-max mode keeps
+// the CTA's running max of the row maxima and merges it into act_max[0]; the
+// fixed-step mode reads its step's max |y| from act_max[0] once.
 //
 // kFull: every thread owns all CH of its chunks (T * CH == K / 8): no bounds checks.
-template <bool kBF16, int NORMK, int CH, bool kGamma, bool kBeta, bool kFull, bool kCalib>
-__global__ void __launch_bounds__(PipeBounds<CH, kCalib>::kMaxThreads,
-                                  PipeBounds<CH, kCalib>::kMinBlocks)
+template <bool kBF16, int NORMK, int CH, bool kGamma, bool kBeta, bool kFull, int kMode>
+__global__ void __launch_bounds__(PipeBounds<CH, kMode>::kMaxThreads,
+                                  PipeBounds<CH, kMode>::kMinBlocks)
     norm_rows_pipe_kernel(const void* __restrict__ x, int64_t ldx, int64_t M, int K,
                           const float* __restrict__ gamma, const float* __restrict__ beta,
                           float eps, int8_t* __restrict__ q, float* __restrict__ scale,
@@ -237,6 +248,17 @@ __global__ void __launch_bounds__(PipeBounds<CH, kCalib>::kMaxThreads,
   {
     const bool ok = (t != 0 || first >= M) ? true : row_landed(bar_base, nbuf, 0);
     if (__syncthreads_or(!ok)) aborted = true;
+  }
+  constexpr bool kCalib = kMode == kModeColMax;
+  constexpr bool kRowMax = kMode == kModeRowQuant || kMode == kModeTensorMax;
+  float cta_max = 0.0f;  // tensor-max mode, thread 0
+  // fixed-step mode: the one step, from the given max |y|
+  float fstep = 0.0f, frstep = 0.0f;
+  bool fexact = false;
+  if constexpr (kMode == kModeFixedQuant) {
+    fstep = div127(__ldg(act_max));
+    fexact = fstep < FLT_MIN;
+    frstep = fexact ? 0.0f : __frcp_rn(fstep);
   }
   float2 cm[kCalib ? CH : 1][4];  // calibration: running max of |y| per owned element
   if constexpr (kCalib) {
@@ -317,7 +339,7 @@ __global__ void __launch_bounds__(PipeBounds<CH, kCalib>::kMaxThreads,
         }
       }
     }
-    if constexpr (kCalib) {
+    if constexpr (!kRowMax) {
       // B (with C folded in): the row scalars are published and the next row is in
       const bool ok = (t != 0 || row + G >= M) ? true : row_landed(bar_base, nbuf, it + 1);
       if (__syncthreads_or(!ok)) {
@@ -367,11 +389,21 @@ __global__ void __launch_bounds__(PipeBounds<CH, kCalib>::kMaxThreads,
           cm[c][i].y = fmaxf(cm[c][i].y, fabsf(y.y));
         } else {
           v[c][i] = y;
-          am = fmaxf(am, fmaxf(fabsf(y.x), fabsf(y.y)));
+          if constexpr (kRowMax) am = fmaxf(am, fmaxf(fabsf(y.x), fabsf(y.y)));
         }
       }
     }
-    if constexpr (!kCalib) {
+    if constexpr (kMode == kModeFixedQuant) {
+      if (t == 0) scale[row] = fstep;
+      int8_t* qrow = q + row * static_cast<int64_t>(K);
+#pragma unroll
+      for (int c = 0; c < CH; ++c) {
+        const int ch = t + c * T;
+        if (!kFull && ch >= nchunks) continue;
+        *reinterpret_cast<uint2*>(qrow + ch * kChunk) = codes8(v[c], frstep, fstep, fexact);
+      }
+    }
+    if constexpr (kRowMax) {
       // non-negative floats order like their bit patterns: integer max reduce
       const unsigned int wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(am));
       if (lane == 0) atomicMax(&smax[slot], wmax);
@@ -386,17 +418,21 @@ __global__ void __launch_bounds__(PipeBounds<CH, kCalib>::kMaxThreads,
       am = __uint_as_float(smax[slot]);
       if (t == 0) smax[slot == 0 ? 2 : slot - 1] = 0u;  // the slot of row it + 2
 
-      // ---- per-token INT8 quantisation
-      const float step = div127(am);
-      const bool exact_only = step < FLT_MIN;  // zero or subnormal step: no reciprocal
-      const float rstep = exact_only ? 0.0f : __frcp_rn(step);
-      if (t == 0) scale[row] = step;
-      int8_t* qrow = q + row * static_cast<int64_t>(K);
+      if constexpr (kMode == kModeTensorMax) {
+        if (t == 0) cta_max = fmaxf(cta_max, am);
+      } else {
+        // ---- per-token INT8 quantisation
+        const float step = div127(am);
+        const bool exact_only = step < FLT_MIN;  // zero or subnormal step: no reciprocal
+        const float rstep = exact_only ? 0.0f : __frcp_rn(step);
+        if (t == 0) scale[row] = step;
+        int8_t* qrow = q + row * static_cast<int64_t>(K);
 #pragma unroll
-      for (int c = 0; c < CH; ++c) {
-        const int ch = t + c * T;
-        if (!kFull && ch >= nchunks) continue;
-        *reinterpret_cast<uint2*>(qrow + ch * kChunk) = codes8(v[c], rstep, step, exact_only);
+        for (int c = 0; c < CH; ++c) {
+          const int ch = t + c * T;
+          if (!kFull && ch >= nchunks) continue;
+          *reinterpret_cast<uint2*>(qrow + ch * kChunk) = codes8(v[c], rstep, step, exact_only);
+        }
       }
     }
   }
@@ -415,6 +451,13 @@ __global__ void __launch_bounds__(PipeBounds<CH, kCalib>::kMaxThreads,
       }
     }
     return;
+  }
+  if constexpr (kMode == kModeTensorMax) {
+    if (t == 0) {
+      unsigned int* dst = reinterpret_cast<unsigned int*>(act_max);
+      const unsigned int bits = __float_as_uint(cta_max);
+      if (bits > __ldcg(dst)) atomicMax(dst, bits);
+    }
   }
   if constexpr (kCalib) {
     // merge into the running maximum: an atomic only where this CTA's value is
@@ -485,9 +528,10 @@ struct RowArgs {
   int* err;
 };
 
-template <bool kBF16, int NORMK, int CH, bool kG, bool kB, bool kF, bool kC>
+template <bool kBF16, int NORMK, int CH, bool kG, bool kB, bool kF, int kMode>
 cudaError_t launch_pipe_k(const RowArgs& a, PipeShape ps, cudaStream_t st) {
-  auto kern = norm_rows_pipe_kernel<kBF16, NORMK, CH, kG, kB, kF, kC>;
+  constexpr bool kC = kMode == kModeColMax;
+  auto kern = norm_rows_pipe_kernel<kBF16, NORMK, CH, kG, kB, kF, kMode>;
   const void* key = reinterpret_cast<const void*>(kern);
   LaunchCache& lc = launch_cache();
   int per_sm = 0;
@@ -514,47 +558,47 @@ cudaError_t launch_pipe_k(const RowArgs& a, PipeShape ps, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-template <bool kBF16, int NORMK, int CH, bool kG, bool kB, bool kC>
+template <bool kBF16, int NORMK, int CH, bool kG, bool kB, int kMode>
 cudaError_t launch_pipe_t(const RowArgs& a, const PipeShape& ps, cudaStream_t st) {
   // bf16 rows whose chunks split evenly over the threads skip the bounds checks
   if constexpr (kBF16) {
     if (ps.threads * ps.ch == a.K / kChunk)
-      return launch_pipe_k<kBF16, NORMK, CH, kG, kB, true, kC>(a, ps, st);
+      return launch_pipe_k<kBF16, NORMK, CH, kG, kB, true, kMode>(a, ps, st);
   }
-  return launch_pipe_k<kBF16, NORMK, CH, kG, kB, false, kC>(a, ps, st);
+  return launch_pipe_k<kBF16, NORMK, CH, kG, kB, false, kMode>(a, ps, st);
 }
 
-template <bool kBF16, int NORMK, int CH, bool kC>
+template <bool kBF16, int NORMK, int CH, int kMode>
 cudaError_t launch_pipe_c(const RowArgs& a, const PipeShape& ps, cudaStream_t st) {
   // beta only matters for LayerNorm
   const bool hb = NORMK == 2 && a.beta != nullptr;
   if (a.gamma) {
-    if (hb) return launch_pipe_t<kBF16, NORMK, CH, true, NORMK == 2, kC>(a, ps, st);
-    return launch_pipe_t<kBF16, NORMK, CH, true, false, kC>(a, ps, st);
+    if (hb) return launch_pipe_t<kBF16, NORMK, CH, true, NORMK == 2, kMode>(a, ps, st);
+    return launch_pipe_t<kBF16, NORMK, CH, true, false, kMode>(a, ps, st);
   }
-  if (hb) return launch_pipe_t<kBF16, NORMK, CH, false, NORMK == 2, kC>(a, ps, st);
-  return launch_pipe_t<kBF16, NORMK, CH, false, false, kC>(a, ps, st);
+  if (hb) return launch_pipe_t<kBF16, NORMK, CH, false, NORMK == 2, kMode>(a, ps, st);
+  return launch_pipe_t<kBF16, NORMK, CH, false, false, kMode>(a, ps, st);
 }
 
-template <bool kBF16, int NORMK, bool kC>
+template <bool kBF16, int NORMK, int kMode>
 cudaError_t launch_pipe_n(const RowArgs& a, const PipeShape& ps, cudaStream_t st) {
-  if (ps.ch == 4) return launch_pipe_c<kBF16, NORMK, 4, kC>(a, ps, st);
-  if constexpr (kC) return cudaErrorInvalidValue;  // calibration: 4-chunk shapes only
-  else return launch_pipe_c<kBF16, NORMK, 8, kC>(a, ps, st);
+  if (ps.ch == 4) return launch_pipe_c<kBF16, NORMK, 4, kMode>(a, ps, st);
+  if constexpr (kMode == kModeColMax) return cudaErrorInvalidValue;  // 4-chunk shapes only
+  else return launch_pipe_c<kBF16, NORMK, 8, kMode>(a, ps, st);
 }
 
-template <bool kC>
+template <int kMode>
 cudaError_t launch_rows(const RowArgs& a, bool bf16, int norm, cudaStream_t st) {
   PipeShape ps;
   if (!pipe_shape(a.K, bf16, &ps)) return cudaErrorInvalidValue;
   if (bf16) {
-    if (norm == SQ_NORM_RMS) return launch_pipe_n<true, 1, kC>(a, ps, st);
-    if (norm == SQ_NORM_LAYER) return launch_pipe_n<true, 2, kC>(a, ps, st);
-    return launch_pipe_n<true, 0, kC>(a, ps, st);
+    if (norm == SQ_NORM_RMS) return launch_pipe_n<true, 1, kMode>(a, ps, st);
+    if (norm == SQ_NORM_LAYER) return launch_pipe_n<true, 2, kMode>(a, ps, st);
+    return launch_pipe_n<true, 0, kMode>(a, ps, st);
   }
-  if (norm == SQ_NORM_RMS) return launch_pipe_n<false, 1, kC>(a, ps, st);
-  if (norm == SQ_NORM_LAYER) return launch_pipe_n<false, 2, kC>(a, ps, st);
-  return launch_pipe_n<false, 0, kC>(a, ps, st);
+  if (norm == SQ_NORM_RMS) return launch_pipe_n<false, 1, kMode>(a, ps, st);
+  if (norm == SQ_NORM_LAYER) return launch_pipe_n<false, 2, kMode>(a, ps, st);
+  return launch_pipe_n<false, 0, kMode>(a, ps, st);
 }
 
 }  // namespace
@@ -574,7 +618,7 @@ cudaError_t launch_norm_quant_pipe(const void* x, bool bf16, int64_t M, int K, i
                                    int8_t* q, float* scale, int* err, cudaStream_t st) {
   if (M == 0) return cudaSuccess;
   const RowArgs a{x, M, K, ldx, gamma, beta, eps, q, scale, nullptr, err};
-  return launch_rows<false>(a, bf16, norm, st);
+  return launch_rows<kModeRowQuant>(a, bf16, norm, st);
 }
 
 cudaError_t launch_calibrate_pipe(const void* x, bool bf16, int64_t M, int K, int64_t ldx,
@@ -582,7 +626,24 @@ cudaError_t launch_calibrate_pipe(const void* x, bool bf16, int64_t M, int K, in
                                   float* act_max, int* err, cudaStream_t st) {
   if (M == 0) return cudaSuccess;
   const RowArgs a{x, M, K, ldx, gamma, beta, eps, nullptr, nullptr, act_max, err};
-  return launch_rows<true>(a, bf16, norm, st);
+  return launch_rows<kModeColMax>(a, bf16, norm, st);
+}
+
+cudaError_t launch_tensor_absmax_pipe(const void* x, bool bf16, int64_t M, int K, int64_t ldx,
+                                      int norm, const float* gamma, const float* beta, float eps,
+                                      float* absmax, int* err, cudaStream_t st) {
+  if (M == 0) return cudaSuccess;
+  const RowArgs a{x, M, K, ldx, gamma, beta, eps, nullptr, nullptr, absmax, err};
+  return launch_rows<kModeTensorMax>(a, bf16, norm, st);
+}
+
+cudaError_t launch_quant_fixed_pipe(const void* x, bool bf16, int64_t M, int K, int64_t ldx,
+                                    int norm, const float* gamma, const float* beta, float eps,
+                                    const float* absmax, int8_t* q, float* scale, int* err,
+                                    cudaStream_t st) {
+  if (M == 0) return cudaSuccess;
+  const RowArgs a{x, M, K, ldx, gamma, beta, eps, q, scale, const_cast<float*>(absmax), err};
+  return launch_rows<kModeFixedQuant>(a, bf16, norm, st);
 }
 
 }  // namespace sq

@@ -84,6 +84,14 @@ bool calibrate_pipe_supported(int K, bool bf16);
 cudaError_t launch_calibrate_pipe(const void* x, bool bf16, int64_t M, int K, int64_t ldx,
                                   int norm, const float* gamma, const float* beta, float eps,
                                   float* act_max, int* err, cudaStream_t st);
+// Per-tensor variants (rows the shared-memory ring holds: norm_quant_pipe_supported).
+cudaError_t launch_tensor_absmax_pipe(const void* x, bool bf16, int64_t M, int K, int64_t ldx,
+                                      int norm, const float* gamma, const float* beta, float eps,
+                                      float* absmax, int* err, cudaStream_t st);
+cudaError_t launch_quant_fixed_pipe(const void* x, bool bf16, int64_t M, int K, int64_t ldx,
+                                    int norm, const float* gamma, const float* beta, float eps,
+                                    const float* absmax, int8_t* q, float* scale, int* err,
+                                    cudaStream_t st);
 cudaError_t launch_calibrate(const void* x, bool bf16, int64_t M, int K, int64_t ldx, int norm,
                              const float* gamma, const float* beta, float eps, float* act_max,
                              int* err, cudaStream_t st);

@@ -33,7 +33,8 @@ EXPORTS = (
     "sq_calibrate_absmax", "sq_compute_smooth_scales", "sq_smooth_quantize_weights",
     "sq_norm_smooth_quant_per_token", "sq_w8a8_gemm_workspace_size", "sq_w8a8_gemm_dequant",
     "sq_linear_w8a8", "sq_status_string", "sq_get_device_error", "sq_set_wait_limit",
-    "sq_w8a8_gemm_dequant_noalloc", "sq_w8a8_gemm_plan",
+    "sq_w8a8_gemm_dequant_noalloc", "sq_w8a8_gemm_plan", "sq_norm_smooth_absmax",
+    "sq_norm_smooth_quant_per_tensor", "sq_smooth_quantize_weights_per_tensor",
 )
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -101,6 +102,11 @@ def _declare(L):
     L.sq_status_string.argtypes = [_I32]
     L.sq_status_string.restype = ctypes.c_char_p
     L.sq_get_device_error.argtypes = [_P]
+    L.sq_norm_smooth_absmax.argtypes = [_P, _I32, _I64, _I64, _I64, _I32, _P, _P, _F32, _P, _P]
+    L.sq_norm_smooth_quant_per_tensor.argtypes = [_P, _I32, _I64, _I64, _I64, _I32, _P, _P, _F32,
+                                                  _P, _P, _P, _P]
+    L.sq_smooth_quantize_weights_per_tensor.argtypes = [_P, _I32, _I64, _I64, _I64, _P, _P, _P,
+                                                        _P, _P]
     L.sq_w8a8_gemm_plan.argtypes = [_I64, _I64, _I64, _I32, _I32, ctypes.POINTER(GemmPlanInfo)]
     L.sq_set_wait_limit.argtypes = [_I64]
     L.sq_set_wait_limit.restype = None
@@ -229,6 +235,50 @@ def norm_smooth_quant_per_token(x: torch.Tensor, norm: int, gamma_folded=None, b
         _ptr(_vec(beta_folded, K, "beta_folded")), eps, _ptr(Xq), _ptr(x_scale), _stream(stream)),
         "sq_norm_smooth_quant_per_token")
     return Xq, x_scale
+
+
+def norm_smooth_absmax(x: torch.Tensor, norm: int, gamma_folded=None, beta_folded=None,
+                       eps: float = 1e-5, absmax=None, stream=None) -> torch.Tensor:
+    """Running max over all of |norm(x)| into a 1-element fp32 device tensor."""
+    M, K, ld = _rows(x, "x")
+    if absmax is None:
+        absmax = torch.zeros(1, dtype=torch.float32, device=x.device)
+    _check(lib().sq_norm_smooth_absmax(_ptr(x), _dtype_code(x), M, K, ld, norm,
+                                       _ptr(_vec(gamma_folded, K, "gamma_folded")),
+                                       _ptr(_vec(beta_folded, K, "beta_folded")), eps,
+                                       _ptr(absmax), _stream(stream)), "sq_norm_smooth_absmax")
+    return absmax
+
+
+def norm_smooth_quant_per_tensor(x: torch.Tensor, norm: int, absmax: torch.Tensor,
+                                 gamma_folded=None, beta_folded=None, eps: float = 1e-5,
+                                 Xq=None, x_scale=None, stream=None):
+    """Codes with the one step fl32(absmax / 127); x_scale holds it per row."""
+    M, K, ld = _rows(x, "x")
+    if Xq is None:
+        Xq = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    if x_scale is None:
+        x_scale = torch.empty(M, dtype=torch.float32, device=x.device)
+    _check(lib().sq_norm_smooth_quant_per_tensor(
+        _ptr(x), _dtype_code(x), M, K, ld, norm, _ptr(_vec(gamma_folded, K, "gamma_folded")),
+        _ptr(_vec(beta_folded, K, "beta_folded")), eps, _ptr(absmax), _ptr(Xq), _ptr(x_scale),
+        _stream(stream)), "sq_norm_smooth_quant_per_tensor")
+    return Xq, x_scale
+
+
+def smooth_quantize_weights_per_tensor(W: torch.Tensor, s: Optional[torch.Tensor] = None,
+                                       Wq=None, w_scale=None, w_absmax=None, stream=None):
+    N, K, ld = _rows(W, "W")
+    if Wq is None:
+        Wq = torch.empty((N, K), dtype=torch.int8, device=W.device)
+    if w_scale is None:
+        w_scale = torch.empty(N, dtype=torch.float32, device=W.device)
+    if w_absmax is None:
+        w_absmax = torch.empty(1, dtype=torch.float32, device=W.device)
+    _check(lib().sq_smooth_quantize_weights_per_tensor(
+        _ptr(W), _dtype_code(W), N, K, ld, _ptr(_vec(s, K, "s")), _ptr(Wq), _ptr(w_scale),
+        _ptr(w_absmax), _stream(stream)), "sq_smooth_quantize_weights_per_tensor")
+    return Wq, w_scale
 
 
 def gemm_plan(M: int, N: int, K: int, path_hint: int = 0, split_k: int = 0) -> GemmPlanInfo:
