@@ -362,7 +362,7 @@ def run_gpu(args, w):
     W = {k: to_dev(v) for k, v in inp.W.items()}
     g = {k: to_dev(v) for k, v in inp.gamma.items()}
     b = {k: to_dev(v) for k, v in inp.beta.items()}
-    blk = pipeline.Block(w, w.M, dev)
+    blk = pipeline.Block(w, w.M, dev, args.granularity)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -507,6 +507,7 @@ def run_gpu(args, w):
         "config": {"workload": w.name, "tokens": w.M, "calib_tokens": w.M_cal, "alpha": w.alpha,
                    "linears": ["%s %dx%d" % (l.name, w.site(l.site).K, l.N) for l in w.linears],
                    "step": "calibrate + smooth scales/fold + weight quant + norm-quant + GEMM",
+                   "granularity": args.granularity,
                    "launch": "the whole step as one CUDA graph, replayed per timed step",
                    "l2": "flushed before every step (256 MiB write, not timed)",
                    "parallelism": "dp%d (independent token batches, weights replicated)" % world},
@@ -527,7 +528,8 @@ def run_gpu(args, w):
         dist.barrier()
         dist.destroy_process_group()
 
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    # the oracle's baseline is the per-token path (the method's default scheme)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.granularity == "per_token":
         import oracle
         oracle.build()
         full, spent, desc = oracle_sample_step(w, inp)
@@ -603,6 +605,10 @@ def main(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--granularity", default="per_token",
+                    choices=["per_token", "per_tensor_dynamic", "per_tensor_static"],
+                    help="activation / weight scale sharing (per-token + per-channel, or the "
+                         "per-tensor O2 / O3 levels)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -8,7 +8,7 @@ import numpy as np
 import oracle
 
 
-def prepare(w, inp):
+def prepare(w, inp, granularity="per_token"):
     sites = {}
     for site in w.sites:
         st = {"norm": site.norm, "s": None, "s64": None}
@@ -21,12 +21,21 @@ def prepare(w, inp):
             st.update(act_max=am, s=s, s64=s64, gamma_f=gf, beta_f=bf)
         else:
             st.update(gamma_f=g, beta_f=b)
+        st["static_absmax"] = None
+        if granularity == "per_tensor_static" and site.smoothed and site.calibrated:
+            yc, _, _ = oracle.norm(inp.x_cal[site.name], site.norm, st["gamma_f"], st["beta_f"],
+                                   w.eps)
+            st["static_absmax"] = oracle.absmax_all(yc)
         sites[site.name] = st
     lins = {}
     for lin in w.linears:
-        Wq, ws = oracle.quantize_weights(inp.W[lin.name], sites[lin.site]["s"])
+        if granularity == "per_token":
+            Wq, ws = oracle.quantize_weights(inp.W[lin.name], sites[lin.site]["s"])
+        else:
+            Wq, step = oracle.quantize_weights_per_tensor(inp.W[lin.name], sites[lin.site]["s"])
+            ws = np.full(lin.N, step, np.float32)
         lins[lin.name] = {"Wq": Wq, "w_scale": ws}
-    return {"sites": sites, "linears": lins}
+    return {"sites": sites, "linears": lins, "granularity": granularity}
 
 
 def forward_rows(w, prep, inp, rows):
@@ -40,7 +49,12 @@ def forward_rows(w, prep, inp, rows):
         else:
             x = np.ascontiguousarray(inp.x[site.name][rows])
         st = prep["sites"][site.name]
-        Xq, xs = oracle.norm_quant(x, site.norm, st["gamma_f"], st["beta_f"], w.eps)
+        if prep.get("granularity", "per_token") == "per_token":
+            Xq, xs = oracle.norm_quant(x, site.norm, st["gamma_f"], st["beta_f"], w.eps)
+        else:  # per-tensor: `rows` must be the whole tensor for O2
+            Xq, step = oracle.norm_quant_per_tensor(x, site.norm, st["gamma_f"], st["beta_f"],
+                                                    w.eps, absmax=st["static_absmax"])
+            xs = np.full(x.shape[0], step, np.float32)
         res["sites"][site.name] = {"x": x, "Xq": Xq, "xs": xs}
         for lin in w.linears_of(site.name):
             L = prep["linears"][lin.name]

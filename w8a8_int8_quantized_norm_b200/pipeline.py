@@ -33,6 +33,9 @@ def _run(timer: Timer, kind: str, units: float, fn: Callable[[], None]) -> None:
         timer(kind, units, fn)
 
 
+GRANULARITIES = ("per_token", "per_tensor_dynamic", "per_tensor_static")
+
+
 class Block:
     """Device state of one workload for M tokens per forward.
 
@@ -40,11 +43,23 @@ class Block:
     weight smoothing + quantisation); ``forward`` the runtime rows (fused norm
     + per-token quantisation, INT8 GEMM with the dequant epilogue).  An optional
     ``timer`` hook brackets every library call (the benchmark records CUDA
-    events there)."""
+    events there).
 
-    def __init__(self, w: Workload, M: int, device):
+    ``granularity`` (see "SmoothQuant, in depth" -- "Granularity: O1, O2, O3"):
+    ``per_token`` is the serving-stack scheme (per-token dynamic activation
+    scales, per-output-channel weight scales); ``per_tensor_dynamic`` (O2) and
+    ``per_tensor_static`` (O3) use one weight scale per matrix and one
+    activation scale per tensor -- the tensor's own max |y| (O2), or the max
+    over the calibration tokens through the folded norm, fixed in ``prepare``
+    (O3; a site without calibration tokens, i.e. an unsmoothed Linear input,
+    falls back to its own max)."""
+
+    def __init__(self, w: Workload, M: int, device, granularity: str = "per_token"):
+        if granularity not in GRANULARITIES:
+            raise ValueError("granularity must be one of %s" % (GRANULARITIES,))
         self.w = w
         self.M = M
+        self.granularity = granularity
         dev = torch.device(device)
         f32 = dict(dtype=torch.float32, device=dev)
         self.act_max: Dict[str, torch.Tensor] = {}
@@ -73,9 +88,16 @@ class Block:
             self.ws[lin.name] = torch.empty(need, dtype=torch.uint8, device=dev) if need else None
         self.xq: Dict[str, torch.Tensor] = {}
         self.xs: Dict[str, torch.Tensor] = {}
+        self.x_absmax: Dict[str, torch.Tensor] = {}  # per-tensor modes: max |y| per site
+        self.static: Dict[str, bool] = {}            # O3: the site's max is calibrated
         for site in w.sites:
             self.xq[site.name] = torch.empty((M, site.K), dtype=torch.int8, device=dev)
             self.xs[site.name] = torch.empty(M, **f32)
+            self.x_absmax[site.name] = torch.zeros(1, **f32)
+            self.static[site.name] = (granularity == "per_tensor_static" and site.smoothed
+                                      and site.calibrated)
+        self.w_absmax: Dict[str, torch.Tensor] = {l.name: torch.zeros(1, **f32)
+                                                  for l in w.linears}
 
     # -- offline rows -------------------------------------------------------
     def prepare(self, x_cal: Dict[str, torch.Tensor], W: Dict[str, torch.Tensor],
@@ -103,12 +125,30 @@ class Block:
                                                       stream=stream))
             else:
                 self.gamma_f[site.name], self.beta_f[site.name] = g, b
+            if self.static[site.name]:
+                # O3: the static max |y| of the calibration tokens through the folded norm
+                xc = x_cal[site.name]
+                am = self.x_absmax[site.name]
+                am.zero_()
+                _run(timer, "static_absmax", xc.numel() * xc.element_size(),
+                     lambda: sq.norm_smooth_absmax(xc, site.norm, self.gamma_f[site.name],
+                                                   self.beta_f[site.name], w.eps, absmax=am,
+                                                   stream=stream))
+        per_tensor = self.granularity != "per_token"
         for lin in w.linears:
             Wl = W[lin.name]
-            _run(timer, "weight_quant", Wl.numel() * (Wl.element_size() + 1) + 4 * lin.N,
-                 lambda: sq.smooth_quantize_weights(Wl, self.s[lin.site], Wq=self.Wq[lin.name],
-                                                    w_scale=self.w_scale[lin.name],
-                                                    stream=stream))
+            units = Wl.numel() * (Wl.element_size() + 1) + 4 * lin.N
+            if per_tensor:  # one more read of W for the matrix-wide max
+                _run(timer, "weight_quant", units + Wl.numel() * Wl.element_size(),
+                     lambda: sq.smooth_quantize_weights_per_tensor(
+                         Wl, self.s[lin.site], Wq=self.Wq[lin.name],
+                         w_scale=self.w_scale[lin.name], w_absmax=self.w_absmax[lin.name],
+                         stream=stream))
+            else:
+                _run(timer, "weight_quant", units,
+                     lambda: sq.smooth_quantize_weights(Wl, self.s[lin.site], Wq=self.Wq[lin.name],
+                                                        w_scale=self.w_scale[lin.name],
+                                                        stream=stream))
         return self
 
     # -- runtime rows -------------------------------------------------------
@@ -119,12 +159,24 @@ class Block:
             src = next((l.source for l in w.linears if l.site == site.name and l.source), None)
             xin = self.out[src] if src else x[site.name]
             nparam = (self.gamma_f[site.name] is not None) + (self.beta_f[site.name] is not None)
-            _run(timer, "norm_quant",
-                 xin.numel() * (xin.element_size() + 1) + 4 * self.M + 4 * site.K * nparam,
-                 lambda: sq.norm_smooth_quant_per_token(xin, site.norm, self.gamma_f[site.name],
-                                                        self.beta_f[site.name], w.eps,
-                                                        self.xq[site.name], self.xs[site.name],
-                                                        stream=stream))
+            units = xin.numel() * (xin.element_size() + 1) + 4 * self.M + 4 * site.K * nparam
+            gf, bf = self.gamma_f[site.name], self.beta_f[site.name]
+            if self.granularity == "per_token":
+                _run(timer, "norm_quant", units,
+                     lambda: sq.norm_smooth_quant_per_token(xin, site.norm, gf, bf, w.eps,
+                                                            self.xq[site.name],
+                                                            self.xs[site.name], stream=stream))
+            else:
+                am = self.x_absmax[site.name]
+                if not self.static[site.name]:  # O2: this tensor's own max first
+                    am.zero_()
+                    _run(timer, "absmax", xin.numel() * xin.element_size() + 4 * site.K * nparam,
+                         lambda: sq.norm_smooth_absmax(xin, site.norm, gf, bf, w.eps, absmax=am,
+                                                       stream=stream))
+                _run(timer, "norm_quant", units,
+                     lambda: sq.norm_smooth_quant_per_tensor(xin, site.norm, am, gf, bf, w.eps,
+                                                             self.xq[site.name],
+                                                             self.xs[site.name], stream=stream))
             for lin in w.linears_of(site.name):
                 def gemm(lin=lin, site=site):
                     sq.w8a8_gemm_dequant(self.xq[site.name], self.Wq[lin.name],
@@ -144,13 +196,18 @@ class Block:
         for site in self.w.sites:
             if site.smoothed:
                 n += 2 + len(self.w.linears_of(site.name))
-        return n + len(self.w.linears)
+            if self.static[site.name]:
+                n += 1  # the static max over the calibration tokens
+        per_tensor = self.granularity != "per_token"
+        return n + len(self.w.linears) * (2 if per_tensor else 1)
 
     def forward_launches(self) -> int:
         """Kernels one ``forward`` launches: norm-quant per site, and per Linear
         the kernels of its GEMM plan (the main kernel, plus the split-K
         reduction or stream-K fix-up where the plan has one)."""
         n = len(self.w.sites)
+        if self.granularity != "per_token":
+            n += sum(1 for site in self.w.sites if not self.static[site.name])  # O2 max pass
         for lin in self.w.linears:
             n += sq.gemm_plan(self.M, lin.N, self.w.site(lin.site).K).launches
         return n
@@ -180,5 +237,6 @@ class Block:
 # Thin functional wrappers (used by tests and the smoke check).
 
 def prepare(w: Workload, x_cal, W, gamma, beta, M: Optional[int] = None, device="cuda",
-            stream=None) -> Block:
-    return Block(w, w.M if M is None else M, device).prepare(x_cal, W, gamma, beta, stream)
+            stream=None, granularity: str = "per_token") -> Block:
+    return Block(w, w.M if M is None else M, device, granularity).prepare(x_cal, W, gamma, beta,
+                                                                           stream)
