@@ -82,11 +82,16 @@ __device__ __forceinline__ double warp_sum(double v) {
 // clamp(rne(fl32(v / step)), -127, 127).  Fast path: one fused multiply-add
 // rounds the exact product P = v * rstep (rstep = fl32(1 / step)) to an
 // integer, ties to even, as the low mantissa bits of P + 1.5 * 2^23; P is
-// within 3 * 2^-24 relative of v / step and |P| < 127.5, so the code equals
-// the exact one -- no clamp needed -- unless v / step lies within 1e-4 of a
-// half-integer.  The residual P - n (one more fused multiply-add) flags that
-// case; a chunk holding such a value, or a step without a finite reciprocal,
-// is recomputed from the exact quotient.
+// within 3 * 2^-24 relative of v / step and, when step is the row's own
+// max / 127, |P| < 127.5, so the code equals the exact one -- no clamp
+// needed -- unless v / step lies within 1e-4 of a half-integer.  The residual
+// P - n (one more fused multiply-add) flags that case; a chunk holding such a
+// value, or a step without a finite reciprocal, is recomputed from the exact
+// quotient.  kClamp: the step may be smaller than max |v| / 127 (a fixed,
+// per-tensor step), so the rounded integer is clamped to [-127, 127] in the
+// magic domain (the only boundary, 127.5, is a half-integer: the residual
+// test sends it to the exact path, which clamps too).
+template <bool kClamp = false>
 __device__ __forceinline__ uint2 codes8(const float2 (&v)[4], float rstep, float step,
                                         bool exact_only) {
   uint32_t m[8];
@@ -96,10 +101,14 @@ __device__ __forceinline__ uint2 codes8(const float2 (&v)[4], float rstep, float
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     // paired fp32 instructions: each component rounds exactly like the scalar op
-    const float2 mf = __ffma2_rn(v[i], rs, mg);
+    float2 mf = __ffma2_rn(v[i], rs, mg);
     const float2 n = __fadd2_rn(mf, make_float2(-kMagic, -kMagic));
     const float2 d = __ffma2_rn(v[i], rs, make_float2(-n.x, -n.y));
     dmax = fmaxf(dmax, fmaxf(fabsf(d.x), fabsf(d.y)));
+    if constexpr (kClamp) {
+      mf.x = fminf(fmaxf(mf.x, kMagic - 127.0f), kMagic + 127.0f);
+      mf.y = fminf(fmaxf(mf.y, kMagic - 127.0f), kMagic + 127.0f);
+    }
     m[2 * i] = __float_as_uint(mf.x);
     m[2 * i + 1] = __float_as_uint(mf.y);
   }
@@ -400,7 +409,8 @@ __global__ void __launch_bounds__(PipeBounds<CH, kMode>::kMaxThreads,
       for (int c = 0; c < CH; ++c) {
         const int ch = t + c * T;
         if (!kFull && ch >= nchunks) continue;
-        *reinterpret_cast<uint2*>(qrow + ch * kChunk) = codes8(v[c], frstep, fstep, fexact);
+        *reinterpret_cast<uint2*>(qrow + ch * kChunk) =
+            codes8<true>(v[c], frstep, fstep, fexact);
       }
     }
     if constexpr (kRowMax) {
