@@ -146,10 +146,9 @@ __device__ __forceinline__ float div127(float a) {
   return __fmaf_rn(r, c, q0);
 }
 
-// Bounded wait for the copy of the CTA's row number `i` (buffer i mod nbuf).
-__device__ __forceinline__ bool row_landed(uint32_t bar_base, int nbuf, int i) {
-  const uint32_t bar = bar_base + 8u * static_cast<uint32_t>(i % nbuf);
-  const uint32_t parity = static_cast<uint32_t>((i / nbuf) & 1);
+// Bounded wait for a row copy: buffer `b`, phase parity `parity`.
+__device__ __forceinline__ bool row_landed(uint32_t bar_base, int b, uint32_t parity) {
+  const uint32_t bar = bar_base + 8u * static_cast<uint32_t>(b);
   if (mbar_try_wait(bar, parity)) return true;
   const long long c0 = clock64();
   for (uint32_t k = 0;; ++k) {
@@ -158,13 +157,12 @@ __device__ __forceinline__ bool row_landed(uint32_t bar_base, int nbuf, int i) {
   }
 }
 
-// The buffer of row number `i` has been read: load the row nbuf further on
-// into it (if there is one).  Returns the new count of issued copies.
+// The buffer `pb` of row number `i` has been read: load the row nbuf further
+// on into it (if there is one).  Returns the new count of issued copies.
 __device__ __forceinline__ int refill_row(uint32_t smem_base, uint32_t bar_base,
                                           uint32_t buf_stride, uint32_t row_bytes, int nbuf, int i,
-                                          int64_t row, int64_t G, int64_t M, const uint8_t* xb,
-                                          int64_t row_pitch, int issued) {
-  const int pb = i % nbuf;
+                                          int pb, int64_t row, int64_t G, int64_t M,
+                                          const uint8_t* xb, int64_t row_pitch, int issued) {
   const int64_t nrow = row + static_cast<int64_t>(nbuf) * G;
   if (nrow >= M) return issued;
   mbar_arrive_expect_tx(bar_base + 8u * pb, row_bytes);
@@ -255,7 +253,7 @@ __global__ void __launch_bounds__(PipeBounds<CH, kMode>::kMaxThreads,
   }
   bool aborted = false;
   {
-    const bool ok = (t != 0 || first >= M) ? true : row_landed(bar_base, nbuf, 0);
+    const bool ok = (t != 0 || first >= M) ? true : row_landed(bar_base, 0, 0u);
     if (__syncthreads_or(!ok)) aborted = true;
   }
   constexpr bool kCalib = kMode == kModeColMax;
@@ -278,9 +276,15 @@ __global__ void __launch_bounds__(PipeBounds<CH, kMode>::kMaxThreads,
   }
 
   int it = 0;
-  for (int64_t row = first; row < M && !aborted; row += G, ++it) {
-    const int slot = it % 3;
-    const uint8_t* rowp = smem + (it % nbuf) * buf_stride;
+  int buf = 0;            // it mod nbuf
+  int slot = 0;           // it mod 3
+  int nbuf_next = nbuf > 1 ? 1 : 0;  // (it + 1) mod nbuf
+  uint32_t par_next = nbuf > 1 ? 0u : 1u;  // phase parity of row it + 1's copy
+  for (int64_t row = first; row < M && !aborted;
+       row += G, ++it, buf = nbuf_next, slot = (slot == 2 ? 0 : slot + 1),
+               par_next ^= (nbuf_next + 1 == nbuf) ? 1u : 0u,
+               nbuf_next = (nbuf_next + 1 == nbuf) ? 0 : nbuf_next + 1) {
+    const uint8_t* rowp = smem + buf * buf_stride;
 
     // ---- this thread's chunks of the row, from shared memory
     float2 v[CH][4];
@@ -319,8 +323,8 @@ __global__ void __launch_bounds__(PipeBounds<CH, kMode>::kMaxThreads,
       }
       __syncthreads();  // A
       if (t == 0)
-        issued = refill_row(smem_base, bar_base, buf_stride, row_bytes, nbuf, it, row, G, M, xb,
-                            row_pitch, issued);
+        issued = refill_row(smem_base, bar_base, buf_stride, row_bytes, nbuf, it, buf, row, G, M,
+                            xb, row_pitch, issued);
       // one warp turns the sums into the row's scalars (the fp64 divide and
       // square root are long instruction sequences: not worth repeating in
       // every warp)
@@ -350,14 +354,14 @@ __global__ void __launch_bounds__(PipeBounds<CH, kMode>::kMaxThreads,
     }
     if constexpr (!kRowMax) {
       // B (with C folded in): the row scalars are published and the next row is in
-      const bool ok = (t != 0 || row + G >= M) ? true : row_landed(bar_base, nbuf, it + 1);
+      const bool ok = (t != 0 || row + G >= M) ? true : row_landed(bar_base, nbuf_next, par_next);
       if (__syncthreads_or(!ok)) {
         aborted = true;
         break;
       }
       if (NORMK == 0 && t == 0)
-        issued = refill_row(smem_base, bar_base, buf_stride, row_bytes, nbuf, it, row, G, M, xb,
-                            row_pitch, issued);
+        issued = refill_row(smem_base, bar_base, buf_stride, row_bytes, nbuf, it, buf, row, G, M,
+                            xb, row_pitch, issued);
     } else if constexpr (NORMK != 0) {
       __syncthreads();  // B
     }
@@ -417,14 +421,14 @@ __global__ void __launch_bounds__(PipeBounds<CH, kMode>::kMaxThreads,
       // non-negative floats order like their bit patterns: integer max reduce
       const unsigned int wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(am));
       if (lane == 0) atomicMax(&smax[slot], wmax);
-      const bool ok = (t != 0 || row + G >= M) ? true : row_landed(bar_base, nbuf, it + 1);
+      const bool ok = (t != 0 || row + G >= M) ? true : row_landed(bar_base, nbuf_next, par_next);
       if (__syncthreads_or(!ok)) {  // C
         aborted = true;
         break;
       }
       if (NORMK == 0 && t == 0)
-        issued = refill_row(smem_base, bar_base, buf_stride, row_bytes, nbuf, it, row, G, M, xb,
-                            row_pitch, issued);
+        issued = refill_row(smem_base, bar_base, buf_stride, row_bytes, nbuf, it, buf, row, G, M,
+                            xb, row_pitch, issued);
       am = __uint_as_float(smax[slot]);
       if (t == 0) smax[slot == 0 ? 2 : slot - 1] = 0u;  // the slot of row it + 2
 
@@ -499,11 +503,15 @@ struct PipeShape {
 // row buffers, their barriers, 64 doubles of partial sums, r and mu, 3 absmax slots
 size_t pipe_smem(size_t stride, int nbuf) { return nbuf * stride + 8 * nbuf + 64 * 8 + 4 * 8; }
 
-bool pipe_shape(int K, bool bf16, PipeShape* ps) {
+bool pipe_shape(int K, bool bf16, bool calib, PipeShape* ps) {
   const int nchunks = K / kChunk;
   // chunks per thread and threads per CTA within the variant's register budget
-  int ch = nchunks <= 4 * PipeBounds<4, false>::kMaxThreads ? 4
-           : (nchunks <= 8 * PipeBounds<8, false>::kMaxThreads ? 8 : 0);
+  int ch = nchunks <= 4 * PipeBounds<4, kModeRowQuant>::kMaxThreads ? 4
+           : (nchunks <= 8 * PipeBounds<8, kModeRowQuant>::kMaxThreads ? 8 : 0);
+  // rows of 2048-4096 elements: eight chunks per thread (32-64 threads a row)
+  // halve the per-row work (barriers, step, bookkeeping) per element; the
+  // calibration variant keeps four (it also holds a column max per element)
+  if (!calib && nchunks >= 8 * 32 && nchunks <= 8 * 64) ch = 8;
   if (!ch) return false;
   int threads = (nchunks + ch - 1) / ch;
   threads = (threads + 31) / 32 * 32;
@@ -600,7 +608,7 @@ cudaError_t launch_pipe_n(const RowArgs& a, const PipeShape& ps, cudaStream_t st
 template <int kMode>
 cudaError_t launch_rows(const RowArgs& a, bool bf16, int norm, cudaStream_t st) {
   PipeShape ps;
-  if (!pipe_shape(a.K, bf16, &ps)) return cudaErrorInvalidValue;
+  if (!pipe_shape(a.K, bf16, kMode == kModeColMax, &ps)) return cudaErrorInvalidValue;
   if (bf16) {
     if (norm == SQ_NORM_RMS) return launch_pipe_n<true, 1, kMode>(a, ps, st);
     if (norm == SQ_NORM_LAYER) return launch_pipe_n<true, 2, kMode>(a, ps, st);
@@ -615,12 +623,12 @@ cudaError_t launch_rows(const RowArgs& a, bool bf16, int norm, cudaStream_t st) 
 
 bool norm_quant_pipe_supported(int K, bool bf16) {
   PipeShape ps;
-  return pipe_shape(K, bf16, &ps);
+  return pipe_shape(K, bf16, false, &ps);
 }
 
 bool calibrate_pipe_supported(int K, bool bf16) {
   PipeShape ps;
-  return pipe_shape(K, bf16, &ps) && ps.ch == 4;
+  return pipe_shape(K, bf16, true, &ps) && ps.ch == 4;
 }
 
 cudaError_t launch_norm_quant_pipe(const void* x, bool bf16, int64_t M, int K, int64_t ldx,
