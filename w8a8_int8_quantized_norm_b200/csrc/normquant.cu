@@ -72,15 +72,6 @@ __device__ __forceinline__ void param8(const float* p, int ch, float2 (&v)[4]) {
   v[3] = make_float2(b.z, b.w);
 }
 
-__device__ __forceinline__ void param8_smem(const float* p, int ch, float2 (&v)[4]) {
-  const float4* q = reinterpret_cast<const float4*>(p + ch * kChunk);
-  const float4 a = q[0], b = q[1];
-  v[0] = make_float2(a.x, a.y);
-  v[1] = make_float2(a.z, a.w);
-  v[2] = make_float2(b.x, b.y);
-  v[3] = make_float2(b.z, b.w);
-}
-
 __device__ __forceinline__ double warp_sum(double v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = __dadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -215,8 +206,7 @@ __global__ void __launch_bounds__(PipeBounds<CH, kMode>::kMaxThreads,
     norm_rows_pipe_kernel(const void* __restrict__ x, int64_t ldx, int64_t M, int K,
                           const float* __restrict__ gamma, const float* __restrict__ beta,
                           float eps, int8_t* __restrict__ q, float* __restrict__ scale,
-                          float* __restrict__ act_max, int nbuf, int stage_params,
-                          int* error_word) {
+                          float* __restrict__ act_max, int nbuf, int* error_word) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int kEsz = kBF16 ? 2 : 4;
   const uint32_t row_bytes = static_cast<uint32_t>(K) * kEsz;
@@ -228,12 +218,6 @@ __global__ void __launch_bounds__(PipeBounds<CH, kMode>::kMaxThreads,
   // barrier C and reads it after; thread 0 clears the slot of row i + 2 after
   // C, which every thread passes again (C of row i + 1) before touching it
   unsigned int* smax = reinterpret_cast<unsigned int*>(fscr + 2);
-  // stage_params: gamma (and beta) copied once into shared memory, read per
-  // row from there (with the SM's shared memory full of row buffers there is
-  // little L1 left, and per-row global re-reads of the same vector stall)
-  float* gs = reinterpret_cast<float*>(
-      (reinterpret_cast<uintptr_t>(smax + 3) + 15u) & ~static_cast<uintptr_t>(15u));
-  float* bs = gs + K;
   const uint32_t smem_base = smem_u32(smem);
   const uint32_t bar_base = smem_u32(bars);
 
@@ -245,19 +229,6 @@ __global__ void __launch_bounds__(PipeBounds<CH, kMode>::kMaxThreads,
   const uint8_t* xb = static_cast<const uint8_t*>(x);
   const int64_t row_pitch = ldx * kEsz;
 
-  if (stage_params) {
-    const int n4 = K / 4;
-    if constexpr (kGamma) {
-      const float4* src = reinterpret_cast<const float4*>(gamma);
-      float4* dst = reinterpret_cast<float4*>(gs);
-      for (int i = t; i < n4; i += T) dst[i] = __ldg(src + i);
-    }
-    if constexpr (kBeta) {
-      const float4* src = reinterpret_cast<const float4*>(beta);
-      float4* dst = reinterpret_cast<float4*>(bs);
-      for (int i = t; i < n4; i += T) dst[i] = __ldg(src + i);
-    }
-  }
   if (t == 0) {
     for (int b = 0; b < nbuf; ++b) mbar_init(bar_base + 8u * b, 1);
     smax[0] = 0u;
@@ -409,12 +380,8 @@ __global__ void __launch_bounds__(PipeBounds<CH, kMode>::kMaxThreads,
       const int ch = t + c * T;
       if (!kFull && ch >= nchunks) continue;
       float2 g[4], bt[4];
-      if constexpr (kGamma) {
-        if (stage_params) param8_smem(gs, ch, g); else param8(gamma, ch, g);
-      }
-      if constexpr (kBeta) {
-        if (stage_params) param8_smem(bs, ch, bt); else param8(beta, ch, bt);
-      }
+      if constexpr (kGamma) param8(gamma, ch, g);
+      if constexpr (kBeta) param8(beta, ch, bt);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         float2 y = v[c][i];
@@ -533,12 +500,8 @@ struct PipeShape {
   size_t smem;
 };
 
-// row buffers, their barriers, 64 doubles of partial sums, r and mu, 3 absmax
-// slots, then (staged parameters) 16-byte aligned gamma and beta
-size_t pipe_smem(size_t stride, int nbuf, size_t param_bytes = 0) {
-  const size_t head = nbuf * stride + 8 * nbuf + 64 * 8 + 4 * 5;
-  return param_bytes ? (head + 15) / 16 * 16 + param_bytes : head;
-}
+// row buffers, their barriers, 64 doubles of partial sums, r and mu, 3 absmax slots
+size_t pipe_smem(size_t stride, int nbuf) { return nbuf * stride + 8 * nbuf + 64 * 8 + 4 * 8; }
 
 bool pipe_shape(int K, bool bf16, bool calib, PipeShape* ps) {
   const int nchunks = K / kChunk;
@@ -592,10 +555,6 @@ cudaError_t launch_pipe_k(const RowArgs& a, PipeShape ps, cudaStream_t st) {
   int per_sm = 0;
   // fewer row buffers when each CTA sees only a few rows: more CTAs fit an SM
   const size_t stride = (static_cast<size_t>(a.K) * (kBF16 ? 2 : 4) + 127) / 128 * 128;
-  // gamma / beta staged in shared memory when they take at most 32 KB
-  const size_t param_bytes = static_cast<size_t>(a.K) * 4 * ((kG ? 1 : 0) + (kB ? 1 : 0));
-  const int stage = param_bytes > 0 && param_bytes <= (32u << 10) ? 1 : 0;
-  ps.smem = pipe_smem(stride, ps.nbuf, stage ? param_bytes : 0);
   for (;;) {
     cudaError_t e = lc.ensure_smem(key, ps.smem);
     if (e != cudaSuccess) return e;
@@ -605,7 +564,7 @@ cudaError_t launch_pipe_k(const RowArgs& a, PipeShape ps, cudaStream_t st) {
     const int64_t rows_per_cta = (a.M + ctas - 1) / ctas;
     if (ps.nbuf <= 2 || rows_per_cta >= ps.nbuf) break;
     ps.nbuf = rows_per_cta < 2 ? 2 : static_cast<int>(rows_per_cta);
-    ps.smem = pipe_smem(stride, ps.nbuf, stage ? param_bytes : 0);
+    ps.smem = pipe_smem(stride, ps.nbuf);
   }
   int64_t grid = static_cast<int64_t>(per_sm) * lc.sms();
   // calibration merges every CTA's column maxima with atomics: at least four
@@ -613,8 +572,7 @@ cudaError_t launch_pipe_k(const RowArgs& a, PipeShape ps, cudaStream_t st) {
   const int64_t max_grid = kC ? (a.M + 3) / 4 : a.M;
   if (grid > max_grid) grid = max_grid;
   kern<<<static_cast<unsigned>(grid), ps.threads, ps.smem, st>>>(
-      a.x, a.ldx, a.M, a.K, a.gamma, a.beta, a.eps, a.q, a.scale, a.act_max, ps.nbuf, stage,
-      a.err);
+      a.x, a.ldx, a.M, a.K, a.gamma, a.beta, a.eps, a.q, a.scale, a.act_max, ps.nbuf, a.err);
   return cudaGetLastError();
 }
 
