@@ -508,10 +508,7 @@ bool pipe_shape(int K, bool bf16, bool calib, PipeShape* ps) {
   // chunks per thread and threads per CTA within the variant's register budget
   int ch = nchunks <= 4 * PipeBounds<4, kModeRowQuant>::kMaxThreads ? 4
            : (nchunks <= 8 * PipeBounds<8, kModeRowQuant>::kMaxThreads ? 8 : 0);
-  // rows of 2048-4096 elements: eight chunks per thread (32-64 threads a row)
-  // halve the per-row work (barriers, step, bookkeeping) per element; the
-  // calibration variant keeps four (it also holds a column max per element)
-  if (!calib && nchunks >= 8 * 32 && nchunks <= 8 * 64) ch = 8;
+  (void)calib;  // the calibration variant uses the same shape (4-chunk rows only)
   if (!ch) return false;
   int threads = (nchunks + ch - 1) / ch;
   threads = (threads + 31) / 32 * 32;
