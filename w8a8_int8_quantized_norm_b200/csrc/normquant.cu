@@ -474,23 +474,32 @@ __global__ void __launch_bounds__(PipeBounds<CH, kMode>::kMaxThreads,
     }
   }
   if constexpr (kCalib) {
-    // merge into the running maximum: an atomic only where this CTA's value is
-    // larger than what act_max already holds (the maximum only grows, so a
-    // stale read costs an extra atomic, never a lost update)
-    unsigned int* am_bits = reinterpret_cast<unsigned int*>(act_max);
+    // merge into the running maximum.  The CTA's column maxima go to shared
+    // memory first (the row ring is idle now: it holds K floats) and are
+    // merged in an order rotated by CTA, so concurrent CTAs hit different L2
+    // lines instead of queueing on the same ones; an atomic only where this
+    // CTA's value is larger than what act_max already holds (the maximum only
+    // grows, so a stale read costs an extra atomic, never a lost update).
+    unsigned int* colmax = reinterpret_cast<unsigned int*>(smem);
+    __syncthreads();  // every thread is done with the row buffers
 #pragma unroll
     for (int c = 0; c < CH; ++c) {
       const int ch = t + c * T;
       if (!kFull && ch >= nchunks) continue;
-      const uint4 cur0 = __ldcg(reinterpret_cast<const uint4*>(am_bits + ch * kChunk));
-      const uint4 cur1 = __ldcg(reinterpret_cast<const uint4*>(am_bits + ch * kChunk + 4));
-      const unsigned int cur[8] = {cur0.x, cur0.y, cur0.z, cur0.w, cur1.x, cur1.y, cur1.z, cur1.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const unsigned int a0 = __float_as_uint(cm[c][i].x), a1 = __float_as_uint(cm[c][i].y);
-        if (a0 > cur[2 * i]) atomicMax(am_bits + ch * kChunk + 2 * i, a0);
-        if (a1 > cur[2 * i + 1]) atomicMax(am_bits + ch * kChunk + 2 * i + 1, a1);
-      }
+      uint4* dst = reinterpret_cast<uint4*>(colmax + ch * kChunk);
+      dst[0] = make_uint4(__float_as_uint(cm[c][0].x), __float_as_uint(cm[c][0].y),
+                          __float_as_uint(cm[c][1].x), __float_as_uint(cm[c][1].y));
+      dst[1] = make_uint4(__float_as_uint(cm[c][2].x), __float_as_uint(cm[c][2].y),
+                          __float_as_uint(cm[c][3].x), __float_as_uint(cm[c][3].y));
+    }
+    __syncthreads();
+    unsigned int* am_bits = reinterpret_cast<unsigned int*>(act_max);
+    const int rot = static_cast<int>((blockIdx.x * 613u) % static_cast<unsigned>(K));
+    for (int i = t; i < K; i += T) {
+      int j = i + rot;
+      if (j >= K) j -= K;
+      const unsigned int a = colmax[j];
+      if (a > __ldcg(am_bits + j)) atomicMax(am_bits + j, a);
     }
   }
 }

@@ -266,7 +266,9 @@ __global__ void __launch_bounds__(256) weight_colmax_kernel(const void* __restri
   dst[0] = make_float4(m[0], m[1], m[2], m[3]);
   dst[1] = make_float4(m[4], m[5], m[6], m[7]);
   __syncthreads();
-  const int j = threadIdx.x;  // column of the slab
+  // column of the slab, rotated by the CTA's row run so that concurrent CTAs
+  // of one slab merge into different L2 lines
+  const int j = static_cast<int>((threadIdx.x + blockIdx.y * 37u) % (kChunk * 32));
   float v = red[0][j];
 #pragma unroll
   for (int w = 1; w < 8; ++w) v = fmaxf(v, red[w][j]);
