@@ -357,6 +357,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   const int64_t polls = prm.wait_polls;
   int64_t producer_issued = 0;  // TMA stage loads issued (warp 0)
+  // the stream-K fix-up kernel (launched as a programmatic dependent) may be
+  // scheduled now; it waits for this grid's completion before reading
+  if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -856,6 +859,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 constexpr int kFixQ = 8;  // tokens per fix-up block
 
 __global__ void __launch_bounds__(BM) streamk_fixup_kernel(const Params prm, int G) {
+  // launched as a programmatic dependent of the main kernel: everything that
+  // grid wrote is visible once this returns
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int c = static_cast<int>(blockIdx.x) + 1;
   const int64_t kbt = prm.k_blocks;
   const int64_t b = static_cast<int64_t>(c) * prm.sk_iters / G;
@@ -1153,7 +1159,18 @@ cudaError_t launch_gemm(const GemmPlan& plan, const int8_t* Xq, const int8_t* Wq
     if (plan.workspace_bytes == 0 || plan.grid < 2) return cudaSuccess;
     const dim3 fgrid(static_cast<unsigned>(plan.grid - 1),
                      static_cast<unsigned>((prm.Q + kFixQ - 1) / kFixQ));
-    streamk_fixup_kernel<<<fgrid, BM, 0, st>>>(prm, plan.grid);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = fgrid;
+    cfg.blockDim = dim3(BM);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t fe = cudaLaunchKernelEx(&cfg, streamk_fixup_kernel, prm, plan.grid);
+    if (fe != cudaSuccess) return fe;
     return cudaGetLastError();
   }
   if (plan.splits <= 1) return e;
