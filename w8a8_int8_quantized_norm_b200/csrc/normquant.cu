@@ -477,9 +477,8 @@ __global__ void __launch_bounds__(PipeBounds<CH, kMode>::kMaxThreads,
     // merge into the running maximum.  The CTA's column maxima go to shared
     // memory first (the row ring is idle now: it holds K floats) and are
     // merged in an order rotated by CTA, so concurrent CTAs hit different L2
-    // lines instead of queueing on the same ones; an atomic only where this
-    // CTA's value is larger than what act_max already holds (the maximum only
-    // grows, so a stale read costs an extra atomic, never a lost update).
+    // lines instead of queueing on the same ones.  The atomics return nothing
+    // (reductions the L2 performs): no thread waits on a global round trip.
     unsigned int* colmax = reinterpret_cast<unsigned int*>(smem);
     __syncthreads();  // every thread is done with the row buffers
 #pragma unroll
@@ -495,11 +494,12 @@ __global__ void __launch_bounds__(PipeBounds<CH, kMode>::kMaxThreads,
     __syncthreads();
     unsigned int* am_bits = reinterpret_cast<unsigned int*>(act_max);
     const int rot = static_cast<int>((blockIdx.x * 613u) % static_cast<unsigned>(K));
+#pragma unroll 4
     for (int i = t; i < K; i += T) {
       int j = i + rot;
       if (j >= K) j -= K;
       const unsigned int a = colmax[j];
-      if (a > __ldcg(am_bits + j)) atomicMax(am_bits + j, a);
+      if (a != 0u) atomicMax(am_bits + j, a);
     }
   }
 }
