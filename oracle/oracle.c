@@ -471,6 +471,9 @@ void oracle_gemm_i64(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N,
  * then converted to FP16/BF16.  Evaluation order and precision:
  *   o32 = fl32(fl32(fl32(acc) * xs[m]) * ws[n]); optional ReLU max(o32, 0);
  *   out = bf16_rne(o32).
+ * The ReLU's max orders -0 below +0 (IEEE 754-2019 maximum): a negative
+ * product that underflowed to -0 (a zero scale) becomes +0, like every other
+ * non-positive value.
  * o32_out and out_bf16 are each nullable.
  * Parity: pinned against numpy float32 arithmetic and torch's bf16 cast.
  */
@@ -482,7 +485,7 @@ void oracle_epilogue(const int64_t* acc, const float* xs, const float* ws,
       float a = (float)acc[m * N + n];
       float t = a * xs[m];
       float o = t * ws[n];
-      if (relu && o < 0.0f) o = 0.0f;
+      if (relu && !(o > 0.0f)) o = 0.0f;
       if (o32_out) o32_out[m * N + n] = o;
       if (out_bf16) out_bf16[m * N + n] = oracle_f32_to_bf16_bits(o);
     }

@@ -462,3 +462,17 @@ def test_epilogue_matches_float32_and_torch_bf16():
         assert np.array_equal(o32, ref)
         tb = torch.from_numpy(ref).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
         assert np.array_equal(out, tb)
+
+
+def test_epilogue_relu_of_negative_zero_is_positive_zero():
+    """max(o32, 0) orders -0 below +0 (IEEE 754-2019 maximum): a negative
+    accumulator times a zero token scale gives -0, which the ReLU maps to +0;
+    without the ReLU the -0 stays."""
+    acc = np.array([[-5, 0, 7]], np.int64)
+    xs = np.zeros(1, np.float32)
+    ws = np.ones(3, np.float32)
+    o32, out = oracle.epilogue(acc, xs, ws, False)
+    assert out[0, 0] == 0x8000 and out[0, 1] == 0 and out[0, 2] == 0
+    o32, out = oracle.epilogue(acc, xs, ws, True)
+    assert np.array_equal(out, np.zeros((1, 3), np.uint16))
+    assert not np.signbit(o32).any()
