@@ -215,6 +215,24 @@ sq_status sq_norm_smooth_quant_per_tensor(const void* x, sq_dtype dtype, int64_t
                                           void* stream);
 
 /*
+ * sq_quant_per_token_given_absmax -- per-token quantisation of rows whose
+ * maxima are already known (no norm): step_m = fl32(row_absmax[m] / 127),
+ * Xq[m, k] = clamp(rne(fl32(x[m, k] / step_m)), -127, 127) (0 where the step
+ * is 0).  With row_absmax[m] = max_k |x[m, k]| (sq_w8a8_gemm_dequant_rowmax)
+ * the result equals sq_norm_smooth_quant_per_token with SQ_NORM_NONE and no
+ * multiplier, bit for bit.
+ * [SQ-depth] "Granularity": per-token scales, max / 127 per row.
+ *   x          device [M, K] bf16 or fp32, row stride ldx
+ *   row_absmax device [M] fp32 IN, 16-byte aligned
+ *   Xq, x_scale as for sq_norm_smooth_quant_per_token
+ * Rows up to 40960 elements (bf16) / 25600 (fp32), else SQ_ERR_UNSUPPORTED.
+ * Errors: those of sq_norm_smooth_quant_per_token.
+ */
+sq_status sq_quant_per_token_given_absmax(const void* x, sq_dtype dtype, int64_t M, int64_t K,
+                                          int64_t ldx, const float* row_absmax, int8_t* Xq,
+                                          float* x_scale, void* stream);
+
+/*
  * sq_smooth_quantize_weights_per_tensor -- W-hat = W diag(s) quantised with
  * one step for the whole matrix, fl32(max |W-hat| / 127).
  *   w_scale  device [N] fp32 OUT: the step in every entry
@@ -289,6 +307,31 @@ sq_status sq_w8a8_gemm_dequant(const int8_t* Xq, const int8_t* Wq, const float* 
                                const float* w_scale, int64_t M, int64_t N, int64_t K,
                                sq_epilogue epi, void* out, int64_t ldo, void* workspace,
                                size_t ws_bytes, int path_hint, int split_k, void* stream);
+
+/*
+ * sq_w8a8_gemm_dequant_rowmax -- sq_w8a8_gemm_dequant on prefill tiles that
+ * also reduces, per output row, max_n |out[m, n]| over the stored bf16 values
+ * (after the ReLU for SQ_EPI_BF16_RELU).
+ * [SQ-depth] "Where the scales go in a decoder block": Linears with no norm in
+ * front (fc2, whose input is fc1's ReLU output) are still quantised with
+ * per-token scales; each token's scale needs the maximum over the whole row,
+ * which spans all of the GEMM's column tiles.  Every tile's
+ * epilogue merges its rows' maxima with an atomic max, so the following
+ * quantisation (sq_quant_per_token_given_absmax) reads each row once and needs
+ * no reduction of its own.
+ *   epi        SQ_EPI_BF16 or SQ_EPI_BF16_RELU (else SQ_ERR_INVALID_ARG)
+ *   row_absmax device [M] fp32 OUT, 16-byte aligned; zeroed by the call
+ *              (on the stream) before the GEMM runs
+ *   path_hint  0 (= 1), 1 or 3 as for sq_w8a8_gemm_dequant; 2 (decode tiles)
+ *              is SQ_ERR_INVALID_ARG
+ * Other arguments as for sq_w8a8_gemm_dequant; no workspace is used.  out is
+ * bit-identical to sq_w8a8_gemm_dequant's.
+ * Errors: those of sq_w8a8_gemm_dequant.
+ */
+sq_status sq_w8a8_gemm_dequant_rowmax(const int8_t* Xq, const int8_t* Wq, const float* x_scale,
+                                      const float* w_scale, int64_t M, int64_t N, int64_t K,
+                                      sq_epilogue epi, void* out, int64_t ldo, float* row_absmax,
+                                      int path_hint, void* stream);
 
 /*
  * sq_linear_w8a8 -- the whole runtime layer: sq_norm_smooth_quant_per_token

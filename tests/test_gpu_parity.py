@@ -333,6 +333,90 @@ def test_gemm_bf16_epilogue(shape, relu, path):
 
 
 # ---------------------------------------------------------------------------
+# fc1 -> ReLU -> fc2: row maxima reduced in the GEMM epilogue, then the
+# per-token quantisation with those maxima given
+# ---------------------------------------------------------------------------
+
+def _bf16_to_f32(bits):
+    return (bits.astype(np.uint32) << 16).view(np.float32)
+
+
+@pytest.mark.parametrize("shape", [(16, 64, 64), (129, 257, 4112), (512, 384, 256),
+                                   (300, 2304, 512), (1024, 3000, 272)],
+                         ids=lambda s: "%dx%dx%d" % s)
+@pytest.mark.parametrize("relu", [False, True])
+@pytest.mark.parametrize("path", [0, 3])
+def test_gemm_rowmax_epilogue(shape, relu, path):
+    M, N, K = shape
+    A, B = _codes(M, K), _codes(N, K)
+    xs = (RNG.random(M) * 0.05 + 1e-3).astype(np.float32)
+    ws = (RNG.random(N) * 0.002 + 1e-5).astype(np.float32)
+    xs[M // 2] = 0.0  # an all-zero output row: its max is 0
+    o32, out_o = oracle.epilogue(oracle.gemm_i64(A, B), xs, ws, relu)
+    am_o = np.abs(_bf16_to_f32(out_o)).max(axis=1)
+    am = torch.full((M,), 3e38, dtype=torch.float32, device="cuda")  # the call zeroes it
+    out_g, am_g = sq.w8a8_gemm_dequant_rowmax(to_gpu(A), to_gpu(B), to_gpu(xs), to_gpu(ws),
+                                              "bf16_relu" if relu else "bf16", row_absmax=am,
+                                              path_hint=path)
+    assert np.array_equal(bf16_bits(out_g), out_o)
+    assert np.array_equal(am_g.cpu().numpy().view(np.uint32), am_o.view(np.uint32))
+    # the plain call's output is the same
+    ref = sq.w8a8_gemm_dequant(to_gpu(A), to_gpu(B), to_gpu(xs), to_gpu(ws),
+                               "bf16_relu" if relu else "bf16", path_hint=path or 1)
+    assert torch.equal(ref, out_g)
+
+
+def test_gemm_rowmax_rejects_other_epilogues_and_decode_tiles():
+    A, B = to_gpu(_codes(8, 64)), to_gpu(_codes(32, 64))
+    xs, ws = torch.ones(8, device="cuda"), torch.ones(32, device="cuda")
+    with pytest.raises(sq.SQError) as e:
+        sq.w8a8_gemm_dequant_rowmax(A, B, xs, ws, "i32",
+                                    out=torch.empty((8, 32), dtype=torch.bfloat16, device="cuda"))
+    assert e.value.status == 1  # SQ_ERR_INVALID_ARG
+    with pytest.raises(sq.SQError) as e:
+        sq.w8a8_gemm_dequant_rowmax(A, B, xs, ws, "bf16", path_hint=2)
+    assert e.value.status == 1  # SQ_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("shape", [(1, 16), (17, 4096), (300, 4112), (64, 9216), (40, 36864),
+                                   (5, 28672)], ids=lambda s: "%dx%d" % s)
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_quant_given_absmax_equals_per_token(shape, dtype):
+    M, K = shape
+    if dtype == "f32" and K > 25600:
+        pytest.skip("fp32 rows above 25600 elements are unsupported")
+    x = _acts(M, K, dtype)
+    if M > 2:
+        x[1] = 0  # a zero row: step 0, codes 0
+    y, _, _ = oracle.norm(x, oracle.NORM_NONE)
+    am = np.abs(y).max(axis=1).astype(np.float32)
+    Xq_o, xs_o = oracle.norm_quant(x, oracle.NORM_NONE)
+    Xq_g, xs_g = sq.quant_per_token_given_absmax(to_gpu(x), to_gpu(am))
+    assert np.array_equal(xs_g.cpu().numpy().view(np.uint32), xs_o.view(np.uint32))
+    assert np.array_equal(Xq_g.cpu().numpy(), Xq_o)
+
+
+def test_quant_given_absmax_below_the_row_max_saturates():
+    M, K = 33, 4096
+    x = _acts(M, K, "bf16")
+    y, _, _ = oracle.norm(x, oracle.NORM_NONE)
+    am = (np.abs(y).max(axis=1) * np.float32(0.3)).astype(np.float32)
+    Xq_g, xs_g = sq.quant_per_token_given_absmax(to_gpu(x), to_gpu(am))
+    for m in range(M):
+        step = oracle.step_of(am[m])
+        assert xs_g[m].item() == step
+        Xq_o = oracle.quantize_with_step(y[m:m + 1], step)
+        assert np.count_nonzero(np.abs(Xq_o) == 127) > 0
+        assert np.array_equal(Xq_g[m:m + 1].cpu().numpy(), Xq_o), m
+
+
+def test_workload_opt66b_uses_the_rowmax_epilogue():
+    blk = pipeline.Block(S.OPT66B_MLP, 256, "cuda")
+    assert set(blk.rowmax) == {"fc1"}
+    assert pipeline.Block(S.OPT66B_MLP, 64, "cuda").rowmax == {}  # decode tiles: no fusion
+
+
+# ---------------------------------------------------------------------------
 # whole workloads
 # ---------------------------------------------------------------------------
 

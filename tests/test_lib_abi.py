@@ -138,3 +138,39 @@ def test_gemm_rejects_bad_arguments(L):
 def test_workspace_size_is_host_only_for_empty_shapes(L):
     assert L.sq_w8a8_gemm_workspace_size(0, 10, 64, 0) == 0
     assert L.sq_w8a8_gemm_workspace_size(10, 10, 64, -1) == 0
+
+
+def test_rowmax_gemm_rejects_bad_arguments(L):
+    f = L.sq_w8a8_gemm_dequant_rowmax
+
+    def call(Xq=A16, Wq=A16, xs=A16, ws=A16, M=16, N=64, K=64, epi=0, out=A16, ldo=64,
+             am=A16, path=0):
+        return f(Xq, Wq, xs, ws, M, N, K, epi, out, ldo, am, path, None)
+
+    assert call(epi=2) == 1             # the INT32 epilogue has no output values to reduce
+    assert call(epi=5) == 1
+    assert call(path=2) == 1            # decode tiles: not supported here
+    assert call(path=4) == 1
+    assert call(am=None) == 1
+    assert call(am=A8) == 3
+    assert call(K=40) == 3
+    assert call(M=-1) == 1
+    assert call(M=0, Xq=None, xs=None, out=None, am=None) == 0
+
+
+def test_given_absmax_quant_rejects_bad_arguments(L):
+    f = L.sq_quant_per_token_given_absmax
+
+    def call(x=A16, dt=1, M=4, K=64, ld=64, am=A16, q=A16, s=A16):
+        return f(x, dt, M, K, ld, am, q, s, None)
+
+    assert call(x=None) == 1
+    assert call(dt=7) == 1
+    assert call(ld=32) == 1
+    assert call(am=None) == 1
+    assert call(q=None) == 1
+    assert call(s=None) == 1
+    assert call(am=A8) == 3
+    assert call(K=60) == 3              # int8 rows: K % 16
+    assert call(K=48000, ld=48000) == 2  # longer rows than one CTA holds
+    assert call(M=0, am=None, q=None, s=None) == 0

@@ -263,6 +263,24 @@ sq_status sq_norm_smooth_quant_per_tensor(const void* x, sq_dtype dtype, int64_t
                                            err, as_stream(stream)));
 }
 
+sq_status sq_quant_per_token_given_absmax(const void* x, sq_dtype dtype, int64_t M, int64_t K,
+                                          int64_t ldx, const float* row_absmax, int8_t* Xq,
+                                          float* x_scale, void* stream) {
+  sq_status st = check_tensor_rows(x, dtype, M, K, ldx, SQ_NORM_NONE, nullptr, nullptr, 0.0f);
+  if (st != SQ_OK) return st;
+  if (M > 0) {
+    if (!Xq) return SQ_ERR_INVALID_ARG;
+    if (!aligned16(Xq)) return SQ_ERR_ALIGNMENT;
+    if ((st = check_vec(x_scale, true)) != SQ_OK) return st;
+    if ((st = check_vec(row_absmax, true)) != SQ_OK) return st;
+  }
+  if (M == 0) return SQ_OK;
+  int* err = device_error_word();
+  if (!err) return SQ_ERR_CUDA;
+  return from_cuda(launch_quant_given_pipe(x, dtype == SQ_BF16, M, static_cast<int>(K), ldx,
+                                           row_absmax, Xq, x_scale, err, as_stream(stream)));
+}
+
 sq_status sq_smooth_quantize_weights_per_tensor(const void* W, sq_dtype dtype, int64_t N,
                                                 int64_t K, int64_t ldw, const float* s,
                                                 int8_t* Wq, float* w_scale, float* w_absmax,
@@ -345,6 +363,28 @@ sq_status sq_w8a8_gemm_dequant(const int8_t* Xq, const int8_t* Wq, const float* 
   if (!err) return SQ_ERR_CUDA;
   return from_cuda(launch_gemm(plan, Xq, Wq, x_scale, w_scale, M, N, K, epi, out, ldo, workspace,
                                sms, g_wait_polls.load(), err, as_stream(stream)));
+}
+
+sq_status sq_w8a8_gemm_dequant_rowmax(const int8_t* Xq, const int8_t* Wq, const float* x_scale,
+                                      const float* w_scale, int64_t M, int64_t N, int64_t K,
+                                      sq_epilogue epi, void* out, int64_t ldo, float* row_absmax,
+                                      int path_hint, void* stream) {
+  if (epi != SQ_EPI_BF16 && epi != SQ_EPI_BF16_RELU) return SQ_ERR_INVALID_ARG;
+  if (path_hint == 2) return SQ_ERR_INVALID_ARG;
+  sq_status st = check_gemm(Xq, Wq, x_scale, w_scale, M, N, K, epi, out, ldo, path_hint, 1);
+  if (st != SQ_OK) return st;
+  if (M == 0) return SQ_OK;
+  if ((st = check_vec(row_absmax, true)) != SQ_OK) return st;
+  cudaStream_t cs = as_stream(stream);
+  // the running maxima start from zero (every output is >= 0 in magnitude)
+  cudaError_t e = cudaMemsetAsync(row_absmax, 0, static_cast<size_t>(M) * sizeof(float), cs);
+  if (e != cudaSuccess || N == 0) return from_cuda(e);
+  const int sms = sms_cached();
+  const GemmPlan plan = plan_gemm(M, N, K, path_hint == 0 ? 1 : path_hint, 1, sms);
+  int* err = device_error_word();
+  if (!err) return SQ_ERR_CUDA;
+  return from_cuda(launch_gemm(plan, Xq, Wq, x_scale, w_scale, M, N, K, epi, out, ldo, nullptr,
+                               sms, g_wait_polls.load(), err, cs, row_absmax));
 }
 
 sq_status sq_linear_w8a8(const void* x, sq_dtype dtype, int64_t M, int64_t K, int64_t ldx,

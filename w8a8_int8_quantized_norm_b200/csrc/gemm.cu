@@ -112,6 +112,9 @@ struct Params {
   int streamk;
   int64_t sk_iters;
   int32_t* sk_partial;
+  // prefill bf16 epilogues: running max of |out| per P row (token), as
+  // binary32 bits, for a following per-token requantisation (or null)
+  float* row_absmax;
 };
 
 // Give-up point of a pipeline wait, in SM clock cycles (about 2 s at the
@@ -210,16 +213,17 @@ __device__ __forceinline__ bool work_next(const Params& p, Work& w, int& pb, int
 
 // Epilogue for one CHUNK of accumulator columns held by this thread (row p of
 // the P side, columns q0 .. q0 + CHUNK - 1 of the Q side).
+// Returns the chunk's max |bf16 out| when prm.row_absmax asks for it (else 0).
 template <int CHUNK>
-__device__ __forceinline__ void store_chunk(const Params& prm, const uint32_t (&r)[32], int p,
-                                            int q0, int split, int slot) {
-  if (p >= prm.P) return;
+__device__ __forceinline__ float store_chunk(const Params& prm, const uint32_t (&r)[32], int p,
+                                             int q0, int split, int slot) {
+  if (p >= prm.P) return 0.0f;
   if (slot >= 0) {  // stream-K partial sums of a decode tile: [slot][Q][128]
     int32_t* dst = prm.sk_partial + static_cast<int64_t>(slot) * prm.Q * BM + (p % BM);
 #pragma unroll
     for (int j = 0; j < CHUNK; ++j)
       if (q0 + j < prm.Q) dst[static_cast<int64_t>(q0 + j) * BM] = static_cast<int32_t>(r[j]);
-    return;
+    return 0.0f;
   }
   if (prm.partial) {  // split-K partial sums, [split][M][N] with M = Q (tokens), N = P
 #pragma unroll
@@ -229,7 +233,7 @@ __device__ __forceinline__ void store_chunk(const Params& prm, const uint32_t (&
         prm.partial[(static_cast<int64_t>(split) * prm.Q + q) * prm.P + p] =
             static_cast<int32_t>(r[j]);
     }
-    return;
+    return 0.0f;
   }
   if (prm.epi == SQ_EPI_I32_RAW) {
     int32_t* o = static_cast<int32_t*>(prm.out);
@@ -249,7 +253,7 @@ __device__ __forceinline__ void store_chunk(const Params& prm, const uint32_t (&
       for (int j = 0; j < CHUNK; ++j)
         if (q0 + j < prm.Q) o[static_cast<int64_t>(q0 + j) * prm.ldo + p] = static_cast<int32_t>(r[j]);
     }
-    return;
+    return 0.0f;
   }
   const bool relu = prm.epi == SQ_EPI_BF16_RELU;
   __nv_bfloat16* o = static_cast<__nv_bfloat16*>(prm.out);
@@ -271,10 +275,13 @@ __device__ __forceinline__ void store_chunk(const Params& prm, const uint32_t (&
 #pragma unroll
     for (int j = 0; j < CHUNK; ++j) {
       float t = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(r[j])), xs), ws[j]);
-      if (relu) t = fmaxf(t, 0.0f);
+      if (relu) t = t > 0.0f ? t : 0.0f;  // -0 (a zero scale) becomes +0
       v[j] = t;
     }
     __nv_bfloat16* dst = o + static_cast<int64_t>(p) * prm.ldo + q0;
+    // max |bf16 out| of the chunk, as bf16 bits (magnitudes order like ints)
+    const bool track = prm.row_absmax != nullptr;
+    uint32_t am = 0;
     if (prm.vec_out && q0 + CHUNK <= prm.Q) {
 #pragma unroll
       for (int j = 0; j < CHUNK; j += 8) {
@@ -283,14 +290,21 @@ __device__ __forceinline__ void store_chunk(const Params& prm, const uint32_t (&
         for (int i = 0; i < 4; ++i) {
           const __nv_bfloat162 h = __floats2bfloat162_rn(v[j + 2 * i], v[j + 2 * i + 1]);
           w[i] = *reinterpret_cast<const uint32_t*>(&h);
+          if (track) am = max(am, max(w[i] & 0x7fffu, (w[i] >> 16) & 0x7fffu));
         }
         *reinterpret_cast<uint4*>(dst + j) = make_uint4(w[0], w[1], w[2], w[3]);
       }
     } else {
 #pragma unroll
       for (int j = 0; j < CHUNK; ++j)
-        if (q0 + j < prm.Q) dst[j] = __float2bfloat16_rn(v[j]);
+        if (q0 + j < prm.Q) {
+          const __nv_bfloat16 h = __float2bfloat16_rn(v[j]);
+          dst[j] = h;
+          if (track)
+            am = max(am, static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(&h)) & 0x7fffu);
+        }
     }
+    return __uint_as_float(am << 16);
   } else {
     // channel scale for this row (weight row p), token scale per column
     const float ws = __ldg(prm.p_scale + p);
@@ -300,11 +314,12 @@ __device__ __forceinline__ void store_chunk(const Params& prm, const uint32_t (&
       if (q < prm.Q) {
         const float xs = __ldg(prm.q_scale + q);
         float t = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(r[j])), xs), ws);
-        if (relu) t = fmaxf(t, 0.0f);
+        if (relu) t = t > 0.0f ? t : 0.0f;  // -0 (a zero scale) becomes +0
         o[static_cast<int64_t>(q) * prm.ldo + p] = __float2bfloat16_rn(t);
       }
     }
   }
+  return 0.0f;
 }
 
 template <int BN>
@@ -501,6 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const int p = pb * BM + quarter * 32 + lane;
+      float rmax = 0.0f;
 #pragma unroll 1
       for (int c = 0; c < BN / C::CHUNK; ++c) {
         uint32_t r[32];
@@ -512,8 +528,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         else
           tmem_ld_32x32b_x16(taddr, r);
         tmem_wait_ld();
-        store_chunk<C::CHUNK>(prm, r, p, qb * BN + c * C::CHUNK, split, slot);
+        rmax = fmaxf(rmax, store_chunk<C::CHUNK>(prm, r, p, qb * BN + c * C::CHUNK, split, slot));
       }
+      if (prm.row_absmax && rmax > 0.0f && p < prm.P)
+        atomicMax(reinterpret_cast<unsigned int*>(prm.row_absmax) + p, __float_as_uint(rmax));
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(TEMPTY_BAR(acc));
@@ -798,6 +816,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const int p = pb * TILE_M + static_cast<int>(rank) * ROWS + quarter * 32 + lane;
+      float rmax = 0.0f;
 #pragma unroll 1
       for (int c = 0; c < TN / 32; ++c) {
         uint32_t r[32];
@@ -806,8 +825,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                                static_cast<uint32_t>(acc * TN + c * 32);
         tmem_ld_32x32b_x32(taddr, r);
         tmem_wait_ld();
-        store_chunk<32>(prm, r, p, qb * TN + c * 32, 0, -1);
+        rmax = fmaxf(rmax, store_chunk<32>(prm, r, p, qb * TN + c * 32, 0, -1));
       }
+      if (prm.row_absmax && rmax > 0.0f && p < prm.P)
+        atomicMax(reinterpret_cast<unsigned int*>(prm.row_absmax) + p, __float_as_uint(rmax));
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -1097,7 +1118,8 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int path_hint, int split_k, 
 cudaError_t launch_gemm(const GemmPlan& plan, const int8_t* Xq, const int8_t* Wq,
                         const float* x_scale, const float* w_scale, int64_t M, int64_t N,
                         int64_t K, int epi, void* out, int64_t ldo, void* workspace, int num_sms,
-                        int64_t wait_polls, int* error_word, cudaStream_t st) {
+                        int64_t wait_polls, int* error_word, cudaStream_t st,
+                        float* row_absmax) {
   if (M == 0 || N == 0) return cudaSuccess;
   Params prm{};
   const int8_t* Pptr = plan.swap ? Wq : Xq;
@@ -1122,6 +1144,8 @@ cudaError_t launch_gemm(const GemmPlan& plan, const int8_t* Xq, const int8_t* Wq
   prm.streamk = plan.streamk;
   prm.sk_iters = plan.sk_iters;
   prm.sk_partial = plan.streamk ? static_cast<int32_t*>(workspace) : nullptr;
+  if (row_absmax && (plan.swap || epi == SQ_EPI_I32_RAW)) return cudaErrorInvalidValue;
+  prm.row_absmax = row_absmax;
   prm.wait_polls = wait_polls;
   prm.error_word = error_word;
   {

@@ -177,6 +177,7 @@ enum RowMode : int {
   kModeColMax = 1,      // calibration: running per-column max of |y|
   kModeTensorMax = 2,   // one running max of |y| over the whole tensor
   kModeFixedQuant = 3,  // codes with one given step (per-tensor: O2 / O3)
+  kModeGivenQuant = 4,  // per-row codes, each row's max |y| given in act_max[row]
 };
 
 template <int CH, int kMode>
@@ -197,7 +198,8 @@ struct PipeBounds {
 // fold C into B.  Calibration keeps a per-thread running max of |y| over the
 // rows it sees, merged into act_max[K] at the end; the tensor-max mode keeps
 // the CTA's running max of the row maxima and merges it into act_max[0]; the
-// fixed-step mode reads its step's max |y| from act_max[0] once.
+// fixed-step mode reads its step's max |y| from act_max[0] once; the given-max
+// mode reads row i's from act_max[i] (a producer already reduced it).
 //
 // kFull: every thread owns all CH of its chunks (T * CH == K / 8): no bounds checks.
 template <bool kBF16, int NORMK, int CH, bool kGamma, bool kBeta, bool kFull, int kMode>
@@ -267,6 +269,12 @@ __global__ void __launch_bounds__(PipeBounds<CH, kMode>::kMaxThreads,
     fexact = fstep < FLT_MIN;
     frstep = fexact ? 0.0f : __frcp_rn(fstep);
   }
+  // given-max mode: row i's max is loaded one row ahead (its global-load
+  // latency hides behind the previous row's work)
+  float gmax_next = 0.0f;
+  if constexpr (kMode == kModeGivenQuant) {
+    if (first < M) gmax_next = __ldg(act_max + first);
+  }
   float2 cm[kCalib ? CH : 1][4];  // calibration: running max of |y| per owned element
   if constexpr (kCalib) {
 #pragma unroll
@@ -285,6 +293,11 @@ __global__ void __launch_bounds__(PipeBounds<CH, kMode>::kMaxThreads,
                par_next ^= (nbuf_next + 1 == nbuf) ? 1u : 0u,
                nbuf_next = (nbuf_next + 1 == nbuf) ? 0 : nbuf_next + 1) {
     const uint8_t* rowp = smem + buf * buf_stride;
+    float gmax = 0.0f;
+    if constexpr (kMode == kModeGivenQuant) {
+      gmax = gmax_next;
+      if (row + G < M) gmax_next = __ldg(act_max + row + G);
+    }
 
     // ---- this thread's chunks of the row, from shared memory
     float2 v[CH][4];
@@ -406,15 +419,23 @@ __global__ void __launch_bounds__(PipeBounds<CH, kMode>::kMaxThreads,
         }
       }
     }
-    if constexpr (kMode == kModeFixedQuant) {
-      if (t == 0) scale[row] = fstep;
+    if constexpr (kMode == kModeFixedQuant || kMode == kModeGivenQuant) {
+      float step = fstep, rstep = frstep;
+      bool exact_only = fexact;
+      if constexpr (kMode == kModeGivenQuant) {
+        step = div127(gmax);
+        exact_only = step < FLT_MIN;
+        rstep = exact_only ? 0.0f : __frcp_rn(step);
+      }
+      if (t == 0) scale[row] = step;
       int8_t* qrow = q + row * static_cast<int64_t>(K);
 #pragma unroll
       for (int c = 0; c < CH; ++c) {
         const int ch = t + c * T;
         if (!kFull && ch >= nchunks) continue;
+        // clamped: a given max below the row's true max saturates at +-127
         *reinterpret_cast<uint2*>(qrow + ch * kChunk) =
-            codes8<true>(v[c], frstep, fstep, fexact);
+            codes8<true>(v[c], rstep, step, exact_only);
       }
     }
     if constexpr (kRowMax) {
@@ -668,6 +689,18 @@ cudaError_t launch_quant_fixed_pipe(const void* x, bool bf16, int64_t M, int K, 
   if (M == 0) return cudaSuccess;
   const RowArgs a{x, M, K, ldx, gamma, beta, eps, q, scale, const_cast<float*>(absmax), err};
   return launch_rows<kModeFixedQuant>(a, bf16, norm, st);
+}
+
+cudaError_t launch_quant_given_pipe(const void* x, bool bf16, int64_t M, int K, int64_t ldx,
+                                    const float* row_absmax, int8_t* q, float* scale, int* err,
+                                    cudaStream_t st) {
+  if (M == 0) return cudaSuccess;
+  PipeShape ps;
+  if (!pipe_shape(K, bf16, false, &ps)) return cudaErrorInvalidValue;
+  const RowArgs a{x, M, K, ldx, nullptr, nullptr, 0.0f, q, scale,
+                  const_cast<float*>(row_absmax), err};
+  if (bf16) return launch_pipe_n<true, 0, kModeGivenQuant>(a, ps, st);
+  return launch_pipe_n<false, 0, kModeGivenQuant>(a, ps, st);
 }
 
 }  // namespace sq

@@ -92,6 +92,11 @@ cudaError_t launch_quant_fixed_pipe(const void* x, bool bf16, int64_t M, int K, 
                                     int norm, const float* gamma, const float* beta, float eps,
                                     const float* absmax, int8_t* q, float* scale, int* err,
                                     cudaStream_t st);
+// Per-row codes from given row maxima (no norm): row i's step is
+// fl32(row_absmax[i] / 127); codes clamp to +-127.
+cudaError_t launch_quant_given_pipe(const void* x, bool bf16, int64_t M, int K, int64_t ldx,
+                                    const float* row_absmax, int8_t* q, float* scale, int* err,
+                                    cudaStream_t st);
 cudaError_t launch_calibrate(const void* x, bool bf16, int64_t M, int K, int64_t ldx, int norm,
                              const float* gamma, const float* beta, float eps, float* act_max,
                              int* err, cudaStream_t st);
@@ -116,7 +121,8 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int path_hint, int split_k, 
 cudaError_t launch_gemm(const GemmPlan& plan, const int8_t* Xq, const int8_t* Wq,
                         const float* x_scale, const float* w_scale, int64_t M, int64_t N,
                         int64_t K, int epi, void* out, int64_t ldo, void* workspace,
-                        int num_sms, int64_t wait_polls, int* error_word, cudaStream_t st);
+                        int num_sms, int64_t wait_polls, int* error_word, cudaStream_t st,
+                        float* row_absmax = nullptr);
 int num_sms_current_device();
 
 }  // namespace sq

@@ -5,6 +5,8 @@
     python -m w8a8_int8_quantized_norm_b200.kbench calibrate --M 4096 --K 8192 --norm layer
     python -m w8a8_int8_quantized_norm_b200.kbench weight_quant --N 28672 --K 8192
     python -m w8a8_int8_quantized_norm_b200.kbench smooth_scales --N 12288 --K 4096
+    python -m w8a8_int8_quantized_norm_b200.kbench quant_given --M 4096 --K 36864
+    python -m w8a8_int8_quantized_norm_b200.kbench gemm --M 4096 --N 36864 --K 9216 --rowmax
 
 Each call is captured once as a CUDA graph; every timed replay is bracketed by
 CUDA events on the launching stream, with L2 emptied before it (256 MiB
@@ -100,7 +102,7 @@ def _time(fn, iters, warmup, flush):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("op", choices=["norm_quant", "gemm", "calibrate", "weight_quant",
-                                   "smooth_scales"])
+                                   "smooth_scales", "quant_given"])
     ap.add_argument("--M", type=int, default=4096)
     ap.add_argument("--N", type=int, default=4096)
     ap.add_argument("--K", type=int, default=4096)
@@ -109,6 +111,8 @@ def main(argv=None):
     ap.add_argument("--path", type=int, default=0, help="GEMM path hint (0 = auto)")
     ap.add_argument("--split", type=int, default=0, help="GEMM split-K (0 = auto)")
     ap.add_argument("--epi", choices=["bf16", "bf16_relu", "i32"], default="bf16")
+    ap.add_argument("--rowmax", action="store_true",
+                    help="GEMM: also reduce each output row's max |out| (prefill tiles)")
     ap.add_argument("--iters", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--seed", type=int, default=0)
@@ -135,6 +139,14 @@ def main(argv=None):
         fn = lambda: sq.norm_smooth_quant_per_token(x, norm, g, b, 1e-5, xq, xs)
         units = M * K * (esz + 1) + 4 * M + 4 * K * ((g is not None) + (b is not None))
         shape = {"M": M, "K": K, "norm": a.norm, "dtype": a.dtype}
+    elif a.op == "quant_given":
+        x = _acts(M, K, a.dtype, gen, dev)
+        am = x.float().abs().amax(dim=1).contiguous()
+        xq = torch.empty((M, K), dtype=torch.int8, device=dev)
+        xs = torch.empty(M, dtype=torch.float32, device=dev)
+        fn = lambda: sq.quant_per_token_given_absmax(x, am, xq, xs)
+        units = M * K * (esz + 1) + 8 * M
+        shape = {"M": M, "K": K, "dtype": a.dtype}
     elif a.op == "calibrate":
         x = _acts(M, K, a.dtype, gen, dev)
         g = torch.empty(K, device=dev).uniform_(0.5, 1.5, generator=gen) if norm else None
@@ -174,7 +186,12 @@ def main(argv=None):
         scales = (None, None) if a.epi == "i32" else (xs, wsc)
         fn = lambda: sq.w8a8_gemm_dequant(A, B, scales[0], scales[1], a.epi, out=out,
                                           path_hint=a.path, split_k=a.split, workspace=ws)
-        shape = {"M": M, "N": N, "K": K, "path": a.path, "split": a.split, "epi": a.epi}
+        if a.rowmax:
+            rm = torch.empty(M, dtype=torch.float32, device=dev)
+            fn = lambda: sq.w8a8_gemm_dequant_rowmax(A, B, xs, wsc, a.epi, out=out,
+                                                     row_absmax=rm, path_hint=a.path)
+        shape = {"M": M, "N": N, "K": K, "path": a.path, "split": a.split, "epi": a.epi,
+                 "rowmax": a.rowmax}
         units = None
     us = _time(fn, a.iters, a.warmup, flush)
     err = sq.get_device_error()

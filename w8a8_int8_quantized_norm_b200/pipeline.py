@@ -98,6 +98,20 @@ class Block:
                                       and site.calibrated)
         self.w_absmax: Dict[str, torch.Tensor] = {l.name: torch.zeros(1, **f32)
                                                   for l in w.linears}
+        # A Linear whose bf16 output is the whole input of a later per-token
+        # site (no norm, no multiplier: fc1 -> ReLU -> fc2) reduces each
+        # output row's max |out| in its GEMM epilogue, so that site's
+        # quantisation reads the row once with its max already known.  Only
+        # on prefill tiles (the decode plan keeps its own tiles).
+        self.rowmax: Dict[str, torch.Tensor] = {}  # source Linear -> [M] row maxima
+        if granularity == "per_token":
+            for lin in w.linears:
+                site = w.site(lin.site)
+                if lin.source and site.norm == sq.NORM_NONE and not site.smoothed:
+                    src = next(l for l in w.linears if l.name == lin.source)
+                    K_src = w.site(src.site).K
+                    if sq.gemm_plan(M, src.N, K_src).kernel != 2:
+                        self.rowmax[src.name] = torch.empty(M, **f32)
 
     # -- offline rows -------------------------------------------------------
     def prepare(self, x_cal: Dict[str, torch.Tensor], W: Dict[str, torch.Tensor],
@@ -161,7 +175,12 @@ class Block:
             nparam = (self.gamma_f[site.name] is not None) + (self.beta_f[site.name] is not None)
             units = xin.numel() * (xin.element_size() + 1) + 4 * self.M + 4 * site.K * nparam
             gf, bf = self.gamma_f[site.name], self.beta_f[site.name]
-            if self.granularity == "per_token":
+            if src in self.rowmax:
+                am = self.rowmax[src]
+                _run(timer, "norm_quant", units,
+                     lambda: sq.quant_per_token_given_absmax(xin, am, self.xq[site.name],
+                                                             self.xs[site.name], stream=stream))
+            elif self.granularity == "per_token":
                 _run(timer, "norm_quant", units,
                      lambda: sq.norm_smooth_quant_per_token(xin, site.norm, gf, bf, w.eps,
                                                             self.xq[site.name],
@@ -179,6 +198,13 @@ class Block:
                                                              self.xs[site.name], stream=stream))
             for lin in w.linears_of(site.name):
                 def gemm(lin=lin, site=site):
+                    if lin.name in self.rowmax:
+                        sq.w8a8_gemm_dequant_rowmax(
+                            self.xq[site.name], self.Wq[lin.name], self.xs[site.name],
+                            self.w_scale[lin.name], "bf16_relu" if lin.relu else "bf16",
+                            out=self.out[lin.name], row_absmax=self.rowmax[lin.name],
+                            stream=stream)
+                        return
                     sq.w8a8_gemm_dequant(self.xq[site.name], self.Wq[lin.name],
                                          self.xs[site.name], self.w_scale[lin.name],
                                          "bf16_relu" if lin.relu else "bf16",
@@ -209,7 +235,10 @@ class Block:
         if self.granularity != "per_token":
             n += sum(1 for site in self.w.sites if not self.static[site.name])  # O2 max pass
         for lin in self.w.linears:
-            n += sq.gemm_plan(self.M, lin.N, self.w.site(lin.site).K).launches
+            if lin.name in self.rowmax:
+                n += 1  # prefill tiles, one kernel (the zeroing is a memset)
+            else:
+                n += sq.gemm_plan(self.M, lin.N, self.w.site(lin.site).K).launches
         return n
 
     # -- CUDA graph ----------------------------------------------------------

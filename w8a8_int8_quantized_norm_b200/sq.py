@@ -35,6 +35,7 @@ EXPORTS = (
     "sq_linear_w8a8", "sq_status_string", "sq_get_device_error", "sq_set_wait_limit",
     "sq_w8a8_gemm_dequant_noalloc", "sq_w8a8_gemm_plan", "sq_norm_smooth_absmax",
     "sq_norm_smooth_quant_per_tensor", "sq_smooth_quantize_weights_per_tensor",
+    "sq_w8a8_gemm_dequant_rowmax", "sq_quant_per_token_given_absmax",
 )
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -107,11 +108,16 @@ def _declare(L):
                                                   _P, _P, _P, _P]
     L.sq_smooth_quantize_weights_per_tensor.argtypes = [_P, _I32, _I64, _I64, _I64, _P, _P, _P,
                                                         _P, _P]
+    L.sq_w8a8_gemm_dequant_rowmax.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _I32, _P, _I64,
+                                              _P, _I32, _P]
+    L.sq_quant_per_token_given_absmax.argtypes = [_P, _I32, _I64, _I64, _I64, _P, _P, _P, _P]
     L.sq_w8a8_gemm_plan.argtypes = [_I64, _I64, _I64, _I32, _I32, ctypes.POINTER(GemmPlanInfo)]
     L.sq_set_wait_limit.argtypes = [_I64]
     L.sq_set_wait_limit.restype = None
     for name in EXPORTS:
         f = getattr(L, name)
+        if f.argtypes is None:  # every call passes 64-bit sizes: no implicit int conversion
+            raise RuntimeError("no argument types declared for %s" % name)
         if name not in ("sq_w8a8_gemm_workspace_size", "sq_status_string", "sq_set_wait_limit"):
             f.restype = _I32
 
@@ -266,6 +272,20 @@ def norm_smooth_quant_per_tensor(x: torch.Tensor, norm: int, absmax: torch.Tenso
     return Xq, x_scale
 
 
+def quant_per_token_given_absmax(x: torch.Tensor, row_absmax: torch.Tensor, Xq=None,
+                                 x_scale=None, stream=None):
+    """Per-token codes of x [M, K] with each row's max |x| given (no norm)."""
+    M, K, ld = _rows(x, "x")
+    if Xq is None:
+        Xq = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    if x_scale is None:
+        x_scale = torch.empty(M, dtype=torch.float32, device=x.device)
+    _check(lib().sq_quant_per_token_given_absmax(
+        _ptr(x), _dtype_code(x), M, K, ld, _ptr(_vec(row_absmax, M, "row_absmax")), _ptr(Xq),
+        _ptr(x_scale), _stream(stream)), "sq_quant_per_token_given_absmax")
+    return Xq, x_scale
+
+
 def smooth_quantize_weights_per_tensor(W: torch.Tensor, s: Optional[torch.Tensor] = None,
                                        Wq=None, w_scale=None, w_absmax=None, stream=None):
     N, K, ld = _rows(W, "W")
@@ -314,6 +334,27 @@ def w8a8_gemm_dequant(Xq: torch.Tensor, Wq: torch.Tensor, x_scale: Optional[torc
                                       path_hint, split_k, _stream(stream)),
            "sq_w8a8_gemm_dequant")
     return out
+
+
+def w8a8_gemm_dequant_rowmax(Xq: torch.Tensor, Wq: torch.Tensor, x_scale: torch.Tensor,
+                             w_scale: torch.Tensor, epi: str = "bf16", out=None,
+                             row_absmax=None, path_hint: int = 0, stream=None):
+    """The prefill GEMM that also returns max_n |out[m, n]| per row (bf16
+    epilogues only).  Returns (out, row_absmax)."""
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    if Xq.dtype != torch.int8 or Wq.dtype != torch.int8 or not Xq.is_contiguous() \
+            or not Wq.is_contiguous() or Wq.shape[1] != K:
+        raise ValueError("Xq [M,K] and Wq [N,K] must be contiguous int8")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=Xq.device)
+    if row_absmax is None:
+        row_absmax = torch.empty(M, dtype=torch.float32, device=Xq.device)
+    _check(lib().sq_w8a8_gemm_dequant_rowmax(
+        _ptr(Xq), _ptr(Wq), _ptr(x_scale), _ptr(w_scale), M, N, K, EPI[epi], _ptr(out),
+        out.stride(0), _ptr(_vec(row_absmax, M, "row_absmax")), path_hint, _stream(stream)),
+        "sq_w8a8_gemm_dequant_rowmax")
+    return out, row_absmax
 
 
 def w8a8_gemm_dequant_noalloc(Xq: torch.Tensor, Wq: torch.Tensor,
