@@ -90,6 +90,10 @@ def _declare(L):
     L.oracle_step_of.argtypes = [ctypes.c_float]
     L.oracle_quantize_with_step.restype = None
     L.oracle_quantize_with_step.argtypes = [_P, _I64, _I64, ctypes.c_float, _P]
+    L.oracle_exp_cw.restype = None
+    L.oracle_exp_cw.argtypes = [_P, _I64, _P]
+    L.oracle_silu_mul.restype = None
+    L.oracle_silu_mul.argtypes = [_P, ctypes.c_int, _I64, _I64, _I64, _P, _P]
     L.oracle_num_threads.restype = ctypes.c_int
     L.oracle_num_threads.argtypes = []
 
@@ -296,6 +300,38 @@ def f32_to_bf16_bits(x) -> np.ndarray:
     x = np.asarray(x, dtype=np.float32)
     f = lib().oracle_f32_to_bf16_bits
     return np.array([f(float(v)) for v in x.ravel()], dtype=np.uint16).reshape(x.shape)
+
+
+def exp_cw(t) -> np.ndarray:
+    """e^t by Cody-Waite reduction and a degree-7 Taylor polynomial in fp32
+    (the exponential of the SiLU step; see oracle.c)."""
+    t = np.ascontiguousarray(t, dtype=np.float32)
+    out = np.empty_like(t)
+    lib().oracle_exp_cw(_ptr(t), t.size, _ptr(out))
+    return out
+
+
+def silu_mul(gu):
+    """The down projection's input from gate_up's output [M, 2I] (gate in the
+    first I columns, up in the last I): h = SiLU(gate) * up in fp32, and h
+    rounded to bf16.  Returns (h32 fp32 [M, I], h bf16 bits uint16 [M, I])."""
+    gu = np.ascontiguousarray(gu)
+    M, K2 = gu.shape
+    if K2 % 2:
+        raise ValueError("gate_up rows hold two halves")
+    I = K2 // 2
+    h32 = np.empty((M, I), np.float32)
+    hb = np.empty((M, I), np.uint16)
+    lib().oracle_silu_mul(_ptr(gu), _dtype_code(gu), M, I, K2, _ptr(h32), _ptr(hb))
+    return h32, hb
+
+
+def silu_mul_quant(gu):
+    """SiLU(gate) * up stored as bf16, then per-token quantised (steps 5 on
+    h, no norm).  Returns (Xq int8 [M, I], x_scale fp32 [M], h bf16 bits)."""
+    _, hb = silu_mul(gu)
+    Xq, xs = norm_quant(hb, NORM_NONE)
+    return Xq, xs, hb
 
 
 def linear(x, norm_kind, gamma_f, beta_f, eps, Wq, w_scale, relu=False):

@@ -491,6 +491,88 @@ void oracle_epilogue(const int64_t* acc, const float* xs, const float* ws,
     }
 }
 
+/* ------------------------------------------------------------------------ */
+/* The down projection's input: SiLU(gate) * up                              */
+/* ------------------------------------------------------------------------ */
+/*
+ * [SQ-depth] "Where the scales go in a decoder block": the down_proj input is
+ * SiLU(gate) times up; it has no norm in front, is not smoothed and is
+ * quantised with per-token scales.  The pages give neither the SiLU formula's
+ * precision nor the layout of the merged gate/up projection.  Readings:
+ *   - gate_up's output row holds gate in columns [0, I) and up in [I, 2I);
+ *   - silu(g) = g * sigma(g), sigma(g) = 1 / (1 + e^-g), in fp32;
+ *   - h = fl32(fl32(g * fl32(1 / fl32(1 + e))) * u), e = exp_cw(-g) below,
+ *     and h is stored in the model dtype (bf16, round to nearest even) before
+ *     it is quantised, as an unfused model would write it.
+ *
+ * exp_cw: e^t in fp32 by Cody and Waite's argument reduction (W. J. Cody and
+ * W. Waite, "Software Manual for the Elementary Functions", 1980) followed by
+ * the degree-7 Taylor polynomial of e^r, so that the result is a fixed
+ * sequence of IEEE operations that any implementation can repeat bit for bit:
+ *   t is first clamped to [-87, 87] (beyond that sigma is 0 or 1 to far below
+ *   an fp32 ulp of silu, and 2^n below stays a normal number);
+ *   n = rint(fl32(t * L2E)), L2E = fl32(1 / ln 2);
+ *   r = fma(-n, LN2_HI, t), then r = fma(-n, LN2_LO, r), where LN2_HI is ln 2
+ *       cut to 16 significant bits (n * LN2_HI is exact for |n| < 2^8) and
+ *       LN2_LO = fl32(ln 2 - LN2_HI);
+ *   p = 1/7!, then p = fma(p, r, 1/k!) for k = 6 .. 0 (coefficients fl32);
+ *   e^t = fl32(p * 2^n), 2^n exact.
+ * |r| <= about ln2 / 2, so the truncation term is below 1e-8 relative; the
+ * rounding of the Horner steps adds a few fp32 ulps.
+ * Parity: pinned against float64 exp (relative error bound), and SiLU * up
+ * against the float64 formula (within one bf16 ulp of the exact value).
+ */
+#define CW_L2E 1.44269504088896340736f
+#define CW_LN2_HI 0.693145751953125f      /* 45426 / 65536 */
+#define CW_LN2_LO 1.428606765330187e-06f  /* ln 2 - LN2_HI, rounded to fp32 */
+
+static float exp_cw(float t) {
+  if (t > 87.0f) t = 87.0f;
+  if (t < -87.0f) t = -87.0f;
+  const float n = rintf(t * CW_L2E);
+  float r = fmaf(-n, CW_LN2_HI, t);
+  r = fmaf(-n, CW_LN2_LO, r);
+  float p = 1.0f / 5040.0f;
+  p = fmaf(p, r, 1.0f / 720.0f);
+  p = fmaf(p, r, 1.0f / 120.0f);
+  p = fmaf(p, r, 1.0f / 24.0f);
+  p = fmaf(p, r, 1.0f / 6.0f);
+  p = fmaf(p, r, 0.5f);
+  p = fmaf(p, r, 1.0f);
+  p = fmaf(p, r, 1.0f);
+  const uint32_t bits = (uint32_t)((int32_t)n + 127) << 23; /* 2^n, n in [-126, 126] */
+  float two_n;
+  memcpy(&two_n, &bits, sizeof two_n);
+  return p * two_n;
+}
+
+void oracle_exp_cw(const float* t, int64_t n, float* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = exp_cw(t[i]);
+}
+
+/* One element of the down projection's input, before the bf16 store. */
+static float silu_mul_one(float g, float u) {
+  const float e = exp_cw(-g);
+  const float sigma = 1.0f / (1.0f + e);
+  const float silu = g * sigma;
+  return silu * u;
+}
+
+/* gu: [M, 2I] (row stride ld) bf16 or fp32; h32 [M, I] fp32 and h_bf16
+ * [M, I] bf16 bits, each nullable. */
+void oracle_silu_mul(const void* gu, int dtype, int64_t M, int64_t I, int64_t ld, float* h32,
+                     uint16_t* h_bf16) {
+#pragma omp parallel for schedule(static)
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t j = 0; j < I; ++j) {
+      const float g = load_elem(gu, dtype, m * ld + j);
+      const float u = load_elem(gu, dtype, m * ld + I + j);
+      const float h = silu_mul_one(g, u);
+      if (h32) h32[m * I + j] = h;
+      if (h_bf16) h_bf16[m * I + j] = oracle_f32_to_bf16_bits(h);
+    }
+}
+
 /* Thread count the OpenMP loops will use (for the CPU-baseline report). */
 int oracle_num_threads(void) {
 #ifdef _OPENMP

@@ -476,3 +476,76 @@ def test_epilogue_relu_of_negative_zero_is_positive_zero():
     o32, out = oracle.epilogue(acc, xs, ws, True)
     assert np.array_equal(out, np.zeros((1, 3), np.uint16))
     assert not np.signbit(o32).any()
+
+
+# ---------------------------------------------------------------------------
+# SiLU(gate) * up: the down projection's input
+# ---------------------------------------------------------------------------
+
+def test_exp_cw_within_a_few_ulps_of_float64_exp():
+    t = np.concatenate([np.linspace(-87, 87, 400001, dtype=np.float32),
+                        np.float32([0.0, -0.0, 1e-30, -1e-30, 0.5, -0.5, 1.0, -1.0, 86.99, -86.99]),
+                        (np.arange(-125, 126) * np.log(2)).astype(np.float32)])
+    e = oracle.exp_cw(t)
+    ref = np.exp(t.astype(np.float64))
+    rel = np.abs(e.astype(np.float64) / ref - 1.0)
+    assert rel.max() < 4 * 2.0 ** -23, rel.max()
+    assert oracle.exp_cw(np.float32([0.0]))[0] == np.float32(1.0)
+    # the argument is clamped to [-87, 87]
+    big = oracle.exp_cw(np.float32([87.0, 100.0, 1e30, -87.0, -100.0, -1e30]))
+    assert big[0] == big[1] == big[2] and big[3] == big[4] == big[5]
+    assert np.isfinite(big).all() and (big > 0).all()
+
+
+def _gu(M, I, g_scale=3.0, seed=5):
+    r = np.random.default_rng(seed)
+    g = (r.standard_normal((M, I)) * g_scale).astype(np.float32)
+    u = r.standard_normal((M, I)).astype(np.float32)
+    return S.to_bf16_bits(np.concatenate([g, u], axis=1))
+
+
+def test_silu_mul_against_the_float64_formula():
+    M, I = 7, 4096
+    gu = _gu(M, I)
+    gf = (gu.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    g, u = gf[:, :I], gf[:, I:]
+    exact = g * u / (1.0 + np.exp(-g))
+    h32, hb = oracle.silu_mul(gu)
+    nz = exact != 0
+    rel = np.abs(h32[nz] / exact[nz] - 1.0)
+    assert rel.max() < 8 * 2.0 ** -23, rel.max()
+    # bf16 h within one bf16 ulp of the exact value (RNE of a nearly exact fp32)
+    hv = (hb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    ulp = np.exp2(np.floor(np.log2(np.abs(exact[nz]))) - 7)
+    assert np.all(np.abs(hv[nz] - exact[nz]) <= ulp)
+    assert np.array_equal(hb, oracle.f32_to_bf16_bits(h32))
+    # gate is the first half: swapping the halves changes the result
+    swapped = np.concatenate([gu[:, I:], gu[:, :I]], axis=1)
+    assert not np.array_equal(oracle.silu_mul(swapped)[1], hb)
+
+
+def test_silu_mul_special_values():
+    g = np.float32([0.0, 0.0, 80.0, 200.0, -80.0, -200.0, 1.0, -1.0])
+    u = np.float32([1.0, -3.0, 1.5, 1.0, 1.0, 7.0, 0.0, 2.0])
+    gu = S.to_bf16_bits(np.concatenate([g, u])[None, :])
+    h32, hb = oracle.silu_mul(gu)
+    h32 = h32[0]
+    assert h32[0] == 0 and h32[1] == 0           # silu(0) = 0
+    assert h32[2] == np.float32(120.0)           # sigma(80) rounds to 1
+    assert h32[3] == np.float32(200.0)           # beyond the clamp: sigma = 1
+    assert 0 < -h32[4] < 1e-30 and 0 < -h32[5] < 1e-30   # sigma(-80) ~ e^-80
+    assert h32[6] == 0                           # up = 0
+    ref = -1.0 / (1.0 + np.exp(1.0)) * 2.0       # silu(-1) * 2
+    assert abs(h32[7] / ref - 1) < 4 * 2.0 ** -23
+
+
+def test_silu_mul_quant_is_the_per_token_quant_of_bf16_h():
+    M, I = 5, 320
+    gu = _gu(M, I, seed=9)
+    Xq, xs, hb = oracle.silu_mul_quant(gu)
+    h = (hb.astype(np.uint32) << 16).view(np.float32)
+    am = np.abs(h).max(axis=1)
+    step = (am / np.float32(127)).astype(np.float32)   # numpy float32 division is IEEE
+    assert np.array_equal(xs, step)
+    q = np.clip(np.rint((h / step[:, None]).astype(np.float32)), -127, 127).astype(np.int8)
+    assert np.array_equal(Xq, q)
