@@ -178,7 +178,10 @@ def oracle_sample_step(w, inp, cal_rows=512, weight_elems=48 << 20, token_rows=1
         x = outs[src] if src else np.ascontiguousarray(inp.x[site.name][rows])
         s, gf, bf = prep[site.name]
         t0 = time.perf_counter()
-        Xq, xs = oracle.norm_quant(x, site.norm, gf, bf, w.eps)
+        if site.act == "silu_mul":
+            Xq, xs, _ = oracle.silu_mul_quant(x)
+        else:
+            Xq, xs = oracle.norm_quant(x, site.norm, gf, bf, w.eps)
         t_rows += time.perf_counter() - t0
         for lin in w.linears_of(site.name):
             Wq, ws, n, N = lin_q[lin.name]

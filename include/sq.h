@@ -233,6 +233,35 @@ sq_status sq_quant_per_token_given_absmax(const void* x, sq_dtype dtype, int64_t
                                           float* x_scale, void* stream);
 
 /*
+ * sq_silu_mul_quant_per_token -- the down projection's input, SiLU(gate) * up,
+ * computed from the merged gate/up projection's output and quantised per
+ * token in the same pass (h is never written unless h_out is given).
+ * [SQ-depth] "Where the scales go in a decoder block": the down_proj input is
+ * SiLU(gate) times up; it has no norm in front, is not smoothed, and is
+ * quantised with per-token scales.
+ *   gate_up  device [M, 2I] bf16, row stride ld_gu: gate in columns [0, I),
+ *            up in [I, 2I) (e.g. sq_w8a8_gemm_dequant's output for the
+ *            merged projection)
+ *   Xq       device [M, I] int8 OUT (stride I);  x_scale device [M] fp32 OUT
+ *   h_out    device [M, I] bf16 OUT (stride ld_h) or NULL: h itself
+ * Arithmetic (fp32, one IEEE rounding per step):
+ *   e = exp(-g) by Cody-Waite reduction and a degree-7 Taylor polynomial, the
+ *       argument clamped to [-87, 87] (a fixed operation sequence, under one
+ *       ulp from the exact exponential);
+ *   h = bf16(fl32(fl32(g * fl32(1 / fl32(1 + e))) * u));
+ *   x_scale = fl32(max_k |h| / 127), Xq = clamp(rne(fl32(h / x_scale)), +-127)
+ *   (0 where the row is all zero): sq_norm_smooth_quant_per_token of h with
+ *   SQ_NORM_NONE, bit for bit.
+ * I up to 28928 (two bf16 half-rows in shared memory), else SQ_ERR_UNSUPPORTED;
+ * dtype must be SQ_BF16 (else SQ_ERR_UNSUPPORTED).
+ * Errors: SQ_ERR_INVALID_ARG, SQ_ERR_ALIGNMENT (16-byte rows and pointers,
+ *         I % 16), SQ_ERR_UNSUPPORTED, SQ_ERR_CUDA.
+ */
+sq_status sq_silu_mul_quant_per_token(const void* gate_up, sq_dtype dtype, int64_t M, int64_t I,
+                                      int64_t ld_gu, int8_t* Xq, float* x_scale, void* h_out,
+                                      int64_t ld_h, void* stream);
+
+/*
  * sq_smooth_quantize_weights_per_tensor -- W-hat = W diag(s) quantised with
  * one step for the whole matrix, fl32(max |W-hat| / 127).
  *   w_scale  device [N] fp32 OUT: the step in every entry

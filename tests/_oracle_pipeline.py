@@ -46,6 +46,8 @@ def forward_rows(w, prep, inp, rows):
         src = next((l.source for l in w.linears if l.site == site.name and l.source), None)
         if src:
             x = res["linears"][src]["out"]
+            if site.act == "silu_mul":  # h = SiLU(gate) * up, stored in bf16
+                _, x = oracle.silu_mul(x)
         else:
             x = np.ascontiguousarray(inp.x[site.name][rows])
         st = prep["sites"][site.name]

@@ -410,6 +410,59 @@ def test_quant_given_absmax_below_the_row_max_saturates():
         assert np.array_equal(Xq_g[m:m + 1].cpu().numpy(), Xq_o), m
 
 
+# SiLU(gate) * up quantised per token (the down projection's input)
+SILU_SHAPES = [(1, 16), (3, 64), (17, 4096), (300, 4112), (64, 28672), (5, 28928), (2000, 1024)]
+
+
+def _gate_up(M, I, seed=0):
+    r = np.random.default_rng(seed)
+    g = (r.standard_normal((M, I)) * 2.5).astype(np.float32)
+    u = r.standard_normal((M, I)).astype(np.float32)
+    if I >= 16:
+        g[:, :8] = np.float32([0.0, -0.0, 90.0, -90.0, 1e-20, 40.0, -40.0, 87.5])
+        u[:, 8] *= 60.0  # an outlier channel of up
+    if M > 2:
+        g[1] = 0.0  # a row whose h is all zero: step 0, codes 0
+    return S.to_bf16_bits(np.concatenate([g, u], axis=1))
+
+
+@pytest.mark.parametrize("shape", SILU_SHAPES, ids=lambda s: "%dx%d" % s)
+def test_silu_mul_quant_matches_oracle(shape):
+    M, I = shape
+    gu = _gate_up(M, I)
+    Xq_o, xs_o, hb_o = oracle.silu_mul_quant(gu)
+    h = torch.empty((M, I), dtype=torch.bfloat16, device="cuda")
+    Xq_g, xs_g = sq.silu_mul_quant_per_token(to_gpu(gu), h_out=h)
+    assert np.array_equal(bf16_bits(h), hb_o)
+    assert np.array_equal(xs_g.cpu().numpy().view(np.uint32), xs_o.view(np.uint32))
+    assert np.array_equal(Xq_g.cpu().numpy(), Xq_o)
+    Xq2, xs2 = sq.silu_mul_quant_per_token(to_gpu(gu))  # without storing h
+    assert torch.equal(Xq2, Xq_g) and torch.equal(xs2, xs_g)
+
+
+def test_silu_mul_quant_strided_rows():
+    M, I = 37, 2048
+    gu = _gate_up(M, I, seed=3)
+    buf = torch.zeros((M, 2 * I + 64), dtype=torch.bfloat16, device="cuda")
+    buf[:, :2 * I] = to_gpu(gu)
+    hbuf = torch.full((M, I + 24), 2.0, dtype=torch.bfloat16, device="cuda")
+    Xq_g, xs_g = sq.silu_mul_quant_per_token(buf[:, :2 * I], h_out=hbuf[:, :I])
+    Xq_o, xs_o, hb_o = oracle.silu_mul_quant(gu)
+    assert np.array_equal(Xq_g.cpu().numpy(), Xq_o)
+    assert np.array_equal(bf16_bits(hbuf[:, :I].contiguous()), hb_o)
+    assert torch.all(hbuf[:, I:] == 2.0)
+
+
+def test_silu_mul_quant_rejects_what_it_cannot_run():
+    gu = torch.zeros((2, 2 * 28944), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(sq.SQError) as e:  # two half-rows beyond one CTA's shared memory
+        sq.silu_mul_quant_per_token(gu)
+    assert e.value.status == 2
+    with pytest.raises(sq.SQError) as e:  # bf16 rows only
+        sq.silu_mul_quant_per_token(torch.zeros((2, 64), dtype=torch.float32, device="cuda"))
+    assert e.value.status == 2
+
+
 def test_workload_opt66b_uses_the_rowmax_epilogue():
     blk = pipeline.Block(S.OPT66B_MLP, 256, "cuda")
     assert set(blk.rowmax) == {"fc1"}

@@ -174,3 +174,25 @@ def test_given_absmax_quant_rejects_bad_arguments(L):
     assert call(K=60) == 3              # int8 rows: K % 16
     assert call(K=48000, ld=48000) == 2  # longer rows than one CTA holds
     assert call(M=0, am=None, q=None, s=None) == 0
+
+
+def test_silu_mul_quant_rejects_bad_arguments(L):
+    f = L.sq_silu_mul_quant_per_token
+
+    def call(gu=A16, dt=1, M=4, I=64, ld=128, q=A16, s=A16, h=None, ldh=0):
+        return f(gu, dt, M, I, ld, q, s, h, ldh, None)
+
+    assert call(gu=None) == 1
+    assert call(dt=7) == 1
+    assert call(ld=64) == 1             # a row holds gate and up: ld >= 2I
+    assert call(I=0) == 1
+    assert call(M=-1) == 1
+    assert call(q=None) == 1
+    assert call(s=None) == 1
+    assert call(h=A16, ldh=32) == 1     # ld_h < I
+    assert call(dt=0) == 2              # bf16 rows only
+    assert call(I=40, ld=80) == 3       # I % 16
+    assert call(s=A8) == 3
+    assert call(h=A8, ldh=64) == 3
+    assert call(I=28944, ld=2 * 28944) == 2  # beyond one CTA's shared memory
+    assert call(M=0, gu=None, q=None, s=None) == 0

@@ -281,6 +281,27 @@ sq_status sq_quant_per_token_given_absmax(const void* x, sq_dtype dtype, int64_t
                                            row_absmax, Xq, x_scale, err, as_stream(stream)));
 }
 
+sq_status sq_silu_mul_quant_per_token(const void* gate_up, sq_dtype dtype, int64_t M, int64_t I,
+                                      int64_t ld_gu, int8_t* Xq, float* x_scale, void* h_out,
+                                      int64_t ld_h, void* stream) {
+  if (!valid_dtype(dtype) || M < 0 || I <= 0 || ld_gu < 2 * I) return SQ_ERR_INVALID_ARG;
+  if (h_out && ld_h < I) return SQ_ERR_INVALID_ARG;
+  if (dtype != SQ_BF16) return SQ_ERR_UNSUPPORTED;
+  if (M > 0x7fffffff || I > 0x7fffffff) return SQ_ERR_UNSUPPORTED;
+  if (M > 0 && (!gate_up || !Xq)) return SQ_ERR_INVALID_ARG;
+  sq_status st = check_vec(x_scale, M > 0);
+  if (st != SQ_OK) return st;
+  if (I % 16 != 0 || (ld_gu * 2) % 16 != 0 || !aligned16(gate_up) || !aligned16(Xq))
+    return SQ_ERR_ALIGNMENT;
+  if (h_out && (!aligned16(h_out) || (ld_h * 2) % 16 != 0)) return SQ_ERR_ALIGNMENT;
+  if (!silu_mul_pipe_supported(static_cast<int>(I))) return SQ_ERR_UNSUPPORTED;
+  if (M == 0) return SQ_OK;
+  int* err = device_error_word();
+  if (!err) return SQ_ERR_CUDA;
+  return from_cuda(launch_silu_mul_quant_pipe(gate_up, M, static_cast<int>(I), ld_gu, Xq, x_scale,
+                                              h_out, ld_h, err, as_stream(stream)));
+}
+
 sq_status sq_smooth_quantize_weights_per_tensor(const void* W, sq_dtype dtype, int64_t N,
                                                 int64_t K, int64_t ldw, const float* s,
                                                 int8_t* Wq, float* w_scale, float* w_absmax,

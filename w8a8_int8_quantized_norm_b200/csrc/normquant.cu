@@ -63,6 +63,64 @@ __device__ __forceinline__ void smem_chunk(const uint8_t* row, int ch, float2 (&
   }
 }
 
+// ---- SiLU(gate) * up ---------------------------------------------------
+// e^t as a fixed sequence of IEEE fp32 operations: Cody and Waite's argument
+// reduction (W. J. Cody, W. Waite, "Software Manual for the Elementary
+// Functions", 1980) with ln 2 split into a 16-significant-bit head (n * head
+// is exact for |n| < 256) and an fp32 tail, then the degree-7 Taylor
+// polynomial of e^r by Horner's rule in fused multiply-adds, then the exact
+// scaling by 2^n.  t is clamped to [-87, 87]: 2^n stays normal and sigma is
+// already 0 or 1 to far below an ulp of the product beyond that.
+// Max relative error against the exact exponential: under one fp32 ulp.
+constexpr float kLog2e = 1.44269504088896340736f;       // fl32(1 / ln 2)
+constexpr float kLn2Head = 0.693145751953125f;          // floor(ln 2 * 2^16) / 2^16
+constexpr float kLn2Tail = 1.4286067653301870e-06f;     // fl32(ln 2 - head)
+
+__device__ __forceinline__ float2 exp_cw2(float2 t) {
+  t.x = fminf(fmaxf(t.x, -87.0f), 87.0f);
+  t.y = fminf(fmaxf(t.y, -87.0f), 87.0f);
+  // n = rint(fl32(t * log2 e)): adding 1.5 * 2^23 rounds |x| < 2^22 to an
+  // integer (nearest, ties to even) and subtracting it back is exact; the
+  // integer itself sits in the low bits of the sum
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  const float2 sum = __fadd2_rn(__fmul2_rn(t, make_float2(kLog2e, kLog2e)),
+                                make_float2(kMagic, kMagic));
+  const float2 nn = __fadd2_rn(make_float2(kMagic, kMagic), make_float2(-sum.x, -sum.y));  // -n
+  float2 r = __ffma2_rn(nn, make_float2(kLn2Head, kLn2Head), t);
+  r = __ffma2_rn(nn, make_float2(kLn2Tail, kLn2Tail), r);
+  // Taylor coefficients 1/k!, each rounded to fp32
+  constexpr float c7 = 1.0f / 5040.0f, c6 = 1.0f / 720.0f, c5 = 1.0f / 120.0f,
+                  c4 = 1.0f / 24.0f, c3 = 1.0f / 6.0f;
+  float2 p = make_float2(c7, c7);
+  p = __ffma2_rn(p, r, make_float2(c6, c6));
+  p = __ffma2_rn(p, r, make_float2(c5, c5));
+  p = __ffma2_rn(p, r, make_float2(c4, c4));
+  p = __ffma2_rn(p, r, make_float2(c3, c3));
+  p = __ffma2_rn(p, r, make_float2(0.5f, 0.5f));
+  p = __ffma2_rn(p, r, make_float2(1.0f, 1.0f));
+  p = __ffma2_rn(p, r, make_float2(1.0f, 1.0f));
+  // 2^n from the integer in the sum's low bits: bits(sum) = 0x4b400000 + n
+  const float2 two_n =
+      make_float2(__int_as_float((__float_as_int(sum.x) - (0x4b400000 - 127)) << 23),
+                  __int_as_float((__float_as_int(sum.y) - (0x4b400000 - 127)) << 23));
+  return __fmul2_rn(p, two_n);
+}
+
+// Eight outputs h = bf16(fl32(fl32(g * fl32(1 / fl32(1 + e^-g))) * u)) of a
+// chunk, as packed bf16 pairs.
+__device__ __forceinline__ void silu_mul8(const float2 (&g)[4], const float2 (&u)[4],
+                                          uint32_t (&hb)[4]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 e = exp_cw2(make_float2(-g[i].x, -g[i].y));
+    const float2 d = __fadd2_rn(make_float2(1.0f, 1.0f), e);
+    const float2 sig = make_float2(__frcp_rn(d.x), __frcp_rn(d.y));
+    const float2 h = __fmul2_rn(__fmul2_rn(g[i], sig), u[i]);
+    const __nv_bfloat162 b = __floats2bfloat162_rn(h.x, h.y);
+    hb[i] = *reinterpret_cast<const uint32_t*>(&b);
+  }
+}
+
 __device__ __forceinline__ void param8(const float* p, int ch, float2 (&v)[4]) {
   const float4* q = reinterpret_cast<const float4*>(p + ch * kChunk);
   const float4 a = __ldg(q), b = __ldg(q + 1);
@@ -178,14 +236,23 @@ enum RowMode : int {
   kModeTensorMax = 2,   // one running max of |y| over the whole tensor
   kModeFixedQuant = 3,  // codes with one given step (per-tensor: O2 / O3)
   kModeGivenQuant = 4,  // per-row codes, each row's max |y| given in act_max[row]
+  kModeSiluMul = 5,     // per-row codes of h = SiLU(gate) * up (rows hold [gate | up])
 };
+
+// Bytes of one input row: SiLU * up rows hold both halves.
+template <int kMode>
+constexpr int kInRowFactor = kMode == kModeSiluMul ? 2 : 1;
 
 template <int CH, int kMode>
 struct PipeBounds {
-  static constexpr int kMaxThreads = CH <= 4 ? 512 : 640;
+  // SiLU * up rows (at most 28928 outputs: 3616 chunks) run 4 chunks a thread
+  // on up to 1024 threads: the row holds one CTA per SM (two 113 KB input
+  // buffers), so its warps are the only latency hiding there is
+  static constexpr int kMaxThreads = kMode == kModeSiluMul ? 1024 : (CH <= 4 ? 512 : 640);
   // 4-chunk CTAs keep to 64 registers a thread so four 256-thread CTAs fit
   // an SM; calibration also keeps a running column max per element
-  static constexpr int kMinBlocks = (CH <= 4 && kMode != kModeColMax) ? 2 : 1;
+  static constexpr int kMinBlocks =
+      (CH <= 4 && kMode != kModeColMax && kMode != kModeSiluMul) ? 2 : 1;
 };
 
 // One row per iteration, three CTA barriers per row (two when calibrating):
@@ -208,10 +275,13 @@ __global__ void __launch_bounds__(PipeBounds<CH, kMode>::kMaxThreads,
     norm_rows_pipe_kernel(const void* __restrict__ x, int64_t ldx, int64_t M, int K,
                           const float* __restrict__ gamma, const float* __restrict__ beta,
                           float eps, int8_t* __restrict__ q, float* __restrict__ scale,
-                          float* __restrict__ act_max, int nbuf, int* error_word) {
+                          float* __restrict__ act_max, int nbuf, int* error_word,
+                          __nv_bfloat16* __restrict__ h_out, int64_t ldh) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int kEsz = kBF16 ? 2 : 4;
-  const uint32_t row_bytes = static_cast<uint32_t>(K) * kEsz;
+  constexpr bool kGLU = kMode == kModeSiluMul;
+  static_assert(!kGLU || (kBF16 && NORMK == 0 && !kGamma && !kBeta), "SiLU * up: bf16, no norm");
+  const uint32_t row_bytes = static_cast<uint32_t>(K) * kEsz * kInRowFactor<kMode>;
   const uint32_t buf_stride = (row_bytes + 127u) & ~127u;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + nbuf * buf_stride);
   double* dscr = reinterpret_cast<double*>(bars + nbuf);      // [64]: sum x^2, sum x per warp
@@ -259,7 +329,7 @@ __global__ void __launch_bounds__(PipeBounds<CH, kMode>::kMaxThreads,
     if (__syncthreads_or(!ok)) aborted = true;
   }
   constexpr bool kCalib = kMode == kModeColMax;
-  constexpr bool kRowMax = kMode == kModeRowQuant || kMode == kModeTensorMax;
+  constexpr bool kRowMax = kMode == kModeRowQuant || kMode == kModeTensorMax || kGLU;
   float cta_max = 0.0f;  // tensor-max mode, thread 0
   // fixed-step mode: the one step, from the given max |y|
   float fstep = 0.0f, frstep = 0.0f;
@@ -300,15 +370,34 @@ __global__ void __launch_bounds__(PipeBounds<CH, kMode>::kMaxThreads,
     }
 
     // ---- this thread's chunks of the row, from shared memory
-    float2 v[CH][4];
+    // (SiLU * up keeps h as packed bf16 pairs instead: half the registers)
+    float2 v[kGLU ? 1 : CH][4];
+    uint32_t hbv[kGLU ? CH : 1][4];
+    uint32_t amb = 0;  // SiLU * up: max |h| as bf16 bits (magnitudes order like ints)
 #pragma unroll
     for (int c = 0; c < CH; ++c) {
       const int ch = t + c * T;
       if (kFull || ch < nchunks) {
-        smem_chunk<kBF16>(rowp, ch, v[c]);
+        if constexpr (kGLU) {
+          float2 g[4], u[4];
+          smem_chunk<true>(rowp, ch, g);
+          smem_chunk<true>(rowp + static_cast<uint32_t>(K) * 2u, ch, u);
+          silu_mul8(g, u, hbv[c]);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            amb = max(amb, max(hbv[c][i] & 0x7fffu, (hbv[c][i] >> 16) & 0x7fffu));
+          if (h_out)
+            *reinterpret_cast<uint4*>(h_out + row * ldh + ch * kChunk) =
+                make_uint4(hbv[c][0], hbv[c][1], hbv[c][2], hbv[c][3]);
+        } else {
+          smem_chunk<kBF16>(rowp, ch, v[c]);
+        }
       } else {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) v[c][i] = make_float2(0.0f, 0.0f);
+        for (int i = 0; i < 4; ++i) {
+          if constexpr (kGLU) hbv[c][i] = 0u;
+          else v[c][i] = make_float2(0.0f, 0.0f);
+        }
       }
     }
     // ---- row statistics in fp64 (two accumulators per sum for ILP)
@@ -386,10 +475,10 @@ __global__ void __launch_bounds__(PipeBounds<CH, kMode>::kMaxThreads,
     // ---- the norm output (paired fp32 ops, same roundings; a multiply
     // followed by an add uses the scalar intrinsics, which are never
     // contracted into a fused multiply-add)
-    float am = 0.0f;
+    float am = kGLU ? __uint_as_float(amb << 16) : 0.0f;
     const float2 r2 = make_float2(r, r), nmu2 = make_float2(-mu, -mu);
 #pragma unroll
-    for (int c = 0; c < CH; ++c) {
+    for (int c = 0; c < (kGLU ? 0 : CH); ++c) {
       const int ch = t + c * T;
       if (!kFull && ch >= nchunks) continue;
       float2 g[4], bt[4];
@@ -466,7 +555,17 @@ __global__ void __launch_bounds__(PipeBounds<CH, kMode>::kMaxThreads,
         for (int c = 0; c < CH; ++c) {
           const int ch = t + c * T;
           if (!kFull && ch >= nchunks) continue;
-          *reinterpret_cast<uint2*>(qrow + ch * kChunk) = codes8(v[c], rstep, step, exact_only);
+          if constexpr (kGLU) {
+            float2 hv[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              hv[i] = make_float2(__uint_as_float(hbv[c][i] << 16),
+                                  __uint_as_float(hbv[c][i] & 0xffff0000u));
+            *reinterpret_cast<uint2*>(qrow + ch * kChunk) = codes8(hv, rstep, step, exact_only);
+          } else {
+            *reinterpret_cast<uint2*>(qrow + ch * kChunk) =
+                codes8(v[c], rstep, step, exact_only);
+          }
         }
       }
     }
@@ -533,17 +632,19 @@ struct PipeShape {
 // row buffers, their barriers, 64 doubles of partial sums, r and mu, 3 absmax slots
 size_t pipe_smem(size_t stride, int nbuf) { return nbuf * stride + 8 * nbuf + 64 * 8 + 4 * 8; }
 
-bool pipe_shape(int K, bool bf16, bool calib, PipeShape* ps) {
+bool pipe_shape(int K, bool bf16, bool calib, PipeShape* ps, int in_factor = 1) {
   const int nchunks = K / kChunk;
   // chunks per thread and threads per CTA within the variant's register budget
   int ch = nchunks <= 4 * PipeBounds<4, kModeRowQuant>::kMaxThreads ? 4
            : (nchunks <= 8 * PipeBounds<8, kModeRowQuant>::kMaxThreads ? 8 : 0);
   (void)calib;  // the calibration variant uses the same shape (4-chunk rows only)
+  if (in_factor > 1) ch = 4;  // SiLU * up: four chunks a thread, up to 1024 threads
   if (!ch) return false;
   int threads = (nchunks + ch - 1) / ch;
   threads = (threads + 31) / 32 * 32;
   if (threads < 32) threads = 32;
-  const size_t row_bytes = static_cast<size_t>(K) * (bf16 ? 2 : 4);
+  if (threads > 1024) return false;
+  const size_t row_bytes = static_cast<size_t>(K) * (bf16 ? 2 : 4) * in_factor;
   const size_t stride = (row_bytes + 127) / 128 * 128;
   // about 24 KB of row buffers per CTA: with small rows that leaves room for
   // eight CTAs per SM (more rows in flight, shorter per-CTA row chains)
@@ -551,7 +652,8 @@ bool pipe_shape(int K, bool bf16, bool calib, PipeShape* ps) {
   if (nbuf < 3) nbuf = 3;
   if (nbuf > 8) nbuf = 8;
   while (nbuf > 2 && nbuf * stride > (150u << 10)) --nbuf;
-  if (nbuf * stride > (200u << 10)) return false;
+  // two-half rows (SiLU * up) may take two buffers up to the 227 KB a CTA can have
+  if (nbuf * stride > (in_factor > 1 ? (226u << 10) : (200u << 10))) return false;
   ps->ch = ch;
   ps->threads = threads;
   ps->nbuf = nbuf;
@@ -571,6 +673,8 @@ struct RowArgs {
   float* scale;
   float* act_max;
   int* err;
+  __nv_bfloat16* h_out = nullptr;
+  int64_t ldh = 0;
 };
 
 template <bool kBF16, int NORMK, int CH, bool kG, bool kB, bool kF, int kMode>
@@ -581,7 +685,8 @@ cudaError_t launch_pipe_k(const RowArgs& a, PipeShape ps, cudaStream_t st) {
   LaunchCache& lc = launch_cache();
   int per_sm = 0;
   // fewer row buffers when each CTA sees only a few rows: more CTAs fit an SM
-  const size_t stride = (static_cast<size_t>(a.K) * (kBF16 ? 2 : 4) + 127) / 128 * 128;
+  const size_t stride =
+      (static_cast<size_t>(a.K) * (kBF16 ? 2 : 4) * kInRowFactor<kMode> + 127) / 128 * 128;
   for (;;) {
     cudaError_t e = lc.ensure_smem(key, ps.smem);
     if (e != cudaSuccess) return e;
@@ -599,7 +704,8 @@ cudaError_t launch_pipe_k(const RowArgs& a, PipeShape ps, cudaStream_t st) {
   const int64_t max_grid = kC ? (a.M + 3) / 4 : a.M;
   if (grid > max_grid) grid = max_grid;
   kern<<<static_cast<unsigned>(grid), ps.threads, ps.smem, st>>>(
-      a.x, a.ldx, a.M, a.K, a.gamma, a.beta, a.eps, a.q, a.scale, a.act_max, ps.nbuf, a.err);
+      a.x, a.ldx, a.M, a.K, a.gamma, a.beta, a.eps, a.q, a.scale, a.act_max, ps.nbuf, a.err,
+      a.h_out, a.ldh);
   return cudaGetLastError();
 }
 
@@ -701,6 +807,23 @@ cudaError_t launch_quant_given_pipe(const void* x, bool bf16, int64_t M, int K, 
                   const_cast<float*>(row_absmax), err};
   if (bf16) return launch_pipe_n<true, 0, kModeGivenQuant>(a, ps, st);
   return launch_pipe_n<false, 0, kModeGivenQuant>(a, ps, st);
+}
+
+bool silu_mul_pipe_supported(int I) {
+  PipeShape ps;
+  return pipe_shape(I, true, false, &ps, 2);
+}
+
+cudaError_t launch_silu_mul_quant_pipe(const void* gu, int64_t M, int I, int64_t ldgu,
+                                       int8_t* q, float* scale, void* h_out, int64_t ldh,
+                                       int* err, cudaStream_t st) {
+  if (M == 0) return cudaSuccess;
+  PipeShape ps;
+  if (!pipe_shape(I, true, false, &ps, 2)) return cudaErrorInvalidValue;
+  RowArgs a{gu, M, I, ldgu, nullptr, nullptr, 0.0f, q, scale, nullptr, err};
+  a.h_out = static_cast<__nv_bfloat16*>(h_out);
+  a.ldh = ldh;
+  return launch_pipe_t<true, 0, 4, false, false, kModeSiluMul>(a, ps, st);
 }
 
 }  // namespace sq

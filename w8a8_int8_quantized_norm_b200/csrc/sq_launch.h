@@ -97,6 +97,12 @@ cudaError_t launch_quant_fixed_pipe(const void* x, bool bf16, int64_t M, int K, 
 cudaError_t launch_quant_given_pipe(const void* x, bool bf16, int64_t M, int K, int64_t ldx,
                                     const float* row_absmax, int8_t* q, float* scale, int* err,
                                     cudaStream_t st);
+// Per-row codes of h = SiLU(gate) * up from bf16 rows [gate (I) | up (I)],
+// h rounded to bf16 first (and stored to h_out [M, I], stride ldh, if given).
+bool silu_mul_pipe_supported(int I);
+cudaError_t launch_silu_mul_quant_pipe(const void* gu, int64_t M, int I, int64_t ldgu,
+                                       int8_t* q, float* scale, void* h_out, int64_t ldh,
+                                       int* err, cudaStream_t st);
 cudaError_t launch_calibrate(const void* x, bool bf16, int64_t M, int K, int64_t ldx, int norm,
                              const float* gamma, const float* beta, float eps, float* act_max,
                              int* err, cudaStream_t st);

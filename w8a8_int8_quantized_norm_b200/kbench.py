@@ -6,6 +6,7 @@
     python -m w8a8_int8_quantized_norm_b200.kbench weight_quant --N 28672 --K 8192
     python -m w8a8_int8_quantized_norm_b200.kbench smooth_scales --N 12288 --K 4096
     python -m w8a8_int8_quantized_norm_b200.kbench quant_given --M 4096 --K 36864
+    python -m w8a8_int8_quantized_norm_b200.kbench silu_mul_quant --M 16384 --K 28672
     python -m w8a8_int8_quantized_norm_b200.kbench gemm --M 4096 --N 36864 --K 9216 --rowmax
 
 Each call is captured once as a CUDA graph; every timed replay is bracketed by
@@ -102,7 +103,7 @@ def _time(fn, iters, warmup, flush):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("op", choices=["norm_quant", "gemm", "calibrate", "weight_quant",
-                                   "smooth_scales", "quant_given"])
+                                   "smooth_scales", "quant_given", "silu_mul_quant"])
     ap.add_argument("--M", type=int, default=4096)
     ap.add_argument("--N", type=int, default=4096)
     ap.add_argument("--K", type=int, default=4096)
@@ -147,6 +148,14 @@ def main(argv=None):
         fn = lambda: sq.quant_per_token_given_absmax(x, am, xq, xs)
         units = M * K * (esz + 1) + 8 * M
         shape = {"M": M, "K": K, "dtype": a.dtype}
+    elif a.op == "silu_mul_quant":
+        # K is the width of h; the input rows hold gate and up (2K)
+        gu = (torch.randn((M, 2 * K), generator=gen, device=dev) * 2.0).to(torch.bfloat16)
+        xq = torch.empty((M, K), dtype=torch.int8, device=dev)
+        xs = torch.empty(M, dtype=torch.float32, device=dev)
+        fn = lambda: sq.silu_mul_quant_per_token(gu, xq, xs)
+        units = M * 2 * K * 2 + M * K + 4 * M
+        shape = {"M": M, "I": K, "dtype": "bf16"}
     elif a.op == "calibrate":
         x = _acts(M, K, a.dtype, gen, dev)
         g = torch.empty(K, device=dev).uniform_(0.5, 1.5, generator=gen) if norm else None

@@ -104,10 +104,15 @@ class Block:
         # quantisation reads the row once with its max already known.  Only
         # on prefill tiles (the decode plan keeps its own tiles).
         self.rowmax: Dict[str, torch.Tensor] = {}  # source Linear -> [M] row maxima
+        # per-tensor variants keep SiLU(gate) * up in bf16 (its tensor-wide max)
+        self.h: Dict[str, torch.Tensor] = {
+            site.name: torch.empty((M, site.K), dtype=torch.bfloat16, device=dev)
+            for site in w.sites if site.act == "silu_mul" and granularity != "per_token"}
         if granularity == "per_token":
             for lin in w.linears:
                 site = w.site(lin.site)
-                if lin.source and site.norm == sq.NORM_NONE and not site.smoothed:
+                if (lin.source and not site.act and site.norm == sq.NORM_NONE
+                        and not site.smoothed):
                     src = next(l for l in w.linears if l.name == lin.source)
                     K_src = w.site(src.site).K
                     if sq.gemm_plan(M, src.N, K_src).kernel != 2:
@@ -172,10 +177,27 @@ class Block:
         for site in w.sites:
             src = next((l.source for l in w.linears if l.site == site.name and l.source), None)
             xin = self.out[src] if src else x[site.name]
+            fused_act = site.act == "silu_mul" and self.granularity == "per_token"
+            if site.act == "silu_mul":
+                # the down projection's input, SiLU(gate) * up of the merged
+                # projection's output: per-token codes in the same pass; the
+                # per-tensor variants store h and quantise it as a tensor
+                h = self.h.get(site.name)
+                gu = xin
+                _run(timer, "silu_mul_quant",
+                     gu.numel() * gu.element_size() + self.M * site.K * (1 + 2 * (h is not None))
+                     + 4 * self.M,
+                     lambda: sq.silu_mul_quant_per_token(gu, self.xq[site.name],
+                                                         self.xs[site.name], h_out=h,
+                                                         stream=stream))
+                if h is not None:
+                    xin = h
             nparam = (self.gamma_f[site.name] is not None) + (self.beta_f[site.name] is not None)
             units = xin.numel() * (xin.element_size() + 1) + 4 * self.M + 4 * site.K * nparam
             gf, bf = self.gamma_f[site.name], self.beta_f[site.name]
-            if src in self.rowmax:
+            if fused_act:
+                pass
+            elif src in self.rowmax:
                 am = self.rowmax[src]
                 _run(timer, "norm_quant", units,
                      lambda: sq.quant_per_token_given_absmax(xin, am, self.xq[site.name],
@@ -232,6 +254,7 @@ class Block:
         the kernels of its GEMM plan (the main kernel, plus the split-K
         reduction or stream-K fix-up where the plan has one)."""
         n = len(self.w.sites)
+        n += sum(1 for site in self.w.sites if site.name in self.h)  # h, then its codes
         if self.granularity != "per_token":
             n += sum(1 for site in self.w.sites if not self.static[site.name])  # O2 max pass
         for lin in self.w.linears:

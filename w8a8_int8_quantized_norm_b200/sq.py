@@ -36,6 +36,7 @@ EXPORTS = (
     "sq_w8a8_gemm_dequant_noalloc", "sq_w8a8_gemm_plan", "sq_norm_smooth_absmax",
     "sq_norm_smooth_quant_per_tensor", "sq_smooth_quantize_weights_per_tensor",
     "sq_w8a8_gemm_dequant_rowmax", "sq_quant_per_token_given_absmax",
+    "sq_silu_mul_quant_per_token",
 )
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -111,6 +112,7 @@ def _declare(L):
     L.sq_w8a8_gemm_dequant_rowmax.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _I32, _P, _I64,
                                               _P, _I32, _P]
     L.sq_quant_per_token_given_absmax.argtypes = [_P, _I32, _I64, _I64, _I64, _P, _P, _P, _P]
+    L.sq_silu_mul_quant_per_token.argtypes = [_P, _I32, _I64, _I64, _I64, _P, _P, _P, _I64, _P]
     L.sq_w8a8_gemm_plan.argtypes = [_I64, _I64, _I64, _I32, _I32, ctypes.POINTER(GemmPlanInfo)]
     L.sq_set_wait_limit.argtypes = [_I64]
     L.sq_set_wait_limit.restype = None
@@ -283,6 +285,29 @@ def quant_per_token_given_absmax(x: torch.Tensor, row_absmax: torch.Tensor, Xq=N
     _check(lib().sq_quant_per_token_given_absmax(
         _ptr(x), _dtype_code(x), M, K, ld, _ptr(_vec(row_absmax, M, "row_absmax")), _ptr(Xq),
         _ptr(x_scale), _stream(stream)), "sq_quant_per_token_given_absmax")
+    return Xq, x_scale
+
+
+def silu_mul_quant_per_token(gate_up: torch.Tensor, Xq=None, x_scale=None, h_out=None,
+                             stream=None):
+    """Per-token codes of h = SiLU(gate) * up from gate_up [M, 2I] (gate in the
+    first I columns).  ``h_out`` (bf16 [M, I]) also receives h when given."""
+    M, K2, ld = _rows(gate_up, "gate_up")
+    if K2 % 2:
+        raise ValueError("gate_up rows hold two halves")
+    I = K2 // 2
+    if Xq is None:
+        Xq = torch.empty((M, I), dtype=torch.int8, device=gate_up.device)
+    if x_scale is None:
+        x_scale = torch.empty(M, dtype=torch.float32, device=gate_up.device)
+    ldh = 0
+    if h_out is not None:
+        if h_out.dtype != torch.bfloat16 or tuple(h_out.shape) != (M, I):
+            raise ValueError("h_out must be bf16 [M, I]")
+        _, _, ldh = _rows(h_out, "h_out")
+    _check(lib().sq_silu_mul_quant_per_token(_ptr(gate_up), _dtype_code(gate_up), M, I, ld,
+                                             _ptr(Xq), _ptr(x_scale), _ptr(h_out), ldh,
+                                             _stream(stream)), "sq_silu_mul_quant_per_token")
     return Xq, x_scale
 
 

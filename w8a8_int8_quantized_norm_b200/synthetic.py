@@ -66,6 +66,9 @@ class Site:
     norm: int
     smoothed: bool
     calibrated: bool = True  # smoothed sites need a calibration batch
+    # how a site fed by a Linear's output is formed from it: "" = the output
+    # itself; "silu_mul" = SiLU(first half) * second half (gate, up), K wide
+    act: str = ""
 
 
 @dataclasses.dataclass(frozen=True)
@@ -74,7 +77,7 @@ class Linear:
     site: str        # activation site it reads
     N: int
     relu: bool = False
-    source: Optional[str] = None  # Linear whose (ReLU'd) output this site is, if any
+    source: Optional[str] = None  # Linear whose output forms this Linear's site, if any
 
 
 @dataclasses.dataclass(frozen=True)
@@ -107,11 +110,11 @@ def _llama_block(M: int, name: str) -> Workload:
         sites=(Site("attn_norm", 8192, NORM_RMS, True),
                Site("attn_out", 8192, NORM_NONE, False, calibrated=False),
                Site("mlp_norm", 8192, NORM_RMS, True),
-               Site("mlp_act", 28672, NORM_NONE, False, calibrated=False)),
+               Site("mlp_act", 28672, NORM_NONE, False, calibrated=False, act="silu_mul")),
         linears=(Linear("qkv", "attn_norm", 10240),
                  Linear("o_proj", "attn_out", 8192),
                  Linear("gate_up", "mlp_norm", 57344),
-                 Linear("down", "mlp_act", 8192)),
+                 Linear("down", "mlp_act", 8192, source="gate_up")),
         outliers=OutlierLaw(fraction=0.001, factor=50.0))
 
 
