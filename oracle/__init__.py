@@ -94,6 +94,16 @@ def _declare(L):
     L.oracle_exp_cw.argtypes = [_P, _I64, _P]
     L.oracle_silu_mul.restype = None
     L.oracle_silu_mul.argtypes = [_P, ctypes.c_int, _I64, _I64, _I64, _P, _P]
+    L.oracle_e4m3_to_f32.restype = ctypes.c_float
+    L.oracle_e4m3_to_f32.argtypes = [ctypes.c_uint8]
+    L.oracle_f32_to_e4m3.restype = ctypes.c_uint8
+    L.oracle_f32_to_e4m3.argtypes = [ctypes.c_float]
+    L.oracle_quantize_rows_fp8.restype = None
+    L.oracle_quantize_rows_fp8.argtypes = [_P, _I64, _I64, _P, _P]
+    L.oracle_gemm_fp8.restype = None
+    L.oracle_gemm_fp8.argtypes = [_P, _P, _I64, _I64, _I64, _P]
+    L.oracle_epilogue_f32.restype = None
+    L.oracle_epilogue_f32.argtypes = [_P, _P, _P, _I64, _I64, ctypes.c_int, _P, _P]
     L.oracle_num_threads.restype = ctypes.c_int
     L.oracle_num_threads.argtypes = []
 
@@ -332,6 +342,70 @@ def silu_mul_quant(gu):
     _, hb = silu_mul(gu)
     Xq, xs = norm_quant(hb, NORM_NONE)
     return Xq, xs, hb
+
+
+# ---- FP8 (e4m3) W8A8 (see oracle.c for the readings) ----------------------
+
+def e4m3_decode(codes) -> np.ndarray:
+    """Values of e4m3 codes (uint8) as fp32."""
+    c = np.asarray(codes, dtype=np.uint8)
+    f = lib().oracle_e4m3_to_f32
+    table = np.array([f(i) for i in range(256)], dtype=np.float32)
+    return table[c]
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """fp32 -> e4m3 codes, nearest-even, saturating at +-448."""
+    x = np.asarray(x, dtype=np.float32)
+    f = lib().oracle_f32_to_e4m3
+    return np.array([f(float(v)) for v in x.ravel()], dtype=np.uint8).reshape(x.shape)
+
+
+def quantize_rows_fp8(y: np.ndarray):
+    """Per-row FP8: step = fl32(max|y| / 448), code = e4m3(fl32(y * fl32(1/step))).
+    Returns (q uint8 [M, K], step fp32 [M])."""
+    y = np.ascontiguousarray(y, dtype=np.float32)
+    M, K = y.shape
+    q = np.empty((M, K), np.uint8)
+    step = np.empty(M, np.float32)
+    lib().oracle_quantize_rows_fp8(_ptr(y), M, K, _ptr(q), _ptr(step))
+    return q, step
+
+
+def norm_quant_fp8(x, norm_kind, gamma_f=None, beta_f=None, eps=1e-5):
+    """The norm (step 4) then per-token FP8 codes.  Returns (Xq8, x_scale)."""
+    y, _, _ = norm(x, norm_kind, gamma_f, beta_f, eps)
+    return quantize_rows_fp8(y)
+
+
+def quantize_weights_fp8(W, s=None):
+    """W-hat = fl32(W * s) per output channel in FP8.  Returns (Wq8, w_scale)."""
+    return quantize_rows_fp8(smooth_weights(W, s))
+
+
+def gemm_fp8(Xq8, Wq8) -> np.ndarray:
+    """Exact sum of the decoded products, fp64 [M, N]."""
+    Xq8 = np.ascontiguousarray(Xq8, dtype=np.uint8)
+    Wq8 = np.ascontiguousarray(Wq8, dtype=np.uint8)
+    M, K = Xq8.shape
+    N = Wq8.shape[0]
+    if K > (1 << 17):
+        raise ValueError("the fp64 sum is exact for K <= 2^17")
+    acc = np.empty((M, N), np.float64)
+    lib().oracle_gemm_fp8(_ptr(Xq8), _ptr(Wq8), M, N, K, _ptr(acc))
+    return acc
+
+
+def epilogue_f32(acc32, x_scale, w_scale, relu=False):
+    """Epilogue from an fp32 accumulator: (o32 [M, N], out bf16 bits [M, N])."""
+    acc32 = np.ascontiguousarray(acc32, dtype=np.float32)
+    M, N = acc32.shape
+    xs, ws = _f32(x_scale), _f32(w_scale)
+    o32 = np.empty((M, N), np.float32)
+    out = np.empty((M, N), np.uint16)
+    lib().oracle_epilogue_f32(_ptr(acc32), _ptr(xs), _ptr(ws), M, N, int(bool(relu)), _ptr(o32),
+                              _ptr(out))
+    return o32, out
 
 
 def linear(x, norm_kind, gamma_f, beta_f, eps, Wq, w_scale, relu=False):

@@ -573,6 +573,109 @@ void oracle_silu_mul(const void* gu, int dtype, int64_t M, int64_t I, int64_t ld
     }
 }
 
+/* ------------------------------------------------------------------------ */
+/* FP8 (e4m3) W8A8                                                           */
+/* ------------------------------------------------------------------------ */
+/*
+ * [LLMint8] "example . what you get": on GPUs with FP8 support, FP8 W8A8 has
+ * largely taken over INT8's role, with the same smoothing applied before the
+ * activations are quantised; [SQ-map] "What it did NOT solve": FP8 hardware
+ * later overtook INT8 serving.  The pages give no FP8 arithmetic.  Readings:
+ *   - format: e4m3 without infinities (OCP FP8 E4M3, "fn"): sign, 4 exponent
+ *     bits with bias 7, 3 mantissa bits; largest finite 448, smallest
+ *     subnormal 2^-9; 0x7f / 0xff are NaN and never produced here;
+ *   - encoding: round to nearest even; magnitudes beyond 448 saturate to 448;
+ *   - per-token (and per-output-channel) scaling as for INT8 with the grid's
+ *     largest value 448 in place of 127: step = fl32(absmax / 448);
+ *   - the code multiplies by the correctly rounded reciprocal of the step,
+ *     code = e4m3(fl32(y * fl32(1 / step))): the stored step is what the
+ *     epilogue multiplies by; (the pages quantise by division for INT8 only);
+ *   - a row whose step is zero or subnormal (absmax below 448 * 2^-126) is
+ *     all zero codes with step 0;
+ *   - the GEMM accumulates the products of the decoded codes; its exact value
+ *     is computed here in fp64 (every product is a multiple of 2^-18 below
+ *     2^18, so sums of up to 2^17 of them are exact);
+ *   - epilogue as for INT8 from the fp32 accumulator:
+ *     out = bf16(fl32(fl32(acc * xs[m]) * ws[n])).
+ */
+#define E4M3_MAX 448.0f
+
+float oracle_e4m3_to_f32(uint8_t c) {
+  const int sign = c >> 7, e = (c >> 3) & 15, m = c & 7;
+  float v;
+  if (e == 0) v = ldexpf((float)m, -9);                /* subnormal: m * 2^-9 */
+  else v = ldexpf((float)(8 + m), e - 10);             /* (1 + m/8) * 2^(e-7) */
+  return sign ? -v : v;
+}
+
+/* Round |x| (finite) to the e4m3 grid, nearest, ties to even; saturate. */
+uint8_t oracle_f32_to_e4m3(float x) {
+  const uint8_t sign = signbit(x) ? 0x80 : 0x00;
+  double a = fabs((double)x);
+  if (a >= 464.0) return sign | 0x7e;  /* at or past the midpoint above 448 */
+  /* the grid spacing at a: 2^-9 below 2^-6, else 2^(floor(log2 a) - 3) */
+  int e2 = -6;
+  if (a >= ldexp(1.0, -6)) e2 = ilogb(a);
+  const double q = ldexp(1.0, e2 - 3);
+  double n = a / q;                       /* exact: a power-of-two scaling */
+  double r = nearbyint(n);                /* current rounding mode: to nearest even */
+  /* the integer multiple r of q: 8..16 in the normal binade, 0..8 below */
+  double val = r * q;
+  if (val >= 464.0) return sign | 0x7e;
+  if (val == 0.0) return sign;
+  int ev = ilogb(val);
+  if (ev < -6) return sign | (uint8_t)(val / ldexp(1.0, -9)); /* subnormal code */
+  const int m = (int)(val / ldexp(1.0, ev - 3)) - 8;
+  return sign | (uint8_t)(((ev + 7) << 3) | m);
+}
+
+/* Per-row FP8 quantisation of y [M, K]: q [M, K] e4m3 codes, step [M]. */
+void oracle_quantize_rows_fp8(const float* y, int64_t M, int64_t K, uint8_t* q, float* step) {
+#pragma omp parallel for schedule(static)
+  for (int64_t m = 0; m < M; ++m) {
+    float am = 0.0f;
+    for (int64_t k = 0; k < K; ++k) {
+      const float a = fabsf(y[m * K + k]);
+      if (a > am) am = a;
+    }
+    float st = am / E4M3_MAX;
+    if (!(st >= 1.17549435e-38f)) st = 0.0f; /* zero or subnormal step: zero row */
+    step[m] = st;
+    const float inv = st > 0.0f ? 1.0f / st : 0.0f;
+    for (int64_t k = 0; k < K; ++k)
+      q[m * K + k] = st > 0.0f ? oracle_f32_to_e4m3(y[m * K + k] * inv) : 0;
+  }
+}
+
+/* Exact acc[m, n] = sum_k dec(Xq[m, k]) * dec(Wq[n, k]) in fp64 (K <= 2^17). */
+void oracle_gemm_fp8(const uint8_t* Xq, const uint8_t* Wq, int64_t M, int64_t N, int64_t K,
+                     double* acc) {
+  float lut[256];
+  for (int c = 0; c < 256; ++c) lut[c] = oracle_e4m3_to_f32((uint8_t)c);
+#pragma omp parallel for collapse(2) schedule(static)
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t n = 0; n < N; ++n) {
+      double s = 0.0;
+      for (int64_t k = 0; k < K; ++k)
+        s += (double)lut[Xq[m * K + k]] * (double)lut[Wq[n * K + k]];
+      acc[m * N + n] = s;
+    }
+}
+
+/* Epilogue from an fp32 accumulator: o32 = fl32(fl32(acc * xs) * ws), ReLU
+ * as in oracle_epilogue, out = bf16(o32). */
+void oracle_epilogue_f32(const float* acc, const float* xs, const float* ws, int64_t M,
+                         int64_t N, int relu, float* o32_out, uint16_t* out_bf16) {
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t n = 0; n < N; ++n) {
+      float t = acc[m * N + n] * xs[m];
+      float o = t * ws[n];
+      if (relu && !(o > 0.0f)) o = 0.0f;
+      if (o32_out) o32_out[m * N + n] = o;
+      if (out_bf16) out_bf16[m * N + n] = oracle_f32_to_bf16_bits(o);
+    }
+}
+
 /* Thread count the OpenMP loops will use (for the CPU-baseline report). */
 int oracle_num_threads(void) {
 #ifdef _OPENMP

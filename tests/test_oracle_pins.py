@@ -549,3 +549,111 @@ def test_silu_mul_quant_is_the_per_token_quant_of_bf16_h():
     assert np.array_equal(xs, step)
     q = np.clip(np.rint((h / step[:, None]).astype(np.float32)), -127, 127).astype(np.int8)
     assert np.array_equal(Xq, q)
+
+
+# ---------------------------------------------------------------------------
+# FP8 (e4m3) W8A8
+# ---------------------------------------------------------------------------
+
+def _e4m3_by_definition(c):
+    """The value of an e4m3 ("fn") code from the format: bias 7, 3 mantissa bits."""
+    sign = -1.0 if c & 0x80 else 1.0
+    e, m = (c >> 3) & 15, c & 7
+    if e == 15 and m == 7:
+        return float("nan")
+    if e == 0:
+        return sign * m * 2.0 ** -9
+    return sign * (1 + m / 8) * 2.0 ** (e - 7)
+
+
+def test_e4m3_decode_follows_the_format_and_torch():
+    d = oracle.e4m3_decode(np.arange(256))
+    ref = np.array([_e4m3_by_definition(c) for c in range(256)])
+    finite = ~np.isnan(ref)
+    assert np.array_equal(d[finite].astype(np.float64), ref[finite])
+    t = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).float().numpy()
+    assert np.array_equal(d[finite], t[finite])
+    assert d[0x7e] == 448 and d[0x01] == 2.0 ** -9 and d[0x08] == 2.0 ** -6
+
+
+def test_e4m3_encode_rounds_to_nearest_even_and_saturates():
+    vals = np.sort(np.unique(np.abs(oracle.e4m3_decode(np.arange(0x7f)))))
+    mids = ((vals[:-1].astype(np.float64) + vals[1:]) / 2).astype(np.float32)  # exact in fp32
+    codes = oracle.e4m3_encode(mids)
+    lo = oracle.e4m3_encode(vals[:-1])
+    hi = oracle.e4m3_encode(vals[1:])
+    # a tie goes to the neighbour whose code (mantissa) is even
+    expect = np.where(lo % 2 == 0, lo, hi)
+    assert np.array_equal(codes, expect)
+    # just off the midpoints: nearest
+    assert np.array_equal(oracle.e4m3_encode(np.nextafter(mids, np.float32(0))), lo)
+    assert np.array_equal(oracle.e4m3_encode(np.nextafter(mids, np.float32(1e9))), hi)
+    # saturation at 448 (464 is the tie with the non-finite 480: even -> 448)
+    big = np.float32([448, 455, 464, 465, 1e6, 3e38, -448, -470, -3e38])
+    assert list(oracle.e4m3_encode(big)) == [0x7e] * 6 + [0xfe] * 3
+    assert list(oracle.e4m3_encode(np.float32([0.0, -0.0]))) == [0x00, 0x80]
+    # random values inside the range: torch's cast (nearest even) agrees
+    x = (np.random.default_rng(3).standard_normal(100000) * 40).astype(np.float32)
+    x = np.concatenate([x[np.abs(x) < 448], np.float32(np.random.default_rng(4).uniform(
+        -2.0 ** -5, 2.0 ** -5, 20000))])
+    t = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.e4m3_encode(x), t)
+
+
+def test_fp8_row_quantisation():
+    r = np.random.default_rng(11)
+    y = (r.standard_normal((6, 4096)) * 3).astype(np.float32)
+    y[0, 17] = 60.0                 # the row max: code 448 exactly
+    y[1] = 0.0                      # zero row
+    y[2] = 1e-37 * np.sign(y[2])    # step would be subnormal: zero row
+    y[3, :] = np.abs(y[3, :])       # one sign
+    q, step = oracle.quantize_rows_fp8(y)
+    am = np.abs(y).max(axis=1)
+    st = (am / np.float32(448)).astype(np.float32)
+    st[st < np.finfo(np.float32).tiny] = 0
+    assert np.array_equal(step, st)
+    assert step[0] == np.float32(60) / np.float32(448) and q[0, 17] == 0x7e
+    assert not q[1].any() and not q[2].any() and step[1] == step[2] == 0
+    # every other row: the decoded code times the step is y to within half an
+    # e4m3 spacing (relative 2^-4 for normals, 2^-10 * step absolute below)
+    for m in (0, 3, 4, 5):
+        dq = oracle.e4m3_decode(q[m]).astype(np.float64) * step[m]
+        err = np.abs(dq - y[m])
+        assert np.all(err <= np.abs(y[m]) * 2.0 ** -4 + 2.0 ** -10 * step[m] * 1.0001)
+        assert np.abs(oracle.e4m3_decode(q[m])).max() == 448
+    # the code is the cast of fl32(y * fl32(1 / step)) (numpy float32, torch cast)
+    inv = (np.float32(1) / step[4]).astype(np.float32)
+    t = torch.from_numpy((y[4] * inv).astype(np.float32)).to(torch.float8_e4m3fn)
+    assert np.array_equal(q[4], t.view(torch.uint8).numpy())
+
+
+def test_fp8_gemm_is_the_exact_sum():
+    r = np.random.default_rng(12)
+    codes = np.concatenate([np.arange(0, 0x7f), np.arange(0x80, 0xff)]).astype(np.uint8)
+    A = r.choice(codes, (5, 40)).astype(np.uint8)
+    B = r.choice(codes, (7, 40)).astype(np.uint8)
+    acc = oracle.gemm_fp8(A, B)
+    da = [[Fraction(_e4m3_by_definition(int(c))) for c in row] for row in A]
+    db = [[Fraction(_e4m3_by_definition(int(c))) for c in row] for row in B]
+    for m in range(5):
+        for n in range(7):
+            assert Fraction(acc[m, n]) == sum(x * w for x, w in zip(da[m], db[n]))
+    # extremes: 448 * 448 * K exactly
+    K = 4096
+    full = oracle.gemm_fp8(np.full((1, K), 0x7e, np.uint8), np.full((2, K), 0xfe, np.uint8))
+    assert np.all(full == -448.0 * 448.0 * K)
+
+
+def test_fp8_epilogue_matches_float32_arithmetic():
+    r = np.random.default_rng(13)
+    acc = (r.standard_normal((9, 31)) * 1e4).astype(np.float32)
+    xs = (r.random(9) * 0.05).astype(np.float32)
+    ws = (r.random(31) * 0.002).astype(np.float32)
+    for relu in (False, True):
+        o32, out = oracle.epilogue_f32(acc, xs, ws, relu)
+        ref = ((acc * xs[:, None]).astype(np.float32) * ws[None, :]).astype(np.float32)
+        if relu:
+            ref = np.where(ref > 0, ref, np.float32(0))
+        assert np.array_equal(o32, ref)
+        tb = torch.from_numpy(ref).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        assert np.array_equal(out, tb)
