@@ -78,7 +78,8 @@ typedef enum { SQ_NORM_NONE = 0, SQ_NORM_RMS = 1, SQ_NORM_LAYER = 2 } sq_norm;
 typedef enum {
   SQ_EPI_BF16 = 0,      /* out bf16 = bf16(fp32(fp32(float(acc) * xs[m]) * ws[n])) */
   SQ_EPI_BF16_RELU = 1, /* the same with max(., 0) before the bf16 rounding */
-  SQ_EPI_I32_RAW = 2    /* out int32 = acc (no scaling; for exactness checks) */
+  SQ_EPI_I32_RAW = 2,   /* out int32 = acc (no scaling; for exactness checks) */
+  SQ_EPI_F32_RAW = 3    /* FP8 GEMMs only: out fp32 = the fp32 accumulator */
 } sq_epilogue;
 
 /* Largest K for which |sum_k q_a q_b| <= 127*127*K fits in INT32. */
@@ -231,6 +232,57 @@ sq_status sq_norm_smooth_quant_per_tensor(const void* x, sq_dtype dtype, int64_t
 sq_status sq_quant_per_token_given_absmax(const void* x, sq_dtype dtype, int64_t M, int64_t K,
                                           int64_t ldx, const float* row_absmax, int8_t* Xq,
                                           float* x_scale, void* stream);
+
+/*
+ * FP8 (e4m3) W8A8: the same smoothing, FP8 codes instead of INT8.
+ * [LLMint8] "example . what you get": on GPUs with FP8 support, FP8 W8A8
+ * took over INT8's role and the same smoothing still tames the activation
+ * outliers before they are quantised; [SQ-map] "What it did NOT solve".
+ * The pages give no FP8 arithmetic; this library's reading:
+ *   e4m3 without infinities (largest finite 448), round to nearest even,
+ *   saturating; step = fl32(max |y| / 448) per row; code =
+ *   e4m3(fl32(y * fl32(1 / step))); a zero or subnormal step gives step 0 and
+ *   all-zero codes.  The GEMM runs tcgen05 kind::f8f6f4 with an fp32
+ *   accumulator; out = bf16(fl32(fl32(acc * x_scale[m]) * w_scale[n])).
+ *
+ * sq_norm_smooth_quant_per_token_fp8 -- sq_norm_smooth_quant_per_token with
+ * FP8 codes: Xq8 device [M, K] e4m3 bytes OUT; x_scale device [M] fp32 OUT.
+ * Rows up to 40960 (bf16) / 25600 (fp32) elements, else SQ_ERR_UNSUPPORTED.
+ * Errors: those of sq_norm_smooth_quant_per_token.
+ */
+sq_status sq_norm_smooth_quant_per_token_fp8(const void* x, sq_dtype dtype, int64_t M, int64_t K,
+                                             int64_t ldx, sq_norm norm,
+                                             const float* gamma_folded, const float* beta_folded,
+                                             float eps, uint8_t* Xq8, float* x_scale,
+                                             void* stream);
+
+/*
+ * sq_smooth_quantize_weights_fp8 -- W-hat = fl32(W * s) per output channel in
+ * FP8: Wq8 device [N, K] e4m3 bytes OUT, w_scale device [N] fp32 OUT.
+ * Arguments and errors as for sq_smooth_quantize_weights (rows up to the
+ * limits of sq_norm_smooth_quant_per_token_fp8).
+ */
+sq_status sq_smooth_quantize_weights_fp8(const void* W, sq_dtype dtype, int64_t N, int64_t K,
+                                         int64_t ldw, const float* s, uint8_t* Wq8,
+                                         float* w_scale, void* stream);
+
+/*
+ * sq_fp8_gemm_dequant -- e4m3 x e4m3 GEMM (fp32 accumulator in tensor memory)
+ * with the dequantising epilogue fused.
+ *   Xq8 device [M, K] e4m3 (stride K); Wq8 device [N, K] e4m3 (stride K)
+ *   epi      SQ_EPI_BF16, SQ_EPI_BF16_RELU (out bf16 [M, N], stride ldo) or
+ *            SQ_EPI_F32_RAW (out fp32 [M, N] = the accumulator)
+ *   path_hint as for sq_w8a8_gemm_dequant; every tile runs its whole K (no
+ *            split-K or stream-K partial sums), so no workspace is needed.
+ * The tensor cores' fp32 accumulation order is theirs: the accumulator
+ * equals the exact sum of the decoded products to within the rounding of
+ * the accumulation (not bit-exact with a sequential sum).
+ * Errors: those of sq_w8a8_gemm_dequant (K <= SQ_MAX_K as there).
+ */
+sq_status sq_fp8_gemm_dequant(const uint8_t* Xq8, const uint8_t* Wq8, const float* x_scale,
+                              const float* w_scale, int64_t M, int64_t N, int64_t K,
+                              sq_epilogue epi, void* out, int64_t ldo, int path_hint,
+                              void* stream);
 
 /*
  * sq_silu_mul_quant_per_token -- the down projection's input, SiLU(gate) * up,

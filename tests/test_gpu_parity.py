@@ -745,3 +745,95 @@ def test_workload_per_tensor_granularity(wname, granularity):
                                        lin.relu)
             idx = torch.from_numpy(rows).cuda()
             assert np.array_equal(bf16_bits(out_g[lin.name][idx].contiguous()), out_o), lin.name
+
+
+# ---------------------------------------------------------------------------
+# FP8 (e4m3) W8A8
+# ---------------------------------------------------------------------------
+
+F8_SHAPES = [(1, 16), (3, 48), (17, 64), (129, 4112), (64, 8192), (5, 28672), (1000, 4096)]
+
+
+@pytest.mark.parametrize("shape", F8_SHAPES, ids=lambda s: "%dx%d" % s)
+@pytest.mark.parametrize("kind", KINDS, ids=lambda k: k[0])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_fp8_norm_quant_matches_oracle(shape, kind, dtype):
+    M, K = shape
+    if dtype == "f32" and K > 25600:
+        pytest.skip("fp32 rows above 25600 elements are unsupported")
+    _, norm, with_params = kind
+    x = _acts(M, K, dtype)
+    if M > 2:
+        x[1] = 0  # zero row: step 0, codes 0
+    g = RNG.uniform(0.5, 1.5, K).astype(np.float32) if with_params else None
+    b = (RNG.standard_normal(K) * 0.1).astype(np.float32) \
+        if (with_params and norm == oracle.NORM_LAYER) else None
+    Xq_o, xs_o = oracle.norm_quant_fp8(x, norm, g, b, 1e-5)
+    Xq_g, xs_g = sq.norm_smooth_quant_per_token_fp8(
+        to_gpu(x), norm, None if g is None else to_gpu(g), None if b is None else to_gpu(b), 1e-5)
+    compare_rows_quant(Xq_g.cpu().numpy(), xs_g.cpu().numpy(), Xq_o, xs_o,
+                       norm_near_tie_rows(x, norm, 1e-5))
+
+
+@pytest.mark.parametrize("NK", [(1, 16), (300, 4096), (129, 4112), (64, 28672)],
+                         ids=lambda s: "%dx%d" % s)
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_fp8_weights_match_oracle(NK, dtype):
+    N, K = NK
+    if dtype == "f32" and K > 25600:
+        pytest.skip("fp32 rows above 25600 elements are unsupported")
+    W = (RNG.standard_normal((N, K)) * 0.02).astype(np.float32)
+    W = S.to_bf16_bits(W) if dtype == "bf16" else W
+    s = RNG.uniform(0.25, 4.0, K).astype(np.float32)
+    Wq_o, ws_o = oracle.quantize_weights_fp8(W, s)
+    Wq_g, ws_g = sq.smooth_quantize_weights_fp8(to_gpu(W), to_gpu(s))
+    assert np.array_equal(Wq_g.cpu().numpy(), Wq_o)
+    assert np.array_equal(ws_g.cpu().numpy().view(np.uint32), ws_o.view(np.uint32))
+
+
+_F8_CODES = np.concatenate([np.arange(0, 0x7f), np.arange(0x80, 0xff)]).astype(np.uint8)
+F8_GEMM_SHAPES = [(16, 64, 64), (3, 5, 16), (129, 257, 4112), (256, 512, 1024), (300, 777, 160),
+                  (1024, 768, 2048), (2048, 1536, 512)]
+
+
+@pytest.mark.parametrize("shape", F8_GEMM_SHAPES, ids=lambda s: "%dx%dx%d" % s)
+@pytest.mark.parametrize("path", [1, 2, 3])
+def test_fp8_gemm_accumulator_and_epilogue(shape, path):
+    """The fp32 accumulator is the exact sum of the decoded products to within
+    the rounding of K/32 accumulation steps (each of the 32-deep MMA steps adds
+    its partial sum into fp32: at most one rounding of relative 2^-24 of the
+    running magnitude, bounded by sum |a b|; a factor 2 covers the rounding
+    inside a step).  Given that accumulator, the bf16 epilogue is bit-exact."""
+    M, N, K = shape
+    if path == 2 and M > 256:
+        pytest.skip("decode tiles take at most 256 tokens")
+    A = RNG.choice(_F8_CODES, (M, K)).astype(np.uint8)
+    B = RNG.choice(_F8_CODES, (N, K)).astype(np.uint8)
+    exact = oracle.gemm_fp8(A, B)
+    da = oracle.e4m3_decode(A).astype(np.float64)
+    db = oracle.e4m3_decode(B).astype(np.float64)
+    absum = np.abs(da) @ np.abs(db).T
+    acc = sq.fp8_gemm_dequant(to_gpu(A), to_gpu(B), None, None, "f32", path_hint=path)
+    acc_g = acc.cpu().numpy()
+    steps = max(1, (K + 31) // 32)
+    assert np.all(np.abs(acc_g.astype(np.float64) - exact) <= steps * 2.0 ** -23 * absum)
+    xs = (RNG.random(M) * 0.05 + 1e-3).astype(np.float32)
+    ws = (RNG.random(N) * 0.002 + 1e-5).astype(np.float32)
+    for relu in (False, True):
+        out = sq.fp8_gemm_dequant(to_gpu(A), to_gpu(B), to_gpu(xs), to_gpu(ws),
+                                  "bf16_relu" if relu else "bf16", path_hint=path)
+        _, out_o = oracle.epilogue_f32(acc_g, xs, ws, relu)
+        assert np.array_equal(bf16_bits(out), out_o)
+
+
+def test_fp8_gemm_rejects_int8_only_epilogues():
+    A = torch.zeros((8, 64), dtype=torch.uint8, device="cuda")
+    B = torch.zeros((32, 64), dtype=torch.uint8, device="cuda")
+    with pytest.raises(sq.SQError) as e:
+        sq.fp8_gemm_dequant(A, B, None, None, "i32",
+                            out=torch.empty((8, 32), dtype=torch.int32, device="cuda"))
+    assert e.value.status == 1
+    with pytest.raises(sq.SQError) as e:  # the INT8 GEMM has no fp32 accumulator
+        sq.w8a8_gemm_dequant(A.view(torch.int8), B.view(torch.int8), None, None, "f32",
+                             out=torch.empty((8, 32), dtype=torch.float32, device="cuda"))
+    assert e.value.status == 1

@@ -196,3 +196,25 @@ def test_silu_mul_quant_rejects_bad_arguments(L):
     assert call(h=A8, ldh=64) == 3
     assert call(I=28944, ld=2 * 28944) == 2  # beyond one CTA's shared memory
     assert call(M=0, gu=None, q=None, s=None) == 0
+
+
+def test_fp8_calls_reject_bad_arguments(L):
+    g = L.sq_fp8_gemm_dequant
+
+    def gemm(Xq=A16, Wq=A16, xs=A16, ws=A16, M=16, N=64, K=64, epi=0, out=A16, ldo=64, path=0):
+        return g(Xq, Wq, xs, ws, M, N, K, epi, out, ldo, path, None)
+
+    assert gemm(epi=2) == 1             # INT32 output: INT8 GEMMs only
+    assert gemm(epi=7) == 1
+    assert gemm(path=5) == 1
+    assert gemm(xs=None) == 1           # bf16 epilogues need both scales
+    assert gemm(K=40) == 3
+    assert gemm(M=0, Xq=None, xs=None, out=None) == 0
+    q = L.sq_norm_smooth_quant_per_token_fp8
+    assert q(A16, 1, 4, 64, 64, 1, None, None, 1e-5, None, A16, None) == 1
+    assert q(A16, 1, 4, 64, 64, 9, None, None, 1e-5, A16, A16, None) == 1
+    assert q(A16, 1, 4, 64, 64, 1, None, None, 1e-5, A8, A16, None) == 3
+    assert q(A16, 1, 0, 64, 64, 1, None, None, 1e-5, None, None, None) == 0
+    w = L.sq_smooth_quantize_weights_fp8
+    assert w(A16, 1, 4, 64, 64, None, None, A16, None) == 1
+    assert w(A16, 1, 4, 64, 64, A8, A16, A16, None) == 3

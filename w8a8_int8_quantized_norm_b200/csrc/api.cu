@@ -281,6 +281,59 @@ sq_status sq_quant_per_token_given_absmax(const void* x, sq_dtype dtype, int64_t
                                            row_absmax, Xq, x_scale, err, as_stream(stream)));
 }
 
+sq_status sq_norm_smooth_quant_per_token_fp8(const void* x, sq_dtype dtype, int64_t M, int64_t K,
+                                             int64_t ldx, sq_norm norm,
+                                             const float* gamma_folded, const float* beta_folded,
+                                             float eps, uint8_t* Xq8, float* x_scale,
+                                             void* stream) {
+  sq_status st = check_tensor_rows(x, dtype, M, K, ldx, norm, gamma_folded, beta_folded, eps);
+  if (st != SQ_OK) return st;
+  if (M > 0) {
+    if (!Xq8) return SQ_ERR_INVALID_ARG;
+    if (!aligned16(Xq8)) return SQ_ERR_ALIGNMENT;
+    if ((st = check_vec(x_scale, true)) != SQ_OK) return st;
+  }
+  if (M == 0) return SQ_OK;
+  int* err = device_error_word();
+  if (!err) return SQ_ERR_CUDA;
+  return from_cuda(launch_norm_quant_fp8_pipe(x, dtype == SQ_BF16, M, static_cast<int>(K), ldx,
+                                              norm, gamma_folded, beta_folded, eps, Xq8, x_scale,
+                                              err, as_stream(stream)));
+}
+
+sq_status sq_smooth_quantize_weights_fp8(const void* W, sq_dtype dtype, int64_t N, int64_t K,
+                                         int64_t ldw, const float* s, uint8_t* Wq8,
+                                         float* w_scale, void* stream) {
+  // a weight row smoothed by s is the no-norm row path with s as multiplier
+  return sq_norm_smooth_quant_per_token_fp8(W, dtype, N, K, ldw, SQ_NORM_NONE, s, nullptr, 0.0f,
+                                            Wq8, w_scale, stream);
+}
+
+sq_status sq_fp8_gemm_dequant(const uint8_t* Xq8, const uint8_t* Wq8, const float* x_scale,
+                              const float* w_scale, int64_t M, int64_t N, int64_t K,
+                              sq_epilogue epi, void* out, int64_t ldo, int path_hint,
+                              void* stream) {
+  if (epi != SQ_EPI_BF16 && epi != SQ_EPI_BF16_RELU && epi != SQ_EPI_F32_RAW)
+    return SQ_ERR_INVALID_ARG;
+  // the shape, alignment and scale checks of the INT8 call (a raw fp32
+  // accumulator has the raw INT32 output's size and needs no scales)
+  const sq_epilogue e = epi == SQ_EPI_F32_RAW ? SQ_EPI_I32_RAW : epi;
+  sq_status st = check_gemm(reinterpret_cast<const int8_t*>(Xq8),
+                            reinterpret_cast<const int8_t*>(Wq8), x_scale, w_scale, M, N, K, e,
+                            out, ldo, path_hint, 1);
+  if (st != SQ_OK) return st;
+  if (M == 0 || N == 0) return SQ_OK;
+  const int sms = sms_cached();
+  // whole-K tiles only: the fp32 accumulator has no exact split-K sum
+  const GemmPlan plan = plan_gemm(M, N, K, path_hint, 1, sms);
+  int* err = device_error_word();
+  if (!err) return SQ_ERR_CUDA;
+  return from_cuda(launch_gemm(plan, reinterpret_cast<const int8_t*>(Xq8),
+                               reinterpret_cast<const int8_t*>(Wq8), x_scale, w_scale, M, N, K,
+                               epi, out, ldo, nullptr, sms, g_wait_polls.load(), err,
+                               as_stream(stream), nullptr, true));
+}
+
 sq_status sq_silu_mul_quant_per_token(const void* gate_up, sq_dtype dtype, int64_t M, int64_t I,
                                       int64_t ld_gu, int8_t* Xq, float* x_scale, void* h_out,
                                       int64_t ld_h, void* stream) {

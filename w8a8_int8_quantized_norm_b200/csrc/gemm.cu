@@ -213,8 +213,16 @@ __device__ __forceinline__ bool work_next(const Params& p, Work& w, int& pb, int
 
 // Epilogue for one CHUNK of accumulator columns held by this thread (row p of
 // the P side, columns q0 .. q0 + CHUNK - 1 of the Q side).
+// The accumulator word as a float: INT32 sums convert (rounding above 2^24),
+// FP8 GEMMs accumulate in fp32 already.
+template <bool kF8>
+__device__ __forceinline__ float acc_value(uint32_t r) {
+  if constexpr (kF8) return __uint_as_float(r);
+  else return __int2float_rn(static_cast<int>(r));
+}
+
 // Returns the chunk's max |bf16 out| when prm.row_absmax asks for it (else 0).
-template <int CHUNK>
+template <int CHUNK, bool kF8 = false>
 __device__ __forceinline__ float store_chunk(const Params& prm, const uint32_t (&r)[32], int p,
                                              int q0, int split, int slot) {
   if (p >= prm.P) return 0.0f;
@@ -235,7 +243,7 @@ __device__ __forceinline__ float store_chunk(const Params& prm, const uint32_t (
     }
     return 0.0f;
   }
-  if (prm.epi == SQ_EPI_I32_RAW) {
+  if (prm.epi == SQ_EPI_I32_RAW || prm.epi == SQ_EPI_F32_RAW) {  // the accumulator's bits
     int32_t* o = static_cast<int32_t*>(prm.out);
     if (!prm.swap) {
       int32_t* dst = o + static_cast<int64_t>(p) * prm.ldo + q0;
@@ -274,7 +282,7 @@ __device__ __forceinline__ float store_chunk(const Params& prm, const uint32_t (
     float v[CHUNK];
 #pragma unroll
     for (int j = 0; j < CHUNK; ++j) {
-      float t = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(r[j])), xs), ws[j]);
+      float t = __fmul_rn(__fmul_rn(acc_value<kF8>(r[j]), xs), ws[j]);
       if (relu) t = t > 0.0f ? t : 0.0f;  // -0 (a zero scale) becomes +0
       v[j] = t;
     }
@@ -313,7 +321,7 @@ __device__ __forceinline__ float store_chunk(const Params& prm, const uint32_t (
       const int q = q0 + j;
       if (q < prm.Q) {
         const float xs = __ldg(prm.q_scale + q);
-        float t = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(r[j])), xs), ws);
+        float t = __fmul_rn(__fmul_rn(acc_value<kF8>(r[j]), xs), ws);
         if (relu) t = t > 0.0f ? t : 0.0f;  // -0 (a zero scale) becomes +0
         o[static_cast<int64_t>(q) * prm.ldo + p] = __float2bfloat16_rn(t);
       }
@@ -322,7 +330,7 @@ __device__ __forceinline__ float store_chunk(const Params& prm, const uint32_t (
   return 0.0f;
 }
 
-template <int BN>
+template <int BN, bool kF8>
 __global__ void __launch_bounds__(kThreads, 1)
     w8a8_gemm_kernel(const __grid_constant__ CUtensorMap mapP,
                      const __grid_constant__ CUtensorMap mapQ, const Params prm) {
@@ -411,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    constexpr uint32_t kIdesc = idesc_i8(BM, BN);
+    constexpr uint32_t kIdesc = kF8 ? idesc_f8(BM, BN) : idesc_i8(BM, BN);
     int stage = 0;
     uint32_t phase = 0;
     int acc = 0;
@@ -438,8 +446,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t sb = b_base + stage * C::B_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BK / UMMA_K; ++kk) {
-            mma_i8(d_tmem, smem_desc_k_sw128(sa + kk * UMMA_K), smem_desc_k_sw128(sb + kk * UMMA_K),
-                   kIdesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+            if constexpr (kF8)
+              mma_f8(d_tmem, smem_desc_k_sw128(sa + kk * UMMA_K),
+                     smem_desc_k_sw128(sb + kk * UMMA_K), kIdesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+            else
+              mma_i8(d_tmem, smem_desc_k_sw128(sa + kk * UMMA_K),
+                     smem_desc_k_sw128(sb + kk * UMMA_K), kIdesc, (kb > kb0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(EMPTY_BAR(stage));
         }
@@ -528,7 +540,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         else
           tmem_ld_32x32b_x16(taddr, r);
         tmem_wait_ld();
-        rmax = fmaxf(rmax, store_chunk<C::CHUNK>(prm, r, p, qb * BN + c * C::CHUNK, split, slot));
+        rmax = fmaxf(rmax,
+                     store_chunk<C::CHUNK, kF8>(prm, r, p, qb * BN + c * C::CHUNK, split, slot));
       }
       if (prm.row_absmax && rmax > 0.0f && p < prm.P)
         atomicMax(reinterpret_cast<unsigned int*>(prm.row_absmax) + p, __float_as_uint(rmax));
@@ -597,7 +610,7 @@ __device__ __forceinline__ int64_t loads_on_stage(int64_t total, int s, int stag
   return total / stages + (s < total % stages ? 1 : 0);
 }
 
-template <int TN>
+template <int TN, bool kF8>
 __global__ void __launch_bounds__(kThreads, 1)
     w8a8_gemm_pair_kernel(const __grid_constant__ CUtensorMap mapP,
                           const __grid_constant__ CUtensorMap mapQ, const Params prm) {
@@ -705,7 +718,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader only)
     if (leader) {
-      constexpr uint32_t kIdesc = idesc_i8(TILE_M, TN);
+      constexpr uint32_t kIdesc = kF8 ? idesc_f8(TILE_M, TN) : idesc_i8(TILE_M, TN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -731,9 +744,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t sb = b_base + stage * B_BYTES;
 #pragma unroll
             for (int kk = 0; kk < BK / UMMA_K; ++kk) {
-              mma_i8_pair(d_tmem, smem_desc_k_sw128(sa + kk * UMMA_K),
-                          smem_desc_k_sw128(sb + kk * UMMA_K), kIdesc,
-                          (kb > kb0 || kk > 0) ? 1u : 0u);
+              if constexpr (kF8)
+                mma_f8_pair(d_tmem, smem_desc_k_sw128(sa + kk * UMMA_K),
+                            smem_desc_k_sw128(sb + kk * UMMA_K), kIdesc,
+                            (kb > kb0 || kk > 0) ? 1u : 0u);
+              else
+                mma_i8_pair(d_tmem, smem_desc_k_sw128(sa + kk * UMMA_K),
+                            smem_desc_k_sw128(sb + kk * UMMA_K), kIdesc,
+                            (kb > kb0 || kk > 0) ? 1u : 0u);
             }
             // the stage is free in both CTAs once these MMAs have read it
             mma_commit_pair(EMPTY_BAR(stage));
@@ -825,7 +843,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                static_cast<uint32_t>(acc * TN + c * 32);
         tmem_ld_32x32b_x32(taddr, r);
         tmem_wait_ld();
-        rmax = fmaxf(rmax, store_chunk<32>(prm, r, p, qb * TN + c * 32, 0, -1));
+        rmax = fmaxf(rmax, store_chunk<32, kF8>(prm, r, p, qb * TN + c * 32, 0, -1));
       }
       if (prm.row_absmax && rmax > 0.0f && p < prm.P)
         atomicMax(reinterpret_cast<unsigned int*>(prm.row_absmax) + p, __float_as_uint(rmax));
@@ -984,22 +1002,22 @@ bool make_map(CUtensorMap* map, const int8_t* ptr, int64_t rows, int64_t K, int 
   return r == CUDA_SUCCESS;
 }
 
-template <int BN>
+template <int BN, bool kF8>
 cudaError_t launch_bn(const Params& prm, const CUtensorMap& mp, const CUtensorMap& mq, int grid,
                       cudaStream_t st) {
   using C = Cfg<BN>;
-  cudaError_t e = launch_cache().ensure_smem(reinterpret_cast<const void*>(w8a8_gemm_kernel<BN>),
-                                             C::SMEM_BYTES);
+  cudaError_t e = launch_cache().ensure_smem(
+      reinterpret_cast<const void*>(w8a8_gemm_kernel<BN, kF8>), C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  w8a8_gemm_kernel<BN><<<grid, kThreads, C::SMEM_BYTES, st>>>(mp, mq, prm);
+  w8a8_gemm_kernel<BN, kF8><<<grid, kThreads, C::SMEM_BYTES, st>>>(mp, mq, prm);
   return cudaGetLastError();
 }
 
-template <int TN>
+template <int TN, bool kF8>
 cudaError_t launch_pair(const Params& prm, const CUtensorMap& mp, const CUtensorMap& mq,
                         int max_pairs, cudaStream_t st) {
   using C = PairCfg<TN>;
-  auto kern = w8a8_gemm_pair_kernel<TN>;
+  auto kern = w8a8_gemm_pair_kernel<TN, kF8>;
   cudaError_t e = launch_cache().ensure_smem(reinterpret_cast<const void*>(kern), C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   cudaLaunchAttribute attr[1];
@@ -1014,7 +1032,7 @@ cudaError_t launch_pair(const Params& prm, const CUtensorMap& mp, const CUtensor
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   // as many co-resident CTA pairs as the device holds (one per SM pair)
-  static int max_clusters[64] = {};
+  static int max_clusters[64] = {};  // per instantiation
   const int dev = LaunchCache::device();
   if (dev >= 0 && dev < 64 && max_clusters[dev] == 0) {
     cfg.gridDim = dim3(2 * max_pairs);
@@ -1119,8 +1137,12 @@ cudaError_t launch_gemm(const GemmPlan& plan, const int8_t* Xq, const int8_t* Wq
                         const float* x_scale, const float* w_scale, int64_t M, int64_t N,
                         int64_t K, int epi, void* out, int64_t ldo, void* workspace, int num_sms,
                         int64_t wait_polls, int* error_word, cudaStream_t st,
-                        float* row_absmax) {
+                        float* row_absmax, bool fp8) {
   if (M == 0 || N == 0) return cudaSuccess;
+  // FP8 accumulators are fp32: no INT32 partial sums to add exactly
+  if (fp8 && (plan.splits > 1 || plan.streamk || epi == SQ_EPI_I32_RAW))
+    return cudaErrorInvalidValue;
+  if (!fp8 && epi == SQ_EPI_F32_RAW) return cudaErrorInvalidValue;
   Params prm{};
   const int8_t* Pptr = plan.swap ? Wq : Xq;
   const int8_t* Qptr = plan.swap ? Xq : Wq;
@@ -1144,12 +1166,13 @@ cudaError_t launch_gemm(const GemmPlan& plan, const int8_t* Xq, const int8_t* Wq
   prm.streamk = plan.streamk;
   prm.sk_iters = plan.sk_iters;
   prm.sk_partial = plan.streamk ? static_cast<int32_t*>(workspace) : nullptr;
-  if (row_absmax && (plan.swap || epi == SQ_EPI_I32_RAW)) return cudaErrorInvalidValue;
+  if (row_absmax && (plan.swap || epi == SQ_EPI_I32_RAW || epi == SQ_EPI_F32_RAW))
+    return cudaErrorInvalidValue;
   prm.row_absmax = row_absmax;
   prm.wait_polls = wait_polls;
   prm.error_word = error_word;
   {
-    const int64_t esz = epi == SQ_EPI_I32_RAW ? 4 : 2;
+    const int64_t esz = (epi == SQ_EPI_I32_RAW || epi == SQ_EPI_F32_RAW) ? 4 : 2;
     prm.vec_out = ((reinterpret_cast<uintptr_t>(out) & 15u) == 0 && (ldo * esz) % 16 == 0) ? 1 : 0;
   }
 
@@ -1160,9 +1183,11 @@ cudaError_t launch_gemm(const GemmPlan& plan, const int8_t* Xq, const int8_t* Wq
     // each CTA of a pair loads 128 rows of A and 128 rows of B
     if (!make_map(&mp, Pptr, prm.P, K, 128) || !make_map(&mq, Qptr, prm.Q, K, plan.bn / 2))
       return cudaErrorInvalidValue;
-    switch (plan.bn) {
-      case 256: return launch_pair<256>(prm, mp, mq, sms / 2, st);
-      case 192: return launch_pair<192>(prm, mp, mq, sms / 2, st);
+    switch (plan.bn * 2 + (fp8 ? 1 : 0)) {
+      case 512: return launch_pair<256, false>(prm, mp, mq, sms / 2, st);
+      case 384: return launch_pair<192, false>(prm, mp, mq, sms / 2, st);
+      case 513: return launch_pair<256, true>(prm, mp, mq, sms / 2, st);
+      case 385: return launch_pair<192, true>(prm, mp, mq, sms / 2, st);
       default: return cudaErrorInvalidValue;
     }
   }
@@ -1170,12 +1195,23 @@ cudaError_t launch_gemm(const GemmPlan& plan, const int8_t* Xq, const int8_t* Wq
     return cudaErrorInvalidValue;
   const int grid = plan.streamk ? plan.grid : (prm.units < sms ? prm.units : sms);
   cudaError_t e;
+  if (fp8) {
+    switch (plan.bn) {
+      case 16: e = launch_bn<16, true>(prm, mp, mq, grid, st); break;
+      case 32: e = launch_bn<32, true>(prm, mp, mq, grid, st); break;
+      case 64: e = launch_bn<64, true>(prm, mp, mq, grid, st); break;
+      case 128: e = launch_bn<128, true>(prm, mp, mq, grid, st); break;
+      case 256: e = launch_bn<256, true>(prm, mp, mq, grid, st); break;
+      default: return cudaErrorInvalidValue;
+    }
+    return e;
+  }
   switch (plan.bn) {
-    case 16: e = launch_bn<16>(prm, mp, mq, grid, st); break;
-    case 32: e = launch_bn<32>(prm, mp, mq, grid, st); break;
-    case 64: e = launch_bn<64>(prm, mp, mq, grid, st); break;
-    case 128: e = launch_bn<128>(prm, mp, mq, grid, st); break;
-    case 256: e = launch_bn<256>(prm, mp, mq, grid, st); break;
+    case 16: e = launch_bn<16, false>(prm, mp, mq, grid, st); break;
+    case 32: e = launch_bn<32, false>(prm, mp, mq, grid, st); break;
+    case 64: e = launch_bn<64, false>(prm, mp, mq, grid, st); break;
+    case 128: e = launch_bn<128, false>(prm, mp, mq, grid, st); break;
+    case 256: e = launch_bn<256, false>(prm, mp, mq, grid, st); break;
     default: return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;

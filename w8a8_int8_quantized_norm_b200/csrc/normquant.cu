@@ -22,6 +22,7 @@
 //     with the exact division (branch-free otherwise).  Rounding to the
 //     nearest integer (ties to even) is the float add of 1.5 * 2^23, whose low
 //     8 mantissa bits are then the two's-complement INT8 code.
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <float.h>
 #include <stdint.h>
@@ -119,6 +120,23 @@ __device__ __forceinline__ void silu_mul8(const float2 (&g)[4], const float2 (&u
     const __nv_bfloat162 b = __floats2bfloat162_rn(h.x, h.y);
     hb[i] = *reinterpret_cast<const uint32_t*>(&b);
   }
+}
+
+// FP8 (e4m3) codes of 8 values, packed little-endian: e4m3(fl32(v * inv)),
+// nearest even, saturating at +-448 (cvt.rn.satfinite), where inv is the
+// correctly rounded reciprocal of the row's step.
+__device__ __forceinline__ uint2 codes8_f8(const float2 (&v)[4], float inv) {
+  const float2 inv2 = make_float2(inv, inv);
+  uint32_t w[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t lo = __nv_cvt_float2_to_fp8x2(__fmul2_rn(v[2 * h], inv2), __NV_SATFINITE,
+                                                 __NV_E4M3);
+    const uint32_t hi = __nv_cvt_float2_to_fp8x2(__fmul2_rn(v[2 * h + 1], inv2), __NV_SATFINITE,
+                                                 __NV_E4M3);
+    w[h] = (lo & 0xffffu) | (hi << 16);
+  }
+  return make_uint2(w[0], w[1]);
 }
 
 __device__ __forceinline__ void param8(const float* p, int ch, float2 (&v)[4]) {
@@ -237,6 +255,7 @@ enum RowMode : int {
   kModeFixedQuant = 3,  // codes with one given step (per-tensor: O2 / O3)
   kModeGivenQuant = 4,  // per-row codes, each row's max |y| given in act_max[row]
   kModeSiluMul = 5,     // per-row codes of h = SiLU(gate) * up (rows hold [gate | up])
+  kModeRowQuantF8 = 6,  // per-row step and FP8 (e4m3) codes
 };
 
 // Bytes of one input row: SiLU * up rows hold both halves.
@@ -329,7 +348,8 @@ __global__ void __launch_bounds__(PipeBounds<CH, kMode>::kMaxThreads,
     if (__syncthreads_or(!ok)) aborted = true;
   }
   constexpr bool kCalib = kMode == kModeColMax;
-  constexpr bool kRowMax = kMode == kModeRowQuant || kMode == kModeTensorMax || kGLU;
+  constexpr bool kF8 = kMode == kModeRowQuantF8;
+  constexpr bool kRowMax = kMode == kModeRowQuant || kMode == kModeTensorMax || kGLU || kF8;
   float cta_max = 0.0f;  // tensor-max mode, thread 0
   // fixed-step mode: the one step, from the given max |y|
   float fstep = 0.0f, frstep = 0.0f;
@@ -544,6 +564,21 @@ __global__ void __launch_bounds__(PipeBounds<CH, kMode>::kMaxThreads,
 
       if constexpr (kMode == kModeTensorMax) {
         if (t == 0) cta_max = fmaxf(cta_max, am);
+      } else if constexpr (kF8) {
+        // ---- per-token FP8 quantisation: step = fl32(max / 448); a zero or
+        // subnormal step makes the row all zero codes with step 0
+        float step = __fdiv_rn(am, 448.0f);
+        if (!(step >= FLT_MIN)) step = 0.0f;
+        const float inv = step > 0.0f ? __frcp_rn(step) : 0.0f;
+        if (t == 0) scale[row] = step;
+        int8_t* qrow = q + row * static_cast<int64_t>(K);
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+          const int ch = t + c * T;
+          if (!kFull && ch >= nchunks) continue;
+          *reinterpret_cast<uint2*>(qrow + ch * kChunk) =
+              step > 0.0f ? codes8_f8(v[c], inv) : make_uint2(0u, 0u);
+        }
       } else {
         // ---- per-token INT8 quantisation
         const float step = div127(am);
@@ -824,6 +859,16 @@ cudaError_t launch_silu_mul_quant_pipe(const void* gu, int64_t M, int I, int64_t
   a.h_out = static_cast<__nv_bfloat16*>(h_out);
   a.ldh = ldh;
   return launch_pipe_t<true, 0, 4, false, false, kModeSiluMul>(a, ps, st);
+}
+
+cudaError_t launch_norm_quant_fp8_pipe(const void* x, bool bf16, int64_t M, int K, int64_t ldx,
+                                       int norm, const float* gamma, const float* beta,
+                                       float eps, uint8_t* q, float* scale, int* err,
+                                       cudaStream_t st) {
+  if (M == 0) return cudaSuccess;
+  const RowArgs a{x, M, K, ldx, gamma, beta, eps, reinterpret_cast<int8_t*>(q), scale, nullptr,
+                  err};
+  return launch_rows<kModeRowQuantF8>(a, bf16, norm, st);
 }
 
 }  // namespace sq

@@ -114,6 +114,17 @@ __device__ __forceinline__ void mma_i8(uint32_t tmem_d, uint64_t adesc, uint64_t
       : "memory");
 }
 
+// The same MMA on FP8 operands (e4m3 x e4m3 -> fp32 accumulator).
+__device__ __forceinline__ void mma_f8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive once on an mbarrier when all tcgen05 ops issued so far by this
 // thread have completed.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
@@ -222,6 +233,16 @@ __device__ __forceinline__ void mma_i8_pair(uint32_t tmem_d, uint64_t adesc, uin
       : "memory");
 }
 
+__device__ __forceinline__ void mma_f8_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive once on an mbarrier (cluster address, either CTA of the pair) when
 // the pair MMAs issued so far by this thread have completed.
 __device__ __forceinline__ void mma_commit_pair(uint32_t bar_cluster) {
@@ -255,6 +276,17 @@ __host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {
   return (2u << 4)                                  // accumulator format S32
          | (1u << 7)                                // A: signed 8-bit
          | (1u << 10)                               // B: signed 8-bit
+         | (static_cast<uint32_t>(N >> 3) << 17)    // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
+}
+
+// Instruction descriptor for kind::f8f6f4 with e4m3 A and B (format code 0
+// in bits 7-9 and 10-12), FP32 accumulator (format 1 in bits 4-5), both
+// operands K-major, shape M x N.
+__host__ __device__ constexpr uint32_t idesc_f8(int M, int N) {
+  return (1u << 4)                                  // accumulator format F32
+         | (0u << 7)                                // A: e4m3
+         | (0u << 10)                               // B: e4m3
          | (static_cast<uint32_t>(N >> 3) << 17)    // N / 8
          | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
 }

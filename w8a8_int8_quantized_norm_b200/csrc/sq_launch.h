@@ -99,6 +99,12 @@ cudaError_t launch_quant_given_pipe(const void* x, bool bf16, int64_t M, int K, 
                                     cudaStream_t st);
 // Per-row codes of h = SiLU(gate) * up from bf16 rows [gate (I) | up (I)],
 // h rounded to bf16 first (and stored to h_out [M, I], stride ldh, if given).
+// Norm + per-row FP8 (e4m3) codes: step = fl32(max |y| / 448), codes
+// e4m3(fl32(y * fl32(1 / step))); rows the pipeline supports only.
+cudaError_t launch_norm_quant_fp8_pipe(const void* x, bool bf16, int64_t M, int K, int64_t ldx,
+                                       int norm, const float* gamma, const float* beta,
+                                       float eps, uint8_t* q, float* scale, int* err,
+                                       cudaStream_t st);
 bool silu_mul_pipe_supported(int I);
 cudaError_t launch_silu_mul_quant_pipe(const void* gu, int64_t M, int I, int64_t ldgu,
                                        int8_t* q, float* scale, void* h_out, int64_t ldh,
@@ -128,7 +134,7 @@ cudaError_t launch_gemm(const GemmPlan& plan, const int8_t* Xq, const int8_t* Wq
                         const float* x_scale, const float* w_scale, int64_t M, int64_t N,
                         int64_t K, int epi, void* out, int64_t ldo, void* workspace,
                         int num_sms, int64_t wait_polls, int* error_word, cudaStream_t st,
-                        float* row_absmax = nullptr);
+                        float* row_absmax = nullptr, bool fp8 = false);
 int num_sms_current_device();
 
 }  // namespace sq

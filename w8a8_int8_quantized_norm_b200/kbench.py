@@ -112,6 +112,7 @@ def main(argv=None):
     ap.add_argument("--path", type=int, default=0, help="GEMM path hint (0 = auto)")
     ap.add_argument("--split", type=int, default=0, help="GEMM split-K (0 = auto)")
     ap.add_argument("--epi", choices=["bf16", "bf16_relu", "i32"], default="bf16")
+    ap.add_argument("--fp8", action="store_true", help="GEMM: e4m3 operands (kind::f8f6f4)")
     ap.add_argument("--rowmax", action="store_true",
                     help="GEMM: also reduce each output row's max |out| (prefill tiles)")
     ap.add_argument("--iters", type=int, default=50)
@@ -195,12 +196,18 @@ def main(argv=None):
         scales = (None, None) if a.epi == "i32" else (xs, wsc)
         fn = lambda: sq.w8a8_gemm_dequant(A, B, scales[0], scales[1], a.epi, out=out,
                                           path_hint=a.path, split_k=a.split, workspace=ws)
+        if a.fp8:
+            A8, B8 = A.view(torch.uint8) & 0x77, B.view(torch.uint8) & 0xf7  # finite e4m3 codes
+            fn = lambda: sq.fp8_gemm_dequant(A8, B8, scales[0], scales[1],
+                                             "f32" if a.epi == "i32" else a.epi,
+                                             out=out.view(torch.float32) if a.epi == "i32" else out,
+                                             path_hint=a.path)
         if a.rowmax:
             rm = torch.empty(M, dtype=torch.float32, device=dev)
             fn = lambda: sq.w8a8_gemm_dequant_rowmax(A, B, xs, wsc, a.epi, out=out,
                                                      row_absmax=rm, path_hint=a.path)
         shape = {"M": M, "N": N, "K": K, "path": a.path, "split": a.split, "epi": a.epi,
-                 "rowmax": a.rowmax}
+                 "rowmax": a.rowmax, "fp8": a.fp8}
         units = None
     us = _time(fn, a.iters, a.warmup, flush)
     err = sq.get_device_error()

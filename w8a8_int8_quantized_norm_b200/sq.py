@@ -25,7 +25,7 @@ STATUS_NAMES = {
 }
 SQ_F32, SQ_BF16 = 0, 1
 NORM_NONE, NORM_RMS, NORM_LAYER = 0, 1, 2
-EPI = {"bf16": 0, "bf16_relu": 1, "i32": 2}
+EPI = {"bf16": 0, "bf16_relu": 1, "i32": 2, "f32": 3}
 MAX_K = 133144
 
 # Every symbol include/sq.h declares.
@@ -36,7 +36,8 @@ EXPORTS = (
     "sq_w8a8_gemm_dequant_noalloc", "sq_w8a8_gemm_plan", "sq_norm_smooth_absmax",
     "sq_norm_smooth_quant_per_tensor", "sq_smooth_quantize_weights_per_tensor",
     "sq_w8a8_gemm_dequant_rowmax", "sq_quant_per_token_given_absmax",
-    "sq_silu_mul_quant_per_token",
+    "sq_silu_mul_quant_per_token", "sq_norm_smooth_quant_per_token_fp8",
+    "sq_smooth_quantize_weights_fp8", "sq_fp8_gemm_dequant",
 )
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -113,6 +114,10 @@ def _declare(L):
                                               _P, _I32, _P]
     L.sq_quant_per_token_given_absmax.argtypes = [_P, _I32, _I64, _I64, _I64, _P, _P, _P, _P]
     L.sq_silu_mul_quant_per_token.argtypes = [_P, _I32, _I64, _I64, _I64, _P, _P, _P, _I64, _P]
+    L.sq_norm_smooth_quant_per_token_fp8.argtypes = [_P, _I32, _I64, _I64, _I64, _I32, _P, _P,
+                                                     _F32, _P, _P, _P]
+    L.sq_smooth_quantize_weights_fp8.argtypes = [_P, _I32, _I64, _I64, _I64, _P, _P, _P, _P]
+    L.sq_fp8_gemm_dequant.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _I32, _P, _I64, _I32, _P]
     L.sq_w8a8_gemm_plan.argtypes = [_I64, _I64, _I64, _I32, _I32, ctypes.POINTER(GemmPlanInfo)]
     L.sq_set_wait_limit.argtypes = [_I64]
     L.sq_set_wait_limit.restype = None
@@ -309,6 +314,53 @@ def silu_mul_quant_per_token(gate_up: torch.Tensor, Xq=None, x_scale=None, h_out
                                              _ptr(Xq), _ptr(x_scale), _ptr(h_out), ldh,
                                              _stream(stream)), "sq_silu_mul_quant_per_token")
     return Xq, x_scale
+
+
+# ---- FP8 (e4m3) W8A8: codes are uint8 tensors holding e4m3 bytes ----------
+
+def norm_smooth_quant_per_token_fp8(x: torch.Tensor, norm: int, gamma_folded=None,
+                                    beta_folded=None, eps: float = 1e-5, Xq8=None, x_scale=None,
+                                    stream=None):
+    M, K, ld = _rows(x, "x")
+    if Xq8 is None:
+        Xq8 = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+    if x_scale is None:
+        x_scale = torch.empty(M, dtype=torch.float32, device=x.device)
+    _check(lib().sq_norm_smooth_quant_per_token_fp8(
+        _ptr(x), _dtype_code(x), M, K, ld, norm, _ptr(_vec(gamma_folded, K, "gamma_folded")),
+        _ptr(_vec(beta_folded, K, "beta_folded")), eps, _ptr(Xq8), _ptr(x_scale),
+        _stream(stream)), "sq_norm_smooth_quant_per_token_fp8")
+    return Xq8, x_scale
+
+
+def smooth_quantize_weights_fp8(W: torch.Tensor, s: Optional[torch.Tensor] = None, Wq8=None,
+                                w_scale=None, stream=None):
+    N, K, ld = _rows(W, "W")
+    if Wq8 is None:
+        Wq8 = torch.empty((N, K), dtype=torch.uint8, device=W.device)
+    if w_scale is None:
+        w_scale = torch.empty(N, dtype=torch.float32, device=W.device)
+    _check(lib().sq_smooth_quantize_weights_fp8(_ptr(W), _dtype_code(W), N, K, ld,
+                                                _ptr(_vec(s, K, "s")), _ptr(Wq8), _ptr(w_scale),
+                                                _stream(stream)), "sq_smooth_quantize_weights_fp8")
+    return Wq8, w_scale
+
+
+def fp8_gemm_dequant(Xq8: torch.Tensor, Wq8: torch.Tensor, x_scale: Optional[torch.Tensor],
+                     w_scale: Optional[torch.Tensor], epi: str = "bf16", out=None,
+                     path_hint: int = 0, stream=None) -> torch.Tensor:
+    M, K = Xq8.shape
+    N = Wq8.shape[0]
+    if Xq8.dtype != torch.uint8 or Wq8.dtype != torch.uint8 or not Xq8.is_contiguous() \
+            or not Wq8.is_contiguous() or Wq8.shape[1] != K:
+        raise ValueError("Xq8 [M,K] and Wq8 [N,K] must be contiguous uint8 (e4m3 bytes)")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float32 if epi == "f32" else torch.bfloat16,
+                          device=Xq8.device)
+    _check(lib().sq_fp8_gemm_dequant(_ptr(Xq8), _ptr(Wq8), _ptr(x_scale), _ptr(w_scale), M, N, K,
+                                     EPI[epi], _ptr(out), out.stride(0), path_hint,
+                                     _stream(stream)), "sq_fp8_gemm_dequant")
+    return out
 
 
 def smooth_quantize_weights_per_tensor(W: torch.Tensor, s: Optional[torch.Tensor] = None,
