@@ -384,7 +384,7 @@ def run_gpu(args, w):
     W = {k: to_dev(v) for k, v in inp.W.items()}
     g = {k: to_dev(v) for k, v in inp.gamma.items()}
     b = {k: to_dev(v) for k, v in inp.beta.items()}
-    blk = pipeline.Block(w, w.M, dev, args.granularity)
+    blk = pipeline.Block(w, w.M, dev, args.granularity, args.format)
     flusher = L2Flush(dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -506,11 +506,15 @@ def run_gpu(args, w):
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TOPS",
                 "frac": achieved / peak,
                 "peak_sustained": peaks.get("bf16_tflops_sustained", 0.0) * INT8_PER_BF16}
+    fp8 = args.format == "fp8"
     roof["peak_source"] = "%s (%s)" % (peak_src, "HBM copy" if decode else
-                                       "2 x bf16 cuBLAS, the nominal INT8:BF16 ratio")
-    plan = sq.gemm_plan(w.M, w.linears[0].N, w.site(w.linears[0].site).K)
+                                       "2 x bf16 cuBLAS, the nominal %s:BF16 ratio"
+                                       % ("FP8" if fp8 else "INT8"))
+    # FP8 GEMMs run whole-K tiles (split 1)
+    plan = sq.gemm_plan(w.M, w.linears[0].N, w.site(w.linears[0].site).K, 0, 1 if fp8 else 0)
     kname = sq.GemmPlanInfo.KERNELS[plan.kernel].split(" ")[0]
-    tr = profile_traffic(kname, w.name)
+    # the committed DRAM-traffic summaries cover the INT8 instantiations
+    tr = None if fp8 else profile_traffic(kname, w.name)
     roof["traffic"] = None if tr is None else tr
     roof["algorithmic_per_launch"] = (g_bytes if decode else g_ops) / g_n
     roof["kernel"] = kname
@@ -524,12 +528,13 @@ def run_gpu(args, w):
     line = {
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_max * 1e3 / args.steps,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8-e4m3" if args.format == "fp8" else "int8",
         "data": "synthetic (seeded outlier-channel activations, N(0,0.02) weights)",
         "config": {"workload": w.name, "tokens": w.M, "calib_tokens": w.M_cal, "alpha": w.alpha,
                    "linears": ["%s %dx%d" % (l.name, w.site(l.site).K, l.N) for l in w.linears],
                    "step": "calibrate + smooth scales/fold + weight quant + norm-quant + GEMM",
-                   "granularity": args.granularity,
+                   "granularity": args.granularity, "format": args.format,
                    "launch": "the whole step as one CUDA graph, replayed per timed step",
                    "l2": "flushed before every step (256 MiB written, then another 256 MiB "
                          "read so no dirty line is left to write back; not timed)",
@@ -552,7 +557,8 @@ def run_gpu(args, w):
         dist.destroy_process_group()
 
     # the oracle's baseline is the per-token path (the method's default scheme)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.granularity == "per_token":
+    if (rank == 0 and world == 1 and not args.no_cpu_baseline and args.granularity == "per_token"
+            and args.format == "int8"):
         import oracle
         oracle.build()
         full, spent, desc = oracle_sample_step(w, inp)
@@ -632,6 +638,9 @@ def main(argv=None):
                     choices=["per_token", "per_tensor_dynamic", "per_tensor_static"],
                     help="activation / weight scale sharing (per-token + per-channel, or the "
                          "per-tensor O2 / O3 levels)")
+    ap.add_argument("--format", choices=["int8", "fp8"], default="int8",
+                    help="code format: INT8 (the method as published) or FP8 e4m3 with the "
+                         "same smoothing")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -837,3 +837,71 @@ def test_fp8_gemm_rejects_int8_only_epilogues():
         sq.w8a8_gemm_dequant(A.view(torch.int8), B.view(torch.int8), None, None, "f32",
                              out=torch.empty((8, 32), dtype=torch.float32, device="cuda"))
     assert e.value.status == 1
+
+
+def _check_workload_fp8(w, rows=None, seed=0):
+    """The whole block with FP8 codes.  Offline results and every site's codes
+    are bit-exact (a site fed by a GEMM is checked stage-wise, from the GPU's
+    own bf16 output of that GEMM); each GEMM output is within the
+    accumulation bound of the exact product of the codes, plus bf16 rounding."""
+    inp_w, prep_o, prep_g = _family_state(w, seed)
+    inp = S.make_inputs(w, seed=seed, weights=False)
+    inp.W = inp_w.W
+    x = {k: to_gpu(v) for k, v in inp.x.items()}
+    blk = pipeline.Block(w, w.M, "cuda", fmt="fp8")
+    blk.prepare(prep_g["xc"], prep_g["W"], prep_g["g"], prep_g["b"])
+    out_g = blk.forward(x)
+    torch.cuda.synchronize()
+    wq = {}
+    for lin in w.linears:
+        so = prep_o["sites"][lin.site]
+        if so["s64"] is not None and scale_near_tie_channels(so["s64"]).any():
+            pytest.skip("certified smoothing-factor near-tie")
+        Wq_o, ws_o = oracle.quantize_weights_fp8(inp.W[lin.name], so["s"])
+        assert np.array_equal(blk.Wq[lin.name].cpu().numpy(), Wq_o), lin.name
+        assert np.array_equal(blk.w_scale[lin.name].cpu().numpy().view(np.uint32),
+                              ws_o.view(np.uint32))
+        wq[lin.name] = (Wq_o, ws_o)
+    rows = np.arange(w.M) if rows is None else np.asarray(rows)
+    idx = torch.from_numpy(rows).cuda()
+    for site in w.sites:
+        so = prep_o["sites"][site.name]
+        src = next((l.source for l in w.linears if l.site == site.name and l.source), None)
+        if src:
+            xs_in = bf16_bits(out_g[src][idx].contiguous())
+            if site.act == "silu_mul":
+                _, xs_in = oracle.silu_mul(xs_in)
+        else:
+            xs_in = np.ascontiguousarray(inp.x[site.name][rows])
+        Xq_o, xsc_o = oracle.norm_quant_fp8(xs_in, site.norm, so["gamma_f"], so["beta_f"], w.eps)
+        Xq_g = blk.xq[site.name][idx].cpu().numpy()
+        xsc_g = blk.xs[site.name][idx].cpu().numpy()
+        compare_rows_quant(Xq_g, xsc_g, Xq_o, xsc_o, norm_near_tie_rows(xs_in, site.norm, w.eps))
+        for lin in w.linears_of(site.name):
+            Wq_o, ws_o = wq[lin.name]
+            exact = oracle.gemm_fp8(Xq_g, Wq_o)      # the GPU's codes (equal but for ties)
+            absum = np.abs(oracle.e4m3_decode(Xq_g).astype(np.float64)) @ \
+                np.abs(oracle.e4m3_decode(Wq_o).astype(np.float64)).T
+            scale = xsc_g.astype(np.float64)[:, None] * ws_o.astype(np.float64)[None, :]
+            o_exact = exact * scale
+            if lin.relu:
+                o_exact = np.maximum(o_exact, 0.0)
+            steps = (site.K + 31) // 32
+            o = bf16_bits(out_g[lin.name][idx].contiguous())
+            o = (o.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+            tol = steps * 2.0 ** -23 * absum * scale + 2.0 ** -8 * np.abs(o_exact) + 1e-30
+            assert np.all(np.abs(o - o_exact) <= tol), lin.name
+    return blk
+
+
+def test_workload_fp8_small_smoothed_linear():
+    _check_workload_fp8(S.SMALL)
+
+
+def test_workload_fp8_opt_prefill_qkv():
+    _check_workload_fp8(S.OPT_QKV, rows=_sample_rows(S.OPT_QKV.M))
+
+
+@pytest.mark.parametrize("M", [8, 128])
+def test_workload_fp8_llama_block_decode(M):
+    _check_workload_fp8(S.WORKLOADS["llama-block-8192-decode-m%d" % M])

@@ -34,6 +34,7 @@ def _run(timer: Timer, kind: str, units: float, fn: Callable[[], None]) -> None:
 
 
 GRANULARITIES = ("per_token", "per_tensor_dynamic", "per_tensor_static")
+FORMATS = ("int8", "fp8")
 
 
 class Block:
@@ -52,14 +53,26 @@ class Block:
     activation scale per tensor -- the tensor's own max |y| (O2), or the max
     over the calibration tokens through the folded norm, fixed in ``prepare``
     (O3; a site without calibration tokens, i.e. an unsmoothed Linear input,
-    falls back to its own max)."""
+    falls back to its own max).
 
-    def __init__(self, w: Workload, M: int, device, granularity: str = "per_token"):
+    ``fmt`` = ``"fp8"`` runs the same smoothing with FP8 (e4m3) codes and the
+    kind::f8f6f4 GEMM (per-token scales only; "LLM.int8() and SmoothQuant" --
+    "example . what you get": FP8 W8A8 on FP8-capable GPUs keeps the
+    smoothing).  Code tensors are then uint8 holding e4m3 bytes."""
+
+    def __init__(self, w: Workload, M: int, device, granularity: str = "per_token",
+                 fmt: str = "int8"):
         if granularity not in GRANULARITIES:
             raise ValueError("granularity must be one of %s" % (GRANULARITIES,))
+        if fmt not in FORMATS:
+            raise ValueError("fmt must be one of %s" % (FORMATS,))
+        if fmt == "fp8" and granularity != "per_token":
+            raise ValueError("FP8 runs with per-token scales")
         self.w = w
         self.M = M
         self.granularity = granularity
+        self.fmt = fmt
+        code_dtype = torch.uint8 if fmt == "fp8" else torch.int8
         dev = torch.device(device)
         f32 = dict(dtype=torch.float32, device=dev)
         self.act_max: Dict[str, torch.Tensor] = {}
@@ -81,17 +94,17 @@ class Block:
         self.ws: Dict[str, Optional[torch.Tensor]] = {}
         for lin in w.linears:
             K = w.site(lin.site).K
-            self.Wq[lin.name] = torch.empty((lin.N, K), dtype=torch.int8, device=dev)
+            self.Wq[lin.name] = torch.empty((lin.N, K), dtype=code_dtype, device=dev)
             self.w_scale[lin.name] = torch.empty(lin.N, **f32)
             self.out[lin.name] = torch.empty((M, lin.N), dtype=torch.bfloat16, device=dev)
-            need = sq.gemm_workspace_size(M, lin.N, K, 0)
+            need = 0 if fmt == "fp8" else sq.gemm_workspace_size(M, lin.N, K, 0)
             self.ws[lin.name] = torch.empty(need, dtype=torch.uint8, device=dev) if need else None
         self.xq: Dict[str, torch.Tensor] = {}
         self.xs: Dict[str, torch.Tensor] = {}
         self.x_absmax: Dict[str, torch.Tensor] = {}  # per-tensor modes: max |y| per site
         self.static: Dict[str, bool] = {}            # O3: the site's max is calibrated
         for site in w.sites:
-            self.xq[site.name] = torch.empty((M, site.K), dtype=torch.int8, device=dev)
+            self.xq[site.name] = torch.empty((M, site.K), dtype=code_dtype, device=dev)
             self.xs[site.name] = torch.empty(M, **f32)
             self.x_absmax[site.name] = torch.zeros(1, **f32)
             self.static[site.name] = (granularity == "per_tensor_static" and site.smoothed
@@ -107,8 +120,9 @@ class Block:
         # per-tensor variants keep SiLU(gate) * up in bf16 (its tensor-wide max)
         self.h: Dict[str, torch.Tensor] = {
             site.name: torch.empty((M, site.K), dtype=torch.bfloat16, device=dev)
-            for site in w.sites if site.act == "silu_mul" and granularity != "per_token"}
-        if granularity == "per_token":
+            for site in w.sites if site.act == "silu_mul"
+            and (granularity != "per_token" or fmt == "fp8")}
+        if granularity == "per_token" and fmt == "int8":
             for lin in w.linears:
                 site = w.site(lin.site)
                 if (lin.source and not site.act and site.norm == sq.NORM_NONE
@@ -157,7 +171,13 @@ class Block:
         for lin in w.linears:
             Wl = W[lin.name]
             units = Wl.numel() * (Wl.element_size() + 1) + 4 * lin.N
-            if per_tensor:  # one more read of W for the matrix-wide max
+            if self.fmt == "fp8":
+                _run(timer, "weight_quant", units,
+                     lambda: sq.smooth_quantize_weights_fp8(Wl, self.s[lin.site],
+                                                            Wq8=self.Wq[lin.name],
+                                                            w_scale=self.w_scale[lin.name],
+                                                            stream=stream))
+            elif per_tensor:  # one more read of W for the matrix-wide max
                 _run(timer, "weight_quant", units + Wl.numel() * Wl.element_size(),
                      lambda: sq.smooth_quantize_weights_per_tensor(
                          Wl, self.s[lin.site], Wq=self.Wq[lin.name],
@@ -177,18 +197,20 @@ class Block:
         for site in w.sites:
             src = next((l.source for l in w.linears if l.site == site.name and l.source), None)
             xin = self.out[src] if src else x[site.name]
-            fused_act = site.act == "silu_mul" and self.granularity == "per_token"
+            fused_act = site.act == "silu_mul" and site.name not in self.h
             if site.act == "silu_mul":
                 # the down projection's input, SiLU(gate) * up of the merged
                 # projection's output: per-token codes in the same pass; the
                 # per-tensor variants store h and quantise it as a tensor
                 h = self.h.get(site.name)
                 gu = xin
+                # (INT8 codes: FP8 runs keep h and quantise it below, so the
+                # INT8 codes go to a scratch view of the same bytes)
+                xq_i8 = self.xq[site.name].view(torch.int8)
                 _run(timer, "silu_mul_quant",
                      gu.numel() * gu.element_size() + self.M * site.K * (1 + 2 * (h is not None))
                      + 4 * self.M,
-                     lambda: sq.silu_mul_quant_per_token(gu, self.xq[site.name],
-                                                         self.xs[site.name], h_out=h,
+                     lambda: sq.silu_mul_quant_per_token(gu, xq_i8, self.xs[site.name], h_out=h,
                                                          stream=stream))
                 if h is not None:
                     xin = h
@@ -197,6 +219,12 @@ class Block:
             gf, bf = self.gamma_f[site.name], self.beta_f[site.name]
             if fused_act:
                 pass
+            elif self.fmt == "fp8":
+                _run(timer, "norm_quant", units,
+                     lambda: sq.norm_smooth_quant_per_token_fp8(xin, site.norm, gf, bf, w.eps,
+                                                                self.xq[site.name],
+                                                                self.xs[site.name],
+                                                                stream=stream))
             elif src in self.rowmax:
                 am = self.rowmax[src]
                 _run(timer, "norm_quant", units,
@@ -220,6 +248,12 @@ class Block:
                                                              self.xs[site.name], stream=stream))
             for lin in w.linears_of(site.name):
                 def gemm(lin=lin, site=site):
+                    if self.fmt == "fp8":
+                        sq.fp8_gemm_dequant(self.xq[site.name], self.Wq[lin.name],
+                                            self.xs[site.name], self.w_scale[lin.name],
+                                            "bf16_relu" if lin.relu else "bf16",
+                                            out=self.out[lin.name], stream=stream)
+                        return
                     if lin.name in self.rowmax:
                         sq.w8a8_gemm_dequant_rowmax(
                             self.xq[site.name], self.Wq[lin.name], self.xs[site.name],
@@ -258,8 +292,8 @@ class Block:
         if self.granularity != "per_token":
             n += sum(1 for site in self.w.sites if not self.static[site.name])  # O2 max pass
         for lin in self.w.linears:
-            if lin.name in self.rowmax:
-                n += 1  # prefill tiles, one kernel (the zeroing is a memset)
+            if lin.name in self.rowmax or self.fmt == "fp8":
+                n += 1  # one kernel (FP8: whole-K tiles; row max: the zeroing is a memset)
             else:
                 n += sq.gemm_plan(self.M, lin.N, self.w.site(lin.site).K).launches
         return n
@@ -289,6 +323,6 @@ class Block:
 # Thin functional wrappers (used by tests and the smoke check).
 
 def prepare(w: Workload, x_cal, W, gamma, beta, M: Optional[int] = None, device="cuda",
-            stream=None, granularity: str = "per_token") -> Block:
-    return Block(w, w.M if M is None else M, device, granularity).prepare(x_cal, W, gamma, beta,
-                                                                           stream)
+            stream=None, granularity: str = "per_token", fmt: str = "int8") -> Block:
+    return Block(w, w.M if M is None else M, device, granularity, fmt).prepare(
+        x_cal, W, gamma, beta, stream)
