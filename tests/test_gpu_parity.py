@@ -366,6 +366,21 @@ def test_gemm_rowmax_epilogue(shape, relu, path):
     assert torch.equal(ref, out_g)
 
 
+@pytest.mark.parametrize("split", [0, 2])
+def test_decode_fixup_relu_of_negative_zero(split):
+    """The stream-K fix-up and the split-K reduction apply the same ReLU as
+    the main epilogue: a zero token scale gives +0, never -0."""
+    M, N, K = 5, 4096, 8192
+    A, B = _codes(M, K), _codes(N, K)
+    xs = (RNG.random(M) * 0.05 + 1e-3).astype(np.float32)
+    ws = (RNG.random(N) * 0.002 + 1e-5).astype(np.float32)
+    xs[2] = 0.0
+    _, out_o = oracle.epilogue(oracle.gemm_i64(A, B), xs, ws, True)
+    out = sq.w8a8_gemm_dequant(to_gpu(A), to_gpu(B), to_gpu(xs), to_gpu(ws), "bf16_relu",
+                               path_hint=2, split_k=split)
+    assert np.array_equal(bf16_bits(out), out_o)
+
+
 def test_gemm_rowmax_rejects_other_epilogues_and_decode_tiles():
     A, B = to_gpu(_codes(8, 64)), to_gpu(_codes(32, 64))
     xs, ws = torch.ones(8, device="cuda"), torch.ones(32, device="cuda")

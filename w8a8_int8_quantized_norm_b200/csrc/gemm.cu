@@ -936,7 +936,7 @@ __global__ void __launch_bounds__(BM) streamk_fixup_kernel(const Params prm, int
       static_cast<int32_t*>(prm.out)[o] = acc[j];
     } else {
       float t = __fmul_rn(__fmul_rn(__int2float_rn(acc[j]), __ldg(prm.q_scale + q0 + j)), ws);
-      if (prm.epi == SQ_EPI_BF16_RELU) t = fmaxf(t, 0.0f);
+      if (prm.epi == SQ_EPI_BF16_RELU) t = t > 0.0f ? t : 0.0f;
       static_cast<__nv_bfloat16*>(prm.out)[o] = __float2bfloat16_rn(t);
     }
   }
@@ -958,7 +958,7 @@ __global__ void splitk_reduce_kernel(const int32_t* __restrict__ partial, int sp
       static_cast<int32_t*>(out)[m * ldo + n] = acc;
     } else {
       float t = __fmul_rn(__fmul_rn(__int2float_rn(acc), x_scale[m]), w_scale[n]);
-      if (epi == SQ_EPI_BF16_RELU) t = fmaxf(t, 0.0f);
+      if (epi == SQ_EPI_BF16_RELU) t = t > 0.0f ? t : 0.0f;
       static_cast<__nv_bfloat16*>(out)[m * ldo + n] = __float2bfloat16_rn(t);
     }
   }
