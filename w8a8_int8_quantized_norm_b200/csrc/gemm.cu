@@ -221,6 +221,65 @@ __device__ __forceinline__ float acc_value(uint32_t r) {
   else return __int2float_rn(static_cast<int>(r));
 }
 
+// Prefill (tokens on the P side) bf16 epilogue of CHUNK accumulator columns
+// of row p (< P), starting at column q0, with the row's token scale xs and
+// the columns' channel scales ws.  Returns the chunk's max |bf16 out| when
+// prm.row_absmax asks for it (else 0).
+template <int CHUNK, bool kF8>
+__device__ __forceinline__ float epi_row_bf16(const Params& prm, const uint32_t (&r)[32], int p,
+                                              int q0, float xs, const float (&ws)[CHUNK]) {
+  const bool relu = prm.epi == SQ_EPI_BF16_RELU;
+  float v[CHUNK];
+#pragma unroll
+  for (int j = 0; j < CHUNK; ++j) {
+    float t = __fmul_rn(__fmul_rn(acc_value<kF8>(r[j]), xs), ws[j]);
+    if (relu) t = t > 0.0f ? t : 0.0f;  // -0 (a zero scale) becomes +0
+    v[j] = t;
+  }
+  __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(prm.out) + static_cast<int64_t>(p) * prm.ldo + q0;
+  // max |bf16 out| of the chunk, as bf16 bits (magnitudes order like ints)
+  const bool track = prm.row_absmax != nullptr;
+  uint32_t am = 0;
+  if (prm.vec_out && q0 + CHUNK <= prm.Q) {
+#pragma unroll
+    for (int j = 0; j < CHUNK; j += 8) {
+      uint32_t w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(v[j + 2 * i], v[j + 2 * i + 1]);
+        w[i] = *reinterpret_cast<const uint32_t*>(&h);
+        if (track) am = max(am, max(w[i] & 0x7fffu, (w[i] >> 16) & 0x7fffu));
+      }
+      *reinterpret_cast<uint4*>(dst + j) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < CHUNK; ++j)
+      if (q0 + j < prm.Q) {
+        const __nv_bfloat16 h = __float2bfloat16_rn(v[j]);
+        dst[j] = h;
+        if (track)
+          am = max(am, static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(&h)) & 0x7fffu);
+      }
+  }
+  return __uint_as_float(am << 16);
+}
+
+// The channel scales of columns q0 .. q0 + CHUNK - 1 (0 past the matrix).
+template <int CHUNK>
+__device__ __forceinline__ void load_col_scales(const Params& prm, int q0, float (&ws)[CHUNK]) {
+  if (q0 + CHUNK <= prm.Q) {
+#pragma unroll
+    for (int j = 0; j < CHUNK; j += 4) {
+      const float4 t = __ldg(reinterpret_cast<const float4*>(prm.q_scale + q0 + j));
+      ws[j] = t.x; ws[j + 1] = t.y; ws[j + 2] = t.z; ws[j + 3] = t.w;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < CHUNK; ++j) ws[j] = (q0 + j < prm.Q) ? __ldg(prm.q_scale + q0 + j) : 0.0f;
+  }
+}
+
 // Returns the chunk's max |bf16 out| when prm.row_absmax asks for it (else 0).
 template <int CHUNK, bool kF8 = false>
 __device__ __forceinline__ float store_chunk(const Params& prm, const uint32_t (&r)[32], int p,
@@ -269,50 +328,8 @@ __device__ __forceinline__ float store_chunk(const Params& prm, const uint32_t (
     // token scale for this row, channel scale per column
     const float xs = __ldg(prm.p_scale + p);
     float ws[CHUNK];
-    if (q0 + CHUNK <= prm.Q) {
-#pragma unroll
-      for (int j = 0; j < CHUNK; j += 4) {
-        const float4 t = __ldg(reinterpret_cast<const float4*>(prm.q_scale + q0 + j));
-        ws[j] = t.x; ws[j + 1] = t.y; ws[j + 2] = t.z; ws[j + 3] = t.w;
-      }
-    } else {
-#pragma unroll
-      for (int j = 0; j < CHUNK; ++j) ws[j] = (q0 + j < prm.Q) ? __ldg(prm.q_scale + q0 + j) : 0.0f;
-    }
-    float v[CHUNK];
-#pragma unroll
-    for (int j = 0; j < CHUNK; ++j) {
-      float t = __fmul_rn(__fmul_rn(acc_value<kF8>(r[j]), xs), ws[j]);
-      if (relu) t = t > 0.0f ? t : 0.0f;  // -0 (a zero scale) becomes +0
-      v[j] = t;
-    }
-    __nv_bfloat16* dst = o + static_cast<int64_t>(p) * prm.ldo + q0;
-    // max |bf16 out| of the chunk, as bf16 bits (magnitudes order like ints)
-    const bool track = prm.row_absmax != nullptr;
-    uint32_t am = 0;
-    if (prm.vec_out && q0 + CHUNK <= prm.Q) {
-#pragma unroll
-      for (int j = 0; j < CHUNK; j += 8) {
-        uint32_t w[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const __nv_bfloat162 h = __floats2bfloat162_rn(v[j + 2 * i], v[j + 2 * i + 1]);
-          w[i] = *reinterpret_cast<const uint32_t*>(&h);
-          if (track) am = max(am, max(w[i] & 0x7fffu, (w[i] >> 16) & 0x7fffu));
-        }
-        *reinterpret_cast<uint4*>(dst + j) = make_uint4(w[0], w[1], w[2], w[3]);
-      }
-    } else {
-#pragma unroll
-      for (int j = 0; j < CHUNK; ++j)
-        if (q0 + j < prm.Q) {
-          const __nv_bfloat16 h = __float2bfloat16_rn(v[j]);
-          dst[j] = h;
-          if (track)
-            am = max(am, static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(&h)) & 0x7fffu);
-        }
-    }
-    return __uint_as_float(am << 16);
+    load_col_scales<CHUNK>(prm, q0, ws);
+    return epi_row_bf16<CHUNK, kF8>(prm, r, p, q0, xs, ws);
   } else {
     // channel scale for this row (weight row p), token scale per column
     const float ws = __ldg(prm.p_scale + p);
@@ -825,6 +842,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int u = pair_id; u < prm.units; u += num_pairs) {
       int pb, qb, kb0, kb1, split;
       decode_unit(prm, u, pb, qb, kb0, kb1, split);
+      // the row's token scale, fetched before the accumulator is ready
+      const int p_row = pb * TILE_M + static_cast<int>(rank) * ROWS + quarter * 32 + lane;
+      const float xs = (prm.epi != SQ_EPI_I32_RAW && prm.epi != SQ_EPI_F32_RAW && p_row < prm.P)
+                           ? __ldg(prm.p_scale + p_row) : 0.0f;
       bool w = false;
       if (lane == 0) w = wait_phase(TFULL_BAR(acc), acc_phase, polls, abort_flag);
       w = __shfl_sync(0xffffffffu, w, 0);
@@ -835,15 +856,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int p = pb * TILE_M + static_cast<int>(rank) * ROWS + quarter * 32 + lane;
       float rmax = 0.0f;
+      const uint32_t trow = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                            static_cast<uint32_t>(acc * TN);
+      if (prm.epi == SQ_EPI_I32_RAW || prm.epi == SQ_EPI_F32_RAW) {
 #pragma unroll 1
-      for (int c = 0; c < TN / 32; ++c) {
-        uint32_t r[32];
+        for (int c = 0; c < TN / 32; ++c) {
+          uint32_t r[32];
+          __syncwarp();
+          tmem_ld_32x32b_x32(trow + static_cast<uint32_t>(c * 32), r);
+          tmem_wait_ld();
+          store_chunk<32, kF8>(prm, r, p, qb * TN + c * 32, 0, -1);
+        }
+      } else {
+        // software-pipelined: chunk c + 1's accumulator load (tensor memory)
+        // and channel scales (L2) are in flight while chunk c is converted
+        // and stored; the token scale was loaded before the accumulator wait
+        uint32_t ra[32], rb[32];
+        float wa[32], wb[32];
+        const bool row_in = p < prm.P;
         __syncwarp();
-        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                               static_cast<uint32_t>(acc * TN + c * 32);
-        tmem_ld_32x32b_x32(taddr, r);
+        tmem_ld_32x32b_x32(trow, ra);
+        load_col_scales<32>(prm, qb * TN, wa);
         tmem_wait_ld();
-        rmax = fmaxf(rmax, store_chunk<32, kF8>(prm, r, p, qb * TN + c * 32, 0, -1));
+#pragma unroll 1
+        for (int c = 0; c < TN / 32; c += 2) {
+          __syncwarp();
+          tmem_ld_32x32b_x32(trow + static_cast<uint32_t>((c + 1) * 32), rb);
+          load_col_scales<32>(prm, qb * TN + (c + 1) * 32, wb);
+          if (row_in) rmax = fmaxf(rmax, epi_row_bf16<32, kF8>(prm, ra, p, qb * TN + c * 32, xs, wa));
+          tmem_wait_ld();
+          if (c + 2 < TN / 32) {
+            __syncwarp();
+            tmem_ld_32x32b_x32(trow + static_cast<uint32_t>((c + 2) * 32), ra);
+            load_col_scales<32>(prm, qb * TN + (c + 2) * 32, wa);
+          }
+          if (row_in)
+            rmax = fmaxf(rmax, epi_row_bf16<32, kF8>(prm, rb, p, qb * TN + (c + 1) * 32, xs, wb));
+          if (c + 2 < TN / 32) tmem_wait_ld();
+        }
       }
       if (prm.row_absmax && rmax > 0.0f && p < prm.P)
         atomicMax(reinterpret_cast<unsigned int*>(prm.row_absmax) + p, __float_as_uint(rmax));
