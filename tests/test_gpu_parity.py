@@ -478,12 +478,6 @@ def test_silu_mul_quant_rejects_what_it_cannot_run():
     assert e.value.status == 2
 
 
-def test_workload_opt66b_uses_the_rowmax_epilogue():
-    blk = pipeline.Block(S.OPT66B_MLP, 256, "cuda")
-    assert set(blk.rowmax) == {"fc1"}
-    assert pipeline.Block(S.OPT66B_MLP, 64, "cuda").rowmax == {}  # decode tiles: no fusion
-
-
 # ---------------------------------------------------------------------------
 # whole workloads
 # ---------------------------------------------------------------------------
