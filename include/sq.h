@@ -138,6 +138,30 @@ sq_status sq_compute_smooth_scales(const float* act_max, const void* const* W,
                                    float* beta_folded, void* stream);
 
 /*
+ * The two halves of sq_compute_smooth_scales, for callers that overlap the
+ * weight column maxima (which need no calibration data) with calibration:
+ *
+ * sq_weight_column_max -- w_max[j] = max over the num_w weights l and their
+ * rows n of |W_l[n, j]| (the weights exactly widened to fp32).
+ *   W, N, num_w, dtype, K  as for sq_compute_smooth_scales
+ *   w_max     device [K] fp32 OUT (zeroed by the call on the stream first)
+ * Errors: SQ_ERR_INVALID_ARG, SQ_ERR_ALIGNMENT, SQ_ERR_UNSUPPORTED, SQ_ERR_CUDA.
+ */
+sq_status sq_weight_column_max(const void* const* W, const int64_t* N, int num_w, sq_dtype dtype,
+                               int64_t K, float* w_max, void* stream);
+
+/*
+ * sq_smooth_scales_from_maxima -- s, gamma_folded and beta_folded of
+ * sq_compute_smooth_scales from both maxima: act_max (sq_calibrate_absmax)
+ * and w_max (sq_weight_column_max).  s may be w_max itself (updated in place).
+ * Other arguments and errors as for sq_compute_smooth_scales.
+ */
+sq_status sq_smooth_scales_from_maxima(const float* act_max, const float* w_max, int64_t K,
+                                       double alpha, float clamp_eps, const float* gamma,
+                                       const float* beta, float* s, float* gamma_folded,
+                                       float* beta_folded, void* stream);
+
+/*
  * sq_smooth_quantize_weights -- W-hat = W diag(s), INT8 per output channel.
  * [LLMint8] "going deeper": W-hat = diag(s) W (column j of an nn.Linear
  * weight times s_j), then quantised per channel; [SQ-depth] "Granularity":

@@ -584,16 +584,22 @@ def test_workload_llama_block_decode(M):
     _check_workload(S.WORKLOADS["llama-block-8192-decode-m%d" % M])
 
 
-@pytest.mark.parametrize("wname", ["opt-prefill-rmsnorm-qkv-2048x4096x12288",
-                                   "llama-block-8192-decode-m1"])
-def test_graph_replay_matches_eager_step(wname):
-    """The benchmark replays the whole step as one CUDA graph: every buffer the
-    step writes must come out bit-identical to the eager calls' results."""
+@pytest.mark.parametrize("wname,granularity,fmt", [
+    ("opt-prefill-rmsnorm-qkv-2048x4096x12288", "per_token", "int8"),
+    ("llama-block-8192-decode-m1", "per_token", "int8"),
+    ("llama-block-8192-decode-m8", "per_tensor_static", "int8"),
+    ("llama-block-8192-decode-m8", "per_token", "fp8"),
+    ("opt66b-mlp-layernorm-fc1-relu-fc2-4096x9216x36864", "per_token", "int8")])
+def test_graph_replay_matches_eager_step(wname, granularity, fmt):
+    """The benchmark replays the whole step as one CUDA graph, with
+    independent work on a second stream: every buffer the step writes must
+    come out bit-identical to the one-stream eager calls' results, both from
+    the graph and from an eager overlapped step."""
     w = S.WORKLOADS[wname]
     inp_w, _, prep_g = _family_state(w)
     inp = S.make_inputs(w, seed=0, weights=False)
     x = {k: to_gpu(v) for k, v in inp.x.items()}
-    blk = pipeline.Block(w, w.M, "cuda")
+    blk = pipeline.Block(w, w.M, "cuda", granularity, fmt)
     blk.prepare(prep_g["xc"], prep_g["W"], prep_g["g"], prep_g["b"])
     blk.forward(x)
     torch.cuda.synchronize()
@@ -604,6 +610,13 @@ def test_graph_replay_matches_eager_step(wname):
                 if v is not None}
 
     eager = snapshot()
+    for d in (blk.out, blk.xq, blk.Wq):
+        for v in d.values():
+            v.zero_()
+    blk.step(prep_g["xc"], prep_g["W"], prep_g["g"], prep_g["b"], x)
+    torch.cuda.synchronize()
+    for key, v in snapshot().items():
+        assert torch.equal(v, eager[key]), ("step", key)
     graph = blk.capture(prep_g["xc"], prep_g["W"], prep_g["g"], prep_g["b"], x)
     for d in (blk.out, blk.xq, blk.Wq):
         for v in d.values():

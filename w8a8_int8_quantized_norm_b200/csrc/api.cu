@@ -143,6 +143,42 @@ sq_status sq_calibrate_absmax(const void* x, sq_dtype dtype, int64_t M, int64_t 
                                     beta, eps, act_max, err, as_stream(stream)));
 }
 
+sq_status sq_weight_column_max(const void* const* W, const int64_t* N, int num_w, sq_dtype dtype,
+                               int64_t K, float* w_max, void* stream) {
+  if (!W || !N || num_w < 1 || !valid_dtype(dtype) || K <= 0) return SQ_ERR_INVALID_ARG;
+  sq_status st;
+  if ((st = check_vec(w_max, true)) != SQ_OK) return st;
+  for (int l = 0; l < num_w; ++l) {
+    if ((st = check_rows(W[l], dtype, N[l], K, K)) != SQ_OK) return st;
+  }
+  cudaStream_t cs = as_stream(stream);
+  // the maxima accumulate as bit patterns (non-negative floats order like them)
+  cudaError_t e = cudaMemsetAsync(w_max, 0, static_cast<size_t>(K) * sizeof(float), cs);
+  for (int l = 0; l < num_w && e == cudaSuccess; ++l)
+    e = launch_weight_colmax(W[l], dtype == SQ_BF16, N[l], static_cast<int>(K), w_max, cs);
+  return from_cuda(e);
+}
+
+sq_status sq_smooth_scales_from_maxima(const float* act_max, const float* w_max, int64_t K,
+                                       double alpha, float clamp_eps, const float* gamma,
+                                       const float* beta, float* s, float* gamma_folded,
+                                       float* beta_folded, void* stream) {
+  if (K <= 0) return SQ_ERR_INVALID_ARG;
+  if (!(alpha >= 0.0 && alpha <= 1.0) || !(clamp_eps > 0.0f) || isinf(clamp_eps))
+    return SQ_ERR_INVALID_ARG;
+  sq_status st;
+  if ((st = check_vec(act_max, true)) != SQ_OK) return st;
+  if ((st = check_vec(w_max, true)) != SQ_OK) return st;
+  if ((st = check_vec(s, true)) != SQ_OK) return st;
+  if ((st = check_vec(gamma_folded, true)) != SQ_OK) return st;
+  if ((st = check_vec(gamma, false)) != SQ_OK) return st;
+  if ((st = check_vec(beta, false)) != SQ_OK) return st;
+  if ((st = check_vec(beta_folded, false)) != SQ_OK) return st;
+  return from_cuda(launch_smooth_finalize(act_max, w_max, s, static_cast<int>(K), alpha,
+                                          clamp_eps, gamma, beta, gamma_folded, beta_folded,
+                                          as_stream(stream)));
+}
+
 sq_status sq_compute_smooth_scales(const float* act_max, const void* const* W, const int64_t* N,
                                    int num_w, sq_dtype dtype, int64_t K, double alpha,
                                    float clamp_eps, const float* gamma, const float* beta,
@@ -161,16 +197,11 @@ sq_status sq_compute_smooth_scales(const float* act_max, const void* const* W, c
   for (int l = 0; l < num_w; ++l) {
     if ((st = check_rows(W[l], dtype, N[l], K, K)) != SQ_OK) return st;
   }
-  cudaStream_t cs = as_stream(stream);
-  // s first accumulates the weight column maxima (as bit patterns), then is
-  // overwritten with the smoothing factors
-  cudaError_t e = cudaMemsetAsync(s, 0, static_cast<size_t>(K) * sizeof(float), cs);
-  for (int l = 0; l < num_w && e == cudaSuccess; ++l)
-    e = launch_weight_colmax(W[l], dtype == SQ_BF16, N[l], static_cast<int>(K), s, cs);
-  if (e == cudaSuccess)
-    e = launch_smooth_finalize(act_max, s, static_cast<int>(K), alpha, clamp_eps, gamma, beta,
-                               gamma_folded, beta_folded, cs);
-  return from_cuda(e);
+  // s first holds the weight column maxima, then the smoothing factors
+  st = sq_weight_column_max(W, N, num_w, dtype, K, s, stream);
+  if (st != SQ_OK) return st;
+  return sq_smooth_scales_from_maxima(act_max, s, K, alpha, clamp_eps, gamma, beta, s,
+                                      gamma_folded, beta_folded, stream);
 }
 
 sq_status sq_smooth_quantize_weights(const void* W, sq_dtype dtype, int64_t N, int64_t K,

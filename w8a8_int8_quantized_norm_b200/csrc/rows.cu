@@ -281,9 +281,10 @@ __global__ void __launch_bounds__(256) weight_colmax_kernel(const void* __restri
 }
 
 // s_j = max(max(a,eps)^alpha / max(w,eps)^(1-alpha), eps) in binary64, stored
-// as binary32; gamma' = gamma / s, beta' = beta / s.  `s` holds the weight
-// column maxima on entry and the smoothing factors on exit.
-__global__ void smooth_finalize_kernel(const float* __restrict__ act_max, float* s, int K,
+// as binary32; gamma' = gamma / s, beta' = beta / s.  w = wmax[j]; `s` may be
+// `wmax` itself (each thread reads its channel before writing it).
+__global__ void smooth_finalize_kernel(const float* __restrict__ act_max, const float* wmax,
+                                       float* s, int K,
                                        double alpha, float clamp_eps,
                                        const float* __restrict__ gamma,
                                        const float* __restrict__ beta, float* __restrict__ gf,
@@ -292,7 +293,7 @@ __global__ void smooth_finalize_kernel(const float* __restrict__ act_max, float*
   if (j >= K) return;
   const double eps = static_cast<double>(clamp_eps);
   const double a = fmax(static_cast<double>(act_max[j]), eps);
-  const double w = fmax(static_cast<double>(s[j]), eps);
+  const double w = fmax(static_cast<double>(wmax[j]), eps);
   double sj = __ddiv_rn(pow(a, alpha), pow(w, __dsub_rn(1.0, alpha)));
   if (sj < eps) sj = eps;
   const float s32 = __double2float_rn(sj);
@@ -392,12 +393,12 @@ cudaError_t launch_weight_colmax(const void* W, bool bf16, int64_t N, int K, flo
   return cudaGetLastError();
 }
 
-cudaError_t launch_smooth_finalize(const float* act_max, float* s, int K, double alpha,
-                                   float clamp_eps, const float* gamma, const float* beta,
-                                   float* gf, float* bfo, cudaStream_t st) {
+cudaError_t launch_smooth_finalize(const float* act_max, const float* wmax, float* s, int K,
+                                   double alpha, float clamp_eps, const float* gamma,
+                                   const float* beta, float* gf, float* bfo, cudaStream_t st) {
   const int threads = 256;
   smooth_finalize_kernel<<<(K + threads - 1) / threads, threads, 0, st>>>(
-      act_max, s, K, alpha, clamp_eps, gamma, beta, gf, bfo);
+      act_max, wmax, s, K, alpha, clamp_eps, gamma, beta, gf, bfo);
   return cudaGetLastError();
 }
 

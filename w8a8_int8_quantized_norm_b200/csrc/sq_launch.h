@@ -114,9 +114,9 @@ cudaError_t launch_calibrate(const void* x, bool bf16, int64_t M, int K, int64_t
                              int* err, cudaStream_t st);
 cudaError_t launch_weight_colmax(const void* W, bool bf16, int64_t N, int K, float* wmax,
                                  cudaStream_t st);
-cudaError_t launch_smooth_finalize(const float* act_max, float* s, int K, double alpha,
-                                   float clamp_eps, const float* gamma, const float* beta,
-                                   float* gf, float* bfo, cudaStream_t st);
+cudaError_t launch_smooth_finalize(const float* act_max, const float* wmax, float* s, int K,
+                                   double alpha, float clamp_eps, const float* gamma,
+                                   const float* beta, float* gf, float* bfo, cudaStream_t st);
 
 // gemm.cu
 struct GemmPlan {

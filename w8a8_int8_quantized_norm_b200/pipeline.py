@@ -116,6 +116,7 @@ class Block:
         # output row's max |out| in its GEMM epilogue, so that site's
         # quantisation reads the row once with its max already known.  Only
         # on prefill tiles (the decode plan keeps its own tiles).
+        self._side = None  # second stream of `step`, created on first use
         self.rowmax: Dict[str, torch.Tensor] = {}  # source Linear -> [M] row maxima
         # per-tensor variants keep SiLU(gate) * up in bf16 (its tensor-wide max)
         self.h: Dict[str, torch.Tensor] = {
@@ -136,19 +137,44 @@ class Block:
     def prepare(self, x_cal: Dict[str, torch.Tensor], W: Dict[str, torch.Tensor],
                 gamma: Dict[str, Optional[torch.Tensor]], beta: Dict[str, Optional[torch.Tensor]],
                 stream=None, timer: Timer = None) -> "Block":
+        for site in self.w.sites:
+            self._site_scales(site, x_cal, W, gamma, beta, stream, timer)
+        for lin in self.w.linears:
+            self._weight_quant(lin, W, stream, timer)
+        return self
+
+    def _calibrate(self, site, x_cal, gamma, beta, stream, timer):
+        g, b = gamma.get(site.name), beta.get(site.name)
+        am = self.act_max[site.name]
+        xc = x_cal[site.name]
+        am.zero_()
+        _run(timer, "calibrate", xc.numel() * xc.element_size() + 4 * site.K,
+             lambda: sq.calibrate_absmax(xc, site.norm, g, b, self.w.eps, act_max=am,
+                                         stream=stream))
+
+    def _site_weights(self, site, W):
+        return [W[l.name] for l in self.w.linears_of(site.name)]
+
+    def _site_scales(self, site, x_cal, W, gamma, beta, stream, timer, calibrated=False,
+                     w_max_done=False):
+        """Smoothing factors and the folded norm of one site (calibration
+        first unless `calibrated`; the weight column maxima, already in
+        s, when `w_max_done`), then O3's static max."""
         w = self.w
-        for site in w.sites:
-            g, b = gamma.get(site.name), beta.get(site.name)
-            if site.smoothed:
-                if b is not None and self.beta_f[site.name] is None:
-                    self.beta_f[site.name] = torch.empty_like(self.gamma_f[site.name])
-                am = self.act_max[site.name]
-                xc = x_cal[site.name]
-                am.zero_()
-                _run(timer, "calibrate", xc.numel() * xc.element_size() + 4 * site.K,
-                     lambda: sq.calibrate_absmax(xc, site.norm, g, b, w.eps, act_max=am,
-                                                 stream=stream))
-                Ws = [W[l.name] for l in w.linears_of(site.name)]
+        g, b = gamma.get(site.name), beta.get(site.name)
+        if site.smoothed:
+            if b is not None and self.beta_f[site.name] is None:
+                self.beta_f[site.name] = torch.empty_like(self.gamma_f[site.name])
+            if not calibrated:
+                self._calibrate(site, x_cal, gamma, beta, stream, timer)
+            am = self.act_max[site.name]
+            Ws = self._site_weights(site, W)
+            if w_max_done:
+                sq.smooth_scales_from_maxima(am, self.s[site.name], w.alpha, w.clamp_eps, g, b,
+                                             s=self.s[site.name],
+                                             gamma_folded=self.gamma_f[site.name],
+                                             beta_folded=self.beta_f[site.name], stream=stream)
+            else:
                 _run(timer, "smooth_scales",
                      sum(t.numel() * t.element_size() for t in Ws) + 16 * site.K,
                      lambda: sq.compute_smooth_scales(am, Ws, w.alpha, w.clamp_eps, g, b,
@@ -156,117 +182,167 @@ class Block:
                                                       gamma_folded=self.gamma_f[site.name],
                                                       beta_folded=self.beta_f[site.name],
                                                       stream=stream))
-            else:
-                self.gamma_f[site.name], self.beta_f[site.name] = g, b
-            if self.static[site.name]:
-                # O3: the static max |y| of the calibration tokens through the folded norm
-                xc = x_cal[site.name]
-                am = self.x_absmax[site.name]
-                am.zero_()
-                _run(timer, "static_absmax", xc.numel() * xc.element_size(),
-                     lambda: sq.norm_smooth_absmax(xc, site.norm, self.gamma_f[site.name],
-                                                   self.beta_f[site.name], w.eps, absmax=am,
-                                                   stream=stream))
-        per_tensor = self.granularity != "per_token"
-        for lin in w.linears:
-            Wl = W[lin.name]
-            units = Wl.numel() * (Wl.element_size() + 1) + 4 * lin.N
-            if self.fmt == "fp8":
-                _run(timer, "weight_quant", units,
-                     lambda: sq.smooth_quantize_weights_fp8(Wl, self.s[lin.site],
-                                                            Wq8=self.Wq[lin.name],
-                                                            w_scale=self.w_scale[lin.name],
-                                                            stream=stream))
-            elif per_tensor:  # one more read of W for the matrix-wide max
-                _run(timer, "weight_quant", units + Wl.numel() * Wl.element_size(),
-                     lambda: sq.smooth_quantize_weights_per_tensor(
-                         Wl, self.s[lin.site], Wq=self.Wq[lin.name],
-                         w_scale=self.w_scale[lin.name], w_absmax=self.w_absmax[lin.name],
-                         stream=stream))
-            else:
-                _run(timer, "weight_quant", units,
-                     lambda: sq.smooth_quantize_weights(Wl, self.s[lin.site], Wq=self.Wq[lin.name],
+        else:
+            self.gamma_f[site.name], self.beta_f[site.name] = g, b
+        if self.static[site.name]:
+            # O3: the static max |y| of the calibration tokens through the folded norm
+            xc = x_cal[site.name]
+            am = self.x_absmax[site.name]
+            am.zero_()
+            _run(timer, "static_absmax", xc.numel() * xc.element_size(),
+                 lambda: sq.norm_smooth_absmax(xc, site.norm, self.gamma_f[site.name],
+                                               self.beta_f[site.name], w.eps, absmax=am,
+                                               stream=stream))
+
+    def _weight_quant(self, lin, W, stream, timer):
+        Wl = W[lin.name]
+        units = Wl.numel() * (Wl.element_size() + 1) + 4 * lin.N
+        if self.fmt == "fp8":
+            _run(timer, "weight_quant", units,
+                 lambda: sq.smooth_quantize_weights_fp8(Wl, self.s[lin.site],
+                                                        Wq8=self.Wq[lin.name],
                                                         w_scale=self.w_scale[lin.name],
                                                         stream=stream))
-        return self
+        elif self.granularity != "per_token":  # one more read of W for the matrix-wide max
+            _run(timer, "weight_quant", units + Wl.numel() * Wl.element_size(),
+                 lambda: sq.smooth_quantize_weights_per_tensor(
+                     Wl, self.s[lin.site], Wq=self.Wq[lin.name],
+                     w_scale=self.w_scale[lin.name], w_absmax=self.w_absmax[lin.name],
+                     stream=stream))
+        else:
+            _run(timer, "weight_quant", units,
+                 lambda: sq.smooth_quantize_weights(Wl, self.s[lin.site], Wq=self.Wq[lin.name],
+                                                    w_scale=self.w_scale[lin.name],
+                                                    stream=stream))
 
     # -- runtime rows -------------------------------------------------------
     def forward(self, x: Dict[str, torch.Tensor], stream=None, timer: Timer = None
                 ) -> Dict[str, torch.Tensor]:
+        for site in self.w.sites:
+            self._quantize_site(site, x, stream, timer)
+            self._gemms(site, stream, timer)
+        return self.out
+
+    def _source(self, site):
+        return next((l.source for l in self.w.linears if l.site == site.name and l.source), None)
+
+    def _quantize_site(self, site, x, stream, timer):
         w = self.w
-        for site in w.sites:
-            src = next((l.source for l in w.linears if l.site == site.name and l.source), None)
-            xin = self.out[src] if src else x[site.name]
-            fused_act = site.act == "silu_mul" and site.name not in self.h
-            if site.act == "silu_mul":
-                # the down projection's input, SiLU(gate) * up of the merged
-                # projection's output: per-token codes in the same pass; the
-                # per-tensor variants store h and quantise it as a tensor
-                h = self.h.get(site.name)
-                gu = xin
-                # (INT8 codes: FP8 runs keep h and quantise it below, so the
-                # INT8 codes go to a scratch view of the same bytes)
-                xq_i8 = self.xq[site.name].view(torch.int8)
-                _run(timer, "silu_mul_quant",
-                     gu.numel() * gu.element_size() + self.M * site.K * (1 + 2 * (h is not None))
-                     + 4 * self.M,
-                     lambda: sq.silu_mul_quant_per_token(gu, xq_i8, self.xs[site.name], h_out=h,
-                                                         stream=stream))
-                if h is not None:
-                    xin = h
-            nparam = (self.gamma_f[site.name] is not None) + (self.beta_f[site.name] is not None)
-            units = xin.numel() * (xin.element_size() + 1) + 4 * self.M + 4 * site.K * nparam
-            gf, bf = self.gamma_f[site.name], self.beta_f[site.name]
-            if fused_act:
-                pass
-            elif self.fmt == "fp8":
-                _run(timer, "norm_quant", units,
-                     lambda: sq.norm_smooth_quant_per_token_fp8(xin, site.norm, gf, bf, w.eps,
-                                                                self.xq[site.name],
-                                                                self.xs[site.name],
-                                                                stream=stream))
-            elif src in self.rowmax:
-                am = self.rowmax[src]
-                _run(timer, "norm_quant", units,
-                     lambda: sq.quant_per_token_given_absmax(xin, am, self.xq[site.name],
-                                                             self.xs[site.name], stream=stream))
-            elif self.granularity == "per_token":
-                _run(timer, "norm_quant", units,
-                     lambda: sq.norm_smooth_quant_per_token(xin, site.norm, gf, bf, w.eps,
+        src = self._source(site)
+        xin = self.out[src] if src else x[site.name]
+        fused_act = site.act == "silu_mul" and site.name not in self.h
+        if site.act == "silu_mul":
+            # the down projection's input, SiLU(gate) * up of the merged
+            # projection's output: per-token codes in the same pass; the
+            # per-tensor variants store h and quantise it as a tensor
+            h = self.h.get(site.name)
+            gu = xin
+            # (INT8 codes: FP8 runs keep h and quantise it below, so the
+            # INT8 codes go to a scratch view of the same bytes)
+            xq_i8 = self.xq[site.name].view(torch.int8)
+            _run(timer, "silu_mul_quant",
+                 gu.numel() * gu.element_size() + self.M * site.K * (1 + 2 * (h is not None))
+                 + 4 * self.M,
+                 lambda: sq.silu_mul_quant_per_token(gu, xq_i8, self.xs[site.name], h_out=h,
+                                                     stream=stream))
+            if h is not None:
+                xin = h
+        nparam = (self.gamma_f[site.name] is not None) + (self.beta_f[site.name] is not None)
+        units = xin.numel() * (xin.element_size() + 1) + 4 * self.M + 4 * site.K * nparam
+        gf, bf = self.gamma_f[site.name], self.beta_f[site.name]
+        if fused_act:
+            return
+        if self.fmt == "fp8":
+            _run(timer, "norm_quant", units,
+                 lambda: sq.norm_smooth_quant_per_token_fp8(xin, site.norm, gf, bf, w.eps,
                                                             self.xq[site.name],
                                                             self.xs[site.name], stream=stream))
+        elif src in self.rowmax:
+            am = self.rowmax[src]
+            _run(timer, "norm_quant", units,
+                 lambda: sq.quant_per_token_given_absmax(xin, am, self.xq[site.name],
+                                                         self.xs[site.name], stream=stream))
+        elif self.granularity == "per_token":
+            _run(timer, "norm_quant", units,
+                 lambda: sq.norm_smooth_quant_per_token(xin, site.norm, gf, bf, w.eps,
+                                                        self.xq[site.name],
+                                                        self.xs[site.name], stream=stream))
+        else:
+            am = self.x_absmax[site.name]
+            if not self.static[site.name]:  # O2: this tensor's own max first
+                am.zero_()
+                _run(timer, "absmax", xin.numel() * xin.element_size() + 4 * site.K * nparam,
+                     lambda: sq.norm_smooth_absmax(xin, site.norm, gf, bf, w.eps, absmax=am,
+                                                   stream=stream))
+            _run(timer, "norm_quant", units,
+                 lambda: sq.norm_smooth_quant_per_tensor(xin, site.norm, am, gf, bf, w.eps,
+                                                         self.xq[site.name],
+                                                         self.xs[site.name], stream=stream))
+
+    def _gemms(self, site, stream, timer):
+        for lin in self.w.linears_of(site.name):
+            def gemm(lin=lin, site=site):
+                if self.fmt == "fp8":
+                    sq.fp8_gemm_dequant(self.xq[site.name], self.Wq[lin.name],
+                                        self.xs[site.name], self.w_scale[lin.name],
+                                        "bf16_relu" if lin.relu else "bf16",
+                                        out=self.out[lin.name], stream=stream)
+                    return
+                if lin.name in self.rowmax:
+                    sq.w8a8_gemm_dequant_rowmax(
+                        self.xq[site.name], self.Wq[lin.name], self.xs[site.name],
+                        self.w_scale[lin.name], "bf16_relu" if lin.relu else "bf16",
+                        out=self.out[lin.name], row_absmax=self.rowmax[lin.name],
+                        stream=stream)
+                    return
+                sq.w8a8_gemm_dequant(self.xq[site.name], self.Wq[lin.name],
+                                     self.xs[site.name], self.w_scale[lin.name],
+                                     "bf16_relu" if lin.relu else "bf16",
+                                     out=self.out[lin.name], workspace=self.ws[lin.name],
+                                     stream=stream)
+            _run(timer, "gemm", 2.0 * self.M * lin.N * site.K, gemm)
+
+    # -- the whole step, independent work on two streams ----------------------
+    def step(self, x_cal, W, gamma, beta, x) -> Dict[str, torch.Tensor]:
+        """``prepare`` then ``forward`` (the same kernels, the same results),
+        with work that does not depend on each other run concurrently on a
+        second stream: calibration beside the weight column maxima, and the
+        weight quantisation beside the quantisation of the block's input
+        sites.  Both streams join the current one before the GEMMs and at the
+        end, so the step is ordered like one stream to its caller (and can be
+        captured in a CUDA graph)."""
+        main = torch.cuda.current_stream()
+        if self._side is None:
+            self._side = torch.cuda.Stream()
+        side = self._side
+        w = self.w
+        smoothed = [site for site in w.sites if site.smoothed]
+        # calibration on the side stream, weight column maxima on this one
+        side.wait_stream(main)
+        with torch.cuda.stream(side):
+            for site in smoothed:
+                self._calibrate(site, x_cal, gamma, beta, None, None)
+        for site in smoothed:
+            sq.weight_column_max(self._site_weights(site, W), w_max=self.s[site.name])
+        main.wait_stream(side)
+        for site in w.sites:
+            self._site_scales(site, x_cal, W, gamma, beta, None, None, calibrated=True,
+                              w_max_done=True)
+        # weights on the side stream, the input sites' codes on this one
+        side.wait_stream(main)
+        with torch.cuda.stream(side):
+            for lin in w.linears:
+                self._weight_quant(lin, W, None, None)
+        inputs = [site for site in w.sites if self._source(site) is None]
+        for site in inputs:
+            self._quantize_site(site, x, None, None)
+        main.wait_stream(side)
+        for site in w.sites:
+            if site in inputs:
+                self._gemms(site, None, None)
             else:
-                am = self.x_absmax[site.name]
-                if not self.static[site.name]:  # O2: this tensor's own max first
-                    am.zero_()
-                    _run(timer, "absmax", xin.numel() * xin.element_size() + 4 * site.K * nparam,
-                         lambda: sq.norm_smooth_absmax(xin, site.norm, gf, bf, w.eps, absmax=am,
-                                                       stream=stream))
-                _run(timer, "norm_quant", units,
-                     lambda: sq.norm_smooth_quant_per_tensor(xin, site.norm, am, gf, bf, w.eps,
-                                                             self.xq[site.name],
-                                                             self.xs[site.name], stream=stream))
-            for lin in w.linears_of(site.name):
-                def gemm(lin=lin, site=site):
-                    if self.fmt == "fp8":
-                        sq.fp8_gemm_dequant(self.xq[site.name], self.Wq[lin.name],
-                                            self.xs[site.name], self.w_scale[lin.name],
-                                            "bf16_relu" if lin.relu else "bf16",
-                                            out=self.out[lin.name], stream=stream)
-                        return
-                    if lin.name in self.rowmax:
-                        sq.w8a8_gemm_dequant_rowmax(
-                            self.xq[site.name], self.Wq[lin.name], self.xs[site.name],
-                            self.w_scale[lin.name], "bf16_relu" if lin.relu else "bf16",
-                            out=self.out[lin.name], row_absmax=self.rowmax[lin.name],
-                            stream=stream)
-                        return
-                    sq.w8a8_gemm_dequant(self.xq[site.name], self.Wq[lin.name],
-                                         self.xs[site.name], self.w_scale[lin.name],
-                                         "bf16_relu" if lin.relu else "bf16",
-                                         out=self.out[lin.name], workspace=self.ws[lin.name],
-                                         stream=stream)
-                _run(timer, "gemm", 2.0 * self.M * lin.N * site.K, gemm)
+                self._quantize_site(site, x, None, None)
+                self._gemms(site, None, None)
         return self.out
 
     # -- launch accounting ---------------------------------------------------
@@ -299,24 +375,34 @@ class Block:
         return n
 
     # -- CUDA graph ----------------------------------------------------------
-    def capture(self, x_cal, W, gamma, beta, x, timer: Timer = None, warmup: int = 1):
-        """Records one whole step (``prepare`` then ``forward``) into a CUDA
-        graph and returns it; ``graph.replay()`` reruns every kernel of the
-        step on the current stream with no host work per kernel.  The step's
-        tensors must stay where they are between replays (the graph holds their
-        addresses).  ``timer`` hooks are captured too (e.g. CUDA event records,
-        which then time each call inside every replay)."""
+    def capture(self, x_cal, W, gamma, beta, x, timer: Timer = None, warmup: int = 1,
+                overlap: bool = True):
+        """Records one whole step into a CUDA graph and returns it;
+        ``graph.replay()`` reruns every kernel of the step on the current
+        stream with no host work per kernel.  With ``overlap`` the step is
+        ``step`` (independent work on a second stream, joined inside the
+        graph); otherwise ``prepare`` then ``forward`` in one stream, with the
+        ``timer`` hooks captured too (e.g. CUDA event records, which then time
+        each call inside every replay).  The step's tensors must stay where
+        they are between replays (the graph holds their addresses)."""
+        overlap = overlap and timer is None
         side = torch.cuda.Stream()
         side.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(side):  # first use of each kernel outside the capture
             for _ in range(warmup):
-                self.prepare(x_cal, W, gamma, beta)
-                self.forward(x)
+                if overlap:
+                    self.step(x_cal, W, gamma, beta, x)
+                else:
+                    self.prepare(x_cal, W, gamma, beta)
+                    self.forward(x)
         torch.cuda.current_stream().wait_stream(side)
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
-            self.prepare(x_cal, W, gamma, beta, timer=timer)
-            self.forward(x, timer=timer)
+            if overlap:
+                self.step(x_cal, W, gamma, beta, x)
+            else:
+                self.prepare(x_cal, W, gamma, beta, timer=timer)
+                self.forward(x, timer=timer)
         return graph
 
 

@@ -37,7 +37,8 @@ EXPORTS = (
     "sq_norm_smooth_quant_per_tensor", "sq_smooth_quantize_weights_per_tensor",
     "sq_w8a8_gemm_dequant_rowmax", "sq_quant_per_token_given_absmax",
     "sq_silu_mul_quant_per_token", "sq_norm_smooth_quant_per_token_fp8",
-    "sq_smooth_quantize_weights_fp8", "sq_fp8_gemm_dequant",
+    "sq_smooth_quantize_weights_fp8", "sq_fp8_gemm_dequant", "sq_weight_column_max",
+    "sq_smooth_scales_from_maxima",
 )
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -118,6 +119,8 @@ def _declare(L):
                                                      _F32, _P, _P, _P]
     L.sq_smooth_quantize_weights_fp8.argtypes = [_P, _I32, _I64, _I64, _I64, _P, _P, _P, _P]
     L.sq_fp8_gemm_dequant.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _I32, _P, _I64, _I32, _P]
+    L.sq_weight_column_max.argtypes = [_P, _P, _I32, _I32, _I64, _P, _P]
+    L.sq_smooth_scales_from_maxima.argtypes = [_P, _P, _I64, _F64, _F32, _P, _P, _P, _P, _P, _P]
     L.sq_w8a8_gemm_plan.argtypes = [_I64, _I64, _I64, _I32, _I32, ctypes.POINTER(GemmPlanInfo)]
     L.sq_set_wait_limit.argtypes = [_I64]
     L.sq_set_wait_limit.restype = None
@@ -219,6 +222,44 @@ def compute_smooth_scales(act_max: torch.Tensor, weights: Sequence[torch.Tensor]
                                           float(alpha), clamp_eps, _ptr(_vec(gamma, K, "gamma")),
                                           _ptr(_vec(beta, K, "beta")), _ptr(s), _ptr(gf), _ptr(bf),
                                           _stream(stream)), "sq_compute_smooth_scales")
+    return s, gf, bf
+
+
+def weight_column_max(weights: Sequence[torch.Tensor], w_max=None, stream=None) -> torch.Tensor:
+    """max over the weights and their rows of |W[n, j]|, per input column j."""
+    K = weights[0].shape[1]
+    dt = _dtype_code(weights[0])
+    for w in weights:
+        _rows(w, "W")
+        if not w.is_contiguous() or w.shape[1] != K or _dtype_code(w) != dt:
+            raise ValueError("weights must be contiguous [N, K] of one dtype")
+    ptrs = (ctypes.c_void_p * len(weights))(*[w.data_ptr() for w in weights])
+    ns = (ctypes.c_int64 * len(weights))(*[w.shape[0] for w in weights])
+    if w_max is None:
+        w_max = torch.empty(K, dtype=torch.float32, device=weights[0].device)
+    _check(lib().sq_weight_column_max(ctypes.cast(ptrs, ctypes.c_void_p),
+                                      ctypes.cast(ns, ctypes.c_void_p), len(weights), dt, K,
+                                      _ptr(_vec(w_max, K, "w_max")), _stream(stream)),
+           "sq_weight_column_max")
+    return w_max
+
+
+def smooth_scales_from_maxima(act_max: torch.Tensor, w_max: torch.Tensor, alpha: float,
+                              clamp_eps: float = 1e-5, gamma=None, beta=None, s=None,
+                              gamma_folded=None, beta_folded=None, stream=None):
+    """s, gamma / s and beta / s from the two maxima (s may be w_max)."""
+    K = act_max.numel()
+    dev = act_max.device
+    s = torch.empty(K, dtype=torch.float32, device=dev) if s is None else s
+    gf = torch.empty(K, dtype=torch.float32, device=dev) if gamma_folded is None else gamma_folded
+    bf = None
+    if beta is not None:
+        bf = torch.empty(K, dtype=torch.float32, device=dev) if beta_folded is None else beta_folded
+    _check(lib().sq_smooth_scales_from_maxima(
+        _ptr(_vec(act_max, K, "act_max")), _ptr(_vec(w_max, K, "w_max")), K, float(alpha),
+        clamp_eps, _ptr(_vec(gamma, K, "gamma")), _ptr(_vec(beta, K, "beta")),
+        _ptr(_vec(s, K, "s")), _ptr(_vec(gf, K, "gamma_folded")),
+        _ptr(_vec(bf, K, "beta_folded")), _stream(stream)), "sq_smooth_scales_from_maxima")
     return s, gf, bf
 
 
