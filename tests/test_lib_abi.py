@@ -218,3 +218,32 @@ def test_fp8_calls_reject_bad_arguments(L):
     w = L.sq_smooth_quantize_weights_fp8
     assert w(A16, 1, 4, 64, 64, None, None, A16, None) == 1
     assert w(A16, 1, 4, 64, 64, A8, A16, A16, None) == 3
+
+
+def test_split_smoothing_calls_reject_bad_arguments(L):
+    ns = (ctypes.c_int64 * 1)(64)
+    ws = (ctypes.c_void_p * 1)(0x10000)
+    P = ctypes.cast(ws, ctypes.c_void_p)
+    Nn = ctypes.cast(ns, ctypes.c_void_p)
+    cm = L.sq_weight_column_max
+    assert cm(None, Nn, 1, 1, 64, A16, None) == 1
+    assert cm(P, Nn, 0, 1, 64, A16, None) == 1      # no weights
+    assert cm(P, Nn, 1, 7, 64, A16, None) == 1      # dtype
+    assert cm(P, Nn, 1, 1, 64, None, None) == 1     # w_max
+    assert cm(P, Nn, 1, 1, 64, A8, None) == 3
+    assert cm(P, Nn, 1, 1, 40, A16, None) == 3      # K % 16
+    fm = L.sq_smooth_scales_from_maxima
+
+    def fin(am=A16, wm=A16, K=64, alpha=0.5, eps=1e-5, g=None, b=None, s=A16, gf=A16, bf=None):
+        return fm(am, wm, K, alpha, eps, g, b, s, gf, bf, None)
+
+    assert fin(alpha=1.5) == 1
+    assert fin(alpha=float("nan")) == 1
+    assert fin(eps=0.0) == 1
+    assert fin(K=0) == 1
+    assert fin(am=None) == 1
+    assert fin(wm=None) == 1
+    assert fin(s=None) == 1
+    assert fin(gf=None) == 1
+    assert fin(wm=A8) == 3
+    assert fin(g=A8) == 3
