@@ -22,6 +22,22 @@
  *      out = acc * scale_token[i] * scale_channel[j] emitted as bf16
  *      ([SQ-depth] "Granularity"; "The problem SmoothQuant solves").
  *
+ * Around that path:
+ *   - inputs with no norm in front, still quantised per token ([SQ-depth]
+ *     "Where the scales go in a decoder block"): a ReLU GEMM output whose row
+ *     maxima the GEMM epilogue reduces (sq_w8a8_gemm_dequant_rowmax, then
+ *     sq_quant_per_token_given_absmax), and SiLU(gate) * up of a merged
+ *     gate/up projection quantised in one pass (sq_silu_mul_quant_per_token);
+ *   - one scale per tensor (the O2 / O3 levels of [SQ-depth] "Granularity"):
+ *     sq_norm_smooth_absmax, sq_norm_smooth_quant_per_tensor,
+ *     sq_smooth_quantize_weights_per_tensor;
+ *   - FP8 (e4m3) codes with the same smoothing ([LLMint8] "example . what you
+ *     get"): sq_norm_smooth_quant_per_token_fp8, sq_smooth_quantize_weights_fp8,
+ *     sq_fp8_gemm_dequant;
+ *   - planning and allocation-free variants: sq_w8a8_gemm_plan,
+ *     sq_w8a8_gemm_workspace_size, sq_w8a8_gemm_dequant_noalloc; the two
+ *     halves of step 2 (sq_weight_column_max, sq_smooth_scales_from_maxima).
+ *
  * Conventions shared by every call
  * --------------------------------
  * - Layout: activations are row-major [M, K] (M tokens, K input channels) with
