@@ -33,7 +33,7 @@
  *     sq_smooth_quantize_weights_per_tensor;
  *   - FP8 (e4m3) codes with the same smoothing ([LLMint8] "example . what you
  *     get"): sq_norm_smooth_quant_per_token_fp8, sq_smooth_quantize_weights_fp8,
- *     sq_fp8_gemm_dequant;
+ *     sq_silu_mul_quant_per_token_fp8, sq_fp8_gemm_dequant;
  *   - planning and allocation-free variants: sq_w8a8_gemm_plan,
  *     sq_w8a8_gemm_workspace_size, sq_w8a8_gemm_dequant_noalloc; the two
  *     halves of step 2 (sq_weight_column_max, sq_smooth_scales_from_maxima).
@@ -352,6 +352,18 @@ sq_status sq_fp8_gemm_dequant(const uint8_t* Xq8, const uint8_t* Wq8, const floa
 sq_status sq_silu_mul_quant_per_token(const void* gate_up, sq_dtype dtype, int64_t M, int64_t I,
                                       int64_t ld_gu, int8_t* Xq, float* x_scale, void* h_out,
                                       int64_t ld_h, void* stream);
+
+/*
+ * sq_silu_mul_quant_per_token_fp8 -- sq_silu_mul_quant_per_token with FP8
+ * (e4m3) codes: h as there, then the per-token FP8 quantisation of
+ * sq_norm_smooth_quant_per_token_fp8 (step = fl32(max |h| / 448), codes
+ * e4m3(fl32(h * fl32(1 / step)))).  Xq8 device [M, I] e4m3 bytes OUT.
+ * Other arguments, limits and errors as for sq_silu_mul_quant_per_token.
+ */
+sq_status sq_silu_mul_quant_per_token_fp8(const void* gate_up, sq_dtype dtype, int64_t M,
+                                          int64_t I, int64_t ld_gu, uint8_t* Xq8,
+                                          float* x_scale, void* h_out, int64_t ld_h,
+                                          void* stream);
 
 /*
  * sq_smooth_quantize_weights_per_tensor -- W-hat = W diag(s) quantised with

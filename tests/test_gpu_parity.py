@@ -455,6 +455,21 @@ def test_silu_mul_quant_matches_oracle(shape):
     assert torch.equal(Xq2, Xq_g) and torch.equal(xs2, xs_g)
 
 
+@pytest.mark.parametrize("shape", [(1, 16), (17, 4096), (64, 28672), (2000, 1024)],
+                         ids=lambda s: "%dx%d" % s)
+def test_silu_mul_quant_fp8_matches_oracle(shape):
+    M, I = shape
+    gu = _gate_up(M, I, seed=4)
+    _, hb_o = oracle.silu_mul(gu)
+    Xq_o, xs_o = oracle.norm_quant_fp8(hb_o, oracle.NORM_NONE)
+    h = torch.empty((M, I), dtype=torch.bfloat16, device="cuda")
+    Xq_g, xs_g = sq.silu_mul_quant_per_token(to_gpu(gu), h_out=h, fp8=True)
+    assert Xq_g.dtype == torch.uint8
+    assert np.array_equal(bf16_bits(h), hb_o)
+    assert np.array_equal(xs_g.cpu().numpy().view(np.uint32), xs_o.view(np.uint32))
+    assert np.array_equal(Xq_g.cpu().numpy(), Xq_o)
+
+
 def test_silu_mul_quant_strided_rows():
     M, I = 37, 2048
     gu = _gate_up(M, I, seed=3)

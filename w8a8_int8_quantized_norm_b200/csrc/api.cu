@@ -365,9 +365,9 @@ sq_status sq_fp8_gemm_dequant(const uint8_t* Xq8, const uint8_t* Wq8, const floa
                                as_stream(stream), nullptr, true));
 }
 
-sq_status sq_silu_mul_quant_per_token(const void* gate_up, sq_dtype dtype, int64_t M, int64_t I,
-                                      int64_t ld_gu, int8_t* Xq, float* x_scale, void* h_out,
-                                      int64_t ld_h, void* stream) {
+static sq_status silu_mul_quant(const void* gate_up, sq_dtype dtype, int64_t M, int64_t I,
+                                int64_t ld_gu, void* Xq, float* x_scale, void* h_out,
+                                int64_t ld_h, void* stream, bool fp8) {
   if (!valid_dtype(dtype) || M < 0 || I <= 0 || ld_gu < 2 * I) return SQ_ERR_INVALID_ARG;
   if (h_out && ld_h < I) return SQ_ERR_INVALID_ARG;
   if (dtype != SQ_BF16) return SQ_ERR_UNSUPPORTED;
@@ -382,8 +382,22 @@ sq_status sq_silu_mul_quant_per_token(const void* gate_up, sq_dtype dtype, int64
   if (M == 0) return SQ_OK;
   int* err = device_error_word();
   if (!err) return SQ_ERR_CUDA;
-  return from_cuda(launch_silu_mul_quant_pipe(gate_up, M, static_cast<int>(I), ld_gu, Xq, x_scale,
-                                              h_out, ld_h, err, as_stream(stream)));
+  return from_cuda(launch_silu_mul_quant_pipe(gate_up, M, static_cast<int>(I), ld_gu,
+                                              static_cast<int8_t*>(Xq), x_scale, h_out, ld_h,
+                                              err, as_stream(stream), fp8));
+}
+
+sq_status sq_silu_mul_quant_per_token(const void* gate_up, sq_dtype dtype, int64_t M, int64_t I,
+                                      int64_t ld_gu, int8_t* Xq, float* x_scale, void* h_out,
+                                      int64_t ld_h, void* stream) {
+  return silu_mul_quant(gate_up, dtype, M, I, ld_gu, Xq, x_scale, h_out, ld_h, stream, false);
+}
+
+sq_status sq_silu_mul_quant_per_token_fp8(const void* gate_up, sq_dtype dtype, int64_t M,
+                                          int64_t I, int64_t ld_gu, uint8_t* Xq8,
+                                          float* x_scale, void* h_out, int64_t ld_h,
+                                          void* stream) {
+  return silu_mul_quant(gate_up, dtype, M, I, ld_gu, Xq8, x_scale, h_out, ld_h, stream, true);
 }
 
 sq_status sq_smooth_quantize_weights_per_tensor(const void* W, sq_dtype dtype, int64_t N,

@@ -256,22 +256,24 @@ enum RowMode : int {
   kModeGivenQuant = 4,  // per-row codes, each row's max |y| given in act_max[row]
   kModeSiluMul = 5,     // per-row codes of h = SiLU(gate) * up (rows hold [gate | up])
   kModeRowQuantF8 = 6,  // per-row step and FP8 (e4m3) codes
+  kModeSiluMulF8 = 7,   // SiLU * up rows with FP8 codes
 };
 
 // Bytes of one input row: SiLU * up rows hold both halves.
 template <int kMode>
-constexpr int kInRowFactor = kMode == kModeSiluMul ? 2 : 1;
+constexpr int kInRowFactor = (kMode == kModeSiluMul || kMode == kModeSiluMulF8) ? 2 : 1;
 
 template <int CH, int kMode>
 struct PipeBounds {
   // SiLU * up rows (at most 28928 outputs: 3616 chunks) run 4 chunks a thread
   // on up to 1024 threads: the row holds one CTA per SM (two 113 KB input
   // buffers), so its warps are the only latency hiding there is
-  static constexpr int kMaxThreads = kMode == kModeSiluMul ? 1024 : (CH <= 4 ? 512 : 640);
+  static constexpr bool kGLU = kMode == kModeSiluMul || kMode == kModeSiluMulF8;
+  static constexpr int kMaxThreads = kGLU ? 1024 : (CH <= 4 ? 512 : 640);
   // 4-chunk CTAs keep to 64 registers a thread so four 256-thread CTAs fit
   // an SM; calibration also keeps a running column max per element
   static constexpr int kMinBlocks =
-      (CH <= 4 && kMode != kModeColMax && kMode != kModeSiluMul) ? 2 : 1;
+      (CH <= 4 && kMode != kModeColMax && !kGLU) ? 2 : 1;
 };
 
 // One row per iteration, three CTA barriers per row (two when calibrating):
@@ -298,7 +300,7 @@ __global__ void __launch_bounds__(PipeBounds<CH, kMode>::kMaxThreads,
                           __nv_bfloat16* __restrict__ h_out, int64_t ldh) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int kEsz = kBF16 ? 2 : 4;
-  constexpr bool kGLU = kMode == kModeSiluMul;
+  constexpr bool kGLU = kMode == kModeSiluMul || kMode == kModeSiluMulF8;
   static_assert(!kGLU || (kBF16 && NORMK == 0 && !kGamma && !kBeta), "SiLU * up: bf16, no norm");
   const uint32_t row_bytes = static_cast<uint32_t>(K) * kEsz * kInRowFactor<kMode>;
   const uint32_t buf_stride = (row_bytes + 127u) & ~127u;
@@ -348,7 +350,7 @@ __global__ void __launch_bounds__(PipeBounds<CH, kMode>::kMaxThreads,
     if (__syncthreads_or(!ok)) aborted = true;
   }
   constexpr bool kCalib = kMode == kModeColMax;
-  constexpr bool kF8 = kMode == kModeRowQuantF8;
+  constexpr bool kF8 = kMode == kModeRowQuantF8 || kMode == kModeSiluMulF8;
   constexpr bool kRowMax = kMode == kModeRowQuant || kMode == kModeTensorMax || kGLU || kF8;
   float cta_max = 0.0f;  // tensor-max mode, thread 0
   // fixed-step mode: the one step, from the given max |y|
@@ -576,8 +578,20 @@ __global__ void __launch_bounds__(PipeBounds<CH, kMode>::kMaxThreads,
         for (int c = 0; c < CH; ++c) {
           const int ch = t + c * T;
           if (!kFull && ch >= nchunks) continue;
-          *reinterpret_cast<uint2*>(qrow + ch * kChunk) =
-              step > 0.0f ? codes8_f8(v[c], inv) : make_uint2(0u, 0u);
+          uint2 code = make_uint2(0u, 0u);
+          if (step > 0.0f) {
+            if constexpr (kGLU) {
+              float2 hv[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                hv[i] = make_float2(__uint_as_float(hbv[c][i] << 16),
+                                    __uint_as_float(hbv[c][i] & 0xffff0000u));
+              code = codes8_f8(hv, inv);
+            } else {
+              code = codes8_f8(v[c], inv);
+            }
+          }
+          *reinterpret_cast<uint2*>(qrow + ch * kChunk) = code;
         }
       } else {
         // ---- per-token INT8 quantisation
@@ -851,13 +865,14 @@ bool silu_mul_pipe_supported(int I) {
 
 cudaError_t launch_silu_mul_quant_pipe(const void* gu, int64_t M, int I, int64_t ldgu,
                                        int8_t* q, float* scale, void* h_out, int64_t ldh,
-                                       int* err, cudaStream_t st) {
+                                       int* err, cudaStream_t st, bool fp8) {
   if (M == 0) return cudaSuccess;
   PipeShape ps;
   if (!pipe_shape(I, true, false, &ps, 2)) return cudaErrorInvalidValue;
   RowArgs a{gu, M, I, ldgu, nullptr, nullptr, 0.0f, q, scale, nullptr, err};
   a.h_out = static_cast<__nv_bfloat16*>(h_out);
   a.ldh = ldh;
+  if (fp8) return launch_pipe_t<true, 0, 4, false, false, kModeSiluMulF8>(a, ps, st);
   return launch_pipe_t<true, 0, 4, false, false, kModeSiluMul>(a, ps, st);
 }
 

@@ -108,7 +108,7 @@ cudaError_t launch_norm_quant_fp8_pipe(const void* x, bool bf16, int64_t M, int 
 bool silu_mul_pipe_supported(int I);
 cudaError_t launch_silu_mul_quant_pipe(const void* gu, int64_t M, int I, int64_t ldgu,
                                        int8_t* q, float* scale, void* h_out, int64_t ldh,
-                                       int* err, cudaStream_t st);
+                                       int* err, cudaStream_t st, bool fp8 = false);
 cudaError_t launch_calibrate(const void* x, bool bf16, int64_t M, int K, int64_t ldx, int norm,
                              const float* gamma, const float* beta, float eps, float* act_max,
                              int* err, cudaStream_t st);

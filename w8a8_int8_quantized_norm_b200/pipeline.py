@@ -121,8 +121,7 @@ class Block:
         # per-tensor variants keep SiLU(gate) * up in bf16 (its tensor-wide max)
         self.h: Dict[str, torch.Tensor] = {
             site.name: torch.empty((M, site.K), dtype=torch.bfloat16, device=dev)
-            for site in w.sites if site.act == "silu_mul"
-            and (granularity != "per_token" or fmt == "fp8")}
+            for site in w.sites if site.act == "silu_mul" and granularity != "per_token"}
         if granularity == "per_token" and fmt == "int8":
             for lin in w.linears:
                 site = w.site(lin.site)
@@ -237,14 +236,12 @@ class Block:
             # per-tensor variants store h and quantise it as a tensor
             h = self.h.get(site.name)
             gu = xin
-            # (INT8 codes: FP8 runs keep h and quantise it below, so the
-            # INT8 codes go to a scratch view of the same bytes)
-            xq_i8 = self.xq[site.name].view(torch.int8)
             _run(timer, "silu_mul_quant",
                  gu.numel() * gu.element_size() + self.M * site.K * (1 + 2 * (h is not None))
                  + 4 * self.M,
-                 lambda: sq.silu_mul_quant_per_token(gu, xq_i8, self.xs[site.name], h_out=h,
-                                                     stream=stream))
+                 lambda: sq.silu_mul_quant_per_token(gu, self.xq[site.name], self.xs[site.name],
+                                                     h_out=h, stream=stream,
+                                                     fp8=self.fmt == "fp8"))
             if h is not None:
                 xin = h
         nparam = (self.gamma_f[site.name] is not None) + (self.beta_f[site.name] is not None)

@@ -38,7 +38,7 @@ EXPORTS = (
     "sq_w8a8_gemm_dequant_rowmax", "sq_quant_per_token_given_absmax",
     "sq_silu_mul_quant_per_token", "sq_norm_smooth_quant_per_token_fp8",
     "sq_smooth_quantize_weights_fp8", "sq_fp8_gemm_dequant", "sq_weight_column_max",
-    "sq_smooth_scales_from_maxima",
+    "sq_smooth_scales_from_maxima", "sq_silu_mul_quant_per_token_fp8",
 )
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -119,6 +119,8 @@ def _declare(L):
                                                      _F32, _P, _P, _P]
     L.sq_smooth_quantize_weights_fp8.argtypes = [_P, _I32, _I64, _I64, _I64, _P, _P, _P, _P]
     L.sq_fp8_gemm_dequant.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _I32, _P, _I64, _I32, _P]
+    L.sq_silu_mul_quant_per_token_fp8.argtypes = [_P, _I32, _I64, _I64, _I64, _P, _P, _P, _I64,
+                                                  _P]
     L.sq_weight_column_max.argtypes = [_P, _P, _I32, _I32, _I64, _P, _P]
     L.sq_smooth_scales_from_maxima.argtypes = [_P, _P, _I64, _F64, _F32, _P, _P, _P, _P, _P, _P]
     L.sq_w8a8_gemm_plan.argtypes = [_I64, _I64, _I64, _I32, _I32, ctypes.POINTER(GemmPlanInfo)]
@@ -335,15 +337,16 @@ def quant_per_token_given_absmax(x: torch.Tensor, row_absmax: torch.Tensor, Xq=N
 
 
 def silu_mul_quant_per_token(gate_up: torch.Tensor, Xq=None, x_scale=None, h_out=None,
-                             stream=None):
+                             stream=None, fp8: bool = False):
     """Per-token codes of h = SiLU(gate) * up from gate_up [M, 2I] (gate in the
-    first I columns).  ``h_out`` (bf16 [M, I]) also receives h when given."""
+    first I columns): INT8, or with ``fp8`` e4m3 bytes (uint8).  ``h_out``
+    (bf16 [M, I]) also receives h when given."""
     M, K2, ld = _rows(gate_up, "gate_up")
     if K2 % 2:
         raise ValueError("gate_up rows hold two halves")
     I = K2 // 2
     if Xq is None:
-        Xq = torch.empty((M, I), dtype=torch.int8, device=gate_up.device)
+        Xq = torch.empty((M, I), dtype=torch.uint8 if fp8 else torch.int8, device=gate_up.device)
     if x_scale is None:
         x_scale = torch.empty(M, dtype=torch.float32, device=gate_up.device)
     ldh = 0
@@ -351,9 +354,9 @@ def silu_mul_quant_per_token(gate_up: torch.Tensor, Xq=None, x_scale=None, h_out
         if h_out.dtype != torch.bfloat16 or tuple(h_out.shape) != (M, I):
             raise ValueError("h_out must be bf16 [M, I]")
         _, _, ldh = _rows(h_out, "h_out")
-    _check(lib().sq_silu_mul_quant_per_token(_ptr(gate_up), _dtype_code(gate_up), M, I, ld,
-                                             _ptr(Xq), _ptr(x_scale), _ptr(h_out), ldh,
-                                             _stream(stream)), "sq_silu_mul_quant_per_token")
+    call = "sq_silu_mul_quant_per_token_fp8" if fp8 else "sq_silu_mul_quant_per_token"
+    _check(getattr(lib(), call)(_ptr(gate_up), _dtype_code(gate_up), M, I, ld, _ptr(Xq),
+                                _ptr(x_scale), _ptr(h_out), ldh, _stream(stream)), call)
     return Xq, x_scale
 
 
