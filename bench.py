@@ -1,10 +1,15 @@
 #!/usr/bin/env python3
 """Benchmark of the SmoothQuant W8A8 linear path on B200 (one JSON line).
 
-A step is one pass of the whole path over one batch of synthetic input:
-calibration, smoothing factors + fold, weight smoothing + INT8 quantisation
-(the offline rows) and fused norm + per-token quantisation, INT8 GEMM with
-the dequant epilogue (the runtime rows), for every Linear of the workload.
+The default workload is the Llama-style decoder block (hidden 8192, 8 x 2048
+tokens: RMSNorm -> QKV, o_proj, RMSNorm -> gate_up, SiLU(gate)*up -> down).
+A timed step is the runtime forward of every Linear of the block: fused norm
++ per-token INT8 quantisation (or SiLU(gate)*up + quantisation), INT8 GEMM
+with the dequant epilogue; ``value`` is its throughput.  The offline rows
+(calibration, smoothing factors + fold, weight smoothing + INT8 quantisation)
+run in the same job and are reported under ``offline_prep``; the decode
+sweep (M = 1, 8, 32, 128 tokens per step on the same weights) under
+``decode``.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
   python bench.py --impl reference ...   # the CPU oracle, on a bounded sample
@@ -31,7 +36,8 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "W8A8 linear TOPS & tokens/s (prefill, decode); % of INT8 tensor peak / HBM BW"
-DEFAULT_WORKLOAD = "opt-prefill-rmsnorm-qkv-2048x4096x12288"
+DEFAULT_WORKLOAD = "llama-block-8192-prefill-16384tok"
+DECODE_TOKENS = (1, 8, 32, 128)
 L2_FLUSH_BYTES = 256 << 20
 # nominal dense INT8 : BF16 tensor throughput on B200 (4.5 : 2.25 PFLOP/s)
 INT8_PER_BF16 = 2.0
@@ -116,22 +122,39 @@ def aggregate(units_per_rank: float, seconds_per_rank: float, world: int, device
 # ---------------------------------------------------------------------------
 
 def _sample_rows(n, k, seed=11):
-    if k >= n:
+    if k is None or k >= n:
         return np.arange(n)
     return np.sort(np.random.default_rng(seed).choice(n, size=k, replace=False))
 
 
-def oracle_sample_step(w, inp, cal_rows=512, weight_elems=48 << 20, token_rows=16):
-    """One oracle step on a bounded sample: `cal_rows` calibration tokens, up
-    to `weight_elems` weight elements per Linear (whole rows) and `token_rows`
-    runtime tokens.  Each phase's time is scaled linearly to the full workload.
-    Returns (extrapolated seconds for the full step, seconds spent, text)."""
+# the oracle's sample of each workload for the CPU baseline: the two small
+# workloads run in full; the larger ones run the weight rows (K2) and the
+# calibration in full, K1 on 1024 tokens and the GEMMs on 16, each phase's
+# time scaled to the full step
+FULL_SAMPLE = dict(cal_rows=None, weight_elems=None, norm_rows=None, gemm_rows=None)
+LARGE_SAMPLE = dict(cal_rows=None, weight_elems=None, norm_rows=1024, gemm_rows=16)
+
+
+def cpu_sample_for(w):
+    return FULL_SAMPLE if w.gemm_ops() <= 4e11 else LARGE_SAMPLE
+
+
+def oracle_sample_step(w, inp, cal_rows=None, weight_elems=None, norm_rows=None, gemm_rows=None):
+    """One oracle step (the offline rows, then the forward) on a sample of
+    the workload: ``cal_rows`` calibration tokens, at most ``weight_elems``
+    weight elements per Linear (whole rows), ``norm_rows`` tokens through the
+    norm + quantisation and ``gemm_rows`` of them through the GEMMs (None =
+    all).  Each phase's time is scaled linearly to the full workload.
+    Returns (seconds for the full step, seconds spent, text, full)."""
     import oracle
     spent = 0.0
-    full = 0.0
+    est = 0.0
     prep = {}
+    extrap = False
 
     def wrows(Wl):
+        if weight_elems is None:
+            return np.arange(Wl.shape[0])
         n = max(1, min(Wl.shape[0], weight_elems // Wl.shape[1]))
         return _sample_rows(Wl.shape[0], n)
 
@@ -147,7 +170,7 @@ def oracle_sample_step(w, inp, cal_rows=512, weight_elems=48 << 20, token_rows=1
             for l in w.linears_of(site.name):
                 Wl = inp.W[l.name]
                 r = wrows(Wl)
-                Ws.append(np.ascontiguousarray(Wl[r]))
+                Ws.append(Wl if len(r) == Wl.shape[0] else np.ascontiguousarray(Wl[r]))
                 fr.append(len(r) / Wl.shape[0])
             t0 = time.perf_counter()
             am = oracle.calibrate_absmax(xcs, site.norm, g, b, w.eps)
@@ -156,64 +179,78 @@ def oracle_sample_step(w, inp, cal_rows=512, weight_elems=48 << 20, token_rows=1
             gf, bf = oracle.fold_norm(s, g, b)
             t2 = time.perf_counter()
             spent += t2 - t0
-            full += (t1 - t0) * xc.shape[0] / len(cr) + (t2 - t1) / min(fr)
+            est += (t1 - t0) * xc.shape[0] / len(cr) + (t2 - t1) / min(fr)
+            extrap |= len(cr) < xc.shape[0] or min(fr) < 1.0
         prep[site.name] = (s, gf, bf)
     lin_q = {}
     for lin in w.linears:
         Wl = inp.W[lin.name]
         r = wrows(Wl)
-        Wsub = np.ascontiguousarray(Wl[r])
+        Wsub = Wl if len(r) == Wl.shape[0] else np.ascontiguousarray(Wl[r])
         t0 = time.perf_counter()
         Wq, ws = oracle.quantize_weights(Wsub, prep[lin.site][0])
         dt = time.perf_counter() - t0
         spent += dt
-        full += dt * Wl.shape[0] / len(r)
+        est += dt * Wl.shape[0] / len(r)
+        extrap |= len(r) < Wl.shape[0]
         lin_q[lin.name] = (Wq, ws, len(r), Wl.shape[0])
-    rows = _sample_rows(w.M, token_rows)
-    R = len(rows)
-    t_rows = 0.0
+    nrows = _sample_rows(w.M, norm_rows)
+    R = len(nrows)
+    G = R if gemm_rows is None else min(R, gemm_rows)
+    extrap |= R < w.M or G < w.M
     outs = {}
     for site in w.sites:
         src = next((l.source for l in w.linears if l.site == site.name and l.source), None)
-        x = outs[src] if src else np.ascontiguousarray(inp.x[site.name][rows])
+        # a site fed by a Linear's output has the GEMM's rows only
+        x = outs[src] if src else np.ascontiguousarray(inp.x[site.name][nrows])
+        rows = x.shape[0]
         s, gf, bf = prep[site.name]
         t0 = time.perf_counter()
         if site.act == "silu_mul":
             Xq, xs, _ = oracle.silu_mul_quant(x)
         else:
             Xq, xs = oracle.norm_quant(x, site.norm, gf, bf, w.eps)
-        t_rows += time.perf_counter() - t0
+        dt = time.perf_counter() - t0
+        spent += dt
+        est += dt * w.M / rows
         for lin in w.linears_of(site.name):
             Wq, ws, n, N = lin_q[lin.name]
+            Xg = np.ascontiguousarray(Xq[:G])
             t0 = time.perf_counter()
-            acc = oracle.gemm_i64(Xq, Wq)
-            _, out = oracle.epilogue(acc, xs, ws, lin.relu)
+            acc = oracle.gemm_i64(Xg, Wq)
+            _, out = oracle.epilogue(acc, xs[:G], ws, lin.relu)
             dt = time.perf_counter() - t0
             spent += dt
-            t_rows += dt * N / n  # the GEMM scales with the output channels too
+            est += dt * (w.M / G) * (N / n)  # the GEMM scales with tokens and channels
             if any(l.source == lin.name for l in w.linears):
                 # a downstream site reads this output: it needs every channel
                 if n < N:
                     out = np.concatenate([out] * ((N + n - 1) // n), axis=1)[:, :N]
                 outs[lin.name] = np.ascontiguousarray(out)
-    spent += t_rows
-    full += t_rows * w.M / R
-    desc = ("oracle on %d of %d tokens, %d of %d calibration tokens and up to %d weight "
-            "elements per Linear, each phase extrapolated linearly to the full step" %
-            (R, w.M, min(cal_rows, w.M_cal), w.M_cal, weight_elems))
-    return full, spent, desc
+    if not extrap:
+        desc = "the oracle on the whole step (all %d tokens, %d calibration tokens, every weight)" % (
+            w.M, w.M_cal)
+    else:
+        desc = ("oracle: %d of %d calibration tokens, %s weight rows, %d of %d tokens through "
+                "norm + quantisation and %d through the GEMMs; each phase's time extrapolated "
+                "linearly to the full step" %
+                (w.M_cal if cal_rows is None else min(cal_rows, w.M_cal), w.M_cal,
+                 "all" if weight_elems is None else "up to %d elements of" % weight_elems,
+                 R, w.M, G))
+    return est, spent, desc, not extrap
 
 
 def reference_sample_sizes(w, inp, steps, budget_s=150.0):
     """Sample sizes for `steps` oracle steps to fit in about `budget_s`
     seconds: a tiny probe step measures the cost, the sizes scale from it."""
-    probe = dict(cal_rows=8, weight_elems=1 << 20, token_rows=1)
-    _, spent, _ = oracle_sample_step(w, inp, **probe)
+    probe = dict(cal_rows=8, weight_elems=1 << 20, norm_rows=1, gemm_rows=1)
+    _, spent, _, _ = oracle_sample_step(w, inp, **probe)
     per_step = max(0.05, (budget_s - spent) / max(1, steps))
     k = max(1.0, per_step / max(spent, 1e-3))
     return dict(cal_rows=int(min(w.M_cal, 8 * k)),
                 weight_elems=int(min(48 << 20, (1 << 20) * k)),
-                token_rows=int(max(1, min(16, k))))
+                norm_rows=int(max(1, min(w.M, 64 * k))),
+                gemm_rows=int(max(1, min(16, k))))
 
 
 def run_reference(args, w):
@@ -227,9 +264,9 @@ def run_reference(args, w):
     times = []
     desc = ""
     for i in range(args.warmup + args.steps):
-        full, spent, desc = oracle_sample_step(w, inp, **sizes)
+        est, spent, desc, _ = oracle_sample_step(w, inp, **sizes)
         if i >= args.warmup:
-            times.append(full)
+            times.append(est)
     t = sum(times) / len(times)
     ops = workload_ops(w)
     value = ops / t / 1e12
@@ -240,7 +277,7 @@ def run_reference(args, w):
         "data": "synthetic", "config": {"workload": w.name, "tokens": w.M},
         "tokens_per_s": w.M / t,
         "cpu_baseline": {"value": value, "unit": "TOPS", "cores": cores, "kind": "oracle",
-                         "sample": desc},
+                         "sample": desc + "; the oracle's whole step (offline rows + forward)"},
         "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -352,12 +389,159 @@ def profile_traffic(kernel: str, workload: str):
     return None
 
 
+def _to_dev(a, dev):
+    import torch
+    if a is None:
+        return None
+    t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16 \
+        else torch.from_numpy(a)
+    return t.to(dev)
+
+
+def _timed_replays(graph, n, flusher, stream):
+    """Device time (ms) of each of ``n`` replays of ``graph``, every replay
+    bracketed by CUDA events on the launching stream after an untimed L2
+    flush."""
+    import torch
+    ev = []
+    for _ in range(n):
+        flusher()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        graph.replay()
+        e1.record(stream)
+        ev.append((e0, e1))
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def _call_breakdown(run_step, n, flusher, stream, head_cycles, dev):
+    """Per library call device times: ``n`` eager steps, every call
+    bracketed by CUDA events (the ``timer`` hook of the pipeline).  Each step
+    waits behind an untimed GPU spin sized from the host's enqueue time, so
+    the queue runs ahead and no host gap enters an interval (each event
+    record still drains the stream: a few microseconds per call).  Returns
+    {kind: [calls, units, seconds]}."""
+    import torch
+    events = []
+
+    def timer(kind, units, fn):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        events.append((kind, units, e0, e1))
+
+    for i in range(n):
+        flusher()
+        torch.cuda._sleep(head_cycles)
+        run_step(timer)
+        if i % 8 == 7:
+            torch.cuda.synchronize(dev)
+    torch.cuda.synchronize(dev)
+    kinds = {}
+    for (kind, units, a, b_) in events:
+        k = kinds.setdefault(kind, [0, 0.0, 0.0])
+        k[0] += 1
+        k[1] += units
+        k[2] += a.elapsed_time(b_) / 1e3
+    return kinds
+
+
+def _row_kernels(kinds, n_steps, hbm):
+    out = {}
+    for kind, (n, units, secs) in kinds.items():
+        if kind.startswith("gemm:"):
+            continue
+        gbs = units / secs / 1e9
+        out[kind] = {"calls": n // n_steps, "ms_per_call": secs * 1e3 / n, "achieved_gbs": gbs,
+                     "frac_hbm": gbs / hbm, "bytes_per_call": units / n}
+    return out
+
+
+def _gemm_calls(w, M, kinds, peaks):
+    """Per-Linear GEMM call times: TOPS against the INT8 peak for prefill
+    shapes, algorithmic GB/s against HBM for decode shapes (M <= 128)."""
+    out = {}
+    for lin in w.linears:
+        K = w.site(lin.site).K
+        n, ops, secs = kinds["gemm:" + lin.name]
+        t = secs / n
+        d = {"shape": "%dx%dx%d" % (M, lin.N, K), "ms_per_call": t * 1e3,
+             "tops": 2.0 * M * lin.N * K / t / 1e12}
+        if M <= 128:
+            gb = gemm_bytes(M, lin.N, K)
+            d.update(bytes_per_call=gb, achieved_gbs=gb / t / 1e9,
+                     frac_hbm=gb / t / 1e9 / peaks["hbm_gbs"])
+        else:
+            d["frac_int8_peak"] = d["tops"] / (peaks["bf16_tflops"] * INT8_PER_BF16)
+        out[lin.name] = d
+    return out
+
+
+def _forward_bytes(w, M, blk):
+    """Algorithmic bytes of one forward: every GEMM's operands, scales and
+    bf16 output, and every row kernel's input read, codes written, scales and
+    norm parameters."""
+    total = 0
+    for lin in w.linears:
+        total += gemm_bytes(M, lin.N, w.site(lin.site).K)
+    for site in w.sites:
+        nparam = (blk.gamma_f[site.name] is not None) + (blk.beta_f[site.name] is not None)
+        width = 2 * site.K if site.act == "silu_mul" else site.K
+        total += M * width * 2 + M * site.K + 4 * M + 4 * site.K * nparam
+    return total
+
+
+def decode_sweep(args, w, blk, dev, stream, flusher, peaks, seed, rank):
+    """The decode configurations on the prefill block's weights: for M tokens
+    per step, the runtime forward (norm + per-token quantisation, the four
+    GEMMs) as one CUDA graph, timed like the main loop; plus each GEMM call's
+    time from eager steps.  Weight bytes dominate: every step streams all the
+    INT8 weights once."""
+    import torch
+    from w8a8_int8_quantized_norm_b200 import pipeline
+    from w8a8_int8_quantized_norm_b200 import synthetic as S
+    res = {}
+    for M in DECODE_TOKENS:
+        wd = S.WORKLOADS["llama-block-8192-decode-m%d" % M]
+        inp = S.make_inputs(wd, seed=seed, weights=False, token_seed=seed + 1000003 * rank)
+        x = {k: _to_dev(v, dev) for k, v in inp.x.items()}
+        bd = pipeline.Block(wd, M, dev, args.granularity, args.format, shared=blk)
+        graph = pipeline.capture_forward(bd, x)
+        for _ in range(3):
+            flusher()
+            graph.replay()
+        n = max(10, args.steps)
+        ms = _timed_replays(graph, n, flusher, stream)
+        t = sum(ms) / n / 1e3
+        del graph
+        kinds = _call_breakdown(lambda timer: bd.forward(x, timer=timer), min(n, 20), flusher,
+                                stream, int(2.0e9 * 200e-6), dev)
+        gemms = _gemm_calls(wd, M, kinds, peaks)
+        gb = sum(g["bytes_per_call"] for g in gemms.values())
+        gt = sum(g["ms_per_call"] for g in gemms.values()) / 1e3
+        fb = _forward_bytes(wd, M, bd)
+        res["m%d" % M] = {
+            "tokens": M, "us_per_step": t * 1e6, "tokens_per_s": M / t,
+            "tops": wd.gemm_ops() / t / 1e12, "bytes_per_step": fb,
+            "achieved_gbs": fb / t / 1e9, "frac_hbm": fb / t / 1e9 / peaks["hbm_gbs"],
+            "gemm_calls": {"achieved_gbs": gb / gt / 1e9,
+                           "frac_hbm": gb / gt / 1e9 / peaks["hbm_gbs"],
+                           "per_linear": gemms},
+            "row_kernels": _row_kernels(kinds, min(n, 20), peaks["hbm_gbs"]),
+            "launches_per_step": bd.forward_launches(),
+        }
+    return res
+
+
 def run_gpu(args, w):
     import torch
     import torch.distributed as dist
 
     from w8a8_int8_quantized_norm_b200 import pipeline, sq
-    from w8a8_int8_quantized_norm_b200 import synthetic as S
 
     world, rank, local = dist_env()
     if not torch.cuda.is_available():
@@ -371,52 +555,31 @@ def run_gpu(args, w):
     sq.lib()
 
     inp = rank_inputs(w, args.seed, rank)
-
-    def to_dev(a):
-        if a is None:
-            return None
-        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16 \
-            else torch.from_numpy(a)
-        return t.to(dev)
-
-    x = {k: to_dev(v) for k, v in inp.x.items()}
-    xc = {k: to_dev(v) for k, v in inp.x_cal.items()}
-    W = {k: to_dev(v) for k, v in inp.W.items()}
-    g = {k: to_dev(v) for k, v in inp.gamma.items()}
-    b = {k: to_dev(v) for k, v in inp.beta.items()}
+    x = {k: _to_dev(v, dev) for k, v in inp.x.items()}
+    xc = {k: _to_dev(v, dev) for k, v in inp.x_cal.items()}
+    W = {k: _to_dev(v, dev) for k, v in inp.W.items()}
+    g = {k: _to_dev(v, dev) for k, v in inp.gamma.items()}
+    b = {k: _to_dev(v, dev) for k, v in inp.beta.items()}
     blk = pipeline.Block(w, w.M, dev, args.granularity, args.format)
     flusher = L2Flush(dev)
     stream = torch.cuda.current_stream(dev)
 
-    events = []  # (kind, units, start event, end event) of every library call in a step
-
-    def timer(kind, units, fn):
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        fn()
-        e1.record(stream)
-        events.append((kind, units, e0, e1))
-
-    def step(timed):
-        blk.prepare(xc, W, g, b, timer=timer if timed else None)
-        blk.forward(x, timer=timer if timed else None)
-
-    # warm-up (eager), then the step captured once as a CUDA graph: the timed
-    # region replays it, each replay bracketed by events on the launching
-    # stream after an untimed L2 overwrite
+    # warm-up (eager), measuring the host's enqueue time of one step
     enqueue_s = 0.0
     for _ in range(args.warmup):
         flusher()
         torch.cuda.synchronize(dev)
         t0 = time.perf_counter()
-        step(True)
+        blk.prepare(xc, W, g, b)
+        blk.forward(x)
         enqueue_s = max(enqueue_s, time.perf_counter() - t0)
-        events.clear()
-    graph = blk.capture(xc, W, g, b, x)
+    # the offline rows and the runtime forward, each captured once as a graph
+    prep_graph = pipeline.capture_prepare(blk, xc, W, g, b)
+    fwd_graph = pipeline.capture_forward(blk, x)
+    prep_graph.replay()
     for _ in range(args.warmup):
         flusher()
-        graph.replay()
+        fwd_graph.replay()
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
@@ -428,125 +591,128 @@ def run_gpu(args, w):
         pci = "%08X:%02X:%02X.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
     except Exception:
         pass
+    # ---- the timed region: K forward steps (runtime rows of every Linear)
     sampler = ClockSampler(pci)
     sampler.start()
     wall0 = time.perf_counter()
-    step_ev = []
-    for _ in range(args.steps):
-        flusher()  # L2 holds nothing of the step's inputs when it starts (untimed)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        graph.replay()
-        e1.record(stream)
-        step_ev.append((e0, e1))
-    torch.cuda.synchronize(dev)
+    step_ms = _timed_replays(fwd_graph, args.steps, flusher, stream)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     wall = time.perf_counter() - wall0
-    step_ms = [a.elapsed_time(b_) for a, b_ in step_ev]
-
-    # per-call breakdown: the same step run eagerly, each call bracketed by
-    # events; every step waits behind an untimed GPU spin sized from the host's
-    # enqueue time, so the queue runs ahead and no host gap enters an interval
-    # (each event record still drains the stream: a few microseconds per call)
-    head_cycles = int(2.0e9 * (2.0 * enqueue_s + 50e-6))
-    n_calls = max(1, min(args.steps, 50))
-    for i in range(n_calls):
-        flusher()
-        torch.cuda._sleep(head_cycles)
-        step(True)
-        if i % 8 == 7:
-            torch.cuda.synchronize(dev)
-    torch.cuda.synchronize(dev)
     clocks = sampler.stop()
-    err = sq.get_device_error()
-    if err:
-        raise SystemExit("device error %s during the benchmark" % sq.status_string(err))
-    del graph
-    kinds = {}  # kind -> [calls, units, seconds]
-    for (kind, units, a, b_) in events:
-        k = kinds.setdefault(kind, [0, 0.0, 0.0])
-        k[0] += 1
-        k[1] += units
-        k[2] += a.elapsed_time(b_) / 1e3
-    calls_steps = n_calls
 
     t_rank = sum(step_ms) / 1e3
     ops = workload_ops(w)
     tops_total, t_max = aggregate(ops * args.steps, t_rank, world, dev)
     value = tops_total / 1e12
     tokens_per_s = w.M * args.steps * world / t_max
-
-    # per library call: CUDA events recorded around every call inside the graph
     peaks, peak_src = load_peaks()
-    kernels = {}
-    for kind, (n, units, secs) in kinds.items():
-        if kind == "gemm":
-            continue
-        gbs = units / secs / 1e9
-        kernels[kind] = {"calls": n // calls_steps, "ms_per_call": secs * 1e3 / n,
-                         "achieved_gbs": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
-                         "bytes_per_call": units / n}
-    # dominant kernel: the GEMM
-    g_n, g_ops, g_time = kinds["gemm"]
-    g_bytes = 0
-    for lin in w.linears:
-        g_bytes += gemm_bytes(w.M, lin.N, w.site(lin.site).K) * calls_steps
+
+    # ---- the offline rows, timed the same way (one-time work per weight set)
+    n_prep = max(3, min(args.steps, 10))
+    prep_ms = _timed_replays(prep_graph, n_prep, flusher, stream)
+    prep_t = sum(prep_ms) / n_prep / 1e3
+    del prep_graph, fwd_graph
+
+    # ---- per-call breakdown from eager steps
+    head_cycles = int(2.0e9 * (2.0 * enqueue_s + 50e-6))
+    n_calls = max(1, min(args.steps, 20))
+
+    def eager_step(timer):
+        blk.prepare(xc, W, g, b, timer=timer)
+        blk.forward(x, timer=timer)
+
+    kinds = _call_breakdown(eager_step, n_calls, flusher, stream, head_cycles, dev)
+    kernels = _row_kernels(kinds, n_calls, peaks["hbm_gbs"])
+    gemms = _gemm_calls(w, w.M, kinds, peaks)
+    prep_kinds = ("calibrate", "smooth_scales", "weight_quant", "static_absmax")
+    prep_bytes = sum(kinds[k][1] for k in prep_kinds if k in kinds) / n_calls
+
+    # dominant kernel: the GEMM call with the most work
+    dom = max(w.linears, key=lambda l: l.N * w.site(l.site).K)
+    K_dom = w.site(dom.site).K
+    n_dom, _, secs_dom = kinds["gemm:" + dom.name]
+    t_dom = secs_dom / n_dom
     decode = w.M <= 128
+    fp8 = args.format == "fp8"
     if decode:
-        achieved = g_bytes / g_time / 1e9
+        alg = gemm_bytes(w.M, dom.N, K_dom)
+        achieved = alg / t_dom / 1e9
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak}
     else:
-        achieved = g_ops / g_time / 1e12
+        alg = 2.0 * w.M * dom.N * K_dom
+        achieved = alg / t_dom / 1e12
         peak = peaks["bf16_tflops"] * INT8_PER_BF16
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TOPS",
                 "frac": achieved / peak,
                 "peak_sustained": peaks.get("bf16_tflops_sustained", 0.0) * INT8_PER_BF16}
-    fp8 = args.format == "fp8"
     roof["peak_source"] = "%s (%s)" % (peak_src, "HBM copy" if decode else
                                        "2 x bf16 cuBLAS, the nominal %s:BF16 ratio"
                                        % ("FP8" if fp8 else "INT8"))
     # FP8 GEMMs run whole-K tiles (split 1)
-    plan = sq.gemm_plan(w.M, w.linears[0].N, w.site(w.linears[0].site).K, 0, 1 if fp8 else 0)
+    plan = sq.gemm_plan(w.M, dom.N, K_dom, 0, 1 if fp8 else 0)
     kname = sq.GemmPlanInfo.KERNELS[plan.kernel].split(" ")[0]
     # the committed DRAM-traffic summaries cover the INT8 instantiations
-    tr = None if fp8 else profile_traffic(kname, w.name)
-    roof["traffic"] = None if tr is None else tr
-    roof["algorithmic_per_launch"] = (g_bytes if decode else g_ops) / g_n
+    tr = None
+    if not fp8:
+        tr = profile_traffic(kname, "%s:%s" % (w.name, dom.name))
+        if tr is None and len(w.linears) == 1:
+            tr = profile_traffic(kname, w.name)
+    roof["traffic"] = tr
+    roof["algorithmic_per_launch"] = alg
     roof["kernel"] = kname
+    roof["linear"] = "%s %dx%dx%d (M x N x K)" % (dom.name, w.M, dom.N, K_dom)
     roof["plan"] = {k: v for k, v in plan.as_dict().items() if k != "kernel"}
-    roof["launch_ms_mean"] = g_time * 1e3 / g_n
-    roof["timing"] = ("CUDA events on the launching stream around each GEMM call, in %d eager "
-                      "steps run right after the graph-timed ones (a call = the main kernel "
+    roof["launch_ms_mean"] = t_dom * 1e3
+    roof["timing"] = ("CUDA events on the launching stream around each %s GEMM call, in %d "
+                      "eager steps run right after the timed ones (a call = the main kernel "
                       "plus its fix-up kernel when the plan has one; the interval includes "
-                      "the event records' own drain)" % calls_steps)
+                      "the event records' own drain)" % (dom.name, n_calls))
 
     line = {
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_max * 1e3 / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "fp8-e4m3" if args.format == "fp8" else "int8",
+        "dtype": "fp8-e4m3" if fp8 else "int8",
         "data": "synthetic (seeded outlier-channel activations, N(0,0.02) weights)",
         "config": {"workload": w.name, "tokens": w.M, "calib_tokens": w.M_cal, "alpha": w.alpha,
                    "linears": ["%s %dx%d" % (l.name, w.site(l.site).K, l.N) for l in w.linears],
-                   "step": "calibrate + smooth scales/fold + weight quant + norm-quant + GEMM",
+                   "step": "the runtime forward of every Linear: norm + per-token quant (or "
+                           "SiLU(gate)*up + quant), INT8 GEMM with the dequant epilogue; the "
+                           "offline rows (calibration, smoothing factors + fold, weight "
+                           "quant) are timed separately under offline_prep",
                    "granularity": args.granularity, "format": args.format,
-                   "launch": "the whole step as one CUDA graph, replayed per timed step",
+                   "launch": "the forward as one CUDA graph, replayed per timed step",
                    "l2": "flushed before every step (256 MiB written, then another 256 MiB "
                          "read so no dirty line is left to write back; not timed)",
                    "parallelism": "dp%d (independent token batches, weights replicated)" % world},
         "tokens_per_s": tokens_per_s,
-        "forward_gemm_tops": g_ops / g_time / 1e12,
+        "forward_gemm_tops": sum(kinds["gemm:" + l.name][1] for l in w.linears)
+        / sum(kinds["gemm:" + l.name][2] for l in w.linears) / 1e12,
         "roofline": roof,
+        "gemms": gemms,
         "kernels": kernels,
-        "gpu_launches": args.steps * (blk.prepare_launches() + blk.forward_launches()),
+        "offline_prep": {
+            "ms": prep_t * 1e3, "bytes": prep_bytes, "achieved_gbs": prep_bytes / prep_t / 1e9,
+            "frac_hbm": prep_bytes / prep_t / 1e9 / peaks["hbm_gbs"],
+            "launches": blk.prepare_launches(), "replays": n_prep,
+            "what": "calibration (beside the weight column maxima, two streams), smoothing "
+                    "factors + fold, weight smoothing + quantisation of every Linear, as one "
+                    "CUDA graph; bytes = the calls' algorithmic bytes"},
+        "whole_path_ms": t_max * 1e3 / args.steps + prep_t * 1e3,
+        "gpu_launches": args.steps * blk.forward_launches(),
         "clocks": clocks,
         "wall_s_timed": wall,
     }
+    if (not args.no_decode and not decode and w.name.startswith("llama-block-8192")
+            and args.format == "int8" and args.granularity == "per_token"):
+        line["decode"] = decode_sweep(args, w, blk, dev, stream, flusher, peaks, args.seed, rank)
+    err = sq.get_device_error()
+    if err:
+        raise SystemExit("device error %s during the benchmark" % sq.status_string(err))
 
     # end to end through the public API: pinned host inputs in, results out
     if not args.no_e2e:
@@ -561,50 +727,45 @@ def run_gpu(args, w):
             and args.format == "int8"):
         import oracle
         oracle.build()
-        full, spent, desc = oracle_sample_step(w, inp)
-        line["cpu_baseline"] = {"value": workload_ops(w) / full / 1e12, "unit": "TOPS",
-                                "cores": oracle.num_threads(), "kind": "oracle",
-                                "sample": desc + " (%.1f s of CPU time)" % spent}
+        est, spent, desc, full = oracle_sample_step(w, inp, **cpu_sample_for(w))
+        line["cpu_baseline"] = {
+            "value": workload_ops(w) / est / 1e12, "unit": "TOPS",
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "measured": "in full" if full else "extrapolated from a sample",
+            "sample": desc + " (%.1f s of CPU time; the oracle's whole step, offline rows "
+                             "included)" % spent}
     if rank == 0:
         print(json.dumps(line), flush=True)
 
 
 def e2e_leg(args, w, inp, blk, dev, stream, world):
+    """The forward through the public API with its activations in pinned host
+    memory: every step copies the step's input tokens in, runs the library
+    calls and copies the block's results (the outputs no later Linear of the
+    block consumes) back to pinned host memory; timed by events on the
+    stream."""
     import torch
 
     def pinned(a):
-        if a is None:
-            return None
         t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16 \
             else torch.from_numpy(a)
         return t.pin_memory()
 
     hx = {k: pinned(v) for k, v in inp.x.items()}
-    hxc = {k: pinned(v) for k, v in inp.x_cal.items()}
-    hW = {k: pinned(v) for k, v in inp.W.items()}
-    hg = {k: pinned(v) for k, v in inp.gamma.items()}
-    hb = {k: pinned(v) for k, v in inp.beta.items()}
     dx = {k: torch.empty(v.shape, dtype=v.dtype, device=dev) for k, v in hx.items()}
-    dxc = {k: torch.empty(v.shape, dtype=v.dtype, device=dev) for k, v in hxc.items()}
-    dW = {k: torch.empty(v.shape, dtype=v.dtype, device=dev) for k, v in hW.items()}
-    dg = {k: (None if v is None else torch.empty(v.shape, dtype=v.dtype, device=dev))
-          for k, v in hg.items()}
-    db = {k: (None if v is None else torch.empty(v.shape, dtype=v.dtype, device=dev))
-          for k, v in hb.items()}
-    hout = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in blk.out.items()}
-    h2d = sum(t.numel() * t.element_size() for d in (hx, hxc, hW, hg, hb) for t in d.values()
-              if t is not None)
+    consumed = {l.source for l in w.linears if l.source}
+    results = [k for k in blk.out if k not in consumed]
+    hout = {k: torch.empty(blk.out[k].shape, dtype=blk.out[k].dtype).pin_memory()
+            for k in results}
+    h2d = sum(t.numel() * t.element_size() for t in hx.values())
     d2h = sum(t.numel() * t.element_size() for t in hout.values())
 
     def step():
-        for src, dst in ((hx, dx), (hxc, dxc), (hW, dW), (hg, dg), (hb, db)):
-            for k, t in src.items():
-                if t is not None:
-                    dst[k].copy_(t, non_blocking=True)
-        blk.prepare(dxc, dW, dg, db)
+        for k, t in hx.items():
+            dx[k].copy_(t, non_blocking=True)
         out = blk.forward(dx)
-        for k, t in out.items():
-            hout[k].copy_(t, non_blocking=True)
+        for k in results:
+            hout[k].copy_(out[k], non_blocking=True)
 
     for _ in range(max(1, args.warmup)):
         step()
@@ -621,19 +782,22 @@ def e2e_leg(args, w, inp, blk, dev, stream, world):
     value, _ = aggregate(workload_ops(w) * n, t, world, dev)
     return {"value": value / 1e12, "unit": "TOPS", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": n,
-            "path": "pinned host -> device copies, the six C-ABI calls, device -> pinned host"}
+            "path": "pinned host tokens -> device, the forward's C-ABI calls (Block.forward), "
+                    "the block's results -> pinned host; weights prepared once beforehand"}
 
 
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true",
+                    help="skip the decode sweep (M = 1, 8, 32, 128 on the Llama block weights)")
     ap.add_argument("--granularity", default="per_token",
                     choices=["per_token", "per_tensor_dynamic", "per_tensor_static"],
                     help="activation / weight scale sharing (per-token + per-channel, or the "

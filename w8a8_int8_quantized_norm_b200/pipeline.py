@@ -21,8 +21,8 @@ from . import sq
 from .synthetic import Workload
 
 # timer(kind, algorithmic_units, fn): a caller hook around every library call;
-# kind names the kernel family, units are its algorithmic bytes (row kernels)
-# or integer ops (the GEMM).
+# kind names the kernel family ("gemm:<linear>" for a GEMM call), units are its
+# algorithmic bytes (row kernels) or integer ops (the GEMM).
 Timer = Optional[Callable[[str, float, Callable[[], None]], None]]
 
 
@@ -61,7 +61,12 @@ class Block:
     smoothing).  Code tensors are then uint8 holding e4m3 bytes."""
 
     def __init__(self, w: Workload, M: int, device, granularity: str = "per_token",
-                 fmt: str = "int8"):
+                 fmt: str = "int8", shared: Optional["Block"] = None):
+        """``shared``: a Block of the same layer shapes whose prepared state
+        (smoothing factors, folded norm parameters, INT8 weights and their
+        scales) this one reads instead of holding its own -- one set of
+        weights serving several token counts, as a decode step beside a
+        prefill step does.  Only the per-token buffers are allocated here."""
         if granularity not in GRANULARITIES:
             raise ValueError("granularity must be one of %s" % (GRANULARITIES,))
         if fmt not in FORMATS:
@@ -92,10 +97,24 @@ class Block:
         self.w_scale: Dict[str, torch.Tensor] = {}
         self.out: Dict[str, torch.Tensor] = {}
         self.ws: Dict[str, Optional[torch.Tensor]] = {}
+        if shared is not None:
+            same = ([(s.name, s.K, s.norm, s.smoothed) for s in shared.w.sites]
+                    == [(s.name, s.K, s.norm, s.smoothed) for s in w.sites]
+                    and [(l.name, l.site, l.N) for l in shared.w.linears]
+                    == [(l.name, l.site, l.N) for l in w.linears])
+            if not same or shared.granularity != granularity or shared.fmt != fmt:
+                raise ValueError("a shared Block must have the same layers, granularity "
+                                 "and format")
+            # the dicts themselves are shared: what the other Block's prepare
+            # writes is what this one's forward reads
+            self.act_max, self.s = shared.act_max, shared.s
+            self.gamma_f, self.beta_f = shared.gamma_f, shared.beta_f
+            self.Wq, self.w_scale = shared.Wq, shared.w_scale
         for lin in w.linears:
             K = w.site(lin.site).K
-            self.Wq[lin.name] = torch.empty((lin.N, K), dtype=code_dtype, device=dev)
-            self.w_scale[lin.name] = torch.empty(lin.N, **f32)
+            if shared is None:
+                self.Wq[lin.name] = torch.empty((lin.N, K), dtype=code_dtype, device=dev)
+                self.w_scale[lin.name] = torch.empty(lin.N, **f32)
             self.out[lin.name] = torch.empty((M, lin.N), dtype=torch.bfloat16, device=dev)
             need = 0 if fmt == "fp8" else sq.gemm_workspace_size(M, lin.N, K, 0)
             self.ws[lin.name] = torch.empty(need, dtype=torch.uint8, device=dev) if need else None
@@ -111,6 +130,11 @@ class Block:
                                       and site.calibrated)
         self.w_absmax: Dict[str, torch.Tensor] = {l.name: torch.zeros(1, **f32)
                                                   for l in w.linears}
+        if shared is not None:
+            self.w_absmax = shared.w_absmax
+            for site in w.sites:  # O3's static maxima are prepared state too
+                if self.static[site.name]:
+                    self.x_absmax[site.name] = shared.x_absmax[site.name]
         # A Linear whose bf16 output is the whole input of a later per-token
         # site (no norm, no multiplier: fc1 -> ReLU -> fc2) reduces each
         # output row's max |out| in its GEMM epilogue, so that site's
@@ -297,7 +321,7 @@ class Block:
                                      "bf16_relu" if lin.relu else "bf16",
                                      out=self.out[lin.name], workspace=self.ws[lin.name],
                                      stream=stream)
-            _run(timer, "gemm", 2.0 * self.M * lin.N * site.K, gemm)
+            _run(timer, "gemm:" + lin.name, 2.0 * self.M * lin.N * site.K, gemm)
 
     # -- the whole step, independent work on two streams ----------------------
     def step(self, x_cal, W, gamma, beta, x) -> Dict[str, torch.Tensor]:
@@ -309,22 +333,8 @@ class Block:
         end, so the step is ordered like one stream to its caller (and can be
         captured in a CUDA graph)."""
         main = torch.cuda.current_stream()
-        if self._side is None:
-            self._side = torch.cuda.Stream()
-        side = self._side
+        side = self._scales_two_streams(x_cal, W, gamma, beta)
         w = self.w
-        smoothed = [site for site in w.sites if site.smoothed]
-        # calibration on the side stream, weight column maxima on this one
-        side.wait_stream(main)
-        with torch.cuda.stream(side):
-            for site in smoothed:
-                self._calibrate(site, x_cal, gamma, beta, None, None)
-        for site in smoothed:
-            sq.weight_column_max(self._site_weights(site, W), w_max=self.s[site.name])
-        main.wait_stream(side)
-        for site in w.sites:
-            self._site_scales(site, x_cal, W, gamma, beta, None, None, calibrated=True,
-                              w_max_done=True)
         # weights on the side stream, the input sites' codes on this one
         side.wait_stream(main)
         with torch.cuda.stream(side):
@@ -341,6 +351,37 @@ class Block:
                 self._quantize_site(site, x, None, None)
                 self._gemms(site, None, None)
         return self.out
+
+    def _scales_two_streams(self, x_cal, W, gamma, beta):
+        """Calibration on a second stream beside the weight column maxima on
+        the current one, joined; then the smoothing factors and the fold.
+        Returns the second stream."""
+        main = torch.cuda.current_stream()
+        if self._side is None:
+            self._side = torch.cuda.Stream()
+        side = self._side
+        smoothed = [site for site in self.w.sites if site.smoothed]
+        side.wait_stream(main)
+        with torch.cuda.stream(side):
+            for site in smoothed:
+                self._calibrate(site, x_cal, gamma, beta, None, None)
+        for site in smoothed:
+            sq.weight_column_max(self._site_weights(site, W), w_max=self.s[site.name])
+        main.wait_stream(side)
+        for site in self.w.sites:
+            self._site_scales(site, x_cal, W, gamma, beta, None, None, calibrated=True,
+                              w_max_done=True)
+        return side
+
+    def prepare_two_streams(self, x_cal, W, gamma, beta) -> "Block":
+        """``prepare`` with the calibration running beside the weight column
+        maxima on a second stream (joined before the smoothing factors); the
+        same kernels and the same results, ordered like one stream to the
+        caller."""
+        self._scales_two_streams(x_cal, W, gamma, beta)
+        for lin in self.w.linears:
+            self._weight_quant(lin, W, None, None)
+        return self
 
     # -- launch accounting ---------------------------------------------------
     def prepare_launches(self) -> int:
@@ -401,6 +442,36 @@ class Block:
                 self.prepare(x_cal, W, gamma, beta, timer=timer)
                 self.forward(x, timer=timer)
         return graph
+
+
+def _capture(fn, warmup: int = 1):
+    """Records ``fn`` (a sequence of library calls on the current stream,
+    possibly forking to others and joining back) into a CUDA graph after
+    ``warmup`` runs outside the capture (the first use of each kernel sets
+    its launch attributes)."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for _ in range(warmup):
+            fn()
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        fn()
+    return graph
+
+
+def capture_forward(blk: Block, x, warmup: int = 1):
+    """The runtime rows of one step (norm + per-token quantisation, GEMMs with
+    the dequant epilogue, for every Linear) as one CUDA graph."""
+    return _capture(lambda: blk.forward(x), warmup)
+
+
+def capture_prepare(blk: Block, x_cal, W, gamma, beta, warmup: int = 1):
+    """The offline rows (calibration, smoothing factors and fold, weight
+    smoothing and quantisation) as one CUDA graph, calibration beside the
+    weight column maxima."""
+    return _capture(lambda: blk.prepare_two_streams(x_cal, W, gamma, beta), warmup)
 
 
 # Thin functional wrappers (used by tests and the smoke check).
