@@ -15,11 +15,13 @@
 //   * the norm kind is a template parameter (no per-element branches); row
 //     sums are fp64 (x^2 of a bf16 / fp32 value is exact in fp64), reduced in
 //     a fixed order so results repeat bit for bit;
-//   * the quantiser avoids a division per element: with r = fl32(1/step) the
-//     product t = fl32(y r) is within 3 * 2^-24 relative of y/step, so
+//   * the quantiser avoids a division per element.  With a row's own step
+//     (max / 127) the codes come from two fused multiply-adds that bracket
+//     y / step (codes8_bracket); with a given step, from r = fl32(1/step),
+//     whose product t = fl32(y r) is within 3 * 2^-24 relative of y/step, so
 //     rne(fl32(y/step)) = rne(t) unless y/step lies within 1e-4 of a
-//     half-integer; a chunk of 8 values holding such a quotient is redone
-//     with the exact division (branch-free otherwise).  Rounding to the
+//     half-integer (codes8).  Either way a chunk of 8 values that the fast
+//     test cannot decide is redone with the exact division.  Rounding to the
 //     nearest integer (ties to even) is the float add of 1.5 * 2^23, whose low
 //     8 mantissa bits are then the two's-complement INT8 code.
 #include <cuda_fp8.h>
@@ -206,6 +208,104 @@ __device__ __forceinline__ uint2 codes8(const float2 (&v)[4], float rstep, float
   const uint32_t hi = __byte_perm(__byte_perm(m[4], m[5], 0x0040), __byte_perm(m[6], m[7], 0x0040),
                                   0x5410);
   return make_uint2(lo, hi);
+}
+
+// INT8 codes of 8 values, packed little-endian, by bracketing: with
+// rhi >= (1 + 2^-24) / step and rlo <= (1 - 2^-24) / step (both finite,
+// step normal), the exact quotient q = v / step and its fp32 rounding lie
+// between v rlo and v rhi; round-half-even to an integer is monotone, so
+// when the two fused multiply-adds rne(v rhi) and rne(v rlo) (as the low
+// bits of the product + 1.5 * 2^23, one rounding each) agree, that integer
+// is rne(fl32(q)) -- no clamp needed when |v| <= 127 step.  They disagree
+// only when an integer + 1/2 lies within about 2^-21 |q| of q (at most
+// 2^-13 of the values); a chunk holding one, or a step without a finite
+// reciprocal, is recomputed from the exact quotient.
+__device__ __forceinline__ uint2 codes8_bracket(const float2 (&v)[4], float rhi, float rlo,
+                                                float step, bool exact_only) {
+  uint32_t m[8];
+  uint32_t diff = 0u;
+  const float2 rh = make_float2(rhi, rhi), rl = make_float2(rlo, rlo);
+  const float2 mg = make_float2(kMagic, kMagic);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 a = __ffma2_rn(v[i], rh, mg);
+    const float2 b = __ffma2_rn(v[i], rl, mg);
+    diff |= __float_as_uint(a.x) ^ __float_as_uint(b.x);
+    diff |= __float_as_uint(a.y) ^ __float_as_uint(b.y);
+    m[2 * i] = __float_as_uint(a.x);
+    m[2 * i + 1] = __float_as_uint(a.y);
+  }
+  if (exact_only || diff != 0u) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float vv[2] = {v[i].x, v[i].y};
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        float e = (step == 0.0f) ? 0.0f : __fdiv_rn(vv[j], step);
+        e = fminf(fmaxf(e, -127.0f), 127.0f);
+        m[2 * i + j] = __float_as_uint(__fadd_rn(e, kMagic));
+      }
+    }
+  }
+  const uint32_t lo = __byte_perm(__byte_perm(m[0], m[1], 0x0040), __byte_perm(m[2], m[3], 0x0040),
+                                  0x5410);
+  const uint32_t hi = __byte_perm(__byte_perm(m[4], m[5], 0x0040), __byte_perm(m[6], m[7], 0x0040),
+                                  0x5410);
+  return make_uint2(lo, hi);
+}
+
+// The bracketing codes of 8 values without the fallback: returns the packed
+// codes of v rhi and ORs into `diff` a non-zero word when some value's two
+// roundings disagree (the caller then recomputes with exact8).
+__device__ __forceinline__ uint2 bracket8(const float2 (&v)[4], float2 rh, float2 rl,
+                                          uint32_t& diff) {
+  uint32_t m[8];
+  const float2 mg = make_float2(kMagic, kMagic);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 a = __ffma2_rn(v[i], rh, mg);
+    const float2 b = __ffma2_rn(v[i], rl, mg);
+    diff |= __float_as_uint(a.x) ^ __float_as_uint(b.x);
+    diff |= __float_as_uint(a.y) ^ __float_as_uint(b.y);
+    m[2 * i] = __float_as_uint(a.x);
+    m[2 * i + 1] = __float_as_uint(a.y);
+  }
+  const uint32_t lo = __byte_perm(__byte_perm(m[0], m[1], 0x0040), __byte_perm(m[2], m[3], 0x0040),
+                                  0x5410);
+  const uint32_t hi = __byte_perm(__byte_perm(m[4], m[5], 0x0040), __byte_perm(m[6], m[7], 0x0040),
+                                  0x5410);
+  return make_uint2(lo, hi);
+}
+
+// clamp(rne(fl32(v / step)), -127, 127) of 8 values by the exact division
+// (step 0: zero codes).
+__device__ __forceinline__ uint2 exact8(const float2 (&v)[4], float step) {
+  uint32_t m[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float vv[2] = {v[i].x, v[i].y};
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      float e = (step == 0.0f) ? 0.0f : __fdiv_rn(vv[j], step);
+      e = fminf(fmaxf(e, -127.0f), 127.0f);
+      m[2 * i + j] = __float_as_uint(__fadd_rn(e, kMagic));
+    }
+  }
+  const uint32_t lo = __byte_perm(__byte_perm(m[0], m[1], 0x0040), __byte_perm(m[2], m[3], 0x0040),
+                                  0x5410);
+  const uint32_t hi = __byte_perm(__byte_perm(m[4], m[5], 0x0040), __byte_perm(m[6], m[7], 0x0040),
+                                  0x5410);
+  return make_uint2(lo, hi);
+}
+
+// The bracketing multipliers of a row's step (normal): rs = fl32(1 / step)
+// is within 2^-24 of 1 / step, and fl32(rs (1 +- 2^-21)) stay more than
+// 2^-22 away from rs on their side, so rhi >= (1 + 2^-24) / step and
+// rlo <= (1 - 2^-24) / step.
+__device__ __forceinline__ void bracket_of(float step, float& rhi, float& rlo) {
+  const float rs = __frcp_rn(step);
+  rhi = __fmul_rn(rs, 1.0f + 0x1p-21f);
+  rlo = __fmul_rn(rs, 1.0f - 0x1p-21f);
 }
 
 // fl32(a / 127) for every non-negative finite binary32 a, in three
@@ -594,10 +694,11 @@ __global__ void __launch_bounds__(PipeBounds<CH, kMode>::kMaxThreads,
           *reinterpret_cast<uint2*>(qrow + ch * kChunk) = code;
         }
       } else {
-        // ---- per-token INT8 quantisation
+        // ---- per-token INT8 quantisation (the row's own step: no clamp)
         const float step = div127(am);
         const bool exact_only = step < FLT_MIN;  // zero or subnormal step: no reciprocal
-        const float rstep = exact_only ? 0.0f : __frcp_rn(step);
+        float rhi = 0.0f, rlo = 0.0f;
+        if (!exact_only) bracket_of(step, rhi, rlo);
         if (t == 0) scale[row] = step;
         int8_t* qrow = q + row * static_cast<int64_t>(K);
 #pragma unroll
@@ -610,10 +711,11 @@ __global__ void __launch_bounds__(PipeBounds<CH, kMode>::kMaxThreads,
             for (int i = 0; i < 4; ++i)
               hv[i] = make_float2(__uint_as_float(hbv[c][i] << 16),
                                   __uint_as_float(hbv[c][i] & 0xffff0000u));
-            *reinterpret_cast<uint2*>(qrow + ch * kChunk) = codes8(hv, rstep, step, exact_only);
+            *reinterpret_cast<uint2*>(qrow + ch * kChunk) =
+                codes8_bracket(hv, rhi, rlo, step, exact_only);
           } else {
             *reinterpret_cast<uint2*>(qrow + ch * kChunk) =
-                codes8(v[c], rstep, step, exact_only);
+                codes8_bracket(v[c], rhi, rlo, step, exact_only);
           }
         }
       }
@@ -801,6 +903,500 @@ cudaError_t launch_rows(const RowArgs& a, bool bf16, int norm, cudaStream_t st) 
   return launch_pipe_n<false, 0, kMode>(a, ps, st);
 }
 
+
+// ---- norm + per-token quantisation, pipelined across a CTA's rows --------
+//
+// The per-token modes with a norm (INT8 or FP8 codes) at one CTA barrier per
+// row, and without the CTA waiting on a row's scalar chain.  Iteration i of a
+// CTA (rows i, i + 1 of its own row sequence):
+//   phase 1: the fp64 sums of row i + 1 (read from its buffer) and the
+//            normalised values y of row i (its buffer again, with r_i, mu_i)
+//            with their partial absmax;
+//   barrier X_i (thread 0 has also seen row i + 2 land);
+//   phase 2: row i's step and codes; one warp, rotating with the row, turns
+//            row i + 1's sums into (r, mu) and publishes them through an
+//            mbarrier, which the other warps wait on only when they reach
+//            row i + 1's y in the next iteration.
+// Row i's buffer is refilled after X_i (both of its reads precede it), so
+// nbuf - 2 rows per CTA are in flight while the CTA computes.
+
+struct RowScalars {
+  float r, mu;
+};
+
+// (r, mu) of a row from its fp64 sums S2 = sum x^2 and S1 = sum x, equal to
+// the fp32 roundings of the exact chain
+//   ms = fl64(S2 / K), mu64 = fl64(S1 / K),
+//   var = max(0, fl64(ms - fl64(mu64 mu64)))   (LayerNorm; RMSNorm: var = ms),
+//   r = fl32(fl64(1 / fl64(sqrt(fl64(var + eps))))),  mu = fl32(mu64).
+// Fast path: the divisions are products with invK = fl64(1 / K) (exact for a
+// power-of-two K) and 1 / sqrt(v) is rsqrt(v) = A, whose own relative error
+// d is measured: with t = fl64(v A), e = fl64(1 - t A) (one fused
+// multiply-add) gives |d| <= 0.51 (|e| (1 + u) + 1.01 u), u = 2^-53.  Against
+// the exact chain, the fast v differs by at most u (6 ms + 11 mu^2 + 2.1 v)
+// (the product roundings: 2u on ms and mu against u in the chain, the
+// square, the difference and the eps sum), the chain's own sqrt and
+// reciprocal add 2.01u, so A is within
+//   E = 1.05 (d + 2.01u + (3 ms + 5.5 mu^2) u / v + 1.05u) + 2^-60
+// of the chain's fp64 r.  r's fp32 rounding is the chain's whenever the
+// distance from A to the nearest fp32 rounding midpoint, in units of A's last
+// place (the low 29 bits of its significand against 2^28), exceeds E 2^53 + 1;
+// the test below checks 0.6 |e| 2^53 + 0.6 (6 ms + 11 mu^2) / v + 6 >= that
+// (both sides times v).  mu's: |fast - chain| <= 3.02u |mu| (at most 6.04
+// units of the last place; 8 is checked).  Otherwise (about one row in 10^7,
+// or a value outside the normal ranges) the exact chain runs.
+template <int NORMK>
+__device__ __forceinline__ RowScalars row_scalars(double S2, double S1, double invK, double Kd,
+                                                  float eps) {
+  const double e64 = static_cast<double>(eps);
+  const double ms = __dmul_rn(S2, invK);
+  double mu = 0.0, m2 = 0.0, var = ms;
+  if constexpr (NORMK == 2) {
+    mu = __dmul_rn(S1, invK);
+    m2 = __dmul_rn(mu, mu);
+    var = __dsub_rn(ms, m2);
+    if (var < 0.0) var = 0.0;
+  }
+  const double v = __dadd_rn(var, e64);
+  const double A = rsqrt(v);
+  const double e = __fma_rn(-__dmul_rn(v, A), A, 1.0);
+  const double tau_v = 0.6 * fabs(e) * 0x1p53 * v + 0.6 * (6.0 * ms + 11.0 * m2) + 6.0 * v;
+  const long long ab = __double_as_longlong(A);
+  const double dist = fabs(static_cast<double>((ab & 0x1fffffffLL) - 0x10000000LL));
+  bool ok = v >= 0x1p-1000 && v <= 0x1p1000 && fabs(e) <= 0x1p-20 && A >= 0x1p-125 &&
+            A <= 0x1p125 && dist * v > tau_v;
+  RowScalars rs;
+  rs.r = __double2float_rn(A);
+  rs.mu = 0.0f;
+  if constexpr (NORMK == 2) {
+    rs.mu = __double2float_rn(mu);
+    if (mu != 0.0) {
+      const long long dl = (__double_as_longlong(mu) & 0x1fffffffLL) - 0x10000000LL;
+      ok = ok && fabs(mu) >= 0x1p-125 && fabs(mu) <= 0x1p125 && (dl > 8 || dl < -8);
+    }
+  }
+  if (!ok) {
+    // the exact chain, one IEEE operation per step
+    const double msx = __ddiv_rn(S2, Kd);
+    double varx = msx;
+    if constexpr (NORMK == 2) {
+      const double mux = __ddiv_rn(S1, Kd);
+      varx = __dsub_rn(msx, __dmul_rn(mux, mux));
+      if (varx < 0.0) varx = 0.0;
+      rs.mu = __double2float_rn(mux);
+    }
+    rs.r = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(varx, e64))));
+  }
+  return rs;
+}
+
+// This thread's fp64 partial sums (x^2; x for LayerNorm) over its chunks of
+// a row in shared memory, two accumulators per sum.
+// bf16 pair (low, high half of a word) -> two fp64 values, exactly
+__device__ __forceinline__ void bf16x2_to_f64(uint32_t w, double& lo, double& hi) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "cvt.f64.bf16 %0, l;\n\tcvt.f64.bf16 %1, h;\n\t}"
+      : "=d"(lo), "=d"(hi)
+      : "r"(w));
+}
+
+template <bool kBF16, int NORMK, int CH, bool kFull>
+__device__ __forceinline__ void row_partial_sums(const uint8_t* rowp, int t, int T, int nchunks,
+                                                 double& s2, double& s1) {
+  // four accumulators per sum (element i of a chunk feeds accumulator i mod 4)
+  double a1[4] = {0.0, 0.0, 0.0, 0.0}, a2[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+  for (int c = 0; c < CH; ++c) {
+    const int ch = t + c * T;
+    if (kFull || ch < nchunks) {
+      double d[8];
+      if constexpr (kBF16) {
+        const uint4 u = *reinterpret_cast<const uint4*>(rowp + ch * 16);
+        bf16x2_to_f64(u.x, d[0], d[1]);
+        bf16x2_to_f64(u.y, d[2], d[3]);
+        bf16x2_to_f64(u.z, d[4], d[5]);
+        bf16x2_to_f64(u.w, d[6], d[7]);
+      } else {
+        float2 v[4];
+        smem_chunk<false>(rowp, ch, v);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          d[2 * i] = static_cast<double>(v[i].x);
+          d[2 * i + 1] = static_cast<double>(v[i].y);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if constexpr (NORMK == 2) a1[i & 3] = __dadd_rn(a1[i & 3], d[i]);
+        a2[i & 3] = __fma_rn(d[i], d[i], a2[i & 3]);
+      }
+    }
+  }
+  s2 = __dadd_rn(__dadd_rn(a2[0], a2[1]), __dadd_rn(a2[2], a2[3]));
+  s1 = __dadd_rn(__dadd_rn(a1[0], a1[1]), __dadd_rn(a1[2], a1[3]));
+}
+
+// Bounded wait for the scalars of a row (parity = the row's number in the
+// CTA's sequence, mod 2).
+__device__ __forceinline__ bool scalars_ready(uint32_t bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long c0 = clock64();
+  for (uint32_t k = 0;; ++k) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((k & 63u) == 63u && clock64() - c0 > kWaitBudgetCycles) return false;
+  }
+}
+
+// One warp: the row's sums (per-warp partials in a fixed order) -> (r, mu) in
+// scal[2 slot .. 2 slot + 1]; lane 0 stores them and arrives on the barrier
+// (release; the waiters' try_wait acquires).
+template <int NORMK>
+__device__ __forceinline__ void publish_scalars(const double* dslot, int nwarps, float* sslot,
+                                                uint32_t sbar, double invK, double Kd, float eps,
+                                                int lane) {
+  double S2 = dslot[0], S1 = dslot[8];
+  for (int w = 1; w < nwarps; ++w) {
+    S2 = __dadd_rn(S2, dslot[w]);
+    if constexpr (NORMK == 2) S1 = __dadd_rn(S1, dslot[8 + w]);
+  }
+  const RowScalars rs = row_scalars<NORMK>(S2, S1, invK, Kd, eps);
+  if (lane == 0) {
+    sslot[0] = rs.r;
+    sslot[1] = rs.mu;
+    mbar_arrive(sbar);
+  }
+}
+
+// At most 8 warps (256 threads) a CTA, 4 or 8 chunks a thread.  TF > 0: the
+// thread count is the compile-time constant TF and TF * CH chunks are the
+// whole row (kFull), so every chunk offset is an immediate.
+template <int TF, int CH>
+struct RowsBounds {
+  static constexpr int kThreads = TF > 0 ? TF : 256;
+  static constexpr int kMinBlocks = (TF > 0 && TF <= 128) ? 4 : (CH <= 4 ? 3 : 2);
+};  // 128 threads: 128 registers; 256 threads, 4 chunks: 85; 8 chunks: 128
+
+template <bool kBF16, int NORMK, int CH, bool kGamma, bool kBeta, bool kFull, bool kF8, int TF>
+__global__ void __launch_bounds__(RowsBounds<TF, CH>::kThreads, RowsBounds<TF, CH>::kMinBlocks)
+    norm_quant_rows_kernel(const void* __restrict__ x, int64_t ldx, int64_t M, int K, double invK,
+                           const float* __restrict__ gamma, const float* __restrict__ beta,
+                           float eps, int8_t* __restrict__ q, float* __restrict__ scale, int nbuf,
+                           int* error_word) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  constexpr int kEsz = kBF16 ? 2 : 4;
+  static_assert(NORMK == 1 || NORMK == 2, "a norm kind");
+  const uint32_t row_bytes = static_cast<uint32_t>(K) * kEsz;
+  const uint32_t buf_stride = (row_bytes + 127u) & ~127u;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + nbuf * buf_stride);  // [nbuf] + scalars
+  double* dscr = reinterpret_cast<double*>(bars + nbuf + 1);  // [2 slots][sum x^2, sum x][8]
+  float* scal = reinterpret_cast<float*>(dscr + 32);          // [2 slots][r, mu]
+  unsigned int* smax = reinterpret_cast<unsigned int*>(scal + 4);  // [3] row absmax bits
+  const uint32_t smem_base = smem_u32(smem);
+  const uint32_t bar_base = smem_u32(bars);
+  const uint32_t sbar = bar_base + 8u * static_cast<uint32_t>(nbuf);
+
+  static_assert(TF == 0 || kFull, "a compile-time thread count covers the whole row");
+  const int t = threadIdx.x;
+  const int T = TF > 0 ? TF : static_cast<int>(blockDim.x);
+  const int warp = t >> 5, lane = t & 31, nwarps = T >> 5;
+  const int nchunks = TF > 0 ? TF * CH : K / kChunk;
+  const int64_t G = gridDim.x;
+  const int64_t first = blockIdx.x;
+  const uint8_t* xb = static_cast<const uint8_t*>(x);
+  const int64_t row_pitch = ldx * kEsz;
+  const double Kd = static_cast<double>(K);
+
+  if (t == 0) {
+    for (int b = 0; b <= nbuf; ++b) mbar_init(bar_base + 8u * b, 1);
+    smax[0] = 0u;
+    smax[1] = 0u;
+    smax[2] = 0u;
+    mbar_fence_init();
+  }
+  __syncthreads();
+  int issued = 0;  // thread 0: row copies issued, in the CTA's row order
+  if (t == 0) {
+    for (int b = 0; b < nbuf; ++b) {
+      const int64_t row = first + b * G;
+      if (row < M) {
+        mbar_arrive_expect_tx(bar_base + 8u * b, row_bytes);
+        bulk_load(smem_base + b * buf_stride, xb + row * row_pitch, row_bytes, bar_base + 8u * b);
+        issued = b + 1;
+      }
+    }
+  }
+  if (first >= M) return;
+
+  // prologue: the sums and scalars of the CTA's first row
+  bool aborted = false;
+  {
+    const bool ok = t != 0 || row_landed(bar_base, 0, 0u);
+    if (__syncthreads_or(!ok)) aborted = true;
+  }
+  if (!aborted) {
+    double s2, s1;
+    row_partial_sums<kBF16, NORMK, CH, kFull>(smem, t, T, nchunks, s2, s1);
+    s2 = warp_sum(s2);
+    if constexpr (NORMK == 2) s1 = warp_sum(s1);
+    if (lane == 0) {
+      dscr[warp] = s2;
+      dscr[8 + warp] = s1;
+    }
+    const bool ok = (t != 0 || first + G >= M) ? true : row_landed(bar_base, 1, 0u);
+    if (__syncthreads_or(!ok)) aborted = true;
+    else if (warp == 0)
+      publish_scalars<NORMK>(dscr, nwarps, scal, sbar, invK, Kd, eps, lane);
+  }
+
+  int it = 0;
+  int b_cur = 0, b_nxt = 1, b_nn = 2;  // buffers of rows it, it + 1, it + 2
+  uint32_t p_nn = 0u;                  // phase parity of row it + 2's copy
+  int s_cur = 0;                       // it mod 3
+  int pub_warp = 0;                    // it mod nwarps: the warp that published row it
+  for (int64_t row = first; row < M && !aborted; row += G, ++it) {
+    const bool has_next = row + G < M;
+    const int slot = it & 1, nslot = slot ^ 1;
+    // ---- phase 1a: row it + 1's sums
+    if (has_next) {
+      double s2, s1;
+      row_partial_sums<kBF16, NORMK, CH, kFull>(smem + b_nxt * buf_stride, t, T, nchunks, s2, s1);
+      s2 = warp_sum(s2);
+      if constexpr (NORMK == 2) s1 = warp_sum(s1);
+      if (lane == 0) {
+        dscr[nslot * 16 + warp] = s2;
+        dscr[nslot * 16 + 8 + warp] = s1;
+      }
+    }
+    // ---- phase 1b: row it's normalised values and their absmax
+    bool ok = scalars_ready(sbar, static_cast<uint32_t>(slot));
+    const float r = scal[2 * slot], mu = scal[2 * slot + 1];
+    const float2 r2 = make_float2(r, r), nmu2 = make_float2(-mu, -mu);
+    const uint8_t* rowp = smem + b_cur * buf_stride;
+    float2 y[CH][4];
+    float am = 0.0f;
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+      const int ch = t + c * T;
+      if (kFull || ch < nchunks) {
+        float2 v[4], g[4], bt[4];
+        smem_chunk<kBF16>(rowp, ch, v);
+        if constexpr (kGamma) param8(gamma, ch, g);
+        if constexpr (kBeta) param8(beta, ch, bt);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float2 yy = v[i];
+          if constexpr (NORMK == 1) yy = __fmul2_rn(yy, r2);
+          if constexpr (NORMK == 2) yy = __fmul2_rn(__fadd2_rn(yy, nmu2), r2);
+          if constexpr (kBeta) {
+            // a multiply followed by an add: the scalar intrinsics, which are
+            // never contracted into a fused multiply-add (paired ones were, in
+            // a LayerNorm test row, both as intrinsics and as explicit .rn PTX)
+            if constexpr (kGamma) {
+              yy.x = __fmul_rn(yy.x, g[i].x);
+              yy.y = __fmul_rn(yy.y, g[i].y);
+            }
+            yy.x = __fadd_rn(yy.x, bt[i].x);
+            yy.y = __fadd_rn(yy.y, bt[i].y);
+          } else if constexpr (kGamma) {
+            yy = __fmul2_rn(yy, g[i]);
+          }
+          am = fmaxf(am, fmaxf(fabsf(yy.x), fabsf(yy.y)));
+          y[c][i] = yy;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) y[c][i] = make_float2(0.0f, 0.0f);
+      }
+    }
+    // non-negative floats order like their bit patterns: integer max reduce
+    const unsigned int wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(am));
+    if (lane == 0) atomicMax(&smax[s_cur], wmax);
+    if (t == 0 && row + 2 * G < M) ok = ok && row_landed(bar_base, b_nn, p_nn);
+    if (__syncthreads_or(!ok)) {  // X
+      aborted = true;
+      break;
+    }
+    // ---- phase 2: row it's step and codes; row it + 1's scalars
+    if (t == 0) {
+      smax[s_cur == 0 ? 2 : s_cur - 1] = 0u;  // the slot of row it + 2
+      issued = refill_row(smem_base, bar_base, buf_stride, row_bytes, nbuf, it, b_cur, row, G, M,
+                          xb, row_pitch, issued);
+    }
+    const float amax = __uint_as_float(smax[s_cur]);
+    int8_t* qrow = q + row * static_cast<int64_t>(K);
+    if constexpr (kF8) {
+      float step = __fdiv_rn(amax, 448.0f);
+      if (!(step >= FLT_MIN)) step = 0.0f;
+      const float inv = step > 0.0f ? __frcp_rn(step) : 0.0f;
+      if (t == 0) scale[row] = step;
+#pragma unroll
+      for (int c = 0; c < CH; ++c) {
+        const int ch = t + c * T;
+        if (!kFull && ch >= nchunks) continue;
+        const uint2 code = step > 0.0f ? codes8_f8(y[c], inv) : make_uint2(0u, 0u);
+        *reinterpret_cast<uint2*>(qrow + ch * kChunk) = code;
+      }
+    } else {
+      const float step = div127(amax);
+      const bool exact_only = step < FLT_MIN;  // zero or subnormal step: no reciprocal
+      float rhi = 0.0f, rlo = 0.0f;
+      if (!exact_only) bracket_of(step, rhi, rlo);
+      if (t == 0) scale[row] = step;
+      // all of this thread's codes by bracketing, stored at once; then one
+      // branch: any value the two roundings disagreed on (or a step without a
+      // reciprocal) sends the thread's chunks of the row to the exact
+      // division, whose codes overwrite them
+      uint32_t diff = exact_only ? 1u : 0u;
+      const float2 rh = make_float2(rhi, rhi), rl = make_float2(rlo, rlo);
+#pragma unroll
+      for (int c = 0; c < CH; ++c) {
+        const int ch = t + c * T;
+        const uint2 code = bracket8(y[c], rh, rl, diff);
+        if (kFull || ch < nchunks) *reinterpret_cast<uint2*>(qrow + ch * kChunk) = code;
+      }
+      if (diff != 0u) {
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+          const int ch = t + c * T;
+          if (kFull || ch < nchunks)
+            *reinterpret_cast<uint2*>(qrow + ch * kChunk) = exact8(y[c], step);
+        }
+      }
+    }
+    if (++pub_warp == nwarps) pub_warp = 0;  // (it + 1) mod nwarps
+    if (has_next && warp == pub_warp)
+      publish_scalars<NORMK>(dscr + nslot * 16, nwarps, scal + 2 * nslot, sbar, invK, Kd, eps,
+                             lane);
+    b_cur = b_nxt;
+    b_nxt = b_nn;
+    if (++b_nn == nbuf) {
+      b_nn = 0;
+      p_nn ^= 1u;
+    }
+    s_cur = s_cur == 2 ? 0 : s_cur + 1;
+  }
+  if (aborted && t == 0) {
+    record_device_error(error_word, SQ_ERR_PIPELINE_TIMEOUT);
+    // let every bulk copy still in flight land before the CTA exits (the
+    // latest copy into buffer b is the one of row number s = b mod nbuf,
+    // s < issued, which completes phase s / nbuf of the buffer's barrier)
+    for (int b = 0; b < nbuf && b < issued; ++b) {
+      const int s_last = b + (issued - 1 - b) / nbuf * nbuf;
+      const uint32_t par = static_cast<uint32_t>((s_last / nbuf) & 1);
+      const long long c0 = clock64();
+      while (!mbar_try_wait(bar_base + 8u * b, par) && clock64() - c0 < kWaitBudgetCycles) {
+      }
+    }
+  }
+}
+
+struct RowsShape {
+  int ch, threads, nbuf;
+  size_t smem;
+};
+
+// row buffers, nbuf + 1 barriers, 32 doubles of sums, 4 floats of scalars, 3 absmax slots
+size_t rows_smem(size_t stride, int nbuf) { return nbuf * stride + 8 * (nbuf + 1) + 32 * 8 + 32; }
+
+// Rows up to kRows4 chunks (8 elements each) run 4 chunks a thread, wider
+// ones 8 (at most 256 threads either way).
+constexpr int kRows4 = 4 * 128;
+
+bool rows_shape(int K, bool bf16, RowsShape* rs) {
+  const int nchunks = K / kChunk;
+  const int ch = nchunks <= kRows4 ? 4 : (nchunks <= 8 * 256 ? 8 : 0);
+  if (!ch || nchunks < 1) return false;
+  int threads = (nchunks + ch - 1) / ch;
+  threads = (threads + 31) / 32 * 32;
+  const size_t stride = (static_cast<size_t>(K) * (bf16 ? 2 : 4) + 127) / 128 * 128;
+  // about 200 KB of row buffers per SM over the CTAs that fit it (their
+  // registers decide: four of 128 threads, three of 256): two rows of each
+  // CTA in use and the rest in flight
+  const int ctas = (threads <= 128) ? 4 : 3;
+  int nbuf = static_cast<int>((200u << 10) / ctas / stride);
+  if (nbuf < 3) nbuf = 3;
+  if (nbuf > 8) nbuf = 8;
+  if (nbuf * stride > (200u << 10)) return false;
+  rs->ch = ch;
+  rs->threads = threads;
+  rs->nbuf = nbuf;
+  rs->smem = rows_smem(stride, nbuf);
+  return true;
+}
+
+template <bool kBF16, int NORMK, int CH, bool kG, bool kB, bool kF, bool kF8, int TF = 0>
+cudaError_t launch_rows_k(const RowArgs& a, RowsShape rs, cudaStream_t st) {
+  auto kern = norm_quant_rows_kernel<kBF16, NORMK, CH, kG, kB, kF, kF8, TF>;
+  const void* key = reinterpret_cast<const void*>(kern);
+  LaunchCache& lc = launch_cache();
+  const size_t stride = (static_cast<size_t>(a.K) * (kBF16 ? 2 : 4) + 127) / 128 * 128;
+  int per_sm = 0;
+  // fewer row buffers when each CTA sees only a few rows: more CTAs fit an SM
+  for (;;) {
+    const cudaError_t e = lc.ensure_smem(key, rs.smem);
+    if (e != cudaSuccess) return e;
+    per_sm = lc.blocks_per_sm(key, rs.threads, rs.smem);
+    const int64_t ctas = static_cast<int64_t>(per_sm) * lc.sms();
+    const int64_t rows_per_cta = (a.M + ctas - 1) / ctas;
+    if (rs.nbuf <= 3 || rows_per_cta >= rs.nbuf) break;
+    rs.nbuf = rows_per_cta < 3 ? 3 : static_cast<int>(rows_per_cta);
+    rs.smem = rows_smem(stride, rs.nbuf);
+  }
+  int64_t grid = static_cast<int64_t>(per_sm) * lc.sms();
+  if (grid > a.M) grid = a.M;
+  const double invK = 1.0 / static_cast<double>(a.K);
+  kern<<<static_cast<unsigned>(grid), rs.threads, rs.smem, st>>>(
+      a.x, a.ldx, a.M, a.K, invK, a.gamma, a.beta, a.eps, a.q, a.scale, rs.nbuf, a.err);
+  return cudaGetLastError();
+}
+
+template <bool kBF16, int NORMK, int CH, bool kG, bool kB, bool kF8>
+cudaError_t launch_rows_f(const RowArgs& a, const RowsShape& rs, cudaStream_t st) {
+  // bf16 rows whose chunks split evenly over the threads skip the bounds
+  // checks; the common widths also fix the thread count at compile time
+  // (4096: 128 x 4 chunks, 8192: 128 x 8, 16384: 256 x 8)
+  if constexpr (kBF16) {
+    if (rs.threads * rs.ch == a.K / kChunk) {
+      if (rs.threads == 128) return launch_rows_k<kBF16, NORMK, CH, kG, kB, true, kF8, 128>(a, rs, st);
+      if (rs.threads == 256) return launch_rows_k<kBF16, NORMK, CH, kG, kB, true, kF8, 256>(a, rs, st);
+      return launch_rows_k<kBF16, NORMK, CH, kG, kB, true, kF8>(a, rs, st);
+    }
+  }
+  return launch_rows_k<kBF16, NORMK, CH, kG, kB, false, kF8>(a, rs, st);
+}
+
+template <bool kBF16, int NORMK, int CH, bool kF8>
+cudaError_t launch_rows_g(const RowArgs& a, const RowsShape& rs, cudaStream_t st) {
+  const bool hb = NORMK == 2 && a.beta != nullptr;
+  if (a.gamma) {
+    if (hb) return launch_rows_f<kBF16, NORMK, CH, true, NORMK == 2, kF8>(a, rs, st);
+    return launch_rows_f<kBF16, NORMK, CH, true, false, kF8>(a, rs, st);
+  }
+  if (hb) return launch_rows_f<kBF16, NORMK, CH, false, NORMK == 2, kF8>(a, rs, st);
+  return launch_rows_f<kBF16, NORMK, CH, false, false, kF8>(a, rs, st);
+}
+
+template <bool kBF16, int NORMK, bool kF8>
+cudaError_t launch_rows_c(const RowArgs& a, const RowsShape& rs, cudaStream_t st) {
+  if (rs.ch == 4) return launch_rows_g<kBF16, NORMK, 4, kF8>(a, rs, st);
+  return launch_rows_g<kBF16, NORMK, 8, kF8>(a, rs, st);
+}
+
+// Per-token quantisation with a norm through norm_quant_rows_kernel; false
+// when the shape is not one it takes.
+template <bool kF8>
+bool launch_norm_rows(const RowArgs& a, bool bf16, int norm, cudaStream_t st, cudaError_t* e) {
+  RowsShape rs;
+  if ((norm != SQ_NORM_RMS && norm != SQ_NORM_LAYER) || !rows_shape(a.K, bf16, &rs)) return false;
+  if (bf16)
+    *e = norm == SQ_NORM_RMS ? launch_rows_c<true, 1, kF8>(a, rs, st)
+                             : launch_rows_c<true, 2, kF8>(a, rs, st);
+  else
+    *e = norm == SQ_NORM_RMS ? launch_rows_c<false, 1, kF8>(a, rs, st)
+                             : launch_rows_c<false, 2, kF8>(a, rs, st);
+  return true;
+}
+
 }  // namespace
 
 bool norm_quant_pipe_supported(int K, bool bf16) {
@@ -818,6 +1414,8 @@ cudaError_t launch_norm_quant_pipe(const void* x, bool bf16, int64_t M, int K, i
                                    int8_t* q, float* scale, int* err, cudaStream_t st) {
   if (M == 0) return cudaSuccess;
   const RowArgs a{x, M, K, ldx, gamma, beta, eps, q, scale, nullptr, err};
+  cudaError_t e = cudaSuccess;
+  if (launch_norm_rows<false>(a, bf16, norm, st, &e)) return e;
   return launch_rows<kModeRowQuant>(a, bf16, norm, st);
 }
 
@@ -883,6 +1481,8 @@ cudaError_t launch_norm_quant_fp8_pipe(const void* x, bool bf16, int64_t M, int 
   if (M == 0) return cudaSuccess;
   const RowArgs a{x, M, K, ldx, gamma, beta, eps, reinterpret_cast<int8_t*>(q), scale, nullptr,
                   err};
+  cudaError_t e = cudaSuccess;
+  if (launch_norm_rows<true>(a, bf16, norm, st, &e)) return e;
   return launch_rows<kModeRowQuantF8>(a, bf16, norm, st);
 }
 
