@@ -143,6 +143,43 @@ def test_worked_example_row_on_gpu(golden_dir):
     assert q[mask].min() >= -4 and q[mask].max() <= 4
 
 
+@pytest.mark.parametrize("case", [(2048, 4096, 12288, oracle.NORM_RMS, "bf16", False),
+                                  (37, 4112, 1000, oracle.NORM_LAYER, "bf16", True),
+                                  (5, 64, 48, oracle.NORM_RMS, "f32", False)],
+                         ids=["opt-qkv-2048x4096x12288-rms", "37x4112x1000-layer-relu",
+                              "5x64x48-rms-f32"])
+def test_linear_w8a8_matches_oracle(case):
+    """sq_linear_w8a8, the whole runtime layer in one call (norm + per-token
+    quantisation into caller scratch, then the GEMM with its epilogue), against
+    the oracle's linear: codes, scales and the bf16 output bit for bit; the
+    output and scratch buffers have guard regions that must stay untouched."""
+    M, K, N, norm, dtype, relu = case
+    x = _acts(M, K, dtype)
+    g = RNG.uniform(0.5, 1.5, K).astype(np.float32)
+    b = (RNG.standard_normal(K) * 0.1).astype(np.float32) if norm == oracle.NORM_LAYER else None
+    W = (RNG.standard_normal((N, K)) * 0.02).astype(np.float32)
+    Wq_o, ws_o = oracle.quantize_weights(W, None)
+    Xq_o, xs_o, _, _, out_o = oracle.linear(x, norm, g, b, 1e-5, Wq_o, ws_o, relu)
+    ld = N + 24
+    out_buf = torch.full((M + 2, ld), -7.0, dtype=torch.bfloat16, device="cuda")
+    q_buf = torch.full((M + 2, K), 55, dtype=torch.int8, device="cuda")
+    s_buf = torch.full((M + 8,), -3.0, dtype=torch.float32, device="cuda")
+    out = out_buf[1:M + 1, :N]
+    sq.linear_w8a8(to_gpu(x), norm, to_gpu(g), None if b is None else to_gpu(b), 1e-5,
+                   to_gpu(Wq_o), to_gpu(ws_o), "bf16_relu" if relu else "bf16", out=out,
+                   Xq_scratch=q_buf[1:M + 1], xscale_scratch=s_buf[4:M + 4])
+    assert sq.get_device_error() == 0
+    tie = norm_near_tie_rows(x, norm, 1e-5)
+    assert compare_rows_quant(q_buf[1:M + 1].cpu().numpy(), s_buf[4:M + 4].cpu().numpy(), Xq_o,
+                              xs_o, tie) == 0
+    assert np.array_equal(bf16_bits(out), out_o)
+    ob = bf16_bits(out_buf)
+    assert (ob[0] == bf16_bits(torch.tensor([-7.0], dtype=torch.bfloat16))[0]).all()
+    assert (ob[M + 1] == ob[0]).all() and (ob[1:M + 1, N:] == ob[0, 0]).all()
+    assert torch.all(q_buf[0] == 55) and torch.all(q_buf[M + 1] == 55)
+    assert torch.all(s_buf[:4] == -3.0) and torch.all(s_buf[M + 4:] == -3.0)
+
+
 # ---------------------------------------------------------------------------
 # K2: calibration, smoothing factors + fold, weight smoothing + quantisation
 # ---------------------------------------------------------------------------
@@ -367,8 +404,8 @@ def test_gemm_rowmax_epilogue(shape, relu, path):
 
 
 @pytest.mark.parametrize("split", [0, 2])
-def test_decode_fixup_relu_of_negative_zero(split):
-    """The stream-K fix-up and the split-K reduction apply the same ReLU as
+def test_decode_split_tiles_relu_of_negative_zero(split):
+    """The stream-K tile finish and the split-K reduction apply the same ReLU as
     the main epilogue: a zero token scale gives +0, never -0."""
     M, N, K = 5, 4096, 8192
     A, B = _codes(M, K), _codes(N, K)
@@ -379,6 +416,33 @@ def test_decode_fixup_relu_of_negative_zero(split):
     out = sq.w8a8_gemm_dequant(to_gpu(A), to_gpu(B), to_gpu(xs), to_gpu(ws), "bf16_relu",
                                path_hint=2, split_k=split)
     assert np.array_equal(bf16_bits(out), out_o)
+
+
+@pytest.mark.parametrize("shape", [(1, 10240, 8192), (8, 8192, 8192), (32, 1000, 4112),
+                                   (128, 3000, 2048), (3, 28672, 8192)],
+                         ids=lambda s: "%dx%dx%d" % s)
+def test_decode_streamk_on_a_dirty_workspace_twice(shape):
+    """The stream-K plan's tile counters start every call at zero whatever the
+    workspace holds: a workspace full of garbage, then reused by a second call
+    with other inputs, gives the oracle's bits both times."""
+    M, N, K = shape
+    need = sq.gemm_workspace_size(M, N, K, 0)
+    plan = sq.gemm_plan(M, N, K, 0, 0)
+    assert plan.stream_k == 1 and plan.launches == 1
+    ws_buf = torch.full((max(need, 1),), 0x7f, dtype=torch.uint8, device="cuda")
+    for _ in range(2):
+        A, B = _codes(M, K), _codes(N, K)
+        xs = (RNG.random(M) * 0.05 + 1e-3).astype(np.float32)
+        ws = (RNG.random(N) * 0.002 + 1e-5).astype(np.float32)
+        acc = oracle.gemm_i64(A, B)
+        _, out_o = oracle.epilogue(acc, xs, ws)
+        out = sq.w8a8_gemm_dequant(to_gpu(A), to_gpu(B), to_gpu(xs), to_gpu(ws), "bf16",
+                                   workspace=ws_buf if need else None)
+        raw = sq.w8a8_gemm_dequant(to_gpu(A), to_gpu(B), None, None, "i32",
+                                   workspace=ws_buf if need else None)
+        assert sq.get_device_error() == 0
+        assert np.array_equal(bf16_bits(out), out_o)
+        assert np.array_equal(raw.cpu().numpy().astype(np.int64), acc)
 
 
 def test_gemm_rowmax_rejects_other_epilogues_and_decode_tiles():

@@ -4,9 +4,11 @@ Some callers cannot allocate device memory at the moment they launch the
 GEMM -- an inference-engine plugin whose enqueue path must not allocate, or a
 serving loop whose memory a framework reserved up front.  This entry point
 takes no workspace: its split-K partial sums live in a fixed array owned by the
-library.  The test checks, through the C ABI, that two calls in a row give the
-same output as the allocating entry point with a caller-provided workspace,
-and that a plan needing more scratch than the array holds is refused.
+library.  The tests check, through the C ABI, that two calls in a row give the
+same output as the allocating entry point with a caller-provided workspace
+and as the oracle, that an automatic plan too big for the array falls back to
+whole tiles, and that a plan needing more scratch than the array holds (or an
+output of the wrong shape) is refused.
 
 This file is named so that pytest collects it last.
 """
@@ -14,6 +16,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from w8a8_int8_quantized_norm_b200 import sq
 
 pytestmark = pytest.mark.gpu
@@ -47,7 +50,46 @@ def test_noalloc_matches_allocating_entry_point_twice(epi):
         sq.w8a8_gemm_dequant_noalloc(Xq, Wq, xs, ws, out, epi)
         torch.cuda.synchronize()
         assert torch.equal(out, ref)
+        _check_oracle(out, Xq, Wq, xs, ws, epi)
     assert sq.get_device_error() == 0
+
+
+def _check_oracle(out, Xq, Wq, xs, ws, epi):
+    """The output against the oracle: the exact integer sums, or the
+    oracle's epilogue of them bit for bit."""
+    acc = oracle.gemm_i64(Xq.cpu().numpy(), Wq.cpu().numpy())
+    if epi == "i32":
+        assert np.array_equal(out.cpu().numpy().astype(np.int64), acc)
+    else:
+        _, ref = oracle.epilogue(acc, xs.cpu().numpy(), ws.cpu().numpy())
+        assert np.array_equal(out.view(torch.int16).cpu().numpy().view(np.uint16), ref)
+
+
+def test_noalloc_automatic_plan_falls_back_to_whole_tiles():
+    """With split_k = 0, a decode plan whose stream-K slots would not fit the
+    library's array runs whole tiles (no scratch) and gives the same bits as
+    the allocating entry point's whole-tile plan."""
+    rng = np.random.default_rng(5)
+    M, N, K = 128, 8192, 8192
+    assert sq.gemm_workspace_size(M, N, K, 0) > sq.NOALLOC_SCRATCH_BYTES
+    Xq, Wq, xs, ws = _problem(rng, M, N, K)
+    ref = sq.w8a8_gemm_dequant(Xq, Wq, xs, ws, "bf16", split_k=1)
+    out = torch.full((M, N), 3, dtype=torch.bfloat16, device="cuda")
+    sq.w8a8_gemm_dequant_noalloc(Xq, Wq, xs, ws, out, "bf16")
+    torch.cuda.synchronize()
+    assert sq.get_device_error() == 0
+    assert torch.equal(out, ref)
+    _check_oracle(out, Xq, Wq, xs, ws, "bf16")
+
+
+def test_noalloc_rejects_an_output_of_the_wrong_shape():
+    rng = np.random.default_rng(6)
+    Xq, Wq, xs, ws = _problem(rng, 4, 256, 128)
+    for bad in (torch.empty((4, 255), dtype=torch.bfloat16, device="cuda"),
+                torch.empty((4, 256), dtype=torch.int32, device="cuda"),
+                torch.empty((256, 4), dtype=torch.bfloat16, device="cuda").t()):
+        with pytest.raises(ValueError):
+            sq.w8a8_gemm_dequant_noalloc(Xq, Wq, xs, ws, bad, "bf16")
 
 
 def test_noalloc_refuses_plans_beyond_its_scratch():

@@ -490,6 +490,13 @@ def w8a8_gemm_dequant_noalloc(Xq: torch.Tensor, Wq: torch.Tensor,
     if Xq.dtype != torch.int8 or Wq.dtype != torch.int8 or not Xq.is_contiguous() \
             or not Wq.is_contiguous() or Wq.shape[1] != K:
         raise ValueError("Xq [M,K] and Wq [N,K] must be contiguous int8")
+    # the C ABI cannot see the output's extent: a wrong one would be written past
+    want = torch.int32 if epi == "i32" else torch.bfloat16
+    if (out.dim() != 2 or tuple(out.shape) != (M, N) or out.dtype != want
+            or (N > 1 and out.stride(1) != 1) or out.stride(0) < N
+            or out.device != Xq.device or Wq.device != Xq.device):
+        raise ValueError("out must be a [M, N] = [%d, %d] %s tensor with unit column stride "
+                         "on the device of Xq" % (M, N, want))
     _check(lib().sq_w8a8_gemm_dequant_noalloc(_ptr(Xq), _ptr(Wq), _ptr(x_scale), _ptr(w_scale),
                                               M, N, K, EPI[epi], _ptr(out), out.stride(0),
                                               path_hint, split_k, _stream(stream)),
