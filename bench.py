@@ -669,7 +669,7 @@ def run_gpu(args, w):
     roof["launch_ms_mean"] = t_dom * 1e3
     roof["timing"] = ("CUDA events on the launching stream around each %s GEMM call, in %d "
                       "eager steps run right after the timed ones (a call = the main kernel "
-                      "plus the tile-counter clear or the split-K reduction when the plan has one; the interval includes "
+                      "plus its fix-up kernel when the plan has one; the interval includes "
                       "the event records' own drain)" % (dom.name, n_calls))
 
     line = {

@@ -41,7 +41,7 @@ def test_forward_launch_counts():
     w = S.OPT66B_MLP
     assert pipeline.Block(w, 256, "cpu").forward_launches() == 2 + 1 + \
         sq.gemm_plan(256, 9216, 36864).launches
-    # Llama decode, INT8: four sites, the GEMMs' plans (one kernel each for stream-K)
+    # Llama decode, INT8: four sites, the GEMMs' plans (stream-K fix-ups included)
     w = S.WORKLOADS["llama-block-8192-decode-m8"]
     assert pipeline.Block(w, 8, "cpu").forward_launches() == 4 + _plan_launches(8, w)
     # FP8: whole-K tiles (one kernel per GEMM), the SiLU*up site in one pass

@@ -3,14 +3,11 @@ stream-K work split of decode tiles checked by enumeration.
 
 The stream-K model below restates the kernel's rules (CTA c runs the flattened
 iterations [c*L/G, (c+1)*L/G); a unit that does not cover its whole tile
-writes slot 2c if it is the CTA's first unit, else 2c+1, then takes one ticket
-of its tile; the tile's contributors are the CTA holding its first k-block
-(found from t0*G/L and a step forward) up to the last CTA starting inside it,
-and the one taking the last ticket sums slot 2c of each contributor starting
-inside the tile and 2c+1 of the one starting before it) and checks on many
-shapes that every (tile, k-block) is computed exactly once and that every
-split tile is summed exactly once, from exactly the slots its contributors
-wrote, with as many tickets as contributors."""
+writes slot 2c if it is the CTA's first unit, else 2c+1; the fix-up block of
+boundary c sums, for the tile that boundary falls in, the slots of CTA c-1 and
+of every CTA starting inside the tile) and checks on many shapes that every
+(tile, k-block) is computed exactly once and that every split tile is summed
+exactly once, from exactly the slots its contributors wrote."""
 import ctypes
 
 import pytest
@@ -32,9 +29,8 @@ def _plan(M, N, K, path=0, split=0):
 def test_plan_kinds_and_workspace_agree_with_the_size_query(L):
     p = _plan(1, 28672, 8192)
     assert (p.kernel, p.stream_k, p.split_k, p.tile_m, p.tile_n) == (2, 1, 1, 128, 16)
-    assert p.ctas == SMS and p.launches == 1
-    # two slots of [M][128] INT32 per CTA, then 224 tile tickets (rounded to 256 bytes)
-    assert p.workspace_bytes == 2 * SMS * 128 * 1 * 4 + 1024
+    assert p.ctas == SMS and p.launches == 2
+    assert p.workspace_bytes == 2 * SMS * 128 * 1 * 4
     # 8 x 48 tiles of 256 x 256 fill 74 SM pairs in 6 rounds; 8 x 64 of 256 x 192
     # need 7 rounds of a step that is not proportionally shorter: 256 wins
     p = _plan(2048, 12288, 4096)
@@ -47,7 +43,7 @@ def test_plan_kinds_and_workspace_agree_with_the_size_query(L):
     assert (p.kernel, p.tile_m, p.tile_n, p.ctas) == (0, 128, 256, SMS)
     p = _plan(16, 1024, 8192, split=4)
     assert (p.kernel, p.stream_k, p.split_k, p.workspace_bytes) == (2, 0, 4, 4 * 16 * 1024 * 4)
-    # one whole tile per SM: no tile is shared, no tickets, no workspace
+    # one whole tile per SM: no tile is shared, no fix-up, no workspace
     p = _plan(4, 128 * SMS, 128)
     assert (p.stream_k, p.launches, p.workspace_bytes) == (1, 1, 0)
     for M, N, K, split in [(1, 28672, 8192, 0), (16, 1024, 8192, 0), (128, 57344, 8192, 0),
@@ -87,21 +83,20 @@ def _streamk_model(tiles, kbt, G):
             first = False
     assert len(computed) == L_
     summed = {}
-    tickets = {}
-    for slot, (tile, _, _) in slots.items():
-        tickets[tile] = tickets.get(tile, 0) + 1
-    for tile in sorted(tickets):
+    for c in range(1, G):
+        b = start[c]
+        if b % kbt == 0:
+            continue
+        tile = b // kbt
         t0, t1 = tile * kbt, tile * kbt + kbt
-        c0 = t0 * G // L_  # the kernel's first-contributor search
-        while c0 + 1 < G and start[c0 + 1] <= t0:
-            c0 += 1
-        assert computed[(tile, 0)] == c0
+        if start[c - 1] > t0:
+            continue
         used = []
-        for cc in range(c0, G):
+        for cc in range(c - 1, G):
             if start[cc] >= t1:
                 break
-            used.append(2 * cc if start[cc] >= t0 else 2 * cc + 1)
-        assert len(used) == tickets[tile]  # the last ticket is number len(used)
+            used.append(2 * cc if start[cc] // kbt == tile else 2 * cc + 1)
+        assert tile not in summed
         summed[tile] = used
     # every split tile summed once, from exactly its slots, covering its K range once
     split_tiles = {t for (t, _, _) in slots.values()}
@@ -119,7 +114,7 @@ def _streamk_model(tiles, kbt, G):
                                          (80, 64, 148), (148, 1, 148), (1, 3, 3), (3, 1, 3),
                                          (296, 2, 148), (7, 13, 148), (1000, 5, 148),
                                          (2, 300, 148), (64, 229, 148)])
-def test_streamk_partition_and_tickets_cover_every_iteration_once(tiles, kbt, G):
+def test_streamk_partition_and_fixup_cover_every_iteration_once(tiles, kbt, G):
     G = min(G, tiles * kbt)
     has_slots = _streamk_model(tiles, kbt, G)
     # the planner's workspace decision matches: slots exist iff a boundary is inside a tile

@@ -458,9 +458,7 @@ sq_status sq_w8a8_gemm_plan(int64_t M, int64_t N, int64_t K, int path_hint, int 
   if (plan.pair) ctas *= 2;
   if (ctas > cap) ctas = cap;
   r.ctas = static_cast<int>(M == 0 || N == 0 ? 0 : ctas);
-  // an explicit split adds the reduction kernel; stream-K finishes its split
-  // tiles in the main kernel
-  r.launches = (M == 0 || N == 0) ? 0 : 1 + (plan.splits > 1 ? 1 : 0);
+  r.launches = (M == 0 || N == 0) ? 0 : 1 + (plan.workspace_bytes > 0 ? 1 : 0);
   r.workspace_bytes = plan.workspace_bytes;
   *info = r;
   return SQ_OK;

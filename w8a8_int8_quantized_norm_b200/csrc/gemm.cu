@@ -15,9 +15,7 @@
 //   decode:  P = weight rows, Q = the few token rows (BN = 16..256), so the
 //            weight stream fills the 128-row MMA, and stream-K (or an
 //            explicit split-K) spreads the weight bytes evenly over all SMs;
-//            INT32 partial sums are added exactly (stream-K: by the last CTA
-//            to finish each split tile, in the same launch; an explicit
-//            split: by a second kernel).
+//            INT32 partial sums are added exactly by a second kernel.
 // Prefill also has a CTA-pair variant (tcgen05 cta_group::2, 256-row tiles).
 // Persistent CTAs (one per SM), warp-specialised:
 //   warp 0      TMA producer: 128-byte-swizzled K-major tiles into an
@@ -109,14 +107,11 @@ struct Params {
   // stream-K (decode tiles): CTA c runs the flattened (tile, k-block)
   // iterations [c * sk_iters / G, (c + 1) * sk_iters / G); a tile whose K
   // range is split between CTAs leaves partial sums in slots 2c (the CTA's
-  // first tile) and 2c + 1 (its last), [slot][Q][128]; each contributor then
-  // takes a ticket of the tile (sk_tickets[tile], zero at launch), and the
-  // one that takes the last sums every contributor's slot and runs the
-  // epilogue (sk_finish_tile)
+  // first tile) and 2c + 1 (its last), [slot][Q][128], summed afterwards by
+  // streamk_fixup_kernel
   int streamk;
   int64_t sk_iters;
   int32_t* sk_partial;
-  int32_t* sk_tickets;
   // prefill bf16 epilogues: running max of |out| per P row (token), as
   // binary32 bits, for a following per-token requantisation (or null)
   float* row_absmax;
@@ -195,11 +190,10 @@ __device__ __forceinline__ void work_init(const Params& p, Work& w) {
 // Next unit of the CTA, or false.  slot < 0: the unit ends in the output (or
 // its split-K slice); slot >= 0: a stream-K partial-sum slot.
 __device__ __forceinline__ bool work_next(const Params& p, Work& w, int& pb, int& qb, int& kb0,
-                                          int& kb1, int& split, int& slot, int* tile_out = nullptr) {
+                                          int& kb1, int& split, int& slot) {
   if (p.streamk) {
     if (w.it >= w.it_end) return false;
     const int tile = static_cast<int>(w.it / p.k_blocks);
-    if (tile_out) *tile_out = tile;
     kb0 = static_cast<int>(w.it - static_cast<int64_t>(tile) * p.k_blocks);
     const int64_t left = w.it_end - w.it;
     kb1 = left < p.k_blocks - kb0 ? kb0 + static_cast<int>(left) : p.k_blocks;
@@ -353,86 +347,6 @@ __device__ __forceinline__ float store_chunk(const Params& prm, const uint32_t (
   return 0.0f;
 }
 
-// Named barrier 2 joins the four epilogue warps (128 threads); the OR of
-// their predicates tells every one of them the same answer.
-__device__ __forceinline__ bool epi_sync_or(bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 q, %1, 0;\n\t"
-      "bar.red.or.pred p, 2, 128, q;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(r)
-      : "r"(v ? 1u : 0u)
-      : "memory");
-  return r != 0;
-}
-
-// The CTAs whose stream-K ranges share tile `tile`: c0 (the one running its
-// first k-block) up to, but not including, the first CTA that starts past it.
-__device__ __forceinline__ int sk_first_contributor(const Params& p, int64_t t0) {
-  const int64_t G = gridDim.x;
-  int64_t c = t0 * G / p.sk_iters;  // sk_start(c) <= t0
-  while (c + 1 < G && sk_start(p, c + 1) <= t0) ++c;
-  return static_cast<int>(c);
-}
-
-__device__ __forceinline__ int sk_contributors(const Params& p, int tile) {
-  const int64_t t0 = static_cast<int64_t>(tile) * p.k_blocks, t1 = t0 + p.k_blocks;
-  int n = 0;
-  for (int64_t c = sk_first_contributor(p, t0); c < gridDim.x && sk_start(p, c) < t1; ++c) ++n;
-  return n;
-}
-
-// The last contributor of a split decode tile: thread pl (< 128) sums row
-// pb * 128 + pl of every contributor's slot for all Q tokens (INT32
-// addition is exact: the unsplit accumulator) and applies the epilogue.
-// Each pass gathers 32 tokens of every contributor into registers before it
-// stores anything, so the loads (128 consecutive words across the threads)
-// are all in flight together.
-__device__ void sk_finish_tile(const Params& prm, int tile, int pb, int pl) {
-  const int p = pb * BM + pl;
-  if (p >= prm.P) return;
-  const int64_t t0 = static_cast<int64_t>(tile) * prm.k_blocks, t1 = t0 + prm.k_blocks;
-  const int c0 = sk_first_contributor(prm, t0);
-  const bool raw = prm.epi == SQ_EPI_I32_RAW;
-  const float ws = raw ? 0.0f : __ldg(prm.p_scale + p);
-  const int32_t* __restrict__ part = prm.sk_partial;
-  constexpr int kQ = 32;  // tokens per pass
-  for (int q0 = 0; q0 < prm.Q; q0 += kQ) {
-    const int nq = min(kQ, prm.Q - q0);
-    int32_t acc[kQ];
-#pragma unroll
-    for (int j = 0; j < kQ; ++j) acc[j] = 0;
-    for (int64_t c = c0; c < gridDim.x; ++c) {
-      const int64_t sc = sk_start(prm, c);
-      if (sc >= t1) break;
-      const int64_t slot = sc >= t0 ? 2 * c : 2 * c + 1;
-      const int32_t* src = part + (slot * prm.Q + q0) * BM + pl;
-      if (nq == kQ) {
-#pragma unroll
-        for (int j = 0; j < kQ; ++j) acc[j] += __ldcg(src + j * BM);
-      } else {
-#pragma unroll
-        for (int j = 0; j < kQ; ++j)
-          if (j < nq) acc[j] += __ldcg(src + j * BM);
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < kQ; ++j) {
-      if (j >= nq) break;
-      const int64_t o = static_cast<int64_t>(q0 + j) * prm.ldo + p;
-      if (raw) {
-        static_cast<int32_t*>(prm.out)[o] = acc[j];
-      } else {
-        float t = __fmul_rn(__fmul_rn(__int2float_rn(acc[j]), __ldg(prm.q_scale + q0 + j)), ws);
-        if (prm.epi == SQ_EPI_BF16_RELU) t = t > 0.0f ? t : 0.0f;  // -0 becomes +0
-        static_cast<__nv_bfloat16*>(prm.out)[o] = __float2bfloat16_rn(t);
-      }
-    }
-  }
-}
-
 template <int BN, bool kF8>
 __global__ void __launch_bounds__(kThreads, 1)
     w8a8_gemm_kernel(const __grid_constant__ CUtensorMap mapP,
@@ -483,8 +397,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   const int64_t polls = prm.wait_polls;
   int64_t producer_issued = 0;  // TMA stage loads issued (warp 0)
-  // a kernel launched as a programmatic dependent of this one may be
-  // scheduled now (it waits for this grid's completion before its reads)
+  // the stream-K fix-up kernel (launched as a programmatic dependent) may be
+  // scheduled now; it waits for this grid's completion before reading
   if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (warp == 0) {
@@ -620,15 +534,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t acc_phase = 0;
     Work wk;
     work_init(prm, wk);
-    int pb, qb, kb0, kb1, split, slot, tile = 0;
-    while (work_next(prm, wk, pb, qb, kb0, kb1, split, slot, &tile)) {
+    int pb, qb, kb0, kb1, split, slot;
+    while (work_next(prm, wk, pb, qb, kb0, kb1, split, slot)) {
       bool w = false;
       if (lane == 0) w = wait_phase(TFULL_BAR(acc), acc_phase, polls, abort_flag);
       w = __shfl_sync(0xffffffffu, w, 0);
-      if (!w && lane == 0) fail(prm.error_word, abort_flag);
-      // stream-K: the four warps meet at named barrier 2 for the tickets, so
-      // they leave the loop together
-      if (prm.streamk ? epi_sync_or(!w) : !w) break;
+      if (!w) {
+        if (lane == 0) fail(prm.error_word, abort_flag);
+        break;
+      }
       tc_fence_after();
       const int p = pb * BM + quarter * 32 + lane;
       float rmax = 0.0f;
@@ -653,19 +567,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(TEMPTY_BAR(acc));
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
-      if (slot >= 0 && prm.sk_tickets) {
-        // this CTA's share of a split tile is stored (every epilogue thread,
-        // the barrier); one thread publishes it device-wide and takes a
-        // ticket; the one that takes the last finishes the tile
-        epi_sync_or(false);
-        bool last = false;
-        if (warp == 2 && lane == 0) {
-          __threadfence();
-          last = atomicAdd(prm.sk_tickets + tile, 1) == sk_contributors(prm, tile) - 1;
-          if (last) __threadfence();
-        }
-        if (epi_sync_or(last)) sk_finish_tile(prm, tile, pb, quarter * 32 + lane);
-      }
     }
   }
   __syncthreads();
@@ -1036,6 +937,61 @@ __global__ void __launch_bounds__(kThreads, 1)
 #undef TEMPTY_BAR
 }
 
+// Stream-K fix-up for decode tiles (weight rows on the P side, tokens on the
+// Q side, one Q block).  Block (b, y) looks at the start of CTA c = b + 1: if
+// that iteration lies inside a tile and no earlier CTA starts inside the same
+// tile, the block sums the tile's partial slots (CTA c - 1 up to the last CTA
+// starting before the tile ends) for tokens q = y * kFixQ ... and applies the
+// epilogue; thread = row of the tile's 128 P rows, so every load and store is
+// 128 consecutive words.  INT32 addition is exact, so the result equals the
+// unsplit accumulation.
+constexpr int kFixQ = 8;  // tokens per fix-up block
+
+__global__ void __launch_bounds__(BM) streamk_fixup_kernel(const Params prm, int G) {
+  // launched as a programmatic dependent of the main kernel: everything that
+  // grid wrote is visible once this returns
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int c = static_cast<int>(blockIdx.x) + 1;
+  const int64_t kbt = prm.k_blocks;
+  const int64_t b = static_cast<int64_t>(c) * prm.sk_iters / G;
+  if (b % kbt == 0) return;
+  const int64_t tile = b / kbt;
+  const int64_t t0 = tile * kbt, t1 = t0 + kbt;
+  if (static_cast<int64_t>(c - 1) * prm.sk_iters / G > t0) return;  // not the first boundary
+  int pb, qb;
+  tile_coords(prm, static_cast<int>(tile), pb, qb);
+  const int pl = static_cast<int>(threadIdx.x);
+  const int p = pb * BM + pl;
+  if (p >= prm.P) return;
+  const int q0 = static_cast<int>(blockIdx.y) * kFixQ;
+  const int nq = min(kFixQ, prm.Q - q0);
+  int32_t acc[kFixQ];
+#pragma unroll
+  for (int j = 0; j < kFixQ; ++j) acc[j] = 0;
+  for (int cc = c - 1; cc < G; ++cc) {
+    const int64_t sc = static_cast<int64_t>(cc) * prm.sk_iters / G;
+    if (sc >= t1) break;
+    const int64_t slot = (sc / kbt == tile) ? 2 * cc : 2 * cc + 1;
+    const int32_t* src = prm.sk_partial + (slot * prm.Q + q0) * BM + pl;
+#pragma unroll
+    for (int j = 0; j < kFixQ; ++j)
+      if (j < nq) acc[j] += __ldcg(src + j * BM);
+  }
+  const float ws = prm.epi == SQ_EPI_I32_RAW ? 0.0f : __ldg(prm.p_scale + p);
+#pragma unroll
+  for (int j = 0; j < kFixQ; ++j) {
+    if (j >= nq) break;
+    const int64_t o = static_cast<int64_t>(q0 + j) * prm.ldo + p;
+    if (prm.epi == SQ_EPI_I32_RAW) {
+      static_cast<int32_t*>(prm.out)[o] = acc[j];
+    } else {
+      float t = __fmul_rn(__fmul_rn(__int2float_rn(acc[j]), __ldg(prm.q_scale + q0 + j)), ws);
+      if (prm.epi == SQ_EPI_BF16_RELU) t = t > 0.0f ? t : 0.0f;
+      static_cast<__nv_bfloat16*>(prm.out)[o] = __float2bfloat16_rn(t);
+    }
+  }
+}
+
 // out[m][n] = epilogue(sum_s partial[s][m][n]); INT32 addition is exact, so
 // the split does not change the result.
 __global__ void splitk_reduce_kernel(const int32_t* __restrict__ partial, int splits, int64_t M,
@@ -1191,11 +1147,8 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int path_hint, int split_k, 
     p.sk_iters = iters;
     bool split_tiles = false;
     for (int64_t c = 1; c < G && !split_tiles; ++c) split_tiles = (c * iters / G) % kblocks != 0;
-    // two slots of [M][128] INT32 partial sums per CTA, then one ticket per tile
-    p.workspace_bytes =
-        split_tiles ? static_cast<size_t>(2 * G) * BM * static_cast<size_t>(M) * 4u +
-                          static_cast<size_t>((tiles * 4 + 255) / 256 * 256)
-                    : 0u;
+    p.workspace_bytes = split_tiles ? static_cast<size_t>(2 * G) * BM * static_cast<size_t>(M) * 4u
+                                    : 0u;
     return p;
   } else {
     p.bn = bn_for_tokens(M);
@@ -1263,11 +1216,6 @@ cudaError_t launch_gemm(const GemmPlan& plan, const int8_t* Xq, const int8_t* Wq
   prm.streamk = plan.streamk;
   prm.sk_iters = plan.sk_iters;
   prm.sk_partial = plan.streamk ? static_cast<int32_t*>(workspace) : nullptr;
-  prm.sk_tickets = nullptr;
-  if (plan.streamk && plan.workspace_bytes > 0)
-    prm.sk_tickets = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) +
-                                                static_cast<size_t>(2 * plan.grid) * BM *
-                                                    static_cast<size_t>(M) * 4u);
   if (row_absmax && (plan.swap || epi == SQ_EPI_I32_RAW || epi == SQ_EPI_F32_RAW))
     return cudaErrorInvalidValue;
   prm.row_absmax = row_absmax;
@@ -1296,13 +1244,6 @@ cudaError_t launch_gemm(const GemmPlan& plan, const int8_t* Xq, const int8_t* Wq
   if (!make_map(&mp, Pptr, prm.P, K, BM) || !make_map(&mq, Qptr, prm.Q, K, plan.bn))
     return cudaErrorInvalidValue;
   const int grid = plan.streamk ? plan.grid : (prm.units < sms ? prm.units : sms);
-  if (prm.sk_tickets) {
-    // the tickets start every call at zero (whatever an earlier call, even an
-    // aborted one, left there)
-    const int64_t tiles = (N + BM - 1) / BM;
-    const cudaError_t me = cudaMemsetAsync(prm.sk_tickets, 0, static_cast<size_t>(tiles) * 4u, st);
-    if (me != cudaSuccess) return me;
-  }
   cudaError_t e;
   if (fp8) {
     switch (plan.bn) {
@@ -1324,7 +1265,24 @@ cudaError_t launch_gemm(const GemmPlan& plan, const int8_t* Xq, const int8_t* Wq
     default: return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;
-  if (plan.streamk) return cudaSuccess;  // split tiles were finished in the launch
+  if (plan.streamk) {
+    if (plan.workspace_bytes == 0 || plan.grid < 2) return cudaSuccess;
+    const dim3 fgrid(static_cast<unsigned>(plan.grid - 1),
+                     static_cast<unsigned>((prm.Q + kFixQ - 1) / kFixQ));
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = fgrid;
+    cfg.blockDim = dim3(BM);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t fe = cudaLaunchKernelEx(&cfg, streamk_fixup_kernel, prm, plan.grid);
+    if (fe != cudaSuccess) return fe;
+    return cudaGetLastError();
+  }
   if (plan.splits <= 1) return e;
   const int64_t total = M * N;
   int blocks = static_cast<int>((total + 255) / 256);

@@ -400,7 +400,7 @@ class Block:
     def forward_launches(self) -> int:
         """Kernels one ``forward`` launches: norm-quant per site, and per Linear
         the kernels of its GEMM plan (the main kernel, plus the split-K
-        reduction where the plan has an explicit split)."""
+        reduction or stream-K fix-up where the plan has one)."""
         n = len(self.w.sites)
         n += sum(1 for site in self.w.sites if site.name in self.h)  # h, then its codes
         if self.granularity != "per_token":
