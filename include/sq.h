@@ -391,10 +391,9 @@ typedef struct sq_gemm_plan_info {
   int tile_m;      /* rows of a tile on the MMA M side (tokens, or weight rows for decode) */
   int tile_n;      /* columns of a tile on the MMA N side */
   int split_k;     /* K slices per tile (1: none) */
-  int stream_k;    /* 1: balanced K ranges per SM; split tiles finished in the same launch */
+  int stream_k;    /* 1: balanced K ranges per SM with a fix-up kernel */
   int ctas;        /* CTAs of the main kernel (persistent: at most one per SM) */
-  int launches;    /* kernels the call launches (a stream-K plan with split tiles also
-                      clears its tile counters with one cudaMemsetAsync) */
+  int launches;    /* kernels the call launches */
   size_t workspace_bytes;
 } sq_gemm_plan_info;
 
@@ -420,11 +419,11 @@ sq_status sq_w8a8_gemm_plan(int64_t M, int64_t N, int64_t K, int path_hint, int 
  *   epi      SQ_EPI_BF16, SQ_EPI_BF16_RELU (out is bf16 [M, N], stride ldo)
  *            or SQ_EPI_I32_RAW (out is int32 [M, N], stride ldo)
  *   workspace / ws_bytes  device scratch for partial sums (split-K slices,
- *            or the stream-K slots of decode tiles and one counter per tile,
- *            which the call clears on its stream before its kernel runs); at
- *            least sq_w8a8_gemm_workspace_size(M, N, K, split_k) bytes when
- *            that is non-zero, else may be NULL.  Nothing in it outlives the
- *            call; two calls that overlap on the GPU need two workspaces.
+ *            or the stream-K slots of decode tiles); at least
+ *            sq_w8a8_gemm_workspace_size(M, N, K, split_k) bytes when that is
+ *            non-zero, else may be NULL.  Nothing in it outlives the call, and
+ *            nothing in it has to start at any value; two calls that overlap
+ *            on the GPU need two workspaces.
  *   path_hint 0 = automatic, 1 = prefill tiles (tokens on the MMA M side;
  *            CTA pairs, 256-row tiles 256 or 192 wide on two SMs, the width
  *            chosen to fill the SMs evenly), 2 = decode tiles (weight
@@ -433,10 +432,9 @@ sq_status sq_w8a8_gemm_plan(int64_t M, int64_t N, int64_t K, int path_hint, int 
  *   split_k  0 = automatic, else the number of K slices (decode path only;
  *            the INT32 partial sums are added exactly, so the result does not
  *            depend on it).  The automatic decode plan is stream-K: every SM
- *            runs the same number of 128-deep K steps across tile boundaries;
- *            each SM sharing a tile stores its INT32 partial sums and takes a
- *            ticket of the tile, and the one that takes the last sums the
- *            shares and runs the epilogue (no SM waits for another).
+ *            runs the same number of 128-deep K steps across tile boundaries,
+ *            and tiles shared by two SMs are summed by a second, small kernel
+ *            (launched as a programmatic dependent of the first).
  * Accumulation is exact for K <= SQ_MAX_K (else SQ_ERR_OVERFLOW_RISK).
  * Errors: SQ_ERR_INVALID_ARG, SQ_ERR_ALIGNMENT, SQ_ERR_OVERFLOW_RISK,
  *         SQ_ERR_WORKSPACE, SQ_ERR_UNSUPPORTED, SQ_ERR_CUDA.
@@ -510,8 +508,7 @@ sq_status sq_linear_w8a8(const void* x, sq_dtype dtype, int64_t M, int64_t K, in
  *   - All calls share the one array: calls whose kernels overlap on the GPU
  *     (different streams, or different host threads) race on it.  Calls in
  *     one stream are ordered and safe.  No state carries over between calls:
- *     every partial sum is written before it is read, and the per-tile
- *     counters of a stream-K plan are cleared at the start of every call.
+ *     every partial sum is written before it is read.
  *   - With split_k = 0, a decode plan whose stream-K slots would not fit the
  *     array runs whole tiles instead (split_k = 1, no scratch).  An explicit
  *     split whose partial sums need more than SQ_NOALLOC_SCRATCH_BYTES

@@ -422,13 +422,13 @@ def test_decode_split_tiles_relu_of_negative_zero(split):
                                    (128, 3000, 2048), (3, 28672, 8192)],
                          ids=lambda s: "%dx%dx%d" % s)
 def test_decode_streamk_on_a_dirty_workspace_twice(shape):
-    """The stream-K plan's tile counters start every call at zero whatever the
-    workspace holds: a workspace full of garbage, then reused by a second call
-    with other inputs, gives the oracle's bits both times."""
+    """Nothing of the stream-K plan's workspace has to start at any value: a
+    workspace full of garbage, then reused by a second call with other
+    inputs, gives the oracle's bits both times."""
     M, N, K = shape
     need = sq.gemm_workspace_size(M, N, K, 0)
     plan = sq.gemm_plan(M, N, K, 0, 0)
-    assert plan.stream_k == 1 and plan.launches == 1
+    assert plan.stream_k == 1 and plan.launches == (2 if need else 1)
     ws_buf = torch.full((max(need, 1),), 0x7f, dtype=torch.uint8, device="cuda")
     for _ in range(2):
         A, B = _codes(M, K), _codes(N, K)

@@ -30,15 +30,19 @@ def _cuda():
     assert sq.get_device_error() == 0
 
 
-# (M, N, K, path hint): CTA-pair prefill tiles, single-SM prefill tiles, and
-# decode tiles with split-K partials plus the reduction kernel.  K is long
-# enough that an accumulator is never ready at the epilogue's first probe.
-CASES = [(512, 1024, 16384, 1), (512, 1024, 16384, 3), (16, 2048, 16384, 2)]
+# (M, N, K, path hint, split-K): CTA-pair prefill tiles, single-SM prefill
+# tiles, decode tiles on the automatic stream-K plan (partial sums in the
+# workspace, then the fix-up kernel launched as a programmatic dependent), and
+# decode tiles with an explicit split into four K slices plus the reduction
+# kernel.  K is long enough that an accumulator is never ready at the
+# epilogue's first probe.
+CASES = [(512, 1024, 16384, 1, 0), (512, 1024, 16384, 3, 0), (16, 2048, 16384, 2, 0),
+         (16, 2048, 16384, 2, 4)]
 
 
-@pytest.mark.parametrize("case", CASES, ids=lambda c: "%dx%dx%d-path%d" % c)
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "%dx%dx%d-path%d-split%d" % c)
 def test_wait_limit_reports_timeout_then_recovers(case):
-    M, N, K, path = case
+    M, N, K, path, split = case
     rng = np.random.default_rng(7 + path)
     A = rng.integers(-127, 128, (M, K)).astype(np.int8)
     B = rng.integers(-127, 128, (N, K)).astype(np.int8)
@@ -46,13 +50,13 @@ def test_wait_limit_reports_timeout_then_recovers(case):
     out = torch.zeros((M, N), dtype=torch.int32, device=a.device)
     try:
         sq.set_wait_limit(1)
-        sq.w8a8_gemm_dequant(a, b, None, None, "i32", out=out, path_hint=path)
+        sq.w8a8_gemm_dequant(a, b, None, None, "i32", out=out, path_hint=path, split_k=split)
         status = sq.get_device_error()
     finally:
         sq.set_wait_limit(0)
     assert status == TIMEOUT, sq.status_string(status)
     # the error word was read and cleared; a normal call is exact again
     assert sq.get_device_error() == 0
-    sq.w8a8_gemm_dequant(a, b, None, None, "i32", out=out, path_hint=path)
+    sq.w8a8_gemm_dequant(a, b, None, None, "i32", out=out, path_hint=path, split_k=split)
     assert sq.get_device_error() == 0
     assert np.array_equal(out.cpu().numpy().astype(np.int64), oracle.gemm_i64(A, B))
