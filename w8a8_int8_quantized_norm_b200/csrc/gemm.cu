@@ -80,8 +80,10 @@ struct Cfg {
   static constexpr int A_BYTES = BM * BK;
   static constexpr int B_BYTES = BN * BK;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES_FIT = (196 * 1024) / STAGE_BYTES;
-  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
+  // as many stages as fit 220 KB (at most 12: the narrow decode tiles keep
+  // up to 216 KB of weight blocks in flight per SM)
+  static constexpr int STAGES_FIT = (220 * 1024) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_FIT > 12 ? 12 : STAGES_FIT;
   static constexpr int TMEM_COLS =
       2 * BN <= 32 ? 32 : 2 * BN <= 64 ? 64 : 2 * BN <= 128 ? 128 : 2 * BN <= 256 ? 256 : 512;
   static constexpr int NUM_BARS = 2 * STAGES + 5;
@@ -397,9 +399,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   const int64_t polls = prm.wait_polls;
   int64_t producer_issued = 0;  // TMA stage loads issued (warp 0)
-  // the stream-K fix-up kernel (launched as a programmatic dependent) may be
-  // scheduled now; it waits for this grid's completion before reading
+  // the next kernel (launched as a programmatic dependent: the stream-K
+  // fix-up, or the caller's next call) may be scheduled now; it waits for
+  // this grid's completion before its own reads.  This grid was launched the
+  // same way: everything above touched only its own shared and tensor
+  // memory, and nothing below reads or writes global memory before the
+  // previous grid has completed
   if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -683,6 +690,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   cluster_sync_all();  // both CTAs' barriers exist before any cross-CTA signal
   tc_fence_after();
+  // programmatic launch: let the next kernel be scheduled, then wait for the
+  // previous grid before any global-memory access (above: shared and tensor
+  // memory only)
+  if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const uint32_t tmem_base = *tmem_slot;
   const int64_t polls = prm.wait_polls;
   // the partner's abort flag, so a failing CTA stops its partner quickly
@@ -1059,7 +1071,20 @@ cudaError_t launch_bn(const Params& prm, const CUtensorMap& mp, const CUtensorMa
   cudaError_t e = launch_cache().ensure_smem(
       reinterpret_cast<const void*>(w8a8_gemm_kernel<BN, kF8>), C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  w8a8_gemm_kernel<BN, kF8><<<grid, kThreads, C::SMEM_BYTES, st>>>(mp, mq, prm);
+  // a programmatic dependent of the previous kernel in the stream: its CTAs
+  // set up their barriers and tensor memory while that kernel finishes
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, w8a8_gemm_kernel<BN, kF8>, mp, mq, prm);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -1070,17 +1095,20 @@ cudaError_t launch_pair(const Params& prm, const CUtensorMap& mp, const CUtensor
   auto kern = w8a8_gemm_pair_kernel<TN, kF8>;
   cudaError_t e = launch_cache().ensure_smem(reinterpret_cast<const void*>(kern), C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // a programmatic dependent of the previous kernel in the stream
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = st;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   // as many co-resident CTA pairs as the device holds (one per SM pair)
   static int max_clusters[64] = {};  // per instantiation
   const int dev = LaunchCache::device();

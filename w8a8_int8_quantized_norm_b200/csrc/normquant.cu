@@ -421,6 +421,10 @@ __global__ void __launch_bounds__(PipeBounds<CH, kMode>::kMaxThreads,
   const int64_t first = blockIdx.x;
   const uint8_t* xb = static_cast<const uint8_t*>(x);
   const int64_t row_pitch = ldx * kEsz;
+  // launched as a programmatic dependent: let the next kernel be scheduled,
+  // and touch no global memory before the previous grid has completed
+  if (t == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (t == 0) {
     for (int b = 0; b < nbuf; ++b) mbar_init(bar_base + 8u * b, 1);
@@ -775,6 +779,27 @@ __global__ void __launch_bounds__(PipeBounds<CH, kMode>::kMaxThreads,
   }
 }
 
+// Launch configuration of a row kernel: a programmatic dependent of the
+// previous kernel in the stream (the kernel waits for that grid at its top,
+// so it may start while that grid finishes).
+cudaLaunchConfig_t pdl_config(unsigned grid, int threads, size_t smem, cudaStream_t st) {
+  // initialised once (thread-safe), read-only afterwards
+  static const cudaLaunchAttribute attr = [] {
+    cudaLaunchAttribute a{};
+    a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    a.val.programmaticStreamSerializationAllowed = 1;
+    return a;
+  }();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(static_cast<unsigned>(threads));
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = const_cast<cudaLaunchAttribute*>(&attr);
+  cfg.numAttrs = 1;
+  return cfg;
+}
+
 struct PipeShape {
   int ch, threads, nbuf;
   size_t smem;
@@ -854,9 +879,11 @@ cudaError_t launch_pipe_k(const RowArgs& a, PipeShape ps, cudaStream_t st) {
   // rows per CTA keeps their number (CTAs x K) down
   const int64_t max_grid = kC ? (a.M + 3) / 4 : a.M;
   if (grid > max_grid) grid = max_grid;
-  kern<<<static_cast<unsigned>(grid), ps.threads, ps.smem, st>>>(
-      a.x, a.ldx, a.M, a.K, a.gamma, a.beta, a.eps, a.q, a.scale, a.act_max, ps.nbuf, a.err,
-      a.h_out, a.ldh);
+  cudaLaunchConfig_t cfg = pdl_config(static_cast<unsigned>(grid), ps.threads, ps.smem, st);
+  const cudaError_t le = cudaLaunchKernelEx(&cfg, kern, a.x, a.ldx, a.M, a.K, a.gamma, a.beta,
+                                            a.eps, a.q, a.scale, a.act_max, ps.nbuf, a.err,
+                                            a.h_out, a.ldh);
+  if (le != cudaSuccess) return le;
   return cudaGetLastError();
 }
 
@@ -1105,6 +1132,10 @@ __global__ void __launch_bounds__(RowsBounds<TF, CH>::kThreads, RowsBounds<TF, C
   const uint8_t* xb = static_cast<const uint8_t*>(x);
   const int64_t row_pitch = ldx * kEsz;
   const double Kd = static_cast<double>(K);
+  // launched as a programmatic dependent: let the next kernel be scheduled,
+  // and touch no global memory before the previous grid has completed
+  if (t == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (t == 0) {
     for (int b = 0; b <= nbuf; ++b) mbar_init(bar_base + 8u * b, 1);
@@ -1345,8 +1376,10 @@ cudaError_t launch_rows_k(const RowArgs& a, RowsShape rs, cudaStream_t st) {
   int64_t grid = static_cast<int64_t>(per_sm) * lc.sms();
   if (grid > a.M) grid = a.M;
   const double invK = 1.0 / static_cast<double>(a.K);
-  kern<<<static_cast<unsigned>(grid), rs.threads, rs.smem, st>>>(
-      a.x, a.ldx, a.M, a.K, invK, a.gamma, a.beta, a.eps, a.q, a.scale, rs.nbuf, a.err);
+  cudaLaunchConfig_t cfg = pdl_config(static_cast<unsigned>(grid), rs.threads, rs.smem, st);
+  const cudaError_t le = cudaLaunchKernelEx(&cfg, kern, a.x, a.ldx, a.M, a.K, invK, a.gamma,
+                                            a.beta, a.eps, a.q, a.scale, rs.nbuf, a.err);
+  if (le != cudaSuccess) return le;
   return cudaGetLastError();
 }
 
