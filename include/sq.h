@@ -34,6 +34,8 @@
  *   - FP8 (e4m3) codes with the same smoothing ([LLMint8] "example . what you
  *     get"): sq_norm_smooth_quant_per_token_fp8, sq_smooth_quantize_weights_fp8,
  *     sq_silu_mul_quant_per_token_fp8, sq_fp8_gemm_dequant;
+ *   - the row split of a Linear over several GPUs (exact collectives between
+ *     the calls): sq_row_absmax, sq_dequant_i32;
  *   - planning and allocation-free variants: sq_w8a8_gemm_plan,
  *     sq_w8a8_gemm_workspace_size, sq_w8a8_gemm_dequant_noalloc; the two
  *     halves of step 2 (sq_weight_column_max, sq_smooth_scales_from_maxima).
@@ -272,6 +274,48 @@ sq_status sq_norm_smooth_quant_per_tensor(const void* x, sq_dtype dtype, int64_t
 sq_status sq_quant_per_token_given_absmax(const void* x, sq_dtype dtype, int64_t M, int64_t K,
                                           int64_t ldx, const float* row_absmax, int8_t* Xq,
                                           float* x_scale, void* stream);
+
+/*
+ * The row split of a Linear over several GPUs (each GPU holds a slice of the
+ * input channels of x and of W; [SQ-depth] "Where the scales go in a decoder
+ * block": o_proj / down_proj read unsmoothed inputs, still quantised per
+ * token).  The per-token step must be the whole row's, and the accumulator
+ * the whole sum, so the slices meet twice, both times exactly:
+ *   1. sq_row_absmax on the local slice; all-reduce MAX of the [M] maxima;
+ *   2. sq_quant_per_token_given_absmax with the reduced maxima (the step and
+ *      the codes are those of the unsplit row), then sq_w8a8_gemm_dequant
+ *      with SQ_EPI_I32_RAW on the local slice; all-reduce SUM of the [M, N]
+ *      INT32 partial sums (integer addition: the unsplit accumulator);
+ *   3. sq_dequant_i32: the epilogue of the summed accumulator.
+ * The weights are quantised the same way once: the row maxima of the local
+ * [N, K_slice] slice, all-reduce MAX, sq_quant_per_token_given_absmax.
+ * The result is bit-identical to the unsplit call.
+ *
+ * sq_row_absmax -- row_absmax[m] = max_k |x[m, k]| (no norm).
+ *   x          device [M, K] bf16 or fp32, row stride ldx
+ *   row_absmax device [M] fp32 OUT, 16-byte aligned
+ * Rows as for sq_quant_per_token_given_absmax.
+ * Errors: SQ_ERR_INVALID_ARG, SQ_ERR_ALIGNMENT, SQ_ERR_UNSUPPORTED, SQ_ERR_CUDA.
+ */
+sq_status sq_row_absmax(const void* x, sq_dtype dtype, int64_t M, int64_t K, int64_t ldx,
+                        float* row_absmax, void* stream);
+
+/*
+ * sq_dequant_i32 -- the GEMM's dequantising epilogue applied to an INT32
+ * accumulator held in memory: out[m, n] = bf16(fl32(fl32(fl32(acc[m, n]) *
+ * x_scale[m]) * w_scale[n])), ReLU before the rounding for SQ_EPI_BF16_RELU.
+ * [SQ-depth] "Granularity": both scales applied to the INT32 accumulator.
+ *   acc        device [M, N] int32, row stride lda (>= N)
+ *   x_scale    device [M] fp32; w_scale device [N] fp32
+ *   epi        SQ_EPI_BF16 or SQ_EPI_BF16_RELU
+ *   out        device [M, N] bf16, row stride ldo (>= N)
+ * Errors: SQ_ERR_INVALID_ARG (sizes, strides, null pointers, other
+ *         epilogues), SQ_ERR_ALIGNMENT (acc not 4-byte, out not 2-byte
+ *         aligned), SQ_ERR_CUDA.
+ */
+sq_status sq_dequant_i32(const int32_t* acc, int64_t M, int64_t N, int64_t lda,
+                         const float* x_scale, const float* w_scale, sq_epilogue epi, void* out,
+                         int64_t ldo, void* stream);
 
 /*
  * FP8 (e4m3) W8A8: the same smoothing, FP8 codes instead of INT8.

@@ -445,6 +445,49 @@ def test_decode_streamk_on_a_dirty_workspace_twice(shape):
         assert np.array_equal(raw.cpu().numpy().astype(np.int64), acc)
 
 
+@pytest.mark.parametrize("cuts", [(0, 4096, 8192), (0, 1024, 5120, 8192), (0, 16, 8192)],
+                         ids=["2-even", "3-uneven", "2-thin"])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_row_split_slices_equal_the_unsplit_layer(cuts, dtype):
+    """The row split of ksplit through the C ABI, its slices run one after
+    another on this GPU and reduced by torch (max of the row maxima, sum of
+    the INT32 partials): weight codes and scales, token scales, the
+    accumulator and the bf16 output equal the oracle's unsplit layer."""
+    from w8a8_int8_quantized_norm_b200 import ksplit
+    M, N, K = 37, 1000, cuts[-1]
+    x = _acts(M, K, dtype)
+    W = (RNG.standard_normal((N, K)) * 0.02).astype(np.float32)
+    if dtype == "bf16":
+        W = S.to_bf16_bits(W)
+    Wq_o, ws_o = oracle.quantize_weights(W, None)
+    _, xs_o, acc_o, _, out_o = oracle.linear(x, oracle.NORM_NONE, None, None, 1e-5, Wq_o, ws_o)
+    spans = list(zip(cuts, cuts[1:]))
+    xg = [to_gpu(np.ascontiguousarray(x[:, a:b])) for a, b in spans]
+    Wg = [to_gpu(np.ascontiguousarray(W[:, a:b])) for a, b in spans]
+    am_w = torch.stack([ksplit.LibOps.row_absmax(w) for w in Wg]).amax(0)
+    qw = [ksplit.LibOps.quant_given(w, am_w) for w in Wg]
+    am = torch.stack([ksplit.shard_row_max(v) for v in xg]).amax(0)
+    parts = [ksplit.shard_partial(v, am, q[0]) for v, q in zip(xg, qw)]
+    acc = parts[0][0].clone()
+    for p_, _ in parts[1:]:
+        acc += p_
+    out = ksplit.finish(acc, parts[0][1], qw[0][1])
+    assert sq.get_device_error() == 0
+    for (a, b), (wq, ws) in zip(spans, qw):
+        assert np.array_equal(ws.cpu().numpy().view(np.uint32), ws_o.view(np.uint32))
+        assert np.array_equal(wq.cpu().numpy(), Wq_o[:, a:b])
+    for _, xs in parts:
+        assert np.array_equal(xs.cpu().numpy().view(np.uint32), xs_o.view(np.uint32))
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), acc_o)
+    assert np.array_equal(bf16_bits(out), out_o)
+    assert np.array_equal(am.cpu().numpy(), np.abs(x.view(np.float32) if dtype == "f32" else
+                                                   _bf16_to_f32(x)).max(axis=1))
+
+
+def _bf16_to_f32(bits):
+    return (bits.astype(np.uint32) << 16).view(np.float32)
+
+
 def test_gemm_rowmax_rejects_other_epilogues_and_decode_tiles():
     A, B = to_gpu(_codes(8, 64)), to_gpu(_codes(32, 64))
     xs, ws = torch.ones(8, device="cuda"), torch.ones(32, device="cuda")

@@ -176,6 +176,38 @@ def test_given_absmax_quant_rejects_bad_arguments(L):
     assert call(M=0, am=None, q=None, s=None) == 0
 
 
+def test_row_split_calls_reject_bad_arguments(L):
+    f = L.sq_row_absmax
+
+    def call(x=A16, dt=1, M=4, K=64, ld=64, am=A16):
+        return f(x, dt, M, K, ld, am, None)
+
+    assert call(x=None) == 1
+    assert call(dt=7) == 1
+    assert call(ld=32) == 1
+    assert call(am=None) == 1
+    assert call(am=A8) == 3
+    assert call(K=60) == 3
+    assert call(K=48000, ld=48000) == 2
+    assert call(M=0, am=None) == 0
+    g = L.sq_dequant_i32
+
+    def dq(acc=A16, M=4, N=8, lda=8, xs=A16, ws=A16, epi=0, out=A16, ldo=8):
+        return g(acc, M, N, lda, xs, ws, epi, out, ldo, None)
+
+    assert dq(acc=None) == 1
+    assert dq(xs=None) == 1
+    assert dq(ws=None) == 1
+    assert dq(out=None) == 1
+    assert dq(lda=4) == 1
+    assert dq(ldo=4) == 1
+    assert dq(epi=2) == 1               # the raw accumulator is the input, not an epilogue
+    assert dq(M=-1) == 1
+    assert dq(acc=ctypes.c_void_p(0x10002)) == 3
+    assert dq(out=ctypes.c_void_p(0x10001)) == 3
+    assert dq(M=0, acc=None, xs=None, ws=None, out=None) == 0
+
+
 def test_silu_mul_quant_rejects_bad_arguments(L):
     f = L.sq_silu_mul_quant_per_token
 

@@ -312,6 +312,31 @@ sq_status sq_quant_per_token_given_absmax(const void* x, sq_dtype dtype, int64_t
                                            row_absmax, Xq, x_scale, err, as_stream(stream)));
 }
 
+sq_status sq_row_absmax(const void* x, sq_dtype dtype, int64_t M, int64_t K, int64_t ldx,
+                        float* row_absmax, void* stream) {
+  sq_status st = check_tensor_rows(x, dtype, M, K, ldx, SQ_NORM_NONE, nullptr, nullptr, 0.0f);
+  if (st != SQ_OK) return st;
+  if (M == 0) return SQ_OK;
+  if ((st = check_vec(row_absmax, true)) != SQ_OK) return st;
+  int* err = device_error_word();
+  if (!err) return SQ_ERR_CUDA;
+  return from_cuda(launch_row_absmax_pipe(x, dtype == SQ_BF16, M, static_cast<int>(K), ldx,
+                                          row_absmax, err, as_stream(stream)));
+}
+
+sq_status sq_dequant_i32(const int32_t* acc, int64_t M, int64_t N, int64_t lda,
+                         const float* x_scale, const float* w_scale, sq_epilogue epi, void* out,
+                         int64_t ldo, void* stream) {
+  if (M < 0 || N < 0 || lda < N || ldo < N) return SQ_ERR_INVALID_ARG;
+  if (epi != SQ_EPI_BF16 && epi != SQ_EPI_BF16_RELU) return SQ_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return SQ_OK;
+  if (!acc || !out || !x_scale || !w_scale) return SQ_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(acc) & 3u) || (reinterpret_cast<uintptr_t>(out) & 1u))
+    return SQ_ERR_ALIGNMENT;
+  return from_cuda(launch_dequant_i32(acc, M, N, lda, x_scale, w_scale, epi, out, ldo,
+                                      as_stream(stream)));
+}
+
 sq_status sq_norm_smooth_quant_per_token_fp8(const void* x, sq_dtype dtype, int64_t M, int64_t K,
                                              int64_t ldx, sq_norm norm,
                                              const float* gamma_folded, const float* beta_folded,

@@ -59,6 +59,9 @@ constexpr int UMMA_K = 32;  // K of one kind::i8 MMA
 // every four MMAs.)
 constexpr int kThreads = 224;
 constexpr int kSchedWarp = 6;
+// Weight blocks (128 rows x 128 bytes) a decode CTA prefetches into L2 before
+// the previous grid has finished: 256 KB per SM, 38 MB over 148 SMs.
+constexpr int kPrefetchBlocks = 16;
 
 // Named barrier 1 joins the MMA-issuing warp and its scheduling warp once per
 // wait; the OR of the two warps' predicates tells both whether to stop.
@@ -406,6 +409,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   // memory, and nothing below reads or writes global memory before the
   // previous grid has completed
   if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (prm.swap && threadIdx.x == 0) {
+    // decode tiles: while the previous grid finishes, pull the first weight
+    // blocks of this CTA's range into L2 (a prefetch only: the loads below
+    // still come after the wait and see whatever that grid wrote)
+    Work wk;
+    work_init(prm, wk);
+    int pb, qb, kb0, kb1, split, slot, n = 0;
+    while (n < kPrefetchBlocks && work_next(prm, wk, pb, qb, kb0, kb1, split, slot))
+      for (int kb = kb0; kb < kb1 && n < kPrefetchBlocks; ++kb, ++n)
+        tma_prefetch_l2_2d(&mapP, kb * BK, pb * BM);
+  }
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (warp == 0) {
@@ -1004,18 +1018,19 @@ __global__ void __launch_bounds__(BM) streamk_fixup_kernel(const Params prm, int
   }
 }
 
-// out[m][n] = epilogue(sum_s partial[s][m][n]); INT32 addition is exact, so
-// the split does not change the result.
+// out[m][n] = epilogue(sum_s partial[s][m][n]) (slices of lda * M words,
+// rows of stride lda); INT32 addition is exact, so the split does not change
+// the result.  With one slice it is the epilogue of a given accumulator.
 __global__ void splitk_reduce_kernel(const int32_t* __restrict__ partial, int splits, int64_t M,
-                                     int64_t N, const float* __restrict__ x_scale,
+                                     int64_t N, int64_t lda, const float* __restrict__ x_scale,
                                      const float* __restrict__ w_scale, int epi, void* out,
                                      int64_t ldo) {
-  const int64_t total = M * N;
+  const int64_t total = M * N, slice = M * lda;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t m = i / N, n = i - m * N;
     int32_t acc = 0;
-    for (int s = 0; s < splits; ++s) acc += partial[s * total + i];
+    for (int s = 0; s < splits; ++s) acc += partial[s * slice + m * lda + n];
     if (epi == SQ_EPI_I32_RAW) {
       static_cast<int32_t*>(out)[m * ldo + n] = acc;
     } else {
@@ -1316,7 +1331,19 @@ cudaError_t launch_gemm(const GemmPlan& plan, const int8_t* Xq, const int8_t* Wq
   int blocks = static_cast<int>((total + 255) / 256);
   if (blocks > sms * 8) blocks = sms * 8;
   splitk_reduce_kernel<<<blocks, 256, 0, st>>>(static_cast<const int32_t*>(workspace), plan.splits,
-                                               M, N, x_scale, w_scale, epi, out, ldo);
+                                               M, N, N, x_scale, w_scale, epi, out, ldo);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dequant_i32(const int32_t* acc, int64_t M, int64_t N, int64_t lda,
+                               const float* x_scale, const float* w_scale, int epi, void* out,
+                               int64_t ldo, cudaStream_t st) {
+  if (M == 0 || N == 0) return cudaSuccess;
+  const int64_t total = M * N;
+  int blocks = static_cast<int>((total + 255) / 256);
+  const int cap = num_sms_current_device() * 8;
+  if (blocks > cap) blocks = cap;
+  splitk_reduce_kernel<<<blocks, 256, 0, st>>>(acc, 1, M, N, lda, x_scale, w_scale, epi, out, ldo);
   return cudaGetLastError();
 }
 

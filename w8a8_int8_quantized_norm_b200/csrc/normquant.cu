@@ -357,6 +357,7 @@ enum RowMode : int {
   kModeSiluMul = 5,     // per-row codes of h = SiLU(gate) * up (rows hold [gate | up])
   kModeRowQuantF8 = 6,  // per-row step and FP8 (e4m3) codes
   kModeSiluMulF8 = 7,   // SiLU * up rows with FP8 codes
+  kModeRowAbsmax = 8,   // each row's max |y| into act_max[row], no codes
 };
 
 // Bytes of one input row: SiLU * up rows hold both halves.
@@ -455,7 +456,8 @@ __global__ void __launch_bounds__(PipeBounds<CH, kMode>::kMaxThreads,
   }
   constexpr bool kCalib = kMode == kModeColMax;
   constexpr bool kF8 = kMode == kModeRowQuantF8 || kMode == kModeSiluMulF8;
-  constexpr bool kRowMax = kMode == kModeRowQuant || kMode == kModeTensorMax || kGLU || kF8;
+  constexpr bool kRowMax = kMode == kModeRowQuant || kMode == kModeTensorMax || kGLU || kF8 ||
+                           kMode == kModeRowAbsmax;
   float cta_max = 0.0f;  // tensor-max mode, thread 0
   // fixed-step mode: the one step, from the given max |y|
   float fstep = 0.0f, frstep = 0.0f;
@@ -670,6 +672,8 @@ __global__ void __launch_bounds__(PipeBounds<CH, kMode>::kMaxThreads,
 
       if constexpr (kMode == kModeTensorMax) {
         if (t == 0) cta_max = fmaxf(cta_max, am);
+      } else if constexpr (kMode == kModeRowAbsmax) {
+        if (t == 0) act_max[row] = am;
       } else if constexpr (kF8) {
         // ---- per-token FP8 quantisation: step = fl32(max / 448); a zero or
         // subnormal step makes the row all zero codes with step 0
@@ -1487,6 +1491,16 @@ cudaError_t launch_quant_given_pipe(const void* x, bool bf16, int64_t M, int K, 
                   const_cast<float*>(row_absmax), err};
   if (bf16) return launch_pipe_n<true, 0, kModeGivenQuant>(a, ps, st);
   return launch_pipe_n<false, 0, kModeGivenQuant>(a, ps, st);
+}
+
+cudaError_t launch_row_absmax_pipe(const void* x, bool bf16, int64_t M, int K, int64_t ldx,
+                                   float* row_absmax, int* err, cudaStream_t st) {
+  if (M == 0) return cudaSuccess;
+  PipeShape ps;
+  if (!pipe_shape(K, bf16, false, &ps)) return cudaErrorInvalidValue;
+  const RowArgs a{x, M, K, ldx, nullptr, nullptr, 0.0f, nullptr, nullptr, row_absmax, err};
+  if (bf16) return launch_pipe_n<true, 0, kModeRowAbsmax>(a, ps, st);
+  return launch_pipe_n<false, 0, kModeRowAbsmax>(a, ps, st);
 }
 
 bool silu_mul_pipe_supported(int I) {

@@ -92,6 +92,9 @@ cudaError_t launch_quant_fixed_pipe(const void* x, bool bf16, int64_t M, int K, 
                                     int norm, const float* gamma, const float* beta, float eps,
                                     const float* absmax, int8_t* q, float* scale, int* err,
                                     cudaStream_t st);
+// Each row's max |x| (no norm) into row_absmax[M].
+cudaError_t launch_row_absmax_pipe(const void* x, bool bf16, int64_t M, int K, int64_t ldx,
+                                   float* row_absmax, int* err, cudaStream_t st);
 // Per-row codes from given row maxima (no norm): row i's step is
 // fl32(row_absmax[i] / 127); codes clamp to +-127.
 cudaError_t launch_quant_given_pipe(const void* x, bool bf16, int64_t M, int K, int64_t ldx,
@@ -136,5 +139,11 @@ cudaError_t launch_gemm(const GemmPlan& plan, const int8_t* Xq, const int8_t* Wq
                         int num_sms, int64_t wait_polls, int* error_word, cudaStream_t st,
                         float* row_absmax = nullptr, bool fp8 = false);
 int num_sms_current_device();
+// The dequantising epilogue of an INT32 accumulator matrix acc [M, N]
+// (stride lda): out = bf16(fl32(fl32(fl32(acc) x_scale[m]) w_scale[n])), ReLU
+// for SQ_EPI_BF16_RELU.
+cudaError_t launch_dequant_i32(const int32_t* acc, int64_t M, int64_t N, int64_t lda,
+                               const float* x_scale, const float* w_scale, int epi, void* out,
+                               int64_t ldo, cudaStream_t st);
 
 }  // namespace sq

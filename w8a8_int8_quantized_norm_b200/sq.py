@@ -38,7 +38,8 @@ EXPORTS = (
     "sq_w8a8_gemm_dequant_rowmax", "sq_quant_per_token_given_absmax",
     "sq_silu_mul_quant_per_token", "sq_norm_smooth_quant_per_token_fp8",
     "sq_smooth_quantize_weights_fp8", "sq_fp8_gemm_dequant", "sq_weight_column_max",
-    "sq_smooth_scales_from_maxima", "sq_silu_mul_quant_per_token_fp8",
+    "sq_smooth_scales_from_maxima", "sq_silu_mul_quant_per_token_fp8", "sq_row_absmax",
+    "sq_dequant_i32",
 )
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -114,6 +115,8 @@ def _declare(L):
     L.sq_w8a8_gemm_dequant_rowmax.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _I32, _P, _I64,
                                               _P, _I32, _P]
     L.sq_quant_per_token_given_absmax.argtypes = [_P, _I32, _I64, _I64, _I64, _P, _P, _P, _P]
+    L.sq_row_absmax.argtypes = [_P, _I32, _I64, _I64, _I64, _P, _P]
+    L.sq_dequant_i32.argtypes = [_P, _I64, _I64, _I64, _P, _P, _I32, _P, _I64, _P]
     L.sq_silu_mul_quant_per_token.argtypes = [_P, _I32, _I64, _I64, _I64, _P, _P, _P, _I64, _P]
     L.sq_norm_smooth_quant_per_token_fp8.argtypes = [_P, _I32, _I64, _I64, _I64, _I32, _P, _P,
                                                      _F32, _P, _P, _P]
@@ -334,6 +337,36 @@ def quant_per_token_given_absmax(x: torch.Tensor, row_absmax: torch.Tensor, Xq=N
         _ptr(x), _dtype_code(x), M, K, ld, _ptr(_vec(row_absmax, M, "row_absmax")), _ptr(Xq),
         _ptr(x_scale), _stream(stream)), "sq_quant_per_token_given_absmax")
     return Xq, x_scale
+
+
+def row_absmax(x: torch.Tensor, out=None, stream=None) -> torch.Tensor:
+    """max_k |x[m, k]| per row of x [M, K] (no norm), fp32 [M]."""
+    M, K, ld = _rows(x, "x")
+    if out is None:
+        out = torch.empty(M, dtype=torch.float32, device=x.device)
+    _check(lib().sq_row_absmax(_ptr(x), _dtype_code(x), M, K, ld, _ptr(_vec(out, M, "out")),
+                               _stream(stream)), "sq_row_absmax")
+    return out
+
+
+def dequant_i32(acc: torch.Tensor, x_scale: torch.Tensor, w_scale: torch.Tensor,
+                epi: str = "bf16", out=None, stream=None) -> torch.Tensor:
+    """The GEMM's epilogue on an INT32 accumulator acc [M, N]: bf16 [M, N]."""
+    if acc.dim() != 2 or acc.dtype != torch.int32 or (acc.shape[1] > 1 and acc.stride(1) != 1):
+        raise ValueError("acc must be an int32 [M, N] tensor with unit column stride")
+    M, N = acc.shape
+    if epi not in ("bf16", "bf16_relu"):
+        raise ValueError("epi must be bf16 or bf16_relu")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=acc.device)
+    if tuple(out.shape) != (M, N) or out.dtype != torch.bfloat16 or \
+            (N > 1 and out.stride(1) != 1):
+        raise ValueError("out must be a bf16 [M, N] tensor with unit column stride")
+    _check(lib().sq_dequant_i32(_ptr(acc), M, N, max(acc.stride(0), N),
+                                _ptr(_vec(x_scale, M, "x_scale")), _ptr(_vec(w_scale, N, "w_scale")),
+                                EPI[epi], _ptr(out), max(out.stride(0), N), _stream(stream)),
+           "sq_dequant_i32")
+    return out
 
 
 def silu_mul_quant_per_token(gate_up: torch.Tensor, Xq=None, x_scale=None, h_out=None,
