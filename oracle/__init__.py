@@ -76,6 +76,11 @@ def _declare(L):
     L.oracle_fold_norm.argtypes = [_P, _P, _P, _I64, _P, _P]
     L.oracle_smooth_weights.restype = None
     L.oracle_smooth_weights.argtypes = [_P, ctypes.c_int, _I64, _I64, _I64, _P, _P]
+    L.oracle_llmint8_outliers.restype = _I64
+    L.oracle_llmint8_outliers.argtypes = [_P, _I64, ctypes.c_float, _P, _P]
+    L.oracle_llmint8_combine.restype = None
+    L.oracle_llmint8_combine.argtypes = [_P, _I64, _I64, _P, ctypes.c_int, _I64, _P, ctypes.c_int,
+                                         _I64, _P, _I64, ctypes.c_int, _P, _P]
     L.oracle_gemm_i64.restype = None
     L.oracle_gemm_i64.argtypes = [_P, _P, _I64, _I64, _I64, _P]
     L.oracle_epilogue.restype = None
@@ -415,3 +420,50 @@ def linear(x, norm_kind, gamma_f, beta_f, eps, Wq, w_scale, relu=False):
     acc = gemm_i64(Xq, Wq)
     o32, out = epilogue(acc, xs, w_scale, relu)
     return Xq, xs, acc, o32, out
+
+
+# --------------------------------------------------------------------------
+# Comparator: LLM.int8()'s mixed-precision decomposition
+# --------------------------------------------------------------------------
+
+def llmint8_outliers(col_absmax, tau: float = 6.0):
+    """(mask [K] fp32: 0 on outlier channels, idx: the outlier channels
+    ascending) for O = {j : col_absmax[j] >= tau}."""
+    col = _f32(col_absmax)
+    K = col.shape[0]
+    mask = np.empty(K, np.float32)
+    idx = np.empty(K, np.int32)
+    n = lib().oracle_llmint8_outliers(_ptr(col), K, float(np.float32(tau)), _ptr(mask), _ptr(idx))
+    return mask, idx[:n].copy()
+
+
+def llmint8_combine(o32, x, W, idx, relu=False):
+    """(y fp32 [M,N], out bf16 bits): the INT8 lane's o32 plus the 16-bit lane
+    over the channels idx (fp64 accumulation, ascending), one fp32 add."""
+    o32 = np.ascontiguousarray(o32, dtype=np.float32)
+    x = np.ascontiguousarray(x)
+    W = np.ascontiguousarray(W)
+    M, N = o32.shape
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    y = np.empty((M, N), np.float32)
+    out = np.empty((M, N), np.uint16)
+    lib().oracle_llmint8_combine(_ptr(o32), M, N, _ptr(x), _dtype_code(x), x.shape[1], _ptr(W),
+                                 _dtype_code(W), W.shape[1], _ptr(idx), idx.shape[0],
+                                 int(bool(relu)), _ptr(y), _ptr(out))
+    return y, out
+
+
+def llmint8_linear(x, Wq, w_scale, W, tau: float = 6.0, relu: bool = False):
+    """The comparator layer end to end ([LLMint8] "Fix 1", "going deeper"):
+    outlier channels from this batch's column maxima, per-token INT8 codes of
+    the other channels, the INT8 GEMM and its epilogue, the 16-bit lane and
+    the sum.  Wq / w_scale: W quantised per output channel (quantize_weights
+    with no smoothing).  Returns a dict of every stage."""
+    col = calibrate_absmax(x, NORM_NONE)
+    mask, idx = llmint8_outliers(col, tau)
+    Xq, xs = norm_quant(x, NORM_NONE, mask, None)
+    acc = gemm_i64(Xq, Wq)
+    o32, _ = epilogue(acc, xs, w_scale, False)
+    y, out = llmint8_combine(o32, x, W, idx, relu)
+    return {"col_absmax": col, "mask": mask, "idx": idx, "Xq": Xq, "x_scale": xs, "acc": acc,
+            "o32": o32, "y": y, "out": out}

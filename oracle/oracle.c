@@ -684,3 +684,72 @@ int oracle_num_threads(void) {
   return 1;
 #endif
 }
+
+/* ------------------------------------------------------------------------ */
+/* Comparator: LLM.int8()'s mixed-precision decomposition                    */
+/* ------------------------------------------------------------------------ */
+/*
+ * [LLMint8] "Fix 1: give the outliers their own lane (LLM.int8())" and
+ * "going deeper -- LLM.int8() decomposition": the outlier channels are
+ * O = { j : max_t |X[t, j]| >= tau } (tau = 6 in the paper); the layer is
+ * X[:, O] W[O, :] in 16-bit plus the vector-wise INT8 product of the other
+ * channels (one absmax scale per token row of X, one per output channel of
+ * W), and the two results are added.
+ *
+ * oracle_llmint8_outliers: from col_absmax[j] = max_t |X[t, j]| (the
+ * calibration max with no norm), mask[j] = 0 for j in O and 1 otherwise (the
+ * INT8 lane quantises x * mask: the channels of O give code 0 and do not
+ * count towards a token's step), idx = the channels of O in ascending order.
+ * Returns |O|.
+ * Parity: pinned by the pages' one-token example (channels 1512 and 2817
+ * taken out, the step of the rest 2/127), the tau boundary (>=) and an empty
+ * set.
+ */
+int64_t oracle_llmint8_outliers(const float* col_absmax, int64_t K, float tau, float* mask,
+                                int32_t* idx) {
+  int64_t n = 0;
+  for (int64_t j = 0; j < K; ++j) {
+    const int out = col_absmax[j] >= tau;
+    mask[j] = out ? 0.0f : 1.0f;
+    if (out) idx[n++] = (int32_t)j;
+  }
+  return n;
+}
+
+/*
+ * oracle_llmint8_combine: y[m, n] = fl32(o32[m, n] + y16[m, n]), ReLU when
+ * asked (as in oracle_epilogue), out = bf16_rne(y), where o32 is the INT8
+ * lane's dequantised value (oracle_epilogue's o32 without ReLU) and
+ *   y16[m, n] = fl32(s),  s = sum over j in O, ascending, of x[m, j] * w[n, j]
+ * accumulated in fp64 (s starts at +0; each step s = fl64(s + x w)).  The
+ * product of two bf16 (or two fp32) values is exact in fp64, so s is a fixed
+ * sequence of roundings.  Readings (the pages give no precision): the 16-bit
+ * lane multiplies the unquantised inputs in their stored type with a wide
+ * accumulator; W is quantised once per output channel over all its input
+ * channels (the stored INT8 weights, whose outlier columns the INT8 lane
+ * never meets because their activation codes are 0); "add the two results"
+ * is one fp32 addition.
+ * y_out and out_bf16 are each nullable.
+ * Parity: pinned by exact integer dot products on small inputs, by the empty
+ * outlier set (equal to the plain W8A8 layer) and by the all-outlier set
+ * (equal to a sequential fp64 dot product).
+ */
+void oracle_llmint8_combine(const float* o32, int64_t M, int64_t N, const void* x, int xdtype,
+                            int64_t ldx, const void* W, int wdtype, int64_t ldw,
+                            const int32_t* idx, int64_t nout, int relu, float* y_out,
+                            uint16_t* out_bf16) {
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t n = 0; n < N; ++n) {
+      double s = 0.0;
+      for (int64_t i = 0; i < nout; ++i) {
+        const int64_t j = idx[i];
+        const double xv = (double)load_elem(x, xdtype, m * ldx + j);
+        const double wv = (double)load_elem(W, wdtype, n * ldw + j);
+        s = s + xv * wv;
+      }
+      float y = o32[m * N + n] + (float)s;
+      if (relu && !(y > 0.0f)) y = 0.0f;
+      if (y_out) y_out[m * N + n] = y;
+      if (out_bf16) out_bf16[m * N + n] = oracle_f32_to_bf16_bits(y);
+    }
+}

@@ -657,3 +657,120 @@ def test_fp8_epilogue_matches_float32_arithmetic():
         assert np.array_equal(o32, ref)
         tb = torch.from_numpy(ref).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
         assert np.array_equal(out, tb)
+
+
+# ---------------------------------------------------------------------------
+# Comparator: LLM.int8()'s mixed-precision decomposition
+# ---------------------------------------------------------------------------
+
+def test_llmint8_worked_token_row(golden_dir):
+    """[LLMint8] "one token through a layer": LLM.int8() sends channels 1512
+    and 2817 (45 and -60, above tau = 6) through 16-bit; the remaining
+    channels get the step 2/127, about 30 times finer than 60/127."""
+    g = _golden(golden_dir, "token_row_outliers.json")
+    K = g["row_width"]
+    lo, hi = g["ordinary_range"]
+    row = RNG.uniform(lo, hi, K).astype(np.float32)
+    row[[0, 1]] = [lo, hi]
+    for ch, v in g["outliers"].items():
+        row[int(ch)] = v
+    x = row[None, :]
+    col = oracle.calibrate_absmax(x, oracle.NORM_NONE)
+    mask, idx = oracle.llmint8_outliers(col, 6.0)
+    assert list(idx) == sorted(int(c) for c in g["outliers"])
+    assert mask[idx].tolist() == [0.0, 0.0] and mask.sum() == K - 2
+    Xq, xs = oracle.norm_quant(x, oracle.NORM_NONE, mask, None)
+    p, tol = g["printed"], g["printed_precision"]
+    assert xs[0] == np.float32(np.float32(2.0) / np.float32(127.0))
+    assert abs(xs[0] - p["step_without_outliers"]) <= tol["step_without_outliers"]
+    assert Xq[0, idx].tolist() == [0, 0]
+    assert Xq[0].min() == -127 and Xq[0].max() == 127
+
+
+def test_llmint8_threshold_is_inclusive():
+    col = np.array([6.0, np.nextafter(np.float32(6.0), np.float32(0.0)), 7.5, 0.0, 60.0],
+                   np.float32)
+    mask, idx = oracle.llmint8_outliers(col, 6.0)
+    assert idx.tolist() == [0, 2, 4]
+    assert mask.tolist() == [0.0, 1.0, 0.0, 1.0, 0.0]
+
+
+def _small_layer(rng, M, N, K, scale=1.0):
+    x = (rng.standard_normal((M, K)) * scale).astype(np.float32)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    return x, W
+
+
+def test_llmint8_without_outliers_is_the_plain_w8a8_layer():
+    rng = np.random.default_rng(11)
+    x, W = _small_layer(rng, 9, 24, 64, scale=1.0)  # |x| < 6 everywhere
+    assert np.abs(x).max() < 6.0
+    Wq, ws = oracle.quantize_weights(W, None)
+    r = oracle.llmint8_linear(x, Wq, ws, W)
+    assert r["idx"].size == 0 and (r["mask"] == 1.0).all()
+    _, _, acc, o32, out = oracle.linear(x, oracle.NORM_NONE, None, None, 1e-5, Wq, ws)
+    assert np.array_equal(r["acc"], acc)
+    assert np.array_equal(r["y"].view(np.uint32), o32.view(np.uint32))
+    assert np.array_equal(r["out"], out)
+
+
+def test_llmint8_sixteen_bit_lane_is_an_exact_dot_product():
+    """Integer-valued inputs: every product and partial sum is exact, so the
+    16-bit lane is the integer dot product over the outlier channels, and
+    with every channel an outlier (tau = 0: every max is >= 0) the INT8 lane is
+    empty (zero codes, zero steps) and y is that dot product."""
+    rng = np.random.default_rng(12)
+    M, N, K = 5, 7, 48
+    x = rng.integers(-40, 41, (M, K)).astype(np.float32)
+    W = rng.integers(-9, 10, (N, K)).astype(np.float32)
+    Wq, ws = oracle.quantize_weights(W, None)
+    r = oracle.llmint8_linear(x, Wq, ws, W, tau=0.0)
+    assert r["idx"].tolist() == list(range(K))
+    assert (r["Xq"] == 0).all() and (r["x_scale"] == 0).all() and (r["o32"] == 0).all()
+    exact = x.astype(np.int64) @ W.astype(np.int64).T
+    assert np.array_equal(r["y"], exact.astype(np.float32))
+    # a chosen outlier set: the lane sums only those channels
+    col = np.zeros(K, np.float32)
+    chosen = [3, 17, 40]
+    col[chosen] = 10.0
+    _, idx = oracle.llmint8_outliers(col, 6.0)
+    y, _ = oracle.llmint8_combine(np.zeros((M, N), np.float32), x, W, idx)
+    assert np.array_equal(y, (x[:, chosen].astype(np.int64) @
+                              W[:, chosen].astype(np.int64).T).astype(np.float32))
+
+
+def test_llmint8_sixteen_bit_lane_in_fp64_order():
+    """Real-valued bf16 inputs: the lane equals a sequential fp64 sum of the
+    exact products in ascending channel order, rounded once to fp32."""
+    rng = np.random.default_rng(13)
+    M, N, K = 3, 4, 64
+    x = S.to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32) * 9)
+    W = S.to_bf16_bits(rng.standard_normal((N, K)).astype(np.float32) * 0.02)
+    xf = (x.astype(np.uint32) << 16).view(np.float32)
+    wf = (W.astype(np.uint32) << 16).view(np.float32)
+    idx = np.array([1, 5, 6, 30, 63], np.int32)
+    y, out = oracle.llmint8_combine(np.zeros((M, N), np.float32), x, W, idx)
+    for m in range(M):
+        for n in range(N):
+            s = 0.0
+            for j in idx:
+                s = s + float(xf[m, j]) * float(wf[n, j])
+            assert y[m, n] == np.float32(s)
+
+
+def test_llmint8_is_finer_than_plain_int8_on_outlier_channels():
+    """The pages' claim in numbers: with a few outlier channels, the plain
+    per-token INT8 layer's output error is several times LLM.int8()'s."""
+    rng = np.random.default_rng(14)
+    M, N, K = 32, 64, 256
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    x[:, [7, 200]] *= np.float32(50.0)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    Wq, ws = oracle.quantize_weights(W, None)
+    ref = x.astype(np.float64) @ W.astype(np.float64).T
+    _, _, _, o32, _ = oracle.linear(x, oracle.NORM_NONE, None, None, 1e-5, Wq, ws)
+    r = oracle.llmint8_linear(x, Wq, ws, W)
+    assert r["idx"].tolist() == [7, 200]
+    e_plain = np.linalg.norm(o32 - ref) / np.linalg.norm(ref)
+    e_int8 = np.linalg.norm(r["y"] - ref) / np.linalg.norm(ref)
+    assert e_int8 * 5 < e_plain
