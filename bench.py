@@ -537,6 +537,78 @@ def decode_sweep(args, w, blk, dev, stream, flusher, peaks, seed, rank):
     return res
 
 
+def comparator_leg(args, w, inp, dev, stream, flusher, peaks, rank):
+    """LLM.int8()'s decomposition against the W8A8 layer on one Linear of the
+    block that has no norm in front (o_proj, the attention-output activations
+    with their outlier channels): the runtime forward of plain per-token INT8
+    (no smoothing), of LLM.int8() (tau = 6) and of SmoothQuant (alpha of the
+    workload, 1/s as a per-channel multiplier: the fold with gamma = 1), each
+    one CUDA graph timed like the main loop, and each one's output error on
+    sampled token rows against an fp64 product of the same bf16 inputs."""
+    import torch
+    from w8a8_int8_quantized_norm_b200 import llmint8, pipeline, sq
+    from w8a8_int8_quantized_norm_b200 import synthetic as S
+    lin = next(l for l in w.linears if l.name == "o_proj")
+    site = w.site(lin.site)
+    M, K, N = w.M, site.K, lin.N
+    x = _to_dev(inp.x[site.name], dev)
+    W = _to_dev(inp.W[lin.name], dev)
+    xcal = _to_dev(S.activations(w, site.name, w.M_cal, "x_cal", args.seed), dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    # plain per-token INT8 and SmoothQuant: the same two calls, with or without s
+    Wq_p, ws_p = sq.smooth_quantize_weights(W, None)
+    am = torch.zeros(K, **f32)
+    sq.calibrate_absmax(xcal, sq.NORM_NONE, act_max=am)
+    s_, gf = torch.empty(K, **f32), torch.empty(K, **f32)
+    sq.compute_smooth_scales(am, [W], w.alpha, w.clamp_eps, None, None, s=s_, gamma_folded=gf)
+    Wq_s, ws_s = sq.smooth_quantize_weights(W, s_)
+    xq, xs = torch.empty((M, K), dtype=torch.int8, device=dev), torch.empty(M, **f32)
+    outs = {k: torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            for k in ("plain_int8", "llm_int8", "smoothquant")}
+
+    def w8a8(mult, Wq, ws, out):
+        sq.norm_smooth_quant_per_token(x, sq.NORM_NONE, mult, None, 0.0, Xq=xq, x_scale=xs)
+        sq.w8a8_gemm_dequant(xq, Wq, xs, ws, "bf16", out=out)
+
+    comp = llmint8.LLMInt8Linear(W, 6.0).prepare()
+    runs = {"plain_int8": lambda: w8a8(None, Wq_p, ws_p, outs["plain_int8"]),
+            "llm_int8": lambda: comp.forward(x, out=outs["llm_int8"]),
+            "smoothquant": lambda: w8a8(gf, Wq_s, ws_s, outs["smoothquant"])}
+    launches = {"plain_int8": 1 + sq.gemm_plan(M, N, K).launches,
+                "llm_int8": comp.launches(M),
+                "smoothquant": 1 + sq.gemm_plan(M, N, K).launches}
+    res = {}
+    for name, fn in runs.items():
+        graph = pipeline.capture_graph(fn)
+        for _ in range(3):
+            flusher()
+            graph.replay()
+        n = max(5, min(args.steps, 20))
+        ms = _timed_replays(graph, n, flusher, stream)
+        t = sum(ms) / n / 1e3
+        del graph
+        res[name] = {"ms": t * 1e3, "tops": 2.0 * M * N * K / t / 1e12,
+                     "launches": launches[name]}
+    torch.cuda.synchronize(dev)
+    # output error on sampled rows against the fp64 product of the bf16 inputs
+    rows = _sample_rows(M, 64, seed=5)
+    xr = inp.x[site.name][rows]
+    bf = lambda a: (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    ref = bf(xr) @ bf(inp.W[lin.name]).T
+    for name in runs:
+        got = outs[name][torch.from_numpy(rows).to(dev)].float().cpu().numpy().astype(np.float64)
+        res[name]["rel_error"] = float(np.linalg.norm(got - ref) / np.linalg.norm(ref))
+    res["smoothquant"]["alpha"] = w.alpha
+    return {"linear": "%s %dx%dx%d (M x K x N), input: %s activations" % (
+                lin.name, M, K, N, site.name),
+            "tau": 6.0, "outlier_channels": int(comp.count.item()),
+            "error": "relative Frobenius error of the bf16 output on %d token rows against "
+                     "the fp64 product of the same bf16 x and W" % len(rows),
+            "timing": "each method's runtime calls as one CUDA graph, L2 flushed before "
+                      "every replay",
+            **res}
+
+
 def run_gpu(args, w):
     import torch
     import torch.distributed as dist
@@ -710,6 +782,9 @@ def run_gpu(args, w):
     if (not args.no_decode and not decode and w.name.startswith("llama-block-8192")
             and args.format == "int8" and args.granularity == "per_token"):
         line["decode"] = decode_sweep(args, w, blk, dev, stream, flusher, peaks, args.seed, rank)
+    if (not args.no_comparator and w.name.startswith("llama-block-8192") and not decode
+            and args.format == "int8"):
+        line["comparator"] = comparator_leg(args, w, inp, dev, stream, flusher, peaks, rank)
     err = sq.get_device_error()
     if err:
         raise SystemExit("device error %s during the benchmark" % sq.status_string(err))
@@ -796,6 +871,8 @@ def main(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-comparator", action="store_true",
+                    help="skip LLM.int8()'s decomposition against the W8A8 layer on o_proj")
     ap.add_argument("--no-decode", action="store_true",
                     help="skip the decode sweep (M = 1, 8, 32, 128 on the Llama block weights)")
     ap.add_argument("--granularity", default="per_token",

@@ -36,6 +36,8 @@
  *     sq_silu_mul_quant_per_token_fp8, sq_fp8_gemm_dequant;
  *   - the row split of a Linear over several GPUs (exact collectives between
  *     the calls): sq_row_absmax, sq_dequant_i32;
+ *   - LLM.int8()'s decomposition as a comparator on the same inputs
+ *     ([LLMint8] "Fix 1"): sq_llmint8_outliers, sq_llmint8_combine;
  *   - planning and allocation-free variants: sq_w8a8_gemm_plan,
  *     sq_w8a8_gemm_workspace_size, sq_w8a8_gemm_dequant_noalloc; the two
  *     halves of step 2 (sq_weight_column_max, sq_smooth_scales_from_maxima).
@@ -316,6 +318,62 @@ sq_status sq_row_absmax(const void* x, sq_dtype dtype, int64_t M, int64_t K, int
 sq_status sq_dequant_i32(const int32_t* acc, int64_t M, int64_t N, int64_t lda,
                          const float* x_scale, const float* w_scale, sq_epilogue epi, void* out,
                          int64_t ldo, void* stream);
+
+/*
+ * LLM.int8()'s mixed-precision decomposition, a comparator of the smoothed
+ * W8A8 layer on the same inputs.
+ * [LLMint8] "Fix 1: give the outliers their own lane (LLM.int8())", "going
+ * deeper -- LLM.int8() decomposition": the outlier channels
+ * O = { j : max_t |X[t, j]| >= tau } (tau = 6 in the paper) go through a
+ * 16-bit product, the other channels through INT8 with one absmax scale per
+ * token row and one per output channel, and the two results are added.  The
+ * layer is five calls:
+ *   1. col_absmax [K] = max_t |X[t, j]|: sq_weight_column_max with x as its
+ *      one "weight" (or sq_calibrate_absmax, SQ_NORM_NONE, into zeros);
+ *   2. sq_llmint8_outliers: mask (0 on O, 1 elsewhere) and the channels of O;
+ *   3. sq_norm_smooth_quant_per_token (SQ_NORM_NONE, multiplier = mask): the
+ *      other channels' per-token codes (O's codes are 0 and do not set the
+ *      step);
+ *   4. sq_w8a8_gemm_dequant with SQ_EPI_I32_RAW and W quantised per output
+ *      channel (sq_smooth_quantize_weights with s = NULL);
+ *   5. sq_llmint8_combine.
+ *
+ * sq_llmint8_outliers -- mask[j] = col_absmax[j] >= tau ? 0 : 1; idx[0 ..
+ * count) = the channels j with col_absmax[j] >= tau, ascending; *count their
+ * number.
+ *   col_absmax device [K] fp32 IN;  mask device [K] fp32 OUT
+ *   idx        device [K] int32 OUT;  count device [1] int32 OUT
+ *   tau        >= 0
+ * K up to SQ_LLMINT8_MAX_K.  Pointers 4-byte aligned.
+ * Errors: SQ_ERR_INVALID_ARG, SQ_ERR_ALIGNMENT, SQ_ERR_CUDA.
+ */
+#define SQ_LLMINT8_MAX_K 1048576
+
+sq_status sq_llmint8_outliers(const float* col_absmax, int64_t K, float tau, float* mask,
+                              int32_t* idx, int32_t* count, void* stream);
+
+/*
+ * sq_llmint8_combine -- out[m, n] = bf16(y), y = fl32(y8 + y16) (ReLU on y
+ * for SQ_EPI_BF16_RELU), where
+ *   y8  = fl32(fl32(fl32(acc[m, n]) * x_scale[m]) * w_scale[n]), the INT8
+ *         lane dequantised as the GEMM epilogue does;
+ *   y16 = fl32(s), s = the sum over the channels idx[0 .. *count), in that
+ *         order, of x[m, j] * W[n, j] in fp64 (each product is exact in
+ *         fp64: the 16-bit lane on the unquantised inputs).
+ *   acc      device [M, N] int32, row stride lda (the INT8 lane, SQ_EPI_I32_RAW)
+ *   x_scale  device [M] fp32 (step 3);  w_scale device [N] fp32
+ *   x        device [M, K] bf16 / fp32, row stride ldx (the layer's input)
+ *   W        device [N, K] bf16 / fp32, row stride ldw (the unquantised weights)
+ *   idx, count  from sq_llmint8_outliers
+ *   out      device [M, N] bf16, row stride ldo
+ * Errors: SQ_ERR_INVALID_ARG (sizes, strides, dtypes, null pointers, other
+ *         epilogues), SQ_ERR_ALIGNMENT, SQ_ERR_CUDA.
+ */
+sq_status sq_llmint8_combine(const int32_t* acc, int64_t M, int64_t N, int64_t lda,
+                             const float* x_scale, const float* w_scale, const void* x,
+                             sq_dtype x_dtype, int64_t ldx, const void* W, sq_dtype w_dtype,
+                             int64_t ldw, int64_t K, const int32_t* idx, const int32_t* count,
+                             sq_epilogue epi, void* out, int64_t ldo, void* stream);
 
 /*
  * FP8 (e4m3) W8A8: the same smoothing, FP8 codes instead of INT8.

@@ -488,6 +488,48 @@ def _bf16_to_f32(bits):
     return (bits.astype(np.uint32) << 16).view(np.float32)
 
 
+@pytest.mark.parametrize("case", [(37, 4096, 1000, "bf16", 6.0, False),
+                                  (5, 64, 48, "f32", 6.0, True),
+                                  (64, 512, 300, "bf16", 1.0, False),
+                                  (9, 256, 128, "bf16", 1e9, False),
+                                  (2048, 4096, 12288, "bf16", 6.0, False)],
+                         ids=["37x4096x1000", "5x64x48-f32-relu", "many-outliers",
+                              "no-outliers", "opt-qkv-sampled"])
+def test_llmint8_comparator_matches_oracle(case):
+    """LLM.int8()'s decomposition through the C ABI against the oracle: the
+    column maxima, outlier mask and list, codes, token scales, the INT32
+    accumulator and the bf16 output, bit for bit (the full-size case on
+    sampled rows; its outlier set comes from all tokens on both sides)."""
+    from w8a8_int8_quantized_norm_b200 import llmint8
+    M, K, N, dtype, tau, relu = case
+    x = _acts(M, K, dtype, outliers=8)
+    W = (RNG.standard_normal((N, K)) * 0.02).astype(np.float32)
+    if dtype == "bf16":
+        W = S.to_bf16_bits(W)
+    Wq_o, ws_o = oracle.quantize_weights(W, None)
+    lin = llmint8.LLMInt8Linear(to_gpu(W), tau).prepare()
+    out = lin.forward(to_gpu(x), "bf16_relu" if relu else "bf16")
+    assert sq.get_device_error() == 0
+    assert np.array_equal(lin.Wq.cpu().numpy(), Wq_o)
+    col = oracle.calibrate_absmax(x, oracle.NORM_NONE)
+    mask, idx = oracle.llmint8_outliers(col, tau)
+    assert np.array_equal(lin.col.cpu().numpy().view(np.uint32), col.view(np.uint32))
+    assert np.array_equal(lin.mask.cpu().numpy(), mask)
+    n = int(lin.count.item())
+    assert n == idx.size and np.array_equal(lin.idx[:n].cpu().numpy(), idx)
+    rows = np.arange(M) if M <= 64 else np.sort(RNG.choice(M, 48, replace=False))
+    xr = np.ascontiguousarray(x[rows])
+    Xq_o, xs_o = oracle.norm_quant(xr, oracle.NORM_NONE, mask, None)
+    acc_o = oracle.gemm_i64(Xq_o, Wq_o)
+    o32, _ = oracle.epilogue(acc_o, xs_o, ws_o, False)
+    _, out_o = oracle.llmint8_combine(o32, xr, W, idx, relu)
+    st = lin.stages
+    assert np.array_equal(st["Xq"].cpu().numpy()[rows], Xq_o)
+    assert np.array_equal(st["x_scale"].cpu().numpy()[rows].view(np.uint32), xs_o.view(np.uint32))
+    assert np.array_equal(st["acc"].cpu().numpy()[rows].astype(np.int64), acc_o)
+    assert np.array_equal(bf16_bits(out)[rows], out_o)
+
+
 def test_gemm_rowmax_rejects_other_epilogues_and_decode_tiles():
     A, B = to_gpu(_codes(8, 64)), to_gpu(_codes(32, 64))
     xs, ws = torch.ones(8, device="cuda"), torch.ones(32, device="cuda")

@@ -208,6 +208,39 @@ def test_row_split_calls_reject_bad_arguments(L):
     assert dq(M=0, acc=None, xs=None, ws=None, out=None) == 0
 
 
+def test_llmint8_calls_reject_bad_arguments(L):
+    f = L.sq_llmint8_outliers
+
+    def out_(col=A16, K=64, tau=6.0, mask=A16, idx=A16, cnt=A16):
+        return f(col, K, tau, mask, idx, cnt, None)
+
+    assert out_(col=None) == 1
+    assert out_(K=0) == 1
+    assert out_(K=(1 << 20) + 1) == 1
+    assert out_(tau=-1.0) == 1
+    assert out_(tau=float("nan")) == 1
+    assert out_(idx=None) == 1
+    assert out_(cnt=ctypes.c_void_p(0x10002)) == 3
+    g = L.sq_llmint8_combine
+
+    def comb(acc=A16, M=4, N=8, lda=8, xs=A16, ws=A16, x=A16, xd=1, ldx=64, W=A16, wd=1,
+             ldw=64, K=64, idx=A16, cnt=A16, epi=0, out=A16, ldo=8):
+        return g(acc, M, N, lda, xs, ws, x, xd, ldx, W, wd, ldw, K, idx, cnt, epi, out, ldo, None)
+
+    assert comb(acc=None) == 1
+    assert comb(idx=None) == 1
+    assert comb(cnt=None) == 1
+    assert comb(W=None) == 1
+    assert comb(ldx=32) == 1
+    assert comb(ldw=32) == 1
+    assert comb(lda=4) == 1
+    assert comb(xd=7) == 1
+    assert comb(epi=2) == 1
+    assert comb(x=ctypes.c_void_p(0x10001)) == 3
+    assert comb(W=ctypes.c_void_p(0x10002), wd=0) == 3
+    assert comb(M=0, acc=None, out=None) == 0
+
+
 def test_silu_mul_quant_rejects_bad_arguments(L):
     f = L.sq_silu_mul_quant_per_token
 

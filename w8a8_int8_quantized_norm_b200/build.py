@@ -22,7 +22,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 OUT_DIR = os.path.join(PKG, "lib")
 LIB = os.path.join(OUT_DIR, "libsq.so")
-SOURCES = ["rows.cu", "normquant.cu", "gemm.cu", "api.cu", "noalloc.cu"]
+SOURCES = ["rows.cu", "normquant.cu", "gemm.cu", "api.cu", "noalloc.cu", "llmint8.cu"]
 HEADERS = ["sq_device.cuh", "sq_launch.h"]
 PUBLIC_HEADER = os.path.join(ROOT, "include", "sq.h")
 

@@ -337,6 +337,39 @@ sq_status sq_dequant_i32(const int32_t* acc, int64_t M, int64_t N, int64_t lda,
                                       as_stream(stream)));
 }
 
+sq_status sq_llmint8_outliers(const float* col_absmax, int64_t K, float tau, float* mask,
+                              int32_t* idx, int32_t* count, void* stream) {
+  if (K <= 0 || K > SQ_LLMINT8_MAX_K || !(tau >= 0.0f)) return SQ_ERR_INVALID_ARG;
+  if (!col_absmax || !mask || !idx || !count) return SQ_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(col_absmax) | reinterpret_cast<uintptr_t>(mask) |
+       reinterpret_cast<uintptr_t>(idx) | reinterpret_cast<uintptr_t>(count)) & 3u)
+    return SQ_ERR_ALIGNMENT;
+  return from_cuda(launch_llmint8_outliers(col_absmax, K, tau, mask, idx, count,
+                                           as_stream(stream)));
+}
+
+sq_status sq_llmint8_combine(const int32_t* acc, int64_t M, int64_t N, int64_t lda,
+                             const float* x_scale, const float* w_scale, const void* x,
+                             sq_dtype x_dtype, int64_t ldx, const void* W, sq_dtype w_dtype,
+                             int64_t ldw, int64_t K, const int32_t* idx, const int32_t* count,
+                             sq_epilogue epi, void* out, int64_t ldo, void* stream) {
+  if (M < 0 || N < 0 || K <= 0 || lda < N || ldo < N || ldx < K || ldw < K)
+    return SQ_ERR_INVALID_ARG;
+  if (!valid_dtype(x_dtype) || !valid_dtype(w_dtype)) return SQ_ERR_INVALID_ARG;
+  if (epi != SQ_EPI_BF16 && epi != SQ_EPI_BF16_RELU) return SQ_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return SQ_OK;
+  if (!acc || !x_scale || !w_scale || !x || !W || !idx || !count || !out)
+    return SQ_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(acc) & 3u) || (reinterpret_cast<uintptr_t>(out) & 1u) ||
+      (reinterpret_cast<uintptr_t>(x) % dsize(x_dtype)) ||
+      (reinterpret_cast<uintptr_t>(W) % dsize(w_dtype)))
+    return SQ_ERR_ALIGNMENT;
+  return from_cuda(launch_llmint8_combine(acc, M, N, lda, x_scale, w_scale, x, x_dtype == SQ_BF16,
+                                          ldx, W, w_dtype == SQ_BF16, ldw, idx, count,
+                                          epi == SQ_EPI_BF16_RELU ? 1 : 0, out, ldo,
+                                          as_stream(stream)));
+}
+
 sq_status sq_norm_smooth_quant_per_token_fp8(const void* x, sq_dtype dtype, int64_t M, int64_t K,
                                              int64_t ldx, sq_norm norm,
                                              const float* gamma_folded, const float* beta_folded,

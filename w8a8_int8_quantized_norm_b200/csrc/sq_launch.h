@@ -121,6 +121,15 @@ cudaError_t launch_smooth_finalize(const float* act_max, const float* wmax, floa
                                    double alpha, float clamp_eps, const float* gamma,
                                    const float* beta, float* gf, float* bfo, cudaStream_t st);
 
+// llmint8.cu (the LLM.int8() comparator)
+cudaError_t launch_llmint8_outliers(const float* col_absmax, int64_t K, float tau, float* mask,
+                                    int32_t* idx, int32_t* count, cudaStream_t st);
+cudaError_t launch_llmint8_combine(const int32_t* acc, int64_t M, int64_t N, int64_t lda,
+                                   const float* x_scale, const float* w_scale, const void* x,
+                                   bool x_bf16, int64_t ldx, const void* W, bool w_bf16,
+                                   int64_t ldw, const int32_t* idx, const int32_t* count, int relu,
+                                   void* out, int64_t ldo, cudaStream_t st);
+
 // gemm.cu
 struct GemmPlan {
   int swap;       // 0: tokens on the MMA M side (prefill); 1: weight rows (decode)

@@ -444,7 +444,7 @@ class Block:
         return graph
 
 
-def _capture(fn, warmup: int = 1):
+def capture_graph(fn, warmup: int = 1):
     """Records ``fn`` (a sequence of library calls on the current stream,
     possibly forking to others and joining back) into a CUDA graph after
     ``warmup`` runs outside the capture (the first use of each kernel sets
@@ -464,14 +464,14 @@ def _capture(fn, warmup: int = 1):
 def capture_forward(blk: Block, x, warmup: int = 1):
     """The runtime rows of one step (norm + per-token quantisation, GEMMs with
     the dequant epilogue, for every Linear) as one CUDA graph."""
-    return _capture(lambda: blk.forward(x), warmup)
+    return capture_graph(lambda: blk.forward(x), warmup)
 
 
 def capture_prepare(blk: Block, x_cal, W, gamma, beta, warmup: int = 1):
     """The offline rows (calibration, smoothing factors and fold, weight
     smoothing and quantisation) as one CUDA graph, calibration beside the
     weight column maxima."""
-    return _capture(lambda: blk.prepare_two_streams(x_cal, W, gamma, beta), warmup)
+    return capture_graph(lambda: blk.prepare_two_streams(x_cal, W, gamma, beta), warmup)
 
 
 # Thin functional wrappers (used by tests and the smoke check).

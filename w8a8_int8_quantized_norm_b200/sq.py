@@ -39,8 +39,9 @@ EXPORTS = (
     "sq_silu_mul_quant_per_token", "sq_norm_smooth_quant_per_token_fp8",
     "sq_smooth_quantize_weights_fp8", "sq_fp8_gemm_dequant", "sq_weight_column_max",
     "sq_smooth_scales_from_maxima", "sq_silu_mul_quant_per_token_fp8", "sq_row_absmax",
-    "sq_dequant_i32",
+    "sq_dequant_i32", "sq_llmint8_outliers", "sq_llmint8_combine",
 )
+LLMINT8_MAX_K = 1 << 20
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
@@ -116,6 +117,9 @@ def _declare(L):
                                               _P, _I32, _P]
     L.sq_quant_per_token_given_absmax.argtypes = [_P, _I32, _I64, _I64, _I64, _P, _P, _P, _P]
     L.sq_row_absmax.argtypes = [_P, _I32, _I64, _I64, _I64, _P, _P]
+    L.sq_llmint8_outliers.argtypes = [_P, _I64, _F32, _P, _P, _P, _P]
+    L.sq_llmint8_combine.argtypes = [_P, _I64, _I64, _I64, _P, _P, _P, _I32, _I64, _P, _I32,
+                                     _I64, _I64, _P, _P, _I32, _P, _I64, _P]
     L.sq_dequant_i32.argtypes = [_P, _I64, _I64, _I64, _P, _P, _I32, _P, _I64, _P]
     L.sq_silu_mul_quant_per_token.argtypes = [_P, _I32, _I64, _I64, _I64, _P, _P, _P, _I64, _P]
     L.sq_norm_smooth_quant_per_token_fp8.argtypes = [_P, _I32, _I64, _I64, _I64, _I32, _P, _P,
@@ -366,6 +370,48 @@ def dequant_i32(acc: torch.Tensor, x_scale: torch.Tensor, w_scale: torch.Tensor,
                                 _ptr(_vec(x_scale, M, "x_scale")), _ptr(_vec(w_scale, N, "w_scale")),
                                 EPI[epi], _ptr(out), max(out.stride(0), N), _stream(stream)),
            "sq_dequant_i32")
+    return out
+
+
+def llmint8_outliers(col_absmax: torch.Tensor, tau: float = 6.0, mask=None, idx=None, count=None,
+                     stream=None):
+    """(mask [K] fp32, idx [K] int32, count [1] int32) of the LLM.int8()
+    comparator: mask 0 on the channels with col_absmax >= tau, idx[:count] those
+    channels ascending (count stays on the device)."""
+    K = col_absmax.numel()
+    dev = col_absmax.device
+    if mask is None:
+        mask = torch.empty(K, dtype=torch.float32, device=dev)
+    if idx is None:
+        idx = torch.empty(K, dtype=torch.int32, device=dev)
+    if count is None:
+        count = torch.empty(1, dtype=torch.int32, device=dev)
+    if idx.dtype != torch.int32 or idx.numel() < K or count.dtype != torch.int32:
+        raise ValueError("idx [K] and count [1] must be int32")
+    _check(lib().sq_llmint8_outliers(_ptr(_vec(col_absmax, K, "col_absmax")), K, tau,
+                                     _ptr(_vec(mask, K, "mask")), _ptr(idx), _ptr(count),
+                                     _stream(stream)), "sq_llmint8_outliers")
+    return mask, idx, count
+
+
+def llmint8_combine(acc: torch.Tensor, x_scale, w_scale, x: torch.Tensor, W: torch.Tensor, idx,
+                    count, epi: str = "bf16", out=None, stream=None) -> torch.Tensor:
+    """The comparator's merge: the INT8 lane's epilogue plus the 16-bit lane
+    over the outlier channels, bf16 [M, N]."""
+    M, N = acc.shape
+    _, K, ldx = _rows(x, "x")
+    _, Kw, ldw = _rows(W, "W")
+    if Kw != K or W.shape[0] != N or acc.dtype != torch.int32 or \
+            (N > 1 and acc.stride(1) != 1):
+        raise ValueError("acc [M, N] int32, x [M, K], W [N, K]")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=acc.device)
+    _check(lib().sq_llmint8_combine(_ptr(acc), M, N, max(acc.stride(0), N),
+                                    _ptr(_vec(x_scale, M, "x_scale")),
+                                    _ptr(_vec(w_scale, N, "w_scale")), _ptr(x), _dtype_code(x),
+                                    ldx, _ptr(W), _dtype_code(W), ldw, K, _ptr(idx), _ptr(count),
+                                    EPI[epi], _ptr(out), max(out.stride(0), N), _stream(stream)),
+           "sq_llmint8_combine")
     return out
 
 
