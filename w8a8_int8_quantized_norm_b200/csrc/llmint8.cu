@@ -70,9 +70,22 @@ __global__ void __launch_bounds__(kOutThreads)
   }
 }
 
-constexpr int kCombRows = 32;   // output rows per CTA
-constexpr int kCombCols = 256;  // output columns per pass (one per thread)
-constexpr int kLaneCache = 32;  // outlier channels held in shared memory / registers
+constexpr int kCombRows = 16;   // rows per tile
+constexpr int kCombCols = 256;  // columns of a CTA's slab (one per thread)
+constexpr int kStages = 3;      // accumulator tiles in the shared-memory ring
+constexpr int kRegLane = 8;     // outlier channels whose weights sit in registers
+constexpr int kLaneCache = 16;  // outlier channels staged on chip (registers + shared)
+constexpr int kGather = (kCombRows * kLaneCache + kCombCols - 1) / kCombCols;  // per thread
+static_assert(kRegLane % 2 == 0 && kLaneCache % 2 == 0, "xo rows are read as pairs");
+// dynamic shared memory: the accumulator ring [kStages][kCombRows][kCombCols]
+// (int32), xo [2][kCombRows][kLaneCache] and wo [kLaneCache - kRegLane]
+// [kCombCols] (fp64), the tiles' token scales [2][kCombRows] (fp32)
+constexpr size_t kCombSmem =
+    static_cast<size_t>(kStages) * kCombRows * kCombCols * sizeof(int32_t) +
+    (2 * static_cast<size_t>(kCombRows) * kLaneCache +
+     static_cast<size_t>(kLaneCache - kRegLane) * kCombCols) *
+        sizeof(double) +
+    2 * kCombRows * sizeof(float);
 
 // Element i of a bf16 or fp32 array, widened (exactly) to fp64.
 __device__ __forceinline__ double elem(const void* p, int64_t i, bool bf) {
@@ -83,60 +96,189 @@ __device__ __forceinline__ double elem(const void* p, int64_t i, bool bf) {
   return static_cast<double>(static_cast<const float*>(p)[i]);
 }
 
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst),
+               "l"(reinterpret_cast<uint64_t>(src))
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int kPending>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(kPending) : "memory");
+}
+
+// Starts the copies of a tile's accumulators (column n of its rows) into
+// ring slot `slot`, as one commit group (empty past the last tile).
+__device__ __forceinline__ void issue_tile(uint32_t ring, int slot, const int32_t* acc,
+                                           int64_t lda, int64_t tile, int64_t tiles, int64_t M,
+                                           int64_t n, bool col, int t) {
+  if (col && tile < tiles) {
+    const int64_t m0 = tile * kCombRows;
+    const int rows = M - m0 < kCombRows ? static_cast<int>(M - m0) : kCombRows;
+    const uint32_t dst = ring + static_cast<uint32_t>((slot * kCombRows * kCombCols + t) * 4);
+    for (int g = 0; g < rows; ++g)
+      cp_async4(dst + static_cast<uint32_t>(g * kCombCols * 4), acc + (m0 + g) * lda + n);
+  }
+  cp_async_commit();
+}
+
+// This thread's share of a tile's outlier inputs (entry i = r * kLaneCache + c
+// of xo, zero past the rows or the count) and token scales.
+struct TileInputs {
+  double xg[kGather];
+  float xs;
+};
+
+template <bool kXBF16>
+__device__ __forceinline__ void load_inputs(TileInputs& L, int64_t m0, int rows,
+                                            const float* __restrict__ x_scale, const void* x,
+                                            int64_t ldx, const int32_t* __restrict__ idx,
+                                            int ncache, int t) {
+#pragma unroll
+  for (int k = 0; k < kGather; ++k) {
+    const int i = t + k * kCombCols;
+    const int r = i / kLaneCache, c = i - r * kLaneCache;
+    L.xg[k] = i < kCombRows * kLaneCache && r < rows && c < ncache
+                  ? elem(x, (m0 + r) * ldx + idx[c], kXBF16)
+                  : 0.0;
+  }
+  L.xs = t < rows ? x_scale[m0 + t] : 0.0f;
+}
+
+__device__ __forceinline__ void stage_inputs(const TileInputs& L, double* xo, float* xsr, int t) {
+#pragma unroll
+  for (int k = 0; k < kGather; ++k) {
+    const int i = t + k * kCombCols;
+    if (i < kCombRows * kLaneCache) xo[i] = L.xg[k];
+  }
+  if (t < kCombRows) xsr[t] = L.xs;
+}
+
 // out[m, n] = bf16(y), y = fl32(fl32(fl32(fl32(acc) xs[m]) ws[n]) + fl32(s)),
 // ReLU on y when asked, where s = sum over the outlier channels j (ascending)
 // of x[m, j] w[n, j] in fp64 (each product is exact in fp64, and fma rounds
-// s + x w once, as the oracle's s = s + x * w does).  A CTA owns kCombRows
-// rows, whose outlier inputs it gathers once into shared memory, and walks
-// the column passes blockIdx.y, blockIdx.y + gridDim.y, ...; thread = column
-// of a pass, its outlier weights in registers (the first kLaneCache
-// channels; the rest are read as they come).
+// s + x w once, as the oracle's s = s + x * w does).
+//
+// A CTA owns the column slab blockIdx.x (thread = column) and walks the row
+// tiles blockIdx.y, blockIdx.y + gridDim.y, ...  Its columns' outlier weights
+// are read once (one scattered load per channel): the first kRegLane into
+// registers (zero past the count), the next ones into the thread's own column
+// of wo; channels past kLaneCache are read per row from global memory.  Each
+// thread copies its own column of the accumulator tiles into a ring of
+// kStages slots with cp.async, kStages - 1 tiles ahead (it reads back only
+// what it copied, so the ring needs no barrier); the next tile's outlier
+// inputs are loaded into registers before the current tile is computed and
+// stored to the other xo buffer after it.  The register lane runs all
+// kRegLane fused multiply-adds: a padded term adds 0 * 0 to s, which leaves s
+// unchanged (s starts at +0 and a rounded sum is never -0).
 template <bool kXBF16, bool kWBF16>
-__global__ void __launch_bounds__(kCombCols)
+__global__ void __launch_bounds__(kCombCols, 3)
     llmint8_combine_kernel(const int32_t* __restrict__ acc, int64_t M, int64_t N, int64_t lda,
                            const float* __restrict__ x_scale, const float* __restrict__ w_scale,
                            const void* __restrict__ x, int64_t ldx, const void* __restrict__ W,
                            int64_t ldw, const int32_t* __restrict__ idx,
                            const int32_t* __restrict__ count, int relu,
                            __nv_bfloat16* __restrict__ out, int64_t ldo) {
-  __shared__ double xo[kCombRows][kLaneCache];
-  __shared__ float xsr[kCombRows];
+  extern __shared__ __align__(16) unsigned char comb_smem[];
+  const int32_t* accs = reinterpret_cast<const int32_t*>(comb_smem);  // [slot][r][t]
+  double* xo = reinterpret_cast<double*>(comb_smem + static_cast<size_t>(kStages) * kCombRows *
+                                                         kCombCols * 4);  // [2][r][c]
+  double* wo = xo + 2 * kCombRows * kLaneCache;  // [c - kRegLane][t]: thread t's own
+  float* xsr = reinterpret_cast<float*>(wo + (kLaneCache - kRegLane) * kCombCols);  // [2][r]
+  const uint32_t ring = smem_u32(comb_smem);
   const int t = threadIdx.x;
-  const int64_t m0 = static_cast<int64_t>(blockIdx.x) * kCombRows;
-  const int rows = M - m0 < kCombRows ? static_cast<int>(M - m0) : kCombRows;
+  const int64_t n = static_cast<int64_t>(blockIdx.x) * kCombCols + t;
+  const bool col = n < N;
   const int nout = *count;
   const int ncache = min(nout, kLaneCache);
-  for (int i = t; i < kCombRows * ncache; i += kCombCols) {
-    const int r = i / ncache, c = i - r * ncache;
-    xo[r][c] = r < rows ? elem(x, (m0 + r) * ldx + idx[c], kXBF16) : 0.0;
-  }
-  if (t < kCombRows) xsr[t] = t < rows ? x_scale[m0 + t] : 0.0f;
+  const int64_t tiles = (M + kCombRows - 1) / kCombRows;
+  const int64_t G = gridDim.y;
+  int64_t tile = blockIdx.y;
+  if (tile >= tiles) return;
+
+#pragma unroll
+  for (int k = 0; k < kStages - 1; ++k)
+    issue_tile(ring, k, acc, lda, tile + k * G, tiles, M, n, col, t);
+  double wr[kRegLane];
+#pragma unroll
+  for (int c = 0; c < kRegLane; ++c)
+    wr[c] = col && c < ncache ? elem(W, n * ldw + idx[c], kWBF16) : 0.0;
+  if (col)
+    for (int c = kRegLane; c < ncache; ++c)
+      wo[(c - kRegLane) * kCombCols + t] = elem(W, n * ldw + idx[c], kWBF16);
+  const float ws = col ? w_scale[n] : 0.0f;
+
+  auto rows_of = [&](int64_t tl) {
+    const int64_t left = M - tl * kCombRows;
+    return left < kCombRows ? static_cast<int>(left) : kCombRows;
+  };
+  TileInputs in;
+  load_inputs<kXBF16>(in, tile * kCombRows, rows_of(tile), x_scale, x, ldx, idx, ncache, t);
+  stage_inputs(in, xo, xsr, t);
   __syncthreads();
-  for (int64_t n0 = static_cast<int64_t>(blockIdx.y) * kCombCols; n0 < N;
-       n0 += static_cast<int64_t>(gridDim.y) * kCombCols) {
-    const int64_t n = n0 + t;
-    if (n >= N) continue;
-    double wv[kLaneCache];
+  int buf = 0, slot = 0;
+  for (;;) {
+    const int64_t next = tile + G;
+    const bool has_next = next < tiles;
+    // the slot read in the previous iteration takes the tile kStages - 1 ahead
+    issue_tile(ring, slot == 0 ? kStages - 1 : slot - 1, acc, lda, tile + (kStages - 1) * G,
+               tiles, M, n, col, t);
+    if (has_next)
+      load_inputs<kXBF16>(in, next * kCombRows, rows_of(next), x_scale, x, ldx, idx, ncache, t);
+    cp_async_wait<kStages - 1>();  // this thread's copies of the current tile have landed
+    const int64_t m0 = tile * kCombRows;
+    const int rows = rows_of(tile);
+    const double* xb = xo + buf * kCombRows * kLaneCache;
+    const float* sb = xsr + buf * kCombRows;
+    const int32_t* ab = accs + slot * kCombRows * kCombCols + t;
+    if (col) {
+      __nv_bfloat16* op = out + m0 * ldo + n;
+      for (int g = 0; g < rows; ++g, op += ldo) {
+        const double2* xr = reinterpret_cast<const double2*>(xb + g * kLaneCache);
+        double s = 0.0;
 #pragma unroll
-    for (int c = 0; c < kLaneCache; ++c)
-      wv[c] = c < ncache ? elem(W, n * ldw + idx[c], kWBF16) : 0.0;
-    const float ws = w_scale[n];
-    for (int r = 0; r < rows; ++r) {
-      const int64_t m = m0 + r;
-      double s = 0.0;
-#pragma unroll
-      for (int c = 0; c < kLaneCache; ++c)
-        if (c < ncache) s = __fma_rn(xo[r][c], wv[c], s);
-      for (int c = kLaneCache; c < nout; ++c) {
-        const int j = idx[c];
-        s = __fma_rn(elem(x, m * ldx + j, kXBF16), elem(W, n * ldw + j, kWBF16), s);
+        for (int c = 0; c < kRegLane; c += 2) {
+          const double2 v = xr[c / 2];
+          s = __fma_rn(v.x, wr[c], s);
+          s = __fma_rn(v.y, wr[c + 1], s);
+        }
+        for (int c = kRegLane; c < ncache; ++c)
+          s = __fma_rn(xb[g * kLaneCache + c], wo[(c - kRegLane) * kCombCols + t], s);
+        for (int c = kLaneCache; c < nout; ++c) {
+          const int j = idx[c];
+          s = __fma_rn(elem(x, (m0 + g) * ldx + j, kXBF16), elem(W, n * ldw + j, kWBF16), s);
+        }
+        const float y8 = __fmul_rn(__fmul_rn(__int2float_rn(ab[g * kCombCols]), sb[g]), ws);
+        float y = __fadd_rn(y8, __double2float_rn(s));
+        if (relu) y = y > 0.0f ? y : 0.0f;  // -0 becomes +0
+        *op = __float2bfloat16_rn(y);
       }
-      const float y8 = __fmul_rn(__fmul_rn(__int2float_rn(acc[m * lda + n]), xsr[r]), ws);
-      float y = __fadd_rn(y8, __double2float_rn(s));
-      if (relu) y = y > 0.0f ? y : 0.0f;  // -0 becomes +0
-      out[m * ldo + n] = __float2bfloat16_rn(y);
     }
+    if (!has_next) break;
+    // the other buffer was last read before the previous iteration's barrier
+    stage_inputs(in, xo + (buf ^ 1) * kCombRows * kLaneCache, xsr + (buf ^ 1) * kCombRows, t);
+    __syncthreads();
+    buf ^= 1;
+    slot = slot == kStages - 1 ? 0 : slot + 1;
+    tile = next;
   }
+  cp_async_wait<0>();  // no copy outlives the CTA
+}
+
+template <bool kXBF16, bool kWBF16>
+cudaError_t launch_combine(dim3 grid, cudaStream_t st, const int32_t* acc, int64_t M, int64_t N,
+                           int64_t lda, const float* x_scale, const float* w_scale, const void* x,
+                           int64_t ldx, const void* W, int64_t ldw, const int32_t* idx,
+                           const int32_t* count, int relu, __nv_bfloat16* out, int64_t ldo) {
+  cudaError_t e = cudaFuncSetAttribute(llmint8_combine_kernel<kXBF16, kWBF16>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kCombSmem));
+  if (e != cudaSuccess) return e;
+  llmint8_combine_kernel<kXBF16, kWBF16><<<grid, kCombCols, kCombSmem, st>>>(
+      acc, M, N, lda, x_scale, w_scale, x, ldx, W, ldw, idx, count, relu, out, ldo);
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -154,30 +296,28 @@ cudaError_t launch_llmint8_combine(const int32_t* acc, int64_t M, int64_t N, int
                                    int64_t ldw, const int32_t* idx, const int32_t* count, int relu,
                                    void* out, int64_t ldo, cudaStream_t st) {
   if (M == 0 || N == 0) return cudaSuccess;
-  // row blocks, and column passes split over gridDim.y only as far as needed
-  // to give every SM a few CTAs (few row blocks: small M)
-  const int64_t row_blocks = (M + kCombRows - 1) / kCombRows;
-  const int64_t passes = (N + kCombCols - 1) / kCombCols;
-  int64_t col_split = (4 * static_cast<int64_t>(num_sms_current_device()) + row_blocks - 1) /
-                      row_blocks;
-  if (col_split > passes) col_split = passes;
-  if (col_split < 1) col_split = 1;
-  if (col_split > 65535) col_split = 65535;
-  const dim3 grid(static_cast<unsigned>(row_blocks), static_cast<unsigned>(col_split));
+  // one CTA per column slab and row-tile stream; the streams per slab fill
+  // three CTAs per SM (one wave) when the slabs alone do not
+  const int64_t slabs = (N + kCombCols - 1) / kCombCols;
+  const int64_t tiles = (M + kCombRows - 1) / kCombRows;
+  int64_t streams = 3 * static_cast<int64_t>(num_sms_current_device()) / slabs;
+  if (streams > tiles) streams = tiles;
+  if (streams < 1) streams = 1;
+  if (streams > 65535) streams = 65535;
+  if (slabs > 0x7fffffff) return cudaErrorInvalidValue;
+  const dim3 grid(static_cast<unsigned>(slabs), static_cast<unsigned>(streams));
   auto* o = static_cast<__nv_bfloat16*>(out);
   if (x_bf16 && w_bf16)
-    llmint8_combine_kernel<true, true><<<grid, kCombCols, 0, st>>>(
-        acc, M, N, lda, x_scale, w_scale, x, ldx, W, ldw, idx, count, relu, o, ldo);
-  else if (x_bf16)
-    llmint8_combine_kernel<true, false><<<grid, kCombCols, 0, st>>>(
-        acc, M, N, lda, x_scale, w_scale, x, ldx, W, ldw, idx, count, relu, o, ldo);
-  else if (w_bf16)
-    llmint8_combine_kernel<false, true><<<grid, kCombCols, 0, st>>>(
-        acc, M, N, lda, x_scale, w_scale, x, ldx, W, ldw, idx, count, relu, o, ldo);
-  else
-    llmint8_combine_kernel<false, false><<<grid, kCombCols, 0, st>>>(
-        acc, M, N, lda, x_scale, w_scale, x, ldx, W, ldw, idx, count, relu, o, ldo);
-  return cudaGetLastError();
+    return launch_combine<true, true>(grid, st, acc, M, N, lda, x_scale, w_scale, x, ldx, W, ldw,
+                                      idx, count, relu, o, ldo);
+  if (x_bf16)
+    return launch_combine<true, false>(grid, st, acc, M, N, lda, x_scale, w_scale, x, ldx, W, ldw,
+                                       idx, count, relu, o, ldo);
+  if (w_bf16)
+    return launch_combine<false, true>(grid, st, acc, M, N, lda, x_scale, w_scale, x, ldx, W, ldw,
+                                       idx, count, relu, o, ldo);
+  return launch_combine<false, false>(grid, st, acc, M, N, lda, x_scale, w_scale, x, ldx, W, ldw,
+                                      idx, count, relu, o, ldo);
 }
 
 }  // namespace sq
