@@ -774,3 +774,34 @@ def test_llmint8_is_finer_than_plain_int8_on_outlier_channels():
     e_plain = np.linalg.norm(o32 - ref) / np.linalg.norm(ref)
     e_int8 = np.linalg.norm(r["y"] - ref) / np.linalg.norm(ref)
     assert e_int8 * 5 < e_plain
+
+
+def test_llmint8_layer_is_the_exact_product_on_integer_data():
+    """A closed form of the whole decomposition: integer inputs whose ordinary
+    channels lie in [-127, 127] with a +-127 in every token row and every
+    weight row (token and weight steps fl32(127 / 127) = 1, so codes equal the
+    values), outlier channels at 200 or more (tau = 200 sends exactly them to
+    the 16-bit lane).  Both lanes are then exact integer sums below 2^24 and
+    the bf16 output is the rounding of the exact product x W^T.  A lane
+    counted twice, an outlier left in the INT8 lane (its step would no longer
+    be 1) or a dropped lane fails."""
+    import torch
+    rng = np.random.default_rng(15)
+    M, N, K = 6, 10, 40
+    out_ch = [4, 21, 33]
+    x = rng.integers(-127, 128, (M, K)).astype(np.float32)
+    x[:, [0, 1]] = 0.0
+    x[:, 0] = np.where(np.arange(M) % 2 == 0, 127.0, -127.0)
+    x[:, out_ch] = rng.integers(200, 400, (M, len(out_ch))) * rng.choice([-1, 1], (M, len(out_ch)))
+    W = rng.integers(-127, 128, (N, K)).astype(np.float32)
+    W[:, 1] = 127.0
+    Wq, ws = oracle.quantize_weights(W, None)
+    assert (ws == 1.0).all() and np.array_equal(Wq.astype(np.float32), W)
+    r = oracle.llmint8_linear(x, Wq, ws, W, tau=200.0)
+    assert r["idx"].tolist() == out_ch
+    assert (r["x_scale"] == 1.0).all()
+    exact = x.astype(np.int64) @ W.astype(np.int64).T
+    assert np.abs(exact).max() < 2 ** 24
+    assert np.array_equal(r["y"], exact.astype(np.float32))
+    want = torch.from_numpy(exact.astype(np.float32)).to(torch.bfloat16)
+    assert np.array_equal(r["out"], want.view(torch.int16).numpy().view(np.uint16))
