@@ -527,7 +527,7 @@ sq_status sq_w8a8_gemm_plan(int64_t M, int64_t N, int64_t K, int path_hint, int 
  *            nothing in it has to start at any value; two calls that overlap
  *            on the GPU need two workspaces.
  *   path_hint 0 = automatic, 1 = prefill tiles (tokens on the MMA M side;
- *            CTA pairs, 256-row tiles 256 or 192 wide on two SMs, the width
+ *            CTA pairs, 256-row tiles 256, 224 or 192 wide on two SMs, the width
  *            chosen to fill the SMs evenly), 2 = decode tiles (weight
  *            rows on the MMA M side, M <= 256), 3 = prefill tiles on single
  *            SMs (128 x 256)

@@ -31,12 +31,17 @@ def test_plan_kinds_and_workspace_agree_with_the_size_query(L):
     assert (p.kernel, p.stream_k, p.split_k, p.tile_m, p.tile_n) == (2, 1, 1, 128, 16)
     assert p.ctas == SMS and p.launches == 2
     assert p.workspace_bytes == 2 * SMS * 128 * 1 * 4
-    # 8 x 48 tiles of 256 x 256 fill 74 SM pairs in 6 rounds; 8 x 64 of 256 x 192
-    # need 7 rounds of a step that is not proportionally shorter: 256 wins
+    # 8 x 48 tiles of 256 x 256 and 8 x 55 of 256 x 224 fill 74 SM pairs in 6
+    # rounds, 8 x 64 of 256 x 192 in 7; a K step costs about 480 + 0.625 TN
+    # cycles, so 224 wins
     p = _plan(2048, 12288, 4096)
-    assert (p.kernel, p.tile_m, p.tile_n, p.launches, p.workspace_bytes) == (1, 256, 256, 1, 0)
-    # 4 x 12 tiles of 256 x 256 or 4 x 16 of 256 x 192 are one round either way
+    assert (p.kernel, p.tile_m, p.tile_n, p.launches, p.workspace_bytes) == (1, 256, 224, 1, 0)
+    # one round at every width: the narrowest step wins
     assert _plan(1024, 3000, 272).tile_n == 192
+    # 59 / 67 / 79 tiles: one round at 256 and 224, two at 192
+    assert _plan(200, 15000, 64).tile_n == 224
+    # 296 tiles of 256 are 4 full rounds, 344 of 224 take 5: 256 wins
+    assert _plan(2048, 9472, 128).tile_n == 256
     p = _plan(16384, 57344, 8192)
     assert (p.kernel, p.tile_m, p.tile_n) == (1, 256, 256)
     p = _plan(2048, 12288, 4096, path=3)

@@ -619,7 +619,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // stage-free and accumulator-ready barriers with one commit each; both CTAs'
 // epilogue warps drain their own 128 accumulator rows and tell the leader.
 // ---------------------------------------------------------------------------
-// TN: the pair tile's N (Q-side) width, 256 or 192; each CTA loads
+// TN: the pair tile's N (Q-side) width, 256, 224 or 192; each CTA loads
 // TN / 2 rows of B.  As many stages as fit 227 KB of shared memory (at most 8).
 template <int TN>
 struct PairCfg {
@@ -904,21 +904,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_32x32b_x32(trow, ra);
         load_col_scales<32>(prm, qb * TN, wa);
         tmem_wait_ld();
+        constexpr int kChunks = TN / 32;  // odd for TN = 224: the last pair is one chunk
 #pragma unroll 1
-        for (int c = 0; c < TN / 32; c += 2) {
-          __syncwarp();
-          tmem_ld_32x32b_x32(trow + static_cast<uint32_t>((c + 1) * 32), rb);
-          load_col_scales<32>(prm, qb * TN + (c + 1) * 32, wb);
+        for (int c = 0; c < kChunks; c += 2) {
+          const bool two = c + 1 < kChunks;
+          if (two) {
+            __syncwarp();
+            tmem_ld_32x32b_x32(trow + static_cast<uint32_t>((c + 1) * 32), rb);
+            load_col_scales<32>(prm, qb * TN + (c + 1) * 32, wb);
+          }
           if (row_in) rmax = fmaxf(rmax, epi_row_bf16<32, kF8>(prm, ra, p, qb * TN + c * 32, xs, wa));
-          tmem_wait_ld();
-          if (c + 2 < TN / 32) {
+          if (two) tmem_wait_ld();
+          if (c + 2 < kChunks) {
             __syncwarp();
             tmem_ld_32x32b_x32(trow + static_cast<uint32_t>((c + 2) * 32), ra);
             load_col_scales<32>(prm, qb * TN + (c + 2) * 32, wa);
           }
-          if (row_in)
+          if (two && row_in)
             rmax = fmaxf(rmax, epi_row_bf16<32, kF8>(prm, rb, p, qb * TN + (c + 1) * 32, xs, wb));
-          if (c + 2 < TN / 32) tmem_wait_ld();
+          if (c + 2 < kChunks) tmem_wait_ld();
         }
       }
       if (prm.row_absmax && rmax > 0.0f && p < prm.P)
@@ -1161,16 +1165,16 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int path_hint, int split_k, 
     p.pair = path_hint == 3 ? 0 : 1;
     if (p.pair) {
       // pair tile width: rounds of tiles over the SM pairs times the time of
-      // a tile's 128-deep K step, which is the MMA's (proportional to the
-      // width) for 256 but does not drop below about 240/256 of it for
-      // narrower tiles (operand delivery and per-step overhead; measured
-      // 600 vs 640 cycles per step at widths 192 and 256)
+      // a tile's 128-deep K step, which operand delivery sets rather than the
+      // MMA (measured 600 and 640 cycles per step at widths 192 and 256, the
+      // MMA alone taking 384 and 512): step ~ 480 + 0.625 TN cycles, in
+      // units of 1/1.6 cycle 768 + TN
       const int64_t pairs = (num_sms > 0 ? num_sms : 148) / 2;
       const int64_t p_blocks = (M + 255) / 256;
       int64_t best = -1;
-      for (int tn : {256, 192}) {
+      for (int tn : {256, 224, 192}) {
         const int64_t tiles = p_blocks * ((N + tn - 1) / tn);
-        const int64_t cost = ((tiles + pairs - 1) / pairs) * (tn > 240 ? tn : 240);
+        const int64_t cost = ((tiles + pairs - 1) / pairs) * (768 + tn);
         if (best < 0 || cost < best) {
           best = cost;
           p.bn = tn;
@@ -1278,8 +1282,10 @@ cudaError_t launch_gemm(const GemmPlan& plan, const int8_t* Xq, const int8_t* Wq
       return cudaErrorInvalidValue;
     switch (plan.bn * 2 + (fp8 ? 1 : 0)) {
       case 512: return launch_pair<256, false>(prm, mp, mq, sms / 2, st);
+      case 448: return launch_pair<224, false>(prm, mp, mq, sms / 2, st);
       case 384: return launch_pair<192, false>(prm, mp, mq, sms / 2, st);
       case 513: return launch_pair<256, true>(prm, mp, mq, sms / 2, st);
+      case 449: return launch_pair<224, true>(prm, mp, mq, sms / 2, st);
       case 385: return launch_pair<192, true>(prm, mp, mq, sms / 2, st);
       default: return cudaErrorInvalidValue;
     }
