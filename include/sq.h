@@ -414,17 +414,26 @@ sq_status sq_smooth_quantize_weights_fp8(const void* W, sq_dtype dtype, int64_t 
  *   Xq8 device [M, K] e4m3 (stride K); Wq8 device [N, K] e4m3 (stride K)
  *   epi      SQ_EPI_BF16, SQ_EPI_BF16_RELU (out bf16 [M, N], stride ldo) or
  *            SQ_EPI_F32_RAW (out fp32 [M, N] = the accumulator)
- *   path_hint as for sq_w8a8_gemm_dequant; every tile runs its whole K (no
- *            split-K or stream-K partial sums), so no workspace is needed.
+ *   workspace device, caller-owned, 16-byte aligned, ws_bytes long, or NULL.
+ *            With a workspace of at least
+ *            sq_w8a8_gemm_workspace_size(M, N, K, 0) bytes the decode tiles
+ *            (path 2, or automatic with M <= 128) run stream-K: a tile split
+ *            between CTAs leaves fp32 partial sums there, which a fix-up
+ *            kernel adds in ascending CTA order (the same order on every run
+ *            on the same GPU model) before the epilogue.  With NULL every
+ *            tile runs its whole K.  Nothing in it outlives the call.
+ *   path_hint as for sq_w8a8_gemm_dequant (no explicit split-K).
  * The tensor cores' fp32 accumulation order is theirs: the accumulator
  * equals the exact sum of the decoded products to within the rounding of
- * the accumulation (not bit-exact with a sequential sum).
- * Errors: those of sq_w8a8_gemm_dequant (K <= SQ_MAX_K as there).
+ * the accumulation (not bit-exact with a sequential sum); a stream-K tile
+ * adds one fp32 rounding per contributing CTA after the first.
+ * Errors: those of sq_w8a8_gemm_dequant (K <= SQ_MAX_K as there);
+ * SQ_ERR_WORKSPACE for a non-NULL workspace shorter than the plan needs.
  */
 sq_status sq_fp8_gemm_dequant(const uint8_t* Xq8, const uint8_t* Wq8, const float* x_scale,
                               const float* w_scale, int64_t M, int64_t N, int64_t K,
-                              sq_epilogue epi, void* out, int64_t ldo, int path_hint,
-                              void* stream);
+                              sq_epilogue epi, void* out, int64_t ldo, void* workspace,
+                              size_t ws_bytes, int path_hint, void* stream);
 
 /*
  * sq_silu_mul_quant_per_token -- the down projection's input, SiLU(gate) * up,

@@ -986,8 +986,11 @@ def fp8_acc_bound(K):
     each rounding by at most 2^-23 of a partial sum bounded by the step's
     sum |a b| -- and adds the result into the fp32 accumulator with one more
     rounding of at most 2^-23 of sum |a b|.  (The hardware exceeds a model
-    with exact step sums, ceil(K/32) 2^-23, by up to 1.4x at K = 64.)"""
-    return (31 + max(1, (K + 31) // 32)) * 2.0 ** -23
+    with exact step sums, ceil(K/32) 2^-23, by up to 1.4x at K = 64.)  A
+    stream-K decode tile adds its contributors' fp32 partial sums with one
+    more rounding each; they are at most ceil(K/128), one per 128-deep
+    block."""
+    return (31 + max(1, (K + 31) // 32) + max(1, (K + 127) // 128)) * 2.0 ** -23
 
 
 F8_GEMM_SHAPES = [(16, 64, 64), (3, 5, 16), (129, 257, 4112), (256, 512, 1024), (300, 777, 160),
@@ -1009,16 +1012,21 @@ def test_fp8_gemm_accumulator_and_epilogue(shape, path):
     da = oracle.e4m3_decode(A).astype(np.float64)
     db = oracle.e4m3_decode(B).astype(np.float64)
     absum = np.abs(da) @ np.abs(db).T
-    acc = sq.fp8_gemm_dequant(to_gpu(A), to_gpu(B), None, None, "f32", path_hint=path)
-    acc_g = acc.cpu().numpy()
-    assert np.all(np.abs(acc_g.astype(np.float64) - exact) <= fp8_acc_bound(K) * absum)
     xs = (RNG.random(M) * 0.05 + 1e-3).astype(np.float32)
     ws = (RNG.random(N) * 0.002 + 1e-5).astype(np.float32)
-    for relu in (False, True):
-        out = sq.fp8_gemm_dequant(to_gpu(A), to_gpu(B), to_gpu(xs), to_gpu(ws),
-                                  "bf16_relu" if relu else "bf16", path_hint=path)
-        _, out_o = oracle.epilogue_f32(acc_g, xs, ws, relu)
-        assert np.array_equal(bf16_bits(out), out_o)
+    # decode tiles: stream-K (the default, fp32 partials added in CTA order)
+    # and whole-K tiles; the prefill paths have whole-K tiles only
+    for whole_k in ((False, True) if path == 2 else (False,)):
+        acc = sq.fp8_gemm_dequant(to_gpu(A), to_gpu(B), None, None, "f32", path_hint=path,
+                                  whole_k=whole_k)
+        acc_g = acc.cpu().numpy()
+        assert np.all(np.abs(acc_g.astype(np.float64) - exact) <= fp8_acc_bound(K) * absum)
+        for relu in (False, True):
+            out = sq.fp8_gemm_dequant(to_gpu(A), to_gpu(B), to_gpu(xs), to_gpu(ws),
+                                      "bf16_relu" if relu else "bf16", path_hint=path,
+                                      whole_k=whole_k)
+            _, out_o = oracle.epilogue_f32(acc_g, xs, ws, relu)
+            assert np.array_equal(bf16_bits(out), out_o)
 
 
 def test_fp8_gemm_rejects_int8_only_epilogues():
@@ -1032,6 +1040,23 @@ def test_fp8_gemm_rejects_int8_only_epilogues():
         sq.w8a8_gemm_dequant(A.view(torch.int8), B.view(torch.int8), None, None, "f32",
                              out=torch.empty((8, 32), dtype=torch.float32, device="cuda"))
     assert e.value.status == 1
+
+
+def test_fp8_decode_workspace_too_small_is_refused():
+    A = torch.zeros((1, 4096), dtype=torch.uint8, device="cuda")
+    B = torch.zeros((4096, 4096), dtype=torch.uint8, device="cuda")
+    need = sq.gemm_workspace_size(1, 4096, 4096, 0)
+    assert need > 16
+    small = torch.empty(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(sq.SQError) as e:
+        sq.fp8_gemm_dequant(A, B, None, None, "f32", path_hint=2, workspace=small)
+    assert e.value.status == 7
+    # a workspace of the planned size, and none at all (whole-K tiles), both run
+    full = torch.empty(need, dtype=torch.uint8, device="cuda")
+    for ws, whole in ((full, False), (None, True)):
+        out = sq.fp8_gemm_dequant(A, B, None, None, "f32", path_hint=2, workspace=ws,
+                                  whole_k=whole)
+        assert torch.count_nonzero(out).item() == 0
 
 
 def _check_workload_fp8(w, rows=None, seed=0):

@@ -267,7 +267,7 @@ def test_fp8_calls_reject_bad_arguments(L):
     g = L.sq_fp8_gemm_dequant
 
     def gemm(Xq=A16, Wq=A16, xs=A16, ws=A16, M=16, N=64, K=64, epi=0, out=A16, ldo=64, path=0):
-        return g(Xq, Wq, xs, ws, M, N, K, epi, out, ldo, path, None)
+        return g(Xq, Wq, xs, ws, M, N, K, epi, out, ldo, None, 0, path, None)
 
     assert gemm(epi=2) == 1             # INT32 output: INT8 GEMMs only
     assert gemm(epi=7) == 1

@@ -400,8 +400,8 @@ sq_status sq_smooth_quantize_weights_fp8(const void* W, sq_dtype dtype, int64_t 
 
 sq_status sq_fp8_gemm_dequant(const uint8_t* Xq8, const uint8_t* Wq8, const float* x_scale,
                               const float* w_scale, int64_t M, int64_t N, int64_t K,
-                              sq_epilogue epi, void* out, int64_t ldo, int path_hint,
-                              void* stream) {
+                              sq_epilogue epi, void* out, int64_t ldo, void* workspace,
+                              size_t ws_bytes, int path_hint, void* stream) {
   if (epi != SQ_EPI_BF16 && epi != SQ_EPI_BF16_RELU && epi != SQ_EPI_F32_RAW)
     return SQ_ERR_INVALID_ARG;
   // the shape, alignment and scale checks of the INT8 call (a raw fp32
@@ -409,17 +409,22 @@ sq_status sq_fp8_gemm_dequant(const uint8_t* Xq8, const uint8_t* Wq8, const floa
   const sq_epilogue e = epi == SQ_EPI_F32_RAW ? SQ_EPI_I32_RAW : epi;
   sq_status st = check_gemm(reinterpret_cast<const int8_t*>(Xq8),
                             reinterpret_cast<const int8_t*>(Wq8), x_scale, w_scale, M, N, K, e,
-                            out, ldo, path_hint, 1);
+                            out, ldo, path_hint, 0);
   if (st != SQ_OK) return st;
   if (M == 0 || N == 0) return SQ_OK;
   const int sms = sms_cached();
-  // whole-K tiles only: the fp32 accumulator has no exact split-K sum
-  const GemmPlan plan = plan_gemm(M, N, K, path_hint, 1, sms);
+  // decode tiles run stream-K (fp32 partial sums added in a fixed order) when
+  // a workspace is given; without one every tile runs its whole K
+  GemmPlan plan = plan_gemm(M, N, K, path_hint, workspace ? 0 : 1, sms);
+  if (plan.workspace_bytes > 0) {
+    if (ws_bytes < plan.workspace_bytes) return SQ_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return SQ_ERR_ALIGNMENT;
+  }
   int* err = device_error_word();
   if (!err) return SQ_ERR_CUDA;
   return from_cuda(launch_gemm(plan, reinterpret_cast<const int8_t*>(Xq8),
                                reinterpret_cast<const int8_t*>(Wq8), x_scale, w_scale, M, N, K,
-                               epi, out, ldo, nullptr, sms, g_wait_polls.load(), err,
+                               epi, out, ldo, workspace, sms, g_wait_polls.load(), err,
                                as_stream(stream), nullptr, true));
 }
 

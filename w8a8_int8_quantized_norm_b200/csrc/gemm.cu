@@ -974,9 +974,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 // starting before the tile ends) for tokens q = y * kFixQ ... and applies the
 // epilogue; thread = row of the tile's 128 P rows, so every load and store is
 // 128 consecutive words.  INT32 addition is exact, so the result equals the
-// unsplit accumulation.
+// unsplit accumulation.  FP8 partials are fp32: they are added in ascending
+// CTA order, one rounding per contributor after the first, the same order on
+// every run.
 constexpr int kFixQ = 8;  // tokens per fix-up block
 
+template <bool kF8>
 __global__ void __launch_bounds__(BM) streamk_fixup_kernel(const Params prm, int G) {
   // launched as a programmatic dependent of the main kernel: everything that
   // grid wrote is visible once this returns
@@ -995,7 +998,7 @@ __global__ void __launch_bounds__(BM) streamk_fixup_kernel(const Params prm, int
   if (p >= prm.P) return;
   const int q0 = static_cast<int>(blockIdx.y) * kFixQ;
   const int nq = min(kFixQ, prm.Q - q0);
-  int32_t acc[kFixQ];
+  int32_t acc[kFixQ];  // INT32 sums, or the fp32 sums' bits
 #pragma unroll
   for (int j = 0; j < kFixQ; ++j) acc[j] = 0;
   for (int cc = c - 1; cc < G; ++cc) {
@@ -1004,18 +1007,27 @@ __global__ void __launch_bounds__(BM) streamk_fixup_kernel(const Params prm, int
     const int64_t slot = (sc / kbt == tile) ? 2 * cc : 2 * cc + 1;
     const int32_t* src = prm.sk_partial + (slot * prm.Q + q0) * BM + pl;
 #pragma unroll
-    for (int j = 0; j < kFixQ; ++j)
-      if (j < nq) acc[j] += __ldcg(src + j * BM);
+    for (int j = 0; j < kFixQ; ++j) {
+      if (j >= nq) break;
+      const int32_t v = __ldcg(src + j * BM);
+      if constexpr (kF8)
+        acc[j] = cc == c - 1 ? v
+                             : __float_as_int(__fadd_rn(__int_as_float(acc[j]), __int_as_float(v)));
+      else
+        acc[j] += v;
+    }
   }
-  const float ws = prm.epi == SQ_EPI_I32_RAW ? 0.0f : __ldg(prm.p_scale + p);
+  const float ws =
+      (prm.epi == SQ_EPI_I32_RAW || prm.epi == SQ_EPI_F32_RAW) ? 0.0f : __ldg(prm.p_scale + p);
 #pragma unroll
   for (int j = 0; j < kFixQ; ++j) {
     if (j >= nq) break;
     const int64_t o = static_cast<int64_t>(q0 + j) * prm.ldo + p;
-    if (prm.epi == SQ_EPI_I32_RAW) {
-      static_cast<int32_t*>(prm.out)[o] = acc[j];
+    if (prm.epi == SQ_EPI_I32_RAW || prm.epi == SQ_EPI_F32_RAW) {
+      static_cast<int32_t*>(prm.out)[o] = acc[j];  // the accumulator's bits
     } else {
-      float t = __fmul_rn(__fmul_rn(__int2float_rn(acc[j]), __ldg(prm.q_scale + q0 + j)), ws);
+      const float a = kF8 ? __int_as_float(acc[j]) : __int2float_rn(acc[j]);
+      float t = __fmul_rn(__fmul_rn(a, __ldg(prm.q_scale + q0 + j)), ws);
       if (prm.epi == SQ_EPI_BF16_RELU) t = t > 0.0f ? t : 0.0f;
       static_cast<__nv_bfloat16*>(prm.out)[o] = __float2bfloat16_rn(t);
     }
@@ -1236,9 +1248,9 @@ cudaError_t launch_gemm(const GemmPlan& plan, const int8_t* Xq, const int8_t* Wq
                         int64_t wait_polls, int* error_word, cudaStream_t st,
                         float* row_absmax, bool fp8) {
   if (M == 0 || N == 0) return cudaSuccess;
-  // FP8 accumulators are fp32: no INT32 partial sums to add exactly
-  if (fp8 && (plan.splits > 1 || plan.streamk || epi == SQ_EPI_I32_RAW))
-    return cudaErrorInvalidValue;
+  // FP8 accumulators are fp32: stream-K partials are added in a fixed order
+  // by the fix-up; no explicit split-K, no INT32 epilogue
+  if (fp8 && (plan.splits > 1 || epi == SQ_EPI_I32_RAW)) return cudaErrorInvalidValue;
   if (!fp8 && epi == SQ_EPI_F32_RAW) return cudaErrorInvalidValue;
   Params prm{};
   const int8_t* Pptr = plan.swap ? Wq : Xq;
@@ -1303,15 +1315,15 @@ cudaError_t launch_gemm(const GemmPlan& plan, const int8_t* Xq, const int8_t* Wq
       case 256: e = launch_bn<256, true>(prm, mp, mq, grid, st); break;
       default: return cudaErrorInvalidValue;
     }
-    return e;
-  }
-  switch (plan.bn) {
-    case 16: e = launch_bn<16, false>(prm, mp, mq, grid, st); break;
-    case 32: e = launch_bn<32, false>(prm, mp, mq, grid, st); break;
-    case 64: e = launch_bn<64, false>(prm, mp, mq, grid, st); break;
-    case 128: e = launch_bn<128, false>(prm, mp, mq, grid, st); break;
-    case 256: e = launch_bn<256, false>(prm, mp, mq, grid, st); break;
-    default: return cudaErrorInvalidValue;
+  } else {
+    switch (plan.bn) {
+      case 16: e = launch_bn<16, false>(prm, mp, mq, grid, st); break;
+      case 32: e = launch_bn<32, false>(prm, mp, mq, grid, st); break;
+      case 64: e = launch_bn<64, false>(prm, mp, mq, grid, st); break;
+      case 128: e = launch_bn<128, false>(prm, mp, mq, grid, st); break;
+      case 256: e = launch_bn<256, false>(prm, mp, mq, grid, st); break;
+      default: return cudaErrorInvalidValue;
+    }
   }
   if (e != cudaSuccess) return e;
   if (plan.streamk) {
@@ -1328,7 +1340,8 @@ cudaError_t launch_gemm(const GemmPlan& plan, const int8_t* Xq, const int8_t* Wq
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t fe = cudaLaunchKernelEx(&cfg, streamk_fixup_kernel, prm, plan.grid);
+    cudaError_t fe = fp8 ? cudaLaunchKernelEx(&cfg, streamk_fixup_kernel<true>, prm, plan.grid)
+                         : cudaLaunchKernelEx(&cfg, streamk_fixup_kernel<false>, prm, plan.grid);
     if (fe != cudaSuccess) return fe;
     return cudaGetLastError();
   }

@@ -201,7 +201,7 @@ def main(argv=None):
             fn = lambda: sq.fp8_gemm_dequant(A8, B8, scales[0], scales[1],
                                              "f32" if a.epi == "i32" else a.epi,
                                              out=out.view(torch.float32) if a.epi == "i32" else out,
-                                             path_hint=a.path)
+                                             path_hint=a.path, workspace=ws)
         if a.rowmax:
             rm = torch.empty(M, dtype=torch.float32, device=dev)
             fn = lambda: sq.w8a8_gemm_dequant_rowmax(A, B, xs, wsc, a.epi, out=out,

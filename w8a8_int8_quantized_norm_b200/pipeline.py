@@ -116,7 +116,7 @@ class Block:
                 self.Wq[lin.name] = torch.empty((lin.N, K), dtype=code_dtype, device=dev)
                 self.w_scale[lin.name] = torch.empty(lin.N, **f32)
             self.out[lin.name] = torch.empty((M, lin.N), dtype=torch.bfloat16, device=dev)
-            need = 0 if fmt == "fp8" else sq.gemm_workspace_size(M, lin.N, K, 0)
+            need = sq.gemm_workspace_size(M, lin.N, K, 0)
             self.ws[lin.name] = torch.empty(need, dtype=torch.uint8, device=dev) if need else None
         self.xq: Dict[str, torch.Tensor] = {}
         self.xs: Dict[str, torch.Tensor] = {}
@@ -307,7 +307,8 @@ class Block:
                     sq.fp8_gemm_dequant(self.xq[site.name], self.Wq[lin.name],
                                         self.xs[site.name], self.w_scale[lin.name],
                                         "bf16_relu" if lin.relu else "bf16",
-                                        out=self.out[lin.name], stream=stream)
+                                        out=self.out[lin.name], workspace=self.ws[lin.name],
+                                        whole_k=self.ws[lin.name] is None, stream=stream)
                     return
                 if lin.name in self.rowmax:
                     sq.w8a8_gemm_dequant_rowmax(

@@ -125,7 +125,8 @@ def _declare(L):
     L.sq_norm_smooth_quant_per_token_fp8.argtypes = [_P, _I32, _I64, _I64, _I64, _I32, _P, _P,
                                                      _F32, _P, _P, _P]
     L.sq_smooth_quantize_weights_fp8.argtypes = [_P, _I32, _I64, _I64, _I64, _P, _P, _P, _P]
-    L.sq_fp8_gemm_dequant.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _I32, _P, _I64, _I32, _P]
+    L.sq_fp8_gemm_dequant.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _I32, _P, _I64, _P, _SZ,
+                                      _I32, _P]
     L.sq_silu_mul_quant_per_token_fp8.argtypes = [_P, _I32, _I64, _I64, _I64, _P, _P, _P, _I64,
                                                   _P]
     L.sq_weight_column_max.argtypes = [_P, _P, _I32, _I32, _I64, _P, _P]
@@ -471,7 +472,10 @@ def smooth_quantize_weights_fp8(W: torch.Tensor, s: Optional[torch.Tensor] = Non
 
 def fp8_gemm_dequant(Xq8: torch.Tensor, Wq8: torch.Tensor, x_scale: Optional[torch.Tensor],
                      w_scale: Optional[torch.Tensor], epi: str = "bf16", out=None,
-                     path_hint: int = 0, stream=None) -> torch.Tensor:
+                     path_hint: int = 0, workspace=None, whole_k: bool = False,
+                     stream=None) -> torch.Tensor:
+    """e4m3 GEMM with the dequant epilogue.  Decode tiles run stream-K with a
+    workspace (allocated here when not given) unless ``whole_k``."""
     M, K = Xq8.shape
     N = Wq8.shape[0]
     if Xq8.dtype != torch.uint8 or Wq8.dtype != torch.uint8 or not Xq8.is_contiguous() \
@@ -480,9 +484,16 @@ def fp8_gemm_dequant(Xq8: torch.Tensor, Wq8: torch.Tensor, x_scale: Optional[tor
     if out is None:
         out = torch.empty((M, N), dtype=torch.float32 if epi == "f32" else torch.bfloat16,
                           device=Xq8.device)
+    if whole_k:
+        workspace = None
+    else:
+        need = gemm_workspace_size(M, N, K, 0) if path_hint != 1 and path_hint != 3 else 0
+        if workspace is None and need:
+            workspace = torch.empty(need, dtype=torch.uint8, device=Xq8.device)
+    wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(lib().sq_fp8_gemm_dequant(_ptr(Xq8), _ptr(Wq8), _ptr(x_scale), _ptr(w_scale), M, N, K,
-                                     EPI[epi], _ptr(out), out.stride(0), path_hint,
-                                     _stream(stream)), "sq_fp8_gemm_dequant")
+                                     EPI[epi], _ptr(out), out.stride(0), _ptr(workspace), wsb,
+                                     path_hint, _stream(stream)), "sq_fp8_gemm_dequant")
     return out
 
 
