@@ -1006,15 +1006,18 @@ __global__ void __launch_bounds__(BM) streamk_fixup_kernel(const Params prm, int
     if (sc >= t1) break;
     const int64_t slot = (sc / kbt == tile) ? 2 * cc : 2 * cc + 1;
     const int32_t* src = prm.sk_partial + (slot * prm.Q + q0) * BM + pl;
+    // predicated, not a loop exit: the loads of all kFixQ tokens issue together
 #pragma unroll
     for (int j = 0; j < kFixQ; ++j) {
-      if (j >= nq) break;
-      const int32_t v = __ldcg(src + j * BM);
-      if constexpr (kF8)
-        acc[j] = cc == c - 1 ? v
-                             : __float_as_int(__fadd_rn(__int_as_float(acc[j]), __int_as_float(v)));
-      else
-        acc[j] += v;
+      if (j < nq) {
+        const int32_t v = __ldcg(src + j * BM);
+        if constexpr (kF8)
+          acc[j] = cc == c - 1
+                       ? v
+                       : __float_as_int(__fadd_rn(__int_as_float(acc[j]), __int_as_float(v)));
+        else
+          acc[j] += v;
+      }
     }
   }
   const float ws =
