@@ -792,6 +792,22 @@ def test_graph_replay_matches_eager_step(wname, granularity, fmt):
     for key, v in snapshot().items():
         assert torch.equal(v, eager[key]), key
     del graph
+    # the benchmark's offline graph (calibration on the second stream beside
+    # the column maxima) prepares the same weights, factors and folds
+    for d in (blk.Wq, blk.w_scale, blk.s, blk.gamma_f):
+        for v in d.values():
+            if v is not None:
+                v.zero_()
+    graph = pipeline.capture_prepare(blk, prep_g["xc"], prep_g["W"], prep_g["g"], prep_g["b"])
+    for d in (blk.Wq, blk.w_scale):
+        for v in d.values():
+            v.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    for key, v in snapshot().items():
+        if key[0] in (3, 4, 5, 6, 7):  # Wq, w_scale, act_max, s, gamma_f
+            assert torch.equal(v, eager[key]), ("prepare graph", key)
+    del graph
 
 
 # ---------------------------------------------------------------------------
