@@ -8,6 +8,7 @@
     python -m w8a8_int8_quantized_norm_b200.kbench quant_given --M 4096 --K 36864
     python -m w8a8_int8_quantized_norm_b200.kbench silu_mul_quant --M 16384 --K 28672
     python -m w8a8_int8_quantized_norm_b200.kbench gemm --M 4096 --N 36864 --K 9216 --rowmax
+    python -m w8a8_int8_quantized_norm_b200.kbench llmint8_combine --M 16384 --N 8192 --K 8192
 
 Each call is captured once as a CUDA graph; every timed replay is bracketed by
 CUDA events on the launching stream, with L2 emptied before it (256 MiB
@@ -103,7 +104,10 @@ def _time(fn, iters, warmup, flush):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("op", choices=["norm_quant", "gemm", "calibrate", "weight_quant",
-                                   "smooth_scales", "quant_given", "silu_mul_quant"])
+                                   "smooth_scales", "quant_given", "silu_mul_quant",
+                                   "llmint8_combine"])
+    ap.add_argument("--outliers", type=int, default=8,
+                    help="llmint8_combine: outlier channels of x (x50, the rest N(0, 1))")
     ap.add_argument("--M", type=int, default=4096)
     ap.add_argument("--N", type=int, default=4096)
     ap.add_argument("--K", type=int, default=4096)
@@ -157,6 +161,24 @@ def main(argv=None):
         fn = lambda: sq.silu_mul_quant_per_token(gu, xq, xs)
         units = M * 2 * K * 2 + M * K + 4 * M
         shape = {"M": M, "I": K, "dtype": "bf16"}
+    elif a.op == "llmint8_combine":
+        # LLM.int8()'s merge on [M, N] outputs of a K-deep Linear: the INT32
+        # accumulator read, the 16-bit lane over the outlier channels, bf16 out
+        x = torch.randn((M, K), generator=gen, device=dev)
+        ch = torch.randperm(K, generator=gen, device=dev)[:a.outliers]
+        x[:, ch] *= 50.0
+        x = x.to(torch.bfloat16)
+        W = (torch.randn((N, K), generator=gen, device=dev) * 0.02).to(torch.bfloat16)
+        col = sq.weight_column_max([x])
+        mask, idx, count = sq.llmint8_outliers(col, 6.0)
+        acc = torch.randint(-2 ** 20, 2 ** 20, (M, N), generator=gen, device=dev,
+                            dtype=torch.int32)
+        xs = torch.empty(M, device=dev).uniform_(1e-3, 1e-2, generator=gen)
+        wsc = torch.empty(N, device=dev).uniform_(1e-4, 1e-3, generator=gen)
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        fn = lambda: sq.llmint8_combine(acc, xs, wsc, x, W, idx, count, "bf16", out=out)
+        units = M * N * (4 + 2) + 4 * (M + N)
+        shape = {"M": M, "N": N, "K": K, "outliers": int(count.item())}
     elif a.op == "calibrate":
         x = _acts(M, K, a.dtype, gen, dev)
         g = torch.empty(K, device=dev).uniform_(0.5, 1.5, generator=gen) if norm else None
