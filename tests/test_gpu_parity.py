@@ -1037,6 +1037,10 @@ def test_fp8_gemm_accumulator_and_epilogue(shape, path):
                                   whole_k=whole_k)
         acc_g = acc.cpu().numpy()
         assert np.all(np.abs(acc_g.astype(np.float64) - exact) <= fp8_acc_bound(K) * absum)
+        # the partial sums are added in a fixed order: the same bits on every run
+        again = sq.fp8_gemm_dequant(to_gpu(A), to_gpu(B), None, None, "f32", path_hint=path,
+                                    whole_k=whole_k)
+        assert np.array_equal(again.cpu().numpy().view(np.uint32), acc_g.view(np.uint32))
         for relu in (False, True):
             out = sq.fp8_gemm_dequant(to_gpu(A), to_gpu(B), to_gpu(xs), to_gpu(ws),
                                       "bf16_relu" if relu else "bf16", path_hint=path,
