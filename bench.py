@@ -874,7 +874,7 @@ def e2e_leg(args, w, inp, blk, dev, stream, world):
     for i in range(max(2, args.warmup)):
         step(i)
     torch.cuda.synchronize(dev)
-    n = max(2, min(args.steps, 10))
+    n = max(2, min(args.steps, 20))
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(s_in)
